@@ -1,0 +1,147 @@
+"""fp64 oracle for the replay group: GDN layers + SwiGLU MLPs, numpy.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+What the pages fix ("Tail-Replay: Escaping the Curse of Linear Attention in
+Prefix Caching for Hybrid LLMs", Sec. 3; "SuffixReplay: Prefix Caching via
+Suffix Replay for Hybrid LLMs", Algorithm Design 1):
+  * consecutive linear-attention layers between two full-attention layers
+    form a group; a group is replayed from its cached entry hidden (the
+    output of the preceding full-attention layer) with every linear state
+    starting at zero, and full-attention layers are skipped;
+  * the group's final FFN is omitted, because the next group starts from its
+    own cached exact hidden.
+
+What the pages leave open, and the reading taken here (the Qwen3.5-family
+GDN block, Sec. 2 of Tail-Replay names Gated DeltaNet as the linear layer):
+  x_res = x
+  h     = RMSNorm(x) * w_in_norm                     eps = 1e-6
+  p     = h W_in^T  -> [q_pre | k_pre | v_pre | z | b | a]
+  c     = causal depthwise conv, width 4, over [q_pre|k_pre|v_pre], zero
+          left padding at every sequence start (replay starts from zero)
+  q,k,v = SiLU(c);  q, k L2-normalised per head (eps 1e-6 inside the sqrt)
+  g     = -exp(A_log) * softplus(a + dt_bias);  beta = sigmoid(b)
+  o     = gated-delta recurrence (oracle.gdn_replay), scale 1/sqrt(d_k)
+  y     = RMSNorm_head(o) * w_gnorm * SiLU(z)        per V head
+  x     = x_res + y W_out^T
+  x     = x + W_down (SiLU(W_gate hh) * (W_up hh)),  hh = RMSNorm(x) * w_post
+  conv_state = the last (width-1) pre-conv rows of each sequence, oldest
+               first, zero where the sequence is shorter.
+Skip mode (the method): the last layer of the group stops after its
+recurrence -- neither its gated norm, out_proj nor MLP can change any state.
+Full mode: every layer runs to its MLP.
+
+Each primitive below is pinned by closed forms in ``tests/``; the composition
+is parity unpinned by the pages.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import gdn_replay, _f64
+
+
+def rmsnorm(x, w, eps):
+    """x / sqrt(mean(x^2) + eps) * w over the last axis."""
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * w
+
+
+def l2norm(x, eps):
+    """x / sqrt(sum(x^2) + eps) over the last axis."""
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+def sigmoid(x):
+    return 0.5 * (1.0 + np.tanh(0.5 * x))
+
+
+def silu(x):
+    return x * sigmoid(x)
+
+
+def softplus(x):
+    """log(1 + exp(x)), with x returned as is above 20 (overflow guard)."""
+    return np.where(x > 20.0, x, np.log1p(np.exp(np.minimum(x, 20.0))))
+
+
+def causal_conv(pre, w, cu):
+    """Depthwise causal conv: c_t[ch] = sum_i w[ch, i] * pre_{t-W+1+i}[ch],
+    pre = 0 before each sequence start (never across cu_seqlens)."""
+    T, D = pre.shape
+    W = w.shape[1]
+    out = np.zeros_like(pre)
+    for n in range(len(cu) - 1):
+        s, e = int(cu[n]), int(cu[n + 1])
+        seg = pre[s:e]
+        for i in range(W):
+            shift = W - 1 - i  # tap i reads the row `shift` tokens back
+            if shift >= e - s:
+                continue
+            out[s + shift:e] += w[:, i] * seg[: e - s - shift]
+    return out
+
+
+def conv_state(pre, cu, width):
+    """Last (width-1) pre-conv rows per sequence -> [N, D, width-1], oldest first."""
+    N = len(cu) - 1
+    D = pre.shape[1]
+    st = np.zeros((N, D, width - 1))
+    for n in range(N):
+        s, e = int(cu[n]), int(cu[n + 1])
+        for j in range(width - 1):
+            t = e - (width - 1) + j
+            if t >= s:
+                st[n, :, j] = pre[t]
+    return st
+
+
+def gdn_layer(x, lw, cu, shape, *, stop_after_recurrence=False):
+    """One GDN layer (+ its MLP unless stopped).  Returns a dict with the
+    final state S, conv_state, the gates, o (None when stopped) and x_out."""
+    s = shape
+    T = x.shape[0]
+    h = rmsnorm(x, _f64(lw.w_in_norm), s.eps)
+    p = h @ _f64(lw.w_in).T
+    qd, vd = s.qk_dim, s.v_dim
+    pre = p[:, : s.conv_dim]
+    z = p[:, s.conv_dim: s.conv_dim + vd]
+    b = p[:, s.conv_dim + vd: s.conv_dim + vd + s.h_v]
+    a = p[:, s.conv_dim + vd + s.h_v:]
+    c = silu(causal_conv(pre, _f64(lw.conv_w), cu))
+    q = l2norm(c[:, :qd].reshape(T, s.h_k, s.d_k), 1e-6)
+    k = l2norm(c[:, qd: 2 * qd].reshape(T, s.h_k, s.d_k), 1e-6)
+    v = c[:, 2 * qd:].reshape(T, s.h_v, s.d_v)
+    g = -np.exp(_f64(lw.a_log)) * softplus(a + _f64(lw.dt_bias))
+    beta = sigmoid(b)
+    o, S = gdn_replay(q, k, v, g, beta, cu, scale=1.0 / np.sqrt(s.d_k),
+                      want_o=not stop_after_recurrence)
+    out = dict(S=S, conv_state=conv_state(pre, cu, s.conv_w), g=g, beta=beta,
+               q=q, k=k, v=v, o=o, x_out=None)
+    if stop_after_recurrence:
+        return out
+    y = rmsnorm(o, _f64(lw.w_gnorm), s.eps) * silu(z.reshape(T, s.h_v, s.d_v))
+    x1 = x + y.reshape(T, vd) @ _f64(lw.w_out).T
+    hh = rmsnorm(x1, _f64(lw.w_post_norm), s.eps)
+    mid = silu(hh @ _f64(lw.w_gate).T) * (hh @ _f64(lw.w_up).T)
+    out["x_out"] = x1 + mid @ _f64(lw.w_down).T
+    out["x_attn"] = x1
+    return out
+
+
+def group_replay(gi, mode="skip"):
+    """Replay one group from its anchors with every state starting at zero.
+
+    gi: workloads.GroupInputs.  mode: "skip" (last layer stops after its
+    recurrence) or "full".  Returns a list of per-layer dicts (see gdn_layer).
+    """
+    assert mode in ("skip", "full")
+    cu = np.asarray(gi.cu_seqlens.tolist(), dtype=np.int64)
+    x = _f64(gi.anchors)
+    outs = []
+    L = len(gi.layers)
+    for l, lw in enumerate(gi.layers):
+        stop = mode == "skip" and l == L - 1
+        r = gdn_layer(x, lw, cu, gi.shape, stop_after_recurrence=stop)
+        outs.append(r)
+        x = r["x_out"]
+    return outs
