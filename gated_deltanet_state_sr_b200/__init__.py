@@ -1,0 +1,272 @@
+"""Suffix-replay state reconstruction for hybrid LLMs on B200 (sm_100a).
+
+Thin Python binding of the C-ABI library ``libsr.so`` (declared in
+``include/sr/sr.h``).  This module only marshals arguments -- torch tensors to
+device pointers, shapes to the C structs, the current CUDA stream -- and
+allocates outputs / workspaces with torch when the caller does not pass them.
+Every step of the replay runs in the library's CUDA kernels; there is no CPU
+or PyTorch fallback: importing fails loudly when ``libsr.so`` is missing.
+
+Entry points mirror the C ABI:
+    gdn_replay      one Gated DeltaNet layer from raw q/k/v/g/beta
+    mamba2_replay   the Mamba2 per-head-decay variant
+    group_replay    whole groups of GDN layers + MLPs from cached anchors
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsr.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sr", "sr.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gated_deltanet_state_sr_b200.build` "
+                      "(there is no fallback path)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+SR_OK, SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_WORKSPACE, SR_ERR_CUDA, SR_ERR_DEVICE = range(6)
+SR_BF16, SR_FP32 = 0, 1
+SR_GDN_AUTO, SR_GDN_SEQUENTIAL, SR_GDN_CHUNKED = 0, 1, 2
+SR_MODE_SKIP, SR_MODE_FULL = 0, 1
+SR_DEV_BAD_CU_SEQLENS, SR_DEV_SEQ_TOO_LONG = 0x1, 0x2
+_ALGOS = {"auto": SR_GDN_AUTO, "sequential": SR_GDN_SEQUENTIAL, "chunked": SR_GDN_CHUNKED}
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+
+
+class GdnArgs(ctypes.Structure):
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp), ("beta", _vp), ("cu_seqlens", _vp),
+                ("h0", _vp), ("o", _vp), ("s_out", _vp), ("dtype", _i32), ("algo", _i32),
+                ("n_seqs", _i32), ("total_tokens", _i32), ("max_seqlen", _i32), ("h_k", _i32),
+                ("h_v", _i32), ("d_k", _i32), ("d_v", _i32), ("scale", ctypes.c_float)]
+
+
+class Mamba2Args(ctypes.Structure):
+    _fields_ = [("x", _vp), ("B", _vp), ("C", _vp), ("dt", _vp), ("A", _vp), ("cu_seqlens", _vp),
+                ("h0", _vp), ("y", _vp), ("s_out", _vp), ("n_seqs", _i32), ("total_tokens", _i32),
+                ("max_seqlen", _i32), ("n_heads", _i32), ("head_dim", _i32), ("n_groups", _i32),
+                ("d_state", _i32)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("w_in_norm", _vp), ("w_in", _vp), ("conv_w", _vp), ("a_log", _vp),
+                ("dt_bias", _vp), ("w_gnorm", _vp), ("w_out", _vp), ("w_post_norm", _vp),
+                ("w_gate", _vp), ("w_up", _vp), ("w_down", _vp)]
+
+
+class LayerOutputs(ctypes.Structure):
+    _fields_ = [("s_out", _vp), ("conv_out", _vp), ("hidden_out", _vp)]
+
+
+class GroupArgs(ctypes.Structure):
+    _fields_ = [("anchors", ctypes.POINTER(_vp)), ("cu_seqlens", _vp),
+                ("weights", ctypes.POINTER(LayerWeights)), ("outputs", ctypes.POINTER(LayerOutputs)),
+                ("n_groups", _i32), ("n_layers", _i32), ("n_seqs", _i32), ("total_tokens", _i32),
+                ("max_seqlen", _i32), ("hidden", _i32), ("inter", _i32), ("h_k", _i32), ("h_v", _i32),
+                ("d_k", _i32), ("d_v", _i32), ("conv_width", _i32), ("eps", ctypes.c_float),
+                ("mode", _i32)]
+
+
+def _sig(name, restype, *argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(argtypes)
+    return f
+
+
+_gdn_ws = _sig("sr_gdn_replay_workspace", ctypes.c_size_t, ctypes.POINTER(GdnArgs))
+_gdn = _sig("sr_gdn_replay", _i32, ctypes.POINTER(GdnArgs), _vp, ctypes.c_size_t, _vp)
+_m2_ws = _sig("sr_mamba2_replay_workspace", ctypes.c_size_t, ctypes.POINTER(Mamba2Args))
+_m2 = _sig("sr_mamba2_replay", _i32, ctypes.POINTER(Mamba2Args), _vp, ctypes.c_size_t, _vp)
+_grp_ws = _sig("sr_group_replay_workspace", ctypes.c_size_t, ctypes.POINTER(GroupArgs))
+_grp = _sig("sr_group_replay", _i32, ctypes.POINTER(GroupArgs), _vp, ctypes.c_size_t, _vp)
+_last_error = _sig("sr_last_error", ctypes.c_char_p)
+_dev_status = _sig("sr_device_status", _i32, _vp, _vp, ctypes.POINTER(ctypes.c_uint32))
+_version = _sig("sr_version", _i32)
+
+
+def declared_symbols(header=HEADER_PATH):
+    """Names of every entry point ``include/sr/sr.h`` declares."""
+    txt = open(header).read()
+    return sorted(set(re.findall(r"SR_API\s+[\w\s\*]+?\b(sr_\w+)\s*\(", txt)))
+
+
+def library():
+    return _lib
+
+
+class SrError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"sr status {status}: {msg}")
+        self.status = status
+
+
+def last_error() -> str:
+    return (_last_error() or b"").decode()
+
+
+def _check(status):
+    if status != SR_OK:
+        raise SrError(status, last_error())
+
+
+def version() -> int:
+    return int(_version())
+
+
+# ------------------------------------------------------------------ torch glue
+
+
+def _torch():
+    import torch  # plumbing only: device memory and streams
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, ndim=None, device=True):
+    torch = _torch()
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+    return t
+
+
+def workspace(nbytes, device="cuda"):
+    """A 256-byte aligned device workspace of at least nbytes (torch-allocated)."""
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def device_status(ws, stream=None) -> int:
+    """Device status flags (SR_DEV_*) that the last call on ``ws`` recorded."""
+    flags = ctypes.c_uint32(0)
+    st = _dev_status(_ptr(ws), _stream_handle(stream), ctypes.byref(flags))
+    if st not in (SR_OK, SR_ERR_DEVICE):
+        _check(st)
+    return int(flags.value)
+
+
+def gdn_args(q, k, v, g, beta, cu_seqlens, *, n_seqs, max_seqlen, h0=None, o=None, s_out=None,
+             scale=0.0, algo="auto") -> GdnArgs:
+    torch = _torch()
+    T, h_k, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    dtype = SR_FP32 if q.dtype == torch.float32 else SR_BF16
+    return GdnArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(h0),
+                   _ptr(o), _ptr(s_out), dtype, _ALGOS[algo], n_seqs, T, max_seqlen, h_k, h_v,
+                   d_k, d_v, float(scale))
+
+
+def gdn_replay(q, k, v, g, beta, cu_seqlens, *, max_seqlen, h0=None, want_o=True, o=None,
+               s_out=None, scale=0.0, algo="auto", ws=None, stream=None):
+    """Gated DeltaNet replay of every packed sequence (see sr_gdn_replay).
+
+    q, k: [T, H_k, d] bf16/fp32; v: [T, H_v, d]; g, beta: [T, H_v] fp32;
+    cu_seqlens: [N+1] int32 (device); max_seqlen: host int >= every length.
+    Returns (o or None, s_out [N, H_v, d_v, d_k] fp32)."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, 3)
+    _need(g, "g", torch.float32, 2)
+    _need(beta, "beta", torch.float32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    n = cu_seqlens.numel() - 1
+    T, _, d_k = q.shape
+    h_v, d_v = v.shape[1], v.shape[2]
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, 4)
+    if o is None and want_o:
+        o = torch.empty_like(v)
+    if s_out is None:
+        s_out = torch.empty(n, h_v, d_v, d_k, dtype=torch.float32, device=q.device)
+    args = gdn_args(q, k, v, g, beta, cu_seqlens, n_seqs=n, max_seqlen=max_seqlen, h0=h0, o=o,
+                    s_out=s_out, scale=scale, algo=algo)
+    need = _gdn_ws(ctypes.byref(args))
+    if need == 0:
+        _check(_gdn(ctypes.byref(args), None, 0, None))  # raises with the validation message
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, q.device)
+    _check(_gdn(ctypes.byref(args), _ptr(ws), ws.numel(), _stream_handle(stream)))
+    return o, s_out
+
+
+def gdn_workspace_bytes(args: GdnArgs) -> int:
+    return int(_gdn_ws(ctypes.byref(args)))
+
+
+def gdn_call(args: GdnArgs, ws, stream=None) -> int:
+    """Raw C call with a prepared GdnArgs (returns the sr_status)."""
+    return int(_gdn(ctypes.byref(args), _ptr(ws), 0 if ws is None else ws.numel(),
+                    _stream_handle(stream) if ws is not None else None))
+
+
+def mamba2_args(x, B, C, dt, A, cu_seqlens, *, n_seqs, max_seqlen, h0=None, y=None,
+                s_out=None) -> Mamba2Args:
+    T, H, P = x.shape
+    G, Ns = B.shape[1], B.shape[2]
+    return Mamba2Args(_ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(cu_seqlens), _ptr(h0),
+                      _ptr(y), _ptr(s_out), n_seqs, T, max_seqlen, H, P, G, Ns)
+
+
+def mamba2_replay(x, B, C, dt, A, cu_seqlens, *, max_seqlen, h0=None, want_y=True, y=None,
+                  s_out=None, ws=None, stream=None):
+    """Mamba2 replay (see sr_mamba2_replay).  Returns (y or None, s_out)."""
+    torch = _torch()
+    _need(x, "x", torch.bfloat16, 3)
+    _need(B, "B", torch.bfloat16, 3)
+    _need(C, "C", torch.bfloat16, 3)
+    _need(dt, "dt", torch.float32, 2)
+    _need(A, "A", torch.float32, 1)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    n = cu_seqlens.numel() - 1
+    T, H, P = x.shape
+    Ns = B.shape[2]
+    if y is None and want_y:
+        y = torch.empty_like(x)
+    if s_out is None:
+        s_out = torch.empty(n, H, P, Ns, dtype=torch.float32, device=x.device)
+    args = mamba2_args(x, B, C, dt, A, cu_seqlens, n_seqs=n, max_seqlen=max_seqlen, h0=h0, y=y,
+                       s_out=s_out)
+    need = _m2_ws(ctypes.byref(args))
+    if need == 0:
+        _check(_m2(ctypes.byref(args), None, 0, None))
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, x.device)
+    _check(_m2(ctypes.byref(args), _ptr(ws), ws.numel(), _stream_handle(stream)))
+    return y, s_out
+
+
+def mamba2_workspace_bytes(args: Mamba2Args) -> int:
+    return int(_m2_ws(ctypes.byref(args)))
+
+
+def mamba2_call(args: Mamba2Args, ws, stream=None) -> int:
+    return int(_m2(ctypes.byref(args), _ptr(ws), 0 if ws is None else ws.numel(),
+                   _stream_handle(stream) if ws is not None else None))
+
+
+def default_scale(d_k):
+    return 1.0 / math.sqrt(d_k)

@@ -1,0 +1,50 @@
+// Shared device/host helpers of libsr (internal; not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sr/sr.h"
+
+namespace sr {
+
+// Workspace header: the first kWsHeader bytes of every workspace hold the
+// device status word (uint32 at offset 0).  Scratch regions follow.
+constexpr size_t kWsHeader = 256;
+constexpr size_t kWsAlign = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Thread-local last-error plumbing (api.cu).
+sr_status set_error(sr_status s, const char *fmt, ...);
+sr_status cuda_error(cudaError_t e, const char *where);
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Reads and checks the bounds of sequence n.  On a bad entry ORs a flag into
+// the status word and returns false; the caller then skips the sequence.
+__device__ __forceinline__ bool seq_bounds(const int32_t *cu, int n, int total, int max_len,
+                                           uint32_t *status, int &bos, int &eos) {
+    bos = cu[n];
+    eos = cu[n + 1];
+    bool ok = (bos >= 0) && (bos <= eos) && (eos <= total) && (n != 0 || bos == 0);
+    if (!ok) {
+        if (status) atomicOr(status, SR_DEV_BAD_CU_SEQLENS);
+        return false;
+    }
+    if (eos - bos > max_len) {
+        if (status) atomicOr(status, SR_DEV_SEQ_TOO_LONG);
+        return false;
+    }
+    return true;
+}
+
+}  // namespace sr

@@ -1,0 +1,249 @@
+/*
+ * sr.h -- C ABI of the suffix-replay state-reconstruction library (libsr.so).
+ *
+ * What it computes.  A hybrid LLM's linear-attention layers carry recurrent
+ * states that cannot be rolled back to an arbitrary prefix boundary.  Suffix
+ * replay rebuilds them by running the linear state update
+ *         S_t = A_t(S_{t-1}) + B_t,  S_0 = 0
+ * over only a short recent suffix of the matched prefix
+ * ("SuffixReplay: Prefix Caching via Suffix Replay for Hybrid LLMs",
+ *  Theoretical Foundation, Eq. 2 and Eq. 4; "Tail-Replay: Escaping the Curse
+ *  of Linear Attention in Prefix Caching for Hybrid LLMs", Sec. 3, where the
+ *  replay length is k = ceil(r m) for a matched prefix of m tokens and every
+ *  group starts its tail from a zero state).
+ *
+ * Entry points (all asynchronous on the given CUDA stream):
+ *   sr_gdn_replay     one Gated DeltaNet layer from raw q/k/v/g/beta
+ *   sr_group_replay   whole replay groups from cached anchor hiddens plus
+ *                     layer weights (RMSNorm, in_proj, conv, gates, the
+ *                     recurrence, gated norm, out_proj, SwiGLU MLP)
+ *   sr_mamba2_replay  the Mamba2 per-head-decay variant
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Memory.  Every pointer in an args struct is a DEVICE pointer unless its
+ *   comment says "host".  The caller owns all buffers; the library never
+ *   allocates, never frees, and keeps no state between calls except a
+ *   thread-local error string.  Scratch memory is the caller's `workspace`
+ *   (device, 256-byte aligned) of at least the size the matching
+ *   *_workspace() query returns for the same args.
+ * Packing.  Sequences are packed token-major and delimited by `cu_seqlens`
+ *   (device, int32, n_seqs+1 entries, cu[0] = 0, non-decreasing,
+ *   cu[n_seqs] = total_tokens): "Batched replay: multiple hits packed into one
+ *   variable-length execution with device-side boundaries" (SuffixReplay,
+ *   System Design, Pipelined Replay Path).  The host passes n_seqs,
+ *   total_tokens and an upper bound max_seqlen on every sequence length (used
+ *   only to size grids).  Zero-length sequences are allowed.
+ * Layouts are row-major, last index contiguous.  bf16 is IEEE bfloat16.
+ * Asynchrony.  A call validates its host-side arguments, enqueues kernels on
+ *   `stream` (a cudaStream_t; NULL = the legacy default stream) and returns.
+ *   It never synchronises and never allocates.
+ * Errors.  A call returns SR_OK or an error code; sr_last_error() gives a
+ *   message for the calling thread's last failure.  Nothing is enqueued when
+ *   host-side validation fails.  Device-side checks (a cu_seqlens entry out of
+ *   range, a sequence longer than max_seqlen) cannot be seen by the host
+ *   without a sync: the kernels skip the offending sequence, leave its outputs
+ *   untouched and OR a flag into the workspace's device status word, which
+ *   sr_device_status() reads.  Each call clears the status word first.
+ */
+#ifndef SR_SR_H
+#define SR_SR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SR_API __attribute__((visibility("default")))
+#else
+#define SR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sr_status {
+    SR_OK = 0,
+    SR_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent shape  */
+    SR_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head dim)   */
+    SR_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small  */
+    SR_ERR_CUDA = 4,         /* a CUDA runtime call failed (message says)   */
+    SR_ERR_DEVICE = 5        /* reported by sr_device_status only           */
+} sr_status;
+
+typedef enum sr_dtype { SR_BF16 = 0, SR_FP32 = 1 } sr_dtype;
+
+/* Device status word flags (sr_device_status). */
+#define SR_DEV_BAD_CU_SEQLENS 0x1u  /* cu[n] > cu[n+1], cu[n+1] > total, cu[0] != 0 */
+#define SR_DEV_SEQ_TOO_LONG 0x2u    /* a sequence is longer than max_seqlen       */
+
+/* Kernel selection for sr_gdn_replay. */
+typedef enum sr_gdn_algo {
+    SR_GDN_AUTO = 0,        /* chunked tensor-core kernel for bf16, sequential for fp32 */
+    SR_GDN_SEQUENTIAL = 1,  /* token-by-token fp32 FFMA recurrence (any dtype)          */
+    SR_GDN_CHUNKED = 2      /* chunked WY/UT form on tensor cores (bf16 only)           */
+} sr_gdn_algo;
+
+/* ------------------------------------------------------------------------
+ * sr_gdn_replay -- one Gated DeltaNet layer's recurrence over packed suffixes.
+ *
+ * For every sequence n and V head h (QK head h / (h_v / h_k)), starting from
+ * S = h0[n,h] (or 0 when h0 is NULL), for each token t of the sequence:
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     alpha_t = exp(g_t),   o_t = scale * S_t q_t
+ * ("Tail-Replay", Sec. 2: Gated DeltaNet with gate alpha in (0,1] and a rank-1
+ * correction; SuffixReplay, Eq. 4 with S_0 = 0).  S is d_v x d_k (row = value
+ * channel).  The final S of every (n, h) is written to s_out.
+ *
+ *   q, k       [total_tokens, h_k, d_k]   bf16 or fp32 (dtype)
+ *   v          [total_tokens, h_v, d_v]   same dtype
+ *   g          [total_tokens, h_v]        fp32, natural-log decay (<= 0)
+ *   beta       [total_tokens, h_v]        fp32
+ *   h0         [n_seqs, h_v, d_v, d_k]    fp32, may be NULL (zero state)
+ *   o          [total_tokens, h_v, d_v]   dtype, may be NULL (state only)
+ *   s_out      [n_seqs, h_v, d_v, d_k]    fp32, required
+ *   scale      multiplier of the output; 0 selects 1/sqrt(d_k)
+ * Supported: d_k = d_v in {64, 128}; h_v % h_k == 0.  Output buffers must not
+ * alias inputs.
+ * ---------------------------------------------------------------------- */
+typedef struct sr_gdn_args {
+    const void *q;
+    const void *k;
+    const void *v;
+    const float *g;
+    const float *beta;
+    const int32_t *cu_seqlens;
+    const float *h0;
+    void *o;
+    float *s_out;
+    int32_t dtype;        /* sr_dtype */
+    int32_t algo;         /* sr_gdn_algo */
+    int32_t n_seqs;
+    int32_t total_tokens;
+    int32_t max_seqlen;
+    int32_t h_k, h_v, d_k, d_v;
+    float scale;
+} sr_gdn_args;
+
+SR_API size_t sr_gdn_replay_workspace(const sr_gdn_args *args);
+SR_API sr_status sr_gdn_replay(const sr_gdn_args *args, void *workspace, size_t workspace_bytes,
+                        void *stream);
+
+/* ------------------------------------------------------------------------
+ * sr_mamba2_replay -- Mamba2 variant: per-head scalar decay, no erase.
+ *
+ *     S_t = exp(dt_t A_h) S_{t-1} + dt_t x_t B_t^T,   y_t = S_t C_t
+ * (SuffixReplay, Eq. 4: "per-head decay in Mamba2").  S is P x N_s per head;
+ * head h reads B/C group h / (n_heads / n_groups).
+ *
+ *   x          [total_tokens, n_heads, head_dim]   bf16
+ *   B, C       [total_tokens, n_groups, d_state]   bf16
+ *   dt         [total_tokens, n_heads]             fp32 (already positive)
+ *   A          [n_heads]                           fp32 (negative)
+ *   h0         [n_seqs, n_heads, head_dim, d_state] fp32, may be NULL
+ *   y          [total_tokens, n_heads, head_dim]   bf16, may be NULL
+ *   s_out      [n_seqs, n_heads, head_dim, d_state] fp32, required
+ * Supported: head_dim = 64, d_state = 128.
+ * ---------------------------------------------------------------------- */
+typedef struct sr_mamba2_args {
+    const void *x;
+    const void *B;
+    const void *C;
+    const float *dt;
+    const float *A;
+    const int32_t *cu_seqlens;
+    const float *h0;
+    void *y;
+    float *s_out;
+    int32_t n_seqs;
+    int32_t total_tokens;
+    int32_t max_seqlen;
+    int32_t n_heads, head_dim, n_groups, d_state;
+} sr_mamba2_args;
+
+SR_API size_t sr_mamba2_replay_workspace(const sr_mamba2_args *args);
+SR_API sr_status sr_mamba2_replay(const sr_mamba2_args *args, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* ------------------------------------------------------------------------
+ * sr_group_replay -- replay whole linear-attention groups from anchors.
+ *
+ * A group is a run of consecutive Gated DeltaNet layers between two full-
+ * attention layers; its anchor is the cached hidden entering the group (the
+ * preceding full-attention layer's output).  Every layer's recurrent state
+ * starts at zero and full-attention layers are skipped (SuffixReplay,
+ * Algorithm Design 1; Tail-Replay, Sec. 3).  Per layer:
+ *     h = RMSNorm(x) w_in_norm;  p = h W_in^T = [q|k|v|z|b|a]
+ *     causal depthwise conv (width conv_width, zero left padding per
+ *     sequence) + SiLU over [q|k|v]; q, k L2-normalised per head (eps 1e-6)
+ *     g = -exp(A_log) softplus(a + dt_bias);  beta = sigmoid(b)
+ *     gated-delta recurrence as in sr_gdn_replay (scale 1/sqrt(d_k))
+ *     y = RMSNorm_head(o) w_gnorm * SiLU(z);  x = x + y W_out^T
+ *     x = x + W_down(SiLU(W_gate hh) * W_up hh),  hh = RMSNorm(x) w_post_norm
+ * mode SR_MODE_SKIP stops the group's LAST layer after its recurrence (its
+ * gated norm, out_proj and MLP change no state: "Tail-Replay", Sec. 3 omits
+ * the final group FFN); SR_MODE_FULL runs every layer to its MLP.
+ * Groups are independent; n_groups > 1 replays them group-parallel with the
+ * same cu_seqlens (one request's suffix seen by every group).
+ *
+ * Shapes: proj_dim = 2 h_k d_k + 2 h_v d_v + 2 h_v, conv_dim = 2 h_k d_k + h_v d_v.
+ * Supported: hidden % 64 == 0, inter % 128 == 0, d_k = d_v = 128,
+ * conv_width = 4, (h_v d_v) % 64 == 0.
+ * ---------------------------------------------------------------------- */
+typedef struct sr_layer_weights {
+    const void *w_in_norm;   /* [hidden] bf16 */
+    const void *w_in;        /* [proj_dim, hidden] bf16 */
+    const void *conv_w;      /* [conv_dim, conv_width] bf16 */
+    const float *a_log;      /* [h_v] fp32 */
+    const float *dt_bias;    /* [h_v] fp32 */
+    const void *w_gnorm;     /* [d_v] bf16, shared by all V heads */
+    const void *w_out;       /* [hidden, h_v d_v] bf16 */
+    const void *w_post_norm; /* [hidden] bf16 */
+    const void *w_gate;      /* [inter, hidden] bf16 */
+    const void *w_up;        /* [inter, hidden] bf16 */
+    const void *w_down;      /* [hidden, inter] bf16 */
+} sr_layer_weights;
+
+typedef struct sr_layer_outputs {
+    float *s_out;     /* [n_seqs, h_v, d_v, d_k] fp32, required */
+    void *conv_out;   /* [n_seqs, conv_dim, conv_width-1] bf16, oldest row first, required */
+    void *hidden_out; /* [total_tokens, hidden] bf16, may be NULL: hidden after the layer's
+                         MLP; must be NULL for the last layer in SR_MODE_SKIP */
+} sr_layer_outputs;
+
+typedef enum sr_group_mode { SR_MODE_SKIP = 0, SR_MODE_FULL = 1 } sr_group_mode;
+
+typedef struct sr_group_args {
+    const void *const *anchors;       /* host array [n_groups] of device [total_tokens, hidden] bf16 */
+    const int32_t *cu_seqlens;
+    const sr_layer_weights *weights;  /* host array [n_groups * n_layers], group-major */
+    const sr_layer_outputs *outputs;  /* host array [n_groups * n_layers], group-major */
+    int32_t n_groups, n_layers;
+    int32_t n_seqs, total_tokens, max_seqlen;
+    int32_t hidden, inter, h_k, h_v, d_k, d_v, conv_width;
+    float eps;
+    int32_t mode;                     /* sr_group_mode */
+} sr_group_args;
+
+SR_API size_t sr_group_replay_workspace(const sr_group_args *args);
+SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics.
+ * ---------------------------------------------------------------------- */
+/* Message for the calling thread's last failed call ("" if none). */
+SR_API const char *sr_last_error(void);
+
+/* Copies the device status word of `workspace` (written by the last call that
+ * used it) into *flags (SR_DEV_* bits), synchronising `stream`.  Returns
+ * SR_ERR_DEVICE when any flag is set, SR_OK when none is. */
+SR_API sr_status sr_device_status(const void *workspace, void *stream, uint32_t *flags);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+SR_API int32_t sr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SR_SR_H */

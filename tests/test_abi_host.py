@@ -1,0 +1,112 @@
+"""Host-side tests of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every entry point ``include/sr/sr.h`` declares,
+and reject bad arguments during host validation -- before any CUDA call."""
+import ctypes
+
+import pytest
+
+sr = pytest.importorskip("gated_deltanet_state_sr_b200")
+
+FAKE = 0x10000  # an aligned, never-dereferenced address: validation fails first
+
+
+def test_exports_every_declared_symbol():
+    names = sr.declared_symbols()
+    assert {"sr_gdn_replay", "sr_group_replay", "sr_mamba2_replay", "sr_last_error",
+            "sr_device_status"} <= set(names)
+    for n in names:
+        assert hasattr(sr.library(), n), f"libsr.so does not export {n}"
+
+
+def test_version():
+    assert sr.version() == 0x000100
+
+
+def _gdn(**kw):
+    a = sr.GdnArgs(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu_seqlens=FAKE, h0=None, o=FAKE,
+                   s_out=FAKE, dtype=sr.SR_BF16, algo=sr.SR_GDN_AUTO, n_seqs=2, total_tokens=100,
+                   max_seqlen=60, h_k=2, h_v=4, d_k=64, d_v=64, scale=0.0)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("q", None, sr.SR_ERR_INVALID_ARG),
+    ("s_out", None, sr.SR_ERR_INVALID_ARG),
+    ("cu_seqlens", None, sr.SR_ERR_INVALID_ARG),
+    ("h_v", 5, sr.SR_ERR_INVALID_ARG),          # h_v % h_k != 0
+    ("h_k", 0, sr.SR_ERR_INVALID_ARG),
+    ("d_k", 96, sr.SR_ERR_UNSUPPORTED),
+    ("d_v", 128, sr.SR_ERR_UNSUPPORTED),        # d_k != d_v
+    ("n_seqs", -1, sr.SR_ERR_INVALID_ARG),
+    ("max_seqlen", 101, sr.SR_ERR_INVALID_ARG),  # longer than total
+    ("dtype", 7, sr.SR_ERR_INVALID_ARG),
+    ("algo", 9, sr.SR_ERR_INVALID_ARG),
+    ("s_out", FAKE + 4, sr.SR_ERR_INVALID_ARG),  # misaligned
+    ("scale", float("nan"), sr.SR_ERR_INVALID_ARG),
+])
+def test_gdn_validation(field, value, status):
+    a = _gdn(**{field: value})
+    assert sr.gdn_workspace_bytes(a) == 0
+    assert sr.gdn_call(a, None) == status
+    assert sr.last_error() != ""
+
+
+def test_gdn_chunked_requires_bf16():
+    a = _gdn(dtype=sr.SR_FP32, algo=sr.SR_GDN_CHUNKED)
+    assert sr.gdn_call(a, None) == sr.SR_ERR_UNSUPPORTED
+
+
+def test_gdn_workspace_required():
+    a = _gdn()
+    need = sr.gdn_workspace_bytes(a)
+    assert need >= 256
+    assert sr.gdn_call(a, None) == sr.SR_ERR_WORKSPACE
+    assert "workspace" in sr.last_error()
+
+
+def test_gdn_workspace_too_small_and_misaligned():
+    import torch
+    a = _gdn()
+    lib = sr.library()
+    small = ctypes.c_void_p(FAKE)
+    st = lib.sr_gdn_replay(ctypes.byref(a), small, 16, None)
+    assert st == sr.SR_ERR_WORKSPACE and "too small" in sr.last_error()
+    st = lib.sr_gdn_replay(ctypes.byref(a), ctypes.c_void_p(FAKE + 16), 1 << 30, None)
+    assert st == sr.SR_ERR_WORKSPACE and "aligned" in sr.last_error()
+
+
+def _m2(**kw):
+    a = sr.Mamba2Args(x=FAKE, B=FAKE, C=FAKE, dt=FAKE, A=FAKE, cu_seqlens=FAKE, h0=None, y=FAKE,
+                      s_out=FAKE, n_seqs=3, total_tokens=50, max_seqlen=40, n_heads=8, head_dim=64,
+                      n_groups=1, d_state=128)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("x", None, sr.SR_ERR_INVALID_ARG),
+    ("n_groups", 3, sr.SR_ERR_INVALID_ARG),
+    ("head_dim", 32, sr.SR_ERR_UNSUPPORTED),
+    ("d_state", 64, sr.SR_ERR_UNSUPPORTED),
+    ("total_tokens", -5, sr.SR_ERR_INVALID_ARG),
+])
+def test_mamba2_validation(field, value, status):
+    a = _m2(**{field: value})
+    assert sr.mamba2_workspace_bytes(a) == 0
+    assert sr.mamba2_call(a, None) == status
+
+
+def test_mamba2_workspace_required():
+    a = _m2()
+    assert sr.mamba2_workspace_bytes(a) >= 256
+    assert sr.mamba2_call(a, None) == sr.SR_ERR_WORKSPACE
+
+
+def test_device_status_needs_workspace():
+    flags = ctypes.c_uint32(0)
+    st = sr.library().sr_device_status(None, None, ctypes.byref(flags))
+    assert st == sr.SR_ERR_INVALID_ARG

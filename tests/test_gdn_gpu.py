@@ -1,0 +1,128 @@
+"""GPU parity of sr_gdn_replay against the fp64 oracle (same seeded inputs).
+
+Covers the raw-replay workloads at full size (one GDN layer, 1 x 256 tokens at
+2/4 heads d=64, and 8 varlen suffixes of U{512..2048} tokens at 16/32 heads
+d=128), plus edge cases: length-1 and length-2 sequences, empty sequences,
+ragged chunk tails, a nonzero initial state, strong decay, state-only mode,
+the fp32-input mode and device-side rejection of bad cu_seqlens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from _util import OUT_TOL_BF16, STATE_TOL, TOL_FP32, assert_close
+
+pytestmark = pytest.mark.gpu
+
+ALGOS = ["sequential", "chunked"]
+
+
+@pytest.fixture(scope="module")
+def sr():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gated_deltanet_state_sr_b200 as m
+    return m
+
+
+def run_gpu(sr, x: W.GdnInputs, algo, want_o=True, dev="cuda"):
+    t = lambda a: None if a is None else a.to(dev).contiguous()
+    o, s = sr.gdn_replay(t(x.q), t(x.k), t(x.v), t(x.g), t(x.beta), t(x.cu_seqlens),
+                         max_seqlen=max(x.max_seqlen, 1), h0=t(x.h0), want_o=want_o, algo=algo)
+    torch.cuda.synchronize()
+    return o, s
+
+
+def run_oracle(x: W.GdnInputs, want_o=True, units=None):
+    return oracle.gdn_replay(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, h0=x.h0, want_o=want_o,
+                             units=units)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_raw_small_workload(sr, algo):
+    x = W.raw_small()
+    o, s = run_gpu(sr, x, algo)
+    o_ref, s_ref = run_oracle(x)
+    assert_close(s, s_ref, STATE_TOL, "state")
+    assert_close(o, o_ref, OUT_TOL_BF16, "o")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_raw_qwen_workload_full_size(sr, algo):
+    x = W.raw_qwen()
+    o, s = run_gpu(sr, x, algo)
+    o_ref, s_ref = run_oracle(x)
+    assert_close(s, s_ref, STATE_TOL, "state")
+    assert_close(o, o_ref, OUT_TOL_BF16, "o")
+    # per-sequence state check, so one good long sequence cannot hide a bad short one
+    for n in range(x.n_seqs):
+        assert_close(s[n], s_ref[n], STATE_TOL, f"state seq {n}")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("d", [64, 128])
+def test_edge_lengths_with_initial_state(sr, algo, d):
+    lengths = [1, 2, 0, 3, 64, 65, 127, 200, 0, 129]
+    x = W.gdn_inputs(77 + d, lengths, 2, 4, d, d, h0_std=0.5)
+    o, s = run_gpu(sr, x, algo)
+    o_ref, s_ref = run_oracle(x)
+    for n in range(len(lengths)):
+        assert_close(s[n], s_ref[n], STATE_TOL, f"state seq {n} (len {lengths[n]})")
+    assert_close(o, o_ref, OUT_TOL_BF16, "o")
+    # empty sequences return their initial state
+    np.testing.assert_array_equal(s[2].cpu().numpy(), x.h0[2].numpy())
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_strong_decay(sr, algo):
+    """Gates of the group workload: g down to about -11 per token, so the
+    cumulative decay over a chunk leaves the fp32 exp range."""
+    x = W.gdn_inputs(5, [300, 77], 2, 4, 128, 128, g_range=(-12.0, -0.5), norm_q=True)
+    o, s = run_gpu(sr, x, algo)
+    o_ref, s_ref = run_oracle(x)
+    assert_close(s, s_ref, STATE_TOL, "state")
+    assert_close(o, o_ref, OUT_TOL_BF16, "o")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_state_only_mode(sr, algo):
+    x = W.gdn_inputs(6, [150, 40], 2, 4, 64, 64)
+    o, s = run_gpu(sr, x, algo, want_o=False)
+    assert o is None
+    _, s_ref = run_oracle(x, want_o=False)
+    assert_close(s, s_ref, STATE_TOL, "state")
+
+
+def test_fp32_input_mode(sr):
+    x = W.gdn_inputs(8, [1, 70, 333], 2, 4, 128, 128, dtype=torch.float32, h0_std=0.3)
+    o, s = run_gpu(sr, x, "auto")
+    assert o.dtype == torch.float32
+    o_ref, s_ref = run_oracle(x)
+    assert_close(s, s_ref, TOL_FP32, "state (fp32 mode)")
+    assert_close(o, o_ref, TOL_FP32, "o (fp32 mode)")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_bad_cu_seqlens_flagged_on_device(sr, algo):
+    """A decreasing cu_seqlens entry is caught by the kernel's own bounds check:
+    that sequence is skipped (its output untouched) and a flag is recorded."""
+    x = W.gdn_inputs(9, [10, 10, 10], 2, 4, 64, 64)
+    dev = lambda a: a.cuda().contiguous()
+    cu = torch.tensor([0, 10, 5, 30], dtype=torch.int32, device="cuda")  # seq 1 runs backwards
+    s_out = torch.full((3, 4, 64, 64), 7.0, device="cuda")
+    ws = sr.workspace(1 << 20)
+    sr.gdn_replay(dev(x.q), dev(x.k), dev(x.v), dev(x.g), dev(x.beta), cu, max_seqlen=25,
+                  s_out=s_out, want_o=False, algo=algo, ws=ws)
+    flags = sr.device_status(ws)
+    assert flags & sr.SR_DEV_BAD_CU_SEQLENS
+    assert torch.all(s_out[1] == 7.0)
+    # too-long sequence against max_seqlen
+    cu = x.cu_seqlens.cuda()
+    sr.gdn_replay(dev(x.q), dev(x.k), dev(x.v), dev(x.g), dev(x.beta), cu, max_seqlen=5,
+                  s_out=s_out, want_o=False, algo=algo, ws=ws)
+    assert sr.device_status(ws) & sr.SR_DEV_SEQ_TOO_LONG
+    # and a good call clears the word
+    sr.gdn_replay(dev(x.q), dev(x.k), dev(x.v), dev(x.g), dev(x.beta), cu, max_seqlen=10,
+                  s_out=s_out, want_o=False, algo=algo, ws=ws)
+    assert sr.device_status(ws) == 0
