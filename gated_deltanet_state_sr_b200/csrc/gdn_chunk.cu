@@ -1,13 +1,556 @@
-// Chunked gated-delta replay on tensor cores (placeholder until the kernel lands).
+// Chunked gated-delta replay on tensor cores (bf16 operands, fp32 state).
+//
+// Recurrence ("Tail-Replay: Escaping the Curse of Linear Attention in Prefix
+// Caching for Hybrid LLMs", Sec. 2; "SuffixReplay", Eq. 4):
+//     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = scale S_t q_t.
+// Write S_t = alpha_t S_{t-1} + u_t k_t^T with u_t = beta_t (v_t - alpha_t S_{t-1} k_t).
+// Inside a chunk of C tokens with log-decay prefix gamma_t = sum_{r<=t} g_r
+// (relative to the chunk start) and entry state S_0, unrolling gives the
+// lower-triangular system
+//     (I + A) U = diag(beta) V - diag(beta e^gamma) K S_0^T,
+//     A_ts = beta_t e^{gamma_t - gamma_s} (k_t . k_s)   for s < t,
+// so with T = (I + A)^{-1}, W = T diag(beta e^gamma) K and Ut = T diag(beta) V:
+//     U   = Ut - W S_0^T
+//     O   = scale (diag(e^gamma) Q S_0^T + M (U)),  M_ts = e^{gamma_t-gamma_s} q_t.k_s, s <= t
+//     S_C = e^{gamma_C} S_0 + U^T diag(e^{gamma_C - gamma}) K.
+// Only differences gamma_t - gamma_s with s <= t are ever exponentiated (the
+// exp argument is masked to -inf before the call), so strong decay underflows
+// to zero instead of overflowing.
+//
+// One CTA per (sequence, V head) keeps the whole d_v x d_k fp32 state in
+// mma.sync accumulator registers (warp w owns rows 16w..16w+15) and walks the
+// sequence chunk by chunk; the next chunk's q/k/v are prefetched with cp.async
+// while the current one is processed.  (I + A)^{-1} is formed in fp32 on the
+// CUDA cores: 16x16 diagonal blocks by forward substitution, then the
+// off-diagonal blocks by block back-substitution.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace sr {
 
-bool gdn_chunked_supported(const sr_gdn_args &) { return false; }
+namespace {
+
+constexpr int C = 64;        // tokens per chunk
+constexpr int ROWP = C + 8;  // bf16 row pitch of C x C tiles (144 B)
+constexpr int ROWA = C + 4;  // fp32 row pitch of C x C tiles (272 B)
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// D += A(16x16, row) * B(16x8, col), bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi), for a pair of values.
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<uint32_t *>(&h);
+    lo = *reinterpret_cast<uint32_t *>(&l);
+}
+
+// exp(gt - gs) for s <= t, else 0 (masked before the exponential).
+__device__ __forceinline__ float decay(float gt, float gs, bool keep) {
+    return __expf(keep ? gt - gs : -INFINITY);
+}
+
+template <int D>
+struct Smem {
+    static constexpr int ROW = D + 8;  // bf16 row pitch of C x D and D x D tiles
+    __nv_bfloat16 k[2][C * ROW];
+    __nv_bfloat16 q[2][C * ROW];
+    __nv_bfloat16 v[2][C * ROW];
+    __nv_bfloat16 sb[D * ROW];   // bf16 copy of the state entering the chunk
+    __nv_bfloat16 p[C * ROWP];   // masked, decayed, scaled Q K^T
+    // R1: A (fp32) during the solve, then -W (bf16)
+    union { float a[C * ROWA]; __nv_bfloat16 w[C * ROW]; } r1;
+    // R2: T (fp32) during the solve, then U (bf16)
+    union { float t[C * ROWA]; __nv_bfloat16 u[C * ROW]; } r2;
+    // R3: T diag(beta e^gamma) and T diag(beta) as hi + lo bf16 pairs, then
+    // U diag(e^{gamma_C-gamma}) as a hi + lo bf16 pair.  The pairs carry 16
+    // mantissa bits into the products that feed the state.
+    union {
+        struct { __nv_bfloat16 t1[C * ROWP], t2[C * ROWP], t1l[C * ROWP], t2l[C * ROWP]; } s;
+        struct { __nv_bfloat16 ud[C * ROW], udl[C * ROW]; } d;
+    } r3;
+    float gam[C];   // gamma_t, chunk-relative
+    float beta[C];
+};
+
+template <int D>
+__global__ void __launch_bounds__(D * 2)
+gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                 const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
+                 const float *__restrict__ beta, const int32_t *__restrict__ cu,
+                 const float *__restrict__ h0, __nv_bfloat16 *__restrict__ o,
+                 float *__restrict__ s_out, int total, int max_len, int h_k, int h_v,
+                 float scale, uint32_t *status) {
+    constexpr int NW = D / 16;         // warps; warp w owns state rows 16w..16w+15
+    constexpr int NT = NW * 32;
+    constexpr int ROW = Smem<D>::ROW;
+    constexpr int WPM = NW / 4;        // warps per 16-token block of the chunk
+    constexpr int NCOL = D / WPM;      // output columns per warp in the C x D products
+    constexpr int NPW = 32 / NW;       // n8 tiles per warp in the C x C products
+
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    Smem<D> &sm = *reinterpret_cast<Smem<D> *>(smem_raw);
+
+    const int h = blockIdx.x, n = blockIdx.y;
+    const int hk = h / (h_v / h_k);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 2, qd = lane & 3;
+    int bos, eos;
+    if (!seq_bounds(cu, n, total, max_len, status, bos, eos)) return;
+    const int len = eos - bos;
+    const int nchunks = (len + C - 1) / C;
+
+    const size_t qk_stride = size_t(h_k) * D;  // elements between consecutive tokens
+    const size_t v_stride = size_t(h_v) * D;
+    const __nv_bfloat16 *qh = q + size_t(bos) * qk_stride + size_t(hk) * D;
+    const __nv_bfloat16 *kh = k + size_t(bos) * qk_stride + size_t(hk) * D;
+    const __nv_bfloat16 *vh = v + size_t(bos) * v_stride + size_t(h) * D;
+
+    // Stage chunk c's q/k/v rows into buffer b (rows past the sequence end are zero-filled).
+    auto load_chunk = [&](int c, int b) {
+        constexpr int SEG = D / 8;  // 16-byte segments per row
+        for (int e = tid; e < C * SEG; e += NT) {
+            const int r = e / SEG, sgm = e % SEG;
+            const int t = c * C + r;
+            const bool ok = t < len;
+            const size_t tt = ok ? size_t(t) : 0;
+            cp_async16(smem_u32(&sm.k[b][r * ROW + sgm * 8]), kh + tt * qk_stride + sgm * 8, ok);
+            cp_async16(smem_u32(&sm.q[b][r * ROW + sgm * 8]), qh + tt * qk_stride + sgm * 8, ok);
+            cp_async16(smem_u32(&sm.v[b][r * ROW + sgm * 8]), vh + tt * v_stride + sgm * 8, ok);
+        }
+        cp_async_commit();
+    };
+
+    // ---- state: warp w owns rows 16w..16w+15, all D columns (D/8 n-tiles)
+    float S[D / 8][4];
+    const size_t sbase = (size_t(n) * h_v + h) * D * D;
+    {
+        const int r0 = warp * 16 + grp;
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+            const int c0 = j * 8 + 2 * qd;
+            if (h0) {
+                const float2 a = *reinterpret_cast<const float2 *>(h0 + sbase + size_t(r0) * D + c0);
+                const float2 b = *reinterpret_cast<const float2 *>(h0 + sbase + size_t(r0 + 8) * D + c0);
+                S[j][0] = a.x; S[j][1] = a.y; S[j][2] = b.x; S[j][3] = b.y;
+            } else {
+                S[j][0] = S[j][1] = S[j][2] = S[j][3] = 0.f;
+            }
+            *reinterpret_cast<uint32_t *>(&sm.sb[r0 * ROW + c0]) = pack_bf16(S[j][0], S[j][1]);
+            *reinterpret_cast<uint32_t *>(&sm.sb[(r0 + 8) * ROW + c0]) = pack_bf16(S[j][2], S[j][3]);
+        }
+    }
+
+    const float *gh = g + size_t(bos) * h_v + h;
+    const float *bh = beta + size_t(bos) * h_v + h;
+    float g_next = 0.f, b_next = 0.f;
+    if (nchunks > 0) {
+        load_chunk(0, 0);
+        if (tid < C && tid < len) {
+            g_next = gh[size_t(tid) * h_v];
+            b_next = bh[size_t(tid) * h_v];
+        }
+    }
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int cur = c & 1;
+        const int clen = min(C, len - c * C);
+        // ---- gates of this chunk: gamma = inclusive prefix sum of g (padding has g = beta = 0)
+        if (tid < C) {
+            sm.gam[tid] = g_next;
+            sm.beta[tid] = b_next;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        if (warp == 0) {
+            // inclusive scan of 64 values, two per lane
+            float a0 = sm.gam[2 * lane], a1 = sm.gam[2 * lane + 1];
+            float pair = a0 + a1;
+            float incl = pair;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const float excl = incl - pair;
+            sm.gam[2 * lane] = excl + a0;
+            sm.gam[2 * lane + 1] = excl + a0 + a1;
+        }
+        // prefetch the next chunk (other buffer) while this one is processed
+        if (c + 1 < nchunks) {
+            load_chunk(c + 1, cur ^ 1);
+            const int t = (c + 1) * C + tid;
+            g_next = (tid < C && t < len) ? gh[size_t(t) * h_v] : 0.f;
+            b_next = (tid < C && t < len) ? bh[size_t(t) * h_v] : 0.f;
+        }
+        __syncthreads();
+
+        const __nv_bfloat16 *Ks = sm.k[cur];
+        const __nv_bfloat16 *Qs = sm.q[cur];
+        const __nv_bfloat16 *Vs = sm.v[cur];
+        const float gC = sm.gam[C - 1];
+
+        // ---- (1)(2): A = strict-lower(beta_t e^{g_t-g_s} K K^T), P = lower(scale e^{g_t-g_s} Q K^T)
+        {
+            const int mb = warp / WPM;
+            const int nt0 = (warp % WPM) * NPW;
+            float akk[NPW][4], aqk[NPW][4];
+#pragma unroll
+            for (int j = 0; j < NPW; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) akk[j][e] = aqk[j][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                uint32_t ak[4], aq[4];
+                const int arow = mb * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
+                ldsm_x4(ak, smem_u32(&Ks[arow * ROW + acol]));
+                ldsm_x4(aq, smem_u32(&Qs[arow * ROW + acol]));
+#pragma unroll
+                for (int np = 0; np < NPW / 2; ++np) {
+                    uint32_t b[4];
+                    const int brow = (nt0 + 2 * np) * 8 + (lane & 7) + 8 * (lane >> 4);
+                    const int bcol = kk * 16 + 8 * ((lane >> 3) & 1);
+                    ldsm_x4(b, smem_u32(&Ks[brow * ROW + bcol]));
+                    mma16816(akk[2 * np], ak, b[0], b[1]);
+                    mma16816(akk[2 * np + 1], ak, b[2], b[3]);
+                    mma16816(aqk[2 * np], aq, b[0], b[1]);
+                    mma16816(aqk[2 * np + 1], aq, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < NPW; ++j) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int t = mb * 16 + grp + 8 * hh;
+                    const int s = (nt0 + j) * 8 + 2 * qd;
+                    const float gt = sm.gam[t], bt = sm.beta[t];
+                    const float d0 = decay(gt, sm.gam[s], s <= t), d1 = decay(gt, sm.gam[s + 1], s + 1 <= t);
+                    sm.r1.a[t * ROWA + s] = (s < t) ? bt * d0 * akk[j][2 * hh] : 0.f;
+                    sm.r1.a[t * ROWA + s + 1] = (s + 1 < t) ? bt * d1 * akk[j][2 * hh + 1] : 0.f;
+                    *reinterpret_cast<uint32_t *>(&sm.p[t * ROWP + s]) =
+                        pack_bf16(scale * d0 * aqk[j][2 * hh], scale * d1 * aqk[j][2 * hh + 1]);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- (3) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
+        float *Af = sm.r1.a;
+        float *Tf = sm.r2.t;
+        if (tid < C) {
+            const int b = tid >> 4, cc = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+                for (int s = 0; s < r; ++s) acc = fmaf(-Af[(16 * b + r) * ROWA + 16 * b + s], x[s], acc);
+                x[r] = (r < cc) ? 0.f : acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * ROWA + 16 * b + cc] = x[r];
+        }
+        __syncthreads();
+        // off-diagonal blocks: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  The strictly upper
+        // blocks of Tf serve as scratch for the inner sums X_ij (stored at block (j, i)).
+        auto blk = [](int bi, int bj, int r, int cc) { return (16 * bi + r) * ROWA + 16 * bj + cc; };
+        for (int level = 1; level <= 3; ++level) {
+            // X_ij for i - j == level
+            for (int e = tid; e < (4 - level) * 256; e += NT) {
+                const int j = e >> 8, i = j + level, r = (e >> 4) & 15, cc = e & 15;
+                float acc = 0.f;
+                for (int kb = j; kb < i; ++kb)
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) acc = fmaf(Af[blk(i, kb, r, m)], Tf[blk(kb, j, m, cc)], acc);
+                Tf[blk(j, i, r, cc)] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < (4 - level) * 256; e += NT) {
+                const int j = e >> 8, i = j + level, r = (e >> 4) & 15, cc = e & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) acc = fmaf(Tf[blk(i, i, r, m)], Tf[blk(j, i, m, cc)], acc);
+                Tf[blk(i, j, r, cc)] = -acc;
+            }
+            __syncthreads();
+        }
+        // T1 = T diag(beta e^gamma), T2 = T diag(beta)  (bf16, lower triangle incl. diagonal)
+        for (int e = tid; e < C * C / 2; e += NT) {
+            const int t = e / (C / 2), s = (e % (C / 2)) * 2;
+            const float t0 = (s <= t) ? Tf[t * ROWA + s] : 0.f;
+            const float t1 = (s + 1 <= t) ? Tf[t * ROWA + s + 1] : 0.f;
+            const float b0 = sm.beta[s], b1 = sm.beta[s + 1];
+            const float e0 = __expf(sm.gam[s]), e1 = __expf(sm.gam[s + 1]);
+            uint32_t hi, lo;
+            split_bf16(t0 * b0 * e0, t1 * b1 * e1, hi, lo);
+            *reinterpret_cast<uint32_t *>(&sm.r3.s.t1[t * ROWP + s]) = hi;
+            *reinterpret_cast<uint32_t *>(&sm.r3.s.t1l[t * ROWP + s]) = lo;
+            split_bf16(t0 * b0, t1 * b1, hi, lo);
+            *reinterpret_cast<uint32_t *>(&sm.r3.s.t2[t * ROWP + s]) = hi;
+            *reinterpret_cast<uint32_t *>(&sm.r3.s.t2l[t * ROWP + s]) = lo;
+        }
+        __syncthreads();
+
+        // ---- (4) -W = -T1 K  -> smem;  Ut = T2 V -> registers (this warp's U tile)
+        const int mb = warp / WPM;
+        const int n0 = (warp % WPM) * NCOL;
+        const int arow4 = mb * 16 + (lane & 15);
+        float acc_u[NCOL / 8][4];
+        {
+            float acc_w[NCOL / 8][4];
+#pragma unroll
+            for (int j = 0; j < NCOL / 8; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc_w[j][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                uint32_t ah[4], al[4];
+                const int acol = kk * 16 + (lane >> 4) * 8;
+                ldsm_x4(ah, smem_u32(&sm.r3.s.t1[arow4 * ROWP + acol]));
+                ldsm_x4(al, smem_u32(&sm.r3.s.t1l[arow4 * ROWP + acol]));
+#pragma unroll
+                for (int np = 0; np < NCOL / 16; ++np) {
+                    uint32_t bk[4];
+                    const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    const int bcol = n0 + np * 16 + 8 * (lane >> 4);
+                    ldsm_x4_t(bk, smem_u32(&Ks[brow * ROW + bcol]));
+                    mma16816(acc_w[2 * np], ah, bk[0], bk[1]);
+                    mma16816(acc_w[2 * np + 1], ah, bk[2], bk[3]);
+                    mma16816(acc_w[2 * np], al, bk[0], bk[1]);
+                    mma16816(acc_w[2 * np + 1], al, bk[2], bk[3]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < NCOL / 8; ++j) {
+                const int t = mb * 16 + grp, col = n0 + j * 8 + 2 * qd;
+                *reinterpret_cast<uint32_t *>(&sm.r1.w[t * ROW + col]) = pack_bf16(-acc_w[j][0], -acc_w[j][1]);
+                *reinterpret_cast<uint32_t *>(&sm.r1.w[(t + 8) * ROW + col]) = pack_bf16(-acc_w[j][2], -acc_w[j][3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NCOL / 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc_u[j][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+            uint32_t ah[4], al[4];
+            const int acol = kk * 16 + (lane >> 4) * 8;
+            ldsm_x4(ah, smem_u32(&sm.r3.s.t2[arow4 * ROWP + acol]));
+            ldsm_x4(al, smem_u32(&sm.r3.s.t2l[arow4 * ROWP + acol]));
+#pragma unroll
+            for (int np = 0; np < NCOL / 16; ++np) {
+                uint32_t bv[4];
+                const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                const int bcol = n0 + np * 16 + 8 * (lane >> 4);
+                ldsm_x4_t(bv, smem_u32(&Vs[brow * ROW + bcol]));
+                mma16816(acc_u[2 * np], ah, bv[0], bv[1]);
+                mma16816(acc_u[2 * np + 1], ah, bv[2], bv[3]);
+                mma16816(acc_u[2 * np], al, bv[0], bv[1]);
+                mma16816(acc_u[2 * np + 1], al, bv[2], bv[3]);
+            }
+        }
+        __syncthreads();
+
+        // ---- (5) U = Ut - W S_0^T ; store U and U diag(e^{gamma_C - gamma}) (bf16)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(a, smem_u32(&sm.r1.w[(mb * 16 + (lane & 15)) * ROW + kk * 16 + (lane >> 4) * 8]));
+#pragma unroll
+            for (int np = 0; np < NCOL / 16; ++np) {
+                uint32_t b[4];
+                const int brow = n0 + np * 16 + (lane & 7) + 8 * (lane >> 4);
+                const int bcol = kk * 16 + 8 * ((lane >> 3) & 1);
+                ldsm_x4(b, smem_u32(&sm.sb[brow * ROW + bcol]));
+                mma16816(acc_u[2 * np], a, b[0], b[1]);
+                mma16816(acc_u[2 * np + 1], a, b[2], b[3]);
+            }
+        }
+        {
+            const int t = mb * 16 + grp;
+            const float f0 = __expf(gC - sm.gam[t]), f1 = __expf(gC - sm.gam[t + 8]);
+#pragma unroll
+            for (int j = 0; j < NCOL / 8; ++j) {
+                const int col = n0 + j * 8 + 2 * qd;
+                *reinterpret_cast<uint32_t *>(&sm.r2.u[t * ROW + col]) = pack_bf16(acc_u[j][0], acc_u[j][1]);
+                *reinterpret_cast<uint32_t *>(&sm.r2.u[(t + 8) * ROW + col]) = pack_bf16(acc_u[j][2], acc_u[j][3]);
+                uint32_t hi, lo;
+                split_bf16(f0 * acc_u[j][0], f0 * acc_u[j][1], hi, lo);
+                *reinterpret_cast<uint32_t *>(&sm.r3.d.ud[t * ROW + col]) = hi;
+                *reinterpret_cast<uint32_t *>(&sm.r3.d.udl[t * ROW + col]) = lo;
+                split_bf16(f1 * acc_u[j][2], f1 * acc_u[j][3], hi, lo);
+                *reinterpret_cast<uint32_t *>(&sm.r3.d.ud[(t + 8) * ROW + col]) = hi;
+                *reinterpret_cast<uint32_t *>(&sm.r3.d.udl[(t + 8) * ROW + col]) = lo;
+            }
+        }
+        __syncthreads();
+
+        // ---- (6) O = scale e^gamma (Q S_0^T) + P U
+        if (o) {
+            float acc_o[NCOL / 8][4];
+#pragma unroll
+            for (int j = 0; j < NCOL / 8; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc_o[j][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                uint32_t a[4];
+                ldsm_x4(a, smem_u32(&Qs[(mb * 16 + (lane & 15)) * ROW + kk * 16 + (lane >> 4) * 8]));
+#pragma unroll
+                for (int np = 0; np < NCOL / 16; ++np) {
+                    uint32_t b[4];
+                    const int brow = n0 + np * 16 + (lane & 7) + 8 * (lane >> 4);
+                    const int bcol = kk * 16 + 8 * ((lane >> 3) & 1);
+                    ldsm_x4(b, smem_u32(&sm.sb[brow * ROW + bcol]));
+                    mma16816(acc_o[2 * np], a, b[0], b[1]);
+                    mma16816(acc_o[2 * np + 1], a, b[2], b[3]);
+                }
+            }
+            const int t = mb * 16 + grp;
+            const float f0 = scale * __expf(sm.gam[t]), f1 = scale * __expf(sm.gam[t + 8]);
+#pragma unroll
+            for (int j = 0; j < NCOL / 8; ++j) {
+                acc_o[j][0] *= f0; acc_o[j][1] *= f0; acc_o[j][2] *= f1; acc_o[j][3] *= f1;
+            }
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                uint32_t a[4];
+                ldsm_x4(a, smem_u32(&sm.p[(mb * 16 + (lane & 15)) * ROWP + kk * 16 + (lane >> 4) * 8]));
+#pragma unroll
+                for (int np = 0; np < NCOL / 16; ++np) {
+                    uint32_t b[4];
+                    const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    const int bcol = n0 + np * 16 + 8 * (lane >> 4);
+                    ldsm_x4_t(b, smem_u32(&sm.r2.u[brow * ROW + bcol]));
+                    mma16816(acc_o[2 * np], a, b[0], b[1]);
+                    mma16816(acc_o[2 * np + 1], a, b[2], b[3]);
+                }
+            }
+            const size_t tok0 = size_t(bos) + size_t(c) * C;
+#pragma unroll
+            for (int j = 0; j < NCOL / 8; ++j) {
+                const int col = n0 + j * 8 + 2 * qd;
+                if (t < clen)
+                    *reinterpret_cast<uint32_t *>(o + (tok0 + t) * v_stride + size_t(h) * D + col) =
+                        pack_bf16(acc_o[j][0], acc_o[j][1]);
+                if (t + 8 < clen)
+                    *reinterpret_cast<uint32_t *>(o + (tok0 + t + 8) * v_stride + size_t(h) * D + col) =
+                        pack_bf16(acc_o[j][2], acc_o[j][3]);
+            }
+        }
+        __syncthreads();  // every warp is done reading sb before it is overwritten
+
+        // ---- (7) S_C = e^{gamma_C} S_0 + (U diag(e^{gamma_C-gamma}))^T K
+        {
+            const float fC = __expf(gC);
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) S[j][e] *= fC;
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                uint32_t ah[4], al[4];
+                const int arow = kk * 16 + (lane & 7) + 8 * (lane >> 4);
+                const int acol = warp * 16 + 8 * ((lane >> 3) & 1);
+                ldsm_x4_t(ah, smem_u32(&sm.r3.d.ud[arow * ROW + acol]));
+                ldsm_x4_t(al, smem_u32(&sm.r3.d.udl[arow * ROW + acol]));
+#pragma unroll
+                for (int np = 0; np < D / 16; ++np) {
+                    uint32_t b[4];
+                    const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    const int bcol = np * 16 + 8 * (lane >> 4);
+                    ldsm_x4_t(b, smem_u32(&Ks[brow * ROW + bcol]));
+                    mma16816(S[2 * np], ah, b[0], b[1]);
+                    mma16816(S[2 * np + 1], ah, b[2], b[3]);
+                    mma16816(S[2 * np], al, b[0], b[1]);
+                    mma16816(S[2 * np + 1], al, b[2], b[3]);
+                }
+            }
+            const int r0 = warp * 16 + grp;
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j) {
+                const int c0 = j * 8 + 2 * qd;
+                *reinterpret_cast<uint32_t *>(&sm.sb[r0 * ROW + c0]) = pack_bf16(S[j][0], S[j][1]);
+                *reinterpret_cast<uint32_t *>(&sm.sb[(r0 + 8) * ROW + c0]) = pack_bf16(S[j][2], S[j][3]);
+            }
+        }
+        // the next iteration's first barrier orders these writes before any read
+    }
+
+    // ---- final state
+    {
+        const int r0 = warp * 16 + grp;
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+            const int c0 = j * 8 + 2 * qd;
+            *reinterpret_cast<float2 *>(s_out + sbase + size_t(r0) * D + c0) = make_float2(S[j][0], S[j][1]);
+            *reinterpret_cast<float2 *>(s_out + sbase + size_t(r0 + 8) * D + c0) = make_float2(S[j][2], S[j][3]);
+        }
+    }
+}
+
+template <int D>
+cudaError_t launch_chunked(const sr_gdn_args &a, float scale, uint32_t *status, cudaStream_t st) {
+    const size_t smem = sizeof(Smem<D>);
+    cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.h_v, a.n_seqs);
+    gdn_chunk_kernel<D><<<grid, D * 2, smem, st>>>(
+        static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
+        static_cast<const __nv_bfloat16 *>(a.v), a.g, a.beta, a.cu_seqlens, a.h0,
+        static_cast<__nv_bfloat16 *>(a.o), a.s_out, a.total_tokens, a.max_seqlen, a.h_k, a.h_v, scale,
+        status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gdn_chunked_supported(const sr_gdn_args &a) {
+    return a.dtype == SR_BF16 && a.d_k == a.d_v && (a.d_k == 64 || a.d_k == 128);
+}
+
 size_t gdn_scratch_bytes(const sr_gdn_args &) { return 0; }
+
 cudaError_t gdn_chunked(const sr_gdn_args &a, float scale, uint32_t *status, void *, cudaStream_t st) {
-    return gdn_sequential(a, scale, status, st);
+    if (a.n_seqs == 0 || a.h_v == 0) return cudaSuccess;
+    return a.d_k == 64 ? launch_chunked<64>(a, scale, status, st) : launch_chunked<128>(a, scale, status, st);
 }
 
 size_t mamba2_scratch_bytes(const sr_mamba2_args &) { return 0; }
