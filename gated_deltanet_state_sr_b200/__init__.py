@@ -70,7 +70,7 @@ class GroupArgs(ctypes.Structure):
                 ("n_groups", _i32), ("n_layers", _i32), ("n_seqs", _i32), ("total_tokens", _i32),
                 ("max_seqlen", _i32), ("hidden", _i32), ("inter", _i32), ("h_k", _i32), ("h_v", _i32),
                 ("d_k", _i32), ("d_v", _i32), ("conv_width", _i32), ("eps", ctypes.c_float),
-                ("mode", _i32)]
+                ("mode", _i32), ("precision", _i32)]
 
 
 def _sig(name, restype, *argtypes):
@@ -270,3 +270,97 @@ def mamba2_call(args: Mamba2Args, ws, stream=None) -> int:
 
 def default_scale(d_k):
     return 1.0 / math.sqrt(d_k)
+
+
+# ------------------------------------------------------------------ test support (include/sr/sr_testing.h)
+
+_test_gemm = _sig("sr_test_gemm", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp,
+                  ctypes.c_size_t, _vp)
+EPI_STORE, EPI_RESIDUAL, EPI_SWIGLU = 0, 1, 2
+
+
+def test_gemm(a, b0, *, b1=None, r=None, epi=EPI_STORE, c=None, ws=None, stream=None):
+    """One tcgen05 GEMM through sr_test_gemm: c = a b0^T, r + a b0^T, or
+    SiLU(a b0^T) * (a b1^T).  bf16 CUDA tensors, row-major."""
+    torch = _torch()
+    m, k = a.shape
+    n = b0.shape[0]
+    if c is None:
+        c = torch.empty(m, n, dtype=torch.bfloat16, device=a.device)
+    if ws is None:
+        ws = workspace(256, a.device)
+    _check(_test_gemm(_ptr(a), _ptr(b0), _ptr(b1), _ptr(c), _ptr(r), m, n, k, epi, _ptr(ws), ws.numel(),
+                      _stream_handle(stream)))
+    return c
+
+
+# ------------------------------------------------------------------ group replay
+
+SR_PREC_SPLIT, SR_PREC_BF16 = 0, 1
+_LAYER_FIELDS = [f for f, _ in LayerWeights._fields_]
+
+
+def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, inter, h_k, h_v, d=128,
+               conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT):
+    """Builds a GroupArgs (and keeps the ctypes arrays alive on it).
+
+    anchors: list [G] of [T, hidden] bf16 CUDA tensors; weights: list [G] of
+    lists [L] of objects with the sr_layer_weights field names (CUDA tensors);
+    outputs: list [G] of lists [L] of (s_out, conv_out, hidden_out-or-None)."""
+    G, L = len(anchors), len(weights[0])
+    anc = (_vp * G)(*[t.data_ptr() for t in anchors])
+    w_arr = (LayerWeights * (G * L))()
+    o_arr = (LayerOutputs * (G * L))()
+    for g in range(G):
+        for l in range(L):
+            lw = weights[g][l]
+            w_arr[g * L + l] = LayerWeights(*[getattr(lw, f).data_ptr() for f in _LAYER_FIELDS])
+            s, c, h = outputs[g][l]
+            o_arr[g * L + l] = LayerOutputs(s.data_ptr(), c.data_ptr(), None if h is None else h.data_ptr())
+    n = cu_seqlens.numel() - 1
+    T = anchors[0].shape[0]
+    a = GroupArgs(anc, cu_seqlens.data_ptr(), w_arr, o_arr, G, L, n, T, max_seqlen, hidden, inter, h_k, h_v,
+                  d, d, conv_width, float(eps), mode, precision)
+    a._keep = (anc, w_arr, o_arr)
+    return a
+
+
+def group_workspace_bytes(args: GroupArgs) -> int:
+    return int(_grp_ws(ctypes.byref(args)))
+
+
+def group_call(args: GroupArgs, ws, stream=None) -> int:
+    return int(_grp(ctypes.byref(args), None if ws is None else _ptr(ws), 0 if ws is None else ws.numel(),
+                    _stream_handle(stream) if ws is not None else None))
+
+
+def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k, h_v, d=128, conv_width=4,
+                 eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, want_hidden=False, outputs=None,
+                 ws=None, stream=None):
+    """Replays every group of the call (see sr_group_replay).  Returns the
+    outputs list [G][L] of (s_out, conv_out, hidden_out or None)."""
+    torch = _torch()
+    dev = anchors[0].device
+    G, L = len(anchors), len(weights[0])
+    n = cu_seqlens.numel() - 1
+    T = anchors[0].shape[0]
+    conv_dim = 2 * h_k * d + h_v * d
+    if outputs is None:
+        outputs = []
+        for g in range(G):
+            row = []
+            for l in range(L):
+                keep_h = want_hidden and not (mode == SR_MODE_SKIP and l == L - 1)
+                row.append((torch.empty(n, h_v, d, d, dtype=torch.float32, device=dev),
+                            torch.empty(n, conv_dim, conv_width - 1, dtype=torch.bfloat16, device=dev),
+                            torch.empty(T, hidden, dtype=torch.bfloat16, device=dev) if keep_h else None))
+            outputs.append(row)
+    args = group_args(anchors, cu_seqlens, weights, outputs, max_seqlen=max_seqlen, hidden=hidden, inter=inter,
+                      h_k=h_k, h_v=h_v, d=d, conv_width=conv_width, eps=eps, mode=mode, precision=precision)
+    need = group_workspace_bytes(args)
+    if need == 0:
+        _check(group_call(args, None))
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, dev)
+    _check(group_call(args, ws, stream))
+    return outputs

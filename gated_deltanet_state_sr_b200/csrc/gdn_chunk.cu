@@ -11,18 +11,23 @@
 //     A_ts = beta_t e^{gamma_t - gamma_s} (k_t . k_s)   for s < t,
 // so with T = (I + A)^{-1}, W = T diag(beta e^gamma) K and Ut = T diag(beta) V:
 //     U   = Ut - W S_0^T
-//     O   = scale (diag(e^gamma) Q S_0^T + M (U)),  M_ts = e^{gamma_t-gamma_s} q_t.k_s, s <= t
+//     O   = scale (diag(e^gamma) Q S_0^T + M U),  M_ts = e^{gamma_t-gamma_s} q_t.k_s, s <= t
 //     S_C = e^{gamma_C} S_0 + U^T diag(e^{gamma_C - gamma}) K.
 // Only differences gamma_t - gamma_s with s <= t are ever exponentiated (the
 // exp argument is masked to -inf before the call), so strong decay underflows
 // to zero instead of overflowing.
 //
-// One CTA per (sequence, V head) keeps the whole d_v x d_k fp32 state in
-// mma.sync accumulator registers (warp w owns rows 16w..16w+15) and walks the
-// sequence chunk by chunk; the next chunk's q/k/v are prefetched with cp.async
-// while the current one is processed.  (I + A)^{-1} is formed in fp32 on the
-// CUDA cores: 16x16 diagonal blocks by forward substitution, then the
-// off-diagonal blocks by block back-substitution.
+// One CTA per (group, sequence, V head) keeps the whole d_v x d_k fp32 state
+// in mma.sync accumulator registers (warp w owns rows 16w..16w+15) and walks
+// the sequence chunk by chunk.  q/k/v of the next chunk are prefetched with
+// cp.async as soon as the current chunk's last reader of each buffer is done.
+// (I + A)^{-1} is formed in fp32 on the CUDA cores: 16x16 diagonal blocks by
+// forward substitution, then the off-diagonal blocks by block substitution.
+//
+// Precision: T and U enter the products that feed the state as exact hi + lo
+// bf16 pairs.  With SPLIT, k and v also arrive as hi + lo pairs (the layer
+// computes them in fp32) and every product that reaches the state uses the
+// three-term expansion hi*hi + lo*hi + hi*lo.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -86,12 +91,14 @@ __device__ __forceinline__ float decay(float gt, float gs, bool keep) {
     return __expf(keep ? gt - gs : -INFINITY);
 }
 
-template <int D>
+template <int D, bool SPLIT>
 struct Smem {
     static constexpr int ROW = D + 8;  // bf16 row pitch of C x D and D x D tiles
-    __nv_bfloat16 k[2][C * ROW];
-    __nv_bfloat16 q[2][C * ROW];
-    __nv_bfloat16 v[2][C * ROW];
+    __nv_bfloat16 k[C * ROW];
+    __nv_bfloat16 q[C * ROW];
+    __nv_bfloat16 v[C * ROW];
+    __nv_bfloat16 kl[SPLIT ? C * ROW : 8];  // low parts of k, v (SPLIT)
+    __nv_bfloat16 vl[SPLIT ? C * ROW : 8];
     __nv_bfloat16 sb[D * ROW];   // bf16 copy of the state entering the chunk
     __nv_bfloat16 p[C * ROWP];   // masked, decayed, scaled Q K^T
     // R1: A (fp32) during the solve, then -W (bf16)
@@ -99,8 +106,7 @@ struct Smem {
     // R2: T (fp32) during the solve, then U (bf16)
     union { float t[C * ROWA]; __nv_bfloat16 u[C * ROW]; } r2;
     // R3: T diag(beta e^gamma) and T diag(beta) as hi + lo bf16 pairs, then
-    // U diag(e^{gamma_C-gamma}) as a hi + lo bf16 pair.  The pairs carry 16
-    // mantissa bits into the products that feed the state.
+    // U diag(e^{gamma_C-gamma}) as a hi + lo bf16 pair.
     union {
         struct { __nv_bfloat16 t1[C * ROWP], t2[C * ROWP], t1l[C * ROWP], t2l[C * ROWP]; } s;
         struct { __nv_bfloat16 ud[C * ROW], udl[C * ROW]; } d;
@@ -109,52 +115,52 @@ struct Smem {
     float beta[C];
 };
 
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(D * 2)
-gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                 const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
-                 const float *__restrict__ beta, const int32_t *__restrict__ cu,
-                 const float *__restrict__ h0, __nv_bfloat16 *__restrict__ o,
-                 float *__restrict__ s_out, int total, int max_len, int h_k, int h_v,
-                 float scale, uint32_t *status) {
+gdn_chunk_kernel(const __grid_constant__ GdnBatch p) {
     constexpr int NW = D / 16;         // warps; warp w owns state rows 16w..16w+15
     constexpr int NT = NW * 32;
-    constexpr int ROW = Smem<D>::ROW;
+    constexpr int ROW = Smem<D, SPLIT>::ROW;
     constexpr int WPM = NW / 4;        // warps per 16-token block of the chunk
     constexpr int NCOL = D / WPM;      // output columns per warp in the C x D products
     constexpr int NPW = 32 / NW;       // n8 tiles per warp in the C x C products
+    constexpr int SEG = D / 8;         // 16-byte segments per row
 
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem<D> &sm = *reinterpret_cast<Smem<D> *>(smem_raw);
+    Smem<D, SPLIT> &sm = *reinterpret_cast<Smem<D, SPLIT> *>(smem_raw);
 
-    const int h = blockIdx.x, n = blockIdx.y;
+    const int h = blockIdx.x, n = blockIdx.y, grp_i = blockIdx.z;
+    const int h_k = p.h_k, h_v = p.h_v;
     const int hk = h / (h_v / h_k);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int grp = lane >> 2, qd = lane & 3;
     int bos, eos;
-    if (!seq_bounds(cu, n, total, max_len, status, bos, eos)) return;
+    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     const int len = eos - bos;
     const int nchunks = (len + C - 1) / C;
+    const float scale = p.scale;
 
     const size_t qk_stride = size_t(h_k) * D;  // elements between consecutive tokens
     const size_t v_stride = size_t(h_v) * D;
-    const __nv_bfloat16 *qh = q + size_t(bos) * qk_stride + size_t(hk) * D;
-    const __nv_bfloat16 *kh = k + size_t(bos) * qk_stride + size_t(hk) * D;
-    const __nv_bfloat16 *vh = v + size_t(bos) * v_stride + size_t(h) * D;
+    const size_t qk_off = size_t(bos) * qk_stride + size_t(hk) * D;
+    const size_t v_off = size_t(bos) * v_stride + size_t(h) * D;
+    const __nv_bfloat16 *qh = p.q[grp_i] + qk_off;
+    const __nv_bfloat16 *kh = p.k[grp_i] + qk_off;
+    const __nv_bfloat16 *vh = p.v[grp_i] + v_off;
+    const __nv_bfloat16 *klh = SPLIT ? p.k_lo[grp_i] + qk_off : nullptr;
+    const __nv_bfloat16 *vlh = SPLIT ? p.v_lo[grp_i] + v_off : nullptr;
+    __nv_bfloat16 *o = p.o[grp_i];
+    const float *h0 = p.h0[grp_i];
 
-    // Stage chunk c's q/k/v rows into buffer b (rows past the sequence end are zero-filled).
-    auto load_chunk = [&](int c, int b) {
-        constexpr int SEG = D / 8;  // 16-byte segments per row
+    // Stage rows of chunk c from `src` (token pitch `stride`) into `dst`; rows
+    // past the sequence end are zero-filled.
+    auto stage = [&](__nv_bfloat16 *dst, const __nv_bfloat16 *src, size_t stride, int c) {
         for (int e = tid; e < C * SEG; e += NT) {
             const int r = e / SEG, sgm = e % SEG;
             const int t = c * C + r;
             const bool ok = t < len;
-            const size_t tt = ok ? size_t(t) : 0;
-            cp_async16(smem_u32(&sm.k[b][r * ROW + sgm * 8]), kh + tt * qk_stride + sgm * 8, ok);
-            cp_async16(smem_u32(&sm.q[b][r * ROW + sgm * 8]), qh + tt * qk_stride + sgm * 8, ok);
-            cp_async16(smem_u32(&sm.v[b][r * ROW + sgm * 8]), vh + tt * v_stride + sgm * 8, ok);
+            cp_async16(smem_u32(&dst[r * ROW + sgm * 8]), src + (ok ? size_t(t) : 0) * stride + sgm * 8, ok);
         }
-        cp_async_commit();
     };
 
     // ---- state: warp w owns rows 16w..16w+15, all D columns (D/8 n-tiles)
@@ -177,11 +183,18 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
     }
 
-    const float *gh = g + size_t(bos) * h_v + h;
-    const float *bh = beta + size_t(bos) * h_v + h;
+    const float *gh = p.g[grp_i] + size_t(bos) * h_v + h;
+    const float *bh = p.beta[grp_i] + size_t(bos) * h_v + h;
     float g_next = 0.f, b_next = 0.f;
     if (nchunks > 0) {
-        load_chunk(0, 0);
+        stage(sm.k, kh, qk_stride, 0);
+        stage(sm.q, qh, qk_stride, 0);
+        stage(sm.v, vh, v_stride, 0);
+        if (SPLIT) {
+            stage(sm.kl, klh, qk_stride, 0);
+            stage(sm.vl, vlh, v_stride, 0);
+        }
+        cp_async_commit();
         if (tid < C && tid < len) {
             g_next = gh[size_t(tid) * h_v];
             b_next = bh[size_t(tid) * h_v];
@@ -189,8 +202,8 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     }
 
     for (int c = 0; c < nchunks; ++c) {
-        const int cur = c & 1;
         const int clen = min(C, len - c * C);
+        const bool more = c + 1 < nchunks;
         // ---- gates of this chunk: gamma = inclusive prefix sum of g (padding has g = beta = 0)
         if (tid < C) {
             sm.gam[tid] = g_next;
@@ -199,7 +212,6 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         cp_async_wait_all();
         __syncthreads();
         if (warp == 0) {
-            // inclusive scan of 64 values, two per lane
             float a0 = sm.gam[2 * lane], a1 = sm.gam[2 * lane + 1];
             float pair = a0 + a1;
             float incl = pair;
@@ -212,18 +224,13 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             sm.gam[2 * lane] = excl + a0;
             sm.gam[2 * lane + 1] = excl + a0 + a1;
         }
-        // prefetch the next chunk (other buffer) while this one is processed
-        if (c + 1 < nchunks) {
-            load_chunk(c + 1, cur ^ 1);
+        if (more) {
             const int t = (c + 1) * C + tid;
             g_next = (tid < C && t < len) ? gh[size_t(t) * h_v] : 0.f;
             b_next = (tid < C && t < len) ? bh[size_t(t) * h_v] : 0.f;
         }
         __syncthreads();
 
-        const __nv_bfloat16 *Ks = sm.k[cur];
-        const __nv_bfloat16 *Qs = sm.q[cur];
-        const __nv_bfloat16 *Vs = sm.v[cur];
         const float gC = sm.gam[C - 1];
 
         // ---- (1)(2): A = strict-lower(beta_t e^{g_t-g_s} K K^T), P = lower(scale e^{g_t-g_s} Q K^T)
@@ -237,20 +244,28 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 for (int e = 0; e < 4; ++e) akk[j][e] = aqk[j][e] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                uint32_t ak[4], aq[4];
+                uint32_t ak[4], aq[4], akl[4];
                 const int arow = mb * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
-                ldsm_x4(ak, smem_u32(&Ks[arow * ROW + acol]));
-                ldsm_x4(aq, smem_u32(&Qs[arow * ROW + acol]));
+                ldsm_x4(ak, smem_u32(&sm.k[arow * ROW + acol]));
+                ldsm_x4(aq, smem_u32(&sm.q[arow * ROW + acol]));
+                if (SPLIT) ldsm_x4(akl, smem_u32(&sm.kl[arow * ROW + acol]));
 #pragma unroll
                 for (int np = 0; np < NPW / 2; ++np) {
-                    uint32_t b[4];
+                    uint32_t b[4], bl[4];
                     const int brow = (nt0 + 2 * np) * 8 + (lane & 7) + 8 * (lane >> 4);
                     const int bcol = kk * 16 + 8 * ((lane >> 3) & 1);
-                    ldsm_x4(b, smem_u32(&Ks[brow * ROW + bcol]));
+                    ldsm_x4(b, smem_u32(&sm.k[brow * ROW + bcol]));
                     mma16816(akk[2 * np], ak, b[0], b[1]);
                     mma16816(akk[2 * np + 1], ak, b[2], b[3]);
                     mma16816(aqk[2 * np], aq, b[0], b[1]);
                     mma16816(aqk[2 * np + 1], aq, b[2], b[3]);
+                    if (SPLIT) {
+                        ldsm_x4(bl, smem_u32(&sm.kl[brow * ROW + bcol]));
+                        mma16816(akk[2 * np], ak, bl[0], bl[1]);
+                        mma16816(akk[2 * np + 1], ak, bl[2], bl[3]);
+                        mma16816(akk[2 * np], akl, b[0], b[1]);
+                        mma16816(akk[2 * np + 1], akl, b[2], b[3]);
+                    }
                 }
             }
 #pragma unroll
@@ -288,10 +303,9 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
         __syncthreads();
         // off-diagonal blocks: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  The strictly upper
-        // blocks of Tf serve as scratch for the inner sums X_ij (stored at block (j, i)).
+        // blocks of Tf hold the inner sums X_ij (stored at block (j, i)).
         auto blk = [](int bi, int bj, int r, int cc) { return (16 * bi + r) * ROWA + 16 * bj + cc; };
         for (int level = 1; level <= 3; ++level) {
-            // X_ij for i - j == level
             for (int e = tid; e < (4 - level) * 256; e += NT) {
                 const int j = e >> 8, i = j + level, r = (e >> 4) & 15, cc = e & 15;
                 float acc = 0.f;
@@ -310,7 +324,7 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             }
             __syncthreads();
         }
-        // T1 = T diag(beta e^gamma), T2 = T diag(beta)  (bf16, lower triangle incl. diagonal)
+        // T1 = T diag(beta e^gamma), T2 = T diag(beta) as hi + lo bf16 (lower triangle incl. diagonal)
         for (int e = tid; e < C * C / 2; e += NT) {
             const int t = e / (C / 2), s = (e % (C / 2)) * 2;
             const float t0 = (s <= t) ? Tf[t * ROWA + s] : 0.f;
@@ -327,7 +341,7 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
         }
         __syncthreads();
 
-        // ---- (4) -W = -T1 K  -> smem;  Ut = T2 V -> registers (this warp's U tile)
+        // ---- (4) -W = -T1 K -> smem;  Ut = T2 V -> registers (this warp's U tile)
         const int mb = warp / WPM;
         const int n0 = (warp % WPM) * NCOL;
         const int arow4 = mb * 16 + (lane & 15);
@@ -346,14 +360,19 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 ldsm_x4(al, smem_u32(&sm.r3.s.t1l[arow4 * ROWP + acol]));
 #pragma unroll
                 for (int np = 0; np < NCOL / 16; ++np) {
-                    uint32_t bk[4];
+                    uint32_t bk[4], bkl[4];
                     const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
                     const int bcol = n0 + np * 16 + 8 * (lane >> 4);
-                    ldsm_x4_t(bk, smem_u32(&Ks[brow * ROW + bcol]));
+                    ldsm_x4_t(bk, smem_u32(&sm.k[brow * ROW + bcol]));
                     mma16816(acc_w[2 * np], ah, bk[0], bk[1]);
                     mma16816(acc_w[2 * np + 1], ah, bk[2], bk[3]);
                     mma16816(acc_w[2 * np], al, bk[0], bk[1]);
                     mma16816(acc_w[2 * np + 1], al, bk[2], bk[3]);
+                    if (SPLIT) {
+                        ldsm_x4_t(bkl, smem_u32(&sm.kl[brow * ROW + bcol]));
+                        mma16816(acc_w[2 * np], ah, bkl[0], bkl[1]);
+                        mma16816(acc_w[2 * np + 1], ah, bkl[2], bkl[3]);
+                    }
                 }
             }
 #pragma unroll
@@ -375,19 +394,30 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             ldsm_x4(al, smem_u32(&sm.r3.s.t2l[arow4 * ROWP + acol]));
 #pragma unroll
             for (int np = 0; np < NCOL / 16; ++np) {
-                uint32_t bv[4];
+                uint32_t bv[4], bvl[4];
                 const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
                 const int bcol = n0 + np * 16 + 8 * (lane >> 4);
-                ldsm_x4_t(bv, smem_u32(&Vs[brow * ROW + bcol]));
+                ldsm_x4_t(bv, smem_u32(&sm.v[brow * ROW + bcol]));
                 mma16816(acc_u[2 * np], ah, bv[0], bv[1]);
                 mma16816(acc_u[2 * np + 1], ah, bv[2], bv[3]);
                 mma16816(acc_u[2 * np], al, bv[0], bv[1]);
                 mma16816(acc_u[2 * np + 1], al, bv[2], bv[3]);
+                if (SPLIT) {
+                    ldsm_x4_t(bvl, smem_u32(&sm.vl[brow * ROW + bcol]));
+                    mma16816(acc_u[2 * np], ah, bvl[0], bvl[1]);
+                    mma16816(acc_u[2 * np + 1], ah, bvl[2], bvl[3]);
+                }
             }
         }
         __syncthreads();
+        // v (and its low part) are no longer read in this chunk: prefetch the next chunk's
+        if (more) {
+            stage(sm.v, vh, v_stride, c + 1);
+            if (SPLIT) stage(sm.vl, vlh, v_stride, c + 1);
+            cp_async_commit();
+        }
 
-        // ---- (5) U = Ut - W S_0^T ; store U and U diag(e^{gamma_C - gamma}) (bf16)
+        // ---- (5) U = Ut - W S_0^T ; store U and U diag(e^{gamma_C - gamma}) (hi + lo)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             uint32_t a[4];
@@ -431,7 +461,7 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 uint32_t a[4];
-                ldsm_x4(a, smem_u32(&Qs[(mb * 16 + (lane & 15)) * ROW + kk * 16 + (lane >> 4) * 8]));
+                ldsm_x4(a, smem_u32(&sm.q[(mb * 16 + (lane & 15)) * ROW + kk * 16 + (lane >> 4) * 8]));
 #pragma unroll
                 for (int np = 0; np < NCOL / 16; ++np) {
                     uint32_t b[4];
@@ -474,7 +504,11 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                         pack_bf16(acc_o[j][2], acc_o[j][3]);
             }
         }
-        __syncthreads();  // every warp is done reading sb before it is overwritten
+        __syncthreads();  // every warp is done reading sb and q
+        if (more) {
+            stage(sm.q, qh, qk_stride, c + 1);
+            cp_async_commit();
+        }
 
         // ---- (7) S_C = e^{gamma_C} S_0 + (U diag(e^{gamma_C-gamma}))^T K
         {
@@ -492,14 +526,19 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 ldsm_x4_t(al, smem_u32(&sm.r3.d.udl[arow * ROW + acol]));
 #pragma unroll
                 for (int np = 0; np < D / 16; ++np) {
-                    uint32_t b[4];
+                    uint32_t b[4], bl[4];
                     const int brow = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
                     const int bcol = np * 16 + 8 * (lane >> 4);
-                    ldsm_x4_t(b, smem_u32(&Ks[brow * ROW + bcol]));
+                    ldsm_x4_t(b, smem_u32(&sm.k[brow * ROW + bcol]));
                     mma16816(S[2 * np], ah, b[0], b[1]);
                     mma16816(S[2 * np + 1], ah, b[2], b[3]);
                     mma16816(S[2 * np], al, b[0], b[1]);
                     mma16816(S[2 * np + 1], al, b[2], b[3]);
+                    if (SPLIT) {
+                        ldsm_x4_t(bl, smem_u32(&sm.kl[brow * ROW + bcol]));
+                        mma16816(S[2 * np], ah, bl[0], bl[1]);
+                        mma16816(S[2 * np + 1], ah, bl[2], bl[3]);
+                    }
                 }
             }
             const int r0 = warp * 16 + grp;
@@ -510,11 +549,17 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 *reinterpret_cast<uint32_t *>(&sm.sb[(r0 + 8) * ROW + c0]) = pack_bf16(S[j][2], S[j][3]);
             }
         }
-        // the next iteration's first barrier orders these writes before any read
+        __syncthreads();  // k (and its low part) are free
+        if (more) {
+            stage(sm.k, kh, qk_stride, c + 1);
+            if (SPLIT) stage(sm.kl, klh, qk_stride, c + 1);
+            cp_async_commit();
+        }
     }
 
     // ---- final state
     {
+        float *s_out = p.s_out[grp_i];
         const int r0 = warp * 16 + grp;
 #pragma unroll
         for (int j = 0; j < D / 8; ++j) {
@@ -525,18 +570,14 @@ gdn_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     }
 }
 
-template <int D>
-cudaError_t launch_chunked(const sr_gdn_args &a, float scale, uint32_t *status, cudaStream_t st) {
-    const size_t smem = sizeof(Smem<D>);
-    cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int D, bool SPLIT>
+cudaError_t launch_chunked(const GdnBatch &b, int n_groups, int n_seqs, cudaStream_t st) {
+    const size_t smem = sizeof(Smem<D, SPLIT>);
+    cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(smem));
     if (e != cudaSuccess) return e;
-    dim3 grid(a.h_v, a.n_seqs);
-    gdn_chunk_kernel<D><<<grid, D * 2, smem, st>>>(
-        static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
-        static_cast<const __nv_bfloat16 *>(a.v), a.g, a.beta, a.cu_seqlens, a.h0,
-        static_cast<__nv_bfloat16 *>(a.o), a.s_out, a.total_tokens, a.max_seqlen, a.h_k, a.h_v, scale,
-        status);
+    dim3 grid(b.h_v, n_seqs, n_groups);
+    gdn_chunk_kernel<D, SPLIT><<<grid, D * 2, smem, st>>>(b);
     return cudaGetLastError();
 }
 
@@ -548,9 +589,32 @@ bool gdn_chunked_supported(const sr_gdn_args &a) {
 
 size_t gdn_scratch_bytes(const sr_gdn_args &) { return 0; }
 
+cudaError_t gdn_chunked_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st) {
+    if (n_seqs == 0 || b.h_v == 0 || n_groups == 0) return cudaSuccess;
+    if (d == 64) return split ? launch_chunked<64, true>(b, n_groups, n_seqs, st)
+                              : launch_chunked<64, false>(b, n_groups, n_seqs, st);
+    return split ? launch_chunked<128, true>(b, n_groups, n_seqs, st)
+                 : launch_chunked<128, false>(b, n_groups, n_seqs, st);
+}
+
 cudaError_t gdn_chunked(const sr_gdn_args &a, float scale, uint32_t *status, void *, cudaStream_t st) {
-    if (a.n_seqs == 0 || a.h_v == 0) return cudaSuccess;
-    return a.d_k == 64 ? launch_chunked<64>(a, scale, status, st) : launch_chunked<128>(a, scale, status, st);
+    GdnBatch b{};
+    b.q[0] = static_cast<const __nv_bfloat16 *>(a.q);
+    b.k[0] = static_cast<const __nv_bfloat16 *>(a.k);
+    b.v[0] = static_cast<const __nv_bfloat16 *>(a.v);
+    b.g[0] = a.g;
+    b.beta[0] = a.beta;
+    b.h0[0] = a.h0;
+    b.o[0] = static_cast<__nv_bfloat16 *>(a.o);
+    b.s_out[0] = a.s_out;
+    b.cu = a.cu_seqlens;
+    b.total = a.total_tokens;
+    b.max_len = a.max_seqlen;
+    b.h_k = a.h_k;
+    b.h_v = a.h_v;
+    b.scale = scale;
+    b.status = status;
+    return gdn_chunked_batch(b, 1, a.n_seqs, a.d_k, false, st);
 }
 
 size_t mamba2_scratch_bytes(const sr_mamba2_args &) { return 0; }

@@ -1,0 +1,378 @@
+// Persistent, warp-specialised tcgen05 GEMM for the replay group's dense
+// projections:  C[M, N] = A[M, K] * B[N, K]^T  (bf16 in, fp32 accumulate in
+// tensor memory), with the epilogue fused:
+//   EPI_STORE         C = A B^T                       bf16 out
+//   EPI_RESIDUAL      C = R + A B^T                   bf16 out
+//   EPI_SWIGLU        C = SiLU(r A Bg^T) * (r A Bu^T) bf16 out, optional lo part   (MLP gate/up)
+//   EPI_F32_ROWSCALE  C = r A B^T                     fp32 out                     (in_proj)
+//   EPI_F32_RESIDUAL  C += A B^T                      fp32 in place                (out_proj, down)
+// r is an optional fp32 per-row scale (the folded RMSNorm factor).  With two
+// passes the A operand is an exact hi + lo pair of bf16 matrices
+// (A = A_hi + A_lo) and both products accumulate into the same TMEM tile, so
+// the result carries ~16 mantissa bits of the activations: the weights are
+// exact bf16, so A_hi B^T + A_lo B^T is the product of the unrounded A.
+// Roles: warp 0 issues TMA loads (128-byte swizzle) into a 4-stage ring,
+// warp 1 allocates TMEM and issues tcgen05.mma (M=128, N=256, K=16) from one
+// thread, warps 2-5 drain the double-buffered TMEM accumulator (2 x 256
+// columns) with tcgen05.ld and apply the epilogue while the next tile's MMAs
+// run.  Tiles walk M fastest so CTAs running together share the weight tile
+// through L2.  Several problems with identical shapes (one per replay group)
+// are scheduled as one launch.  Every mbarrier wait is bounded; on timeout
+// the kernel records SR_DEV_TIMEOUT, drains its MMAs, frees TMEM and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace sr {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kTileA = BM * BK * 2;  // 16 KB
+constexpr int kTileB = BN * BK * 2;  // 32 KB
+constexpr int kThreads = 192;
+constexpr int kSmemBytes = STAGES * (kTileA + kTileB) + 1024 /*align*/ + 256 /*barriers*/;
+
+struct Problem {
+    CUtensorMap a;   // [M, K], box {64, 128}
+    CUtensorMap a_lo;  // [M, K] low part of A (second pass), box {64, 128}
+    CUtensorMap b0;  // [N, K] box {64, 256}; gate [N, K] box {64, 128} for SwiGLU
+    CUtensorMap b1;  // up [N, K] box {64, 128} (SwiGLU only)
+    void *c;
+    const __nv_bfloat16 *r;
+    __nv_bfloat16 *c_lo;     // SwiGLU: low part of the output (may be null)
+    const float *rowscale;   // per-row scale (may be null)
+};
+
+struct Params {
+    Problem prob[kMaxGemmProblems];
+    int n_problems;
+    int M, N, K;  // N = output columns
+    int ldc;      // row pitch of C and R in elements
+    int m_tiles, n_tiles;
+    int epi;
+    int n_pass;  // 1: A; 2: A_hi then A_lo
+    uint32_t *status;
+};
+
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ float silu(float x) { return x / (1.f + __expf(-x)); }
+
+// Abort-aware bounded wait: gives up when another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort_flag) {
+    for (uint32_t i = 0; i < tc::kMaxPolls; ++i) {
+        if (tc::mbar_try_wait(bar, phase)) return true;
+        if ((i & 1023) == 1023 && *abort_flag) return false;
+    }
+    return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * kTileA;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + STAGES * kTileB);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&tfull[b], 1);
+            tc::mbar_init(&tempty[b], 4);
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < p.n_problems; ++i) {
+            tc::prefetch_tmap(&p.prob[i].a);
+            if (p.n_pass == 2) tc::prefetch_tmap(&p.prob[i].a_lo);
+            tc::prefetch_tmap(&p.prob[i].b0);
+            if (p.epi == EPI_SWIGLU) tc::prefetch_tmap(&p.prob[i].b1);
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int tiles_per_prob = p.m_tiles * p.n_tiles;
+    const int total = p.n_problems * tiles_per_prob;
+    const int kblocks = p.K / BK;
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(p.status, SR_DEV_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                const int pi = tile / tiles_per_prob, rem = tile % tiles_per_prob;
+                const int nt = rem / p.m_tiles, mt = rem % p.m_tiles;
+                const Problem &pr = p.prob[pi];
+                for (int kk = 0; kk < p.n_pass * kblocks; ++kk) {
+                    const int kb = kk % kblocks;
+                    if (!wait_or_abort(&empty[stage], phase ^ 1, abort_flag)) { fail(); break; }
+                    tc::mbar_arrive_expect_tx(&full[stage], kTileA + kTileB);
+                    tc::tma_load_2d(sA + stage * kTileA, kk < kblocks ? &pr.a : &pr.a_lo, &full[stage], kb * BK,
+                                    mt * BM);
+                    if (p.epi == EPI_SWIGLU) {
+                        tc::tma_load_2d(sB + stage * kTileB, &pr.b0, &full[stage], kb * BK, nt * (BN / 2));
+                        tc::tma_load_2d(sB + stage * kTileB + (BN / 2) * BK * 2, &pr.b1, &full[stage], kb * BK,
+                                        nt * (BN / 2));
+                    } else {
+                        tc::tma_load_2d(sB + stage * kTileB, &pr.b0, &full[stage], kb * BK, nt * BN);
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                if (!wait_or_abort(&tempty[acc], acc_phase ^ 1, abort_flag)) { fail(); break; }
+                tc::tc_fence_after();
+                const uint32_t d = tmem + uint32_t(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < p.n_pass * kblocks; ++kb) {
+                    if (!wait_or_abort(&full[stage], phase, abort_flag)) { fail(); ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint32_t a0 = tc::smem_u32(sA + stage * kTileA);
+                    const uint32_t b0 = tc::smem_u32(sB + stage * kTileB);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc::mma_bf16_ss(d, tc::sdesc_k_sw128(a0 + k * 32), tc::sdesc_k_sw128(b0 + k * 32), idesc,
+                                        (kb | k) != 0);
+                    tc::mma_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc::mma_commit(&tfull[acc]);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            // all MMAs issued by this thread complete before TMEM is released
+            tc::mma_commit(drain);
+            if (!tc::mbar_wait(drain, 0)) atomicOr(p.status, SR_DEV_TIMEOUT);
+        }
+    } else {
+        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            const int pi = tile / tiles_per_prob, rem = tile % tiles_per_prob;
+            const int nt = rem / p.m_tiles, mt = rem % p.m_tiles;
+            const Problem &pr = p.prob[pi];
+            if (!wait_or_abort(&tfull[acc], acc_phase, abort_flag)) { fail(); break; }
+            tc::tc_fence_after();
+            const int row = mt * BM + quad * 32 + lane;
+            const bool row_ok = row < p.M;
+            const uint32_t tbase = tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN);
+            const float rs = (pr.rowscale && row_ok) ? pr.rowscale[row] : 1.f;
+            if (p.epi == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < BN / 2; c += 32) {
+                    uint32_t g[32], u[32];
+                    tc::tmem_ld_32x32b_x32(tbase + c, g);
+                    tc::tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
+                    tc::tmem_ld_wait();
+                    const int col = nt * (BN / 2) + c;
+                    const int nvec = min(4, (p.N - col) / 8);  // 8-column groups in range
+                    if (row_ok && nvec > 0) {
+                        __nv_bfloat16 *cb = static_cast<__nv_bfloat16 *>(pr.c);
+                        uint4 *dst = reinterpret_cast<uint4 *>(cb + size_t(row) * p.ldc + col);
+                        uint4 *dlo = pr.c_lo ? reinterpret_cast<uint4 *>(pr.c_lo + size_t(row) * p.ldc + col) : nullptr;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            if (v >= nvec) break;
+                            uint32_t w[4], wl[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = v * 8 + e * 2;
+                                const float h0 = silu(rs * __uint_as_float(g[j])) * (rs * __uint_as_float(u[j]));
+                                const float h1 = silu(rs * __uint_as_float(g[j + 1])) * (rs * __uint_as_float(u[j + 1]));
+                                w[e] = pack2(h0, h1);
+                                wl[e] = pack2(h0 - bf_lo(w[e]), h1 - bf_hi(w[e]));
+                            }
+                            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                            if (dlo) dlo[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                        }
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t x[32];
+                    tc::tmem_ld_32x32b_x32(tbase + c, x);
+                    tc::tmem_ld_wait();
+                    const int col = nt * BN + c;
+                    const int nvec = min(4, (p.N - col) / 8);
+                    if (!row_ok || nvec <= 0) continue;
+                    if (p.epi == EPI_F32_ROWSCALE || p.epi == EPI_F32_RESIDUAL) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(pr.c) + size_t(row) * p.ldc + col);
+                        const bool resid = p.epi == EPI_F32_RESIDUAL;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            if (v >= 2 * nvec) break;
+                            float4 o = make_float4(rs * __uint_as_float(x[4 * v]), rs * __uint_as_float(x[4 * v + 1]),
+                                                   rs * __uint_as_float(x[4 * v + 2]), rs * __uint_as_float(x[4 * v + 3]));
+                            if (resid) {
+                                const float4 rv = dst[v];
+                                o.x += rv.x; o.y += rv.y; o.z += rv.z; o.w += rv.w;
+                            }
+                            dst[v] = o;
+                        }
+                        continue;
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c) + size_t(row) * p.ldc + col);
+                    const uint4 *res = p.epi == EPI_RESIDUAL
+                                           ? reinterpret_cast<const uint4 *>(pr.r + size_t(row) * p.ldc + col)
+                                           : nullptr;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (v >= nvec) break;
+                        uint32_t rr[4] = {0u, 0u, 0u, 0u};
+                        if (res) {
+                            const uint4 rv = res[v];
+                            rr[0] = rv.x; rr[1] = rv.y; rr[2] = rv.z; rr[3] = rv.w;
+                        }
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = v * 8 + e * 2;
+                            w[e] = pack2(bf_lo(rr[e]) + rs * __uint_as_float(x[j]),
+                                         bf_hi(rr[e]) + rs * __uint_as_float(x[j + 1]));
+                        }
+                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+
+    if (*abort_flag) {
+        // let TMA copies already in flight land before the shared memory is released
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    // The driver entry point is looked up once per process.
+    static EncodeTiledFn fn = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            ptr = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix (row pitch `pitch`
+// elements), 64 x box_rows boxes with the 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(pitch) * 2};
+    cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+    cuuint32_t es[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 1;
+}
+
+}  // namespace
+
+cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
+                    int n_pass, uint32_t *status, cudaStream_t st) {
+    if (n_problems <= 0 || n_problems > kMaxGemmProblems || M <= 0 || N <= 0 || K <= 0 || K % BK != 0 ||
+        N % 8 != 0 || ldc % 8 != 0 || ldc < N || (n_pass != 1 && n_pass != 2))
+        return cudaErrorInvalidValue;
+    Params local{};
+    const int bn_out = epi == EPI_SWIGLU ? BN / 2 : BN;
+    for (int i = 0; i < n_problems; ++i) {
+        const GemmProblemDesc &d = probs[i];
+        if (!make_map(&local.prob[i].a, d.a, M, K, K, BM)) return cudaErrorInvalidValue;
+        if (n_pass == 2 && !make_map(&local.prob[i].a_lo, d.a_lo, M, K, K, BM)) return cudaErrorInvalidValue;
+        if (epi == EPI_SWIGLU) {
+            if (!make_map(&local.prob[i].b0, d.b0, N, K, K, BN / 2) ||
+                !make_map(&local.prob[i].b1, d.b1, N, K, K, BN / 2))
+                return cudaErrorInvalidValue;
+        } else if (!make_map(&local.prob[i].b0, d.b0, N, K, K, BN)) {
+            return cudaErrorInvalidValue;
+        }
+        local.prob[i].c = d.c;
+        local.prob[i].r = static_cast<const __nv_bfloat16 *>(d.r);
+        local.prob[i].c_lo = static_cast<__nv_bfloat16 *>(d.c_lo);
+        local.prob[i].rowscale = d.rowscale;
+    }
+    local.n_problems = n_problems;
+    local.M = M;
+    local.N = N;
+    local.K = K;
+    local.ldc = ldc;
+    local.m_tiles = (M + BM - 1) / BM;
+    local.n_tiles = (N + bn_out - 1) / bn_out;
+    local.epi = epi;
+    local.n_pass = n_pass;
+    local.status = status;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int total = n_problems * local.m_tiles * local.n_tiles;
+    const int grid = total < sm_count() ? total : sm_count();
+    gemm_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(local);
+    return cudaGetLastError();
+}
+
+}  // namespace sr

@@ -15,9 +15,96 @@ size_t gdn_scratch_bytes(const sr_gdn_args &a);
 cudaError_t gdn_chunked(const sr_gdn_args &a, float scale, uint32_t *status, void *scratch,
                         cudaStream_t st);
 
+// Chunked replay of several independent problems (replay groups) in one
+// launch: grid = (h_v, n_seqs, n_groups); all groups share cu_seqlens and shapes.
+constexpr int kMaxGroups = 8;
+struct GdnBatch {
+    const __nv_bfloat16 *q[kMaxGroups];
+    const __nv_bfloat16 *k[kMaxGroups];
+    const __nv_bfloat16 *v[kMaxGroups];
+    const __nv_bfloat16 *k_lo[kMaxGroups];  // low parts (split precision), else unused
+    const __nv_bfloat16 *v_lo[kMaxGroups];
+    const float *g[kMaxGroups];
+    const float *beta[kMaxGroups];
+    const float *h0[kMaxGroups];      // may be null
+    __nv_bfloat16 *o[kMaxGroups];     // may be null
+    float *s_out[kMaxGroups];
+    const int32_t *cu;
+    int total, max_len, h_k, h_v;
+    float scale;
+    uint32_t *status;
+};
+cudaError_t gdn_chunked_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st);
+
+// Layer kernels of a replay group (layer_kernels.cu).  Arrays are indexed by group.
+struct RowPrepBatch {
+    const void *x[kMaxGroups];            // [T, H] fp32 (x_f32) or bf16
+    const __nv_bfloat16 *w[kMaxGroups];   // [H] norm weight
+    __nv_bfloat16 *a_hi[kMaxGroups];      // [T, H] x * w (hi part)
+    __nv_bfloat16 *a_lo[kMaxGroups];      // [T, H] low part, may be null
+    float *r[kMaxGroups];                 // [T] 1 / sqrt(mean(x^2) + eps)
+    float *x32_out[kMaxGroups];           // [T, H] fp32 copy of x, may be null
+    int T, H, x_f32;
+    float eps;
+};
+cudaError_t row_prep(const RowPrepBatch &b, int n_groups, cudaStream_t st);
+
+struct ConvBatch {
+    const float *p[kMaxGroups];            // [T, ld] fp32 in_proj output
+    const __nv_bfloat16 *conv_w[kMaxGroups];  // [conv_dim, 4]
+    const float *a_log[kMaxGroups];
+    const float *dt_bias[kMaxGroups];
+    __nv_bfloat16 *q[kMaxGroups];          // [T, h_k, 128]
+    __nv_bfloat16 *k[kMaxGroups];
+    __nv_bfloat16 *k_lo[kMaxGroups];       // may be null
+    __nv_bfloat16 *v[kMaxGroups];          // [T, h_v, 128]
+    __nv_bfloat16 *v_lo[kMaxGroups];       // may be null
+    float *gate[kMaxGroups];               // [T, h_v]
+    float *beta[kMaxGroups];
+    __nv_bfloat16 *conv_out[kMaxGroups];   // [n_seqs, conv_dim, 3]
+    const int32_t *cu;
+    int n_seqs, T, ld, h_k, h_v, conv_dim, b_off;  // b_off: column of b (a follows at + h_v)
+};
+cudaError_t conv_gates(const ConvBatch &b, int n_groups, cudaStream_t st);
+
+struct GatedNormBatch {
+    const __nv_bfloat16 *o[kMaxGroups];   // [T, h_v, 128]
+    const float *p[kMaxGroups];           // [T, ld] (z at column z_off)
+    const __nv_bfloat16 *w[kMaxGroups];   // [128]
+    __nv_bfloat16 *y_hi[kMaxGroups];      // [T, h_v * 128]
+    __nv_bfloat16 *y_lo[kMaxGroups];      // may be null
+    int T, h_v, ld, z_off;
+    float eps;
+};
+cudaError_t gated_norm(const GatedNormBatch &b, int n_groups, cudaStream_t st);
+
+struct CastBatch {
+    const float *src[kMaxGroups];
+    __nv_bfloat16 *dst[kMaxGroups];
+    size_t n;  // elements per group, multiple of 4
+};
+cudaError_t to_bf16(const CastBatch &b, int n_groups, cudaStream_t st);
+
 // Mamba2 replay.
 cudaError_t mamba2_sequential(const sr_mamba2_args &a, uint32_t *status, cudaStream_t st);
 size_t mamba2_scratch_bytes(const sr_mamba2_args &a);
 cudaError_t mamba2_replay(const sr_mamba2_args &a, uint32_t *status, void *scratch, cudaStream_t st);
+
+// Dense projections on tcgen05 (gemm_tc.cu).  C[M,N] = A[M,K] B[N,K]^T with
+// a fused epilogue; all problems of one call share M, N, K and the epilogue.
+enum GemmEpilogue { EPI_STORE = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_F32_ROWSCALE = 3, EPI_F32_RESIDUAL = 4 };
+constexpr int kMaxGemmProblems = 8;
+struct GemmProblemDesc {
+    const void *a;   // [M, K] bf16, row pitch K
+    const void *a_lo;  // [M, K] bf16 low part of A (two-pass GEMMs), else unused
+    const void *b0;  // [N, K] bf16 (SwiGLU: gate)
+    const void *b1;  // [N, K] bf16 (SwiGLU: up), else unused
+    void *c;         // [M, ldc] bf16
+    const void *r;   // residual [M, ldc] bf16 (EPI_RESIDUAL), may equal c
+    void *c_lo;      // SwiGLU low-part output [M, ldc] bf16, may be null
+    const float *rowscale;  // [M] fp32 per-row scale, may be null (= 1)
+};
+cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
+                    int n_pass, uint32_t *status, cudaStream_t st);
 
 }  // namespace sr

@@ -1,0 +1,259 @@
+// Elementwise / reduction kernels of a replay-group layer (HBM-bound; one
+// launch covers every replay group of the call through per-group pointers).
+//
+//   row_prep     A = x * w (as an exact hi + lo bf16 pair when split) and the
+//                RMSNorm factor r_t = 1/sqrt(mean(x_t^2) + eps); the GEMM that
+//                consumes A applies r_t in its epilogue, so RMSNorm(x) w W^T is
+//                formed without rounding the normalised activations.
+//   conv_gates   causal depthwise conv (width 4, zero left padding per
+//                sequence) + SiLU over [q|k|v], per-head L2 norm of q and k,
+//                g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b).
+//   conv_state   the last (width-1) pre-conv rows of each sequence.
+//   gated_norm   y = RMSNorm_head(o) w_g * SiLU(z) (hi + lo when split).
+//   to_bf16      fp32 residual stream -> bf16 hidden output.
+// The layer math is the Qwen3.5-family Gated DeltaNet block ("Tail-Replay",
+// Sec. 2 names Gated DeltaNet as the linear layer of the hybrids replayed).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sr {
+
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ void split2(float a, float b, __nv_bfloat162 &hi, __nv_bfloat162 &lo) {
+    hi = __floats2bfloat162_rn(a, b);
+    const float2 h = __bfloat1622float2(hi);
+    lo = __floats2bfloat162_rn(a - h.x, b - h.y);
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float softplusf_(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+
+// ---------------------------------------------------------------- row_prep
+// One warp per row.  H % 8 == 0.
+__global__ void __launch_bounds__(256) row_prep_kernel(const __grid_constant__ RowPrepBatch p) {
+    const int g = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= p.T) return;
+    const int H = p.H;
+    const size_t base = size_t(row) * H;
+    float ss = 0.f;
+    for (int c = lane * 8; c < H; c += 256) {
+        float xv[8];
+        if (p.x_f32) {
+            const float4 *xs = reinterpret_cast<const float4 *>(static_cast<const float *>(p.x[g]) + base + c);
+            const float4 a = xs[0], b = xs[1];
+            xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w; xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
+        } else {
+            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x[g]) + base + c);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                xv[2 * e] = f.x;
+                xv[2 * e + 1] = f.y;
+            }
+        }
+        const uint4 wu = *reinterpret_cast<const uint4 *>(p.w[g] + c);
+        const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&wu);
+        __nv_bfloat162 hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            ss = fmaf(xv[2 * e], xv[2 * e], ss);
+            ss = fmaf(xv[2 * e + 1], xv[2 * e + 1], ss);
+            const float2 wf = __bfloat1622float2(w2[e]);
+            split2(xv[2 * e] * wf.x, xv[2 * e + 1] * wf.y, hi[e], lo[e]);
+        }
+        *reinterpret_cast<uint4 *>(p.a_hi[g] + base + c) = *reinterpret_cast<uint4 *>(hi);
+        if (p.a_lo[g]) *reinterpret_cast<uint4 *>(p.a_lo[g] + base + c) = *reinterpret_cast<uint4 *>(lo);
+        if (p.x32_out[g]) {
+            float4 *d = reinterpret_cast<float4 *>(p.x32_out[g] + base + c);
+            d[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+            d[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) p.r[g][row] = 1.f / sqrtf(ss / float(H) + p.eps);
+}
+
+// ---------------------------------------------------------------- conv_gates
+constexpr int kConvTok = 32;  // tokens per CTA
+
+// Index n of the sequence holding token t (cu non-decreasing, cu[0] = 0).
+__device__ __forceinline__ int seq_of(const int32_t *cu, int n_seqs, int t) {
+    int lo = 0, hi = n_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cu[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// blockIdx.y < 2 h_k + h_v: one 128-channel head of [q|k|v] (thread = channel);
+// blockIdx.y == 2 h_k + h_v: the gates of kConvTok tokens.
+__global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__ ConvBatch p) {
+    const int g = blockIdx.z;
+    const int head = blockIdx.y;
+    const int t0 = blockIdx.x * kConvTok;
+    const int t1 = min(p.T, t0 + kConvTok);
+    const int tid = threadIdx.x;
+    const float *P = p.p[g];
+    const int n_qk = 2 * p.h_k;
+    if (head == n_qk + p.h_v) {
+        // gates: b at column b_off + h, a at column b_off + h_v + h
+        for (int e = tid; e < (t1 - t0) * p.h_v; e += blockDim.x) {
+            const int t = t0 + e / p.h_v, h = e % p.h_v;
+            const float b = P[size_t(t) * p.ld + p.b_off + h];
+            const float a = P[size_t(t) * p.ld + p.b_off + p.h_v + h];
+            p.gate[g][size_t(t) * p.h_v + h] = -expf(p.a_log[g][h]) * softplusf_(a + p.dt_bias[g][h]);
+            p.beta[g][size_t(t) * p.h_v + h] = sigmoidf_(b);
+        }
+        return;
+    }
+    const int D = 128;
+    const int ch = head * D + tid;
+    const __nv_bfloat16 *cw = p.conv_w[g] + size_t(ch) * 4;
+    const float w0 = __bfloat162float(cw[0]), w1 = __bfloat162float(cw[1]);
+    const float w2 = __bfloat162float(cw[2]), w3 = __bfloat162float(cw[3]);
+    __shared__ float red[4];
+    int n = seq_of(p.cu, p.n_seqs, t0);
+    int bos = max(p.cu[n], 0), eos = p.cu[n + 1];
+    // sliding window of the 3 previous pre-conv values (zero before the sequence start)
+    float x1 = (t0 - 1 >= bos) ? P[size_t(t0 - 1) * p.ld + ch] : 0.f;
+    float x2 = (t0 - 2 >= bos) ? P[size_t(t0 - 2) * p.ld + ch] : 0.f;
+    float x3 = (t0 - 3 >= bos) ? P[size_t(t0 - 3) * p.ld + ch] : 0.f;
+    for (int t = t0; t < t1; ++t) {
+        while (t >= eos && n + 1 < p.n_seqs) {  // next sequence (skips empty ones): the window restarts at zero
+            ++n;
+            bos = max(p.cu[n], 0);
+            eos = p.cu[n + 1];
+            x1 = x2 = x3 = 0.f;
+        }
+        const float x0 = P[size_t(t) * p.ld + ch];
+        float c = w0 * x3 + w1 * x2 + w2 * x1 + w3 * x0;
+        c = c * sigmoidf_(c);
+        x3 = x2;
+        x2 = x1;
+        x1 = x0;
+        if (head < n_qk) {
+            // per-head L2 norm over the 128 channels of this CTA
+            float ss = warp_sum(c * c);
+            if ((tid & 31) == 0) red[tid >> 5] = ss;
+            __syncthreads();
+            ss = red[0] + red[1] + red[2] + red[3];
+            __syncthreads();
+            c = c / sqrtf(ss + 1e-6f);
+        }
+        if (head < p.h_k) {
+            p.q[g][size_t(t) * p.h_k * D + ch] = __float2bfloat16_rn(c);
+        } else if (head < n_qk) {
+            const size_t o = size_t(t) * p.h_k * D + (ch - p.h_k * D);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(c);
+            p.k[g][o] = hi;
+            if (p.k_lo[g]) p.k_lo[g][o] = __float2bfloat16_rn(c - __bfloat162float(hi));
+        } else {
+            const size_t o = size_t(t) * p.h_v * D + (ch - n_qk * D);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(c);
+            p.v[g][o] = hi;
+            if (p.v_lo[g]) p.v_lo[g][o] = __float2bfloat16_rn(c - __bfloat162float(hi));
+        }
+    }
+}
+
+// conv_state[n, ch, j] = pre-conv row (eos - W + 1 + j) of sequence n, 0 before its start.
+__global__ void __launch_bounds__(128) conv_state_kernel(const __grid_constant__ ConvBatch p) {
+    const int g = blockIdx.z, n = blockIdx.x;
+    const int ch = blockIdx.y * 128 + threadIdx.x;
+    if (ch >= p.conv_dim) return;
+    const int bos = max(p.cu[n], 0), eos = min(p.cu[n + 1], p.T);
+    __nv_bfloat16 *out = p.conv_out[g] + (size_t(n) * p.conv_dim + ch) * 3;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int t = eos - 3 + j;
+        out[j] = __float2bfloat16_rn(t >= bos ? p.p[g][size_t(t) * p.ld + ch] : 0.f);
+    }
+}
+
+// ---------------------------------------------------------------- gated_norm
+// One warp per (token, V head); d = 128 (4 values per lane).
+__global__ void __launch_bounds__(256) gated_norm_kernel(const __grid_constant__ GatedNormBatch p) {
+    const int g = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x * 8 + warp;  // t * h_v + h
+    if (item >= p.T * p.h_v) return;
+    const int t = item / p.h_v, h = item % p.h_v;
+    const int c = lane * 4;
+    const uint2 ou = *reinterpret_cast<const uint2 *>(p.o[g] + size_t(item) * 128 + c);
+    const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ou);
+    const float2 oa = __bfloat1622float2(o2[0]), ob = __bfloat1622float2(o2[1]);
+    const float ov[4] = {oa.x, oa.y, ob.x, ob.y};
+    const float ss = warp_sum(ov[0] * ov[0] + ov[1] * ov[1] + ov[2] * ov[2] + ov[3] * ov[3]);
+    const float r = 1.f / sqrtf(ss / 128.f + p.eps);
+    const float4 z = *reinterpret_cast<const float4 *>(p.p[g] + size_t(t) * p.ld + p.z_off + h * 128 + c);
+    const float zv[4] = {z.x, z.y, z.z, z.w};
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        y[e] = ov[e] * r * __bfloat162float(p.w[g][c + e]) * (zv[e] * sigmoidf_(zv[e]));
+    __nv_bfloat162 hi[2], lo[2];
+    split2(y[0], y[1], hi[0], lo[0]);
+    split2(y[2], y[3], hi[1], lo[1]);
+    *reinterpret_cast<uint2 *>(p.y_hi[g] + size_t(item) * 128 + c) = *reinterpret_cast<uint2 *>(hi);
+    if (p.y_lo[g]) *reinterpret_cast<uint2 *>(p.y_lo[g] + size_t(item) * 128 + c) = *reinterpret_cast<uint2 *>(lo);
+}
+
+// ---------------------------------------------------------------- to_bf16
+__global__ void __launch_bounds__(256) to_bf16_kernel(const __grid_constant__ CastBatch p) {
+    const int g = blockIdx.y;
+    const size_t i = (size_t(blockIdx.x) * 256 + threadIdx.x) * 4;
+    if (i >= p.n) return;
+    const float4 v = *reinterpret_cast<const float4 *>(p.src[g] + i);
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p.dst[g] + i) = u;
+}
+
+}  // namespace
+
+cudaError_t row_prep(const RowPrepBatch &b, int n_groups, cudaStream_t st) {
+    if (b.T == 0) return cudaSuccess;
+    dim3 grid((b.T + 7) / 8, n_groups);
+    row_prep_kernel<<<grid, 256, 0, st>>>(b);
+    return cudaGetLastError();
+}
+
+cudaError_t conv_gates(const ConvBatch &b, int n_groups, cudaStream_t st) {
+    if (b.T == 0) return cudaSuccess;
+    dim3 grid((b.T + kConvTok - 1) / kConvTok, 2 * b.h_k + b.h_v + 1, n_groups);
+    conv_gates_kernel<<<grid, 128, 0, st>>>(b);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || b.n_seqs == 0) return e;
+    dim3 g2(b.n_seqs, (b.conv_dim + 127) / 128, n_groups);
+    conv_state_kernel<<<g2, 128, 0, st>>>(b);
+    return cudaGetLastError();
+}
+
+cudaError_t gated_norm(const GatedNormBatch &b, int n_groups, cudaStream_t st) {
+    if (b.T == 0) return cudaSuccess;
+    dim3 grid((b.T * b.h_v + 7) / 8, n_groups);
+    gated_norm_kernel<<<grid, 256, 0, st>>>(b);
+    return cudaGetLastError();
+}
+
+cudaError_t to_bf16(const CastBatch &b, int n_groups, cudaStream_t st) {
+    if (b.n == 0) return cudaSuccess;
+    dim3 grid(unsigned((b.n / 4 + 255) / 256), n_groups);
+    to_bf16_kernel<<<grid, 256, 0, st>>>(b);
+    return cudaGetLastError();
+}
+
+}  // namespace sr

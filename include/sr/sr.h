@@ -76,6 +76,7 @@ typedef enum sr_dtype { SR_BF16 = 0, SR_FP32 = 1 } sr_dtype;
 /* Device status word flags (sr_device_status). */
 #define SR_DEV_BAD_CU_SEQLENS 0x1u  /* cu[n] > cu[n+1], cu[n+1] > total, cu[0] != 0 */
 #define SR_DEV_SEQ_TOO_LONG 0x2u    /* a sequence is longer than max_seqlen       */
+#define SR_DEV_TIMEOUT 0x4u         /* a bounded on-chip wait gave up (kernel exited early) */
 
 /* Kernel selection for sr_gdn_replay. */
 typedef enum sr_gdn_algo {
@@ -187,8 +188,10 @@ SR_API sr_status sr_mamba2_replay(const sr_mamba2_args *args, void *workspace, s
  * same cu_seqlens (one request's suffix seen by every group).
  *
  * Shapes: proj_dim = 2 h_k d_k + 2 h_v d_v + 2 h_v, conv_dim = 2 h_k d_k + h_v d_v.
- * Supported: hidden % 64 == 0, inter % 128 == 0, d_k = d_v = 128,
- * conv_width = 4, (h_v d_v) % 64 == 0.
+ * Supported: n_groups <= 8, d_k = d_v = 128, conv_width = 4, hidden % 64 == 0,
+ * inter % 64 == 0, (h_v d_v) % 64 == 0, h_v % h_k == 0.  Workspace: the size
+ * sr_group_replay_workspace() returns (it grows linearly with total_tokens
+ * and n_groups; about 150 KB per token per group at hidden 2560).
  * ---------------------------------------------------------------------- */
 typedef struct sr_layer_weights {
     const void *w_in_norm;   /* [hidden] bf16 */
@@ -213,6 +216,18 @@ typedef struct sr_layer_outputs {
 
 typedef enum sr_group_mode { SR_MODE_SKIP = 0, SR_MODE_FULL = 1 } sr_group_mode;
 
+/* Arithmetic of the group's activations.
+ * SR_PREC_SPLIT (default): the residual stream, the in_proj output and the
+ *   gates are fp32; every activation operand of a tensor-core product (the
+ *   normalised hidden, the gated-norm output, the SwiGLU output, k and v) is
+ *   carried as an exact pair of bf16 matrices hi + lo, so each projection runs
+ *   two bf16 MMA passes (the weights are exact bf16).  The states then track
+ *   the fp64 layer math to ~1e-4 of max|S| over a 3-layer group.
+ * SR_PREC_BF16: one pass per projection with bf16 activations (the usual bf16
+ *   serving arithmetic); about half the tensor-core work, state error a few
+ *   1e-3 of max|S| after three layers. */
+typedef enum sr_group_precision { SR_PREC_SPLIT = 0, SR_PREC_BF16 = 1 } sr_group_precision;
+
 typedef struct sr_group_args {
     const void *const *anchors;       /* host array [n_groups] of device [total_tokens, hidden] bf16 */
     const int32_t *cu_seqlens;
@@ -223,6 +238,7 @@ typedef struct sr_group_args {
     int32_t hidden, inter, h_k, h_v, d_k, d_v, conv_width;
     float eps;
     int32_t mode;                     /* sr_group_mode */
+    int32_t precision;                /* sr_group_precision */
 } sr_group_args;
 
 SR_API size_t sr_group_replay_workspace(const sr_group_args *args);

@@ -110,3 +110,30 @@ def test_device_status_needs_workspace():
     flags = ctypes.c_uint32(0)
     st = sr.library().sr_device_status(None, None, ctypes.byref(flags))
     assert st == sr.SR_ERR_INVALID_ARG
+
+
+def test_ctypes_structs_match_the_c_header(tmp_path):
+    """The binding's ctypes structs have the C header's sizes and field offsets
+    (compiled here with gcc from include/sr/sr.h)."""
+    import os
+    import subprocess
+    structs = {"sr_gdn_args": sr.GdnArgs, "sr_mamba2_args": sr.Mamba2Args,
+               "sr_layer_weights": sr.LayerWeights, "sr_layer_outputs": sr.LayerOutputs,
+               "sr_group_args": sr.GroupArgs}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "sr/sr.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append("return 0; }")
+    src = tmp_path / "abi.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "abi"
+    inc = os.path.join(os.path.dirname(sr.HEADER_PATH), "..")
+    subprocess.run(["gcc", "-I", inc, str(src), "-o", str(exe)], check=True)
+    out = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                 check=True).stdout.splitlines())
+    for cname, py in structs.items():
+        assert int(out[cname]) == ctypes.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert int(out[f"{cname}.{f}"]) == getattr(py, f).offset, f"{cname}.{f}"

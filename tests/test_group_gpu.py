@@ -1,0 +1,110 @@
+"""GPU parity of sr_group_replay against the fp64 layer oracle.
+
+Covers: the full replay-group workload (3 GDN layers + SwiGLU MLPs,
+hidden 2560, 1638-token suffix) in skip mode; small ragged multi-sequence
+groups in full mode with every intermediate hidden checked; the fast bf16
+precision mode at its derived tolerance; and group-parallel replay (several
+groups in one call give exactly the per-group results)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import layers as OL
+import workloads as W
+from _util import OUT_TOL_BF16, STATE_TOL, assert_close
+
+pytestmark = pytest.mark.gpu
+
+# bf16 precision mode: every bf16 rounding of the hidden stream adds ~2^-9/sqrt(3)
+# relative error that the next layer's k, v and state inherit almost one to one
+# (three layers: a few 1e-3 of max|S|); the bound below allows 5x 2^-9 of max|S|.
+STATE_TOL_BF16_MODE = 1e-2
+
+
+@pytest.fixture(scope="module")
+def sr():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gated_deltanet_state_sr_b200 as m
+    return m
+
+
+class DevLayer:
+    def __init__(self, lw):
+        for f in ("w_in_norm", "w_in", "conv_w", "a_log", "dt_bias", "w_gnorm", "w_out", "w_post_norm",
+                  "w_gate", "w_up", "w_down"):
+            setattr(self, f, getattr(lw, f).cuda().contiguous())
+
+
+def run(sr, gis, mode, precision, want_hidden=False):
+    s = gis[0].shape
+    anchors = [gi.anchors.cuda().contiguous() for gi in gis]
+    weights = [[DevLayer(lw) for lw in gi.layers] for gi in gis]
+    cu = gis[0].cu_seqlens.cuda()
+    out = sr.group_replay(anchors, cu, weights, max_seqlen=max(max(gis[0].lengths), 1), hidden=s.hidden,
+                          inter=s.inter, h_k=s.h_k, h_v=s.h_v, d=s.d_k, eps=s.eps, mode=mode,
+                          precision=precision, want_hidden=want_hidden)
+    torch.cuda.synchronize()
+    return out
+
+
+def small_shape():
+    return W.LayerShape(hidden=256, inter=512, h_k=2, h_v=4, d_k=128, d_v=128)
+
+
+def check_group(out_g, ref, state_tol, mode, check_hidden):
+    L = len(ref)
+    for l in range(L):
+        s, c, h = out_g[l]
+        assert_close(s, ref[l]["S"], state_tol, f"layer {l} state")
+        for n in range(s.shape[0]):
+            if np.abs(ref[l]["S"][n]).max() > 0:
+                assert_close(s[n], ref[l]["S"][n], state_tol * 2, f"layer {l} seq {n} state")
+        assert_close(c, ref[l]["conv_state"], OUT_TOL_BF16, f"layer {l} conv state")
+        if check_hidden and h is not None:
+            assert_close(h, ref[l]["x_out"], OUT_TOL_BF16, f"layer {l} hidden")
+
+
+@pytest.mark.parametrize("mode", ["full", "skip"])
+def test_small_ragged_group_split_precision(sr, mode):
+    gi = W.group_inputs(31, [5, 1, 0, 70, 130, 2], n_layers=2, shape=small_shape())
+    m = sr.SR_MODE_FULL if mode == "full" else sr.SR_MODE_SKIP
+    out = run(sr, [gi], m, sr.SR_PREC_SPLIT, want_hidden=True)
+    ref = OL.group_replay(gi, mode)
+    check_group(out[0], ref, STATE_TOL, mode, True)
+    # an empty sequence leaves zero state
+    assert torch.all(out[0][0][0][2] == 0)
+
+
+def test_small_group_bf16_precision(sr):
+    gi = W.group_inputs(32, [100, 37], n_layers=3, shape=small_shape())
+    out = run(sr, [gi], sr.SR_MODE_FULL, sr.SR_PREC_BF16, want_hidden=True)
+    ref = OL.group_replay(gi, "full")
+    check_group(out[0], ref, STATE_TOL_BF16_MODE, "full", True)
+
+
+def test_group_parallel_equals_single(sr):
+    """Groups replay independently ("SuffixReplay", Algorithm Design 1: errors do
+    not cross group boundaries): a 3-group call gives each group's own result bit
+    for bit."""
+    s = small_shape()
+    gis = [W.group_inputs(40 + g, [33, 64, 1], n_layers=2, shape=s) for g in range(3)]
+    together = run(sr, gis, sr.SR_MODE_FULL, sr.SR_PREC_SPLIT, want_hidden=True)
+    for g in range(3):
+        alone = run(sr, [gis[g]], sr.SR_MODE_FULL, sr.SR_PREC_SPLIT, want_hidden=True)
+        for l in range(2):
+            for a, b in zip(together[g][l], alone[0][l]):
+                if a is not None:
+                    assert torch.equal(a, b), (g, l)
+    ref = OL.group_replay(gis[1], "full")
+    check_group(together[1], ref, STATE_TOL, "full", True)
+
+
+def test_full_group_workload(sr):
+    """The replay-group workload at full size: 3 layers, hidden 2560,
+    intermediate 9216, 16/32 heads, 1638-token suffix, skip mode."""
+    gi = W.group()
+    out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT)
+    ref = OL.group_replay(gi, "skip")
+    check_group(out[0], ref, STATE_TOL, "skip", False)
