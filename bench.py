@@ -203,10 +203,152 @@ class RawGdn:
             oracle.num_threads()
 
 
-WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn}
+
+class GroupReplay:
+    """Whole replay groups from anchors (sr_group_replay): one group of 3 GDN
+    layers + SwiGLU MLPs over a 1638-token suffix, or the 8-group whole-model
+    replay of a [GDN, GDN, GDN, FA] x 8 hybrid with suffix k = ceil(r m)."""
+
+    FULL_LAYER_MFLOP = None  # filled from shapes
+
+    def __init__(self, name, rank, precision="split"):
+        self.name = name
+        if name == "group":
+            self.gis = [W.group(seed=0x5EED0002 + 1000 * rank)]
+            self.desc = "one group: 3 GDN layers + SwiGLU MLP, hidden 2560, inter 9216, 1638-token suffix"
+        elif name.startswith("model_"):
+            _, m, r = name.split("_")
+            prefix = {"8k": 8192, "16k": 16384, "32k": 32768}[m]
+            ratio = {"5": 0.05, "10": 0.10}[r]
+            self.gis = [W.model_group(prefix, ratio, g, seed=0x5EED0003 + 1000 * rank) for g in range(8)]
+            self.desc = (f"whole model: [GDN,GDN,GDN,FA]x8, 8 groups replayed group-parallel, FA skipped, "
+                         f"suffix k = ceil({ratio} * {prefix}) = {W.model_suffix(prefix, ratio)}")
+        else:
+            raise ValueError(name)
+        self.precision = precision
+        s = self.gis[0].shape
+        self.s = s
+        self.G = len(self.gis)
+        self.L = len(self.gis[0].layers)
+        self.tokens = sum(self.gis[0].lengths)
+        T, H, I = self.tokens, s.hidden, s.inter
+        C = 64
+        self.flop = {  # algorithmic flops of one launch (all groups)
+            "gemm_in": 2.0 * T * H * s.proj_dim * self.G,
+            "gemm_out": 2.0 * T * s.v_dim * H * self.G,
+            "gemm_gateup": 2.0 * T * H * 2 * I * self.G,
+            "gemm_down": 2.0 * T * I * H * self.G,
+            "gdn": float(T) * s.h_v * 2 * (C * (3 * s.d_k + 2 * s.d_v) + 3 * s.d_k * s.d_v) * self.G,
+        }
+        full = (self.flop["gemm_in"] + self.flop["gemm_out"] + self.flop["gemm_gateup"] + self.flop["gemm_down"]
+                + self.flop["gdn"])
+        last = self.flop["gemm_in"] + self.flop["gdn"]
+        self.step_flop = (self.L - 1) * full + last  # skip mode
+        self.input_bytes = self.G * T * H * 2 + sum(
+            sum(getattr(lw, f).numel() * getattr(lw, f).element_size() for f in ("w_in", "w_out", "w_gate", "w_up",
+                                                                              "w_down"))
+            for gi in self.gis for lw in gi.layers)
+
+    launches_per_step = None  # counted from the profiler
+
+    def setup(self, sr, dev):
+        self.sr = sr
+        s = self.s
+        self.anchors = [gi.anchors.to(dev).contiguous() for gi in self.gis]
+        keys = ("w_in_norm", "w_in", "conv_w", "a_log", "dt_bias", "w_gnorm", "w_out", "w_post_norm", "w_gate",
+                "w_up", "w_down")
+
+        class L:
+            pass
+
+        self.weights = []
+        for gi in self.gis:
+            row = []
+            for lw in gi.layers:
+                o = L()
+                for k in keys:
+                    setattr(o, k, getattr(lw, k).to(dev).contiguous())
+                row.append(o)
+            self.weights.append(row)
+        self.cu = self.gis[0].cu_seqlens.to(dev)
+        self.max_len = max(self.gis[0].lengths)
+        self.kw = dict(max_seqlen=self.max_len, hidden=s.hidden, inter=s.inter, h_k=s.h_k, h_v=s.h_v, d=s.d_k,
+                       eps=s.eps, mode=sr.SR_MODE_SKIP,
+                       precision=sr.SR_PREC_SPLIT if self.precision == "split" else sr.SR_PREC_BF16)
+        self.outputs = sr.group_replay(self.anchors, self.cu, self.weights, **self.kw)
+        args = sr.group_args(self.anchors, self.cu, self.weights, self.outputs, **self.kw)
+        self.ws = sr.workspace(sr.group_workspace_bytes(args), dev)
+        self.prof = None
+        # pinned host buffers for the end-to-end leg
+        self.h_anchors = [gi.anchors.contiguous().pin_memory() for gi in self.gis]
+        self.h_cu = self.gis[0].cu_seqlens.contiguous().pin_memory()
+        self.h_out = [[(torch.empty(o[0].shape, dtype=o[0].dtype).pin_memory(),
+                        torch.empty(o[1].shape, dtype=o[1].dtype).pin_memory()) for o in row]
+                      for row in self.outputs]
+
+    def step(self, profile=None):
+        self.sr.group_replay(self.anchors, self.cu, self.weights, outputs=self.outputs, ws=self.ws,
+                             profile=profile, **self.kw)
+
+    def step_e2e(self):
+        for h, d in zip(self.h_anchors, self.anchors):
+            d.copy_(h, non_blocking=True)
+        self.cu.copy_(self.h_cu, non_blocking=True)
+        self.step()
+        for hrow, drow in zip(self.h_out, self.outputs):
+            for (hs, hc), (ds, dc, _) in zip(hrow, drow):
+                hs.copy_(ds, non_blocking=True)
+                hc.copy_(dc, non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.h_anchors) + self.h_cu.numel() * 4
+
+    @property
+    def d2h_bytes(self):
+        return sum(hs.numel() * 4 + hc.numel() * 2 for row in self.h_out for hs, hc in row)
+
+    def oracle_sample(self, stride=1, min_s=0.0, tokens=None):
+        """Bounded oracle run: the first layer (in_proj, conv, recurrence,
+        gated norm, out_proj, MLP) of group 0 over the first `tokens` tokens,
+        repeated until min_s seconds; scaled by algorithmic flops to the
+        tokens/s of the whole step."""
+        import numpy as np
+        import oracle
+        from oracle import layers as OL
+        gi = self.gis[0]
+        T = self.tokens if tokens is None else min(tokens, self.tokens)
+        x = oracle._f64(gi.anchors[:T])
+        cu = np.array([0, T])
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            OL.gdn_layer(x, gi.layers[0], cu, gi.shape)
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= min_s:
+                break
+        full_layer_flop_per_tok = sum(v for k, v in self.flop.items()) / self.G / self.tokens
+        sample_flop = full_layer_flop_per_tok * T * reps
+        step_flop_per_tok = self.step_flop / self.tokens
+        tok_per_s = sample_flop / dt / step_flop_per_tok
+        return tok_per_s, (f"group 0, layer 0 (full layer incl. MLP) over {T} tokens x {reps} reps in {dt:.1f} s, "
+                           f"scaled by algorithmic flops to the whole step "
+                           f"({step_flop_per_tok / 1e6:.0f} MFLOP per replayed token)"), oracle.num_threads()
+
+
+WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "group": GroupReplay,
+             **{f"model_{m}_{r}": GroupReplay for m in ("8k", "16k", "32k") for r in ("5", "10")}}
+DEFAULT_WORKLOAD = "model_32k_5"
 
 
 # ------------------------------------------------------------------ arms
+
+
+def make_workload(args, rank):
+    cls = WORKLOADS[args.workload]
+    if cls is GroupReplay:
+        return cls(args.workload, rank, precision=args.precision)
+    return cls(args.workload, rank)
 
 
 def dist_setup():
@@ -225,7 +367,7 @@ def run_ours(args):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
     import gated_deltanet_state_sr_b200 as sr
-    wl = WORKLOADS[args.workload](args.workload, rank)
+    wl = make_workload(args, rank)
     wl.setup(sr, dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -237,20 +379,23 @@ def run_ours(args):
     for _ in range(args.warmup):
         wl.step()
     barrier()
+    profiled = isinstance(wl, GroupReplay)
+    profs = [sr.LaunchProfiler(64) for _ in range(args.steps)] if profiled else None
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
         e0.record(stream)
-        for _ in range(args.steps):
-            wl.step()
+        for i in range(args.steps):
+            if profiled:
+                wl.step(profs[i])
+            else:
+                wl.step()
         e1.record(stream)
         barrier()
         # keep the GPU busy long enough for the clock sampler to see load
-        extra = 0
         t_end = time.perf_counter() + 0.6
         while time.perf_counter() < t_end:
             wl.step()
-            extra += 1
         torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
     if world > 1:
@@ -260,6 +405,23 @@ def run_ours(args):
     ms_per_step = ms / args.steps
     tokens_all = wl.tokens * world * args.steps
     value = tokens_all / (ms / 1e3)
+
+    # per-kernel device time inside the timed region (events on the launching stream)
+    kernels = None
+    launches = None
+    if profiled:
+        tot, cnt = {}, {}
+        launches = 0
+        for pr in profs:
+            for kind, t in pr.times():
+                launches += 2 if kind == "conv" else 1  # conv: conv_gates + conv_state kernels
+                tot[kind] = tot.get(kind, 0.0) + t
+                cnt[kind] = cnt.get(kind, 0) + 1
+        busy = sum(tot.values())
+        kernels = {k: {"ms_per_step": round(tot[k] / args.steps, 4), "launches_per_step": cnt[k] // args.steps,
+                       "share": round(tot[k] / busy, 4)} for k in sorted(tot, key=lambda k: -tot[k])}
+    else:
+        launches = wl.launches_per_step * args.steps
 
     # end-to-end through the C ABI with host buffers (copies inside the timed region)
     for _ in range(2):
@@ -280,21 +442,30 @@ def run_ours(args):
     e2e_value = wl.tokens * world * k_e2e / (ms_e2e / 1e3)
 
     peaks, src = load_peaks()
-    dom = wl.dominant()
-    kern_ms = ms_per_step  # the dominant kernel is the whole step for the raw workloads
-    if dom["bound"] == "tensor":
+    if profiled:
+        # dominant kernel: the kind with the most device time; algorithmic flops per
+        # launch over its average launch duration; timed inside a long step -> sustained peak
+        dom_kind = max((k for k in kernels if k in wl.flop), key=lambda k: kernels[k]["ms_per_step"])
+        per_launch_ms = kernels[dom_kind]["ms_per_step"] / kernels[dom_kind]["launches_per_step"]
+        achieved = wl.flop[dom_kind] / (per_launch_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roofline = {"kernel": f"gemm_tc_kernel ({dom_kind})" if dom_kind.startswith("gemm") else dom_kind,
+                    "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak_source": f"{src} (sustained bf16: kernel timed inside a long step)",
+                    "flop_per_launch": wl.flop[dom_kind], "ms_per_launch": round(per_launch_ms, 4),
+                    "mma_passes": 2 if wl.precision == "split" else 1,
+                    "step_tflops": round(wl.step_flop / (ms_per_step / 1e3) / 1e12, 2)}
+    else:
+        dom = wl.dominant()
+        kern_ms = ms_per_step  # the dominant kernel is the whole step for the raw workloads
         achieved = dom["flop"] / (kern_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops"]
-        unit = "TFLOP/s"
-    else:
-        achieved = dom["bytes"] / (kern_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
-    hbm_gbs = dom["bytes"] / (kern_ms / 1e3) / 1e9
-    roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": round(achieved, 2),
-                "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
-                "peak_source": src, "hbm_gbs": round(hbm_gbs, 1),
-                "hbm_frac": round(hbm_gbs / peaks["hbm_gbs"], 4)}
+        hbm_gbs = dom["bytes"] / (kern_ms / 1e3) / 1e9
+        roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": round(achieved, 2),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak_source": f"{src} (burst bf16)", "hbm_gbs": round(hbm_gbs, 1),
+                    "hbm_frac": round(hbm_gbs / peaks["hbm_gbs"], 4)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -307,15 +478,20 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, workloads.py)",
         "config": {"workload": args.workload, "desc": wl.desc, "tokens_per_step_per_gpu": wl.tokens,
+                   "precision": getattr(wl, "precision", "bf16 inputs"),
                    "l2": f"inputs {wl.input_bytes / 2**20:.0f} MiB > L2, no flush",
                    "parallelism": f"dp{world} (independent replays per GPU)"},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.h2d_bytes,
                 "d2h_bytes_per_step": wl.d2h_bytes},
-        "gpu_launches": wl.launches_per_step * args.steps,
+        "gpu_launches": launches,
         "roofline": roofline,
+        "kernels": kernels,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
     }
+    if isinstance(wl, GroupReplay):
+        line["per_group_ms"] = ms_per_step / wl.G
+        line["group_tokens_per_s"] = value * wl.G
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -327,12 +503,13 @@ def run_reference(args):
     world, rank, local = dist_setup()
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload](args.workload, 0)
+    wl = make_workload(args, 0)
+    kw = dict(stride=8) if isinstance(wl, RawGdn) else dict(tokens=96)
     for _ in range(args.warmup):
-        wl.oracle_sample(stride=8)
+        wl.oracle_sample(**kw)
     vals = []
     for _ in range(args.steps):
-        v, sample, cores = wl.oracle_sample(stride=8)
+        v, sample, cores = wl.oracle_sample(**kw)
         vals.append(v)
     value = statistics.mean(vals)
     line = {"impl": "reference", "metric": "replayed tokens/s", "value": value, "unit": "tokens/s",
@@ -352,7 +529,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="raw_qwen")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--precision", choices=["split", "bf16"], default="split",
+                    help="group workloads: hi/lo activations (parity-checked) or single-pass bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

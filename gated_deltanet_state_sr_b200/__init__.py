@@ -64,13 +64,21 @@ class LayerOutputs(ctypes.Structure):
     _fields_ = [("s_out", _vp), ("conv_out", _vp), ("hidden_out", _vp)]
 
 
+class Profile(ctypes.Structure):
+    _fields_ = [("events", ctypes.POINTER(_vp)), ("kinds", ctypes.POINTER(_i32)), ("capacity", _i32),
+                ("count", _i32)]
+
+
+KERNEL_KINDS = ["row_prep", "gemm_in", "conv", "gdn", "gated_norm", "gemm_out", "gemm_gateup", "gemm_down", "cast"]
+
+
 class GroupArgs(ctypes.Structure):
     _fields_ = [("anchors", ctypes.POINTER(_vp)), ("cu_seqlens", _vp),
                 ("weights", ctypes.POINTER(LayerWeights)), ("outputs", ctypes.POINTER(LayerOutputs)),
                 ("n_groups", _i32), ("n_layers", _i32), ("n_seqs", _i32), ("total_tokens", _i32),
                 ("max_seqlen", _i32), ("hidden", _i32), ("inter", _i32), ("h_k", _i32), ("h_v", _i32),
                 ("d_k", _i32), ("d_v", _i32), ("conv_width", _i32), ("eps", ctypes.c_float),
-                ("mode", _i32), ("precision", _i32)]
+                ("mode", _i32), ("precision", _i32), ("profile", ctypes.POINTER(Profile))]
 
 
 def _sig(name, restype, *argtypes):
@@ -301,7 +309,7 @@ _LAYER_FIELDS = [f for f, _ in LayerWeights._fields_]
 
 
 def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, inter, h_k, h_v, d=128,
-               conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT):
+               conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, profile=None):
     """Builds a GroupArgs (and keeps the ctypes arrays alive on it).
 
     anchors: list [G] of [T, hidden] bf16 CUDA tensors; weights: list [G] of
@@ -320,9 +328,29 @@ def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, int
     n = cu_seqlens.numel() - 1
     T = anchors[0].shape[0]
     a = GroupArgs(anc, cu_seqlens.data_ptr(), w_arr, o_arr, G, L, n, T, max_seqlen, hidden, inter, h_k, h_v,
-                  d, d, conv_width, float(eps), mode, precision)
-    a._keep = (anc, w_arr, o_arr)
+                  d, d, conv_width, float(eps), mode, precision,
+                  ctypes.pointer(profile.struct) if profile is not None else None)
+    a._keep = (anc, w_arr, o_arr, profile)
     return a
+
+
+class LaunchProfiler:
+    """CUDA events for sr_profile: per-launch device time of a group replay,
+    recorded on the launching stream."""
+
+    def __init__(self, capacity=256):
+        torch = _torch()
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.ev:  # torch creates the CUDA event lazily, at its first record
+            e.record()
+        self.handles = (_vp * (2 * capacity))(*[e.cuda_event for e in self.ev])
+        self.kinds = (_i32 * capacity)()
+        self.struct = Profile(self.handles, self.kinds, capacity, 0)
+
+    def times(self):
+        """[(kind name, ms)] of the last profiled call (events must have completed)."""
+        n = min(self.struct.count, self.struct.capacity)
+        return [(KERNEL_KINDS[self.kinds[i]], self.ev[2 * i].elapsed_time(self.ev[2 * i + 1])) for i in range(n)]
 
 
 def group_workspace_bytes(args: GroupArgs) -> int:
@@ -336,7 +364,7 @@ def group_call(args: GroupArgs, ws, stream=None) -> int:
 
 def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k, h_v, d=128, conv_width=4,
                  eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, want_hidden=False, outputs=None,
-                 ws=None, stream=None):
+                 ws=None, stream=None, profile=None):
     """Replays every group of the call (see sr_group_replay).  Returns the
     outputs list [G][L] of (s_out, conv_out, hidden_out or None)."""
     torch = _torch()
@@ -356,7 +384,8 @@ def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k
                             torch.empty(T, hidden, dtype=torch.bfloat16, device=dev) if keep_h else None))
             outputs.append(row)
     args = group_args(anchors, cu_seqlens, weights, outputs, max_seqlen=max_seqlen, hidden=hidden, inter=inter,
-                      h_k=h_k, h_v=h_v, d=d, conv_width=conv_width, eps=eps, mode=mode, precision=precision)
+                      h_k=h_k, h_v=h_v, d=d, conv_width=conv_width, eps=eps, mode=mode, precision=precision,
+                      profile=profile)
     need = group_workspace_bytes(args)
     if need == 0:
         _check(group_call(args, None))

@@ -120,6 +120,25 @@ sr_status validate(const sr_group_args *a) {
     return SR_OK;
 }
 
+// Records caller events around launches when profiling is on.
+struct Prof {
+    sr_profile *p;
+    cudaStream_t st;
+    int i = 0;
+    cudaError_t begin(int kind) {
+        if (!p || i >= p->capacity) return cudaSuccess;
+        p->kinds[i] = kind;
+        return cudaEventRecord(static_cast<cudaEvent_t>(p->events[2 * i]), st);
+    }
+    cudaError_t end() {
+        cudaError_t e = cudaSuccess;
+        if (p && i < p->capacity) e = cudaEventRecord(static_cast<cudaEvent_t>(p->events[2 * i + 1]), st);
+        ++i;
+        if (p) p->count = i;
+        return e;
+    }
+};
+
 #define SR_TRY(expr)                                                        \
     do {                                                                    \
         cudaError_t e_ = (expr);                                            \
@@ -159,6 +178,8 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
     }
     GroupBufs B[kMaxGroups];
     carve(m, static_cast<char *>(ws), B);
+    Prof prof{a->profile, st};
+    if (a->profile) a->profile->count = 0;
     const int G = m.G, T = m.T;
     const int npass = m.split ? 2 : 1;
 
@@ -179,13 +200,17 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             rp.x32_out[g] = l == 0 ? B[g].x32 : nullptr;
         }
         rp.T = T; rp.H = m.H; rp.x_f32 = l == 0 ? 0 : 1; rp.eps = a->eps;
+        SR_TRY(prof.begin(SR_K_ROW_PREP));
         SR_TRY(row_prep(rp, G, st));
+        SR_TRY(prof.end());
 
         // (2) p = r * (A W_in^T), fp32
         GemmProblemDesc gp[kMaxGemmProblems];
         for (int g = 0; g < G; ++g)
             gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_in, nullptr, B[g].p, nullptr, nullptr, B[g].r};
+        SR_TRY(prof.begin(SR_K_GEMM_IN));
         SR_TRY(gemm_tc(gp, G, T, m.proj, m.H, m.proj, EPI_F32_ROWSCALE, npass, status, st));
+        SR_TRY(prof.end());
 
         // (3) conv + SiLU + L2 norm + gates, conv state
         ConvBatch cb{};
@@ -205,7 +230,9 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         }
         cb.cu = a->cu_seqlens; cb.n_seqs = m.N; cb.T = T; cb.ld = m.proj; cb.h_k = m.hk; cb.h_v = m.hv;
         cb.conv_dim = m.conv_dim; cb.b_off = m.conv_dim + m.vd;
+        SR_TRY(prof.begin(SR_K_CONV));
         SR_TRY(conv_gates(cb, G, st));
+        SR_TRY(prof.end());
 
         // (4) gated-delta recurrence from a zero state
         GdnBatch gb{};
@@ -223,7 +250,9 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         }
         gb.cu = a->cu_seqlens; gb.total = T; gb.max_len = a->max_seqlen; gb.h_k = m.hk; gb.h_v = m.hv;
         gb.scale = 1.0f / sqrtf(float(m.d)); gb.status = status;
+        SR_TRY(prof.begin(SR_K_GDN));
         SR_TRY(gdn_chunked_batch(gb, G, m.N, m.d, m.split, st));
+        SR_TRY(prof.end());
         if (stop) break;
 
         // (5) y = RMSNorm_head(o) w_gnorm * SiLU(z) -> A (hi/lo)
@@ -236,12 +265,16 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             gn.y_lo[g] = B[g].a_lo;
         }
         gn.T = T; gn.h_v = m.hv; gn.ld = m.proj; gn.z_off = m.conv_dim; gn.eps = a->eps;
+        SR_TRY(prof.begin(SR_K_GATED_NORM));
         SR_TRY(gated_norm(gn, G, st));
+        SR_TRY(prof.end());
 
         // (6) x += y W_out^T
         for (int g = 0; g < G; ++g)
             gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_out, nullptr, B[g].x32, nullptr, nullptr, nullptr};
+        SR_TRY(prof.begin(SR_K_GEMM_OUT));
         SR_TRY(gemm_tc(gp, G, T, m.H, m.vd, m.H, EPI_F32_RESIDUAL, npass, status, st));
+        SR_TRY(prof.end());
 
         // (7) A = x * w_post_norm, r
         for (int g = 0; g < G; ++g) {
@@ -250,17 +283,23 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             rp.x32_out[g] = nullptr;
         }
         rp.x_f32 = 1;
+        SR_TRY(prof.begin(SR_K_ROW_PREP));
         SR_TRY(row_prep(rp, G, st));
+        SR_TRY(prof.end());
 
         // (8) h = SiLU(r A W_gate^T) * (r A W_up^T) (hi/lo)
         for (int g = 0; g < G; ++g)
             gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_gate, W(g).w_up, B[g].h_hi, nullptr, B[g].h_lo, B[g].r};
+        SR_TRY(prof.begin(SR_K_GEMM_GATEUP));
         SR_TRY(gemm_tc(gp, G, T, m.I, m.H, m.I, EPI_SWIGLU, npass, status, st));
+        SR_TRY(prof.end());
 
         // (9) x += h W_down^T
         for (int g = 0; g < G; ++g)
             gp[g] = GemmProblemDesc{B[g].h_hi, B[g].h_lo, W(g).w_down, nullptr, B[g].x32, nullptr, nullptr, nullptr};
+        SR_TRY(prof.begin(SR_K_GEMM_DOWN));
         SR_TRY(gemm_tc(gp, G, T, m.H, m.I, m.H, EPI_F32_RESIDUAL, npass, status, st));
+        SR_TRY(prof.end());
 
         // (10) optional bf16 copy of the hidden after this layer
         CastBatch cast{};
@@ -273,14 +312,18 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
                 cast.dst[g] = static_cast<__nv_bfloat16 *>(O(g).hidden_out);
             }
             cast.n = size_t(T) * m.H;
+            SR_TRY(prof.begin(SR_K_CAST));
             SR_TRY(to_bf16(cast, G, st));
+            SR_TRY(prof.end());
         } else if (n_cast > 0) {
             for (int g = 0; g < G; ++g) {
                 if (!O(g).hidden_out) continue;
                 cast.src[0] = B[g].x32;
                 cast.dst[0] = static_cast<__nv_bfloat16 *>(O(g).hidden_out);
                 cast.n = size_t(T) * m.H;
+                SR_TRY(prof.begin(SR_K_CAST));
                 SR_TRY(to_bf16(cast, 1, st));
+                SR_TRY(prof.end());
             }
         }
     }

@@ -228,6 +228,32 @@ typedef enum sr_group_mode { SR_MODE_SKIP = 0, SR_MODE_FULL = 1 } sr_group_mode;
  *   1e-3 of max|S| after three layers. */
 typedef enum sr_group_precision { SR_PREC_SPLIT = 0, SR_PREC_BF16 = 1 } sr_group_precision;
 
+/* Optional per-launch timing.  When sr_group_args.profile is non-NULL the
+ * call records events[2i] before and events[2i+1] after its i-th kernel
+ * launch on `stream` (cudaEvent_t handles the caller created) and stores the
+ * launch's kind in kinds[i], for up to `capacity` launches; `count` returns
+ * how many launches the call made (it may exceed capacity: the excess is not
+ * timed).  Recording events adds no synchronisation. */
+typedef enum sr_kernel_kind {
+    SR_K_ROW_PREP = 0,   /* RMSNorm factor + activation split            */
+    SR_K_GEMM_IN = 1,    /* in_proj                                      */
+    SR_K_CONV = 2,       /* conv + SiLU + L2 norm + gates (+ conv state) */
+    SR_K_GDN = 3,        /* chunked gated-delta recurrence               */
+    SR_K_GATED_NORM = 4, /* gated RMSNorm                                */
+    SR_K_GEMM_OUT = 5,   /* out_proj + residual                          */
+    SR_K_GEMM_GATEUP = 6,/* MLP gate/up + SwiGLU                         */
+    SR_K_GEMM_DOWN = 7,  /* MLP down + residual                          */
+    SR_K_CAST = 8,       /* fp32 hidden -> bf16 hidden_out               */
+    SR_K_COUNT = 9
+} sr_kernel_kind;
+
+typedef struct sr_profile {
+    void *const *events;  /* host array [2 * capacity] of cudaEvent_t */
+    int32_t *kinds;       /* host array [capacity] */
+    int32_t capacity;
+    int32_t count;        /* out */
+} sr_profile;
+
 typedef struct sr_group_args {
     const void *const *anchors;       /* host array [n_groups] of device [total_tokens, hidden] bf16 */
     const int32_t *cu_seqlens;
@@ -239,6 +265,7 @@ typedef struct sr_group_args {
     float eps;
     int32_t mode;                     /* sr_group_mode */
     int32_t precision;                /* sr_group_precision */
+    sr_profile *profile;              /* host, may be NULL */
 } sr_group_args;
 
 SR_API size_t sr_group_replay_workspace(const sr_group_args *args);

@@ -119,7 +119,7 @@ def test_ctypes_structs_match_the_c_header(tmp_path):
     import subprocess
     structs = {"sr_gdn_args": sr.GdnArgs, "sr_mamba2_args": sr.Mamba2Args,
                "sr_layer_weights": sr.LayerWeights, "sr_layer_outputs": sr.LayerOutputs,
-               "sr_group_args": sr.GroupArgs}
+               "sr_group_args": sr.GroupArgs, "sr_profile": sr.Profile}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "sr/sr.h"', 'int main(void) {']
     for cname, py in structs.items():
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
