@@ -393,3 +393,28 @@ def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k
         ws = workspace(need, dev)
     _check(group_call(args, ws, stream))
     return outputs
+
+
+# ------------------------------------------------------------------ allocation-free group replay
+
+_grp_noalloc = _sig("sr_group_replay_noalloc", _i32, ctypes.POINTER(GroupArgs), _vp, ctypes.POINTER(_vp))
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def group_replay_noalloc(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, inter, h_k, h_v, d=128,
+                         conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, stream=None):
+    """sr_group_replay_noalloc: the group replay for callers that cannot allocate
+    device memory (scratch in the library's own fixed device array).  The caller
+    passes the anchors, the weights and preallocated outputs [G][L] of
+    (s_out, conv_out, hidden_out or None).  Returns the device address of the
+    scratch array (its first word is the status word)."""
+    args = group_args(anchors, cu_seqlens, weights, outputs, max_seqlen=max_seqlen, hidden=hidden, inter=inter,
+                      h_k=h_k, h_v=h_v, d=d, conv_width=conv_width, eps=eps, mode=mode, precision=precision)
+    scratch = _vp()
+    _check(_grp_noalloc(ctypes.byref(args), _stream_handle(stream), ctypes.byref(scratch)))
+    return scratch.value
+
+
+def group_noalloc_call(args: GroupArgs, stream=None) -> int:
+    """Raw C call (returns the sr_status); no CUDA work before validation passes."""
+    return int(_grp_noalloc(ctypes.byref(args), None if stream is None else _stream_handle(stream), None))

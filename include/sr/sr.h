@@ -273,6 +273,35 @@ SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, siz
                           void *stream);
 
 /* ------------------------------------------------------------------------
+ * sr_group_replay_noalloc -- sr_group_replay without a caller workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: a plug-in given only its input and
+ * output buffers by the host framework, an engine whose spare HBM is all
+ * promised to its KV-cache pool, or a path that cannot afford the implicit
+ * synchronisation of cudaMalloc.  The scratch is a fixed device array of
+ * SR_GROUP_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that
+ * loads the library keeps until the process exits.  The call allocates
+ * nothing and computes exactly what sr_group_replay computes.
+ *
+ * Limit: a replay whose sr_group_replay_workspace() exceeds
+ * SR_GROUP_NOALLOC_SCRATCH_BYTES is rejected with SR_ERR_WORKSPACE (about
+ * 150 KB per token per group at hidden 2560 with SR_PREC_SPLIT, so one group
+ * of up to ~210 tokens fits; ~110 KB and ~290 tokens with SR_PREC_BF16).
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Sharing: every call on a device uses the same
+ * array, which keeps the previous call's contents, so calls whose kernels
+ * overlap on the GPU (for example on two streams) race; serialise them.
+ * status_scratch (may be NULL) receives the array's device address, which
+ * sr_device_status() accepts in place of a workspace.
+ * ---------------------------------------------------------------------- */
+#define SR_GROUP_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+SR_API sr_status sr_group_replay_noalloc(const sr_group_args *args, void *stream,
+                                         const void **status_scratch);
+
+/* ------------------------------------------------------------------------
  * Status and diagnostics.
  * ---------------------------------------------------------------------- */
 /* Message for the calling thread's last failed call ("" if none). */
