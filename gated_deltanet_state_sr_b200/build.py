@@ -1,7 +1,9 @@
 """Build libsr.so in-tree: every csrc/*.cu compiled by nvcc for sm_100a only,
 linked into one shared library with a static CUDA runtime.
 
-    python -m gated_deltanet_state_sr_b200.build [--force] [--verbose]
+    python gated_deltanet_state_sr_b200/build.py [--force] [--verbose]
+
+(Run it by path: importing the package loads the library being built.)
 """
 from __future__ import annotations
 
