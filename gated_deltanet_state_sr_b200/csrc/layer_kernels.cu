@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(256) row_prep_kernel(const __grid_constant__ R
 }
 
 // ---------------------------------------------------------------- conv_gates
-constexpr int kConvTok = 32;  // tokens per CTA
+constexpr int kConvTok = 32;   // tokens per CTA: 4 warps x 8 consecutive tokens
+constexpr int kWarpTok = 8;
 
 // Index n of the sequence holding token t (cu non-decreasing, cu[0] = 0).
 __device__ __forceinline__ int seq_of(const int32_t *cu, int n_seqs, int t) {
@@ -96,18 +97,19 @@ __device__ __forceinline__ int seq_of(const int32_t *cu, int n_seqs, int t) {
     return lo;
 }
 
-// blockIdx.y < 2 h_k + h_v: one 128-channel head of [q|k|v] (thread = channel);
-// blockIdx.y == 2 h_k + h_v: the gates of kConvTok tokens.
+// blockIdx.y < 2 h_k + h_v: one 128-channel head of [q|k|v]; warp w takes
+// tokens t0 + 8w .. t0 + 8w + 7 and lane l channels 4l .. 4l+3, so the
+// per-head L2 norm is a warp reduction.  All 11 input rows (3 of history +
+// 8) are loaded before any arithmetic.  blockIdx.y == 2 h_k + h_v: gates.
 __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__ ConvBatch p) {
     const int g = blockIdx.z;
     const int head = blockIdx.y;
     const int t0 = blockIdx.x * kConvTok;
-    const int t1 = min(p.T, t0 + kConvTok);
     const int tid = threadIdx.x;
     const float *P = p.p[g];
     const int n_qk = 2 * p.h_k;
     if (head == n_qk + p.h_v) {
-        // gates: b at column b_off + h, a at column b_off + h_v + h
+        const int t1 = min(p.T, t0 + kConvTok);
         for (int e = tid; e < (t1 - t0) * p.h_v; e += blockDim.x) {
             const int t = t0 + e / p.h_v, h = e % p.h_v;
             const float b = P[size_t(t) * p.ld + p.b_off + h];
@@ -117,52 +119,72 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
         }
         return;
     }
-    const int D = 128;
-    const int ch = head * D + tid;
-    const __nv_bfloat16 *cw = p.conv_w[g] + size_t(ch) * 4;
-    const float w0 = __bfloat162float(cw[0]), w1 = __bfloat162float(cw[1]);
-    const float w2 = __bfloat162float(cw[2]), w3 = __bfloat162float(cw[3]);
-    __shared__ float red[4];
-    int n = seq_of(p.cu, p.n_seqs, t0);
-    int bos = max(p.cu[n], 0), eos = p.cu[n + 1];
-    // sliding window of the 3 previous pre-conv values (zero before the sequence start)
-    float x1 = (t0 - 1 >= bos) ? P[size_t(t0 - 1) * p.ld + ch] : 0.f;
-    float x2 = (t0 - 2 >= bos) ? P[size_t(t0 - 2) * p.ld + ch] : 0.f;
-    float x3 = (t0 - 3 >= bos) ? P[size_t(t0 - 3) * p.ld + ch] : 0.f;
-    for (int t = t0; t < t1; ++t) {
-        while (t >= eos && n + 1 < p.n_seqs) {  // next sequence (skips empty ones): the window restarts at zero
+    const int warp = tid >> 5, lane = tid & 31;
+    const int tw = t0 + warp * kWarpTok;  // first token of this warp
+    if (tw >= p.T) return;
+    const int ch = head * 128 + lane * 4;
+    float w[4][4];  // w[channel][tap]
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p.conv_w[g] + size_t(ch + c) * 4);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        w[c][0] = a.x; w[c][1] = a.y; w[c][2] = b.x; w[c][3] = b.y;
+    }
+    // rows tw-3 .. tw+7 (clamped into [0, T); masked below)
+    float4 x[kWarpTok + 3];
+#pragma unroll
+    for (int r = 0; r < kWarpTok + 3; ++r) {
+        const int t = tw - 3 + r;
+        const int tc = t < 0 ? 0 : (t >= p.T ? p.T - 1 : t);
+        x[r] = *reinterpret_cast<const float4 *>(P + size_t(tc) * p.ld + ch);
+    }
+    int n = seq_of(p.cu, p.n_seqs, tw);
+    int eos = p.cu[n + 1];
+    int bos = max(p.cu[n], 0);
+#pragma unroll
+    for (int i = 0; i < kWarpTok; ++i) {
+        const int t = tw + i;
+        if (t >= p.T) break;
+        while (t >= eos && n + 1 < p.n_seqs) {
             ++n;
             bos = max(p.cu[n], 0);
             eos = p.cu[n + 1];
-            x1 = x2 = x3 = 0.f;
         }
-        const float x0 = P[size_t(t) * p.ld + ch];
-        float c = w0 * x3 + w1 * x2 + w2 * x1 + w3 * x0;
-        c = c * sigmoidf_(c);
-        x3 = x2;
-        x2 = x1;
-        x1 = x0;
+        float c[4];
+        const float *x0 = reinterpret_cast<const float *>(&x[i + 3]);
+        const float *x1 = reinterpret_cast<const float *>(&x[i + 2]);
+        const float *x2 = reinterpret_cast<const float *>(&x[i + 1]);
+        const float *x3 = reinterpret_cast<const float *>(&x[i]);
+        const bool v1 = t - 1 >= bos, v2 = t - 2 >= bos, v3 = t - 3 >= bos;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float acc = w[e][3] * x0[e];
+            if (v1) acc = fmaf(w[e][2], x1[e], acc);
+            if (v2) acc = fmaf(w[e][1], x2[e], acc);
+            if (v3) acc = fmaf(w[e][0], x3[e], acc);
+            c[e] = acc * sigmoidf_(acc);
+        }
         if (head < n_qk) {
-            // per-head L2 norm over the 128 channels of this CTA
-            float ss = warp_sum(c * c);
-            if ((tid & 31) == 0) red[tid >> 5] = ss;
-            __syncthreads();
-            ss = red[0] + red[1] + red[2] + red[3];
-            __syncthreads();
-            c = c / sqrtf(ss + 1e-6f);
+            const float ss = warp_sum(c[0] * c[0] + c[1] * c[1] + c[2] * c[2] + c[3] * c[3]);
+            const float inv = 1.f / sqrtf(ss + 1e-6f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[e] *= inv;
         }
+        __nv_bfloat162 hi[2], lo[2];
+        split2(c[0], c[1], hi[0], lo[0]);
+        split2(c[2], c[3], hi[1], lo[1]);
+        const uint2 hv = *reinterpret_cast<uint2 *>(hi), lv = *reinterpret_cast<uint2 *>(lo);
         if (head < p.h_k) {
-            p.q[g][size_t(t) * p.h_k * D + ch] = __float2bfloat16_rn(c);
+            *reinterpret_cast<uint2 *>(p.q[g] + size_t(t) * p.h_k * 128 + ch) = hv;
         } else if (head < n_qk) {
-            const size_t o = size_t(t) * p.h_k * D + (ch - p.h_k * D);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(c);
-            p.k[g][o] = hi;
-            if (p.k_lo[g]) p.k_lo[g][o] = __float2bfloat16_rn(c - __bfloat162float(hi));
+            const size_t o = size_t(t) * p.h_k * 128 + (ch - p.h_k * 128);
+            *reinterpret_cast<uint2 *>(p.k[g] + o) = hv;
+            if (p.k_lo[g]) *reinterpret_cast<uint2 *>(p.k_lo[g] + o) = lv;
         } else {
-            const size_t o = size_t(t) * p.h_v * D + (ch - n_qk * D);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(c);
-            p.v[g][o] = hi;
-            if (p.v_lo[g]) p.v_lo[g][o] = __float2bfloat16_rn(c - __bfloat162float(hi));
+            const size_t o = size_t(t) * p.h_v * 128 + (ch - n_qk * 128);
+            *reinterpret_cast<uint2 *>(p.v[g] + o) = hv;
+            if (p.v_lo[g]) *reinterpret_cast<uint2 *>(p.v_lo[g] + o) = lv;
         }
     }
 }
