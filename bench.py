@@ -336,7 +336,86 @@ class GroupReplay:
                            f"({step_flop_per_tok / 1e6:.0f} MFLOP per replayed token)"), oracle.num_threads()
 
 
-WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "group": GroupReplay,
+
+class Mamba2Replay:
+    """Mamba2 replay (sr_mamba2_replay): 64 varlen suffixes of U{256..4096}
+    tokens, 64 heads, P = 64, N = 128, one B/C group."""
+
+    launches_per_step = 1
+    precision = "bf16 inputs, hi/lo state write"
+
+    def __init__(self, name, rank):
+        self.m = W.mamba2(seed=0x5EED0004 + rank)
+        self.desc = "Mamba2: 64 suffixes ~U{256..4096} tok, 64 heads, head dim 64, d_state 128"
+        m = self.m
+        self.tokens = sum(m.lengths)
+        T, H, P = m.x.shape
+        Ns = m.B.shape[2]
+        self.H, self.P, self.Ns = H, P, Ns
+        # algorithmic bytes per token: x, y (bf16), B, C (bf16, shared by heads), dt (fp32)
+        self.bytes_per_tok = H * P * 2 * 2 + 2 * Ns * 2 + H * 4
+        self.state_bytes = len(m.lengths) * H * P * Ns * 4
+        self.flop_per_tok = H * (4 * P * Ns + 2 * 64 * P) + 2 * 64 * Ns
+        self.input_bytes = sum(t.numel() * t.element_size() for t in (m.x, m.B, m.C, m.dt))
+
+    def setup(self, sr, dev):
+        self.sr = sr
+        m = self.m
+        d = lambda t: t.to(dev).contiguous()
+        self.x, self.B, self.C, self.dt, self.A, self.cu = map(d, (m.x, m.B, m.C, m.dt, m.A, m.cu_seqlens))
+        self.y = torch.empty_like(self.x)
+        self.s = torch.empty(len(m.lengths), self.H, self.P, self.Ns, dtype=torch.float32, device=dev)
+        self.ws = sr.workspace(1 << 20, dev)
+        self.max_len = m.max_seqlen
+        pin = lambda t: t.contiguous().pin_memory()
+        self.h_in = [pin(t) for t in (m.x, m.B, m.C, m.dt, m.cu_seqlens)]
+        self.d_in = [self.x, self.B, self.C, self.dt, self.cu]
+        self.h_y = torch.empty(self.y.shape, dtype=self.y.dtype).pin_memory()
+        self.h_s = torch.empty(self.s.shape, dtype=torch.float32).pin_memory()
+
+    def step(self):
+        self.sr.mamba2_replay(self.x, self.B, self.C, self.dt, self.A, self.cu, max_seqlen=self.max_len,
+                              y=self.y, s_out=self.s, ws=self.ws)
+
+    def step_e2e(self):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.h_y.copy_(self.y, non_blocking=True)
+        self.h_s.copy_(self.s, non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.h_in)
+
+    @property
+    def d2h_bytes(self):
+        return self.h_y.numel() * 2 + self.h_s.numel() * 4
+
+    def dominant(self):
+        return {"name": "mamba2_chunk_kernel", "bound": "hbm", "flop": self.flop_per_tok * self.tokens,
+                "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
+
+    def oracle_sample(self, stride=1, min_s=0.0, units=16):
+        """Bounded oracle run over `units` (sequence, head) pairs spread over the
+        batch, repeated until min_s seconds; tokens/s of the whole workload."""
+        import oracle
+        m = self.m
+        n_units = len(m.lengths) * self.H
+        us = list(range(0, n_units, max(1, n_units // units)))[:units]
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.mamba2_replay(m.x, m.B, m.C, m.dt, m.A, m.cu_seqlens, units=us)
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= min_s:
+                break
+        head_tokens = sum(m.lengths[u // self.H] for u in us) * reps
+        return head_tokens / self.H / dt, (f"{len(us)} of {n_units} (sequence, head) units x {reps} reps, "
+                                           f"{head_tokens} head-tokens in {dt:.1f} s; tokens/s = head-tokens / H / s"), \
+            oracle.num_threads()
+
+WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "group": GroupReplay, "mamba2": Mamba2Replay,
              **{f"model_{m}_{r}": GroupReplay for m in ("8k", "16k", "32k") for r in ("5", "10")}}
 DEFAULT_WORKLOAD = "model_32k_5"
 
@@ -459,13 +538,19 @@ def run_ours(args):
     else:
         dom = wl.dominant()
         kern_ms = ms_per_step  # the dominant kernel is the whole step for the raw workloads
-        achieved = dom["flop"] / (kern_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
+        tflops = dom["flop"] / (kern_ms / 1e3) / 1e12
         hbm_gbs = dom["bytes"] / (kern_ms / 1e3) / 1e9
-        roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": round(achieved, 2),
-                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                    "peak_source": f"{src} (burst bf16)", "hbm_gbs": round(hbm_gbs, 1),
-                    "hbm_frac": round(hbm_gbs / peaks["hbm_gbs"], 4)}
+        if dom["bound"] == "hbm":
+            roofline = {"kernel": dom["name"], "bound": "hbm", "achieved": round(hbm_gbs, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(hbm_gbs / peaks["hbm_gbs"], 4),
+                        "traffic": None, "peak_source": f"{src} (HBM copy)",
+                        "bytes_per_launch": dom["bytes"], "tflops": round(tflops, 2)}
+        else:
+            peak = peaks["bf16_tflops"]
+            roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": round(tflops, 2),
+                        "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                        "peak_source": f"{src} (burst bf16)", "hbm_gbs": round(hbm_gbs, 1),
+                        "hbm_frac": round(hbm_gbs / peaks["hbm_gbs"], 4)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -504,7 +589,8 @@ def run_reference(args):
     if rank != 0:
         return
     wl = make_workload(args, 0)
-    kw = dict(stride=8) if isinstance(wl, RawGdn) else dict(tokens=96)
+    kw = dict(stride=8) if isinstance(wl, RawGdn) else (dict(units=2) if isinstance(wl, Mamba2Replay)
+                                                        else dict(tokens=96))
     for _ in range(args.warmup):
         wl.oracle_sample(**kw)
     vals = []
