@@ -24,8 +24,9 @@
 // (I + A)^{-1} is formed in fp32 on the CUDA cores: 16x16 diagonal blocks by
 // forward substitution, then the off-diagonal blocks by block substitution.
 //
-// Precision: T and U enter the products that feed the state as exact hi + lo
-// bf16 pairs.  With SPLIT, k and v also arrive as hi + lo pairs (the layer
+// Precision: T diag(beta) and U enter the products that feed the state as
+// exact hi + lo bf16 pairs (a CPU emulation of these rounding points puts the
+// state error near 1e-4 of max|S|, against 3e-3 with plain bf16 operands).  With SPLIT, k and v also arrive as hi + lo pairs (the layer
 // computes them in fp32) and every product that reaches the state uses the
 // three-term expansion hi*hi + lo*hi + hi*lo.
 #include "common.cuh"
@@ -61,10 +62,11 @@ struct Smem {
     union { float a[C * ROWA]; __nv_bfloat16 w[C * ROW]; } r1;
     // R2: T (fp32) during the solve, then U (bf16)
     union { float t[C * ROWA]; __nv_bfloat16 u[C * ROW]; } r2;
-    // R3: T diag(beta e^gamma) and T diag(beta) as hi + lo bf16 pairs, then
-    // U diag(e^{gamma_C-gamma}) as a hi + lo bf16 pair.
+    // R3: T diag(beta e^gamma) (bf16; it only meets the state through W, where
+    // one rounding stays far inside the tolerance) and T diag(beta) as a hi + lo
+    // bf16 pair, then U diag(e^{gamma_C-gamma}) as a hi + lo bf16 pair.
     union {
-        struct { __nv_bfloat16 t1[C * ROWP], t2[C * ROWP], t1l[C * ROWP], t2l[C * ROWP]; } s;
+        struct { __nv_bfloat16 t1[C * ROWP], t2[C * ROWP], t2l[C * ROWP]; } s;
         struct { __nv_bfloat16 ud[C * ROW], udl[C * ROW]; } d;
     } r3;
     float gam[C];   // gamma_t, chunk-relative
@@ -242,6 +244,8 @@ gdn_chunk_kernel(const __grid_constant__ GdnBatch p) {
         __syncthreads();
 
         // ---- (3) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
+        // (thread = one column of one block; each row of A is read as 4 float4
+        // before it is used, so the loads pipeline ahead of the FMA chain)
         float *Af = sm.r1.a;
         float *Tf = sm.r2.t;
         if (tid < C) {
@@ -249,34 +253,68 @@ gdn_chunk_kernel(const __grid_constant__ GdnBatch p) {
             float x[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
+                const float4 *ar = reinterpret_cast<const float4 *>(&Af[(16 * b + r) * ROWA + 16 * b]);
+                float a[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 f = ar[v];
+                    a[4 * v] = f.x; a[4 * v + 1] = f.y; a[4 * v + 2] = f.z; a[4 * v + 3] = f.w;
+                }
                 float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-                for (int s = 0; s < r; ++s) acc = fmaf(-Af[(16 * b + r) * ROWA + 16 * b + s], x[s], acc);
+                for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-a[s2], x[s2], acc);
                 x[r] = (r < cc) ? 0.f : acc;
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * ROWA + 16 * b + cc] = x[r];
         }
         __syncthreads();
-        // off-diagonal blocks: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.  The strictly upper
-        // blocks of Tf hold the inner sums X_ij (stored at block (j, i)).
+        // Off-diagonal blocks, level by level: T_ij = -T_ii X_ij with
+        // X_ij = sum_{k=j}^{i-1} A_ik T_kj.  X_ij is kept in the (free) strictly
+        // upper block (j, i).  One work item = one row segment of 4 columns.
         auto blk = [](int bi, int bj, int r, int cc) { return (16 * bi + r) * ROWA + 16 * bj + cc; };
         for (int level = 1; level <= 3; ++level) {
-            for (int e = tid; e < (4 - level) * 256; e += NT) {
-                const int j = e >> 8, i = j + level, r = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-                for (int kb = j; kb < i; ++kb)
+            const int items = (4 - level) * 64;
+            for (int it = tid; it < items; it += NT) {
+                const int j = it >> 6, i = j + level, r = (it >> 2) & 15, c4 = (it & 3) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int kb = j; kb < i; ++kb) {
+                    const float4 *ar = reinterpret_cast<const float4 *>(&Af[blk(i, kb, r, 0)]);
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) acc = fmaf(Af[blk(i, kb, r, m)], Tf[blk(kb, j, m, cc)], acc);
-                Tf[blk(j, i, r, cc)] = acc;
+                    for (int v = 0; v < 4; ++v) {
+                        const float4 a = ar[v];
+                        const float am[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float4 t = *reinterpret_cast<const float4 *>(&Tf[blk(kb, j, 4 * v + e, c4)]);
+                            acc.x = fmaf(am[e], t.x, acc.x);
+                            acc.y = fmaf(am[e], t.y, acc.y);
+                            acc.z = fmaf(am[e], t.z, acc.z);
+                            acc.w = fmaf(am[e], t.w, acc.w);
+                        }
+                    }
+                }
+                *reinterpret_cast<float4 *>(&Tf[blk(j, i, r, c4)]) = acc;
             }
             __syncthreads();
-            for (int e = tid; e < (4 - level) * 256; e += NT) {
-                const int j = e >> 8, i = j + level, r = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
+            for (int it = tid; it < items; it += NT) {
+                const int j = it >> 6, i = j + level, r = (it >> 2) & 15, c4 = (it & 3) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 *dr = reinterpret_cast<const float4 *>(&Tf[blk(i, i, r, 0)]);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc = fmaf(Tf[blk(i, i, r, m)], Tf[blk(j, i, m, cc)], acc);
-                Tf[blk(i, j, r, cc)] = -acc;
+                for (int v = 0; v < 4; ++v) {
+                    const float4 d = dr[v];
+                    const float dm[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 xx = *reinterpret_cast<const float4 *>(&Tf[blk(j, i, 4 * v + e, c4)]);
+                        acc.x = fmaf(dm[e], xx.x, acc.x);
+                        acc.y = fmaf(dm[e], xx.y, acc.y);
+                        acc.z = fmaf(dm[e], xx.z, acc.z);
+                        acc.w = fmaf(dm[e], xx.w, acc.w);
+                    }
+                }
+                *reinterpret_cast<float4 *>(&Tf[blk(i, j, r, c4)]) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
         }
@@ -288,9 +326,7 @@ gdn_chunk_kernel(const __grid_constant__ GdnBatch p) {
             const float b0 = sm.beta[s], b1 = sm.beta[s + 1];
             const float e0 = __expf(sm.gam[s]), e1 = __expf(sm.gam[s + 1]);
             uint32_t hi, lo;
-            split_bf16(t0 * b0 * e0, t1 * b1 * e1, hi, lo);
-            *reinterpret_cast<uint32_t *>(&sm.r3.s.t1[t * ROWP + s]) = hi;
-            *reinterpret_cast<uint32_t *>(&sm.r3.s.t1l[t * ROWP + s]) = lo;
+            *reinterpret_cast<uint32_t *>(&sm.r3.s.t1[t * ROWP + s]) = pack_bf16(t0 * b0 * e0, t1 * b1 * e1);
             split_bf16(t0 * b0, t1 * b1, hi, lo);
             *reinterpret_cast<uint32_t *>(&sm.r3.s.t2[t * ROWP + s]) = hi;
             *reinterpret_cast<uint32_t *>(&sm.r3.s.t2l[t * ROWP + s]) = lo;
@@ -310,10 +346,9 @@ gdn_chunk_kernel(const __grid_constant__ GdnBatch p) {
                 for (int e = 0; e < 4; ++e) acc_w[j][e] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                uint32_t ah[4], al[4];
+                uint32_t ah[4];
                 const int acol = kk * 16 + (lane >> 4) * 8;
                 ldsm_x4(ah, smem_u32(&sm.r3.s.t1[arow4 * ROWP + acol]));
-                ldsm_x4(al, smem_u32(&sm.r3.s.t1l[arow4 * ROWP + acol]));
 #pragma unroll
                 for (int np = 0; np < NCOL / 16; ++np) {
                     uint32_t bk[4], bkl[4];
@@ -322,8 +357,6 @@ gdn_chunk_kernel(const __grid_constant__ GdnBatch p) {
                     ldsm_x4_t(bk, smem_u32(&sm.k[brow * ROW + bcol]));
                     mma16816(acc_w[2 * np], ah, bk[0], bk[1]);
                     mma16816(acc_w[2 * np + 1], ah, bk[2], bk[3]);
-                    mma16816(acc_w[2 * np], al, bk[0], bk[1]);
-                    mma16816(acc_w[2 * np + 1], al, bk[2], bk[3]);
                     if (SPLIT) {
                         ldsm_x4_t(bkl, smem_u32(&sm.kl[brow * ROW + bcol]));
                         mma16816(acc_w[2 * np], ah, bkl[0], bkl[1]);
