@@ -437,6 +437,20 @@ def dist_setup():
     return ws, rank, local
 
 
+def max_over_ranks(ms, world, device):
+    """Device-timed milliseconds of this rank -> the slowest rank's (the job's time)."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step_per_rank, world, steps, ms):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_step_per_rank * world * steps / (ms / 1e3)
+
+
 def run_ours(args):
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -476,14 +490,9 @@ def run_ours(args):
         while time.perf_counter() < t_end:
             wl.step()
         torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_step = ms / args.steps
-    tokens_all = wl.tokens * world * args.steps
-    value = tokens_all / (ms / 1e3)
+    value = job_throughput(wl.tokens, world, args.steps, ms)
 
     # per-kernel device time inside the timed region (events on the launching stream)
     kernels = None
@@ -513,12 +522,8 @@ def run_ours(args):
         wl.step_e2e()
     f1.record(stream)
     barrier()
-    ms_e2e = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = wl.tokens * world * k_e2e / (ms_e2e / 1e3)
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1), world, dev)
+    e2e_value = job_throughput(wl.tokens, world, k_e2e, ms_e2e)
 
     peaks, src = load_peaks()
     if profiled:

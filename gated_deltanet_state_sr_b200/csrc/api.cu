@@ -57,9 +57,11 @@ sr_status validate_gdn(const sr_gdn_args *a) {
         return set_error(SR_ERR_UNSUPPORTED, "head dims must satisfy d_k == d_v in {64,128} (got %d,%d)",
                          a->d_k, a->d_v);
     if (a->dtype != SR_BF16 && a->dtype != SR_FP32) return set_error(SR_ERR_INVALID_ARG, "bad dtype");
-    if (a->algo < SR_GDN_AUTO || a->algo > SR_GDN_CHUNKED) return set_error(SR_ERR_INVALID_ARG, "bad algo");
-    if (a->algo == SR_GDN_CHUNKED && a->dtype != SR_BF16)
-        return set_error(SR_ERR_UNSUPPORTED, "the chunked kernel takes bf16 q/k/v only");
+    if (a->algo < SR_GDN_AUTO || a->algo > SR_GDN_TCGEN05) return set_error(SR_ERR_INVALID_ARG, "bad algo");
+    if ((a->algo == SR_GDN_CHUNKED || a->algo == SR_GDN_TCGEN05) && a->dtype != SR_BF16)
+        return set_error(SR_ERR_UNSUPPORTED, "the chunked kernels take bf16 q/k/v only");
+    if (a->algo == SR_GDN_TCGEN05 && !gdn_tc_supported(a->d_k))
+        return set_error(SR_ERR_UNSUPPORTED, "the tcgen05 kernel takes d_k = d_v = 128 only");
     if (!aligned(a->s_out, 16) || (a->h0 && !aligned(a->h0, 16)))
         return set_error(SR_ERR_INVALID_ARG, "s_out and h0 must be 16-byte aligned");
     const size_t esz = a->dtype == SR_BF16 ? 2 : 4;
@@ -97,7 +99,12 @@ sr_status sr_gdn_replay(const sr_gdn_args *a, void *ws, size_t ws_bytes, void *s
     const bool chunked = a->algo == SR_GDN_CHUNKED || (a->algo == SR_GDN_AUTO && a->dtype == SR_BF16 &&
                                                         gdn_chunked_supported(*a));
     void *scratch = static_cast<char *>(ws) + kWsHeader;
-    e = chunked ? gdn_chunked(*a, scale, status, scratch, st) : gdn_sequential(*a, scale, status, st);
+    const bool use_tc = a->algo == SR_GDN_TCGEN05 ||
+                        (a->algo == SR_GDN_AUTO && a->dtype == SR_BF16 && gdn_tc_supported(a->d_k));
+    if (use_tc)
+        e = gdn_tc(*a, scale, status, st);
+    else
+        e = chunked ? gdn_chunked(*a, scale, status, scratch, st) : gdn_sequential(*a, scale, status, st);
     if (e != cudaSuccess) return cuda_error(e, "sr_gdn_replay: kernel launch");
     return SR_OK;
 }

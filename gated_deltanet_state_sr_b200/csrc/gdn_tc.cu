@@ -1,0 +1,679 @@
+// Chunked gated-delta replay on the 5th-generation tensor cores (d = 128).
+//
+// Same chunk algebra as gdn_chunk.cu ("Tail-Replay", Sec. 2; "SuffixReplay",
+// Eq. 4): per chunk of C = 64 tokens with chunk-relative log-decay gamma,
+//     A   = strict-lower(beta_t e^{gamma_t-gamma_s} k_t.k_s),  T = (I + A)^{-1}
+//     W   = T diag(beta e^gamma) K,   Ut = T diag(beta) V,    U = Ut - W S^T
+//     O   = scale (diag(e^gamma) Q S^T + M U),  M = lower(e^{gamma_t-gamma_s} q_t.k_s)
+//     S  <- e^{gamma_C} S + U^T diag(e^{gamma_C-gamma}) K
+// Here every product is a tcgen05.mma with M = 128 issued by one thread, the
+// fp32 state S (d_v x d_k) lives in tensor memory for the whole sequence, and
+// the token dimension is put on N so that M is a head dimension:
+//     [K;Q] K^T  (K and Q rows stacked: one M = 128 product gives K K^T and Q K^T)
+//     W^T = K^T T1^T,  Ut^T = V^T T2^T,  U^T += S (-W)^T,  O^T = S Qg^T + U^T P^T,
+//     S  += (U diag(e^{gamma_C-gamma}))^T K.
+// q, k, v tiles arrive by TMA (128-byte swizzle); T1, T2, P, -W^T, the bf16
+// copies of S and U and the scaled Qg are written by the threads in the same
+// swizzled layouts.  Eight warps do the masking, the fp32 (I + A)^{-1} solve
+// and the conversions; T diag(beta) and U diag(...) enter the products that
+// feed the state as exact hi + lo bf16 pairs, and with split inputs k and v do
+// too (three-term products), exactly as in the mma.sync kernel.
+// Every mbarrier wait is bounded; a timeout records SR_DEV_TIMEOUT, drains the
+// MMAs, frees tensor memory and ends the CTA.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace sr {
+
+namespace {
+
+using namespace tc;
+
+constexpr int C = 64, D = 128;
+constexpr int kThreads = 256;
+constexpr int ROWA = C + 4;  // fp32 row pitch of A and T in the solve
+
+// shared-memory layout (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_KQ = 0;           // [K_j0][Q_j0][K_j1][Q_j1], 8 KB each
+constexpr uint32_t OFF_V = 32768;        // [V_i0][V_i1]
+constexpr uint32_t OFF_KL = 49152;       // [Kl_j0][Kl_j1]    (split)
+constexpr uint32_t OFF_VL = 65536;       // [Vl_i0][Vl_i1]    (split)
+constexpr uint32_t kIn[2] = {49152, 81920};  // end of the inputs (plain, split)
+constexpr uint32_t SZ_P = 8192;          // P   [t][s]
+constexpr uint32_t SZ_TR = 24576;        // T1, T2h, T2l [t][s]; later -W^T [j][t] (16 KB)
+constexpr uint32_t SZ_SB = 32768;        // S bf16 [i][j], two 64-column halves
+constexpr uint32_t SZ_QG = 16384;        // Qg [t][j], two halves
+constexpr uint32_t SZ_XR = 49152;        // A, T fp32 (2 x 17408); later Udh, Udl, Ub [i][t]
+constexpr uint32_t SZ_MISC = 1024;       // gamma, beta, barriers, TMEM address, flags
+
+constexpr uint32_t smem_bytes(bool split) {
+    return kIn[split] + SZ_P + SZ_TR + SZ_SB + SZ_QG + SZ_XR + SZ_MISC + 1024 /* alignment */;
+}
+
+struct GdnTcParams {
+    CUtensorMap q[kMaxGroups], k[kMaxGroups], v[kMaxGroups], kl[kMaxGroups], vl[kMaxGroups];
+    const float *g[kMaxGroups];
+    const float *beta[kMaxGroups];
+    const float *h0[kMaxGroups];
+    __nv_bfloat16 *o[kMaxGroups];
+    float *s_out[kMaxGroups];
+    const int32_t *cu;
+    int total, max_len, h_k, h_v;
+    float scale;
+    uint32_t *status;
+};
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 f = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(a - f.x, b - f.y);
+    hi = *reinterpret_cast<uint32_t *>(&h);
+    lo = *reinterpret_cast<uint32_t *>(&l);
+}
+
+template <bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ GdnTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(sm);
+    const uint32_t oP = kIn[SPLIT], oTR = oP + SZ_P, oSB = oTR + SZ_TR, oQG = oSB + SZ_SB, oXR = oQG + SZ_QG;
+    const uint32_t oMISC = oXR + SZ_XR;
+    float *gam = reinterpret_cast<float *>(sm + oMISC);          // [64]
+    float *bet = gam + C;                                         // [64]
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 512);  // K (+ k low part) landed
+    uint64_t *bar_q = bar_k + 1;                                          // Q landed
+    uint64_t *bar_v = bar_k + 2;                                          // V (+ v low part) landed
+    uint64_t *bar_mma = bar_k + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *Af = reinterpret_cast<float *>(sm + oXR);
+    float *Tf = reinterpret_cast<float *>(sm + oXR + C * ROWA * 4);
+
+    const int h = blockIdx.x, n = blockIdx.y, gi = blockIdx.z;
+    const int h_k = p.h_k, h_v = p.h_v;
+    const int hk = h / (h_v / h_k);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;  // TMEM lane this thread reads
+    int bos, eos;
+    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
+    const int len = eos - bos;
+    const int nchunks = (len + C - 1) / C;
+    const size_t sbase = (size_t(n) * h_v + h) * D * D;
+    const float *h0 = p.h0[gi];
+    float *s_out = p.s_out[gi];
+
+    if (nchunks == 0) {  // empty sequence: the state is h0 (or zero)
+        for (int e = tid; e < D * D / 4; e += kThreads) {
+            const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4 *>(s_out + sbase)[e] = v;
+        }
+        return;
+    }
+
+    if (tid == 0) {
+        mbar_init(bar_k, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t R0 = tmem, R1 = tmem + 64, R2 = tmem + 128, R3 = tmem + 256;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+
+    // ---- initial state into TMEM: thread -> row i = `row`, columns [64 half, 64 half + 64)
+    {
+        uint32_t r[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int j0 = 64 * half + 32 * part;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                r[e] = __float_as_uint(h0 ? h0[sbase + size_t(row) * D + j0 + e] : 0.f);
+            tmem_st_32x32b_x32(R2 + lane_off + j0, r);
+        }
+        tmem_st_wait();
+    }
+
+    const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
+    // Each input is refilled as soon as the last product reading it has completed.
+    auto issue_k = [&](int c) {
+        const int y = bos + c * C;
+        mbar_arrive_expect_tx(bar_k, SPLIT ? 32768u : 16384u);
+        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * D, y);
+        tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * D + 64, y);
+        if (SPLIT) {
+            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * D, y);
+            tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * D + 64, y);
+        }
+    };
+    auto issue_q = [&](int c) {
+        const int y = bos + c * C;
+        mbar_arrive_expect_tx(bar_q, 16384u);
+        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * D, y);
+        tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * D + 64, y);
+    };
+    auto issue_v = [&](int c) {
+        const int y = bos + c * C;
+        mbar_arrive_expect_tx(bar_v, SPLIT ? 32768u : 16384u);
+        tma_load_2d(sm + OFF_V, mv, bar_v, h * D, y);
+        tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * D + 64, y);
+        if (SPLIT) {
+            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * D, y);
+            tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * D + 64, y);
+        }
+    };
+    if (tid == 0) {
+        prefetch_tmap(mq); prefetch_tmap(mk); prefetch_tmap(mv);
+        if (SPLIT) { prefetch_tmap(mkl); prefetch_tmap(mvl); }
+        issue_k(0);
+        issue_q(0);
+        issue_v(0);
+    }
+
+    const float *gh = p.g[gi] + size_t(bos) * h_v + h;
+    const float *bh = p.beta[gi] + size_t(bos) * h_v + h;
+    __nv_bfloat16 *o = p.o[gi];
+    const size_t v_stride = size_t(h_v) * D;
+    const float scale = p.scale;
+    uint32_t kq_phase = 0, v_phase = 0, mma_phase = 0;
+    float g_next = 0.f, b_next = 0.f;  // gates of the next chunk (threads tid < C)
+    if (tid < C && tid < len) {
+        g_next = gh[size_t(tid) * h_v];
+        b_next = bh[size_t(tid) * h_v];
+    }
+    bool ok = true;
+
+    // wait for the next completion of the MMA barrier (all threads), then order TMEM reads
+    auto wait_mma = [&]() -> bool {
+        const bool w = mbar_wait(bar_mma, mma_phase);
+        mma_phase ^= 1;
+        tc_fence_after();
+        return w;
+    };
+    auto check = [&](bool w) -> bool {  // collective barrier: true when any thread's wait failed
+        const bool stop = __syncthreads_or(!w) != 0;
+        if (stop && tid == 0) *abort_flag = 1;
+        return stop;
+    };
+
+    constexpr uint32_t ID_KK = idesc_bf16_f32_major(128, 64, 0, 0);   // K-major A and B
+    constexpr uint32_t ID_MN_K = idesc_bf16_f32_major(128, 64, 1, 0); // MN-major A, K-major B
+    constexpr uint32_t ID_K_MN = idesc_bf16_f32_major(128, 64, 0, 1); // K-major A, MN-major B
+    constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 0, 1);   // state update (N = 128)
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int clen = min(C, len - c * C);
+        // ---- gates of the chunk: gamma = inclusive prefix sum of g; padding has g = beta = 0
+        if (tid < C) {
+            gam[tid] = g_next;
+            bet[tid] = b_next;
+            const int t = (c + 1) * C + tid;
+            g_next = t < len ? gh[size_t(t) * h_v] : 0.f;
+            b_next = t < len ? bh[size_t(t) * h_v] : 0.f;
+        }
+        const bool tma_ok = mbar_wait(bar_k, kq_phase) && mbar_wait(bar_q, kq_phase);
+        kq_phase ^= 1;
+        __syncthreads();
+        if (warp == 0) {
+            const float a0 = gam[2 * lane], a1 = gam[2 * lane + 1];
+            float incl = a0 + a1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const float excl = incl - (a0 + a1);
+            gam[2 * lane] = excl + a0;
+            gam[2 * lane + 1] = excl + a0 + a1;
+        }
+        if (check(tma_ok)) break;
+        const float gC = gam[C - 1];
+
+        // ---- MMA 1: [K;Q] K^T -> R0 (rows 0-63: K K^T, rows 64-127: Q K^T)
+        if (tid == 0) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = base + OFF_KQ + (k >> 2) * 16384 + (k & 3) * 32;
+                mma_bf16_ss(R0, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_KK, k > 0);
+            }
+            if (SPLIT) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {  // [K;Q] Kl^T, and Kl K^T into R1 (rows 0-63)
+                    const uint32_t a = base + OFF_KQ + (k >> 2) * 16384 + (k & 3) * 32;
+                    const uint32_t bl = base + OFF_KL + (k >> 2) * 8192 + (k & 3) * 32;
+                    mma_bf16_ss(R0, sdesc_sw128(a, 16, 1024), sdesc_sw128(bl, 16, 1024), ID_KK, 1);
+                    mma_bf16_ss(R1, sdesc_sw128(bl, 16, 1024), sdesc_sw128(a, 16, 1024), ID_KK, k > 0);
+                }
+            }
+            mma_commit(bar_mma);
+        }
+        // ---- meanwhile: bf16 copy of S (entering the chunk) and S <- e^{gamma_C} S in TMEM
+        {
+            const float fC = __expf(gC);
+            uint32_t r[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                tmem_ld_32x32b_x32(R2 + lane_off + 64 * half + 32 * part, r);
+                tmem_ld_wait();
+                uint8_t *sb = sm + oSB + half * 16384;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 w;
+                    w.x = pack2(__uint_as_float(r[8 * q4 + 0]), __uint_as_float(r[8 * q4 + 1]));
+                    w.y = pack2(__uint_as_float(r[8 * q4 + 2]), __uint_as_float(r[8 * q4 + 3]));
+                    w.z = pack2(__uint_as_float(r[8 * q4 + 4]), __uint_as_float(r[8 * q4 + 5]));
+                    w.w = pack2(__uint_as_float(r[8 * q4 + 6]), __uint_as_float(r[8 * q4 + 7]));
+                    *reinterpret_cast<uint4 *>(sb + sw128(row, 4 * part + q4)) = w;
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
+                tmem_st_32x32b_x32(R2 + lane_off + 64 * half + 32 * part, r);
+            }
+            tmem_st_wait();
+        }
+        // ---- Qg = scale e^{gamma_t} Q (same swizzled geometry as the Q tiles)
+        for (int e = tid; e < 1024; e += kThreads) {
+            const int sub = e >> 9, t = (e >> 3) & 63, ch = e & 7;
+            const uint32_t off = sw128(t, ch);
+            const uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_KQ + 8192 + sub * 16384 + off);
+            const float f = scale * __expf(gam[t]);
+            const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+            uint4 w;
+            uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float2 xf = __bfloat1622float2(x2[q2]);
+                wp[q2] = pack2(xf.x * f, xf.y * f);
+            }
+            *reinterpret_cast<uint4 *>(sm + oQG + sub * 8192 + off) = w;
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (check(true)) break;
+        // ---- O^T = S Qg^T -> R3 (issued now, completes with the next commit)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = base + oSB + (k >> 2) * 16384 + (k & 3) * 32;
+                const uint32_t b = base + oQG + (k >> 2) * 8192 + (k & 3) * 32;
+                mma_bf16_ss(R3, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 16, 1024), ID_KK, k > 0);
+            }
+        }
+        const bool m1 = wait_mma();  // MMA 1 done (the O^T product may still run)
+
+        // ---- A (fp32, for the solve) from K K^T and P (bf16 tile) from Q K^T
+        {
+            uint32_t r[32], r2[32];
+            tmem_ld_32x32b_x32(R0 + lane_off + 32 * half, r);
+            if (SPLIT && quad < 2) tmem_ld_32x32b_x32(R1 + lane_off + 32 * half, r2);
+            tmem_ld_wait();
+            if (quad < 2) {
+                const int t = row;
+                const float gt = gam[t], bt = bet[t];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    float a4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s = 32 * half + e + u;
+                        float kk = __uint_as_float(r[e + u]);
+                        if (SPLIT) kk += __uint_as_float(r2[e + u]);
+                        a4[u] = (s < t) ? bt * __expf(gt - gam[s]) * kk : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(&Af[t * ROWA + 32 * half + e]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+                }
+            } else {
+                const int t = row - 64;
+                const float gt = gam[t];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s = 32 * half + 8 * q4 + 2 * u;
+                        const float d0 = __expf(s <= t ? gt - gam[s] : -INFINITY);
+                        const float d1 = __expf(s + 1 <= t ? gt - gam[s + 1] : -INFINITY);
+                        w[u] = pack2(scale * d0 * __uint_as_float(r[8 * q4 + 2 * u]),
+                                     scale * d1 * __uint_as_float(r[8 * q4 + 2 * u + 1]));
+                    }
+                    *reinterpret_cast<uint4 *>(sm + oP + sw128(t, 4 * half + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        tc_fence_before();
+        if (check(m1)) break;
+        if (tid == 0 && c + 1 < nchunks) issue_q(c + 1);  // Q read by MMA 1 and the Qg copy only
+
+        // ---- T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
+        if (tid < C) {
+            const int b = tid >> 4, cc = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const float4 *ar = reinterpret_cast<const float4 *>(&Af[(16 * b + r) * ROWA + 16 * b]);
+                float a[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 f = ar[v];
+                    a[4 * v] = f.x; a[4 * v + 1] = f.y; a[4 * v + 2] = f.z; a[4 * v + 3] = f.w;
+                }
+                float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-a[s2], x[s2], acc);
+                x[r] = (r < cc) ? 0.f : acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * ROWA + 16 * b + cc] = x[r];
+        }
+        __syncthreads();
+        auto blk = [](int bi, int bj, int r, int cc) { return (16 * bi + r) * ROWA + 16 * bj + cc; };
+        for (int level = 1; level <= 3; ++level) {
+            const int items = (4 - level) * 64;
+            for (int it = tid; it < items; it += kThreads) {
+                const int j = it >> 6, i = j + level, r = (it >> 2) & 15, c4 = (it & 3) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int kb = j; kb < i; ++kb) {
+                    const float4 *ar = reinterpret_cast<const float4 *>(&Af[blk(i, kb, r, 0)]);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float4 a = ar[v];
+                        const float am[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[blk(kb, j, 4 * v + e, c4)]);
+                            acc.x = fmaf(am[e], t4.x, acc.x);
+                            acc.y = fmaf(am[e], t4.y, acc.y);
+                            acc.z = fmaf(am[e], t4.z, acc.z);
+                            acc.w = fmaf(am[e], t4.w, acc.w);
+                        }
+                    }
+                }
+                *reinterpret_cast<float4 *>(&Tf[blk(j, i, r, c4)]) = acc;
+            }
+            __syncthreads();
+            for (int it = tid; it < items; it += kThreads) {
+                const int j = it >> 6, i = j + level, r = (it >> 2) & 15, c4 = (it & 3) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 *dr = reinterpret_cast<const float4 *>(&Tf[blk(i, i, r, 0)]);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 d4 = dr[v];
+                    const float dm[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 xx = *reinterpret_cast<const float4 *>(&Tf[blk(j, i, 4 * v + e, c4)]);
+                        acc.x = fmaf(dm[e], xx.x, acc.x);
+                        acc.y = fmaf(dm[e], xx.y, acc.y);
+                        acc.z = fmaf(dm[e], xx.z, acc.z);
+                        acc.w = fmaf(dm[e], xx.w, acc.w);
+                    }
+                }
+                *reinterpret_cast<float4 *>(&Tf[blk(i, j, r, c4)]) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            }
+            __syncthreads();
+        }
+        // T1 = T diag(beta e^gamma) (bf16), T2 = T diag(beta) (hi + lo): K-major tiles [t][s]
+        for (int e = tid; e < C * 8; e += kThreads) {
+            const int t = e >> 3, ch = e & 7;
+            uint32_t w1[4], wh[4], wl[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = 8 * ch + 2 * u;
+                const float t0 = (s <= t) ? Tf[t * ROWA + s] : 0.f;
+                const float t1 = (s + 1 <= t) ? Tf[t * ROWA + s + 1] : 0.f;
+                const float b0 = bet[s], b1 = bet[s + 1];
+                w1[u] = pack2(t0 * b0 * __expf(gam[s]), t1 * b1 * __expf(gam[s + 1]));
+                split2(t0 * b0, t1 * b1, wh[u], wl[u]);
+            }
+            const uint32_t off = sw128(t, ch);
+            *reinterpret_cast<uint4 *>(sm + oTR + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+            *reinterpret_cast<uint4 *>(sm + oTR + 8192 + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            *reinterpret_cast<uint4 *>(sm + oTR + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (check(true)) break;
+
+        // ---- MMA 2: W^T = K^T T1^T -> R1 ; Ut^T = V^T T2^T -> R0
+        if (tid == 0) {
+            if (!mbar_wait(bar_v, v_phase)) *abort_flag = 1;
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t kmn = base + OFF_KQ + k * 2048;  // K as MN-major A (j blocks 16 KB apart)
+                const uint32_t t1 = base + oTR + k * 32;
+                mma_bf16_ss(R1, sdesc_sw128(kmn, 16384, 1024), sdesc_sw128(t1, 16, 1024), ID_MN_K, k > 0);
+                if (SPLIT)
+                    mma_bf16_ss(R1, sdesc_sw128(base + OFF_KL + k * 2048, 8192, 1024), sdesc_sw128(t1, 16, 1024),
+                                ID_MN_K, 1);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t vmn = base + OFF_V + k * 2048;   // V as MN-major A (i blocks 8 KB apart)
+                const uint32_t t2h = base + oTR + 8192 + k * 32, t2l = base + oTR + 16384 + k * 32;
+                mma_bf16_ss(R0, sdesc_sw128(vmn, 8192, 1024), sdesc_sw128(t2h, 16, 1024), ID_MN_K, k > 0);
+                mma_bf16_ss(R0, sdesc_sw128(vmn, 8192, 1024), sdesc_sw128(t2l, 16, 1024), ID_MN_K, 1);
+                if (SPLIT)
+                    mma_bf16_ss(R0, sdesc_sw128(base + OFF_VL + k * 2048, 8192, 1024), sdesc_sw128(t2h, 16, 1024),
+                                ID_MN_K, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        v_phase ^= 1;
+        const bool m2 = wait_mma() && *abort_flag == 0;
+
+        // ---- -W^T (bf16) as the MN-major B tile [j][t] of the next product
+        {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(R1 + lane_off + 32 * half, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint4 w;
+                w.x = pack2(-__uint_as_float(r[8 * q4 + 0]), -__uint_as_float(r[8 * q4 + 1]));
+                w.y = pack2(-__uint_as_float(r[8 * q4 + 2]), -__uint_as_float(r[8 * q4 + 3]));
+                w.z = pack2(-__uint_as_float(r[8 * q4 + 4]), -__uint_as_float(r[8 * q4 + 5]));
+                w.w = pack2(-__uint_as_float(r[8 * q4 + 6]), -__uint_as_float(r[8 * q4 + 7]));
+                *reinterpret_cast<uint4 *>(sm + oTR + sw128(row, 4 * half + q4)) = w;
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (check(m2)) break;
+        if (tid == 0 && c + 1 < nchunks) issue_v(c + 1);  // V read by MMA 2 only
+
+        // ---- MMA 3: U^T = Ut^T + S (-W)^T -> R0
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = base + oSB + (k >> 2) * 16384 + (k & 3) * 32;
+                const uint32_t b = base + oTR + k * 2048;
+                mma_bf16_ss(R0, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 8192, 1024), ID_K_MN, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        const bool m3 = wait_mma();
+
+        // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16): K-major tiles [i][t]
+        {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(R0 + lane_off + 32 * half, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t wh[4], wl[4], wb[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int t = 32 * half + 8 * q4 + 2 * u;
+                    const float u0 = __uint_as_float(r[8 * q4 + 2 * u]), u1 = __uint_as_float(r[8 * q4 + 2 * u + 1]);
+                    split2(u0 * __expf(gC - gam[t]), u1 * __expf(gC - gam[t + 1]), wh[u], wl[u]);
+                    wb[u] = pack2(u0, u1);
+                }
+                const uint32_t off = sw128(row, 4 * half + q4);
+                *reinterpret_cast<uint4 *>(sm + oXR + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                *reinterpret_cast<uint4 *>(sm + oXR + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                *reinterpret_cast<uint4 *>(sm + oXR + 32768 + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (check(m3)) break;
+
+        // ---- MMA 4: S += (U diag)^T K -> R2 ; O^T += U^T P^T -> R3
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t kmn = base + OFF_KQ + k * 2048;  // K as MN-major B (j blocks 16 KB apart)
+                const uint32_t uh = base + oXR + k * 32, ul = base + oXR + 16384 + k * 32;
+                mma_bf16_ss(R2, sdesc_sw128(uh, 16, 1024), sdesc_sw128(kmn, 16384, 1024), ID_S, 1);
+                mma_bf16_ss(R2, sdesc_sw128(ul, 16, 1024), sdesc_sw128(kmn, 16384, 1024), ID_S, 1);
+                if (SPLIT)
+                    mma_bf16_ss(R2, sdesc_sw128(uh, 16, 1024), sdesc_sw128(base + OFF_KL + k * 2048, 8192, 1024),
+                                ID_S, 1);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t ub = base + oXR + 32768 + k * 32, pb = base + oP + k * 32;
+                mma_bf16_ss(R3, sdesc_sw128(ub, 16, 1024), sdesc_sw128(pb, 16, 1024), ID_KK, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        const bool m4 = wait_mma();
+        if (check(m4)) break;
+        // K is free now: fetch the next chunk's while O is written out
+        if (tid == 0 && c + 1 < nchunks) issue_k(c + 1);
+
+        // ---- o_t (bf16): thread = value channel i, 32 tokens
+        if (o) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(R3 + lane_off + 32 * half, r);
+            tmem_ld_wait();
+            const size_t tok0 = size_t(bos) + size_t(c) * C;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int t = 32 * half + e;
+                if (t < clen) o[(tok0 + t) * v_stride + size_t(h) * D + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    __syncthreads();
+    ok = *abort_flag == 0;
+    if (ok) {
+        // ---- final state: TMEM -> s_out
+        uint32_t r[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int j0 = 64 * half + 32 * part;
+            tmem_ld_32x32b_x32(R2 + lane_off + j0, r);
+            tmem_ld_wait();
+            float4 *dst = reinterpret_cast<float4 *>(s_out + sbase + size_t(row) * D + j0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                     __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+        }
+    } else if (tid == 0) {
+        atomicOr(p.status, SR_DEV_TIMEOUT);
+        // let in-flight MMAs and TMA copies finish before tensor memory and shared memory are released
+        mma_commit(bar_mma);
+        mbar_wait(bar_mma, mma_phase);
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// 2-D bf16 map over [rows, cols] (row pitch `cols`), 64 x 64 boxes, 128-byte swizzle.
+bool map_64x64(CUtensorMap *m, const void *base, int rows, int cols) {
+    return make_map_bf16(m, base, rows, cols, cols, 64, 64);
+}
+
+template <bool SPLIT>
+cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t st) {
+    const int smem = int(smem_bytes(SPLIT));
+    cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.h_v, n_seqs, n_groups);
+    gdn_tc_kernel<SPLIT><<<grid, kThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gdn_tc_supported(int d) { return d == 128; }
+
+cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split, cudaStream_t st) {
+    if (n_seqs == 0 || n_groups == 0 || b.total == 0) return gdn_chunked_batch(b, n_groups, n_seqs, 128, split, st);
+    GdnTcParams p{};
+    const int T = b.total, qkw = b.h_k * D, vw = b.h_v * D;
+    for (int g = 0; g < n_groups; ++g) {
+        if (!map_64x64(&p.q[g], b.q[g], T, qkw) || !map_64x64(&p.k[g], b.k[g], T, qkw) ||
+            !map_64x64(&p.v[g], b.v[g], T, vw))
+            return cudaErrorInvalidValue;
+        if (split && (!map_64x64(&p.kl[g], b.k_lo[g], T, qkw) || !map_64x64(&p.vl[g], b.v_lo[g], T, vw)))
+            return cudaErrorInvalidValue;
+        p.g[g] = b.g[g];
+        p.beta[g] = b.beta[g];
+        p.h0[g] = b.h0[g];
+        p.o[g] = b.o[g];
+        p.s_out[g] = b.s_out[g];
+    }
+    p.cu = b.cu;
+    p.total = b.total;
+    p.max_len = b.max_len;
+    p.h_k = b.h_k;
+    p.h_v = b.h_v;
+    p.scale = b.scale;
+    p.status = b.status;
+    return split ? launch<true>(p, n_groups, n_seqs, st) : launch<false>(p, n_groups, n_seqs, st);
+}
+
+cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, cudaStream_t st) {
+    GdnBatch b{};
+    b.q[0] = static_cast<const __nv_bfloat16 *>(a.q);
+    b.k[0] = static_cast<const __nv_bfloat16 *>(a.k);
+    b.v[0] = static_cast<const __nv_bfloat16 *>(a.v);
+    b.g[0] = a.g;
+    b.beta[0] = a.beta;
+    b.h0[0] = a.h0;
+    b.o[0] = static_cast<__nv_bfloat16 *>(a.o);
+    b.s_out[0] = a.s_out;
+    b.cu = a.cu_seqlens;
+    b.total = a.total_tokens;
+    b.max_len = a.max_seqlen;
+    b.h_k = a.h_k;
+    b.h_v = a.h_v;
+    b.scale = scale;
+    b.status = status;
+    return gdn_tc_batch(b, 1, a.n_seqs, false, st);
+}
+
+}  // namespace sr

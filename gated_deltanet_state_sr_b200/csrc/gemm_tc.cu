@@ -311,20 +311,6 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix (row pitch `pitch`
-// elements), 64 x box_rows boxes with the 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-    cuuint64_t strides[1] = {cuuint64_t(pitch) * 2};
-    cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
-    cuuint32_t es[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int sm_count() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -332,6 +318,26 @@ int sm_count() {
     return n > 0 ? n : 1;
 }
 
+}  // namespace
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix (row pitch `pitch`
+// elements), box_cols x box_rows boxes with the 128-byte swizzle.
+bool make_map_bf16(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(pitch) * 2};
+    cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+    cuuint32_t es[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_rows) {
+    return make_map_bf16(m, base, rows, cols, pitch, 64, box_rows);
+}
 }  // namespace
 
 cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,

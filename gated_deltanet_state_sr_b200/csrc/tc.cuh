@@ -126,6 +126,42 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
+// Store 32 consecutive fp32 columns of this warp's 32 lanes (inverse of tmem_ld_32x32b_x32).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// Shared-memory descriptor of a 128-byte-swizzled operand tile (1024-byte
+// aligned 8-row groups of 128-byte rows).
+//  K-major  (rows = M/N index, 64 K elements per row): lbo unused, sbo = 1024;
+//           step along K by adding 32 bytes per 16 elements.
+//  MN-major (rows = K index, 64 M/N elements per row): sbo = 1024 between
+//           8-row K groups, lbo = byte distance between consecutive 64-wide
+//           M/N blocks; step along K by adding 2048 bytes per 16 rows.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFF);
+    d |= uint64_t((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= uint64_t((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(2) << 61;
+    return d;
+}
+
+// Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte
+// swizzled tile (the layout TMA SWIZZLE_128B writes).
+__host__ __device__ constexpr uint32_t sw128(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
 // Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle
 // layout that a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes: rows of 128 B
 // (64 bf16), 8-row groups 1024 B apart.  `addr` must lie in a 1024-byte
@@ -148,6 +184,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | (1u << 10)                   // B format: bf16
            | (uint32_t(N >> 3) << 17)     // N / 8
            | (uint32_t(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor with operand majors: a_mn / b_mn = 1 selects MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, int a_mn, int b_mn) {
+    return idesc_bf16_f32(M, N) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16);
 }
 
 }  // namespace tc

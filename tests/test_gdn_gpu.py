@@ -15,7 +15,7 @@ from _util import OUT_TOL_BF16, STATE_TOL, TOL_FP32, assert_close
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = ["sequential", "chunked"]
+ALGOS = ["sequential", "chunked", "tcgen05"]
 
 
 @pytest.fixture(scope="module")
@@ -27,6 +27,8 @@ def sr():
 
 
 def run_gpu(sr, x: W.GdnInputs, algo, want_o=True, dev="cuda"):
+    if algo == "tcgen05" and x.q.shape[-1] != 128:
+        pytest.skip("the tcgen05 kernel takes d = 128 only")
     t = lambda a: None if a is None else a.to(dev).contiguous()
     o, s = sr.gdn_replay(t(x.q), t(x.k), t(x.v), t(x.g), t(x.beta), t(x.cu_seqlens),
                          max_seqlen=max(x.max_seqlen, 1), h0=t(x.h0), want_o=want_o, algo=algo)
@@ -86,8 +88,9 @@ def test_strong_decay(sr, algo):
 
 
 @pytest.mark.parametrize("algo", ALGOS)
-def test_state_only_mode(sr, algo):
-    x = W.gdn_inputs(6, [150, 40], 2, 4, 64, 64)
+@pytest.mark.parametrize("d", [64, 128])
+def test_state_only_mode(sr, algo, d):
+    x = W.gdn_inputs(6, [150, 40], 2, 4, d, d)
     o, s = run_gpu(sr, x, algo, want_o=False)
     assert o is None
     _, s_ref = run_oracle(x, want_o=False)
@@ -107,10 +110,10 @@ def test_fp32_input_mode(sr):
 def test_bad_cu_seqlens_flagged_on_device(sr, algo):
     """A decreasing cu_seqlens entry is caught by the kernel's own bounds check:
     that sequence is skipped (its output untouched) and a flag is recorded."""
-    x = W.gdn_inputs(9, [10, 10, 10], 2, 4, 64, 64)
+    x = W.gdn_inputs(9, [10, 10, 10], 2, 4, 128, 128)
     dev = lambda a: a.cuda().contiguous()
     cu = torch.tensor([0, 10, 5, 30], dtype=torch.int32, device="cuda")  # seq 1 runs backwards
-    s_out = torch.full((3, 4, 64, 64), 7.0, device="cuda")
+    s_out = torch.full((3, 4, 128, 128), 7.0, device="cuda")
     ws = sr.workspace(1 << 20)
     sr.gdn_replay(dev(x.q), dev(x.k), dev(x.v), dev(x.g), dev(x.beta), cu, max_seqlen=25,
                   s_out=s_out, want_o=False, algo=algo, ws=ws)
