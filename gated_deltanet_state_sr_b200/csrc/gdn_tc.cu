@@ -47,7 +47,7 @@ constexpr uint32_t SZ_TR = 24576;        // T1, T2h, T2l [t][s]; later -W^T [j][
 constexpr uint32_t SZ_SB = 32768;        // S bf16 [i][j], two 64-column halves
 constexpr uint32_t SZ_QG = 16384;        // Qg [t][j], two halves
 constexpr uint32_t SZ_XR = 49152;        // A, T fp32 (2 x 17408); later Udh, Udl, Ub [i][t]
-constexpr uint32_t SZ_MISC = 1024;       // gamma, beta, barriers, TMEM address, flags
+constexpr uint32_t SZ_MISC = 2048;       // gamma, beta, column factors, barriers, TMEM address, flags
 
 constexpr uint32_t smem_bytes(bool split) {
     return kIn[split] + SZ_P + SZ_TR + SZ_SB + SZ_QG + SZ_XR + SZ_MISC + 1024 /* alignment */;
@@ -87,7 +87,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const uint32_t oMISC = oXR + SZ_XR;
     float *gam = reinterpret_cast<float *>(sm + oMISC);          // [64]
     float *bet = gam + C;                                         // [64]
-    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 512);  // K (+ k low part) landed
+    float *fb = gam + 2 * C;                                      // [64] beta_s e^{gamma_s}
+    float *fu = gam + 3 * C;                                      // [64] e^{gamma_C - gamma_t}
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 1024);  // K (+ k low part) landed
     uint64_t *bar_q = bar_k + 1;                                          // Q landed
     uint64_t *bar_v = bar_k + 2;                                          // V (+ v low part) landed
     uint64_t *bar_mma = bar_k + 3;
@@ -245,6 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         if (check(tma_ok)) break;
         const float gC = gam[C - 1];
+        if (tid < C) {  // per-column factors, read after later barriers
+            fb[tid] = bet[tid] * __expf(gam[tid]);
+            fu[tid] = __expf(gC - gam[tid]);
+        }
 
         // ---- MMA 1: [K;Q] K^T -> R0 (rows 0-63: K K^T, rows 64-127: Q K^T)
         if (tid == 0) {
@@ -430,23 +436,34 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             }
             __syncthreads();
         }
-        // T1 = T diag(beta e^gamma) (bf16), T2 = T diag(beta) (hi + lo): K-major tiles [t][s]
-        for (int e = tid; e < C * 8; e += kThreads) {
-            const int t = e >> 3, ch = e & 7;
-            uint32_t w1[4], wh[4], wl[4];
+        // T1 = T diag(beta e^gamma) (bf16), T2 = T diag(beta) (hi + lo): K-major tiles [t][s].
+        // A thread always covers the same 8 columns, so their factors stay in registers.
+        {
+            const int ch = tid & 7;
+            float cb[8], cbe[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = 8 * ch + 2 * u;
-                const float t0 = (s <= t) ? Tf[t * ROWA + s] : 0.f;
-                const float t1 = (s + 1 <= t) ? Tf[t * ROWA + s + 1] : 0.f;
-                const float b0 = bet[s], b1 = bet[s + 1];
-                w1[u] = pack2(t0 * b0 * __expf(gam[s]), t1 * b1 * __expf(gam[s + 1]));
-                split2(t0 * b0, t1 * b1, wh[u], wl[u]);
+            for (int u = 0; u < 8; ++u) {
+                cb[u] = bet[8 * ch + u];
+                cbe[u] = fb[8 * ch + u];
             }
-            const uint32_t off = sw128(t, ch);
-            *reinterpret_cast<uint4 *>(sm + oTR + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-            *reinterpret_cast<uint4 *>(sm + oTR + 8192 + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-            *reinterpret_cast<uint4 *>(sm + oTR + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            for (int t = tid >> 3; t < C; t += kThreads / 8) {
+                const float4 *tr = reinterpret_cast<const float4 *>(&Tf[t * ROWA + 8 * ch]);
+                const float4 ta = tr[0], tb = tr[1];
+                float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+                uint32_t w1[4], wh[4], wl[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int s0 = 8 * ch + 2 * u;
+                    const float t0 = (s0 <= t) ? tv[2 * u] : 0.f;
+                    const float t1 = (s0 + 1 <= t) ? tv[2 * u + 1] : 0.f;
+                    w1[u] = pack2(t0 * cbe[2 * u], t1 * cbe[2 * u + 1]);
+                    split2(t0 * cb[2 * u], t1 * cb[2 * u + 1], wh[u], wl[u]);
+                }
+                const uint32_t off = sw128(t, ch);
+                *reinterpret_cast<uint4 *>(sm + oTR + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                *reinterpret_cast<uint4 *>(sm + oTR + 8192 + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                *reinterpret_cast<uint4 *>(sm + oTR + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -525,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
                 for (int u = 0; u < 4; ++u) {
                     const int t = 32 * half + 8 * q4 + 2 * u;
                     const float u0 = __uint_as_float(r[8 * q4 + 2 * u]), u1 = __uint_as_float(r[8 * q4 + 2 * u + 1]);
-                    split2(u0 * __expf(gC - gam[t]), u1 * __expf(gC - gam[t + 1]), wh[u], wl[u]);
+                    split2(u0 * fu[t], u1 * fu[t + 1], wh[u], wl[u]);
                     wb[u] = pack2(u0, u1);
                 }
                 const uint32_t off = sw128(row, 4 * half + q4);
