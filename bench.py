@@ -176,7 +176,8 @@ class RawGdn:
         return self.h_o.numel() * self.h_o.element_size() + self.h_s.numel() * 4
 
     def dominant(self):
-        return {"name": "gdn_chunk_kernel", "bound": "tensor",
+        # the default algorithm: the tcgen05 kernel at d = 128, the mma.sync one at d = 64
+        return {"name": "gdn_tc_kernel" if self.d == 128 else "gdn_chunk_kernel", "bound": "tensor",
                 "flop": self.flop_per_tok * self.tokens,
                 "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
 
@@ -244,6 +245,18 @@ class GroupReplay:
                 + self.flop["gdn"])
         last = self.flop["gemm_in"] + self.flop["gdn"]
         self.step_flop = (self.L - 1) * full + last  # skip mode
+        # algorithmic bytes of one launch (all groups) for the HBM-bound layer kernels
+        split = 2 if precision == "split" else 1
+        qd, vd = s.qk_dim, s.v_dim
+        self.bytes = {
+            # p (fp32) of the conv channels and gate columns in; q, k, v (hi/lo) and g, beta out
+            "conv": float(T) * self.G * ((s.conv_dim + 2 * s.h_v) * 4 + qd * 2 + (qd + vd) * 2 * split
+                                          + 2 * s.h_v * 4),
+            # x in (fp32), x * w out (hi/lo), r out
+            "row_prep": float(T) * self.G * (H * 4 + H * 2 * split + 4),
+            # o (bf16) and z (fp32) in, y (hi/lo) out
+            "gated_norm": float(T) * self.G * (vd * 2 + vd * 4 + vd * 2 * split),
+        }
         self.input_bytes = self.G * T * H * 2 + sum(
             sum(getattr(lw, f).numel() * getattr(lw, f).element_size() for f in ("w_in", "w_out", "w_gate", "w_up",
                                                                               "w_down"))
@@ -506,8 +519,20 @@ def run_ours(args):
                 tot[kind] = tot.get(kind, 0.0) + t
                 cnt[kind] = cnt.get(kind, 0) + 1
         busy = sum(tot.values())
-        kernels = {k: {"ms_per_step": round(tot[k] / args.steps, 4), "launches_per_step": cnt[k] // args.steps,
-                       "share": round(tot[k] / busy, 4)} for k in sorted(tot, key=lambda k: -tot[k])}
+        peaks_, _ = load_peaks()
+        kernels = {}
+        for k in sorted(tot, key=lambda k: -tot[k]):
+            per_launch = tot[k] / cnt[k]
+            ent = {"ms_per_step": round(tot[k] / args.steps, 4), "launches_per_step": cnt[k] // args.steps,
+                   "share": round(tot[k] / busy, 4)}
+            if k in wl.flop:
+                tf = wl.flop[k] / (per_launch / 1e3) / 1e12
+                ent.update(bound="tensor", achieved_tflops=round(tf, 1),
+                           frac=round(tf / peaks_.get("bf16_tflops_sustained", peaks_["bf16_tflops"]), 4))
+            elif k in wl.bytes:
+                gbs = wl.bytes[k] / (per_launch / 1e3) / 1e9
+                ent.update(bound="hbm", achieved_gbs=round(gbs, 1), frac=round(gbs / peaks_["hbm_gbs"], 4))
+            kernels[k] = ent
     else:
         launches = wl.launches_per_step * args.steps
 

@@ -129,3 +129,31 @@ def test_bad_cu_seqlens_flagged_on_device(sr, algo):
     sr.gdn_replay(dev(x.q), dev(x.k), dev(x.v), dev(x.g), dev(x.beta), cu, max_seqlen=10,
                   s_out=s_out, want_o=False, algo=algo, ws=ws)
     assert sr.device_status(ws) == 0
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("split_at", [64, 100])
+def test_exact_resume_on_gpu(sr, algo, split_at):
+    """Continuation: replaying b from h0 = Replay(a) gives Replay(a || b) ("Sparse
+    Prefix Caching for Hybrid and Recurrent LLM Serving", exactness of resume; the
+    replayed state hands over to the continuing tokens).  Split on and off a chunk
+    boundary."""
+    T = 300
+    x = W.gdn_inputs(15, [T], 2, 4, 128, 128)
+    d = lambda a: a.cuda().contiguous()
+    if algo == "tcgen05" and x.q.shape[-1] != 128:
+        pytest.skip("d = 128 only")
+    full_o, full_s = sr.gdn_replay(d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.cu_seqlens), max_seqlen=T,
+                                   algo=algo)
+    cu_a = torch.tensor([0, split_at], dtype=torch.int32, device="cuda")
+    cu_b = torch.tensor([0, T - split_at], dtype=torch.int32, device="cuda")
+    sl = lambda t, a, b: d(t[a:b])
+    _, s_a = sr.gdn_replay(sl(x.q, 0, split_at), sl(x.k, 0, split_at), sl(x.v, 0, split_at),
+                           sl(x.g, 0, split_at), sl(x.beta, 0, split_at), cu_a, max_seqlen=split_at, algo=algo)
+    o_b, s_b = sr.gdn_replay(sl(x.q, split_at, T), sl(x.k, split_at, T), sl(x.v, split_at, T),
+                             sl(x.g, split_at, T), sl(x.beta, split_at, T), cu_b, max_seqlen=T - split_at,
+                             h0=s_a, algo=algo)
+    torch.cuda.synchronize()
+    ref = full_s.double().cpu().numpy()
+    assert_close(s_b, ref, STATE_TOL, "resumed state vs full replay")
+    assert_close(o_b, full_o[split_at:].double().cpu().numpy(), OUT_TOL_BF16, "resumed outputs")

@@ -75,3 +75,18 @@ def test_state_only_and_strong_decay(sr):
     torch.cuda.synchronize()
     _, s_ref = oracle.mamba2_replay(m.x, m.B, m.C, m.dt, m.A, m.cu_seqlens, want_y=False)
     assert_close(s, s_ref, STATE_TOL, "state")
+
+
+def test_exact_resume_on_gpu(sr):
+    """Continuation from a replayed state: Replay(a || b) = Replay(b, h0 = Replay(a))."""
+    T, j = 250, 90
+    m = W.mamba2_inputs(24, [T], H=4)
+    d = lambda a: a.cuda().contiguous()
+    y, s = sr.mamba2_replay(d(m.x), d(m.B), d(m.C), d(m.dt), d(m.A), d(m.cu_seqlens), max_seqlen=T)
+    cu = lambda n: torch.tensor([0, n], dtype=torch.int32, device="cuda")
+    _, sa = sr.mamba2_replay(d(m.x[:j]), d(m.B[:j]), d(m.C[:j]), d(m.dt[:j]), d(m.A), cu(j), max_seqlen=j)
+    yb, sb = sr.mamba2_replay(d(m.x[j:]), d(m.B[j:]), d(m.C[j:]), d(m.dt[j:]), d(m.A), cu(T - j),
+                              max_seqlen=T - j, h0=sa)
+    torch.cuda.synchronize()
+    assert_close(sb, s.double().cpu().numpy(), STATE_TOL, "resumed state")
+    assert_close(yb, y[j:].double().cpu().numpy(), OUT_TOL_BF16, "resumed outputs")
