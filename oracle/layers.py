@@ -18,7 +18,8 @@ GDN block, Sec. 2 of Tail-Replay names Gated DeltaNet as the linear layer):
   h     = RMSNorm(x) * w_in_norm                     eps = 1e-6
   p     = h W_in^T  -> [q_pre | k_pre | v_pre | z | b | a]
   c     = causal depthwise conv, width 4, over [q_pre|k_pre|v_pre], zero
-          left padding at every sequence start (replay starts from zero)
+          left padding at every sequence start (replay starts from zero;
+          a continuation supplies the rebuilt conv state instead)
   q,k,v = SiLU(c);  q, k L2-normalised per head (eps 1e-6 inside the sqrt)
   g     = -exp(A_log) * softplus(a + dt_bias);  beta = sigmoid(b)
   o     = gated-delta recurrence (oracle.gdn_replay), scale 1/sqrt(d_k)
@@ -26,7 +27,7 @@ GDN block, Sec. 2 of Tail-Replay names Gated DeltaNet as the linear layer):
   x     = x_res + y W_out^T
   x     = x + W_down (SiLU(W_gate hh) * (W_up hh)),  hh = RMSNorm(x) * w_post
   conv_state = the last (width-1) pre-conv rows of each sequence, oldest
-               first, zero where the sequence is shorter.
+               first, taken from the padding where the sequence is shorter.
 Skip mode (the method): the last layer of the group stops after its
 recurrence -- neither its gated norm, out_proj nor MLP can change any state.
 Full mode: every layer runs to its MLP.
@@ -64,40 +65,52 @@ def softplus(x):
     return np.where(x > 20.0, x, np.log1p(np.exp(np.minimum(x, 20.0))))
 
 
-def causal_conv(pre, w, cu):
-    """Depthwise causal conv: c_t[ch] = sum_i w[ch, i] * pre_{t-W+1+i}[ch],
-    pre = 0 before each sequence start (never across cu_seqlens)."""
+def _history(conv_in, n, width, D):
+    """The (width-1) pre-conv rows that precede sequence n, oldest first:
+    zeros for a replay from zero, conv_in[n] (stored [D, width-1]) for a
+    continuation from a rebuilt conv state."""
+    if conv_in is None:
+        return np.zeros((width - 1, D))
+    return np.asarray(conv_in[n], dtype=np.float64).T
+
+
+def causal_conv(pre, w, cu, conv_in=None):
+    """Depthwise causal conv: c_t[ch] = sum_i w[ch, i] * pre_{t-W+1+i}[ch] over
+    each sequence, never across cu_seqlens.  The W-1 rows before a sequence
+    start are zero (replay from zero, "Tail-Replay", Sec. 3), or conv_in[n]
+    when the sequence continues from a rebuilt state."""
     T, D = pre.shape
     W = w.shape[1]
     out = np.zeros_like(pre)
     for n in range(len(cu) - 1):
         s, e = int(cu[n]), int(cu[n + 1])
-        seg = pre[s:e]
-        for i in range(W):
-            shift = W - 1 - i  # tap i reads the row `shift` tokens back
-            if shift >= e - s:
-                continue
-            out[s + shift:e] += w[:, i] * seg[: e - s - shift]
+        ext = np.concatenate([_history(conv_in, n, W, D), pre[s:e]], axis=0)
+        for t in range(e - s):
+            out[s + t] = np.sum(w * ext[t: t + W].T, axis=1)
     return out
 
 
-def conv_state(pre, cu, width):
-    """Last (width-1) pre-conv rows per sequence -> [N, D, width-1], oldest first."""
+def conv_state(pre, cu, width, conv_in=None):
+    """Last (width-1) pre-conv rows per sequence -> [N, D, width-1], oldest
+    first; rows before the sequence start come from its history (zeros, or
+    conv_in[n] on a continuation)."""
     N = len(cu) - 1
     D = pre.shape[1]
     st = np.zeros((N, D, width - 1))
     for n in range(N):
         s, e = int(cu[n]), int(cu[n + 1])
-        for j in range(width - 1):
-            t = e - (width - 1) + j
-            if t >= s:
-                st[n, :, j] = pre[t]
+        ext = np.concatenate([_history(conv_in, n, width, D), pre[s:e]], axis=0)
+        st[n] = ext[len(ext) - (width - 1):].T
     return st
 
 
-def gdn_layer(x, lw, cu, shape, *, stop_after_recurrence=False):
+def gdn_layer(x, lw, cu, shape, *, stop_after_recurrence=False, s_in=None, conv_in=None):
     """One GDN layer (+ its MLP unless stopped).  Returns a dict with the
-    final state S, conv_state, the gates, o (None when stopped) and x_out."""
+    final state S, conv_state, the gates, o (None when stopped) and x_out.
+
+    s_in [N, h_v, d_v, d_k] and conv_in [N, conv_dim, width-1] continue the
+    layer from rebuilt states (the unmatched tokens after a replay, "Tail-
+    Replay", Sec. 3); None starts from zero, as a replay does."""
     s = shape
     T = x.shape[0]
     h = rmsnorm(x, _f64(lw.w_in_norm), s.eps)
@@ -107,15 +120,15 @@ def gdn_layer(x, lw, cu, shape, *, stop_after_recurrence=False):
     z = p[:, s.conv_dim: s.conv_dim + vd]
     b = p[:, s.conv_dim + vd: s.conv_dim + vd + s.h_v]
     a = p[:, s.conv_dim + vd + s.h_v:]
-    c = silu(causal_conv(pre, _f64(lw.conv_w), cu))
+    c = silu(causal_conv(pre, _f64(lw.conv_w), cu, conv_in))
     q = l2norm(c[:, :qd].reshape(T, s.h_k, s.d_k), 1e-6)
     k = l2norm(c[:, qd: 2 * qd].reshape(T, s.h_k, s.d_k), 1e-6)
     v = c[:, 2 * qd:].reshape(T, s.h_v, s.d_v)
     g = -np.exp(_f64(lw.a_log)) * softplus(a + _f64(lw.dt_bias))
     beta = sigmoid(b)
-    o, S = gdn_replay(q, k, v, g, beta, cu, scale=1.0 / np.sqrt(s.d_k),
+    o, S = gdn_replay(q, k, v, g, beta, cu, scale=1.0 / np.sqrt(s.d_k), h0=s_in,
                       want_o=not stop_after_recurrence)
-    out = dict(S=S, conv_state=conv_state(pre, cu, s.conv_w), g=g, beta=beta,
+    out = dict(S=S, conv_state=conv_state(pre, cu, s.conv_w, conv_in), g=g, beta=beta,
                q=q, k=k, v=v, o=o, x_out=None)
     if stop_after_recurrence:
         return out
@@ -128,20 +141,28 @@ def gdn_layer(x, lw, cu, shape, *, stop_after_recurrence=False):
     return out
 
 
-def group_replay(gi, mode="skip"):
-    """Replay one group from its anchors with every state starting at zero.
+def group_replay(gi, mode="skip", *, initial=None, anchor_index=None, anchors=None):
+    """Replay one group from its anchors.
 
     gi: workloads.GroupInputs.  mode: "skip" (last layer stops after its
-    recurrence) or "full".  Returns a list of per-layer dicts (see gdn_layer).
+    recurrence) or "full".  anchors (default gi.anchors) is the anchor pool;
+    with anchor_index, replay token t reads pool row anchor_index[t] (token-
+    wise sparse anchors gathered from the sidecar, "SuffixReplay", Algorithm
+    Design 2).  initial: None (every state starts at zero: the replay) or a
+    per-layer list of (s_in, conv_in) to continue from.  Returns a list of
+    per-layer dicts (see gdn_layer).
     """
     assert mode in ("skip", "full")
     cu = np.asarray(gi.cu_seqlens.tolist(), dtype=np.int64)
-    x = _f64(gi.anchors)
+    x = _f64(gi.anchors if anchors is None else anchors)
+    if anchor_index is not None:
+        x = x[np.asarray(anchor_index, dtype=np.int64)]
     outs = []
     L = len(gi.layers)
     for l, lw in enumerate(gi.layers):
         stop = mode == "skip" and l == L - 1
-        r = gdn_layer(x, lw, cu, gi.shape, stop_after_recurrence=stop)
+        s_in, c_in = (None, None) if initial is None else initial[l]
+        r = gdn_layer(x, lw, cu, gi.shape, stop_after_recurrence=stop, s_in=s_in, conv_in=c_in)
         outs.append(r)
         x = r["x_out"]
     return outs

@@ -201,3 +201,109 @@ def test_groups_are_independent_of_packing():
         for l in range(2):
             np.testing.assert_allclose(both[l]["S"][n], one[l]["S"][0], rtol=1e-12, atol=1e-14)
             np.testing.assert_allclose(both[l]["x_out"][a:b], one[l]["x_out"], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- continuation
+# After a replay rebuilds a layer's recurrent state and conv state, the
+# unmatched tokens continue from them ("Tail-Replay", Sec. 3).  Continuing
+# from the states of a must give exactly what processing a || b in one pass
+# gives ("Sparse Prefix Caching for Hybrid and Recurrent LLM Serving", exact
+# resume); in fp64 the two differ only by rounding order.
+
+def test_conv_priming_closed_form():
+    """Delta weights turn the conv into a shift; on a continuation the rows
+    shifted in at a sequence start are the stored history, oldest first."""
+    rng = np.random.default_rng(3)
+    cu = [0, 1, 1, 6]  # lengths 1, 0, 5
+    D = 2
+    pre = rng.standard_normal((6, D))
+    hist = rng.standard_normal((3, D, 3))  # [N, D, width-1]
+    w = np.zeros((D, 4))
+    w[:, 1] = 1.0  # two tokens back
+    out = L.causal_conv(pre, w, cu, hist)
+    np.testing.assert_array_equal(out[0], hist[0][:, 1])      # t = 0 of seq 0 reads history slot 1
+    np.testing.assert_array_equal(out[1], hist[2][:, 1])      # seq 2 starts at row 1
+    np.testing.assert_array_equal(out[2], hist[2][:, 2])
+    np.testing.assert_array_equal(out[3], pre[1])
+    np.testing.assert_array_equal(out[5], pre[3])
+    st = L.conv_state(pre, cu, 4, hist)
+    np.testing.assert_array_equal(st[0], np.stack([hist[0][:, 1], hist[0][:, 2], pre[0]], axis=1))
+    np.testing.assert_array_equal(st[1], hist[1])              # empty sequence keeps its history
+    np.testing.assert_array_equal(st[2], pre[3:6].T)
+
+
+def _split_batch(lengths, cuts):
+    """Index arrays of the a-part (first cut_n tokens of every sequence) and
+    the b-part (the rest) of a packed batch, plus their cu_seqlens."""
+    starts = np.concatenate([[0], np.cumsum(lengths)])
+    a_idx = np.concatenate([np.arange(starts[n], starts[n] + c) for n, c in enumerate(cuts)]).astype(np.int64)
+    b_idx = np.concatenate([np.arange(starts[n] + c, starts[n + 1]) for n, c in enumerate(cuts)]).astype(np.int64)
+    cu_a = np.concatenate([[0], np.cumsum(cuts)])
+    cu_b = np.concatenate([[0], np.cumsum(np.asarray(lengths) - np.asarray(cuts))])
+    return a_idx, b_idx, cu_a, cu_b
+
+
+CONT_LENGTHS = [9, 5, 3, 7, 2]
+CONT_CUTS = [4, 1, 3, 0, 2]  # b-parts of 5, 4, 0, 7, 0 tokens; a-parts shorter than the conv window too
+
+
+def test_layer_continuation_is_exact():
+    s = _tiny_shape()
+    gi = W.group_inputs(31, CONT_LENGTHS, n_layers=1, shape=s)
+    lw = gi.layers[0]
+    lw.w_in = W.normal(31, "win", (s.proj_dim, s.hidden), 0.5)
+    lw.conv_w = W.normal(31, "cw", (s.conv_dim, s.conv_w), 0.5)
+    x = oracle._f64(gi.anchors)
+    full = L.gdn_layer(x, lw, np.asarray(gi.cu_seqlens.tolist()), s)
+    a_idx, b_idx, cu_a, cu_b = _split_batch(CONT_LENGTHS, CONT_CUTS)
+    ra = L.gdn_layer(x[a_idx], lw, cu_a, s)
+    rb = L.gdn_layer(x[b_idx], lw, cu_b, s, s_in=ra["S"], conv_in=ra["conv_state"])
+    np.testing.assert_allclose(rb["S"], full["S"], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(rb["conv_state"], full["conv_state"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(rb["x_out"], full["x_out"][b_idx], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(rb["o"], full["o"][b_idx], rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", ["skip", "full"])
+def test_group_continuation_is_exact(mode):
+    s = _tiny_shape()
+    gi = W.group_inputs(32, CONT_LENGTHS, n_layers=3, shape=s)
+    full = L.group_replay(gi, mode)
+    a_idx, b_idx, cu_a, cu_b = _split_batch(CONT_LENGTHS, CONT_CUTS)
+    ga = W.GroupInputs(gi.anchors[torch.from_numpy(a_idx)], torch.tensor(cu_a, dtype=torch.int32), gi.layers, s)
+    gb = W.GroupInputs(gi.anchors[torch.from_numpy(b_idx)], torch.tensor(cu_b, dtype=torch.int32), gi.layers, s)
+    ra = L.group_replay(ga, mode)
+    rb = L.group_replay(gb, mode, initial=[(r["S"], r["conv_state"]) for r in ra])
+    for l in range(3):
+        np.testing.assert_allclose(rb[l]["S"], full[l]["S"], rtol=1e-10, atol=1e-13)
+        np.testing.assert_allclose(rb[l]["conv_state"], full[l]["conv_state"], rtol=1e-10, atol=1e-13)
+
+
+def test_continuation_rejects_a_reversed_conv_history(monkeypatch):
+    """Planted mistake: a conv state stored newest-first breaks the exact
+    continuation, so the test above pins the history's order."""
+    s = _tiny_shape()
+    gi = W.group_inputs(33, CONT_LENGTHS, n_layers=1, shape=s)
+    x = oracle._f64(gi.anchors)
+    lw = gi.layers[0]
+    lw.conv_w = W.normal(33, "cw", (s.conv_dim, s.conv_w), 0.5)
+    full = L.gdn_layer(x, lw, np.asarray(gi.cu_seqlens.tolist()), s)
+    a_idx, b_idx, cu_a, cu_b = _split_batch(CONT_LENGTHS, CONT_CUTS)
+    good = L.conv_state
+    monkeypatch.setattr(L, "conv_state", lambda *a, **k: good(*a, **k)[..., ::-1])
+    ra = L.gdn_layer(x[a_idx], lw, cu_a, s)
+    rb = L.gdn_layer(x[b_idx], lw, cu_b, s, s_in=ra["S"], conv_in=ra["conv_state"])
+    assert np.max(np.abs(rb["S"] - full["S"])) > 1e-6 * np.max(np.abs(full["S"]))
+
+
+def test_sparse_anchor_gather_reads_pool_rows():
+    """Token-wise sparse anchors ("SuffixReplay", Algorithm Design 2): the
+    replay batch is the anchor pool's rows in index order."""
+    s = _tiny_shape()
+    gi = W.group_inputs(34, [6, 3], n_layers=2, shape=s)
+    pool = W.normal(34, "pool", (20, s.hidden), 1.0)
+    idx = np.array([19, 3, 4, 7, 0, 12, 5, 5, 18])
+    a = L.group_replay(gi, "full", anchors=pool, anchor_index=idx)
+    b = L.group_replay(W.GroupInputs(pool[torch.from_numpy(idx)], gi.cu_seqlens, gi.layers, s), "full")
+    for l in range(2):
+        np.testing.assert_array_equal(a[l]["S"], b[l]["S"])
