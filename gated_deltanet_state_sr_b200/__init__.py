@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libsr.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sr", "sr.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gated_deltanet_state_sr_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python gated_deltanet_state_sr_b200/build.py` "
                       "(there is no fallback path)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -33,7 +33,7 @@ SR_OK, SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_WORKSPACE, SR_ERR_CUDA, SR
 SR_BF16, SR_FP32 = 0, 1
 SR_GDN_AUTO, SR_GDN_SEQUENTIAL, SR_GDN_CHUNKED, SR_GDN_TCGEN05 = 0, 1, 2, 3
 SR_MODE_SKIP, SR_MODE_FULL = 0, 1
-SR_DEV_BAD_CU_SEQLENS, SR_DEV_SEQ_TOO_LONG = 0x1, 0x2
+SR_DEV_BAD_CU_SEQLENS, SR_DEV_SEQ_TOO_LONG, SR_DEV_TIMEOUT, SR_DEV_BAD_INDEX = 0x1, 0x2, 0x4, 0x8
 _ALGOS = {"auto": SR_GDN_AUTO, "sequential": SR_GDN_SEQUENTIAL, "chunked": SR_GDN_CHUNKED,
           "tcgen05": SR_GDN_TCGEN05}
 
@@ -65,6 +65,10 @@ class LayerOutputs(ctypes.Structure):
     _fields_ = [("s_out", _vp), ("conv_out", _vp), ("hidden_out", _vp)]
 
 
+class LayerState(ctypes.Structure):
+    _fields_ = [("s_in", _vp), ("conv_in", _vp)]
+
+
 class Profile(ctypes.Structure):
     _fields_ = [("events", ctypes.POINTER(_vp)), ("kinds", ctypes.POINTER(_i32)), ("capacity", _i32),
                 ("count", _i32)]
@@ -79,7 +83,8 @@ class GroupArgs(ctypes.Structure):
                 ("n_groups", _i32), ("n_layers", _i32), ("n_seqs", _i32), ("total_tokens", _i32),
                 ("max_seqlen", _i32), ("hidden", _i32), ("inter", _i32), ("h_k", _i32), ("h_v", _i32),
                 ("d_k", _i32), ("d_v", _i32), ("conv_width", _i32), ("eps", ctypes.c_float),
-                ("mode", _i32), ("precision", _i32), ("profile", ctypes.POINTER(Profile))]
+                ("mode", _i32), ("precision", _i32), ("profile", ctypes.POINTER(Profile)),
+                ("initial", ctypes.POINTER(LayerState)), ("anchor_index", _vp), ("anchor_rows", _i32)]
 
 
 def _sig(name, restype, *argtypes):
@@ -310,13 +315,25 @@ _LAYER_FIELDS = [f for f, _ in LayerWeights._fields_]
 
 
 def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, inter, h_k, h_v, d=128,
-               conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, profile=None):
+               conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, profile=None,
+               initial=None, anchor_index=None, total_tokens=None):
     """Builds a GroupArgs (and keeps the ctypes arrays alive on it).
 
-    anchors: list [G] of [T, hidden] bf16 CUDA tensors; weights: list [G] of
-    lists [L] of objects with the sr_layer_weights field names (CUDA tensors);
-    outputs: list [G] of lists [L] of (s_out, conv_out, hidden_out-or-None)."""
+    anchors: list [G] of [T, hidden] bf16 CUDA tensors (the anchor pools
+    [rows, hidden] when anchor_index, an int32 CUDA tensor [T], is given);
+    weights: list [G] of lists [L] of objects with the sr_layer_weights field
+    names (CUDA tensors); outputs: list [G] of lists [L] of (s_out, conv_out,
+    hidden_out-or-None); initial: None or list [G] of lists [L] of
+    (s_in-or-None, conv_in-or-None) to continue from."""
     G, L = len(anchors), len(weights[0])
+    init_arr = None
+    if initial is not None:
+        init_arr = (LayerState * (G * L))()
+        for g in range(G):
+            for l in range(L):
+                si, ci = initial[g][l]
+                init_arr[g * L + l] = LayerState(None if si is None else si.data_ptr(),
+                                                 None if ci is None else ci.data_ptr())
     anc = (_vp * G)(*[t.data_ptr() for t in anchors])
     w_arr = (LayerWeights * (G * L))()
     o_arr = (LayerOutputs * (G * L))()
@@ -327,11 +344,16 @@ def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, int
             s, c, h = outputs[g][l]
             o_arr[g * L + l] = LayerOutputs(s.data_ptr(), c.data_ptr(), None if h is None else h.data_ptr())
     n = cu_seqlens.numel() - 1
-    T = anchors[0].shape[0]
+    if total_tokens is not None:
+        T = total_tokens
+    else:
+        T = anchors[0].shape[0] if anchor_index is None else anchor_index.numel()
     a = GroupArgs(anc, cu_seqlens.data_ptr(), w_arr, o_arr, G, L, n, T, max_seqlen, hidden, inter, h_k, h_v,
                   d, d, conv_width, float(eps), mode, precision,
-                  ctypes.pointer(profile.struct) if profile is not None else None)
-    a._keep = (anc, w_arr, o_arr, profile)
+                  ctypes.pointer(profile.struct) if profile is not None else None,
+                  init_arr, None if anchor_index is None else anchor_index.data_ptr(),
+                  0 if anchor_index is None else anchors[0].shape[0])
+    a._keep = (anc, w_arr, o_arr, profile, init_arr)
     return a
 
 
@@ -365,14 +387,18 @@ def group_call(args: GroupArgs, ws, stream=None) -> int:
 
 def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k, h_v, d=128, conv_width=4,
                  eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, want_hidden=False, outputs=None,
-                 ws=None, stream=None, profile=None):
+                 ws=None, stream=None, profile=None, initial=None, anchor_index=None):
     """Replays every group of the call (see sr_group_replay).  Returns the
-    outputs list [G][L] of (s_out, conv_out, hidden_out or None)."""
+    outputs list [G][L] of (s_out, conv_out, hidden_out or None).
+
+    anchor_index (int32 CUDA tensor [T]) gathers the replay tokens from the
+    anchor pools ``anchors``; initial ([G][L] of (s_in, conv_in), either may
+    be None) continues from earlier states instead of zero."""
     torch = _torch()
     dev = anchors[0].device
     G, L = len(anchors), len(weights[0])
     n = cu_seqlens.numel() - 1
-    T = anchors[0].shape[0]
+    T = anchors[0].shape[0] if anchor_index is None else anchor_index.numel()
     conv_dim = 2 * h_k * d + h_v * d
     if outputs is None:
         outputs = []
@@ -386,7 +412,7 @@ def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k
             outputs.append(row)
     args = group_args(anchors, cu_seqlens, weights, outputs, max_seqlen=max_seqlen, hidden=hidden, inter=inter,
                       h_k=h_k, h_v=h_v, d=d, conv_width=conv_width, eps=eps, mode=mode, precision=precision,
-                      profile=profile)
+                      profile=profile, initial=initial, anchor_index=anchor_index)
     need = group_workspace_bytes(args)
     if need == 0:
         _check(group_call(args, None))
@@ -419,3 +445,60 @@ def group_replay_noalloc(anchors, cu_seqlens, weights, outputs, *, max_seqlen, h
 def group_noalloc_call(args: GroupArgs, stream=None) -> int:
     """Raw C call (returns the sr_status); no CUDA work before validation passes."""
     return int(_grp_noalloc(ctypes.byref(args), None if stream is None else _stream_handle(stream), None))
+
+
+# ------------------------------------------------------------------ anchor sidecar
+
+class CaptureArgs(ctypes.Structure):
+    _fields_ = [("hidden_states", _vp), ("pool", _vp), ("src_rows", _vp), ("dst_rows", _vp), ("n", _i32),
+                ("hidden", _i32), ("src_rows_total", _i32), ("pool_rows", _i32)]
+
+
+class AnchorPlanArgs(ctypes.Structure):
+    _fields_ = [("n_prefix", ctypes.c_int64), ("page_size", _i32), ("anchors_per_page", _i32), ("layout", _i32),
+                ("k_max", _i32), ("ratio", ctypes.c_double), ("block_table", ctypes.POINTER(_i32))]
+
+
+SR_ANCHORS_PAGE_TAIL, SR_ANCHORS_UNIFORM = 0, 1
+_capture = _sig("sr_anchor_capture", _i32, ctypes.POINTER(CaptureArgs), _vp, ctypes.c_size_t, _vp)
+_plan = _sig("sr_sparse_anchor_plan", _i32, ctypes.POINTER(AnchorPlanArgs), ctypes.POINTER(ctypes.c_int64),
+             ctypes.POINTER(_i32), ctypes.c_int64, ctypes.POINTER(ctypes.c_int64))
+
+
+def capture_args(hidden_states, pool, src_rows, dst_rows) -> CaptureArgs:
+    return CaptureArgs(hidden_states.data_ptr(), pool.data_ptr(), src_rows.data_ptr(), dst_rows.data_ptr(),
+                       src_rows.numel(), hidden_states.shape[1], hidden_states.shape[0], pool.shape[0])
+
+
+def capture_call(args: CaptureArgs, ws, stream=None) -> int:
+    return int(_capture(ctypes.byref(args), None if ws is None else _ptr(ws), 0 if ws is None else ws.numel(),
+                        _stream_handle(stream) if ws is not None else None))
+
+
+def anchor_capture(hidden_states, pool, src_rows, dst_rows, *, ws=None, stream=None):
+    """sr_anchor_capture: pool[dst_rows[i]] = hidden_states[src_rows[i]] (bf16
+    CUDA tensors, int32 index tensors on the same device)."""
+    if ws is None:
+        ws = workspace(256, hidden_states.device)
+    _check(capture_call(capture_args(hidden_states, pool, src_rows, dst_rows), ws, stream))
+    return ws
+
+
+def sparse_anchor_plan(n_prefix, *, page_size=64, anchors_per_page=4, layout=SR_ANCHORS_PAGE_TAIL, k_max=512,
+                       ratio=0.05, block_table=None):
+    """sr_sparse_anchor_plan (host): (positions, pool_rows) of the anchors a
+    token-sparse replay of an n_prefix-token prefix reads, as Python lists."""
+    bt = None
+    if block_table is not None:
+        bt = (_i32 * len(block_table))(*block_table)
+    a = AnchorPlanArgs(int(n_prefix), page_size, anchors_per_page, layout, k_max, float(ratio), bt)
+    count = ctypes.c_int64(0)
+    # first call sizes the arrays: *count is set only once the arguments are valid
+    st = _plan(ctypes.byref(a), None, None, 0, ctypes.byref(count))
+    k = count.value
+    if st != SR_OK and k == 0:
+        _check(st)
+    pos = (ctypes.c_int64 * max(k, 1))()
+    rows = (_i32 * max(k, 1))()
+    _check(_plan(ctypes.byref(a), pos, rows, k, ctypes.byref(count)))
+    return list(pos[:k]), list(rows[:k])

@@ -3,8 +3,12 @@
 // A group is a run of Gated DeltaNet layers between two full-attention
 // layers; its anchor is the hidden entering it.  Every state starts at zero
 // and full-attention layers are skipped ("SuffixReplay", Algorithm Design 1;
-// "Tail-Replay", Sec. 3).  Per layer, all groups of the call advance together
-// (each launch covers every group through per-group pointers):
+// "Tail-Replay", Sec. 3).  Two options widen the replay: anchors gathered
+// from a pool through an index table (token-wise sparse anchors,
+// "SuffixReplay", Algorithm Design 2), and initial states per layer, which
+// continue a previous call exactly (the extend step that follows a replay).
+// Per layer, all groups of the call advance together (each launch covers
+// every group through per-group pointers):
 //   row_prep(x, w_in_norm) -> in_proj GEMM (fp32 out, RMSNorm factor in the
 //   epilogue) -> conv + gates (+ conv state) -> chunked gated-delta recurrence
 //   -> gated norm -> out_proj GEMM (+= residual) -> row_prep(x, w_post_norm)
@@ -103,6 +107,8 @@ sr_status validate(const sr_group_args *a) {
     if (a->precision != SR_PREC_SPLIT && a->precision != SR_PREC_BF16)
         return set_error(SR_ERR_INVALID_ARG, "bad precision");
     if (!(a->eps > 0.f)) return set_error(SR_ERR_INVALID_ARG, "eps must be > 0");
+    if (a->anchor_index && a->anchor_rows < 1)
+        return set_error(SR_ERR_INVALID_ARG, "anchor_index needs anchor_rows >= 1 (got %d)", a->anchor_rows);
     for (int g = 0; g < a->n_groups; ++g) {
         if (!a->anchors[g]) return set_error(SR_ERR_INVALID_ARG, "anchors[%d] is NULL", g);
         for (int l = 0; l < a->n_layers; ++l) {
@@ -167,12 +173,24 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
     uint32_t *status = static_cast<uint32_t *>(ws);
     SR_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
     if (m.T == 0 || m.N == 0) {
-        // nothing to replay: every state is zero, every conv state is zero
+        // no tokens: every state is its initial state (zero for a replay)
+        const size_t s_bytes = size_t(m.N) * m.hv * m.d * m.d * 4, c_bytes = size_t(m.N) * m.conv_dim * 3 * 2;
         for (int g = 0; g < m.G; ++g)
             for (int l = 0; l < m.L; ++l) {
                 const sr_layer_outputs &o = a->outputs[g * m.L + l];
-                SR_TRY(cudaMemsetAsync(o.s_out, 0, size_t(m.N) * m.hv * m.d * m.d * 4, st));
-                SR_TRY(cudaMemsetAsync(o.conv_out, 0, size_t(m.N) * m.conv_dim * 3 * 2, st));
+                const sr_layer_state *in = a->initial ? &a->initial[g * m.L + l] : nullptr;
+                if (in && in->s_in) {
+                    if (in->s_in != o.s_out)
+                        SR_TRY(cudaMemcpyAsync(o.s_out, in->s_in, s_bytes, cudaMemcpyDeviceToDevice, st));
+                } else {
+                    SR_TRY(cudaMemsetAsync(o.s_out, 0, s_bytes, st));
+                }
+                if (in && in->conv_in) {
+                    if (in->conv_in != o.conv_out)
+                        SR_TRY(cudaMemcpyAsync(o.conv_out, in->conv_in, c_bytes, cudaMemcpyDeviceToDevice, st));
+                } else {
+                    SR_TRY(cudaMemsetAsync(o.conv_out, 0, c_bytes, st));
+                }
             }
         return SR_OK;
     }
@@ -188,6 +206,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         const bool stop = last && a->mode == SR_MODE_SKIP;
         auto W = [&](int g) -> const sr_layer_weights & { return a->weights[g * m.L + l]; };
         auto O = [&](int g) -> const sr_layer_outputs & { return a->outputs[g * m.L + l]; };
+        auto I = [&](int g) -> const sr_layer_state * { return a->initial ? &a->initial[g * m.L + l] : nullptr; };
 
         // (1) A = x * w_in_norm (hi/lo), r = RMSNorm factor; layer 0 also seeds the fp32 residual stream
         RowPrepBatch rp{};
@@ -200,6 +219,9 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             rp.x32_out[g] = l == 0 ? B[g].x32 : nullptr;
         }
         rp.T = T; rp.H = m.H; rp.x_f32 = l == 0 ? 0 : 1; rp.eps = a->eps;
+        rp.idx = l == 0 ? a->anchor_index : nullptr;  // sparse anchors: gather from the pool
+        rp.x_rows = a->anchor_index ? a->anchor_rows : T;
+        rp.status = status;
         SR_TRY(prof.begin(SR_K_ROW_PREP));
         SR_TRY(row_prep(rp, G, st));
         SR_TRY(prof.end());
@@ -227,6 +249,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             cb.gate[g] = B[g].gate;
             cb.beta[g] = B[g].beta;
             cb.conv_out[g] = static_cast<__nv_bfloat16 *>(O(g).conv_out);
+            cb.conv_in[g] = I(g) ? static_cast<const __nv_bfloat16 *>(I(g)->conv_in) : nullptr;
         }
         cb.cu = a->cu_seqlens; cb.n_seqs = m.N; cb.T = T; cb.ld = m.proj; cb.h_k = m.hk; cb.h_v = m.hv;
         cb.conv_dim = m.conv_dim; cb.b_off = m.conv_dim + m.vd;
@@ -234,7 +257,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         SR_TRY(conv_gates(cb, G, st));
         SR_TRY(prof.end());
 
-        // (4) gated-delta recurrence from a zero state
+        // (4) gated-delta recurrence from a zero state (or s_in on a continuation)
         GdnBatch gb{};
         for (int g = 0; g < G; ++g) {
             gb.q[g] = B[g].q;
@@ -244,7 +267,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             gb.v_lo[g] = B[g].v_lo;
             gb.g[g] = B[g].gate;
             gb.beta[g] = B[g].beta;
-            gb.h0[g] = nullptr;
+            gb.h0[g] = I(g) ? I(g)->s_in : nullptr;
             gb.o[g] = stop ? nullptr : B[g].o;
             gb.s_out[g] = O(g).s_out;
         }
@@ -284,6 +307,8 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             rp.x32_out[g] = nullptr;
         }
         rp.x_f32 = 1;
+        rp.idx = nullptr;
+        rp.x_rows = T;
         SR_TRY(prof.begin(SR_K_ROW_PREP));
         SR_TRY(row_prep(rp, G, st));
         SR_TRY(prof.end());

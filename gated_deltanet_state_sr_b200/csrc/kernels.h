@@ -52,7 +52,9 @@ struct RowPrepBatch {
     __nv_bfloat16 *a_lo[kMaxGroups];      // [T, H] low part, may be null
     float *r[kMaxGroups];                 // [T] 1 / sqrt(mean(x^2) + eps)
     float *x32_out[kMaxGroups];           // [T, H] fp32 copy of x, may be null
-    int T, H, x_f32;
+    const int32_t *idx;                   // [T] row of x that token t reads, may be null (row t)
+    uint32_t *status;                     // device status word (bad index flag)
+    int T, H, x_f32, x_rows;              // x_rows: rows of x (bounds of idx)
     float eps;
 };
 cudaError_t row_prep(const RowPrepBatch &b, int n_groups, cudaStream_t st);
@@ -70,6 +72,7 @@ struct ConvBatch {
     float *gate[kMaxGroups];               // [T, h_v]
     float *beta[kMaxGroups];
     __nv_bfloat16 *conv_out[kMaxGroups];   // [n_seqs, conv_dim, 3]
+    const __nv_bfloat16 *conv_in[kMaxGroups];  // [n_seqs, conv_dim, 3] history before each sequence, may be null
     const int32_t *cu;
     int n_seqs, T, ld, h_k, h_v, conv_dim, b_off;  // b_off: column of b (a follows at + h_v)
 };

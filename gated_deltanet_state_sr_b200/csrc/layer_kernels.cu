@@ -4,9 +4,11 @@
 //   row_prep     A = x * w (as an exact hi + lo bf16 pair when split) and the
 //                RMSNorm factor r_t = 1/sqrt(mean(x_t^2) + eps); the GEMM that
 //                consumes A applies r_t in its epilogue, so RMSNorm(x) w W^T is
-//                formed without rounding the normalised activations.
-//   conv_gates   causal depthwise conv (width 4, zero left padding per
-//                sequence) + SiLU over [q|k|v], per-head L2 norm of q and k,
+//                formed without rounding the normalised activations.  Row t of
+//                x is optionally gathered through an anchor index table.
+//   conv_gates   causal depthwise conv (width 4; zero left padding per
+//                sequence, or the stored history of a continuation) + SiLU
+//                over [q|k|v], per-head L2 norm of q and k,
 //                g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b).
 //   conv_state   the last (width-1) pre-conv rows of each sequence.
 //   gated_norm   y = RMSNorm_head(o) w_g * SiLU(z) (hi + lo when split).
@@ -43,16 +45,31 @@ __global__ void __launch_bounds__(256) row_prep_kernel(const __grid_constant__ R
     const int row = blockIdx.x * 8 + warp;
     if (row >= p.T) return;
     const int H = p.H;
-    const size_t base = size_t(row) * H;
+    const size_t base = size_t(row) * H;  // destination row (packed token)
+    // source row: the token itself, or its entry of the anchor index table
+    int src = row;
+    bool zero = false;
+    if (p.idx) {
+        src = p.idx[row];
+        if (src < 0 || src >= p.x_rows) {
+            zero = true;
+            src = 0;
+            if (lane == 0) atomicOr(p.status, SR_DEV_BAD_INDEX);
+        }
+    }
+    const size_t sbase = size_t(src) * H;
     float ss = 0.f;
     for (int c = lane * 8; c < H; c += 256) {
         float xv[8];
-        if (p.x_f32) {
-            const float4 *xs = reinterpret_cast<const float4 *>(static_cast<const float *>(p.x[g]) + base + c);
+        if (zero) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xv[e] = 0.f;
+        } else if (p.x_f32) {
+            const float4 *xs = reinterpret_cast<const float4 *>(static_cast<const float *>(p.x[g]) + sbase + c);
             const float4 a = xs[0], b = xs[1];
             xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w; xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
         } else {
-            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x[g]) + base + c);
+            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x[g]) + sbase + c);
             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -153,16 +170,31 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
         }
         float c[4];
         const float *x0 = reinterpret_cast<const float *>(&x[i + 3]);
-        const float *x1 = reinterpret_cast<const float *>(&x[i + 2]);
-        const float *x2 = reinterpret_cast<const float *>(&x[i + 1]);
-        const float *x3 = reinterpret_cast<const float *>(&x[i]);
-        const bool v1 = t - 1 >= bos, v2 = t - 2 >= bos, v3 = t - 3 >= bos;
+        // rows t-1, t-2, t-3: inside the sequence from the loaded window;
+        // before its start zero (replay) or the stored history (continuation)
+        float xm[3][4];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int tj = t - 1 - j;
+            const float *xr = reinterpret_cast<const float *>(&x[i + 2 - j]);
+            if (tj >= bos) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xm[j][e] = xr[e];
+            } else if (p.conv_in[g]) {
+                const __nv_bfloat16 *hp = p.conv_in[g] + (size_t(n) * p.conv_dim + ch) * 3 + (3 - bos + tj);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xm[j][e] = __bfloat162float(hp[e * 3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xm[j][e] = 0.f;
+            }
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             float acc = w[e][3] * x0[e];
-            if (v1) acc = fmaf(w[e][2], x1[e], acc);
-            if (v2) acc = fmaf(w[e][1], x2[e], acc);
-            if (v3) acc = fmaf(w[e][0], x3[e], acc);
+            acc = fmaf(w[e][2], xm[0][e], acc);
+            acc = fmaf(w[e][1], xm[1][e], acc);
+            acc = fmaf(w[e][0], xm[2][e], acc);
             c[e] = acc * sigmoidf_(acc);
         }
         if (head < n_qk) {
@@ -189,18 +221,30 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
     }
 }
 
-// conv_state[n, ch, j] = pre-conv row (eos - W + 1 + j) of sequence n, 0 before its start.
+// conv_state[n, ch, j] = pre-conv row (eos - W + 1 + j) of sequence n; rows
+// before its start come from its history (zero, or conv_in on a continuation).
+// The history is read before anything is written, so conv_in may alias conv_out.
 __global__ void __launch_bounds__(128) conv_state_kernel(const __grid_constant__ ConvBatch p) {
     const int g = blockIdx.z, n = blockIdx.x;
     const int ch = blockIdx.y * 128 + threadIdx.x;
     if (ch >= p.conv_dim) return;
     const int bos = max(p.cu[n], 0), eos = min(p.cu[n + 1], p.T);
-    __nv_bfloat16 *out = p.conv_out[g] + (size_t(n) * p.conv_dim + ch) * 3;
+    const size_t off = (size_t(n) * p.conv_dim + ch) * 3;
+    float hist[3] = {0.f, 0.f, 0.f};
+    if (p.conv_in[g]) {
+#pragma unroll
+        for (int j = 0; j < 3; ++j) hist[j] = __bfloat162float(p.conv_in[g][off + j]);
+    }
+    float val[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
         const int t = eos - 3 + j;
-        out[j] = __float2bfloat16_rn(t >= bos ? p.p[g][size_t(t) * p.ld + ch] : 0.f);
+        const int hj = 3 - bos + t;  // history slot of a row before the start (in [0, 3) when t < bos)
+        val[j] = t >= bos ? p.p[g][size_t(t) * p.ld + ch] : (hj >= 0 ? hist[hj] : 0.f);
     }
+    __nv_bfloat16 *out = p.conv_out[g] + off;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) out[j] = __float2bfloat16_rn(val[j]);
 }
 
 // ---------------------------------------------------------------- gated_norm

@@ -77,6 +77,7 @@ typedef enum sr_dtype { SR_BF16 = 0, SR_FP32 = 1 } sr_dtype;
 #define SR_DEV_BAD_CU_SEQLENS 0x1u  /* cu[n] > cu[n+1], cu[n+1] > total, cu[0] != 0 */
 #define SR_DEV_SEQ_TOO_LONG 0x2u    /* a sequence is longer than max_seqlen       */
 #define SR_DEV_TIMEOUT 0x4u         /* a bounded on-chip wait gave up (kernel exited early) */
+#define SR_DEV_BAD_INDEX 0x8u       /* an anchor or row index outside its table (row read as zero / skipped) */
 
 /* Kernel selection for sr_gdn_replay. */
 typedef enum sr_gdn_algo {
@@ -217,6 +218,20 @@ typedef struct sr_layer_outputs {
                          MLP; must be NULL for the last layer in SR_MODE_SKIP */
 } sr_layer_outputs;
 
+/* Initial states of one layer, for a continuation.  A replay starts every
+ * layer from zero; the unmatched tokens after it are then processed from the
+ * rebuilt states ("Tail-Replay", Sec. 3; "SuffixReplay", Pipelined Replay
+ * Path: extend consumes the reconstructed state).  With these set, layer l's
+ * recurrence starts at s_in and its causal conv reads conv_in's rows as the
+ * (conv_width-1) tokens before each sequence, so the call continues exactly
+ * where a previous call over the preceding tokens stopped (up to the bf16
+ * rounding of the stored conv state).  s_in may equal the layer's s_out and
+ * conv_in its conv_out (in-place continuation). */
+typedef struct sr_layer_state {
+    const float *s_in;    /* [n_seqs, h_v, d_v, d_k] fp32, or NULL: zero state */
+    const void *conv_in;  /* [n_seqs, conv_dim, conv_width-1] bf16, oldest row first, or NULL: zero padding */
+} sr_layer_state;
+
 typedef enum sr_group_mode { SR_MODE_SKIP = 0, SR_MODE_FULL = 1 } sr_group_mode;
 
 /* Arithmetic of the group's activations.
@@ -269,6 +284,17 @@ typedef struct sr_group_args {
     int32_t mode;                     /* sr_group_mode */
     int32_t precision;                /* sr_group_precision */
     sr_profile *profile;              /* host, may be NULL */
+    /* Continuation (see sr_layer_state): host array [n_groups * n_layers],
+     * group-major, or NULL for a replay from zero. */
+    const sr_layer_state *initial;
+    /* Token-wise sparse anchors ("SuffixReplay", Algorithm Design 2): when
+     * non-NULL, a device int32 array [total_tokens]; replay token t of every
+     * group reads row anchor_index[t] of that group's anchor pool
+     * anchors[g] ([anchor_rows, hidden] bf16).  An index outside
+     * [0, anchor_rows) reads a zero row and sets SR_DEV_BAD_INDEX.  NULL:
+     * anchors[g] holds the packed suffix itself ([total_tokens, hidden]). */
+    const int32_t *anchor_index;
+    int32_t anchor_rows;
 } sr_group_args;
 
 SR_API size_t sr_group_replay_workspace(const sr_group_args *args);
@@ -303,6 +329,69 @@ SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, siz
 
 SR_API sr_status sr_group_replay_noalloc(const sr_group_args *args, void *stream,
                                          const void **status_scratch);
+
+/* ------------------------------------------------------------------------
+ * sr_anchor_capture -- write selected hidden rows into an anchor pool.
+ *
+ * The forward pass that serves a request caches, for each replay group, the
+ * hidden entering the group at selected token positions: the anchors that a
+ * later replay starts from.  The pages store them in a sidecar pool beside
+ * the KV pages, written by indexed copies inside captured CUDA graphs from a
+ * destination table prepared on the host ("SuffixReplay", System Design,
+ * Anchor Sidecar).  This call is that indexed copy:
+ *     pool[dst_rows[i], :] = hidden_states[src_rows[i], :]   for i < n.
+ * Layout: hidden_states [src_rows_total, hidden] bf16 and pool [pool_rows,
+ * hidden] bf16, row-major, both 16-byte aligned, hidden % 8 == 0; src_rows and
+ * dst_rows are device int32 [n].  Two entries with the same dst_rows race
+ * (one of them wins).  A pair with an index out of range is skipped and sets
+ * SR_DEV_BAD_INDEX in the workspace status word.  Workspace: 256 bytes (the
+ * status word).  No allocation, no host synchronisation: the call can be
+ * captured into a CUDA graph whose index tables the host rewrites in place
+ * between launches.
+ * ---------------------------------------------------------------------- */
+typedef struct sr_capture_args {
+    const void *hidden_states; /* [src_rows_total, hidden] bf16, device */
+    void *pool;                /* [pool_rows, hidden] bf16, device */
+    const int32_t *src_rows;   /* [n] device */
+    const int32_t *dst_rows;   /* [n] device */
+    int32_t n, hidden, src_rows_total, pool_rows;
+} sr_capture_args;
+
+SR_API sr_status sr_anchor_capture(const sr_capture_args *args, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/* ------------------------------------------------------------------------
+ * sr_sparse_anchor_plan -- host: which anchors a token-sparse replay reads.
+ *
+ * Token-wise sparse anchors ("SuffixReplay", Algorithm Design 2): each page
+ * of page_size tokens (64 on the pages) keeps anchors_per_page of its
+ * positions (density 1/16: 4 per page); SR_ANCHORS_PAGE_TAIL puts them on
+ * the page's last positions (the dense sampling near the page boundary that
+ * the pages prefer), SR_ANCHORS_UNIFORM at offsets (i+1) page_size /
+ * anchors_per_page - 1.  The replay budget is counted in anchors (Algorithm
+ * Design 3): k = min(ceil(ratio * n_prefix), k_max, anchors present), and the
+ * replay reads the last k anchors of the prefix, oldest first.
+ * Outputs (host arrays of `capacity` entries, either may be NULL):
+ * positions[j], the token position of replayed anchor j, and pool_rows[j],
+ * its row in a page-major pool holding anchors_per_page rows per page:
+ * block_table[page] * anchors_per_page + slot (block_table NULL: the page
+ * index itself).  *count receives k; capacity < k is SR_ERR_INVALID_ARG
+ * (with *count set, so the caller can size its arrays).  Pure host code.
+ * ---------------------------------------------------------------------- */
+typedef enum sr_anchor_layout { SR_ANCHORS_PAGE_TAIL = 0, SR_ANCHORS_UNIFORM = 1 } sr_anchor_layout;
+
+typedef struct sr_anchor_plan_args {
+    int64_t n_prefix;             /* matched prefix length in tokens */
+    int32_t page_size;            /* tokens per page (64) */
+    int32_t anchors_per_page;     /* page_size * density (4) */
+    int32_t layout;               /* sr_anchor_layout */
+    int32_t k_max;                /* budget cap in anchors (512 / 256 on the pages) */
+    double ratio;                 /* budget ratio (0.05) */
+    const int32_t *block_table;   /* host [pages], may be NULL */
+} sr_anchor_plan_args;
+
+SR_API sr_status sr_sparse_anchor_plan(const sr_anchor_plan_args *args, int64_t *positions, int32_t *pool_rows,
+                                       int64_t capacity, int64_t *count);
 
 /* ------------------------------------------------------------------------
  * Status and diagnostics.

@@ -119,7 +119,8 @@ def test_ctypes_structs_match_the_c_header(tmp_path):
     import subprocess
     structs = {"sr_gdn_args": sr.GdnArgs, "sr_mamba2_args": sr.Mamba2Args,
                "sr_layer_weights": sr.LayerWeights, "sr_layer_outputs": sr.LayerOutputs,
-               "sr_group_args": sr.GroupArgs, "sr_profile": sr.Profile}
+               "sr_group_args": sr.GroupArgs, "sr_profile": sr.Profile, "sr_layer_state": sr.LayerState,
+               "sr_capture_args": sr.CaptureArgs, "sr_anchor_plan_args": sr.AnchorPlanArgs}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "sr/sr.h"', 'int main(void) {']
     for cname, py in structs.items():
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
@@ -137,3 +138,33 @@ def test_ctypes_structs_match_the_c_header(tmp_path):
         assert int(out[cname]) == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
             assert int(out[f"{cname}.{f}"]) == getattr(py, f).offset, f"{cname}.{f}"
+
+
+def _fake_group_args(**over):
+    """A GroupArgs over fake (never dereferenced) device pointers: host
+    validation runs before any CUDA work, so no GPU is needed."""
+    fake = 0x10000
+    anc = (ctypes.c_void_p * 1)(fake)
+    w = (sr.LayerWeights * 1)(sr.LayerWeights(*([fake] * 11)))
+    o = (sr.LayerOutputs * 1)(sr.LayerOutputs(fake, fake, None))
+    a = sr.GroupArgs(anc, fake, w, o, 1, 1, 1, 16, 16, 256, 512, 2, 4, 128, 128, 4, 1e-6, sr.SR_MODE_SKIP, 0,
+                     None, None, None, 0)
+    for k, v in over.items():
+        setattr(a, k, v)
+    a._keep = (anc, w, o)
+    return a
+
+
+def test_group_sparse_anchors_need_pool_rows():
+    a = _fake_group_args(anchor_index=0x20000, anchor_rows=0)
+    assert sr.group_workspace_bytes(a) == 0
+    assert sr.group_call(a, None) == sr.SR_ERR_INVALID_ARG
+    assert "anchor_rows" in sr.last_error()
+    a = _fake_group_args(anchor_index=0x20000, anchor_rows=5)
+    assert sr.group_workspace_bytes(a) > 0
+
+
+def test_group_workspace_independent_of_continuation():
+    """Initial states are read in place: a continuation needs no extra scratch."""
+    init = (sr.LayerState * 1)(sr.LayerState(0x30000, 0x40000))
+    assert sr.group_workspace_bytes(_fake_group_args(initial=init)) == sr.group_workspace_bytes(_fake_group_args())
