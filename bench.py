@@ -224,8 +224,21 @@ class GroupReplay:
             self.gis = [W.model_group(prefix, ratio, g, seed=0x5EED0003 + 1000 * rank) for g in range(8)]
             self.desc = (f"whole model: [GDN,GDN,GDN,FA]x8, 8 groups replayed group-parallel, FA skipped, "
                          f"suffix k = ceil({ratio} * {prefix}) = {W.model_suffix(prefix, ratio)}")
+        elif name == "sparse_32k":
+            # token-sparse anchors: each group's pool holds the 2048 anchors of a 32K
+            # prefix (4 per 64-token page); the replay gathers the last
+            # k = min(ceil(0.05 * 32768), 512) = 512 through the planner's pool rows
+            n_pages = W.SPARSE_PREFIX // W.SPARSE_PAGE
+            k = min(W.model_suffix(W.SPARSE_PREFIX, 0.05), W.SPARSE_K_MAX)
+            self.gis = [W.anchor_pool_group(n_pages * W.SPARSE_PER_PAGE, k, seed=0x5EED0005 + 1000 * rank + g)
+                        for g in range(8)]
+            self.block_table = W.block_table(n_pages, 0x5EED0005 + 1000 * rank)
+            self.desc = (f"whole model, token-sparse anchors: 8 groups replay k = {k} anchors gathered from "
+                         f"pools of {n_pages * W.SPARSE_PER_PAGE} (32K prefix, 4 per 64-token page, "
+                         f"shuffled block table)")
         else:
             raise ValueError(name)
+        self.sparse = name == "sparse_32k"
         self.precision = precision
         s = self.gis[0].shape
         self.s = s
@@ -288,6 +301,14 @@ class GroupReplay:
         self.kw = dict(max_seqlen=self.max_len, hidden=s.hidden, inter=s.inter, h_k=s.h_k, h_v=s.h_v, d=s.d_k,
                        eps=s.eps, mode=sr.SR_MODE_SKIP,
                        precision=sr.SR_PREC_SPLIT if self.precision == "split" else sr.SR_PREC_BF16)
+        if self.sparse:
+            _, rows = sr.sparse_anchor_plan(W.SPARSE_PREFIX, page_size=W.SPARSE_PAGE,
+                                            anchors_per_page=W.SPARSE_PER_PAGE, k_max=W.SPARSE_K_MAX, ratio=0.05,
+                                            block_table=self.block_table)
+            assert len(rows) == self.tokens
+            self.h_index = torch.tensor(rows, dtype=torch.int32).pin_memory()
+            self.index = self.h_index.to(dev)
+            self.kw["anchor_index"] = self.index
         self.outputs = sr.group_replay(self.anchors, self.cu, self.weights, **self.kw)
         args = sr.group_args(self.anchors, self.cu, self.weights, self.outputs, **self.kw)
         self.ws = sr.workspace(sr.group_workspace_bytes(args), dev)
@@ -307,6 +328,8 @@ class GroupReplay:
         for h, d in zip(self.h_anchors, self.anchors):
             d.copy_(h, non_blocking=True)
         self.cu.copy_(self.h_cu, non_blocking=True)
+        if self.sparse:
+            self.index.copy_(self.h_index, non_blocking=True)
         self.step()
         for hrow, drow in zip(self.h_out, self.outputs):
             for (hs, hc), (ds, dc, _) in zip(hrow, drow):
@@ -315,7 +338,8 @@ class GroupReplay:
 
     @property
     def h2d_bytes(self):
-        return sum(t.numel() * t.element_size() for t in self.h_anchors) + self.h_cu.numel() * 4
+        return (sum(t.numel() * t.element_size() for t in self.h_anchors) + self.h_cu.numel() * 4
+                + (self.h_index.numel() * 4 if self.sparse else 0))
 
     @property
     def d2h_bytes(self):
@@ -331,7 +355,7 @@ class GroupReplay:
         from oracle import layers as OL
         gi = self.gis[0]
         T = self.tokens if tokens is None else min(tokens, self.tokens)
-        x = oracle._f64(gi.anchors[:T])
+        x = oracle._f64(gi.anchors[:T])  # sparse pools: the first T rows (the cost does not depend on which)
         cu = np.array([0, T])
         reps, t0 = 0, time.perf_counter()
         while True:
@@ -429,6 +453,7 @@ class Mamba2Replay:
             oracle.num_threads()
 
 WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "group": GroupReplay, "mamba2": Mamba2Replay,
+             "sparse_32k": GroupReplay,
              **{f"model_{m}_{r}": GroupReplay for m in ("8k", "16k", "32k") for r in ("5", "10")}}
 DEFAULT_WORKLOAD = "model_32k_5"
 

@@ -265,6 +265,27 @@ def model_group(prefix, ratio, g, seed=0x5EED0003, shape=None) -> GroupInputs:
     return group_inputs(seed + g, [model_suffix(prefix, ratio)], shape=shape)
 
 
+SPARSE_PREFIX = 32768     # matched prefix of the token-sparse replay workload
+SPARSE_PAGE = 64          # tokens per page
+SPARSE_PER_PAGE = 4       # anchors per page (density 1/16)
+SPARSE_K_MAX = 512        # replay budget cap in anchors
+
+
+def anchor_pool_group(pool_rows, k, seed, shape=None, n_layers=3) -> GroupInputs:
+    """A group whose `anchors` is an anchor pool of pool_rows random bf16
+    hiddens (N(0,1)) from which a replay of k tokens gathers its rows; the
+    weights follow layer_weights."""
+    s = shape or LayerShape()
+    pool = normal(seed, "pool", (pool_rows, s.hidden), 1.0)
+    layers = [layer_weights(seed, l, s) for l in range(n_layers)]
+    return GroupInputs(pool, cu_from_lengths([k]), layers, s)
+
+
+def block_table(n_pages, seed) -> list:
+    """A seeded page -> pool-block permutation (the sidecar's page table)."""
+    return torch.randperm(n_pages, generator=substream(seed, "block_table")).tolist()
+
+
 # ---------------------------------------------------------------- Mamba2
 
 
