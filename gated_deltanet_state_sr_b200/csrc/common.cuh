@@ -47,4 +47,30 @@ __device__ __forceinline__ bool seq_bounds(const int32_t *cu, int n, int total, 
     return true;
 }
 
+// Longest-first dispatch.  A grid row r of a per-sequence kernel takes the
+// sequence of rank r in the order of decreasing length (ties: lower index
+// first), so the longest replays start in the first wave instead of trailing
+// the last one.  With more than kLongestFirstMax sequences the row keeps its
+// own index.  `scratch` is shared memory for n + 1 ints; every thread of the
+// block calls this, and it ends with a block barrier.
+constexpr int kLongestFirstMax = 256;
+__device__ __forceinline__ int longest_first(const int32_t *cu, int n, int r, int *scratch) {
+    if (n > kLongestFirstMax) return r;
+    for (int m = threadIdx.x; m < n; m += blockDim.x) scratch[m] = cu[m + 1] - cu[m];
+    __syncthreads();
+    for (int m = threadIdx.x; m < n; m += blockDim.x) {
+        const int lm = scratch[m];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) {
+            const int lj = scratch[j];
+            rank += (lj > lm) || (lj == lm && j < m);
+        }
+        if (rank == r) scratch[n] = m;
+    }
+    __syncthreads();
+    const int seq = scratch[n];
+    __syncthreads();  // the scratch may be reused right after
+    return seq;
+}
+
 }  // namespace sr

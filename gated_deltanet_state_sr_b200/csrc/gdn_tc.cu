@@ -98,7 +98,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     float *Af = reinterpret_cast<float *>(sm + oXR);
     float *Tf = reinterpret_cast<float *>(sm + oXR + C * ROWA * 4);
 
-    const int h = blockIdx.x, n = blockIdx.y, gi = blockIdx.z;
+    const int h = blockIdx.x, gi = blockIdx.z;
+    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + oXR));
     const int h_k = p.h_k, h_v = p.h_v;
     const int hk = h / (h_v / h_k);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -56,7 +56,7 @@ mamba2_chunk_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
                     float *__restrict__ s_out, int total, int max_len, int H, uint32_t *status) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     M2Smem &sm = *reinterpret_cast<M2Smem *>(smem_raw);
-    const int n = blockIdx.y;
+    const int n = longest_first(cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm.g));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hh = warp >> 2, wq = warp & 3;  // head of the pair, warp within the head
     const int tid_h = tid & 127;
