@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mma_sync.cuh"
 #include "tc.cuh"
 
 namespace sr {
@@ -55,6 +56,7 @@ constexpr uint32_t smem_bytes(bool split) {
 
 struct GdnTcParams {
     CUtensorMap q[kMaxGroups], k[kMaxGroups], v[kMaxGroups], kl[kMaxGroups], vl[kMaxGroups];
+    CUtensorMap om[kMaxGroups];  // o, for the tile store of full chunks
     const float *g[kMaxGroups];
     const float *beta[kMaxGroups];
     const float *h0[kMaxGroups];
@@ -65,6 +67,44 @@ struct GdnTcParams {
     float scale;
     uint32_t *status;
 };
+
+// One warp: acc (16 x 16 fp32 in the m16n8k16 accumulator layout, two 8-column
+// halves) += X Y for 16 x 16 fp32 blocks X, Y in shared memory (row pitch ROWA).
+// Each operand is split into exact bf16 pairs hi + lo and the product is taken
+// as Xh Yh + Xh Yl + Xl Yh, which leaves out only Xl Yl (2^-16 relative).
+__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, const float *Y, int lane) {
+    const int g = lane >> 2, q = lane & 3;
+    uint32_t ah[4], al[4];
+    const float2 x0 = *reinterpret_cast<const float2 *>(X + g * ROWA + 2 * q);
+    const float2 x1 = *reinterpret_cast<const float2 *>(X + (g + 8) * ROWA + 2 * q);
+    const float2 x2 = *reinterpret_cast<const float2 *>(X + g * ROWA + 2 * q + 8);
+    const float2 x3 = *reinterpret_cast<const float2 *>(X + (g + 8) * ROWA + 2 * q + 8);
+    ms::split_bf16(x0.x, x0.y, ah[0], al[0]);
+    ms::split_bf16(x1.x, x1.y, ah[1], al[1]);
+    ms::split_bf16(x2.x, x2.y, ah[2], al[2]);
+    ms::split_bf16(x3.x, x3.y, ah[3], al[3]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int n = 8 * nt + g;
+        uint32_t bh0, bl0, bh1, bl1;
+        ms::split_bf16(Y[(2 * q) * ROWA + n], Y[(2 * q + 1) * ROWA + n], bh0, bl0);
+        ms::split_bf16(Y[(2 * q + 8) * ROWA + n], Y[(2 * q + 9) * ROWA + n], bh1, bl1);
+        ms::mma16816(acc[nt], ah, bh0, bh1);
+        ms::mma16816(acc[nt], ah, bl0, bl1);
+        ms::mma16816(acc[nt], al, bh0, bh1);
+    }
+}
+
+// Stores sign * acc (accumulator layout of blk_mma) as a 16 x 16 fp32 block.
+__device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], int lane, float sign) {
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2 *>(Z + g * ROWA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
+        *reinterpret_cast<float2 *>(Z + (g + 8) * ROWA + 8 * nt + 2 * q) =
+            make_float2(sign * acc[nt][2], sign * acc[nt][3]);
+    }
+}
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -155,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     }
 
     const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
+    const CUtensorMap *mo = &p.om[gi];
     // Each input is refilled as soon as the last product reading it has completed.
     auto issue_k = [&](int c) {
         const int y = bos + c * C;
@@ -184,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     };
     if (tid == 0) {
         prefetch_tmap(mq); prefetch_tmap(mk); prefetch_tmap(mv);
+        if (p.o[gi]) prefetch_tmap(mo);
         if (SPLIT) { prefetch_tmap(mkl); prefetch_tmap(mvl); }
         issue_k(0);
         issue_q(0);
@@ -233,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         const bool tma_ok = mbar_wait(bar_k, kq_phase) && mbar_wait(bar_q, kq_phase);
         kq_phase ^= 1;
+        if (tid == 0) bulk_wait_read();  // the previous chunk's o tile has left the Qg region
         __syncthreads();
         if (warp == 0) {
             const float a0 = gam[2 * lane], a1 = gam[2 * lane + 1];
@@ -369,7 +412,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (check(m1)) break;
         if (tid == 0 && c + 1 < nchunks) issue_q(c + 1);  // Q read by MMA 1 and the Qg copy only
 
-        // ---- T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
+        // ---- T = (I + A)^{-1} by 16x16 blocks (A strictly lower):
+        //   T_ii  = (I + A_ii)^{-1}, fp32 forward substitution, one column per thread
+        //   B_ik  = T_ii A_ik (k < i), kept in the unused upper blocks of T
+        //   T_ij  = -sum_{k=j}^{i-1} B_ik T_kj, by block distance i - j = 1, 2, 3
+        // The block products run on mma.sync with split bf16 operands (blk_mma).
         if (tid < C) {
             const int b = tid >> 4, cc = tid & 15;
             float x[16];
@@ -391,49 +438,25 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * ROWA + 16 * b + cc] = x[r];
         }
         __syncthreads();
-        auto blk = [](int bi, int bj, int r, int cc) { return (16 * bi + r) * ROWA + 16 * bj + cc; };
-        for (int level = 1; level <= 3; ++level) {
-            const int items = (4 - level) * 64;
-            for (int it = tid; it < items; it += kThreads) {
-                const int j = it >> 6, i = j + level, r = (it >> 2) & 15, c4 = (it & 3) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int kb = j; kb < i; ++kb) {
-                    const float4 *ar = reinterpret_cast<const float4 *>(&Af[blk(i, kb, r, 0)]);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const float4 a = ar[v];
-                        const float am[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[blk(kb, j, 4 * v + e, c4)]);
-                            acc.x = fmaf(am[e], t4.x, acc.x);
-                            acc.y = fmaf(am[e], t4.y, acc.y);
-                            acc.z = fmaf(am[e], t4.z, acc.z);
-                            acc.w = fmaf(am[e], t4.w, acc.w);
-                        }
-                    }
-                }
-                *reinterpret_cast<float4 *>(&Tf[blk(j, i, r, c4)]) = acc;
+        auto blk = [](int bi, int bj) { return 16 * bi * ROWA + 16 * bj; };
+        {
+            // B_ik for (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2): warp w takes pair w
+            if (warp < 6) {
+                const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3), k = warp - i * (i - 1) / 2;
+                float acc[2][4] = {};
+                blk_mma(acc, Tf + blk(i, i), Af + blk(i, k), lane);
+                blk_store(Tf + blk(k, i), acc, lane, 1.f);  // kept in the upper block (k, i)
             }
-            __syncthreads();
-            for (int it = tid; it < items; it += kThreads) {
-                const int j = it >> 6, i = j + level, r = (it >> 2) & 15, c4 = (it & 3) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                const float4 *dr = reinterpret_cast<const float4 *>(&Tf[blk(i, i, r, 0)]);
+        }
+        __syncthreads();
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float4 d4 = dr[v];
-                    const float dm[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float4 xx = *reinterpret_cast<const float4 *>(&Tf[blk(j, i, 4 * v + e, c4)]);
-                        acc.x = fmaf(dm[e], xx.x, acc.x);
-                        acc.y = fmaf(dm[e], xx.y, acc.y);
-                        acc.z = fmaf(dm[e], xx.z, acc.z);
-                        acc.w = fmaf(dm[e], xx.w, acc.w);
-                    }
-                }
-                *reinterpret_cast<float4 *>(&Tf[blk(i, j, r, c4)]) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        for (int level = 1; level <= 3; ++level) {
+            // blocks (j + level, j), j = 0 .. 3 - level: warp j takes block j
+            if (warp + level <= 3) {
+                const int j = warp, i = j + level;
+                float acc[2][4] = {};
+                for (int k = j; k < i; ++k) blk_mma(acc, Tf + blk(k, i), Tf + blk(k, j), lane);
+                blk_store(Tf + blk(i, j), acc, lane, -1.f);
             }
             __syncthreads();
         }
@@ -581,22 +604,44 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         // K is free now: fetch the next chunk's while O is written out
         if (tid == 0 && c + 1 < nchunks) issue_k(c + 1);
 
-        // ---- o_t (bf16): thread = value channel i, 32 tokens
+        // ---- o_t (bf16): thread = value channel i, 32 tokens.  A full chunk goes
+        // through the (now free) Qg region as a [t][i] tile and one TMA store; the
+        // ragged last chunk is stored element by element, so that no row of the
+        // next sequence is touched.
+        const bool tile_store = o != nullptr && clen == C;
         if (o) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(R3 + lane_off + 32 * half, r);
             tmem_ld_wait();
-            const size_t tok0 = size_t(bos) + size_t(c) * C;
+            if (tile_store) {
+                uint8_t *ot = sm + oQG + (row >> 6) * 8192;
+                const uint32_t cofs = uint32_t(row & 7) * 2;
+                const uint32_t chunk = uint32_t(row & 63) >> 3;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int t = 32 * half + e;
-                if (t < clen) o[(tok0 + t) * v_stride + size_t(h) * D + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
+                for (int e = 0; e < 32; ++e)
+                    *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(32 * half + e, chunk) + cofs) =
+                        __float2bfloat16_rn(__uint_as_float(r[e]));
+                fence_async_smem();
+            } else {
+                const size_t tok0 = size_t(bos) + size_t(c) * C;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int t = 32 * half + e;
+                    if (t < clen)
+                        o[(tok0 + t) * v_stride + size_t(h) * D + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
+                }
             }
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0 && tile_store) {
+            tma_store_2d(mo, sm + oQG, h * D, bos + c * C);
+            tma_store_2d(mo, sm + oQG + 8192, h * D + 64, bos + c * C);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();
 
     __syncthreads();
     ok = *abort_flag == 0;
@@ -658,6 +703,7 @@ cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split
             return cudaErrorInvalidValue;
         if (split && (!map_64x64(&p.kl[g], b.k_lo[g], T, qkw) || !map_64x64(&p.vl[g], b.v_lo[g], T, vw)))
             return cudaErrorInvalidValue;
+        if (b.o[g] && !map_64x64(&p.om[g], b.o[g], T, vw)) return cudaErrorInvalidValue;
         p.g[g] = b.g[g];
         p.beta[g] = b.beta[g];
         p.h0[g] = b.h0[g];
