@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     float *bet = gam + C;                                         // [64]
     float *fb = gam + 2 * C;                                      // [64] beta_s e^{gamma_s}
     float *fu = gam + 3 * C;                                      // [64] e^{gamma_C - gamma_t}
+    float *eg = reinterpret_cast<float *>(sm + oMISC + 1536);     // [64] e^{gamma_t}
+    float *ei = eg + C;                                           // [64] e^{-gamma_t}
     uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 1024);  // K (+ k low part) landed
     uint64_t *bar_q = bar_k + 1;                                          // Q landed
     uint64_t *bar_v = bar_k + 2;                                          // V (+ v low part) landed
@@ -292,9 +294,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (check(tma_ok)) break;
         const float gC = gam[C - 1];
         if (tid < C) {  // per-column factors, read after later barriers
-            fb[tid] = bet[tid] * __expf(gam[tid]);
+            const float e = __expf(gam[tid]);
+            fb[tid] = bet[tid] * e;
             fu[tid] = __expf(gC - gam[tid]);
+            eg[tid] = e;
+            ei[tid] = __expf(-gam[tid]);
         }
+        // e^{gamma_t - gamma_s} = e^{gamma_t} e^{-gamma_s} while e^{-gamma_C} stays far from
+        // the fp32 range (gamma_C > -80); stronger decay takes the exponential of each
+        // masked difference
+        const bool fact = gC > -80.f;
 
         // ---- MMA 1: [K;Q] K^T -> R0 (rows 0-63: K K^T, rows 64-127: Q K^T)
         if (tid == 0) {
@@ -377,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             tmem_ld_wait();
             if (quad < 2) {
                 const int t = row;
-                const float gt = gam[t], bt = bet[t];
+                const float gt = gam[t], bt = bet[t], ft = fb[t];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     float a4[4];
@@ -386,23 +395,29 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
                         const int s = 32 * half + e + u;
                         float kk = __uint_as_float(r[e + u]);
                         if (SPLIT) kk += __uint_as_float(r2[e + u]);
-                        a4[u] = (s < t) ? bt * __expf(gt - gam[s]) * kk : 0.f;
+                        const float d = fact ? ft * ei[s] : bt * __expf(gt - gam[s]);
+                        a4[u] = (s < t) ? d * kk : 0.f;
                     }
                     *reinterpret_cast<float4 *>(&Af[t * ROWA + 32 * half + e]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
                 }
             } else {
                 const int t = row - 64;
-                const float gt = gam[t];
+                const float gt = gam[t], st = scale * eg[t];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint32_t w[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int s = 32 * half + 8 * q4 + 2 * u;
-                        const float d0 = __expf(s <= t ? gt - gam[s] : -INFINITY);
-                        const float d1 = __expf(s + 1 <= t ? gt - gam[s + 1] : -INFINITY);
-                        w[u] = pack2(scale * d0 * __uint_as_float(r[8 * q4 + 2 * u]),
-                                     scale * d1 * __uint_as_float(r[8 * q4 + 2 * u + 1]));
+                        float d0, d1;
+                        if (fact) {
+                            d0 = s <= t ? st * ei[s] : 0.f;
+                            d1 = s + 1 <= t ? st * ei[s + 1] : 0.f;
+                        } else {
+                            d0 = scale * __expf(s <= t ? gt - gam[s] : -INFINITY);
+                            d1 = scale * __expf(s + 1 <= t ? gt - gam[s + 1] : -INFINITY);
+                        }
+                        w[u] = pack2(d0 * __uint_as_float(r[8 * q4 + 2 * u]), d1 * __uint_as_float(r[8 * q4 + 2 * u + 1]));
                     }
                     *reinterpret_cast<uint4 *>(sm + oP + sw128(t, 4 * half + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
@@ -417,25 +432,41 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         //   B_ik  = T_ii A_ik (k < i), kept in the unused upper blocks of T
         //   T_ij  = -sum_{k=j}^{i-1} B_ik T_kj, by block distance i - j = 1, 2, 3
         // The block products run on mma.sync with split bf16 operands (blk_mma).
+        // T_ii by 8 x 8 halves: D = (I + N)^{-1} of each half by forward substitution,
+        // then the lower-left half -D2 (N21 D1) (its temporary N21 D1 sits in the
+        // unused upper-right half of the diagonal block of A)
         if (tid < C) {
-            const int b = tid >> 4, cc = tid & 15;
-            float x[16];
+            const int r0 = 8 * (tid >> 3), cc = tid & 7;
+            float x[8];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float4 *ar = reinterpret_cast<const float4 *>(&Af[(16 * b + r) * ROWA + 16 * b]);
-                float a[16];
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float4 f = ar[v];
-                    a[4 * v] = f.x; a[4 * v + 1] = f.y; a[4 * v + 2] = f.z; a[4 * v + 3] = f.w;
-                }
+            for (int r = 0; r < 8; ++r) {
+                const float4 *ar = reinterpret_cast<const float4 *>(&Af[(r0 + r) * ROWA + r0]);
+                const float4 f0 = ar[0], f1 = ar[1];
+                const float a[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
                 float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
                 for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-a[s2], x[s2], acc);
                 x[r] = (r < cc) ? 0.f : acc;
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * ROWA + 16 * b + cc] = x[r];
+            for (int r = 0; r < 8; ++r) Tf[(r0 + r) * ROWA + r0 + cc] = x[r];
+        }
+        __syncthreads();
+        {
+            const int b = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7, d0 = 16 * b;
+            float y = 0.f;  // (N21 D1)[r][cc]
+#pragma unroll
+            for (int m = 0; m < 8; ++m) y = fmaf(Af[(d0 + 8 + r) * ROWA + d0 + m], Tf[(d0 + m) * ROWA + d0 + cc], y);
+            Af[(d0 + r) * ROWA + d0 + 8 + cc] = y;
+            Tf[(d0 + r) * ROWA + d0 + 8 + cc] = 0.f;  // upper-right half of T_ii
+        }
+        __syncthreads();
+        {
+            const int b = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7, d0 = 16 * b;
+            float x = 0.f;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) x = fmaf(Tf[(d0 + 8 + r) * ROWA + d0 + 8 + m], Af[(d0 + m) * ROWA + d0 + 8 + cc], x);
+            Tf[(d0 + 8 + r) * ROWA + d0 + cc] = -x;
         }
         __syncthreads();
         auto blk = [](int bi, int bj) { return 16 * bi * ROWA + 16 * bj; };
