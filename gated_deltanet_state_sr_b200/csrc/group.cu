@@ -251,7 +251,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             cb.conv_out[g] = static_cast<__nv_bfloat16 *>(O(g).conv_out);
             cb.conv_in[g] = I(g) ? static_cast<const __nv_bfloat16 *>(I(g)->conv_in) : nullptr;
         }
-        cb.cu = a->cu_seqlens; cb.n_seqs = m.N; cb.T = T; cb.ld = m.proj; cb.h_k = m.hk; cb.h_v = m.hv;
+        cb.cu = a->cu_seqlens; cb.status = status; cb.n_seqs = m.N; cb.T = T; cb.ld = m.proj; cb.h_k = m.hk; cb.h_v = m.hv;
         cb.conv_dim = m.conv_dim; cb.b_off = m.conv_dim + m.vd;
         SR_TRY(prof.begin(SR_K_CONV));
         SR_TRY(conv_gates(cb, G, st));

@@ -43,6 +43,8 @@ cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split
 
 // 2-D bf16 TMA map (128-byte swizzle) over a row-major [rows, cols] matrix with row pitch `pitch`.
 bool make_map_bf16(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows);
+// fp32 [rows, cols] (row pitch `pitch` elements), unswizzled boxes of box_rows x box_cols.
+bool make_map_f32(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows);
 
 // Layer kernels of a replay group (layer_kernels.cu).  Arrays are indexed by group.
 struct RowPrepBatch {
@@ -60,6 +62,7 @@ struct RowPrepBatch {
 cudaError_t row_prep(const RowPrepBatch &b, int n_groups, cudaStream_t st);
 
 struct ConvBatch {
+    CUtensorMap pmap[kMaxGroups];          // p, boxes of 128 channels x (32 + 3) rows (set by conv_gates)
     const float *p[kMaxGroups];            // [T, ld] fp32 in_proj output
     const __nv_bfloat16 *conv_w[kMaxGroups];  // [conv_dim, 4]
     const float *a_log[kMaxGroups];
@@ -74,6 +77,7 @@ struct ConvBatch {
     __nv_bfloat16 *conv_out[kMaxGroups];   // [n_seqs, conv_dim, 3]
     const __nv_bfloat16 *conv_in[kMaxGroups];  // [n_seqs, conv_dim, 3] history before each sequence, may be null
     const int32_t *cu;
+    uint32_t *status;                      // device status word (timeout flag)
     int n_seqs, T, ld, h_k, h_v, conv_dim, b_off;  // b_off: column of b (a follows at + h_v)
 };
 cudaError_t conv_gates(const ConvBatch &b, int n_groups, cudaStream_t st);

@@ -17,6 +17,7 @@
 // Sec. 2 names Gated DeltaNet as the linear layer of the hybrids replayed).
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace sr {
 
@@ -36,6 +37,11 @@ __device__ __forceinline__ void split2(float a, float b, __nv_bfloat162 &hi, __n
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
 __device__ __forceinline__ float softplusf_(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+// SiLU on the per-element hot paths: hardware exp2-based __expf and the fast
+// division (a few fp32 ulp; the result is carried on as an fp32 value or an
+// exact hi + lo pair, far inside the bf16-level tolerances).  For x -> -inf the
+// quotient goes to zero (x times the reciprocal of +inf).
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 // ---------------------------------------------------------------- row_prep
 // One warp per row.  H % 8 == 0.
@@ -114,11 +120,16 @@ __device__ __forceinline__ int seq_of(const int32_t *cu, int n_seqs, int t) {
     return lo;
 }
 
-// blockIdx.y < 2 h_k + h_v: one 128-channel head of [q|k|v]; warp w takes
-// tokens t0 + 8w .. t0 + 8w + 7 and lane l channels 4l .. 4l+3, so the
-// per-head L2 norm is a warp reduction.  All 11 input rows (3 of history +
-// 8) are loaded before any arithmetic.  blockIdx.y == 2 h_k + h_v: gates.
+constexpr int kConvRows = kConvTok + 3;  // the block's tokens and the 3 rows before them
+
+// blockIdx.y < 2 h_k + h_v: one 128-channel head of [q|k|v].  One TMA tile
+// load brings the block's 32 rows and the 3 rows before them (rows outside
+// [0, T) read as zero) into shared memory; warp w then takes tokens
+// t0 + 8w .. t0 + 8w + 7 and lane l channels 4l .. 4l+3, so the per-head L2
+// norm is a warp reduction.  blockIdx.y == 2 h_k + h_v: gates.
 __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__ ConvBatch p) {
+    __shared__ __align__(128) float tile[kConvRows * 128];
+    __shared__ __align__(8) uint64_t bar;
     const int g = blockIdx.z;
     const int head = blockIdx.y;
     const int t0 = blockIdx.x * kConvTok;
@@ -136,6 +147,21 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
         }
         return;
     }
+    if (tid == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(&bar, kConvRows * 128 * 4);
+        tc::tma_load_2d(tile, &p.pmap[g], &bar, head * 128, t0 - 3);
+    }
+    __syncthreads();
+    if (!tc::mbar_wait(&bar, 0)) {
+        // give the copy a second bounded wait before the block's shared memory goes away
+        if (tid == 0) {
+            atomicOr(p.status, SR_DEV_TIMEOUT);
+            tc::mbar_wait(&bar, 0);
+        }
+        return;
+    }
     const int warp = tid >> 5, lane = tid & 31;
     const int tw = t0 + warp * kWarpTok;  // first token of this warp
     if (tw >= p.T) return;
@@ -148,58 +174,16 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
         const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
         w[c][0] = a.x; w[c][1] = a.y; w[c][2] = b.x; w[c][3] = b.y;
     }
-    // rows tw-3 .. tw+7 (clamped into [0, T); masked below)
-    float4 x[kWarpTok + 3];
-#pragma unroll
-    for (int r = 0; r < kWarpTok + 3; ++r) {
-        const int t = tw - 3 + r;
-        const int tc = t < 0 ? 0 : (t >= p.T ? p.T - 1 : t);
-        x[r] = *reinterpret_cast<const float4 *>(P + size_t(tc) * p.ld + ch);
-    }
+    // tile row j holds token t0 - 3 + j; this warp's rows tw-3 .. tw+7 start at row 8 warp
+    const float4 *x = reinterpret_cast<const float4 *>(tile) + (warp * kWarpTok) * 32 + lane;
     int n = seq_of(p.cu, p.n_seqs, tw);
     int eos = p.cu[n + 1];
     int bos = max(p.cu[n], 0);
-#pragma unroll
-    for (int i = 0; i < kWarpTok; ++i) {
-        const int t = tw + i;
-        if (t >= p.T) break;
-        while (t >= eos && n + 1 < p.n_seqs) {
-            ++n;
-            bos = max(p.cu[n], 0);
-            eos = p.cu[n + 1];
-        }
-        float c[4];
-        const float *x0 = reinterpret_cast<const float *>(&x[i + 3]);
-        // rows t-1, t-2, t-3: inside the sequence from the loaded window;
-        // before its start zero (replay) or the stored history (continuation)
-        float xm[3][4];
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-            const int tj = t - 1 - j;
-            const float *xr = reinterpret_cast<const float *>(&x[i + 2 - j]);
-            if (tj >= bos) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) xm[j][e] = xr[e];
-            } else if (p.conv_in[g]) {
-                const __nv_bfloat16 *hp = p.conv_in[g] + (size_t(n) * p.conv_dim + ch) * 3 + (3 - bos + tj);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) xm[j][e] = __bfloat162float(hp[e * 3]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) xm[j][e] = 0.f;
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float acc = w[e][3] * x0[e];
-            acc = fmaf(w[e][2], xm[0][e], acc);
-            acc = fmaf(w[e][1], xm[1][e], acc);
-            acc = fmaf(w[e][0], xm[2][e], acc);
-            c[e] = acc * sigmoidf_(acc);
-        }
+    // SiLU'd conv output of token t -> (L2 norm for q, k) -> bf16 (hi + lo) stores
+    auto emit = [&](int t, float (&c)[4]) {
         if (head < n_qk) {
             const float ss = warp_sum(c[0] * c[0] + c[1] * c[1] + c[2] * c[2] + c[3] * c[3]);
-            const float inv = 1.f / sqrtf(ss + 1e-6f);
+            const float inv = rsqrtf(ss + 1e-6f);
 #pragma unroll
             for (int e = 0; e < 4; ++e) c[e] *= inv;
         }
@@ -218,6 +202,74 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
             *reinterpret_cast<uint2 *>(p.v[g] + o) = hv;
             if (p.v_lo[g]) *reinterpret_cast<uint2 *>(p.v_lo[g] + o) = lv;
         }
+    };
+    // fast path: the warp's tokens and the 3 rows before them all lie inside one
+    // sequence, so no tap is masked; a rolling window keeps the previous rows in
+    // registers (same arithmetic, in the same order, as the general path)
+    if (tw - 3 >= bos && tw + kWarpTok <= eos && tw + kWarpTok <= p.T) {
+        float4 h3 = x[0], h2 = x[32], h1 = x[64];
+#pragma unroll
+        for (int i = 0; i < kWarpTok; ++i) {
+            const float4 x0 = x[(i + 3) * 32];
+            const float a0[4] = {x0.x, x0.y, x0.z, x0.w}, a1[4] = {h1.x, h1.y, h1.z, h1.w};
+            const float a2[4] = {h2.x, h2.y, h2.z, h2.w}, a3[4] = {h3.x, h3.y, h3.z, h3.w};
+            float c[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float acc = w[e][3] * a0[e];
+                acc = fmaf(w[e][2], a1[e], acc);
+                acc = fmaf(w[e][1], a2[e], acc);
+                acc = fmaf(w[e][0], a3[e], acc);
+                c[e] = silu_fast(acc);
+            }
+            emit(tw + i, c);
+            h3 = h2;
+            h2 = h1;
+            h1 = x0;
+        }
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < kWarpTok; ++i) {
+        const int t = tw + i;
+        if (t >= p.T) break;
+        while (t >= eos && n + 1 < p.n_seqs) {
+            ++n;
+            bos = max(p.cu[n], 0);
+            eos = p.cu[n + 1];
+        }
+        float c[4];
+        const float4 x0v = x[(i + 3) * 32];
+        const float *x0 = reinterpret_cast<const float *>(&x0v);
+        // rows t-1, t-2, t-3: inside the sequence from the tile; before its
+        // start zero (replay) or the stored history (continuation)
+        float xm[3][4];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int tj = t - 1 - j;
+            const float4 xv = x[(i + 2 - j) * 32];
+            const float *xr = reinterpret_cast<const float *>(&xv);
+            if (tj >= bos) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xm[j][e] = xr[e];
+            } else if (p.conv_in[g]) {
+                const __nv_bfloat16 *hp = p.conv_in[g] + (size_t(n) * p.conv_dim + ch) * 3 + (3 - bos + tj);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xm[j][e] = __bfloat162float(hp[e * 3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xm[j][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float acc = w[e][3] * x0[e];
+            acc = fmaf(w[e][2], xm[0][e], acc);
+            acc = fmaf(w[e][1], xm[1][e], acc);
+            acc = fmaf(w[e][0], xm[2][e], acc);
+            c[e] = silu_fast(acc);
+        }
+        emit(t, c);
     }
 }
 
@@ -261,13 +313,13 @@ __global__ void __launch_bounds__(256) gated_norm_kernel(const __grid_constant__
     const float2 oa = __bfloat1622float2(o2[0]), ob = __bfloat1622float2(o2[1]);
     const float ov[4] = {oa.x, oa.y, ob.x, ob.y};
     const float ss = warp_sum(ov[0] * ov[0] + ov[1] * ov[1] + ov[2] * ov[2] + ov[3] * ov[3]);
-    const float r = 1.f / sqrtf(ss / 128.f + p.eps);
+    const float r = rsqrtf(ss / 128.f + p.eps);
     const float4 z = *reinterpret_cast<const float4 *>(p.p[g] + size_t(t) * p.ld + p.z_off + h * 128 + c);
     const float zv[4] = {z.x, z.y, z.z, z.w};
     float y[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-        y[e] = ov[e] * r * __bfloat162float(p.w[g][c + e]) * (zv[e] * sigmoidf_(zv[e]));
+        y[e] = ov[e] * r * __bfloat162float(p.w[g][c + e]) * silu_fast(zv[e]);
     __nv_bfloat162 hi[2], lo[2];
     split2(y[0], y[1], hi[0], lo[0]);
     split2(y[2], y[3], hi[1], lo[1]);
@@ -297,8 +349,11 @@ cudaError_t row_prep(const RowPrepBatch &b, int n_groups, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t conv_gates(const ConvBatch &b, int n_groups, cudaStream_t st) {
-    if (b.T == 0) return cudaSuccess;
+cudaError_t conv_gates(const ConvBatch &b_in, int n_groups, cudaStream_t st) {
+    if (b_in.T == 0) return cudaSuccess;
+    ConvBatch b = b_in;
+    for (int g = 0; g < n_groups; ++g)
+        if (!make_map_f32(&b.pmap[g], b.p[g], b.T, b.ld, b.ld, 128, kConvRows)) return cudaErrorInvalidValue;
     dim3 grid((b.T + kConvTok - 1) / kConvTok, 2 * b.h_k + b.h_v + 1, n_groups);
     conv_gates_kernel<<<grid, 128, 0, st>>>(b);
     cudaError_t e = cudaGetLastError();
