@@ -49,8 +49,12 @@ L2_BYTES = 126 * 1024 * 1024
 # the kernel source it was taken on; once that file changes the figure no
 # longer describes the kernel and the bench reports null.
 MEASURED_TRAFFIC = {
-    # in_proj of the 1-group workload: 81.4 MB read + 36.3 MB written, x 8 groups
-    "model_32k_5": ("gemm_tc.cu", "267fc0b4aafe4f34", 8 * 117.7e6),
+    # in_proj of the 1-group workload: 81.5 MB read + 36.1 MB written, x 8 groups
+    "model_32k_5": ("gemm_tc.cu", "a6f1b53e40f6a63f", 8 * 117.6e6),
+    # the raw workload's launch: 151.8 MB read + 54.0 MB written
+    "raw_qwen": ("gdn_tc.cu", "e32a7269977276f7", 205.8e6),
+    # the Mamba2 workload's launch: 1252.3 MB read + 1216.5 MB written
+    "mamba2": ("mamba2_chunk.cu", "957e765a8ae46ee6", 2468.8e6),
 }
 
 
@@ -696,12 +700,13 @@ def run_ours(args):
         if dom["bound"] == "hbm":
             roofline = {"kernel": dom["name"], "bound": "hbm", "achieved": round(hbm_gbs, 1),
                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(hbm_gbs / peaks["hbm_gbs"], 4),
-                        "traffic": None, "peak_source": f"{src} (HBM copy)",
+                        "traffic": measured_traffic(args.workload), "peak_source": f"{src} (HBM copy)",
                         "bytes_per_launch": dom["bytes"], "tflops": round(tflops, 2)}
         else:
             peak = peaks["bf16_tflops"]
             roofline = {"kernel": dom["name"], "bound": dom["bound"], "achieved": round(tflops, 2),
-                        "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                        "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                        "traffic": measured_traffic(args.workload),
                         "peak_source": f"{src} (burst bf16)", "hbm_gbs": round(hbm_gbs, 1),
                         "hbm_frac": round(hbm_gbs / peaks["hbm_gbs"], 4)}
 
