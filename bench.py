@@ -241,7 +241,7 @@ class GroupReplay:
 
     FULL_LAYER_MFLOP = None  # filled from shapes
 
-    def __init__(self, name, rank, precision="split"):
+    def __init__(self, name, rank, precision="split_fp8"):
         self.name = name
         if name == "group":
             self.gis = [W.group(seed=0x5EED0002 + 1000 * rank)]
@@ -288,16 +288,17 @@ class GroupReplay:
         last = self.flop["gemm_in"] + self.flop["gdn"]
         self.step_flop = (self.L - 1) * full + last  # skip mode
         # algorithmic bytes of one launch (all groups) for the HBM-bound layer kernels
-        split = 2 if precision == "split" else 1
+        split = 1 if precision == "bf16" else 2  # k, v: bf16, or hi + lo bf16
+        act_out = {"split": 4, "split_fp8": 3, "bf16": 2}[precision]  # projection operand bytes per element
         qd, vd = s.qk_dim, s.v_dim
         self.bytes = {
             # p (fp32) of the conv channels and gate columns in; q, k, v (hi/lo) and g, beta out
             "conv": float(T) * self.G * ((s.conv_dim + 2 * s.h_v) * 4 + qd * 2 + (qd + vd) * 2 * split
                                           + 2 * s.h_v * 4),
             # x in (fp32), x * w out (hi/lo), r out
-            "row_prep": float(T) * self.G * (H * 4 + H * 2 * split + 4),
+            "row_prep": float(T) * self.G * (H * 4 + H * act_out + 4),
             # o (bf16) and z (fp32) in, y (hi/lo) out
-            "gated_norm": float(T) * self.G * (vd * 2 + vd * 4 + vd * 2 * split),
+            "gated_norm": float(T) * self.G * (vd * 2 + vd * 4 + vd * act_out),
         }
         self.input_bytes = self.G * T * H * 2 + sum(
             sum(getattr(lw, f).numel() * getattr(lw, f).element_size() for f in ("w_in", "w_out", "w_gate", "w_up",
@@ -327,9 +328,15 @@ class GroupReplay:
             self.weights.append(row)
         self.cu = self.gis[0].cu_seqlens.to(dev)
         self.max_len = max(self.gis[0].lengths)
+        prec = {"split": sr.SR_PREC_SPLIT, "split_fp8": sr.SR_PREC_SPLIT_FP8, "bf16": sr.SR_PREC_BF16}
         self.kw = dict(max_seqlen=self.max_len, hidden=s.hidden, inter=s.inter, h_k=s.h_k, h_v=s.h_v, d=s.d_k,
-                       eps=s.eps, mode=sr.SR_MODE_SKIP,
-                       precision=sr.SR_PREC_SPLIT if self.precision == "split" else sr.SR_PREC_BF16)
+                       eps=s.eps, mode=sr.SR_MODE_SKIP, precision=prec[self.precision])
+        if self.precision == "split_fp8":
+            # the low-pass weight copies are made once, as at model load
+            for row in self.weights:
+                for o in row:
+                    sr.attach_lo8(o)
+            torch.cuda.synchronize(dev)
         if self.sparse:
             _, rows = sr.sparse_anchor_plan(W.SPARSE_PREFIX, page_size=W.SPARSE_PAGE,
                                             anchors_per_page=W.SPARSE_PER_PAGE, k_max=W.SPARSE_K_MAX, ratio=0.05,
@@ -690,7 +697,8 @@ def run_ours(args):
                     "traffic": measured_traffic(args.workload) if dom_kind == "gemm_in" else None,
                     "peak_source": f"{src} (sustained bf16: kernel timed inside a long step)",
                     "flop_per_launch": wl.flop[dom_kind], "ms_per_launch": round(per_launch_ms, 4),
-                    "mma_passes": 2 if wl.precision == "split" else 1,
+                    "mma_passes": {"split": "2 bf16", "split_fp8": "1 bf16 + 1 fp8 (e4m3 x e5m2)",
+                                   "bf16": "1 bf16"}[wl.precision],
                     "step_tflops": round(wl.step_flop / (ms_per_step / 1e3) / 1e12, 2)}
     else:
         dom = wl.dominant()
@@ -776,8 +784,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
-    ap.add_argument("--precision", choices=["split", "bf16"], default="split",
-                    help="group workloads: hi/lo activations (parity-checked) or single-pass bf16")
+    ap.add_argument("--precision", choices=["split", "split_fp8", "bf16"], default="split_fp8",
+                    help="group workloads: split_fp8 (hi/lo activations, low pass on the fp8 tensor cores; "
+                         "parity-checked, the default), split (both passes bf16; parity-checked) or bf16 "
+                         "(single pass)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

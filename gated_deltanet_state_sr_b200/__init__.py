@@ -58,7 +58,11 @@ class Mamba2Args(ctypes.Structure):
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_in_norm", _vp), ("w_in", _vp), ("conv_w", _vp), ("a_log", _vp),
                 ("dt_bias", _vp), ("w_gnorm", _vp), ("w_out", _vp), ("w_post_norm", _vp),
-                ("w_gate", _vp), ("w_up", _vp), ("w_down", _vp)]
+                ("w_gate", _vp), ("w_up", _vp), ("w_down", _vp),
+                ("w_in_lo8", _vp), ("w_out_lo8", _vp), ("w_gate_lo8", _vp), ("w_up_lo8", _vp), ("w_down_lo8", _vp)]
+
+
+LO8_FIELDS = ("w_in_lo8", "w_out_lo8", "w_gate_lo8", "w_up_lo8", "w_down_lo8")
 
 
 class LayerOutputs(ctypes.Structure):
@@ -310,7 +314,7 @@ def test_gemm(a, b0, *, b1=None, r=None, epi=EPI_STORE, c=None, ws=None, stream=
 
 # ------------------------------------------------------------------ group replay
 
-SR_PREC_SPLIT, SR_PREC_BF16 = 0, 1
+SR_PREC_SPLIT, SR_PREC_BF16, SR_PREC_SPLIT_FP8 = 0, 1, 2
 _LAYER_FIELDS = [f for f, _ in LayerWeights._fields_]
 
 
@@ -340,7 +344,8 @@ def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, int
     for g in range(G):
         for l in range(L):
             lw = weights[g][l]
-            w_arr[g * L + l] = LayerWeights(*[getattr(lw, f).data_ptr() for f in _LAYER_FIELDS])
+            w_arr[g * L + l] = LayerWeights(*[None if getattr(lw, f, None) is None else getattr(lw, f).data_ptr()
+                                              for f in _LAYER_FIELDS])
             s, c, h = outputs[g][l]
             o_arr[g * L + l] = LayerOutputs(s.data_ptr(), c.data_ptr(), None if h is None else h.data_ptr())
     n = cu_seqlens.numel() - 1
@@ -502,3 +507,25 @@ def sparse_anchor_plan(n_prefix, *, page_size=64, anchors_per_page=4, layout=SR_
     rows = (_i32 * max(k, 1))()
     _check(_plan(ctypes.byref(a), pos, rows, k, ctypes.byref(count)))
     return list(pos[:k]), list(rows[:k])
+
+
+# ------------------------------------------------------------------ fp8 low-pass weights
+
+_prep_lo8 = _sig("sr_prepare_lo8_weights", _i32, _vp, _vp, ctypes.c_int64, _vp)
+
+
+def prepare_lo8(w, stream=None):
+    """sr_prepare_lo8_weights: the low-pass copy e5m2(w * 2^-8) of a bf16 CUDA
+    weight tensor, as a uint8 tensor of the same shape."""
+    torch = _torch()
+    out = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    _check(_prep_lo8(_ptr(w), _ptr(out), w.numel(), _stream_handle(stream)))
+    return out
+
+
+def attach_lo8(layer, stream=None):
+    """Adds the five *_lo8 low-pass copies to a layer-weights object (its
+    w_in, w_out, w_gate, w_up, w_down CUDA tensors) for SR_PREC_SPLIT_FP8."""
+    for f in LO8_FIELDS:
+        setattr(layer, f, prepare_lo8(getattr(layer, f[:-4]), stream))
+    return layer

@@ -144,6 +144,15 @@ sr_status sr_mamba2_replay(const sr_mamba2_args *a, void *ws, size_t ws_bytes, v
     return SR_OK;
 }
 
+sr_status sr_prepare_lo8_weights(const void *w, void *w_lo8, int64_t n, void *stream) {
+    if (n < 0) return set_error(SR_ERR_INVALID_ARG, "n must be >= 0");
+    if (n > 0 && (!w || !w_lo8)) return set_error(SR_ERR_INVALID_ARG, "w and w_lo8 are required");
+    if (n == 0) return SR_OK;
+    cudaError_t e = prepare_lo8(w, w_lo8, n, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_error(e, "sr_prepare_lo8_weights");
+    return SR_OK;
+}
+
 sr_status sr_device_status(const void *ws, void *stream, uint32_t *flags) {
     if (!ws || !flags) return set_error(SR_ERR_INVALID_ARG, "workspace and flags are required");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -173,7 +182,7 @@ extern "C" sr_status sr_test_gemm(const void *a, const void *b0, const void *b1,
     uint32_t *status = static_cast<uint32_t *>(ws);
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st);
     GemmProblemDesc d{a, nullptr, b0, b1, c, r, nullptr, nullptr};
-    if (e == cudaSuccess) e = gemm_tc(&d, 1, m, n, k, n, epi, 1, status, st);
+    if (e == cudaSuccess) e = gemm_tc(&d, 1, m, n, k, n, epi, 1, 0, status, st);
     if (e != cudaSuccess) return cuda_error(e, "sr_test_gemm");
     return SR_OK;
 }

@@ -25,6 +25,8 @@
 #include "kernels.h"
 #include "tc.cuh"
 
+#include <cuda_fp8.h>
+
 namespace sr {
 
 namespace {
@@ -44,9 +46,11 @@ struct Problem {
     CUtensorMap a_lo;  // [M, K] low part of A (second pass), box {64, 128}
     CUtensorMap b0;  // [N, K] box {64, 256}; gate [N, K] box {64, 128} for SwiGLU
     CUtensorMap b1;  // up [N, K] box {64, 128} (SwiGLU only)
+    CUtensorMap b0_lo;  // fp8 low pass: e5m2 bytes of b0 * 2^-8, box {128 B, as b0}
+    CUtensorMap b1_lo;  // fp8 low pass: e5m2 bytes of b1 * 2^-8 (SwiGLU only)
     void *c;
     const __nv_bfloat16 *r;
-    __nv_bfloat16 *c_lo;     // SwiGLU: low part of the output (may be null)
+    void *c_lo;              // SwiGLU: low part of the output (bf16, or e4m3 of lo * 2^8; may be null)
     const float *rowscale;   // per-row scale (may be null)
 };
 
@@ -58,6 +62,7 @@ struct Params {
     int m_tiles, n_tiles;
     int epi;
     int n_pass;  // 1: A; 2: A_hi then A_lo
+    int lo_fp8;  // the A_lo pass on the fp8 tensor cores (128-byte K blocks of 128 elements)
     uint32_t *status;
 };
 
@@ -68,6 +73,19 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 __device__ __forceinline__ float silu(float x) { return x / (1.f + __expf(-x)); }
+// Eight low parts -> eight e4m3 bytes of lo * 2^8 (round to nearest, saturating).
+__device__ __forceinline__ uint2 lo8_pack8(const float (&lo)[8]) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const __nv_fp8x2_storage_t a = __nv_cvt_float2_to_fp8x2(make_float2(lo[4 * h] * 256.f, lo[4 * h + 1] * 256.f),
+                                                               __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(
+            make_float2(lo[4 * h + 2] * 256.f, lo[4 * h + 3] * 256.f), __NV_SATFINITE, __NV_E4M3);
+        w[h] = uint32_t(a) | (uint32_t(b) << 16);
+    }
+    return make_uint2(w[0], w[1]);
+}
 
 // Abort-aware bounded wait: gives up when another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort_flag) {
@@ -116,6 +134,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         for (int i = 0; i < p.n_problems; ++i) {
             tc::prefetch_tmap(&p.prob[i].a);
             if (p.n_pass == 2) tc::prefetch_tmap(&p.prob[i].a_lo);
+            if (p.lo_fp8) {
+                tc::prefetch_tmap(&p.prob[i].b0_lo);
+                if (p.epi == EPI_SWIGLU) tc::prefetch_tmap(&p.prob[i].b1_lo);
+            }
             tc::prefetch_tmap(&p.prob[i].b0);
             if (p.epi == EPI_SWIGLU) tc::prefetch_tmap(&p.prob[i].b1);
         }
@@ -128,6 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int tiles_per_prob = p.m_tiles * p.n_tiles;
     const int total = p.n_problems * tiles_per_prob;
     const int kblocks = p.K / BK;
+    // k blocks of the low pass: 64 bf16 or 128 fp8 elements, 128 bytes per row either way
+    const int kblocks_lo = p.n_pass == 2 ? (p.lo_fp8 ? p.K / (2 * BK) : kblocks) : 0;
+    const int kblocks_all = kblocks + kblocks_lo;
     auto fail = [&]() {
         *abort_flag = 1;
         atomicOr(p.status, SR_DEV_TIMEOUT);
@@ -141,18 +166,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 const int pi = tile / tiles_per_prob, rem = tile % tiles_per_prob;
                 const int nt = rem / p.m_tiles, mt = rem % p.m_tiles;
                 const Problem &pr = p.prob[pi];
-                for (int kk = 0; kk < p.n_pass * kblocks; ++kk) {
-                    const int kb = kk % kblocks;
+                for (int kk = 0; kk < kblocks_all; ++kk) {
+                    const bool lo = kk >= kblocks;
+                    const bool f8 = lo && p.lo_fp8;
+                    const int kb = lo ? kk - kblocks : kk;
+                    const int kx = f8 ? kb * 2 * BK : kb * BK;  // element column of the 128-byte block
+                    const CUtensorMap *mb0 = f8 ? &pr.b0_lo : &pr.b0, *mb1 = f8 ? &pr.b1_lo : &pr.b1;
                     if (!wait_or_abort(&empty[stage], phase ^ 1, abort_flag)) { fail(); break; }
                     tc::mbar_arrive_expect_tx(&full[stage], kTileA + kTileB);
-                    tc::tma_load_2d(sA + stage * kTileA, kk < kblocks ? &pr.a : &pr.a_lo, &full[stage], kb * BK,
-                                    mt * BM);
+                    tc::tma_load_2d(sA + stage * kTileA, lo ? &pr.a_lo : &pr.a, &full[stage], kx, mt * BM);
                     if (p.epi == EPI_SWIGLU) {
-                        tc::tma_load_2d(sB + stage * kTileB, &pr.b0, &full[stage], kb * BK, nt * (BN / 2));
-                        tc::tma_load_2d(sB + stage * kTileB + (BN / 2) * BK * 2, &pr.b1, &full[stage], kb * BK,
+                        tc::tma_load_2d(sB + stage * kTileB, mb0, &full[stage], kx, nt * (BN / 2));
+                        tc::tma_load_2d(sB + stage * kTileB + (BN / 2) * BK * 2, mb1, &full[stage], kx,
                                         nt * (BN / 2));
                     } else {
-                        tc::tma_load_2d(sB + stage * kTileB, &pr.b0, &full[stage], kb * BK, nt * BN);
+                        tc::tma_load_2d(sB + stage * kTileB, mb0, &full[stage], kx, nt * BN);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -161,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc_f8 = tc::idesc_e4m3_e5m2_f32(BM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
@@ -168,15 +197,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 tc::tc_fence_after();
                 const uint32_t d = tmem + uint32_t(acc * BN);
                 bool ok = true;
-                for (int kb = 0; kb < p.n_pass * kblocks; ++kb) {
+                for (int kb = 0; kb < kblocks_all; ++kb) {
                     if (!wait_or_abort(&full[stage], phase, abort_flag)) { fail(); ok = false; break; }
                     tc::tc_fence_after();
                     const uint32_t a0 = tc::smem_u32(sA + stage * kTileA);
                     const uint32_t b0 = tc::smem_u32(sB + stage * kTileB);
+                    // four MMAs per 128-byte block: K = 16 bf16 or K = 32 fp8 elements, 32 bytes apart
+                    if (p.lo_fp8 && kb >= kblocks) {
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        tc::mma_bf16_ss(d, tc::sdesc_k_sw128(a0 + k * 32), tc::sdesc_k_sw128(b0 + k * 32), idesc,
-                                        (kb | k) != 0);
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_f8_ss(d, tc::sdesc_k_sw128(a0 + k * 32), tc::sdesc_k_sw128(b0 + k * 32), idesc_f8,
+                                          1);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            tc::mma_bf16_ss(d, tc::sdesc_k_sw128(a0 + k * 32), tc::sdesc_k_sw128(b0 + k * 32), idesc,
+                                            (kb | k) != 0);
+                    }
                     tc::mma_commit(&empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -214,21 +251,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     if (row_ok && nvec > 0) {
                         __nv_bfloat16 *cb = static_cast<__nv_bfloat16 *>(pr.c);
                         uint4 *dst = reinterpret_cast<uint4 *>(cb + size_t(row) * p.ldc + col);
-                        uint4 *dlo = pr.c_lo ? reinterpret_cast<uint4 *>(pr.c_lo + size_t(row) * p.ldc + col) : nullptr;
+                        uint4 *dlo = pr.c_lo && !p.lo_fp8
+                                         ? reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c_lo) +
+                                                                     size_t(row) * p.ldc + col)
+                                         : nullptr;
+                        uint2 *dlo8 = pr.c_lo && p.lo_fp8
+                                          ? reinterpret_cast<uint2 *>(static_cast<uint8_t *>(pr.c_lo) +
+                                                                      size_t(row) * p.ldc + col)
+                                          : nullptr;
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             if (v >= nvec) break;
                             uint32_t w[4], wl[4];
+                            float lo[8];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int j = v * 8 + e * 2;
                                 const float h0 = silu(rs * __uint_as_float(g[j])) * (rs * __uint_as_float(u[j]));
                                 const float h1 = silu(rs * __uint_as_float(g[j + 1])) * (rs * __uint_as_float(u[j + 1]));
                                 w[e] = pack2(h0, h1);
-                                wl[e] = pack2(h0 - bf_lo(w[e]), h1 - bf_hi(w[e]));
+                                lo[2 * e] = h0 - bf_lo(w[e]);
+                                lo[2 * e + 1] = h1 - bf_hi(w[e]);
+                                wl[e] = pack2(lo[2 * e], lo[2 * e + 1]);
                             }
                             dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
                             if (dlo) dlo[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                            if (dlo8) dlo8[v] = lo8_pack8(lo);
                         }
                     }
                 }
@@ -341,6 +389,18 @@ bool make_map_bf16(CUtensorMap *m, const void *base, int rows, int cols, int pit
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_u8(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(pitch)};
+    cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+    cuuint32_t es[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_f32(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -363,23 +423,29 @@ namespace {
 
 template <int BN>
 cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
-                        int n_pass, uint32_t *status, cudaStream_t st) {
+                        int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st) {
     Params local{};
     const int bn_out = epi == EPI_SWIGLU ? BN / 2 : BN;
+    const int bn_rows = epi == EPI_SWIGLU ? BN / 2 : BN;  // rows of each weight box
     for (int i = 0; i < n_problems; ++i) {
         const GemmProblemDesc &d = probs[i];
         if (!make_map(&local.prob[i].a, d.a, M, K, K, BM)) return cudaErrorInvalidValue;
-        if (n_pass == 2 && !make_map(&local.prob[i].a_lo, d.a_lo, M, K, K, BM)) return cudaErrorInvalidValue;
-        if (epi == EPI_SWIGLU) {
-            if (!make_map(&local.prob[i].b0, d.b0, N, K, K, BN / 2) ||
-                !make_map(&local.prob[i].b1, d.b1, N, K, K, BN / 2))
+        if (n_pass == 2) {
+            const bool ok = lo_fp8 ? make_map_u8(&local.prob[i].a_lo, d.a_lo, M, K, K, 2 * BK, BM)
+                                   : make_map(&local.prob[i].a_lo, d.a_lo, M, K, K, BM);
+            if (!ok) return cudaErrorInvalidValue;
+        }
+        if (!make_map(&local.prob[i].b0, d.b0, N, K, K, bn_rows)) return cudaErrorInvalidValue;
+        if (epi == EPI_SWIGLU && !make_map(&local.prob[i].b1, d.b1, N, K, K, bn_rows)) return cudaErrorInvalidValue;
+        if (n_pass == 2 && lo_fp8) {
+            if (!d.b0_lo || !make_map_u8(&local.prob[i].b0_lo, d.b0_lo, N, K, K, 2 * BK, bn_rows))
                 return cudaErrorInvalidValue;
-        } else if (!make_map(&local.prob[i].b0, d.b0, N, K, K, BN)) {
-            return cudaErrorInvalidValue;
+            if (epi == EPI_SWIGLU && (!d.b1_lo || !make_map_u8(&local.prob[i].b1_lo, d.b1_lo, N, K, K, 2 * BK, bn_rows)))
+                return cudaErrorInvalidValue;
         }
         local.prob[i].c = d.c;
         local.prob[i].r = static_cast<const __nv_bfloat16 *>(d.r);
-        local.prob[i].c_lo = static_cast<__nv_bfloat16 *>(d.c_lo);
+        local.prob[i].c_lo = d.c_lo;
         local.prob[i].rowscale = d.rowscale;
     }
     local.n_problems = n_problems;
@@ -391,6 +457,7 @@ cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int
     local.n_tiles = (N + bn_out - 1) / bn_out;
     local.epi = epi;
     local.n_pass = n_pass;
+    local.lo_fp8 = n_pass == 2 && lo_fp8;
     local.status = status;
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<BN>::kSmemBytes);
@@ -405,14 +472,15 @@ cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int
 }  // namespace
 
 cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
-                    int n_pass, uint32_t *status, cudaStream_t st) {
+                    int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st) {
     if (n_problems <= 0 || n_problems > kMaxGemmProblems || M <= 0 || N <= 0 || K <= 0 || K % BK != 0 ||
-        N % 8 != 0 || ldc % 8 != 0 || ldc < N || (n_pass != 1 && n_pass != 2))
+        N % 8 != 0 || ldc % 8 != 0 || ldc < N || (n_pass != 1 && n_pass != 2) ||
+        (n_pass == 2 && lo_fp8 && K % (2 * BK) != 0))
         return cudaErrorInvalidValue;
     // 256-wide tiles: measured against 128-wide ones on the group shapes, they stay
     // ahead even where the 128-wide tiling fills the last wave of SMs better
     // (the A tile is then streamed twice as often).
-    return launch_gemm<256>(probs, n_problems, M, N, K, ldc, epi, n_pass, status, st);
+    return launch_gemm<256>(probs, n_problems, M, N, K, ldc, epi, n_pass, lo_fp8, status, st);
 }
 
 }  // namespace sr

@@ -27,7 +27,8 @@ namespace {
 
 struct Dims {
     int G, L, N, T, H, I, hk, hv, d, qd, vd, conv_dim, proj;
-    bool split;
+    bool split;  // activations carried as hi + lo
+    bool lo8;    // the lo parts of the projection operands as e4m3 bytes (fp8 low pass)
 };
 
 Dims dims_of(const sr_group_args &a) {
@@ -45,13 +46,15 @@ Dims dims_of(const sr_group_args &a) {
     m.vd = a.h_v * a.d_v;
     m.conv_dim = 2 * m.qd + m.vd;
     m.proj = m.conv_dim + m.vd + 2 * m.hv;
-    m.split = a.precision == SR_PREC_SPLIT;
+    m.split = a.precision == SR_PREC_SPLIT || a.precision == SR_PREC_SPLIT_FP8;
+    m.lo8 = a.precision == SR_PREC_SPLIT_FP8;
     return m;
 }
 
 struct GroupBufs {
     float *x32, *r, *p, *gate, *beta;
-    __nv_bfloat16 *a_hi, *a_lo, *q, *k, *k_lo, *v, *v_lo, *o, *h_hi, *h_lo;
+    __nv_bfloat16 *a_hi, *q, *k, *k_lo, *v, *v_lo, *o, *h_hi;
+    void *a_lo, *h_lo;  // bf16, or e4m3 bytes with the fp8 low pass
 };
 
 // Carves the per-group scratch buffers out of the workspace (after its header).
@@ -73,7 +76,8 @@ size_t carve(const Dims &m, char *base, GroupBufs *out) {
         b.gate = reinterpret_cast<float *>(take(T * m.hv * 4));
         b.beta = reinterpret_cast<float *>(take(T * m.hv * 4));
         b.a_hi = reinterpret_cast<__nv_bfloat16 *>(take(T * amax * 2));
-        b.a_lo = m.split ? reinterpret_cast<__nv_bfloat16 *>(take(T * amax * 2)) : nullptr;
+        const size_t lo_elem = m.lo8 ? 1 : 2;
+        b.a_lo = m.split ? take(T * amax * lo_elem) : nullptr;
         b.q = reinterpret_cast<__nv_bfloat16 *>(take(T * m.qd * 2));
         b.k = reinterpret_cast<__nv_bfloat16 *>(take(T * m.qd * 2));
         b.k_lo = m.split ? reinterpret_cast<__nv_bfloat16 *>(take(T * m.qd * 2)) : nullptr;
@@ -81,7 +85,7 @@ size_t carve(const Dims &m, char *base, GroupBufs *out) {
         b.v_lo = m.split ? reinterpret_cast<__nv_bfloat16 *>(take(T * m.vd * 2)) : nullptr;
         b.o = reinterpret_cast<__nv_bfloat16 *>(take(T * m.vd * 2));
         b.h_hi = reinterpret_cast<__nv_bfloat16 *>(take(T * m.I * 2));
-        b.h_lo = m.split ? reinterpret_cast<__nv_bfloat16 *>(take(T * m.I * 2)) : nullptr;
+        b.h_lo = m.split ? take(T * m.I * lo_elem) : nullptr;
         if (out) out[g] = b;
     }
     return off;
@@ -104,8 +108,10 @@ sr_status validate(const sr_group_args *a) {
     if (a->hidden <= 0 || a->hidden % 64 || a->inter <= 0 || a->inter % 64)
         return set_error(SR_ERR_UNSUPPORTED, "hidden and inter must be positive multiples of 64");
     if (a->mode != SR_MODE_SKIP && a->mode != SR_MODE_FULL) return set_error(SR_ERR_INVALID_ARG, "bad mode");
-    if (a->precision != SR_PREC_SPLIT && a->precision != SR_PREC_BF16)
+    if (a->precision != SR_PREC_SPLIT && a->precision != SR_PREC_BF16 && a->precision != SR_PREC_SPLIT_FP8)
         return set_error(SR_ERR_INVALID_ARG, "bad precision");
+    if (a->precision == SR_PREC_SPLIT_FP8 && (a->hidden % 128 || a->inter % 128 || (a->h_v * a->d_v) % 128))
+        return set_error(SR_ERR_UNSUPPORTED, "SR_PREC_SPLIT_FP8 needs hidden, inter and h_v d_v multiples of 128");
     if (!(a->eps > 0.f)) return set_error(SR_ERR_INVALID_ARG, "eps must be > 0");
     if (a->anchor_index && a->anchor_rows < 1)
         return set_error(SR_ERR_INVALID_ARG, "anchor_index needs anchor_rows >= 1 (got %d)", a->anchor_rows);
@@ -117,6 +123,10 @@ sr_status validate(const sr_group_args *a) {
             if (!w.w_in_norm || !w.w_in || !w.conv_w || !w.a_log || !w.dt_bias || !w.w_gnorm || !w.w_out ||
                 !w.w_post_norm || !w.w_gate || !w.w_up || !w.w_down)
                 return set_error(SR_ERR_INVALID_ARG, "weights of group %d layer %d incomplete", g, l);
+            if (a->precision == SR_PREC_SPLIT_FP8 &&
+                (!w.w_in_lo8 || !w.w_out_lo8 || !w.w_gate_lo8 || !w.w_up_lo8 || !w.w_down_lo8))
+                return set_error(SR_ERR_INVALID_ARG,
+                                 "SR_PREC_SPLIT_FP8: low-pass weights of group %d layer %d missing", g, l);
             if (!o.s_out || !o.conv_out)
                 return set_error(SR_ERR_INVALID_ARG, "outputs of group %d layer %d need s_out and conv_out", g, l);
             if (o.hidden_out && a->mode == SR_MODE_SKIP && l == a->n_layers - 1)
@@ -218,7 +228,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             rp.r[g] = B[g].r;
             rp.x32_out[g] = l == 0 ? B[g].x32 : nullptr;
         }
-        rp.T = T; rp.H = m.H; rp.x_f32 = l == 0 ? 0 : 1; rp.eps = a->eps;
+        rp.T = T; rp.H = m.H; rp.x_f32 = l == 0 ? 0 : 1; rp.eps = a->eps; rp.lo8 = m.lo8;
         rp.idx = l == 0 ? a->anchor_index : nullptr;  // sparse anchors: gather from the pool
         rp.x_rows = a->anchor_index ? a->anchor_rows : T;
         rp.status = status;
@@ -229,9 +239,10 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         // (2) p = r * (A W_in^T), fp32
         GemmProblemDesc gp[kMaxGemmProblems];
         for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_in, nullptr, B[g].p, nullptr, nullptr, B[g].r};
+            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_in, nullptr, B[g].p, nullptr, nullptr, B[g].r,
+                                    W(g).w_in_lo8, nullptr};
         SR_TRY(prof.begin(SR_K_GEMM_IN));
-        SR_TRY(gemm_tc(gp, G, T, m.proj, m.H, m.proj, EPI_F32_ROWSCALE, npass, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.proj, m.H, m.proj, EPI_F32_ROWSCALE, npass, m.lo8, status, st));
         SR_TRY(prof.end());
 
         // (3) conv + SiLU + L2 norm + gates, conv state
@@ -288,16 +299,17 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             gn.y_hi[g] = B[g].a_hi;
             gn.y_lo[g] = B[g].a_lo;
         }
-        gn.T = T; gn.h_v = m.hv; gn.ld = m.proj; gn.z_off = m.conv_dim; gn.eps = a->eps;
+        gn.T = T; gn.h_v = m.hv; gn.ld = m.proj; gn.z_off = m.conv_dim; gn.eps = a->eps; gn.lo8 = m.lo8;
         SR_TRY(prof.begin(SR_K_GATED_NORM));
         SR_TRY(gated_norm(gn, G, st));
         SR_TRY(prof.end());
 
         // (6) x += y W_out^T
         for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_out, nullptr, B[g].x32, nullptr, nullptr, nullptr};
+            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_out, nullptr, B[g].x32, nullptr, nullptr, nullptr,
+                                    W(g).w_out_lo8, nullptr};
         SR_TRY(prof.begin(SR_K_GEMM_OUT));
-        SR_TRY(gemm_tc(gp, G, T, m.H, m.vd, m.H, EPI_F32_RESIDUAL, npass, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.H, m.vd, m.H, EPI_F32_RESIDUAL, npass, m.lo8, status, st));
         SR_TRY(prof.end());
 
         // (7) A = x * w_post_norm, r
@@ -315,16 +327,18 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
 
         // (8) h = SiLU(r A W_gate^T) * (r A W_up^T) (hi/lo)
         for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_gate, W(g).w_up, B[g].h_hi, nullptr, B[g].h_lo, B[g].r};
+            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_gate, W(g).w_up, B[g].h_hi, nullptr, B[g].h_lo, B[g].r,
+                                    W(g).w_gate_lo8, W(g).w_up_lo8};
         SR_TRY(prof.begin(SR_K_GEMM_GATEUP));
-        SR_TRY(gemm_tc(gp, G, T, m.I, m.H, m.I, EPI_SWIGLU, npass, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.I, m.H, m.I, EPI_SWIGLU, npass, m.lo8, status, st));
         SR_TRY(prof.end());
 
         // (9) x += h W_down^T
         for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].h_hi, B[g].h_lo, W(g).w_down, nullptr, B[g].x32, nullptr, nullptr, nullptr};
+            gp[g] = GemmProblemDesc{B[g].h_hi, B[g].h_lo, W(g).w_down, nullptr, B[g].x32, nullptr, nullptr, nullptr,
+                                    W(g).w_down_lo8, nullptr};
         SR_TRY(prof.begin(SR_K_GEMM_DOWN));
-        SR_TRY(gemm_tc(gp, G, T, m.H, m.I, m.H, EPI_F32_RESIDUAL, npass, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.H, m.I, m.H, EPI_F32_RESIDUAL, npass, m.lo8, status, st));
         SR_TRY(prof.end());
 
         // (10) optional bf16 copy of the hidden after this layer

@@ -43,6 +43,8 @@ cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split
 
 // 2-D bf16 TMA map (128-byte swizzle) over a row-major [rows, cols] matrix with row pitch `pitch`.
 bool make_map_bf16(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows);
+// bytes [rows, cols] (row pitch `pitch` bytes), 128-byte swizzled boxes of box_rows x box_cols.
+bool make_map_u8(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows);
 // fp32 [rows, cols] (row pitch `pitch` elements), unswizzled boxes of box_rows x box_cols.
 bool make_map_f32(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows);
 
@@ -51,12 +53,13 @@ struct RowPrepBatch {
     const void *x[kMaxGroups];            // [T, H] fp32 (x_f32) or bf16
     const __nv_bfloat16 *w[kMaxGroups];   // [H] norm weight
     __nv_bfloat16 *a_hi[kMaxGroups];      // [T, H] x * w (hi part)
-    __nv_bfloat16 *a_lo[kMaxGroups];      // [T, H] low part, may be null
+    void *a_lo[kMaxGroups];               // [T, H] low part (bf16, or e4m3(lo * 2^8) when lo8), may be null
     float *r[kMaxGroups];                 // [T] 1 / sqrt(mean(x^2) + eps)
     float *x32_out[kMaxGroups];           // [T, H] fp32 copy of x, may be null
     const int32_t *idx;                   // [T] row of x that token t reads, may be null (row t)
     uint32_t *status;                     // device status word (bad index flag)
     int T, H, x_f32, x_rows;              // x_rows: rows of x (bounds of idx)
+    int lo8;                              // low part as e4m3 bytes of lo * 2^8
     float eps;
 };
 cudaError_t row_prep(const RowPrepBatch &b, int n_groups, cudaStream_t st);
@@ -87,8 +90,8 @@ struct GatedNormBatch {
     const float *p[kMaxGroups];           // [T, ld] (z at column z_off)
     const __nv_bfloat16 *w[kMaxGroups];   // [128]
     __nv_bfloat16 *y_hi[kMaxGroups];      // [T, h_v * 128]
-    __nv_bfloat16 *y_lo[kMaxGroups];      // may be null
-    int T, h_v, ld, z_off;
+    void *y_lo[kMaxGroups];               // may be null; bf16, or e4m3(lo * 2^8) when lo8
+    int T, h_v, ld, z_off, lo8;
     float eps;
 };
 cudaError_t gated_norm(const GatedNormBatch &b, int n_groups, cudaStream_t st);
@@ -111,15 +114,21 @@ enum GemmEpilogue { EPI_STORE = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_F32_ROW
 constexpr int kMaxGemmProblems = 8;
 struct GemmProblemDesc {
     const void *a;   // [M, K] bf16, row pitch K
-    const void *a_lo;  // [M, K] bf16 low part of A (two-pass GEMMs), else unused
+    const void *a_lo;  // [M, K] low part of A (two-pass GEMMs): bf16, or e4m3(lo * 2^8) bytes (lo_fp8)
     const void *b0;  // [N, K] bf16 (SwiGLU: gate)
     const void *b1;  // [N, K] bf16 (SwiGLU: up), else unused
     void *c;         // [M, ldc] bf16
     const void *r;   // residual [M, ldc] bf16 (EPI_RESIDUAL), may equal c
-    void *c_lo;      // SwiGLU low-part output [M, ldc] bf16, may be null
+    void *c_lo;      // SwiGLU low-part output [M, ldc] (bf16, or e4m3(lo * 2^8) bytes when lo_fp8), may be null
     const float *rowscale;  // [M] fp32 per-row scale, may be null (= 1)
+    const void *b0_lo = nullptr;  // lo_fp8: e5m2(b0 * 2^-8) bytes [N, K]
+    const void *b1_lo = nullptr;  // lo_fp8: e5m2(b1 * 2^-8) bytes [N, K] (SwiGLU)
 };
+// n_pass 1: A only; 2: A_hi then A_lo.  lo_fp8: the A_lo pass runs on the fp8
+// tensor cores (e4m3 A_lo * 2^8 times e5m2 B * 2^-8); needs K % 128 == 0.
 cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
-                    int n_pass, uint32_t *status, cudaStream_t st);
+                    int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st);
+// fp8 low-pass helpers (layer_kernels.cu): e5m2(w * 2^-8) for n bf16 weights.
+cudaError_t prepare_lo8(const void *w, void *w_lo8, int64_t n, cudaStream_t st);
 
 }  // namespace sr

@@ -15,6 +15,8 @@
 //   to_bf16      fp32 residual stream -> bf16 hidden output.
 // The layer math is the Qwen3.5-family Gated DeltaNet block ("Tail-Replay",
 // Sec. 2 names Gated DeltaNet as the linear layer of the hybrids replayed).
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -33,6 +35,12 @@ __device__ __forceinline__ void split2(float a, float b, __nv_bfloat162 &hi, __n
     hi = __floats2bfloat162_rn(a, b);
     const float2 h = __bfloat1622float2(hi);
     lo = __floats2bfloat162_rn(a - h.x, b - h.y);
+}
+// hi = bf16 pair; lo8 = e4m3 bytes of (x - hi) * 2^8 (round to nearest, saturating)
+__device__ __forceinline__ void split2_lo8(float a, float b, __nv_bfloat162 &hi, uint16_t &lo8) {
+    hi = __floats2bfloat162_rn(a, b);
+    const float2 h = __bfloat1622float2(hi);
+    lo8 = __nv_cvt_float2_to_fp8x2(make_float2((a - h.x) * 256.f, (b - h.y) * 256.f), __NV_SATFINITE, __NV_E4M3);
 }
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
@@ -87,15 +95,26 @@ __global__ void __launch_bounds__(256) row_prep_kernel(const __grid_constant__ R
         const uint4 wu = *reinterpret_cast<const uint4 *>(p.w[g] + c);
         const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&wu);
         __nv_bfloat162 hi[4], lo[4];
+        uint16_t lo8[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             ss = fmaf(xv[2 * e], xv[2 * e], ss);
             ss = fmaf(xv[2 * e + 1], xv[2 * e + 1], ss);
             const float2 wf = __bfloat1622float2(w2[e]);
-            split2(xv[2 * e] * wf.x, xv[2 * e + 1] * wf.y, hi[e], lo[e]);
+            if (p.lo8)
+                split2_lo8(xv[2 * e] * wf.x, xv[2 * e + 1] * wf.y, hi[e], lo8[e]);
+            else
+                split2(xv[2 * e] * wf.x, xv[2 * e + 1] * wf.y, hi[e], lo[e]);
         }
         *reinterpret_cast<uint4 *>(p.a_hi[g] + base + c) = *reinterpret_cast<uint4 *>(hi);
-        if (p.a_lo[g]) *reinterpret_cast<uint4 *>(p.a_lo[g] + base + c) = *reinterpret_cast<uint4 *>(lo);
+        if (p.a_lo[g]) {
+            if (p.lo8)
+                *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.a_lo[g]) + base + c) =
+                    make_uint2(uint32_t(lo8[0]) | (uint32_t(lo8[1]) << 16), uint32_t(lo8[2]) | (uint32_t(lo8[3]) << 16));
+            else
+                *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.a_lo[g]) + base + c) =
+                    *reinterpret_cast<uint4 *>(lo);
+        }
         if (p.x32_out[g]) {
             float4 *d = reinterpret_cast<float4 *>(p.x32_out[g] + base + c);
             d[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
@@ -321,10 +340,46 @@ __global__ void __launch_bounds__(256) gated_norm_kernel(const __grid_constant__
     for (int e = 0; e < 4; ++e)
         y[e] = ov[e] * r * __bfloat162float(p.w[g][c + e]) * silu_fast(zv[e]);
     __nv_bfloat162 hi[2], lo[2];
-    split2(y[0], y[1], hi[0], lo[0]);
-    split2(y[2], y[3], hi[1], lo[1]);
+    if (p.lo8) {
+        uint16_t l8[2];
+        split2_lo8(y[0], y[1], hi[0], l8[0]);
+        split2_lo8(y[2], y[3], hi[1], l8[1]);
+        if (p.y_lo[g])
+            *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(p.y_lo[g]) + size_t(item) * 128 + c) =
+                uint32_t(l8[0]) | (uint32_t(l8[1]) << 16);
+    } else {
+        split2(y[0], y[1], hi[0], lo[0]);
+        split2(y[2], y[3], hi[1], lo[1]);
+        if (p.y_lo[g])
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.y_lo[g]) + size_t(item) * 128 + c) =
+                *reinterpret_cast<uint2 *>(lo);
+    }
     *reinterpret_cast<uint2 *>(p.y_hi[g] + size_t(item) * 128 + c) = *reinterpret_cast<uint2 *>(hi);
-    if (p.y_lo[g]) *reinterpret_cast<uint2 *>(p.y_lo[g] + size_t(item) * 128 + c) = *reinterpret_cast<uint2 *>(lo);
+}
+
+// ---------------------------------------------------------------- prepare_lo8
+// w_lo8[i] = e5m2(w[i] * 2^-8); 8 weights per thread (n % 8 handled by the tail loop).
+__global__ void __launch_bounds__(256) prepare_lo8_kernel(const __nv_bfloat16 *__restrict__ w, uint8_t *__restrict__ q,
+                                                          int64_t n) {
+    const int64_t i = (int64_t(blockIdx.x) * 256 + threadIdx.x) * 8;
+    if (i + 8 <= n) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(w + i);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        uint32_t out[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float2 a = __bfloat1622float2(h2[2 * h]), b = __bfloat1622float2(h2[2 * h + 1]);
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a.x * 0.00390625f, a.y * 0.00390625f),
+                                                         __NV_SATFINITE, __NV_E5M2);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(b.x * 0.00390625f, b.y * 0.00390625f),
+                                                         __NV_SATFINITE, __NV_E5M2);
+            out[h] = lo | (hi << 16);
+        }
+        *reinterpret_cast<uint2 *>(q + i) = make_uint2(out[0], out[1]);
+    } else {
+        for (int64_t j = i; j < n; ++j)
+            q[j] = __nv_cvt_float_to_fp8(__bfloat162float(w[j]) * 0.00390625f, __NV_SATFINITE, __NV_E5M2);
+    }
 }
 
 // ---------------------------------------------------------------- to_bf16
@@ -374,6 +429,15 @@ cudaError_t to_bf16(const CastBatch &b, int n_groups, cudaStream_t st) {
     if (b.n == 0) return cudaSuccess;
     dim3 grid(unsigned((b.n / 4 + 255) / 256), n_groups);
     to_bf16_kernel<<<grid, 256, 0, st>>>(b);
+    return cudaGetLastError();
+}
+
+cudaError_t prepare_lo8(const void *w, void *w_lo8, int64_t n, cudaStream_t st) {
+    if (reinterpret_cast<uintptr_t>(w) % 16 || reinterpret_cast<uintptr_t>(w_lo8) % 8) return cudaErrorInvalidValue;
+    const int64_t blocks = (n + 2047) / 2048;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+    prepare_lo8_kernel<<<unsigned(blocks), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(w),
+                                                          static_cast<uint8_t *>(w_lo8), n);
     return cudaGetLastError();
 }
 

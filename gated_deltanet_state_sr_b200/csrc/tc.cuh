@@ -117,6 +117,19 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (8-bit floats in, fp32 accumulate;
+// K = 32 per instruction, i.e. the same 32-byte step along a 128-byte row as bf16).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n"
+        "}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
@@ -195,6 +208,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                      // D format: f32
            | (1u << 7)                    // A format: bf16
            | (1u << 10)                   // B format: bf16
+           | (uint32_t(N >> 3) << 17)     // N / 8
+           | (uint32_t(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor: kind::f8f6f4, A e4m3 x B e5m2 -> fp32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_e5m2_f32(int M, int N) {
+    return (1u << 4)                      // D format: f32
+           | (0u << 7)                    // A format: e4m3
+           | (1u << 10)                   // B format: e5m2
            | (uint32_t(N >> 3) << 17)     // N / 8
            | (uint32_t(M >> 4) << 24);    // M / 16
 }

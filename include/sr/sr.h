@@ -209,6 +209,14 @@ typedef struct sr_layer_weights {
     const void *w_gate;      /* [inter, hidden] bf16 */
     const void *w_up;        /* [inter, hidden] bf16 */
     const void *w_down;      /* [hidden, inter] bf16 */
+    /* SR_PREC_SPLIT_FP8 only (NULL otherwise): the low-pass copies of the five
+     * projections, same shapes, one byte per weight: e5m2(W * 2^-8), written by
+     * sr_prepare_lo8_weights once per model. */
+    const void *w_in_lo8;
+    const void *w_out_lo8;
+    const void *w_gate_lo8;
+    const void *w_up_lo8;
+    const void *w_down_lo8;
 } sr_layer_weights;
 
 typedef struct sr_layer_outputs {
@@ -243,8 +251,16 @@ typedef enum sr_group_mode { SR_MODE_SKIP = 0, SR_MODE_FULL = 1 } sr_group_mode;
  *   the fp64 layer math to ~1e-4 of max|S| over a 3-layer group.
  * SR_PREC_BF16: one pass per projection with bf16 activations (the usual bf16
  *   serving arithmetic); about half the tensor-core work, state error a few
- *   1e-3 of max|S| after three layers. */
-typedef enum sr_group_precision { SR_PREC_SPLIT = 0, SR_PREC_BF16 = 1 } sr_group_precision;
+ *   1e-3 of max|S| after three layers.
+ * SR_PREC_SPLIT_FP8: as SR_PREC_SPLIT, but the low pass of every projection
+ *   runs on the fp8 tensor cores: the activation's low part as
+ *   e4m3(lo * 2^8) times the prepared weight copy e5m2(W * 2^-8), accumulated
+ *   with the bf16 high pass (the powers of two cancel).  The low part's own
+ *   rounding (3 mantissa bits) and the weight copy's (2 bits) act on a term
+ *   2^-9 of the product, so the states stay within about 5e-4 of max|S| over a
+ *   3-layer group, at three quarters of SR_PREC_SPLIT's tensor time.  Needs the
+ *   *_lo8 weight pointers, and hidden, inter and h_v d_v multiples of 128. */
+typedef enum sr_group_precision { SR_PREC_SPLIT = 0, SR_PREC_BF16 = 1, SR_PREC_SPLIT_FP8 = 2 } sr_group_precision;
 
 /* Optional per-launch timing.  When sr_group_args.profile is non-NULL the
  * call records events[2i] before and events[2i+1] after its i-th kernel
@@ -329,6 +345,18 @@ SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, siz
 
 SR_API sr_status sr_group_replay_noalloc(const sr_group_args *args, void *stream,
                                          const void **status_scratch);
+
+/* ------------------------------------------------------------------------
+ * sr_prepare_lo8_weights -- the low-pass weight copy of SR_PREC_SPLIT_FP8.
+ *
+ * The paper has no counterpart: this belongs to this library's split
+ * arithmetic.  Writes w_lo8[i] = e5m2(w[i] * 2^-8) (round to nearest,
+ * saturating) for n bf16 weights, on `stream`.  Run it once per weight matrix
+ * when a model is loaded; every replay then reads the copy.  w and w_lo8 are
+ * device pointers; returns SR_ERR_INVALID_ARG for n < 0 or a NULL pointer
+ * with n > 0.
+ * ---------------------------------------------------------------------- */
+SR_API sr_status sr_prepare_lo8_weights(const void *w, void *w_lo8, int64_t n, void *stream);
 
 /* ------------------------------------------------------------------------
  * sr_anchor_capture -- write selected hidden rows into an anchor pool.

@@ -168,3 +168,22 @@ def test_group_workspace_independent_of_continuation():
     """Initial states are read in place: a continuation needs no extra scratch."""
     init = (sr.LayerState * 1)(sr.LayerState(0x30000, 0x40000))
     assert sr.group_workspace_bytes(_fake_group_args(initial=init)) == sr.group_workspace_bytes(_fake_group_args())
+
+
+def test_prepare_lo8_validation_runs_without_a_gpu():
+    f = sr.library().sr_prepare_lo8_weights
+    assert f(ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), ctypes.c_int64(-1), None) == sr.SR_ERR_INVALID_ARG
+    assert f(None, ctypes.c_void_p(0x20000), ctypes.c_int64(8), None) == sr.SR_ERR_INVALID_ARG
+    assert f(None, None, ctypes.c_int64(0), None) == sr.SR_OK
+
+
+def test_group_fp8_low_pass_needs_its_weights_and_shapes():
+    a = _fake_group_args(precision=sr.SR_PREC_SPLIT_FP8)
+    assert sr.group_call(a, None) == sr.SR_ERR_INVALID_ARG
+    assert "low-pass weights" in sr.last_error()
+    w = a._keep[1]
+    for f in sr.LO8_FIELDS:
+        setattr(w[0], f, 0x50000)
+    assert sr.group_workspace_bytes(a) > 0
+    a.hidden = 192  # a multiple of 64 but not of 128
+    assert sr.group_call(a, None) == sr.SR_ERR_UNSUPPORTED

@@ -3,8 +3,9 @@
 Covers: the full replay-group workload (3 GDN layers + SwiGLU MLPs,
 hidden 2560, 1638-token suffix) in skip mode; small ragged multi-sequence
 groups in full mode with every intermediate hidden checked; the fast bf16
-precision mode at its derived tolerance; and group-parallel replay (several
-groups in one call give exactly the per-group results)."""
+precision mode at its derived tolerance; the fp8 low pass at the state
+tolerance; and group-parallel replay (several groups in one call give exactly
+the per-group results)."""
 import numpy as np
 import pytest
 import torch
@@ -41,6 +42,10 @@ def run(sr, gis, mode, precision, want_hidden=False):
     s = gis[0].shape
     anchors = [gi.anchors.cuda().contiguous() for gi in gis]
     weights = [[DevLayer(lw) for lw in gi.layers] for gi in gis]
+    if precision == sr.SR_PREC_SPLIT_FP8:
+        for row in weights:
+            for lw in row:
+                sr.attach_lo8(lw)
     cu = gis[0].cu_seqlens.cuda()
     out = sr.group_replay(anchors, cu, weights, max_seqlen=max(max(gis[0].lengths), 1), hidden=s.hidden,
                           inter=s.inter, h_k=s.h_k, h_v=s.h_v, d=s.d_k, eps=s.eps, mode=mode,
@@ -106,5 +111,32 @@ def test_full_group_workload(sr):
     intermediate 9216, 16/32 heads, 1638-token suffix, skip mode."""
     gi = W.group()
     out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT)
+    ref = OL.group_replay(gi, "skip")
+    check_group(out[0], ref, STATE_TOL, "skip", False)
+
+
+def test_prepare_lo8_matches_the_e5m2_format(sr):
+    """The low-pass weight copy is e5m2(w * 2^-8), round to nearest even (the
+    format's own conversion, taken here by torch on the CPU)."""
+    w = W.normal(61, "w", (300, 257), 0.02)  # 77100 weights: the vector path and a ragged tail
+    got = sr.prepare_lo8(w.cuda()).cpu()
+    want = (w.float() * 2.0 ** -8).to(torch.float8_e5m2).view(torch.uint8)
+    assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("mode", ["full", "skip"])
+def test_small_ragged_group_fp8_low_pass(sr, mode):
+    gi = W.group_inputs(31, [5, 1, 0, 70, 130, 2], n_layers=2, shape=small_shape())
+    m = sr.SR_MODE_FULL if mode == "full" else sr.SR_MODE_SKIP
+    out = run(sr, [gi], m, sr.SR_PREC_SPLIT_FP8, want_hidden=True)
+    ref = OL.group_replay(gi, mode)
+    check_group(out[0], ref, STATE_TOL, mode, True)
+
+
+def test_full_group_workload_fp8_low_pass(sr):
+    """The full replay-group workload with the projections' low pass on the fp8
+    tensor cores, at the same state tolerance as the exact split."""
+    gi = W.group()
+    out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8)
     ref = OL.group_replay(gi, "skip")
     check_group(out[0], ref, STATE_TOL, "skip", False)
