@@ -53,8 +53,7 @@ MEASURED_TRAFFIC = {
     "model_32k_5": ("gemm_tc.cu", "a6f1b53e40f6a63f", 8 * 117.6e6),
     # the raw workload's launch: 151.8 MB read + 54.0 MB written
     "raw_qwen": ("gdn_tc.cu", "e32a7269977276f7", 205.8e6),
-    # the Mamba2 workload's launch: 1252.3 MB read + 1216.5 MB written
-    "mamba2": ("mamba2_chunk.cu", "957e765a8ae46ee6", 2468.8e6),
+
 }
 
 
@@ -494,7 +493,7 @@ class Mamba2Replay:
         return self.h_y.numel() * 2 + self.h_s.numel() * 4
 
     def dominant(self):
-        return {"name": "mamba2_chunk_kernel", "bound": "hbm", "flop": self.flop_per_tok * self.tokens,
+        return {"name": "mamba2_tc_kernel", "bound": "hbm", "flop": self.flop_per_tok * self.tokens,
                 "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
 
     def oracle_sample(self, stride=1, min_s=0.0, units=16):

@@ -52,7 +52,7 @@ class Mamba2Args(ctypes.Structure):
     _fields_ = [("x", _vp), ("B", _vp), ("C", _vp), ("dt", _vp), ("A", _vp), ("cu_seqlens", _vp),
                 ("h0", _vp), ("y", _vp), ("s_out", _vp), ("n_seqs", _i32), ("total_tokens", _i32),
                 ("max_seqlen", _i32), ("n_heads", _i32), ("head_dim", _i32), ("n_groups", _i32),
-                ("d_state", _i32)]
+                ("d_state", _i32), ("algo", _i32)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -241,16 +241,21 @@ def gdn_call(args: GdnArgs, ws, stream=None) -> int:
                     _stream_handle(stream) if ws is not None else None))
 
 
+SR_MAMBA2_AUTO, SR_MAMBA2_SEQUENTIAL, SR_MAMBA2_CHUNKED, SR_MAMBA2_TCGEN05 = 0, 1, 2, 3
+_M2_ALGOS = {"auto": SR_MAMBA2_AUTO, "sequential": SR_MAMBA2_SEQUENTIAL, "chunked": SR_MAMBA2_CHUNKED,
+             "tcgen05": SR_MAMBA2_TCGEN05}
+
+
 def mamba2_args(x, B, C, dt, A, cu_seqlens, *, n_seqs, max_seqlen, h0=None, y=None,
-                s_out=None) -> Mamba2Args:
+                s_out=None, algo="auto") -> Mamba2Args:
     T, H, P = x.shape
     G, Ns = B.shape[1], B.shape[2]
     return Mamba2Args(_ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(cu_seqlens), _ptr(h0),
-                      _ptr(y), _ptr(s_out), n_seqs, T, max_seqlen, H, P, G, Ns)
+                      _ptr(y), _ptr(s_out), n_seqs, T, max_seqlen, H, P, G, Ns, _M2_ALGOS[algo])
 
 
 def mamba2_replay(x, B, C, dt, A, cu_seqlens, *, max_seqlen, h0=None, want_y=True, y=None,
-                  s_out=None, ws=None, stream=None):
+                  s_out=None, ws=None, stream=None, algo="auto"):
     """Mamba2 replay (see sr_mamba2_replay).  Returns (y or None, s_out)."""
     torch = _torch()
     _need(x, "x", torch.bfloat16, 3)
@@ -267,7 +272,7 @@ def mamba2_replay(x, B, C, dt, A, cu_seqlens, *, max_seqlen, h0=None, want_y=Tru
     if s_out is None:
         s_out = torch.empty(n, H, P, Ns, dtype=torch.float32, device=x.device)
     args = mamba2_args(x, B, C, dt, A, cu_seqlens, n_seqs=n, max_seqlen=max_seqlen, h0=h0, y=y,
-                       s_out=s_out)
+                       s_out=s_out, algo=algo)
     need = _m2_ws(ctypes.byref(args))
     if need == 0:
         _check(_m2(ctypes.byref(args), None, 0, None))

@@ -120,6 +120,9 @@ static sr_status validate_mamba2(const sr_mamba2_args *a) {
         return set_error(SR_ERR_UNSUPPORTED, "supported: head_dim 64, d_state 128 (got %d, %d)",
                          a->head_dim, a->d_state);
     if (a->n_heads > 65535) return set_error(SR_ERR_UNSUPPORTED, "n_heads > 65535");
+    if (a->algo < SR_MAMBA2_AUTO || a->algo > SR_MAMBA2_TCGEN05) return set_error(SR_ERR_INVALID_ARG, "bad algo");
+    if ((a->algo == SR_MAMBA2_CHUNKED || a->algo == SR_MAMBA2_TCGEN05) && (a->n_groups != 1 || a->n_heads % 2))
+        return set_error(SR_ERR_UNSUPPORTED, "the chunk kernels need one B/C group and an even head count");
     if (!aligned(a->s_out, 16) || (a->h0 && !aligned(a->h0, 16)) || !aligned(a->x, 16) ||
         !aligned(a->B, 16) || !aligned(a->C, 16) || (a->y && !aligned(a->y, 16)))
         return set_error(SR_ERR_INVALID_ARG, "tensors must be 16-byte aligned");

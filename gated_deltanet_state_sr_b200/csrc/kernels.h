@@ -107,6 +107,7 @@ cudaError_t to_bf16(const CastBatch &b, int n_groups, cudaStream_t st);
 cudaError_t mamba2_sequential(const sr_mamba2_args &a, uint32_t *status, cudaStream_t st);
 size_t mamba2_scratch_bytes(const sr_mamba2_args &a);
 cudaError_t mamba2_replay(const sr_mamba2_args &a, uint32_t *status, void *scratch, cudaStream_t st);
+cudaError_t mamba2_tc(const sr_mamba2_args &a, uint32_t *status, cudaStream_t st);
 
 // Dense projections on tcgen05 (gemm_tc.cu).  C[M,N] = A[M,K] B[N,K]^T with
 // a fused epilogue; all problems of one call share M, N, K and the epilogue.

@@ -307,11 +307,16 @@ mamba2_chunk_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
 
 size_t mamba2_scratch_bytes(const sr_mamba2_args &) { return 0; }
 
-// Chunked kernel for one B/C group and an even head count; the fp32
-// token-by-token kernel otherwise.
+// The tcgen05 chunk kernel (or, on request, this mma.sync one) for one B/C
+// group and an even head count; the fp32 token-by-token kernel otherwise.
 cudaError_t mamba2_replay(const sr_mamba2_args &a, uint32_t *status, void *, cudaStream_t st) {
     if (a.n_seqs == 0) return cudaSuccess;
-    if (a.n_groups != 1 || a.n_heads % 2 != 0) return mamba2_sequential(a, status, st);
+    const bool chunk_ok = a.n_groups == 1 && a.n_heads % 2 == 0;
+    int algo = a.algo;
+    if (algo == SR_MAMBA2_AUTO) algo = chunk_ok ? SR_MAMBA2_TCGEN05 : SR_MAMBA2_SEQUENTIAL;
+    if (algo == SR_MAMBA2_SEQUENTIAL || a.total_tokens == 0) return mamba2_sequential(a, status, st);
+    if (!chunk_ok) return cudaErrorInvalidValue;
+    if (algo == SR_MAMBA2_TCGEN05) return mamba2_tc(a, status, st);
     const int smem = int(sizeof(M2Smem));
     cudaError_t e = cudaFuncSetAttribute(mamba2_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

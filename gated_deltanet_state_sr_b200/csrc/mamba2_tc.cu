@@ -1,0 +1,458 @@
+// Chunked Mamba2 replay on the 5th-generation tensor cores (head dim 64,
+// d_state 128, one B/C group).
+//
+// Recurrence ("SuffixReplay: Prefix Caching via Suffix Replay for Hybrid
+// LLMs", Eq. 4, the per-head-decay instance with no erase term):
+//     S_t = exp(dt_t A_h) S_{t-1} + dt_t x_t B_t^T,   y_t = S_t C_t.
+// Per chunk of C = 64 tokens with gamma_t = sum_{r<=t} dt_r A_h (chunk
+// relative) and entry state S_0:
+//     y_t = sum_{s<=t} e^{gamma_t-gamma_s} dt_s (C_t . B_s) x_s + e^{gamma_t} S_0 C_t
+//     S_C = e^{gamma_C} S_0 + sum_s dt_s e^{gamma_C-gamma_s} x_s B_s^T.
+// A CTA takes one sequence and two heads.  Their states (64 x 128 each) are
+// stacked into one 128 x 128 fp32 accumulator in tensor memory, so every
+// product is a tcgen05 MMA with M = 128, issued by one thread:
+//     [C; B] B^T          -> G = C B^T in rows 0..63 (the B B^T rows are unused)
+//     [S_h0; S_h1] C^T    -> e^{-gamma} y's state part for both heads (bf16 copy of S)
+//     [x_h0^T; x_h1^T] [Gm_h0 | Gm_h1]^T -> the chunk-internal part; the two
+//                            diagonal 64 x 64 blocks are the two heads' outputs
+//     S += [xw_h0^T; xw_h1^T] B   (xw = x diag(dt e^{gamma_C-gamma}) as hi + lo)
+// with Gm_h = (G o L_h), L_h[t][s] = e^{gamma_t-gamma_s} dt_s for s <= t.  C, B and
+// x tiles arrive by TMA (double-buffered); full chunks of y leave by TMA.
+// Exponentials only ever see differences gamma_t - gamma_s with s <= t.
+// Every mbarrier wait is bounded; a timeout records SR_DEV_TIMEOUT, drains the
+// MMAs, frees tensor memory and ends the CTA.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace sr {
+
+namespace {
+
+using namespace tc;
+
+constexpr int C = 64, P = 64, NS = 128;
+constexpr int kThreads = 256;
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr uint32_t SZ_IN = 49152;        // one input buffer: [C_n0][B_n0][C_n1][B_n1][x_h0][x_h1], 8 KB each
+constexpr uint32_t OFF_IN = 0;           // two buffers
+constexpr uint32_t OFF_SB = 2 * SZ_IN;   // bf16 state [(h,p)][n]: two 64-column halves of 16 KB
+constexpr uint32_t OFF_Q = OFF_SB + 32768;    // masked G rows [(h,t)][s], 16 KB
+constexpr uint32_t OFF_XW = OFF_Q + 16384;    // [xwh_h0][xwh_h1][xwl_h0][xwl_h1] tiles [t][p], 8 KB each
+constexpr uint32_t OFF_YS = OFF_XW + 32768;   // y staging [y_h0][y_h1] tiles [t][p]
+constexpr uint32_t OFF_MISC = OFF_YS + 16384; // gates, tables, barriers
+constexpr uint32_t SZ_MISC = 3072;
+constexpr uint32_t kSmem = OFF_MISC + SZ_MISC + 1024;
+
+struct M2TcParams {
+    CUtensorMap mc, mb, mx, my;
+    const float *dt;
+    const float *A;
+    const int32_t *cu;
+    const float *h0;
+    __nv_bfloat16 *y;
+    float *s_out;
+    int total, max_len, H;
+    uint32_t *status;
+};
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 f = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(a - f.x, b - f.y);
+    hi = *reinterpret_cast<uint32_t *>(&h);
+    lo = *reinterpret_cast<uint32_t *>(&l);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_constant__ M2TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(sm);
+    float *gam = reinterpret_cast<float *>(sm + OFF_MISC);  // [2][64] gamma
+    float *dts = gam + 2 * C;                                // [2][64] dt (0 beyond the sequence)
+    float *wts = gam + 4 * C;                                // [2][64] dt e^{gamma_C - gamma}
+    float *egs = gam + 6 * C;                                // [2][64] e^{gamma}
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 2048);  // [2] input buffers landed
+    uint64_t *bar_g = bar_in + 2;    // C B^T done
+    uint64_t *bar_mma = bar_in + 3;  // state part of y and the state update done
+    uint64_t *bar_y = bar_in + 4;    // chunk-internal part of y done
+    uint64_t *bar_drain = bar_in + 5;  // every issued MMA done (abort path)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 6);
+    float *gs = reinterpret_cast<float *>(sm + OFF_YS);      // G = C B^T staged for the mask (before y uses it)
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;      // TMEM lane = stacked state row (head row >> 6, p = row & 63)
+    const int hrow = row >> 6, prow = row & 63;
+    const int pair = blockIdx.x;
+    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + OFF_SB));
+    int bos, eos;
+    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
+    const int len = eos - bos;
+    const int nchunks = (len + C - 1) / C;
+    const int H = p.H;
+    const size_t sbase0 = (size_t(n) * H + 2 * pair) * P * NS;  // state of head 2 pair; the pair is contiguous
+    const float *h0 = p.h0;
+    float *s_out = p.s_out;
+
+    if (nchunks == 0) {  // empty sequence: the states are h0 (or zero)
+        for (int e = tid; e < 2 * P * NS / 4; e += kThreads) {
+            const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase0)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4 *>(s_out + sbase0)[e] = v;
+        }
+        return;
+    }
+
+    if (tid == 0) {
+        mbar_init(&bar_in[0], 1);
+        mbar_init(&bar_in[1], 1);
+        mbar_init(bar_g, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_y, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t RS = tmem, RG = tmem + 128, RI = tmem + 192, RY = tmem + 256;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+
+    // ---- initial states into TMEM: row (h, p), columns n in [64 half, 64 half + 64)
+    {
+        uint32_t r[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int n0 = 64 * half + 32 * part;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                r[e] = __float_as_uint(h0 ? h0[sbase0 + size_t(row) * NS + n0 + e] : 0.f);
+            tmem_st_32x32b_x32(RS + lane_off + n0, r);
+        }
+        tmem_st_wait();
+    }
+
+    auto issue_in = [&](int c) {
+        const int b = c & 1;
+        const int y0 = bos + c * C;
+        uint8_t *in = sm + OFF_IN + b * SZ_IN;
+        mbar_arrive_expect_tx(&bar_in[b], SZ_IN);
+        tma_load_2d(in, &p.mc, &bar_in[b], 0, y0);
+        tma_load_2d(in + 8192, &p.mb, &bar_in[b], 0, y0);
+        tma_load_2d(in + 16384, &p.mc, &bar_in[b], 64, y0);
+        tma_load_2d(in + 24576, &p.mb, &bar_in[b], 64, y0);
+        tma_load_2d(in + 32768, &p.mx, &bar_in[b], (2 * pair) * P, y0);
+        tma_load_2d(in + 40960, &p.mx, &bar_in[b], (2 * pair + 1) * P, y0);
+    };
+    if (tid == 0) {
+        prefetch_tmap(&p.mc); prefetch_tmap(&p.mb); prefetch_tmap(&p.mx);
+        if (p.y) prefetch_tmap(&p.my);
+        issue_in(0);
+    }
+
+    // dt of the next chunk: thread tid < 128 holds token (tid & 63) of head (tid >> 6) of the pair
+    const int dh = (tid >> 6) & 1, dtok = tid & 63;
+    const float Ah = p.A[2 * pair + (warp & 1)];  // warps 0 and 1 scan heads 0 and 1
+    float dt_next = (tid < 128 && dtok < len) ? p.dt[(size_t(bos) + dtok) * H + 2 * pair + dh] : 0.f;
+    bool ok = true;
+    // each MMA barrier completes once per chunk: its phase parity is the chunk's
+    auto wait_on = [&](uint64_t *bar, int c) -> bool {
+        const bool w = mbar_wait(bar, uint32_t(c & 1));
+        tc_fence_after();
+        return w;
+    };
+    auto check = [&](bool w) -> bool {
+        const bool stop = __syncthreads_or(!w) != 0;
+        if (stop && tid == 0) *abort_flag = 1;
+        return stop;
+    };
+    constexpr uint32_t ID_G = idesc_bf16_f32_major(128, 64, 0, 0);      // [C;B] B^T, [S] C^T
+    constexpr uint32_t ID_Y = idesc_bf16_f32_major(128, 128, 1, 0);     // x^T (MN-major) Q^T
+    constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 1, 1);     // xw^T (MN-major) B (MN-major)
+    const bool want_y = p.y != nullptr;
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int b = c & 1;
+        const uint32_t in = base + OFF_IN + b * SZ_IN;
+        const int clen = min(C, len - c * C);
+        // ---- gates of the chunk: gamma = inclusive prefix sum of dt A (dt = 0 beyond the sequence)
+        if (tid < 128) {
+            dts[dh * C + dtok] = dt_next;
+            const int t = (c + 1) * C + dtok;
+            dt_next = (t < len) ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
+        }
+        const bool tma_ok = mbar_wait(&bar_in[b], (c >> 1) & 1);
+        if (tid == 0) bulk_wait_read();  // the previous chunk's y tiles have left the staging area
+        __syncthreads();
+        if (warp < 2) {
+            const float *d = dts + warp * C;
+            const float a0 = d[2 * lane] * Ah, a1 = d[2 * lane + 1] * Ah;
+            float incl = a0 + a1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const float excl = incl - (a0 + a1);
+            gam[warp * C + 2 * lane] = excl + a0;
+            gam[warp * C + 2 * lane + 1] = excl + a0 + a1;
+        }
+        if (check(tma_ok)) break;
+        // the input buffer of chunk c+1 last served chunk c-1, whose products have completed
+        if (tid == 0 && c + 1 < nchunks) issue_in(c + 1);
+        if (tid < 128) {
+            const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
+            wts[dh * C + dtok] = dts[dh * C + dtok] * __expf(gC - g);
+            egs[dh * C + dtok] = __expf(g);
+        }
+        __syncthreads();
+
+        // ---- bf16 copy of S (for y) and S <- e^{gamma_C} S in TMEM; xw = x diag(w) as hi + lo
+        {
+            const float fC = __expf(gam[hrow * C + C - 1]);
+            uint32_t r[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int n0 = 64 * half + 32 * part;
+                tmem_ld_32x32b_x32(RS + lane_off + n0, r);
+                tmem_ld_wait();
+                if (want_y) {
+                    uint8_t *sb = sm + OFF_SB + half * 16384;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 w;
+                        w.x = pack2(__uint_as_float(r[8 * q4 + 0]), __uint_as_float(r[8 * q4 + 1]));
+                        w.y = pack2(__uint_as_float(r[8 * q4 + 2]), __uint_as_float(r[8 * q4 + 3]));
+                        w.z = pack2(__uint_as_float(r[8 * q4 + 4]), __uint_as_float(r[8 * q4 + 5]));
+                        w.w = pack2(__uint_as_float(r[8 * q4 + 6]), __uint_as_float(r[8 * q4 + 7]));
+                        *reinterpret_cast<uint4 *>(sb + sw128(row, 4 * part + q4)) = w;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
+                tmem_st_32x32b_x32(RS + lane_off + n0, r);
+            }
+            tmem_st_wait();
+        }
+        {
+            // thread: head hx, token tx, 32 p values (4 chunks of 8)
+            const int hx = tid >> 7, tx = (tid >> 1) & 63, c0 = (tid & 1) * 4;
+            const float wgt = wts[hx * C + tx];
+            const uint8_t *xt = sm + OFF_IN + b * SZ_IN + 32768 + hx * 8192;
+            uint8_t *xh = sm + OFF_XW + hx * 8192, *xl = sm + OFF_XW + 16384 + hx * 8192;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint32_t off = sw128(tx, c0 + v);
+                const uint4 u = *reinterpret_cast<const uint4 *>(xt + off);
+                const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(x2[e]);
+                    split2(f.x * wgt, f.y * wgt, hi[e], lo[e]);
+                }
+                *reinterpret_cast<uint4 *>(xh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(xl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (check(true)) break;
+
+        // ---- MMAs: G = [C;B] B^T -> RG (own commit); Yi^T = [S] C^T -> RI; S += xw^T B (hi, lo)
+        if (tid == 0) {
+            tc_fence_after();
+            if (want_y) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
+                }
+                mma_commit(bar_g);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t a = base + OFF_SB + (k >> 2) * 16384 + (k & 3) * 32;
+                    const uint32_t bc = in + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16_ss(RI, sdesc_sw128(a, 16, 1024), sdesc_sw128(bc, 16, 1024), ID_G, k > 0);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t bmn = in + 8192 + k * 2048;  // B as MN-major (n halves 16 KB apart)
+                mma_bf16_ss(RS, sdesc_sw128(base + OFF_XW + k * 2048, 8192, 1024), sdesc_sw128(bmn, 16384, 1024),
+                            ID_S, 1);
+                mma_bf16_ss(RS, sdesc_sw128(base + OFF_XW + 16384 + k * 2048, 8192, 1024),
+                            sdesc_sw128(bmn, 16384, 1024), ID_S, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        if (!want_y) {
+            if (check(wait_on(bar_mma, c))) break;
+            continue;
+        }
+
+        // ---- Gm_h rows: Q[(h, t)][s] = G[t][s] e^{gamma_h,t - gamma_h,s} dt_h,s (s <= t), bf16.
+        // G lives in TMEM lanes 0..63, which half of the warps can read: they stage it
+        // in shared memory (columns XOR-swizzled by row), then all warps build the rows
+        // while the other products run.
+        const bool mg = wait_on(bar_g, c);
+        if (quad < 2) {
+            const int t = row;
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(RG + lane_off + 32 * half, r);
+            tmem_ld_wait();
+            const int sw = (t & 7) << 2;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4 *>(gs + t * C + ((32 * half + 4 * j) ^ sw)) =
+                    make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
+                                __uint_as_float(r[4 * j + 3]));
+        }
+        if (check(mg)) break;
+        {
+            // thread: head hq, token tq, 32 columns s0 .. s0 + 31
+            const int hq = tid >> 7, tq = (tid >> 1) & 63, s0 = (tid & 1) * 32;
+            const float gt = gam[hq * C + tq];
+            const float *gh = gam + hq * C, *dh2 = dts + hq * C;
+            const int sw = (tq & 7) << 2;
+            uint8_t *qrow = sm + OFF_Q;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 ga = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4) ^ sw));
+                const float4 gb = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4 + 4) ^ sw));
+                const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int s = s0 + 8 * q4 + 2 * u;
+                    const float d0 = s <= tq ? __expf(gt - gh[s]) * dh2[s] : 0.f;
+                    const float d1 = s + 1 <= tq ? __expf(gt - gh[s + 1]) * dh2[s + 1] : 0.f;
+                    w[u] = pack2(d0 * gv[2 * u], d1 * gv[2 * u + 1]);
+                }
+                *reinterpret_cast<uint4 *>(qrow + sw128(hq * C + tq, (s0 >> 3) + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (check(true)) break;
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // [x_h0^T; x_h1^T] (MN-major, head blocks 8 KB apart) Q^T
+                mma_bf16_ss(RY, sdesc_sw128(in + 32768 + k * 2048, 8192, 1024),
+                            sdesc_sw128(base + OFF_Q + k * 32, 16, 1024), ID_Y, k > 0);
+            mma_commit(bar_y);
+        }
+        const bool m2 = wait_on(bar_mma, c) && wait_on(bar_y, c);
+        if (check(m2)) break;
+
+        // ---- y_t = e^{gamma_t} Yi + Y (own head's diagonal block); thread = (h, p), 32 tokens
+        {
+            uint32_t ri[32], ry[32];
+            tmem_ld_32x32b_x32(RI + lane_off + 32 * half, ri);
+            tmem_ld_32x32b_x32(RY + lane_off + 64 * hrow + 32 * half, ry);
+            tmem_ld_wait();
+            const float *eg = egs + hrow * C;
+            if (clen == C) {
+                uint8_t *yt = sm + OFF_YS + hrow * 8192;
+                const uint32_t cofs = uint32_t(prow & 7) * 2, chunk = uint32_t(prow) >> 3;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int t = 32 * half + e;
+                    *reinterpret_cast<__nv_bfloat16 *>(yt + sw128(t, chunk) + cofs) =
+                        __float2bfloat16_rn(eg[t] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
+                }
+                fence_async_smem();
+            } else {
+                const size_t tok0 = size_t(bos) + size_t(c) * C;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int t = 32 * half + e;
+                    if (t < clen)
+                        p.y[((tok0 + t) * H + 2 * pair + hrow) * P + prow] =
+                            __float2bfloat16_rn(eg[t] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && clen == C) {
+            tma_store_2d(&p.my, sm + OFF_YS, (2 * pair) * P, bos + c * C);
+            tma_store_2d(&p.my, sm + OFF_YS + 8192, (2 * pair + 1) * P, bos + c * C);
+            bulk_commit();
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+
+    __syncthreads();
+    ok = *abort_flag == 0;
+    if (ok) {
+        uint32_t r[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int n0 = 64 * half + 32 * part;
+            tmem_ld_32x32b_x32(RS + lane_off + n0, r);
+            tmem_ld_wait();
+            float4 *dst = reinterpret_cast<float4 *>(s_out + sbase0 + size_t(row) * NS + n0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                     __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+        }
+    } else if (tid == 0) {
+        atomicOr(p.status, SR_DEV_TIMEOUT);
+        // let in-flight MMAs and TMA copies finish before tensor and shared memory are released
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0);
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t mamba2_tc(const sr_mamba2_args &a, uint32_t *status, cudaStream_t st) {
+    M2TcParams p{};
+    const int T = a.total_tokens, hp = a.n_heads * P;
+    if (!make_map_bf16(&p.mc, a.C, T, NS, NS, 64, 64) || !make_map_bf16(&p.mb, a.B, T, NS, NS, 64, 64) ||
+        !make_map_bf16(&p.mx, a.x, T, hp, hp, 64, 64))
+        return cudaErrorInvalidValue;
+    if (a.y && !make_map_bf16(&p.my, a.y, T, hp, hp, 64, 64)) return cudaErrorInvalidValue;
+    p.dt = a.dt;
+    p.A = a.A;
+    p.cu = a.cu_seqlens;
+    p.h0 = a.h0;
+    p.y = static_cast<__nv_bfloat16 *>(a.y);
+    p.s_out = a.s_out;
+    p.total = a.total_tokens;
+    p.max_len = a.max_seqlen;
+    p.H = a.n_heads;
+    p.status = status;
+    cudaError_t e = cudaFuncSetAttribute(mamba2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.n_heads / 2, a.n_seqs);
+    mamba2_tc_kernel<<<grid, kThreads, kSmem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace sr

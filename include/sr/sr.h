@@ -149,7 +149,19 @@ SR_API sr_status sr_gdn_replay(const sr_gdn_args *args, void *workspace, size_t 
  *   y          [total_tokens, n_heads, head_dim]   bf16, may be NULL
  *   s_out      [n_seqs, n_heads, head_dim, d_state] fp32, required
  * Supported: head_dim = 64, d_state = 128.
+ * algo: SR_MAMBA2_AUTO picks the tcgen05 chunk kernel for one B/C group and
+ *   an even head count, the fp32 token-by-token kernel otherwise;
+ *   SR_MAMBA2_SEQUENTIAL, SR_MAMBA2_CHUNKED (mma.sync chunk kernel, same
+ *   shape limits as the tcgen05 one) and SR_MAMBA2_TCGEN05 force a kernel
+ *   (SR_ERR_UNSUPPORTED when the shape does not fit it).
  * ---------------------------------------------------------------------- */
+typedef enum sr_mamba2_algo {
+    SR_MAMBA2_AUTO = 0,
+    SR_MAMBA2_SEQUENTIAL = 1,
+    SR_MAMBA2_CHUNKED = 2,
+    SR_MAMBA2_TCGEN05 = 3
+} sr_mamba2_algo;
+
 typedef struct sr_mamba2_args {
     const void *x;
     const void *B;
@@ -164,6 +176,7 @@ typedef struct sr_mamba2_args {
     int32_t total_tokens;
     int32_t max_seqlen;
     int32_t n_heads, head_dim, n_groups, d_state;
+    int32_t algo;  /* sr_mamba2_algo */
 } sr_mamba2_args;
 
 SR_API size_t sr_mamba2_replay_workspace(const sr_mamba2_args *args);
