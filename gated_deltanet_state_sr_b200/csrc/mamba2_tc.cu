@@ -35,6 +35,10 @@ using namespace tc;
 
 constexpr int C = 64, P = 64, NS = 128;
 constexpr int kThreads = 256;
+// MMA and TMA issue is spread over threads of warps that are idle at that point:
+// warp 7 (no gate-table work) loads the next chunk and forms C B^T at the chunk
+// start; warp 2 (no part in staging C B^T) issues the products after the state copy.
+constexpr int kIssueIn = 224, kIssueMma = 64;
 
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t SZ_IN = 49152;        // one input buffer: [C_n0][B_n0][C_n1][B_n1][x_h0][x_h1], 8 KB each
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         mbar_init(bar_g, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_y, 1);
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_drain, 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -158,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         tma_load_2d(in + 32768, &p.mx, &bar_in[b], (2 * pair) * P, y0);
         tma_load_2d(in + 40960, &p.mx, &bar_in[b], (2 * pair + 1) * P, y0);
     };
-    if (tid == 0) {
+    if (tid == kIssueIn) {
         prefetch_tmap(&p.mc); prefetch_tmap(&p.mb); prefetch_tmap(&p.mx);
         if (p.y) prefetch_tmap(&p.my);
         issue_in(0);
@@ -212,8 +216,19 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             gam[warp * C + 2 * lane + 1] = excl + a0 + a1;
         }
         if (check(tma_ok)) break;
-        // the input buffer of chunk c+1 last served chunk c-1, whose products have completed
-        if (tid == 0 && c + 1 < nchunks) issue_in(c + 1);
+        if (tid == kIssueIn) {
+            // the input buffer of chunk c+1 last served chunk c-1, whose products have completed
+            if (c + 1 < nchunks) issue_in(c + 1);
+            if (want_y) {  // G = [C;B] B^T -> RG needs only this chunk's inputs
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
+                }
+                mma_commit(bar_g);
+            }
+        }
         if (tid < 128) {
             const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
             wts[dh * C + dtok] = dts[dh * C + dtok] * __expf(gC - g);
@@ -273,16 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         tc_fence_before();
         if (check(true)) break;
 
-        // ---- MMAs: G = [C;B] B^T -> RG (own commit); Yi^T = [S] C^T -> RI; S += xw^T B (hi, lo)
-        if (tid == 0) {
+        // ---- MMAs: Yi^T = [S] C^T -> RI; S += xw^T B (hi, lo)
+        if (tid == kIssueMma) {
             tc_fence_after();
             if (want_y) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
-                }
-                mma_commit(bar_g);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t a = base + OFF_SB + (k >> 2) * 16384 + (k & 3) * 32;
@@ -349,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         fence_async_smem();
         tc_fence_before();
         if (check(true)) break;
-        if (tid == 0) {
+        if (tid == kIssueMma) {
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 4; ++k)  // [x_h0^T; x_h1^T] (MN-major, head blocks 8 KB apart) Q^T
@@ -414,12 +423,15 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
                 dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
                                      __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
         }
-    } else if (tid == 0) {
-        atomicOr(p.status, SR_DEV_TIMEOUT);
-        // let in-flight MMAs and TMA copies finish before tensor and shared memory are released
-        mma_commit(bar_drain);
-        mbar_wait(bar_drain, 0);
-        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    } else {
+        // let in-flight MMAs (of both issuing threads) and TMA copies finish before
+        // tensor and shared memory are released
+        if (tid == kIssueIn || tid == kIssueMma) mma_commit(bar_drain);
+        if (tid == kIssueMma) {
+            atomicOr(p.status, SR_DEV_TIMEOUT);
+            mbar_wait(bar_drain, 0);
+            for (int i = 0; i < 64; ++i) __nanosleep(1000);
+        }
     }
     tc_fence_before();
     __syncthreads();
