@@ -182,6 +182,23 @@ class RawGdn:
         self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
         self.h_s = torch.empty(self.s.shape, dtype=torch.float32).pin_memory()
         self.d_in = [self.q, self.k, self.v, self.g, self.b, self.cu]
+        # second device buffer set for the pipelined end-to-end leg
+        self.alt_in = [t.clone() for t in self.d_in]
+        self.alt_o, self.alt_s = torch.empty_like(self.o), torch.empty_like(self.s)
+
+    def e2e_inputs(self, b):
+        return list(zip(self.h_in, self.d_in if b == 0 else self.alt_in))
+
+    def e2e_outputs(self, b):
+        o, s = (self.o, self.s) if b == 0 else (self.alt_o, self.alt_s)
+        return [(o, self.h_o), (s, self.h_s)]
+
+    def step_on(self, b):
+        if b == 0:
+            self.step()
+            return
+        q, k, v, g, be, cu = self.alt_in
+        self.sr.gdn_replay(q, k, v, g, be, cu, max_seqlen=self.max_len, o=self.alt_o, s_out=self.alt_s, ws=self.ws)
 
     def step(self):
         self.sr.gdn_replay(self.q, self.k, self.v, self.g, self.b, self.cu, max_seqlen=self.max_len,
@@ -473,6 +490,24 @@ class Mamba2Replay:
         self.d_in = [self.x, self.B, self.C, self.dt, self.cu]
         self.h_y = torch.empty(self.y.shape, dtype=self.y.dtype).pin_memory()
         self.h_s = torch.empty(self.s.shape, dtype=torch.float32).pin_memory()
+        # second device buffer set for the pipelined end-to-end leg
+        self.alt_in = [t.clone() for t in self.d_in]
+        self.alt_y, self.alt_s = torch.empty_like(self.y), torch.empty_like(self.s)
+
+    def e2e_inputs(self, b):
+        return list(zip(self.h_in, self.d_in if b == 0 else self.alt_in))
+
+    def e2e_outputs(self, b):
+        y, s = (self.y, self.s) if b == 0 else (self.alt_y, self.alt_s)
+        return [(y, self.h_y), (s, self.h_s)]
+
+    def step_on(self, b):
+        if b == 0:
+            self.step()
+            return
+        x, B, C, dt, cu = self.alt_in
+        self.sr.mamba2_replay(x, B, C, dt, self.A, cu, max_seqlen=self.max_len, y=self.alt_y, s_out=self.alt_s,
+                              ws=self.ws)
 
     def step(self):
         self.sr.mamba2_replay(self.x, self.B, self.C, self.dt, self.A, self.cu, max_seqlen=self.max_len,
