@@ -140,3 +140,15 @@ def test_full_group_workload_fp8_low_pass(sr):
     out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8)
     ref = OL.group_replay(gi, "skip")
     check_group(out[0], ref, STATE_TOL, "skip", False)
+
+
+@pytest.mark.parametrize("prefix,ratio", [(8192, 0.05), (32768, 0.05)])
+def test_whole_model_groups_0_and_7(sr, prefix, ratio):
+    """The whole-model replay (8 groups of 3 GDN layers, group-parallel, FA
+    skipped, suffix k = ceil(r m)) in the bench's default precision: all 8
+    groups in one call, the first and the last checked against the oracle."""
+    gis = [W.model_group(prefix, ratio, g) for g in range(8)]
+    out = run(sr, gis, sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8)
+    for g in (0, 7):
+        ref = OL.group_replay(gis[g], "skip")
+        check_group(out[g], ref, STATE_TOL, "skip", False)
