@@ -95,6 +95,17 @@ __device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float *X, cons
     }
 }
 
+// Loads a 16 x 16 fp32 block into the accumulator layout of blk_mma.
+__device__ __forceinline__ void blk_load(float (&acc)[2][4], const float *Z, int lane) {
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const float2 a = *reinterpret_cast<const float2 *>(Z + g * ROWA + 8 * nt + 2 * q);
+        const float2 b = *reinterpret_cast<const float2 *>(Z + (g + 8) * ROWA + 8 * nt + 2 * q);
+        acc[nt][0] = a.x; acc[nt][1] = a.y; acc[nt][2] = b.x; acc[nt][3] = b.y;
+    }
+}
+
 // Stores sign * acc (accumulator layout of blk_mma) as a 16 x 16 fp32 block.
 __device__ __forceinline__ void blk_store(float *Z, const float (&acc)[2][4], int lane, float sign) {
     const int g = lane >> 2, q = lane & 3;
@@ -430,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         // ---- T = (I + A)^{-1} by 16x16 blocks (A strictly lower):
         //   T_ii  = (I + A_ii)^{-1}, fp32 forward substitution, one column per thread
         //   B_ik  = T_ii A_ik (k < i), kept in the unused upper blocks of T
-        //   T_ij  = -sum_{k=j}^{i-1} B_ik T_kj, by block distance i - j = 1, 2, 3
+        //   T_ij  = -sum_{k=j}^{i-1} B_ik T_kj, in three rounds of independent products
         // The block products run on mma.sync with split bf16 operands (blk_mma).
         // T_ii by 8 x 8 halves: D = (I + N)^{-1} of each half by forward substitution,
         // then the lower-left half -D2 (N21 D1) (its temporary N21 D1 sits in the
@@ -480,17 +491,38 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             }
         }
         __syncthreads();
-#pragma unroll
-        for (int level = 1; level <= 3; ++level) {
-            // blocks (j + level, j), j = 0 .. 3 - level: warp j takes block j
-            if (warp + level <= 3) {
-                const int j = warp, i = j + level;
-                float acc[2][4] = {};
-                for (int k = j; k < i; ++k) blk_mma(acc, Tf + blk(k, i), Tf + blk(k, j), lane);
-                blk_store(Tf + blk(i, j), acc, lane, -1.f);
-            }
-            __syncthreads();
+        // T_ij = -sum_{k=j}^{i-1} B_ik T_kj in three rounds of independent products;
+        // the partial sums of T_20, T_31 and T_30 wait in their own blocks:
+        //   1: T_10, T_21, T_32 and the partials B_20 T_00, B_31 T_11, B_30 T_00
+        //   2: T_20, T_31 (partial + last term) and B_31 T_10 added to T_30's partial
+        //   3: T_30
+        // (B_ik is kept in the upper block (k, i))
+        if (warp < 6) {
+            // warps 0-2: (i, j) = (1,0) (2,1) (3,2); warps 3-5: (2,0) (3,1) (3,0)
+            const int i = warp < 3 ? warp + 1 : (warp == 3 ? 2 : 3);
+            const int j = warp < 3 ? warp : (warp == 4 ? 1 : 0);
+            float acc[2][4] = {};
+            blk_mma(acc, Tf + blk(j, i), Tf + blk(j, j), lane);  // B_ij T_jj
+            blk_store(Tf + blk(i, j), acc, lane, warp < 3 ? -1.f : 1.f);
         }
+        __syncthreads();
+        if (warp < 3) {
+            // warp 0: T_20 = -(P_20 + B_21 T_10); warp 1: T_31 = -(P_31 + B_32 T_21);
+            // warp 2: P_30 += B_31 T_10
+            const int i = warp == 0 ? 2 : 3, j = warp == 1 ? 1 : 0, k = warp == 1 ? 2 : 1;
+            float acc[2][4];
+            blk_load(acc, Tf + blk(i, j), lane);
+            blk_mma(acc, Tf + blk(k, i), Tf + blk(k, j), lane);
+            blk_store(Tf + blk(i, j), acc, lane, warp < 2 ? -1.f : 1.f);
+        }
+        __syncthreads();
+        if (warp == 0) {  // T_30 = -(P_30 + B_32 T_20)
+            float acc[2][4];
+            blk_load(acc, Tf + blk(3, 0), lane);
+            blk_mma(acc, Tf + blk(2, 3), Tf + blk(2, 0), lane);
+            blk_store(Tf + blk(3, 0), acc, lane, -1.f);
+        }
+        __syncthreads();
         // T1 = T diag(beta e^gamma) (bf16), T2 = T diag(beta) (hi + lo): K-major tiles [t][s].
         // A thread always covers the same 8 columns, so their factors stay in registers.
         {
