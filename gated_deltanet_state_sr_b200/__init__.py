@@ -534,3 +534,23 @@ def attach_lo8(layer, stream=None):
     for f in LO8_FIELDS:
         setattr(layer, f, prepare_lo8(getattr(layer, f[:-4]), stream))
     return layer
+
+
+# ------------------------------------------------------------------ checkpoint placement (host)
+
+_ckpt = _sig("sr_checkpoint_plan", _i32, ctypes.POINTER(ctypes.c_double), ctypes.c_int64, _i32,
+             ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double))
+
+
+def checkpoint_plan(p, m_max):
+    """sr_checkpoint_plan (host): (positions, expected recompute) of the best
+    placement of at most m_max checkpoints for depth weights p[0..N]."""
+    import numpy as np
+    w = np.ascontiguousarray(p, dtype=np.float64)
+    n = w.size - 1
+    pos = (ctypes.c_int64 * max(m_max, 1))()
+    cnt = _i32(0)
+    cost = ctypes.c_double(0.0)
+    _check(_ckpt(w.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), n, m_max, pos, ctypes.byref(cnt),
+                 ctypes.byref(cost)))
+    return list(pos[:cnt.value]), cost.value

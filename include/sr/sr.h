@@ -435,6 +435,28 @@ SR_API sr_status sr_sparse_anchor_plan(const sr_anchor_plan_args *args, int64_t 
                                        int64_t capacity, int64_t *count);
 
 /* ------------------------------------------------------------------------
+ * sr_checkpoint_plan -- host: where to keep recurrent-state checkpoints.
+ *
+ * The checkpoint alternative to replay ("Sparse Prefix Caching for Hybrid and
+ * Recurrent LLM Serving", Methodology): a retained prefix of n tokens keeps
+ * exact states at up to m_max positions C in 1..n; a request overlapping the
+ * prefix to depth t resumes from max({0} u {c in C : c <= t}) and recomputes
+ * the rest.  Given p[t] (t = 0..n, any non-negative weights: the overlap-depth
+ * distribution or a histogram of it), the call returns the placement that
+ * minimises sum_t p[t] (t - l(t; C)), by the exact dynamic program of that
+ * page, O(n m_max) with the monotone convex-hull trick.
+ *   positions  host [m_max] out: the chosen positions, increasing (fewer than
+ *              m_max when more checkpoints would not lower the cost)
+ *   count      host out: how many positions were written
+ *   expected_cost  host out (may be NULL): sum_t p[t] r(t; C) of the result
+ * Pure host code.  Errors: SR_ERR_INVALID_ARG for NULL pointers, n < 0,
+ * m_max < 0 or a negative weight; SR_ERR_UNSUPPORTED when n (m_max + 1)
+ * exceeds 2^31.
+ * ---------------------------------------------------------------------- */
+SR_API sr_status sr_checkpoint_plan(const double *p, int64_t n, int32_t m_max, int64_t *positions, int32_t *count,
+                                    double *expected_cost);
+
+/* ------------------------------------------------------------------------
  * Status and diagnostics.
  * ---------------------------------------------------------------------- */
 /* Message for the calling thread's last failed call ("" if none). */

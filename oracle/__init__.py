@@ -12,12 +12,16 @@ Contents
 * ``mamba2_replay``  Mamba2 per-head-decay recurrence, fp64 (C).
 * ``layers``         the GDN layer, the SwiGLU MLP and the replay-group
                      schedule in numpy fp64 (``oracle/layers.py``).
+* ``planning``       checkpoint placement: the objective, exhaustive search
+                     and the literal recurrence (``oracle/planning.py``).
 
 Parity status of each function (what pins it, see ``tests/test_oracle_*``):
 * gdn_replay / mamba2_replay: pinned by closed forms (beta = 0 decay,
   orthonormal-key sum, Mamba2 decay-weighted sum), an explicit unrolled
   transition-product brute force, the contraction bound of the suffix
   approximation and the exact-resume identity.
+* planning.*: pinned by the balanced optimum of uniform overlap depths and
+  by point masses; the recurrence against exhaustive search.
 * layers.*: each primitive pinned by closed forms; the *composition* of a
   GDN layer (order of norm, conv, gates, gated norm, MLP) is not printed on
   the pages -- parity unpinned beyond the readings listed in the design
