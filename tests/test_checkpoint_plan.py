@@ -81,3 +81,25 @@ def test_plan_arguments():
     assert sr.checkpoint_plan([1.0], 3) == ([], 0.0)       # N = 0: nothing to place
     pos, cost = sr.checkpoint_plan(np.zeros(50), 4)         # no weight anywhere: nothing worth placing
     assert pos == [] and cost == 0.0
+
+
+def test_no_budget_and_full_budget():
+    """M = 0 leaves every request at the empty state: the cost is the mean
+    depth.  With M >= N every depth can hold a checkpoint: the cost is 0."""
+    rng = np.random.default_rng(11)
+    p = rng.random(40)
+    mean_depth = float(np.dot(np.arange(40), p))
+    assert PL.optimal_by_enumeration(p[:9], 0)[0] == pytest.approx(float(np.dot(np.arange(9), p[:9])))
+    assert sr.checkpoint_plan(p, 0) == ([], pytest.approx(mean_depth))
+    for m in (39, 60):
+        pos, cost = sr.checkpoint_plan(p, m)
+        assert cost == 0.0 and pos == list(range(1, 40))
+
+
+def test_plan_on_uniform_depths_is_balanced():
+    """The C planner reaches the balanced-spacing optimum on uniform depths."""
+    for N, m in [(100, 3), (257, 7), (64, 63)]:
+        pos, cost = sr.checkpoint_plan(np.ones(N + 1), m)
+        lengths = np.diff([0, *pos, N + 1])
+        assert len(pos) == m and lengths.max() - lengths.min() <= 1
+        assert cost == pytest.approx(sum(L * (L - 1) / 2 for L in lengths))
