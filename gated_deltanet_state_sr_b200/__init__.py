@@ -31,11 +31,11 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 SR_OK, SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_WORKSPACE, SR_ERR_CUDA, SR_ERR_DEVICE = range(6)
 SR_BF16, SR_FP32 = 0, 1
-SR_GDN_AUTO, SR_GDN_SEQUENTIAL, SR_GDN_CHUNKED, SR_GDN_TCGEN05 = 0, 1, 2, 3
+SR_GDN_AUTO, SR_GDN_SEQUENTIAL, SR_GDN_CHUNKED, SR_GDN_TCGEN05, SR_GDN_TCGEN05_FUSED = 0, 1, 2, 3, 4
 SR_MODE_SKIP, SR_MODE_FULL = 0, 1
 SR_DEV_BAD_CU_SEQLENS, SR_DEV_SEQ_TOO_LONG, SR_DEV_TIMEOUT, SR_DEV_BAD_INDEX = 0x1, 0x2, 0x4, 0x8
 _ALGOS = {"auto": SR_GDN_AUTO, "sequential": SR_GDN_SEQUENTIAL, "chunked": SR_GDN_CHUNKED,
-          "tcgen05": SR_GDN_TCGEN05}
+          "tcgen05": SR_GDN_TCGEN05, "tcgen05_fused": SR_GDN_TCGEN05_FUSED}
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32

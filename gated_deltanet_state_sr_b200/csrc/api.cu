@@ -57,11 +57,12 @@ sr_status validate_gdn(const sr_gdn_args *a) {
         return set_error(SR_ERR_UNSUPPORTED, "head dims must satisfy d_k == d_v in {64,128} (got %d,%d)",
                          a->d_k, a->d_v);
     if (a->dtype != SR_BF16 && a->dtype != SR_FP32) return set_error(SR_ERR_INVALID_ARG, "bad dtype");
-    if (a->algo < SR_GDN_AUTO || a->algo > SR_GDN_TCGEN05) return set_error(SR_ERR_INVALID_ARG, "bad algo");
-    if ((a->algo == SR_GDN_CHUNKED || a->algo == SR_GDN_TCGEN05) && a->dtype != SR_BF16)
+    if (a->algo < SR_GDN_AUTO || a->algo > SR_GDN_TCGEN05_FUSED) return set_error(SR_ERR_INVALID_ARG, "bad algo");
+    const bool tc = a->algo == SR_GDN_TCGEN05 || a->algo == SR_GDN_TCGEN05_FUSED;
+    if ((a->algo == SR_GDN_CHUNKED || tc) && a->dtype != SR_BF16)
         return set_error(SR_ERR_UNSUPPORTED, "the chunked kernels take bf16 q/k/v only");
-    if (a->algo == SR_GDN_TCGEN05 && !gdn_tc_supported(a->d_k))
-        return set_error(SR_ERR_UNSUPPORTED, "the tcgen05 kernel takes d_k = d_v = 128 only");
+    if (tc && !gdn_tc_supported(a->d_k))
+        return set_error(SR_ERR_UNSUPPORTED, "the tcgen05 kernels take d_k = d_v = 128 only");
     if (!aligned(a->s_out, 16) || (a->h0 && !aligned(a->h0, 16)))
         return set_error(SR_ERR_INVALID_ARG, "s_out and h0 must be 16-byte aligned");
     const size_t esz = a->dtype == SR_BF16 ? 2 : 4;
@@ -82,14 +83,27 @@ const char *sr_last_error(void) { return g_err; }
 
 int32_t sr_version(void) { return 0x000100; }
 
+// The tcgen05 form a call runs: 0 none, 1 two-phase, 2 fused.
+static int gdn_tc_form(const sr_gdn_args *a) {
+    if (a->algo == SR_GDN_TCGEN05_FUSED) return 2;
+    if (a->algo == SR_GDN_TCGEN05) return 1;
+    return a->algo == SR_GDN_AUTO && a->dtype == SR_BF16 && gdn_tc_supported(a->d_k) ? 1 : 0;
+}
+
+static size_t gdn_need(const sr_gdn_args *a) {
+    const int form = gdn_tc_form(a);
+    if (form == 1) return kWsHeader + gdn_tc_image_bytes(a->total_tokens, a->n_seqs, a->h_v, 1);
+    return kWsHeader + (form == 0 ? gdn_scratch_bytes(*a) : 0);
+}
+
 size_t sr_gdn_replay_workspace(const sr_gdn_args *a) {
     if (validate_gdn(a) != SR_OK) return 0;
-    return kWsHeader + gdn_scratch_bytes(*a);
+    return gdn_need(a);
 }
 
 sr_status sr_gdn_replay(const sr_gdn_args *a, void *ws, size_t ws_bytes, void *stream) {
     if (sr_status s = validate_gdn(a)) return s;
-    const size_t need = kWsHeader + gdn_scratch_bytes(*a);
+    const size_t need = gdn_need(a);
     if (sr_status s = check_workspace(ws, ws_bytes, need)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t *status = static_cast<uint32_t *>(ws);
@@ -99,10 +113,9 @@ sr_status sr_gdn_replay(const sr_gdn_args *a, void *ws, size_t ws_bytes, void *s
     const bool chunked = a->algo == SR_GDN_CHUNKED || (a->algo == SR_GDN_AUTO && a->dtype == SR_BF16 &&
                                                         gdn_chunked_supported(*a));
     void *scratch = static_cast<char *>(ws) + kWsHeader;
-    const bool use_tc = a->algo == SR_GDN_TCGEN05 ||
-                        (a->algo == SR_GDN_AUTO && a->dtype == SR_BF16 && gdn_tc_supported(a->d_k));
-    if (use_tc)
-        e = gdn_tc(*a, scale, status, st);
+    const int form = gdn_tc_form(a);
+    if (form)
+        e = gdn_tc(*a, scale, status, form == 1 ? scratch : nullptr, st);
     else
         e = chunked ? gdn_chunked(*a, scale, status, scratch, st) : gdn_sequential(*a, scale, status, st);
     if (e != cudaSuccess) return cuda_error(e, "sr_gdn_replay: kernel launch");

@@ -6,9 +6,9 @@
 //     W   = T diag(beta e^gamma) K,   Ut = T diag(beta) V,    U = Ut - W S^T
 //     O   = scale (diag(e^gamma) Q S^T + M U),  M = lower(e^{gamma_t-gamma_s} q_t.k_s)
 //     S  <- e^{gamma_C} S + U^T diag(e^{gamma_C-gamma}) K
-// Here every product is a tcgen05.mma with M = 128 issued by one thread, the
-// fp32 state S (d_v x d_k) lives in tensor memory for the whole sequence, and
-// the token dimension is put on N so that M is a head dimension:
+// Every product is a tcgen05.mma with M = 128 issued by one thread, the fp32
+// state S (d_v x d_k) lives in tensor memory for the whole sequence, and the
+// token dimension is put on N so that M is a head dimension:
 //     [K;Q] K^T  (K and Q rows stacked: one M = 128 product gives K K^T and Q K^T)
 //     W^T = K^T T1^T,  Ut^T = V^T T2^T,  U^T += S (-W)^T,  O^T = S Qg^T + U^T P^T,
 //     S  += (U diag(e^{gamma_C-gamma}))^T K.
@@ -18,6 +18,20 @@
 // and the conversions; T diag(beta) and U diag(...) enter the products that
 // feed the state as exact hi + lo bf16 pairs, and with split inputs k and v do
 // too (three-term products), exactly as in the mma.sync kernel.
+//
+// Two forms share these steps:
+//  * fused (gdn_tc_kernel): one CTA per (group, sequence, V head) runs every
+//    step of every chunk in order.  No scratch memory.
+//  * two-phase (gdn_prep_kernel, then gdn_seq_kernel): the gates, P, A, the
+//    solve, T2 and W of a chunk depend only on that chunk's q, k, g and beta,
+//    not on the state.  The prep kernel computes them for every (chunk, V
+//    head) at once (two CTAs per SM) and stores a 40 KB image per unit,
+//    [P | -W^T | T2 hi | T2 lo], in the operand layouts of the products that
+//    read it.  The sequential kernel then walks each sequence with only the
+//    state-dependent chain left per chunk:
+//        S -> bf16 and Qg;  O^T = S Qg^T,  U^T = V^T T2^T + S (-W)^T;
+//        U -> bf16;  S += (U diag)^T K,  O^T += U^T P^T;  o out,
+//    while the next chunk's tiles and image stream in behind each product.
 // Every mbarrier wait is bounded; a timeout records SR_DEV_TIMEOUT, drains the
 // MMAs, frees tensor memory and ends the CTA.
 #include <cuda.h>
@@ -35,24 +49,55 @@ using namespace tc;
 
 constexpr int C = 64, D = 128;
 constexpr int kThreads = 256;
-constexpr int ROWA = C + 4;  // fp32 row pitch of A and T in the solve
+constexpr int ROWA = C + 4;               // fp32 row pitch of A and T in the solve
+constexpr uint32_t SZ_AT = C * ROWA * 4;  // one fp32 64 x 64 matrix with padded rows
 
-// shared-memory layout (bytes from a 1024-aligned base)
+// input tiles (bytes from a 1024-aligned base) of the fused and the sequential kernels
 constexpr uint32_t OFF_KQ = 0;           // [K_j0][Q_j0][K_j1][Q_j1], 8 KB each
 constexpr uint32_t OFF_V = 32768;        // [V_i0][V_i1]
 constexpr uint32_t OFF_KL = 49152;       // [Kl_j0][Kl_j1]    (split)
 constexpr uint32_t OFF_VL = 65536;       // [Vl_i0][Vl_i1]    (split)
 constexpr uint32_t kIn[2] = {49152, 81920};  // end of the inputs (plain, split)
+
 constexpr uint32_t SZ_P = 8192;          // P   [t][s]
 constexpr uint32_t SZ_TR = 24576;        // T1, T2h, T2l [t][s]; later -W^T [j][t] (16 KB)
 constexpr uint32_t SZ_SB = 32768;        // S bf16 [i][j], two 64-column halves
 constexpr uint32_t SZ_QG = 16384;        // Qg [t][j], two halves
-constexpr uint32_t SZ_XR = 49152;        // A, T fp32 (2 x 17408); later Udh, Udl, Ub [i][t]
-constexpr uint32_t SZ_MISC = 2048;       // gamma, beta, column factors, barriers, TMEM address, flags
+constexpr uint32_t SZ_XR = 49152;        // fused: A, T fp32, later Udh, Udl, Ub [i][t]; sequential: U tiles
+constexpr uint32_t SZ_MISC = 2048;       // gates, column factors, barriers, TMEM address, flags
 
-constexpr uint32_t smem_bytes(bool split) {
+constexpr uint32_t smem_fused(bool split) {
     return kIn[split] + SZ_P + SZ_TR + SZ_SB + SZ_QG + SZ_XR + SZ_MISC + 1024 /* alignment */;
 }
+
+// Chunk image of the two-phase form, per (group, chunk slot, V head): bf16
+// tiles in the 128-byte swizzled layouts of the products that read them.
+constexpr uint32_t IMG_P = 0;        // P, K-major [t][s]
+constexpr uint32_t IMG_W = 8192;     // -W^T, MN-major [j][t] (16 KB)
+constexpr uint32_t IMG_T2H = 24576;  // T diag(beta), hi, K-major [t][s]
+constexpr uint32_t IMG_T2L = 32768;  // T diag(beta), lo
+constexpr uint32_t kImg = 40960;
+
+// prep kernel: K/Q (and Kl) tiles, then A and T fp32.  P and T2 hi reuse the
+// Q tiles once the first product has read them, T1 and T2 lo the A matrix
+// after the solve, -W^T the T matrix once T1 and T2 are formed.
+constexpr uint32_t kPrepIn[2] = {32768, 49152};
+constexpr uint32_t smem_prep(bool split) { return kPrepIn[split] + 2 * SZ_AT + SZ_MISC + 1024; }
+
+// sequential kernel: inputs, the chunk image, S bf16, Qg, the U tiles
+constexpr uint32_t smem_seq(bool split) { return kIn[split] + kImg + SZ_SB + SZ_QG + SZ_XR + SZ_MISC + 1024; }
+static_assert(smem_seq(true) <= 232448, "sequential kernel exceeds shared memory");
+static_assert(2 * (smem_prep(true) + 1024) <= 233472, "two prep CTAs must fit one SM");
+
+// Chunk c of the sequence n starting at token bos has the image slot
+// floor(bos / C) + n + c: distinct chunks get distinct slots, all below
+// floor(total / C) + n_seqs.
+__host__ __device__ inline int chunk_slot(int bos, int n, int c) { return bos / C + n + c; }
+
+constexpr uint32_t ID_KK = idesc_bf16_f32_major(128, 64, 0, 0);    // K-major A and B
+constexpr uint32_t ID_MN_K = idesc_bf16_f32_major(128, 64, 1, 0);  // MN-major A, K-major B
+constexpr uint32_t ID_K_MN = idesc_bf16_f32_major(128, 64, 0, 1);  // K-major A, MN-major B
+constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 0, 1);    // state update (N = 128)
 
 struct GdnTcParams {
     CUtensorMap q[kMaxGroups], k[kMaxGroups], v[kMaxGroups], kl[kMaxGroups], vl[kMaxGroups];
@@ -63,7 +108,8 @@ struct GdnTcParams {
     __nv_bfloat16 *o[kMaxGroups];
     float *s_out[kMaxGroups];
     const int32_t *cu;
-    int total, max_len, h_k, h_v;
+    uint8_t *img;  // two-phase: chunk images [group][slot][V head][kImg]
+    int total, max_len, h_k, h_v, n_seqs, slots;
     float scale;
     uint32_t *status;
 };
@@ -129,6 +175,455 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     lo = *reinterpret_cast<uint32_t *>(&l);
 }
 
+// ---------------------------------------------------------------- chunk steps
+// (every thread of the CTA calls each step; `row` = quad * 32 + lane is the
+// TMEM lane a thread reads, `half` = warp / 4 the column half it covers)
+
+// Warp 0: gam[0..63] <- its inclusive prefix sum.
+__device__ __forceinline__ void gate_prefix(float *gam, int lane) {
+    const float a0 = gam[2 * lane], a1 = gam[2 * lane + 1];
+    float incl = a0 + a1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const float excl = incl - (a0 + a1);
+    gam[2 * lane] = excl + a0;
+    gam[2 * lane + 1] = excl + a0 + a1;
+}
+
+// Descriptor of (addr + bytes) from the descriptor of addr.  The start-address
+// field holds addr >> 4, below 2^14 for every shared-memory address, so a byte
+// offset adds without a carry out of the field; the products below form each
+// operand's descriptor once and step it by constants.
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + uint64_t(bytes >> 4); }
+// The shared-memory base, re-read where a product group is issued so that its
+// descriptors live only there (kept out of the registers of the chunk loop).
+__device__ __forceinline__ uint32_t fresh(uint32_t base) {
+    uint32_t b;
+    asm volatile("mov.b32 %0, %1;" : "=r"(b) : "r"(base));
+    return b;
+}
+
+// [K;Q] K^T -> R0 (rows 0-63: K K^T, rows 64-127: Q K^T); with split k also
+// [K;Q] Kl^T into R0 and Kl K^T into R1 (rows 0-63).  One thread issues.
+template <bool SPLIT>
+__device__ __forceinline__ void mma_kqk(uint32_t base, uint32_t R0, uint32_t R1) {
+    base = fresh(base);
+    const uint64_t dk = sdesc_sw128(base + OFF_KQ, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint64_t a = dadd(dk, (k >> 2) * 16384 + (k & 3) * 32);
+        mma_bf16_ss(R0, a, a, ID_KK, k > 0);
+    }
+    if (SPLIT) {
+        const uint64_t dl = sdesc_sw128(base + OFF_KL, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint64_t a = dadd(dk, (k >> 2) * 16384 + (k & 3) * 32);
+            const uint64_t bl = dadd(dl, (k >> 2) * 8192 + (k & 3) * 32);
+            mma_bf16_ss(R0, a, bl, ID_KK, 1);
+            mma_bf16_ss(R1, bl, a, ID_KK, k > 0);
+        }
+    }
+}
+
+// A (fp32 [t][s] with row pitch ROWA) from K K^T and P (bf16 K-major tile [t][s]
+// at p_off) from Q K^T.  e^{gamma_t - gamma_s} = e^{gamma_t} e^{-gamma_s} while
+// e^{-gamma_C} stays far from the fp32 range (`fact`: gamma_C > -80); stronger
+// decay takes the exponential of each masked difference.
+template <bool SPLIT>
+__device__ __forceinline__ void build_a_p(uint8_t *sm, uint32_t p_off, float *Af, uint32_t R0, uint32_t R1,
+                                          uint32_t lane_off, int quad, int half, int row, const float *gam,
+                                          const float *bet, const float *fb, const float *eg, const float *ei,
+                                          bool fact, float scale) {
+    uint32_t r[32], r2[32];
+    tmem_ld_32x32b_x32(R0 + lane_off + 32 * half, r);
+    if (SPLIT && quad < 2) tmem_ld_32x32b_x32(R1 + lane_off + 32 * half, r2);
+    tmem_ld_wait();
+    if (quad < 2) {
+        const int t = row;
+        const float gt = gam[t], bt = bet[t], ft = fb[t];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+            float a4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = 32 * half + e + u;
+                float kk = __uint_as_float(r[e + u]);
+                if (SPLIT) kk += __uint_as_float(r2[e + u]);
+                const float d = fact ? ft * ei[s] : bt * __expf(gt - gam[s]);
+                a4[u] = (s < t) ? d * kk : 0.f;
+            }
+            *reinterpret_cast<float4 *>(&Af[t * ROWA + 32 * half + e]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        }
+    } else {
+        const int t = row - 64;
+        const float gt = gam[t], st = scale * eg[t];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = 32 * half + 8 * q4 + 2 * u;
+                float d0, d1;
+                if (fact) {
+                    d0 = s <= t ? st * ei[s] : 0.f;
+                    d1 = s + 1 <= t ? st * ei[s + 1] : 0.f;
+                } else {
+                    d0 = scale * __expf(s <= t ? gt - gam[s] : -INFINITY);
+                    d1 = scale * __expf(s + 1 <= t ? gt - gam[s + 1] : -INFINITY);
+                }
+                w[u] = pack2(d0 * __uint_as_float(r[8 * q4 + 2 * u]), d1 * __uint_as_float(r[8 * q4 + 2 * u + 1]));
+            }
+            *reinterpret_cast<uint4 *>(sm + p_off + sw128(t, 4 * half + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+// T = (I + A)^{-1} by 16x16 blocks (A strictly lower), into Tf:
+//   T_ii  = (I + A_ii)^{-1}, fp32 forward substitution by 8 x 8 halves
+//   B_ik  = T_ii A_ik (k < i), kept in the unused upper blocks of T
+//   T_ij  = -sum_{k=j}^{i-1} B_ik T_kj, in three rounds of independent products
+// The block products run on mma.sync with split bf16 operands (blk_mma).  Ends
+// with a block barrier.
+__device__ __forceinline__ void t_solve(float *Af, float *Tf, int tid, int warp, int lane) {
+    // T_ii by 8 x 8 halves: D = (I + N)^{-1} of each half by forward substitution,
+    // then the lower-left half -D2 (N21 D1) (its temporary N21 D1 sits in the
+    // unused upper-right half of the diagonal block of A)
+    if (tid < C) {
+        const int r0 = 8 * (tid >> 3), cc = tid & 7;
+        float x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const float4 *ar = reinterpret_cast<const float4 *>(&Af[(r0 + r) * ROWA + r0]);
+            const float4 f0 = ar[0], f1 = ar[1];
+            const float a[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-a[s2], x[s2], acc);
+            x[r] = (r < cc) ? 0.f : acc;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) Tf[(r0 + r) * ROWA + r0 + cc] = x[r];
+    }
+    __syncthreads();
+    {
+        const int b = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7, d0 = 16 * b;
+        float y = 0.f;  // (N21 D1)[r][cc]
+#pragma unroll
+        for (int m = 0; m < 8; ++m) y = fmaf(Af[(d0 + 8 + r) * ROWA + d0 + m], Tf[(d0 + m) * ROWA + d0 + cc], y);
+        Af[(d0 + r) * ROWA + d0 + 8 + cc] = y;
+        Tf[(d0 + r) * ROWA + d0 + 8 + cc] = 0.f;  // upper-right half of T_ii
+    }
+    __syncthreads();
+    {
+        const int b = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7, d0 = 16 * b;
+        float x = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) x = fmaf(Tf[(d0 + 8 + r) * ROWA + d0 + 8 + m], Af[(d0 + m) * ROWA + d0 + 8 + cc], x);
+        Tf[(d0 + 8 + r) * ROWA + d0 + cc] = -x;
+    }
+    __syncthreads();
+    auto blk = [](int bi, int bj) { return 16 * bi * ROWA + 16 * bj; };
+    {
+        // B_ik for (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2): warp w takes pair w
+        if (warp < 6) {
+            const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3), k = warp - i * (i - 1) / 2;
+            float acc[2][4] = {};
+            blk_mma(acc, Tf + blk(i, i), Af + blk(i, k), lane);
+            blk_store(Tf + blk(k, i), acc, lane, 1.f);  // kept in the upper block (k, i)
+        }
+    }
+    __syncthreads();
+    // T_ij = -sum_{k=j}^{i-1} B_ik T_kj in three rounds of independent products;
+    // the partial sums of T_20, T_31 and T_30 wait in their own blocks:
+    //   1: T_10, T_21, T_32 and the partials B_20 T_00, B_31 T_11, B_30 T_00
+    //   2: T_20, T_31 (partial + last term) and B_31 T_10 added to T_30's partial
+    //   3: T_30
+    // (B_ik is kept in the upper block (k, i))
+    if (warp < 6) {
+        // warps 0-2: (i, j) = (1,0) (2,1) (3,2); warps 3-5: (2,0) (3,1) (3,0)
+        const int i = warp < 3 ? warp + 1 : (warp == 3 ? 2 : 3);
+        const int j = warp < 3 ? warp : (warp == 4 ? 1 : 0);
+        float acc[2][4] = {};
+        blk_mma(acc, Tf + blk(j, i), Tf + blk(j, j), lane);  // B_ij T_jj
+        blk_store(Tf + blk(i, j), acc, lane, warp < 3 ? -1.f : 1.f);
+    }
+    __syncthreads();
+    if (warp < 3) {
+        // warp 0: T_20 = -(P_20 + B_21 T_10); warp 1: T_31 = -(P_31 + B_32 T_21);
+        // warp 2: P_30 += B_31 T_10
+        const int i = warp == 0 ? 2 : 3, j = warp == 1 ? 1 : 0, k = warp == 1 ? 2 : 1;
+        float acc[2][4];
+        blk_load(acc, Tf + blk(i, j), lane);
+        blk_mma(acc, Tf + blk(k, i), Tf + blk(k, j), lane);
+        blk_store(Tf + blk(i, j), acc, lane, warp < 2 ? -1.f : 1.f);
+    }
+    __syncthreads();
+    if (warp == 0) {  // T_30 = -(P_30 + B_32 T_20)
+        float acc[2][4];
+        blk_load(acc, Tf + blk(3, 0), lane);
+        blk_mma(acc, Tf + blk(2, 3), Tf + blk(2, 0), lane);
+        blk_store(Tf + blk(3, 0), acc, lane, -1.f);
+    }
+    __syncthreads();
+}
+
+// T1 = T diag(beta e^gamma) (bf16) and T2 = T diag(beta) (hi + lo) as K-major
+// tiles [t][s] at o1, o2h, o2l.  A thread always covers the same 8 columns, so
+// their factors stay in registers.
+__device__ __forceinline__ void write_t12(uint8_t *sm, const float *Tf, const float *bet, const float *fb,
+                                          uint32_t o1, uint32_t o2h, uint32_t o2l, int tid) {
+    const int ch = tid & 7;
+    float cb[8], cbe[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        cb[u] = bet[8 * ch + u];
+        cbe[u] = fb[8 * ch + u];
+    }
+    for (int t = tid >> 3; t < C; t += kThreads / 8) {
+        const float4 *tr = reinterpret_cast<const float4 *>(&Tf[t * ROWA + 8 * ch]);
+        const float4 ta = tr[0], tb = tr[1];
+        float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+        uint32_t w1[4], wh[4], wl[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s0 = 8 * ch + 2 * u;
+            const float t0 = (s0 <= t) ? tv[2 * u] : 0.f;
+            const float t1 = (s0 + 1 <= t) ? tv[2 * u + 1] : 0.f;
+            w1[u] = pack2(t0 * cbe[2 * u], t1 * cbe[2 * u + 1]);
+            split2(t0 * cb[2 * u], t1 * cb[2 * u + 1], wh[u], wl[u]);
+        }
+        const uint32_t off = sw128(t, ch);
+        *reinterpret_cast<uint4 *>(sm + o1 + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        *reinterpret_cast<uint4 *>(sm + o2h + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4 *>(sm + o2l + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+    }
+}
+
+// W^T = K^T T1^T -> RW (split: + Kl^T T1^T).  One thread issues.
+template <bool SPLIT>
+__device__ __forceinline__ void mma_w(uint32_t base, uint32_t o1, uint32_t RW) {
+    base = fresh(base);
+    const uint64_t dk = sdesc_sw128(base + OFF_KQ, 16384, 1024);  // K as MN-major A (j blocks 16 KB apart)
+    const uint64_t dl = sdesc_sw128(base + OFF_KL, 8192, 1024);
+    const uint64_t dt = sdesc_sw128(base + o1, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        mma_bf16_ss(RW, dadd(dk, k * 2048), dadd(dt, k * 32), ID_MN_K, k > 0);
+        if (SPLIT) mma_bf16_ss(RW, dadd(dl, k * 2048), dadd(dt, k * 32), ID_MN_K, 1);
+    }
+}
+
+// Ut^T = V^T T2^T -> RU from the hi and lo tiles of T2 (split: + Vl^T T2h^T).
+template <bool SPLIT>
+__device__ __forceinline__ void mma_ut(uint32_t base, uint32_t o2h, uint32_t o2l, uint32_t RU) {
+    base = fresh(base);
+    const uint64_t dv = sdesc_sw128(base + OFF_V, 8192, 1024);  // V as MN-major A (i blocks 8 KB apart)
+    const uint64_t dvl = sdesc_sw128(base + OFF_VL, 8192, 1024);
+    const uint64_t dh = sdesc_sw128(base + o2h, 16, 1024), dl = sdesc_sw128(base + o2l, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dh, k * 32), ID_MN_K, k > 0);
+        mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dl, k * 32), ID_MN_K, 1);
+        if (SPLIT) mma_bf16_ss(RU, dadd(dvl, k * 2048), dadd(dh, k * 32), ID_MN_K, 1);
+    }
+}
+
+// U^T += S (-W)^T -> RU, S bf16 at sb_off, -W^T (MN-major [j][t]) at w_off.
+__device__ __forceinline__ void mma_sw(uint32_t base, uint32_t sb_off, uint32_t w_off, uint32_t RU) {
+    base = fresh(base);
+    const uint64_t da = sdesc_sw128(base + sb_off, 16, 1024), db = sdesc_sw128(base + w_off, 8192, 1024);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_bf16_ss(RU, dadd(da, (k >> 2) * 16384 + (k & 3) * 32), dadd(db, k * 2048), ID_K_MN, 1);
+}
+
+// O^T = S Qg^T -> RO (the first product of the chunk's output).
+__device__ __forceinline__ void mma_sq(uint32_t base, uint32_t sb_off, uint32_t qg_off, uint32_t RO) {
+    base = fresh(base);
+    const uint64_t da = sdesc_sw128(base + sb_off, 16, 1024), db = sdesc_sw128(base + qg_off, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_bf16_ss(RO, dadd(da, (k >> 2) * 16384 + (k & 3) * 32), dadd(db, (k >> 2) * 8192 + (k & 3) * 32),
+                    ID_KK, k > 0);
+}
+
+// S += (U diag)^T K -> RS and O^T += U^T P^T -> RO, from the U tiles (Udh, Udl,
+// Ub) at xr_off and P at p_off.
+template <bool SPLIT>
+__device__ __forceinline__ void mma_update(uint32_t base, uint32_t xr_off, uint32_t p_off, uint32_t RS,
+                                           uint32_t RO) {
+    base = fresh(base);
+    const uint64_t dk = sdesc_sw128(base + OFF_KQ, 16384, 1024);  // K as MN-major B (j blocks 16 KB apart)
+    const uint64_t dkl = sdesc_sw128(base + OFF_KL, 8192, 1024);
+    const uint64_t du = sdesc_sw128(base + xr_off, 16, 1024), dp = sdesc_sw128(base + p_off, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        mma_bf16_ss(RS, dadd(du, k * 32), dadd(dk, k * 2048), ID_S, 1);
+        mma_bf16_ss(RS, dadd(du, 16384 + k * 32), dadd(dk, k * 2048), ID_S, 1);
+        if (SPLIT) mma_bf16_ss(RS, dadd(du, k * 32), dadd(dkl, k * 2048), ID_S, 1);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mma_bf16_ss(RO, dadd(du, 32768 + k * 32), dadd(dp, k * 32), ID_KK, 1);
+}
+
+// bf16 copy of S (TMEM RS, this thread's row and column half) into the K-major
+// tiles at sb_off (two 64-column halves 16 KB apart), then S <- fC S in TMEM.
+__device__ __forceinline__ void state_copy(uint8_t *sm, uint32_t sb_off, uint32_t RS, uint32_t lane_off, int half,
+                                           int row, float fC) {
+    uint32_t r[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        tmem_ld_32x32b_x32(RS + lane_off + 64 * half + 32 * part, r);
+        tmem_ld_wait();
+        uint8_t *sb = sm + sb_off + half * 16384;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w;
+            w.x = pack2(__uint_as_float(r[8 * q4 + 0]), __uint_as_float(r[8 * q4 + 1]));
+            w.y = pack2(__uint_as_float(r[8 * q4 + 2]), __uint_as_float(r[8 * q4 + 3]));
+            w.z = pack2(__uint_as_float(r[8 * q4 + 4]), __uint_as_float(r[8 * q4 + 5]));
+            w.w = pack2(__uint_as_float(r[8 * q4 + 6]), __uint_as_float(r[8 * q4 + 7]));
+            *reinterpret_cast<uint4 *>(sb + sw128(row, 4 * part + q4)) = w;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
+        tmem_st_32x32b_x32(RS + lane_off + 64 * half + 32 * part, r);
+    }
+    tmem_st_wait();
+}
+
+// Qg = scale e^{gamma_t} Q (same swizzled geometry as the Q tiles) at qg_off.
+__device__ __forceinline__ void build_qg(uint8_t *sm, uint32_t qg_off, const float *gam, float scale, int tid) {
+    for (int e = tid; e < 1024; e += kThreads) {
+        const int sub = e >> 9, t = (e >> 3) & 63, ch = e & 7;
+        const uint32_t off = sw128(t, ch);
+        const uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_KQ + 8192 + sub * 16384 + off);
+        const float f = scale * __expf(gam[t]);
+        const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        uint4 w;
+        uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 xf = __bfloat1622float2(x2[q2]);
+            wp[q2] = pack2(xf.x * f, xf.y * f);
+        }
+        *reinterpret_cast<uint4 *>(sm + qg_off + sub * 8192 + off) = w;
+    }
+}
+
+// -W^T (bf16) from TMEM RW as the MN-major B tile [j][t] at w_off.
+__device__ __forceinline__ void convert_w(uint8_t *sm, uint32_t w_off, uint32_t RW, uint32_t lane_off, int half,
+                                          int row) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(RW + lane_off + 32 * half, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        uint4 w;
+        w.x = pack2(-__uint_as_float(r[8 * q4 + 0]), -__uint_as_float(r[8 * q4 + 1]));
+        w.y = pack2(-__uint_as_float(r[8 * q4 + 2]), -__uint_as_float(r[8 * q4 + 3]));
+        w.z = pack2(-__uint_as_float(r[8 * q4 + 4]), -__uint_as_float(r[8 * q4 + 5]));
+        w.w = pack2(-__uint_as_float(r[8 * q4 + 6]), -__uint_as_float(r[8 * q4 + 7]));
+        *reinterpret_cast<uint4 *>(sm + w_off + sw128(row, 4 * half + q4)) = w;
+    }
+}
+
+// U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16) from TMEM RU as K-major
+// tiles [i][t] at xr_off, xr_off + 16 KB and xr_off + 32 KB.
+__device__ __forceinline__ void convert_u(uint8_t *sm, uint32_t xr_off, uint32_t RU, uint32_t lane_off, int half,
+                                          int row, const float *fu) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(RU + lane_off + 32 * half, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t wh[4], wl[4], wb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int t = 32 * half + 8 * q4 + 2 * u;
+            const float u0 = __uint_as_float(r[8 * q4 + 2 * u]), u1 = __uint_as_float(r[8 * q4 + 2 * u + 1]);
+            split2(u0 * fu[t], u1 * fu[t + 1], wh[u], wl[u]);
+            wb[u] = pack2(u0, u1);
+        }
+        const uint32_t off = sw128(row, 4 * half + q4);
+        *reinterpret_cast<uint4 *>(sm + xr_off + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4 *>(sm + xr_off + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        *reinterpret_cast<uint4 *>(sm + xr_off + 32768 + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    }
+}
+
+// o_t (bf16) from TMEM RO (lane = value channel i, columns = tokens).  A full
+// chunk is staged as a [t][i] tile (two 64-channel halves) at stage_off for one
+// TMA store; the ragged last chunk is stored element by element, so that no row
+// of the next sequence is touched.
+__device__ __forceinline__ void out_chunk(uint8_t *sm, uint32_t stage_off, uint32_t RO, uint32_t lane_off, int half,
+                                          int row, __nv_bfloat16 *o, size_t tok0, int clen, size_t v_stride, int h,
+                                          bool tile_store) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(RO + lane_off + 32 * half, r);
+    tmem_ld_wait();
+    if (tile_store) {
+        uint8_t *ot = sm + stage_off + (row >> 6) * 8192;
+        const uint32_t cofs = uint32_t(row & 7) * 2;
+        const uint32_t chunk = uint32_t(row & 63) >> 3;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(32 * half + e, chunk) + cofs) =
+                __float2bfloat16_rn(__uint_as_float(r[e]));
+        fence_async_smem();
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int t = 32 * half + e;
+            if (t < clen) o[(tok0 + t) * v_stride + size_t(h) * D + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
+        }
+    }
+}
+
+// Initial state (h0, or zero) into TMEM RS: thread -> row `row`, its column half.
+__device__ __forceinline__ void state_init(uint32_t RS, uint32_t lane_off, int half, int row, const float *h0,
+                                           size_t sbase) {
+    uint32_t r[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        const int j0 = 64 * half + 32 * part;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(h0 ? h0[sbase + size_t(row) * D + j0 + e] : 0.f);
+        tmem_st_32x32b_x32(RS + lane_off + j0, r);
+    }
+    tmem_st_wait();
+}
+
+// Final state TMEM RS -> s_out.
+__device__ __forceinline__ void state_out(uint32_t RS, uint32_t lane_off, int half, int row, float *s_out,
+                                          size_t sbase) {
+    uint32_t r[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        const int j0 = 64 * half + 32 * part;
+        tmem_ld_32x32b_x32(RS + lane_off + j0, r);
+        tmem_ld_wait();
+        float4 *dst = reinterpret_cast<float4 *>(s_out + sbase + size_t(row) * D + j0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                 __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+    }
+}
+
+// Copies h0 (or zeros) to s_out for an empty sequence.
+__device__ __forceinline__ void state_passthrough(const float *h0, float *s_out, size_t sbase, int tid) {
+    for (int e = tid; e < D * D / 4; e += kThreads) {
+        const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4 *>(s_out + sbase)[e] = v;
+    }
+}
+
+// ---------------------------------------------------------------- fused form
 template <bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -149,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *Af = reinterpret_cast<float *>(sm + oXR);
-    float *Tf = reinterpret_cast<float *>(sm + oXR + C * ROWA * 4);
+    float *Tf = reinterpret_cast<float *>(sm + oXR + SZ_AT);
 
     const int h = blockIdx.x, gi = blockIdx.z;
     const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + oXR));
@@ -167,10 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     float *s_out = p.s_out[gi];
 
     if (nchunks == 0) {  // empty sequence: the state is h0 (or zero)
-        for (int e = tid; e < D * D / 4; e += kThreads) {
-            const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-            reinterpret_cast<float4 *>(s_out + sbase)[e] = v;
-        }
+        state_passthrough(h0, s_out, sbase, tid);
         return;
     }
 
@@ -193,19 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const uint32_t R0 = tmem, R1 = tmem + 64, R2 = tmem + 128, R3 = tmem + 256;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    // ---- initial state into TMEM: thread -> row i = `row`, columns [64 half, 64 half + 64)
-    {
-        uint32_t r[32];
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int j0 = 64 * half + 32 * part;
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-                r[e] = __float_as_uint(h0 ? h0[sbase + size_t(row) * D + j0 + e] : 0.f);
-            tmem_st_32x32b_x32(R2 + lane_off + j0, r);
-        }
-        tmem_st_wait();
-    }
+    state_init(R2, lane_off, half, row, h0, sbase);
 
     const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const CUtensorMap *mo = &p.om[gi];
@@ -256,7 +736,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         g_next = gh[size_t(tid) * h_v];
         b_next = bh[size_t(tid) * h_v];
     }
-    bool ok = true;
 
     // wait for the next completion of the MMA barrier (all threads), then order TMEM reads
     auto wait_mma = [&]() -> bool {
@@ -270,11 +749,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (stop && tid == 0) *abort_flag = 1;
         return stop;
     };
-
-    constexpr uint32_t ID_KK = idesc_bf16_f32_major(128, 64, 0, 0);   // K-major A and B
-    constexpr uint32_t ID_MN_K = idesc_bf16_f32_major(128, 64, 1, 0); // MN-major A, K-major B
-    constexpr uint32_t ID_K_MN = idesc_bf16_f32_major(128, 64, 0, 1); // K-major A, MN-major B
-    constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 0, 1);   // state update (N = 128)
 
     for (int c = 0; c < nchunks; ++c) {
         const int clen = min(C, len - c * C);
@@ -290,18 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         kq_phase ^= 1;
         if (tid == 0) bulk_wait_read();  // the previous chunk's o tile has left the Qg region
         __syncthreads();
-        if (warp == 0) {
-            const float a0 = gam[2 * lane], a1 = gam[2 * lane + 1];
-            float incl = a0 + a1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            const float excl = incl - (a0 + a1);
-            gam[2 * lane] = excl + a0;
-            gam[2 * lane + 1] = excl + a0 + a1;
-        }
+        if (warp == 0) gate_prefix(gam, lane);
         if (check(tma_ok)) break;
         const float gC = gam[C - 1];
         if (tid < C) {  // per-column factors, read after later barriers
@@ -311,247 +774,34 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             eg[tid] = e;
             ei[tid] = __expf(-gam[tid]);
         }
-        // e^{gamma_t - gamma_s} = e^{gamma_t} e^{-gamma_s} while e^{-gamma_C} stays far from
-        // the fp32 range (gamma_C > -80); stronger decay takes the exponential of each
-        // masked difference
         const bool fact = gC > -80.f;
 
-        // ---- MMA 1: [K;Q] K^T -> R0 (rows 0-63: K K^T, rows 64-127: Q K^T)
+        // ---- MMA 1: [K;Q] K^T -> R0 (and R1)
         if (tid == 0) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t a = base + OFF_KQ + (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16_ss(R0, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_KK, k > 0);
-            }
-            if (SPLIT) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {  // [K;Q] Kl^T, and Kl K^T into R1 (rows 0-63)
-                    const uint32_t a = base + OFF_KQ + (k >> 2) * 16384 + (k & 3) * 32;
-                    const uint32_t bl = base + OFF_KL + (k >> 2) * 8192 + (k & 3) * 32;
-                    mma_bf16_ss(R0, sdesc_sw128(a, 16, 1024), sdesc_sw128(bl, 16, 1024), ID_KK, 1);
-                    mma_bf16_ss(R1, sdesc_sw128(bl, 16, 1024), sdesc_sw128(a, 16, 1024), ID_KK, k > 0);
-                }
-            }
+            mma_kqk<SPLIT>(base, R0, R1);
             mma_commit(bar_mma);
         }
-        // ---- meanwhile: bf16 copy of S (entering the chunk) and S <- e^{gamma_C} S in TMEM
-        {
-            const float fC = __expf(gC);
-            uint32_t r[32];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                tmem_ld_32x32b_x32(R2 + lane_off + 64 * half + 32 * part, r);
-                tmem_ld_wait();
-                uint8_t *sb = sm + oSB + half * 16384;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint4 w;
-                    w.x = pack2(__uint_as_float(r[8 * q4 + 0]), __uint_as_float(r[8 * q4 + 1]));
-                    w.y = pack2(__uint_as_float(r[8 * q4 + 2]), __uint_as_float(r[8 * q4 + 3]));
-                    w.z = pack2(__uint_as_float(r[8 * q4 + 4]), __uint_as_float(r[8 * q4 + 5]));
-                    w.w = pack2(__uint_as_float(r[8 * q4 + 6]), __uint_as_float(r[8 * q4 + 7]));
-                    *reinterpret_cast<uint4 *>(sb + sw128(row, 4 * part + q4)) = w;
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
-                tmem_st_32x32b_x32(R2 + lane_off + 64 * half + 32 * part, r);
-            }
-            tmem_st_wait();
-        }
-        // ---- Qg = scale e^{gamma_t} Q (same swizzled geometry as the Q tiles)
-        for (int e = tid; e < 1024; e += kThreads) {
-            const int sub = e >> 9, t = (e >> 3) & 63, ch = e & 7;
-            const uint32_t off = sw128(t, ch);
-            const uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_KQ + 8192 + sub * 16384 + off);
-            const float f = scale * __expf(gam[t]);
-            const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-            uint4 w;
-            uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-                const float2 xf = __bfloat1622float2(x2[q2]);
-                wp[q2] = pack2(xf.x * f, xf.y * f);
-            }
-            *reinterpret_cast<uint4 *>(sm + oQG + sub * 8192 + off) = w;
-        }
+        // ---- meanwhile: bf16 copy of S (entering the chunk), S <- e^{gamma_C} S, and Qg
+        state_copy(sm, oSB, R2, lane_off, half, row, __expf(gC));
+        build_qg(sm, oQG, gam, scale, tid);
         fence_async_smem();
         tc_fence_before();
         if (check(true)) break;
         // ---- O^T = S Qg^T -> R3 (issued now, completes with the next commit)
         if (tid == 0) {
             tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t a = base + oSB + (k >> 2) * 16384 + (k & 3) * 32;
-                const uint32_t b = base + oQG + (k >> 2) * 8192 + (k & 3) * 32;
-                mma_bf16_ss(R3, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 16, 1024), ID_KK, k > 0);
-            }
+            mma_sq(base, oSB, oQG, R3);
         }
         const bool m1 = wait_mma();  // MMA 1 done (the O^T product may still run)
 
         // ---- A (fp32, for the solve) from K K^T and P (bf16 tile) from Q K^T
-        {
-            uint32_t r[32], r2[32];
-            tmem_ld_32x32b_x32(R0 + lane_off + 32 * half, r);
-            if (SPLIT && quad < 2) tmem_ld_32x32b_x32(R1 + lane_off + 32 * half, r2);
-            tmem_ld_wait();
-            if (quad < 2) {
-                const int t = row;
-                const float gt = gam[t], bt = bet[t], ft = fb[t];
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    float a4[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int s = 32 * half + e + u;
-                        float kk = __uint_as_float(r[e + u]);
-                        if (SPLIT) kk += __uint_as_float(r2[e + u]);
-                        const float d = fact ? ft * ei[s] : bt * __expf(gt - gam[s]);
-                        a4[u] = (s < t) ? d * kk : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(&Af[t * ROWA + 32 * half + e]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-                }
-            } else {
-                const int t = row - 64;
-                const float gt = gam[t], st = scale * eg[t];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int s = 32 * half + 8 * q4 + 2 * u;
-                        float d0, d1;
-                        if (fact) {
-                            d0 = s <= t ? st * ei[s] : 0.f;
-                            d1 = s + 1 <= t ? st * ei[s + 1] : 0.f;
-                        } else {
-                            d0 = scale * __expf(s <= t ? gt - gam[s] : -INFINITY);
-                            d1 = scale * __expf(s + 1 <= t ? gt - gam[s + 1] : -INFINITY);
-                        }
-                        w[u] = pack2(d0 * __uint_as_float(r[8 * q4 + 2 * u]), d1 * __uint_as_float(r[8 * q4 + 2 * u + 1]));
-                    }
-                    *reinterpret_cast<uint4 *>(sm + oP + sw128(t, 4 * half + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-        }
+        build_a_p<SPLIT>(sm, oP, Af, R0, R1, lane_off, quad, half, row, gam, bet, fb, eg, ei, fact, scale);
         tc_fence_before();
         if (check(m1)) break;
         if (tid == 0 && c + 1 < nchunks) issue_q(c + 1);  // Q read by MMA 1 and the Qg copy only
 
-        // ---- T = (I + A)^{-1} by 16x16 blocks (A strictly lower):
-        //   T_ii  = (I + A_ii)^{-1}, fp32 forward substitution, one column per thread
-        //   B_ik  = T_ii A_ik (k < i), kept in the unused upper blocks of T
-        //   T_ij  = -sum_{k=j}^{i-1} B_ik T_kj, in three rounds of independent products
-        // The block products run on mma.sync with split bf16 operands (blk_mma).
-        // T_ii by 8 x 8 halves: D = (I + N)^{-1} of each half by forward substitution,
-        // then the lower-left half -D2 (N21 D1) (its temporary N21 D1 sits in the
-        // unused upper-right half of the diagonal block of A)
-        if (tid < C) {
-            const int r0 = 8 * (tid >> 3), cc = tid & 7;
-            float x[8];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const float4 *ar = reinterpret_cast<const float4 *>(&Af[(r0 + r) * ROWA + r0]);
-                const float4 f0 = ar[0], f1 = ar[1];
-                const float a[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-                float acc = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-                for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-a[s2], x[s2], acc);
-                x[r] = (r < cc) ? 0.f : acc;
-            }
-#pragma unroll
-            for (int r = 0; r < 8; ++r) Tf[(r0 + r) * ROWA + r0 + cc] = x[r];
-        }
-        __syncthreads();
-        {
-            const int b = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7, d0 = 16 * b;
-            float y = 0.f;  // (N21 D1)[r][cc]
-#pragma unroll
-            for (int m = 0; m < 8; ++m) y = fmaf(Af[(d0 + 8 + r) * ROWA + d0 + m], Tf[(d0 + m) * ROWA + d0 + cc], y);
-            Af[(d0 + r) * ROWA + d0 + 8 + cc] = y;
-            Tf[(d0 + r) * ROWA + d0 + 8 + cc] = 0.f;  // upper-right half of T_ii
-        }
-        __syncthreads();
-        {
-            const int b = tid >> 6, r = (tid >> 3) & 7, cc = tid & 7, d0 = 16 * b;
-            float x = 0.f;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) x = fmaf(Tf[(d0 + 8 + r) * ROWA + d0 + 8 + m], Af[(d0 + m) * ROWA + d0 + 8 + cc], x);
-            Tf[(d0 + 8 + r) * ROWA + d0 + cc] = -x;
-        }
-        __syncthreads();
-        auto blk = [](int bi, int bj) { return 16 * bi * ROWA + 16 * bj; };
-        {
-            // B_ik for (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2): warp w takes pair w
-            if (warp < 6) {
-                const int i = warp < 1 ? 1 : (warp < 3 ? 2 : 3), k = warp - i * (i - 1) / 2;
-                float acc[2][4] = {};
-                blk_mma(acc, Tf + blk(i, i), Af + blk(i, k), lane);
-                blk_store(Tf + blk(k, i), acc, lane, 1.f);  // kept in the upper block (k, i)
-            }
-        }
-        __syncthreads();
-        // T_ij = -sum_{k=j}^{i-1} B_ik T_kj in three rounds of independent products;
-        // the partial sums of T_20, T_31 and T_30 wait in their own blocks:
-        //   1: T_10, T_21, T_32 and the partials B_20 T_00, B_31 T_11, B_30 T_00
-        //   2: T_20, T_31 (partial + last term) and B_31 T_10 added to T_30's partial
-        //   3: T_30
-        // (B_ik is kept in the upper block (k, i))
-        if (warp < 6) {
-            // warps 0-2: (i, j) = (1,0) (2,1) (3,2); warps 3-5: (2,0) (3,1) (3,0)
-            const int i = warp < 3 ? warp + 1 : (warp == 3 ? 2 : 3);
-            const int j = warp < 3 ? warp : (warp == 4 ? 1 : 0);
-            float acc[2][4] = {};
-            blk_mma(acc, Tf + blk(j, i), Tf + blk(j, j), lane);  // B_ij T_jj
-            blk_store(Tf + blk(i, j), acc, lane, warp < 3 ? -1.f : 1.f);
-        }
-        __syncthreads();
-        if (warp < 3) {
-            // warp 0: T_20 = -(P_20 + B_21 T_10); warp 1: T_31 = -(P_31 + B_32 T_21);
-            // warp 2: P_30 += B_31 T_10
-            const int i = warp == 0 ? 2 : 3, j = warp == 1 ? 1 : 0, k = warp == 1 ? 2 : 1;
-            float acc[2][4];
-            blk_load(acc, Tf + blk(i, j), lane);
-            blk_mma(acc, Tf + blk(k, i), Tf + blk(k, j), lane);
-            blk_store(Tf + blk(i, j), acc, lane, warp < 2 ? -1.f : 1.f);
-        }
-        __syncthreads();
-        if (warp == 0) {  // T_30 = -(P_30 + B_32 T_20)
-            float acc[2][4];
-            blk_load(acc, Tf + blk(3, 0), lane);
-            blk_mma(acc, Tf + blk(2, 3), Tf + blk(2, 0), lane);
-            blk_store(Tf + blk(3, 0), acc, lane, -1.f);
-        }
-        __syncthreads();
-        // T1 = T diag(beta e^gamma) (bf16), T2 = T diag(beta) (hi + lo): K-major tiles [t][s].
-        // A thread always covers the same 8 columns, so their factors stay in registers.
-        {
-            const int ch = tid & 7;
-            float cb[8], cbe[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                cb[u] = bet[8 * ch + u];
-                cbe[u] = fb[8 * ch + u];
-            }
-            for (int t = tid >> 3; t < C; t += kThreads / 8) {
-                const float4 *tr = reinterpret_cast<const float4 *>(&Tf[t * ROWA + 8 * ch]);
-                const float4 ta = tr[0], tb = tr[1];
-                float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-                uint32_t w1[4], wh[4], wl[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int s0 = 8 * ch + 2 * u;
-                    const float t0 = (s0 <= t) ? tv[2 * u] : 0.f;
-                    const float t1 = (s0 + 1 <= t) ? tv[2 * u + 1] : 0.f;
-                    w1[u] = pack2(t0 * cbe[2 * u], t1 * cbe[2 * u + 1]);
-                    split2(t0 * cb[2 * u], t1 * cb[2 * u + 1], wh[u], wl[u]);
-                }
-                const uint32_t off = sw128(t, ch);
-                *reinterpret_cast<uint4 *>(sm + oTR + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-                *reinterpret_cast<uint4 *>(sm + oTR + 8192 + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                *reinterpret_cast<uint4 *>(sm + oTR + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-            }
-        }
+        t_solve(Af, Tf, tid, warp, lane);
+        write_t12(sm, Tf, bet, fb, oTR, oTR + 8192, oTR + 16384, tid);
         fence_async_smem();
         tc_fence_before();
         if (check(true)) break;
@@ -560,45 +810,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         if (tid == 0) {
             if (!mbar_wait(bar_v, v_phase)) *abort_flag = 1;
             tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t kmn = base + OFF_KQ + k * 2048;  // K as MN-major A (j blocks 16 KB apart)
-                const uint32_t t1 = base + oTR + k * 32;
-                mma_bf16_ss(R1, sdesc_sw128(kmn, 16384, 1024), sdesc_sw128(t1, 16, 1024), ID_MN_K, k > 0);
-                if (SPLIT)
-                    mma_bf16_ss(R1, sdesc_sw128(base + OFF_KL + k * 2048, 8192, 1024), sdesc_sw128(t1, 16, 1024),
-                                ID_MN_K, 1);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t vmn = base + OFF_V + k * 2048;   // V as MN-major A (i blocks 8 KB apart)
-                const uint32_t t2h = base + oTR + 8192 + k * 32, t2l = base + oTR + 16384 + k * 32;
-                mma_bf16_ss(R0, sdesc_sw128(vmn, 8192, 1024), sdesc_sw128(t2h, 16, 1024), ID_MN_K, k > 0);
-                mma_bf16_ss(R0, sdesc_sw128(vmn, 8192, 1024), sdesc_sw128(t2l, 16, 1024), ID_MN_K, 1);
-                if (SPLIT)
-                    mma_bf16_ss(R0, sdesc_sw128(base + OFF_VL + k * 2048, 8192, 1024), sdesc_sw128(t2h, 16, 1024),
-                                ID_MN_K, 1);
-            }
+            mma_w<SPLIT>(base, oTR, R1);
+            mma_ut<SPLIT>(base, oTR + 8192, oTR + 16384, R0);
             mma_commit(bar_mma);
         }
         v_phase ^= 1;
         const bool m2 = wait_mma() && *abort_flag == 0;
 
         // ---- -W^T (bf16) as the MN-major B tile [j][t] of the next product
-        {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(R1 + lane_off + 32 * half, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint4 w;
-                w.x = pack2(-__uint_as_float(r[8 * q4 + 0]), -__uint_as_float(r[8 * q4 + 1]));
-                w.y = pack2(-__uint_as_float(r[8 * q4 + 2]), -__uint_as_float(r[8 * q4 + 3]));
-                w.z = pack2(-__uint_as_float(r[8 * q4 + 4]), -__uint_as_float(r[8 * q4 + 5]));
-                w.w = pack2(-__uint_as_float(r[8 * q4 + 6]), -__uint_as_float(r[8 * q4 + 7]));
-                *reinterpret_cast<uint4 *>(sm + oTR + sw128(row, 4 * half + q4)) = w;
-            }
-        }
+        convert_w(sm, oTR, R1, lane_off, half, row);
         fence_async_smem();
         tc_fence_before();
         if (check(m2)) break;
@@ -607,37 +827,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         // ---- MMA 3: U^T = Ut^T + S (-W)^T -> R0
         if (tid == 0) {
             tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t a = base + oSB + (k >> 2) * 16384 + (k & 3) * 32;
-                const uint32_t b = base + oTR + k * 2048;
-                mma_bf16_ss(R0, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 8192, 1024), ID_K_MN, 1);
-            }
+            mma_sw(base, oSB, oTR, R0);
             mma_commit(bar_mma);
         }
         const bool m3 = wait_mma();
 
         // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16): K-major tiles [i][t]
-        {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(R0 + lane_off + 32 * half, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t wh[4], wl[4], wb[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int t = 32 * half + 8 * q4 + 2 * u;
-                    const float u0 = __uint_as_float(r[8 * q4 + 2 * u]), u1 = __uint_as_float(r[8 * q4 + 2 * u + 1]);
-                    split2(u0 * fu[t], u1 * fu[t + 1], wh[u], wl[u]);
-                    wb[u] = pack2(u0, u1);
-                }
-                const uint32_t off = sw128(row, 4 * half + q4);
-                *reinterpret_cast<uint4 *>(sm + oXR + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                *reinterpret_cast<uint4 *>(sm + oXR + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                *reinterpret_cast<uint4 *>(sm + oXR + 32768 + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-            }
-        }
+        convert_u(sm, oXR, R0, lane_off, half, row, fu);
         fence_async_smem();
         tc_fence_before();
         if (check(m3)) break;
@@ -645,21 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         // ---- MMA 4: S += (U diag)^T K -> R2 ; O^T += U^T P^T -> R3
         if (tid == 0) {
             tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t kmn = base + OFF_KQ + k * 2048;  // K as MN-major B (j blocks 16 KB apart)
-                const uint32_t uh = base + oXR + k * 32, ul = base + oXR + 16384 + k * 32;
-                mma_bf16_ss(R2, sdesc_sw128(uh, 16, 1024), sdesc_sw128(kmn, 16384, 1024), ID_S, 1);
-                mma_bf16_ss(R2, sdesc_sw128(ul, 16, 1024), sdesc_sw128(kmn, 16384, 1024), ID_S, 1);
-                if (SPLIT)
-                    mma_bf16_ss(R2, sdesc_sw128(uh, 16, 1024), sdesc_sw128(base + OFF_KL + k * 2048, 8192, 1024),
-                                ID_S, 1);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t ub = base + oXR + 32768 + k * 32, pb = base + oP + k * 32;
-                mma_bf16_ss(R3, sdesc_sw128(ub, 16, 1024), sdesc_sw128(pb, 16, 1024), ID_KK, 1);
-            }
+            mma_update<SPLIT>(base, oXR, oP, R2, R3);
             mma_commit(bar_mma);
         }
         const bool m4 = wait_mma();
@@ -667,34 +849,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         // K is free now: fetch the next chunk's while O is written out
         if (tid == 0 && c + 1 < nchunks) issue_k(c + 1);
 
-        // ---- o_t (bf16): thread = value channel i, 32 tokens.  A full chunk goes
-        // through the (now free) Qg region as a [t][i] tile and one TMA store; the
-        // ragged last chunk is stored element by element, so that no row of the
-        // next sequence is touched.
+        // ---- o_t (bf16) through the (now free) Qg region
         const bool tile_store = o != nullptr && clen == C;
-        if (o) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(R3 + lane_off + 32 * half, r);
-            tmem_ld_wait();
-            if (tile_store) {
-                uint8_t *ot = sm + oQG + (row >> 6) * 8192;
-                const uint32_t cofs = uint32_t(row & 7) * 2;
-                const uint32_t chunk = uint32_t(row & 63) >> 3;
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    *reinterpret_cast<__nv_bfloat16 *>(ot + sw128(32 * half + e, chunk) + cofs) =
-                        __float2bfloat16_rn(__uint_as_float(r[e]));
-                fence_async_smem();
-            } else {
-                const size_t tok0 = size_t(bos) + size_t(c) * C;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = 32 * half + e;
-                    if (t < clen)
-                        o[(tok0 + t) * v_stride + size_t(h) * D + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
-                }
-            }
-        }
+        if (o) out_chunk(sm, oQG, R3, lane_off, half, row, o, size_t(bos) + size_t(c) * C, clen, v_stride, h, tile_store);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -707,24 +864,412 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     if (tid == 0) bulk_wait_all();
 
     __syncthreads();
-    ok = *abort_flag == 0;
-    if (ok) {
-        // ---- final state: TMEM -> s_out
-        uint32_t r[32];
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int j0 = 64 * half + 32 * part;
-            tmem_ld_32x32b_x32(R2 + lane_off + j0, r);
-            tmem_ld_wait();
-            float4 *dst = reinterpret_cast<float4 *>(s_out + sbase + size_t(row) * D + j0);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                     __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
-        }
+    if (*abort_flag == 0) {
+        state_out(R2, lane_off, half, row, s_out, sbase);
     } else if (tid == 0) {
         atomicOr(p.status, SR_DEV_TIMEOUT);
         // let in-flight MMAs and TMA copies finish before tensor memory and shared memory are released
+        mma_commit(bar_mma);
+        mbar_wait(bar_mma, mma_phase);
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- two-phase form: prep
+// One CTA per (chunk slot, V head, group).  Slots between two sequences' chunks
+// (at most one per sequence) exit at once.
+template <bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(sm);
+    constexpr uint32_t oXR = kPrepIn[SPLIT], oMISC = oXR + 2 * SZ_AT;
+    constexpr uint32_t oP = OFF_KQ + 8192, oT2H = OFF_KQ + 24576;  // the Q tiles
+    constexpr uint32_t oT1 = oXR, oT2L = oXR + 8192;                // A
+    constexpr uint32_t oW = oXR + SZ_AT;                            // T
+    float *Af = reinterpret_cast<float *>(sm + oXR);
+    float *Tf = reinterpret_cast<float *>(sm + oXR + SZ_AT);
+    float *gam = reinterpret_cast<float *>(sm + oMISC);  // [64]
+    float *bet = gam + C;                                 // [64]
+    float *fb = gam + 2 * C;                              // [64] beta_s e^{gamma_s}
+    float *eg = gam + 3 * C;                              // [64] e^{gamma_t}
+    float *ei = gam + 4 * C;                              // [64] e^{-gamma_t}
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + oMISC + 1280);
+    uint64_t *bar_mma = bar_in + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+
+    const int slot = blockIdx.x, h = blockIdx.y, gi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+
+    // the sequence holding this slot: the largest n with floor(cu[n] / C) + n <= slot
+    int lo = 0, hi = p.n_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cu[mid] / C + mid <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    const int n = lo;
+    int bos, eos;
+    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
+    const int len = eos - bos, c = slot - (bos / C + n);
+    if (c < 0 || c * C >= len) return;
+    const int clen = min(C, len - c * C), y = bos + c * C;
+    const int hk = h / (p.h_v / p.h_k);
+
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot, R0 = tmem, R1 = tmem + 64;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    if (tid == 0) {
+        const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mkl = &p.kl[gi];
+        mbar_arrive_expect_tx(bar_in, SPLIT ? 49152u : 32768u);
+        tma_load_2d(sm + OFF_KQ, mk, bar_in, hk * D, y);
+        tma_load_2d(sm + OFF_KQ + 16384, mk, bar_in, hk * D + 64, y);
+        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_in, hk * D, y);
+        tma_load_2d(sm + OFF_KQ + 24576, mq, bar_in, hk * D + 64, y);
+        if (SPLIT) {
+            tma_load_2d(sm + OFF_KL, mkl, bar_in, hk * D, y);
+            tma_load_2d(sm + OFF_KL + 8192, mkl, bar_in, hk * D + 64, y);
+        }
+    }
+    // gates: gamma = inclusive prefix sum of g; padding has g = beta = 0
+    if (tid < C) {
+        const bool in = tid < clen;
+        gam[tid] = in ? p.g[gi][size_t(y + tid) * p.h_v + h] : 0.f;
+        bet[tid] = in ? p.beta[gi][size_t(y + tid) * p.h_v + h] : 0.f;
+    }
+    __syncthreads();
+    if (warp == 0) gate_prefix(gam, lane);
+    __syncthreads();
+    const float gC = gam[C - 1];
+    if (tid < C) {
+        const float e = __expf(gam[tid]);
+        fb[tid] = bet[tid] * e;
+        eg[tid] = e;
+        ei[tid] = __expf(-gam[tid]);
+    }
+    const bool fact = gC > -80.f;
+    uint32_t mma_phase = 0;
+    bool ok = __syncthreads_and(mbar_wait(bar_in, 0)) != 0;
+
+    if (ok) {
+        // ---- [K;Q] K^T, then A and P
+        if (tid == 0) {
+            tc_fence_after();
+            mma_kqk<SPLIT>(base, R0, R1);
+            mma_commit(bar_mma);
+        }
+        const bool w = mbar_wait(bar_mma, mma_phase);
+        mma_phase ^= 1;
+        tc_fence_after();
+        build_a_p<SPLIT>(sm, oP, Af, R0, R1, lane_off, quad, half, row, gam, bet, fb, eg, ei, fact, p.scale);
+        tc_fence_before();
+        ok = __syncthreads_and(w) != 0;
+    }
+    if (ok) {
+        // ---- the solve, T1 and T2, then W^T = K^T T1^T and -W^T
+        t_solve(Af, Tf, tid, warp, lane);
+        write_t12(sm, Tf, bet, fb, oT1, oT2H, oT2L, tid);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            mma_w<SPLIT>(base, oT1, R0);
+            mma_commit(bar_mma);
+        }
+        const bool w = mbar_wait(bar_mma, mma_phase);
+        mma_phase ^= 1;
+        tc_fence_after();
+        convert_w(sm, oW, R0, lane_off, half, row);
+        fence_async_smem();
+        ok = __syncthreads_and(w) != 0;
+    }
+    if (ok) {
+        if (tid == 0) {
+            uint8_t *dst = p.img + ((size_t(gi) * p.slots + slot) * p.h_v + h) * kImg;
+            bulk_store(dst + IMG_P, sm + oP, 8192);
+            bulk_store(dst + IMG_W, sm + oW, 16384);
+            bulk_store(dst + IMG_T2H, sm + oT2H, 8192);
+            bulk_store(dst + IMG_T2L, sm + oT2L, 8192);
+            bulk_commit();
+            bulk_wait_all();
+        }
+    } else if (tid == 0) {
+        atomicOr(p.status, SR_DEV_TIMEOUT);
+        mma_commit(bar_mma);
+        mbar_wait(bar_mma, mma_phase);
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// ---------------------------------------------------------------- two-phase form: sequential
+// o_t (bf16) of one chunk straight from TMEM RO to global memory: a warp stores
+// one token's 32 consecutive value channels per instruction (64 contiguous bytes).
+__device__ __forceinline__ void out_direct(uint32_t RO, uint32_t lane_off, int half, int row, __nv_bfloat16 *o,
+                                           size_t tok0, int clen, size_t v_stride, int h) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(RO + lane_off + 32 * half, r);
+    tmem_ld_wait();
+    __nv_bfloat16 *dst = o + (tok0 + size_t(32 * half)) * v_stride + size_t(h) * D + row;
+    const int n_out = min(32, clen - 32 * half);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        if (e < n_out) *dst = __float2bfloat16_rn(__uint_as_float(r[e]));
+        dst += v_stride;
+    }
+}
+
+// One CTA per (V head, sequence rank, group).  Per chunk c the state chain is
+//   S(c) -> bf16;  [O(c) = S Qg^T,  U^T = V^T T2^T + S (-W)^T];  U -> bf16;
+//   [S += (U diag)^T K,  O(c) += U^T P^T]
+// and the work that feeds only the output or the next chunk runs beside the
+// products: o of chunk c-1 is written while the first group of products of c
+// runs (O alternates between two TMEM accumulators), and the gates and Qg of
+// chunk c+1 are formed while the state update of c runs.
+template <bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_constant__ GdnTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(sm);
+    constexpr uint32_t oIMG = kIn[SPLIT], oSB = oIMG + kImg, oQG = oSB + SZ_SB, oXR = oQG + SZ_QG;
+    constexpr uint32_t oMISC = oXR + SZ_XR;
+    float *gam = reinterpret_cast<float *>(sm + oMISC);  // [64]
+    float *fu = gam + C;                                  // [64] e^{gamma_C - gamma_t}
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 1024);  // K (+ k low part) landed
+    uint64_t *bar_q = bar_k + 1;                                          // Q landed
+    uint64_t *bar_v = bar_k + 2;                                          // V (+ v low part) landed
+    uint64_t *bar_w = bar_k + 3;                                          // -W^T and T2 landed
+    uint64_t *bar_p = bar_k + 4;                                          // P landed
+    uint64_t *bar_mma = bar_k + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int h = blockIdx.x, gi = blockIdx.z;
+    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + oXR));
+    const int h_k = p.h_k, h_v = p.h_v;
+    const int hk = h / (h_v / h_k);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    int bos, eos;
+    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
+    const int len = eos - bos;
+    const int nchunks = (len + C - 1) / C;
+    const size_t sbase = (size_t(n) * h_v + h) * D * D;
+    const float *h0 = p.h0[gi];
+    float *s_out = p.s_out[gi];
+
+    if (nchunks == 0) {
+        state_passthrough(h0, s_out, sbase, tid);
+        return;
+    }
+
+    if (tid == 0) {
+        mbar_init(bar_k, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_w, 1);
+        mbar_init(bar_p, 1);
+        mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t RU = tmem, RS = tmem + 128, RO0 = tmem + 256, RO1 = tmem + 320;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+
+    state_init(RS, lane_off, half, row, h0, sbase);
+
+    const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
+    const uint8_t *img = p.img + (size_t(gi) * p.slots * h_v + h) * kImg;
+    auto img_of = [&](int c) { return img + size_t(chunk_slot(bos, n, c)) * h_v * kImg; };
+    // Each input is refilled as soon as the last reader of its buffer is done:
+    // Q once Qg is formed, V, T2 and -W^T once U is, K and P after the update.
+    auto issue_k = [&](int c) {
+        const int y = bos + c * C;
+        mbar_arrive_expect_tx(bar_k, SPLIT ? 32768u : 16384u);
+        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * D, y);
+        tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * D + 64, y);
+        if (SPLIT) {
+            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * D, y);
+            tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * D + 64, y);
+        }
+    };
+    auto issue_q = [&](int c) {
+        const int y = bos + c * C;
+        mbar_arrive_expect_tx(bar_q, 16384u);
+        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * D, y);
+        tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * D + 64, y);
+    };
+    auto issue_v = [&](int c) {
+        const int y = bos + c * C;
+        mbar_arrive_expect_tx(bar_v, SPLIT ? 32768u : 16384u);
+        tma_load_2d(sm + OFF_V, mv, bar_v, h * D, y);
+        tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * D + 64, y);
+        if (SPLIT) {
+            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * D, y);
+            tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * D + 64, y);
+        }
+    };
+    auto issue_w = [&](int c) {  // -W^T, T2 hi, T2 lo
+        mbar_arrive_expect_tx(bar_w, kImg - IMG_W);
+        bulk_load(sm + oIMG + IMG_W, img_of(c) + IMG_W, kImg - IMG_W, bar_w);
+    };
+    auto issue_p = [&](int c) {
+        mbar_arrive_expect_tx(bar_p, IMG_W - IMG_P);
+        bulk_load(sm + oIMG + IMG_P, img_of(c) + IMG_P, IMG_W - IMG_P, bar_p);
+    };
+    if (tid == 0) {
+        prefetch_tmap(mq); prefetch_tmap(mk); prefetch_tmap(mv);
+        if (SPLIT) { prefetch_tmap(mkl); prefetch_tmap(mvl); }
+        issue_q(0);
+        issue_k(0);
+        issue_v(0);
+        issue_w(0);
+        issue_p(0);
+    }
+
+    const float *gh = p.g[gi] + size_t(bos) * h_v + h;
+    __nv_bfloat16 *o = p.o[gi];
+    const size_t v_stride = size_t(h_v) * D;
+    const float scale = p.scale;
+    uint32_t k_phase = 0, q_phase = 0, v_phase = 0, w_phase = 0, p_phase = 0, mma_phase = 0;
+
+    auto wait_mma = [&]() -> bool {
+        const bool w = mbar_wait(bar_mma, mma_phase);
+        mma_phase ^= 1;
+        tc_fence_after();
+        return w;
+    };
+    auto check = [&](bool w) -> bool {
+        const bool stop = __syncthreads_or(!w) != 0;
+        if (stop && tid == 0) *abort_flag = 1;
+        return stop;
+    };
+    // gates of chunk c in gam (gamma = inclusive prefix sum of g; padding has g = 0),
+    // fu, and Qg = scale e^{gamma_t} Q once Q has landed; false when a wait failed
+    float g_next = 0.f;  // g of the next chunk (threads tid < C)
+    auto next_gates_and_qg = [&](int c) -> bool {
+        if (tid < C) {
+            gam[tid] = g_next;
+            const int t = (c + 1) * C + tid;
+            g_next = t < len ? gh[size_t(t) * h_v] : 0.f;
+        }
+        const bool qok = mbar_wait(bar_q, q_phase);
+        q_phase ^= 1;
+        __syncthreads();
+        if (warp == 0) gate_prefix(gam, lane);
+        if (check(qok)) return false;
+        if (tid < C) fu[tid] = __expf(gam[C - 1] - gam[tid]);  // read after later barriers
+        build_qg(sm, oQG, gam, scale, tid);
+        fence_async_smem();
+        return true;
+    };
+
+    if (tid < C && tid < len) g_next = gh[size_t(tid) * h_v];
+    bool ok = next_gates_and_qg(0);
+    ok = ok && !check(true);
+    if (ok && tid == 0 && nchunks > 1) issue_q(1);
+
+    int c = 0;
+    for (; ok && c < nchunks; ++c) {
+        const uint32_t RO = (c & 1) ? RO1 : RO0, RO_prev = (c & 1) ? RO0 : RO1;
+        // ---- bf16 copy of S (entering the chunk), then S <- e^{gamma_C} S
+        state_copy(sm, oSB, RS, lane_off, half, row, __expf(gam[C - 1]));
+        fence_async_smem();
+        tc_fence_before();
+        if (check(true)) break;
+
+        // ---- O(c) = S Qg^T ;  U^T = V^T T2^T + S (-W)^T
+        if (tid == 0) {
+            const bool w = mbar_wait(bar_v, v_phase) && mbar_wait(bar_w, w_phase);
+            if (!w) *abort_flag = 1;
+            tc_fence_after();
+            mma_sq(base, oSB, oQG, RO);
+            mma_ut<SPLIT>(base, oIMG + IMG_T2H, oIMG + IMG_T2L, RU);
+            mma_sw(base, oSB, oIMG + IMG_W, RU);
+            mma_commit(bar_mma);
+        }
+        v_phase ^= 1;
+        w_phase ^= 1;
+        // ---- meanwhile: o of the previous chunk
+        if (o && c > 0) out_direct(RO_prev, lane_off, half, row, o, size_t(bos) + size_t(c - 1) * C, C, v_stride, h);
+        const bool m2 = wait_mma() && *abort_flag == 0;
+        if (check(m2)) break;
+        if (tid == 0 && c + 1 < nchunks) {
+            issue_v(c + 1);
+            issue_w(c + 1);
+        }
+
+        // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16): K-major tiles [i][t]
+        convert_u(sm, oXR, RU, lane_off, half, row, fu);
+        fence_async_smem();
+        tc_fence_before();
+        if (check(true)) break;
+
+        // ---- S += (U diag)^T K ;  O(c) += U^T P^T
+        if (tid == 0) {
+            const bool w = mbar_wait(bar_k, k_phase) && mbar_wait(bar_p, p_phase);
+            if (!w) *abort_flag = 1;
+            tc_fence_after();
+            mma_update<SPLIT>(base, oXR, oIMG + IMG_P, RS, RO);
+            mma_commit(bar_mma);
+        }
+        k_phase ^= 1;
+        p_phase ^= 1;
+        // ---- meanwhile: gates and Qg of the next chunk (the Qg region was last read
+        // by the first product group, complete at the previous wait)
+        bool nok = true;
+        if (c + 1 < nchunks) nok = next_gates_and_qg(c + 1);
+        const bool m4 = wait_mma() && *abort_flag == 0 && nok;
+        if (check(m4)) break;
+        if (tid == 0 && c + 1 < nchunks) {
+            issue_k(c + 1);
+            issue_p(c + 1);
+            if (c + 2 < nchunks) issue_q(c + 2);
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag == 0) {
+        const int cl = nchunks - 1;
+        if (o) out_direct(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C, len - cl * C,
+                          v_stride, h);
+        state_out(RS, lane_off, half, row, s_out, sbase);
+    } else if (tid == 0) {
+        atomicOr(p.status, SR_DEV_TIMEOUT);
         mma_commit(bar_mma);
         mbar_wait(bar_mma, mma_phase);
         for (int i = 0; i < 64; ++i) __nanosleep(1000);
@@ -744,20 +1289,37 @@ bool map_64x64(CUtensorMap *m, const void *base, int rows, int cols) {
 
 template <bool SPLIT>
 cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t st) {
-    const int smem = int(smem_bytes(SPLIT));
-    cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (!p.img) {
+        const int smem = int(smem_fused(SPLIT));
+        cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        gdn_tc_kernel<SPLIT><<<dim3(p.h_v, n_seqs, n_groups), kThreads, smem, st>>>(p);
+        return cudaGetLastError();
+    }
+    const int s1 = int(smem_prep(SPLIT)), s2 = int(smem_seq(SPLIT));
+    cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.h_v, n_seqs, n_groups);
-    gdn_tc_kernel<SPLIT><<<grid, kThreads, smem, st>>>(p);
+    e = cudaFuncSetAttribute(gdn_seq_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
+    if (e != cudaSuccess) return e;
+    gdn_prep_kernel<SPLIT><<<dim3(p.slots, p.h_v, n_groups), kThreads, s1, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    gdn_seq_kernel<SPLIT><<<dim3(p.h_v, n_seqs, n_groups), kThreads, s2, st>>>(p);
     return cudaGetLastError();
 }
+
+int image_slots(int total, int n_seqs) { return total / C + n_seqs; }
 
 }  // namespace
 
 bool gdn_tc_supported(int d) { return d == 128; }
 
+size_t gdn_tc_image_bytes(int total, int n_seqs, int h_v, int n_groups) {
+    return size_t(n_groups) * size_t(image_slots(total, n_seqs)) * size_t(h_v) * kImg;
+}
+
 cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split, cudaStream_t st) {
     if (n_seqs == 0 || n_groups == 0 || b.total == 0) return gdn_chunked_batch(b, n_groups, n_seqs, 128, split, st);
+    if (b.h_v > 65535) return cudaErrorInvalidValue;
     GdnTcParams p{};
     const int T = b.total, qkw = b.h_k * D, vw = b.h_v * D;
     for (int g = 0; g < n_groups; ++g) {
@@ -774,16 +1336,19 @@ cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split
         p.s_out[g] = b.s_out[g];
     }
     p.cu = b.cu;
+    p.img = static_cast<uint8_t *>(b.img);
     p.total = b.total;
     p.max_len = b.max_len;
     p.h_k = b.h_k;
     p.h_v = b.h_v;
+    p.n_seqs = n_seqs;
+    p.slots = image_slots(b.total, n_seqs);
     p.scale = b.scale;
     p.status = b.status;
     return split ? launch<true>(p, n_groups, n_seqs, st) : launch<false>(p, n_groups, n_seqs, st);
 }
 
-cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, cudaStream_t st) {
+cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, void *img, cudaStream_t st) {
     GdnBatch b{};
     b.q[0] = static_cast<const __nv_bfloat16 *>(a.q);
     b.k[0] = static_cast<const __nv_bfloat16 *>(a.k);
@@ -794,6 +1359,7 @@ cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, cudaStre
     b.o[0] = static_cast<__nv_bfloat16 *>(a.o);
     b.s_out[0] = a.s_out;
     b.cu = a.cu_seqlens;
+    b.img = img;
     b.total = a.total_tokens;
     b.max_len = a.max_seqlen;
     b.h_k = a.h_k;

@@ -57,9 +57,11 @@ struct GroupBufs {
     void *a_lo, *h_lo;  // bf16, or e4m3 bytes with the fp8 low pass
 };
 
-// Carves the per-group scratch buffers out of the workspace (after its header).
-// Returns the bytes used; with base == nullptr only sizes are computed.
-size_t carve(const Dims &m, char *base, GroupBufs *out) {
+// Carves the per-group scratch buffers, then the chunk images of the two-phase
+// gated-delta kernels (shared by the layers; *img), out of the workspace
+// (after its header).  Returns the bytes used; with base == nullptr only sizes
+// are computed.
+size_t carve(const Dims &m, char *base, GroupBufs *out, void **img = nullptr) {
     size_t off = kWsHeader;
     auto take = [&](size_t bytes) {
         char *ptr = base ? base + off : nullptr;
@@ -88,6 +90,8 @@ size_t carve(const Dims &m, char *base, GroupBufs *out) {
         b.h_lo = m.split ? take(T * m.I * lo_elem) : nullptr;
         if (out) out[g] = b;
     }
+    void *im = take(gdn_tc_supported(m.d) ? gdn_tc_image_bytes(m.T, m.N, m.hv, m.G) : 0);
+    if (img) *img = im;
     return off;
 }
 
@@ -205,7 +209,8 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         return SR_OK;
     }
     GroupBufs B[kMaxGroups];
-    carve(m, static_cast<char *>(ws), B);
+    void *img = nullptr;
+    carve(m, static_cast<char *>(ws), B, &img);
     Prof prof{a->profile, st};
     if (a->profile) a->profile->count = 0;
     const int G = m.G, T = m.T;
@@ -282,7 +287,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             gb.o[g] = stop ? nullptr : B[g].o;
             gb.s_out[g] = O(g).s_out;
         }
-        gb.cu = a->cu_seqlens; gb.total = T; gb.max_len = a->max_seqlen; gb.h_k = m.hk; gb.h_v = m.hv;
+        gb.cu = a->cu_seqlens; gb.img = img; gb.total = T; gb.max_len = a->max_seqlen; gb.h_k = m.hk; gb.h_v = m.hv;
         gb.scale = 1.0f / sqrtf(float(m.d)); gb.status = status;
         SR_TRY(prof.begin(SR_K_GDN));
         SR_TRY(gdn_tc_supported(m.d) ? gdn_tc_batch(gb, G, m.N, m.split, st)

@@ -31,6 +31,7 @@ struct GdnBatch {
     __nv_bfloat16 *o[kMaxGroups];     // may be null
     float *s_out[kMaxGroups];
     const int32_t *cu;
+    void *img;  // tcgen05 two-phase form: chunk images (gdn_tc_image_bytes); null selects the fused kernel
     int total, max_len, h_k, h_v;
     float scale;
     uint32_t *status;
@@ -38,7 +39,9 @@ struct GdnBatch {
 cudaError_t gdn_chunked_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st);
 // The same on tcgen05 with the state in tensor memory (d = 128; gdn_tc.cu).
 bool gdn_tc_supported(int d);
-cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, cudaStream_t st);
+cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, void *img, cudaStream_t st);
+// Scratch of the two-phase form: one 40 KB chunk image per (group, chunk slot, V head).
+size_t gdn_tc_image_bytes(int total, int n_seqs, int h_v, int n_groups);
 cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split, cudaStream_t st);
 
 // 2-D bf16 TMA map (128-byte swizzle) over a row-major [rows, cols] matrix with row pitch `pitch`.

@@ -72,6 +72,21 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
                  "r"(smem_u32(src)), "r"(x), "r"(y)
                  : "memory");
 }
+// Untiled bulk copy global -> shared completing on an mbarrier (both addresses
+// 16-byte aligned, `bytes` a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     smem_u32(dst)),
+                 "l"(static_cast<uint64_t>(__cvta_generic_to_global(src))), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Untiled bulk copy shared -> global (bulk-group completion; same alignment rules).
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(
+                     static_cast<uint64_t>(__cvta_generic_to_global(dst))),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
 // Waits until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }

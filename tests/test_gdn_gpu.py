@@ -15,7 +15,7 @@ from _util import OUT_TOL_BF16, STATE_TOL, TOL_FP32, assert_close
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = ["sequential", "chunked", "tcgen05"]
+ALGOS = ["sequential", "chunked", "tcgen05", "tcgen05_fused"]
 
 
 @pytest.fixture(scope="module")
@@ -27,7 +27,7 @@ def sr():
 
 
 def run_gpu(sr, x: W.GdnInputs, algo, want_o=True, dev="cuda"):
-    if algo == "tcgen05" and x.q.shape[-1] != 128:
+    if algo.startswith("tcgen05") and x.q.shape[-1] != 128:
         pytest.skip("the tcgen05 kernel takes d = 128 only")
     t = lambda a: None if a is None else a.to(dev).contiguous()
     o, s = sr.gdn_replay(t(x.q), t(x.k), t(x.v), t(x.g), t(x.beta), t(x.cu_seqlens),
@@ -141,7 +141,7 @@ def test_exact_resume_on_gpu(sr, algo, split_at):
     T = 300
     x = W.gdn_inputs(15, [T], 2, 4, 128, 128)
     d = lambda a: a.cuda().contiguous()
-    if algo == "tcgen05" and x.q.shape[-1] != 128:
+    if algo.startswith("tcgen05") and x.q.shape[-1] != 128:
         pytest.skip("d = 128 only")
     full_o, full_s = sr.gdn_replay(d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.cu_seqlens), max_seqlen=T,
                                    algo=algo)
@@ -157,3 +157,33 @@ def test_exact_resume_on_gpu(sr, algo, split_at):
     ref = full_s.double().cpu().numpy()
     assert_close(s_b, ref, STATE_TOL, "resumed state vs full replay")
     assert_close(o_b, full_o[split_at:].double().cpu().numpy(), OUT_TOL_BF16, "resumed outputs")
+
+
+def test_two_phase_equals_fused(sr):
+    """The two-phase tcgen05 form (state-free chunk work for all chunks first,
+    then the state chain) does the fused kernel's arithmetic in the same order:
+    the results are the same bits."""
+    x = W.raw_qwen()
+    o2, s2 = run_gpu(sr, x, "tcgen05")
+    o1, s1 = run_gpu(sr, x, "tcgen05_fused")
+    assert torch.equal(s1, s2)
+    assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("algo", ["tcgen05", "tcgen05_fused"])
+def test_many_short_sequences(sr, algo):
+    """More sequences than the longest-first ranking handles (300), lengths
+    0..140 with empty ones between: every chunk finds its image slot."""
+    gen = torch.Generator().manual_seed(31)
+    lengths = torch.randint(0, 141, (300,), generator=gen).tolist()
+    for i in range(0, 300, 37):
+        lengths[i] = 0
+    x = W.gdn_inputs(31, lengths, 1, 2, 128, 128, h0_std=0.2)
+    o, s = run_gpu(sr, x, algo)
+    units = [n * 2 + h for n in range(0, 300, 7) for h in range(2)]
+    o_ref, s_ref = run_oracle(x, units=units)
+    cu = x.cu_seqlens.tolist()
+    for u in units:
+        n, h = divmod(u, 2)
+        assert_close(s[n, h], s_ref[n, h], STATE_TOL, f"state seq {n} head {h}")
+        assert_close(o[cu[n]:cu[n + 1], h], o_ref[cu[n]:cu[n + 1], h], OUT_TOL_BF16, f"o seq {n} head {h}")
