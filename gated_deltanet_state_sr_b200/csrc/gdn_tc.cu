@@ -73,7 +73,7 @@ constexpr uint32_t smem_fused(bool split) {
 // Chunk image of the two-phase form, per (group, chunk slot, V head): bf16
 // tiles in the 128-byte swizzled layouts of the products that read them.
 constexpr uint32_t IMG_P = 0;        // P, K-major [t][s]
-constexpr uint32_t IMG_W = 8192;     // -W^T, MN-major [j][t] (16 KB)
+constexpr uint32_t IMG_W = 8192;     // -W, K-major [t][j], columns j 0-63 then 64-127 (16 KB)
 constexpr uint32_t IMG_T2H = 24576;  // T diag(beta), hi, K-major [t][s]
 constexpr uint32_t IMG_T2L = 32768;  // T diag(beta), lo
 constexpr uint32_t kImg = 40960;
@@ -84,8 +84,9 @@ constexpr uint32_t kImg = 40960;
 constexpr uint32_t kPrepIn[2] = {32768, 49152};
 constexpr uint32_t smem_prep(bool split) { return kPrepIn[split] + 2 * SZ_AT + SZ_MISC + 1024; }
 
-// sequential kernel: inputs, the chunk image, S bf16, Qg, the U tiles
-constexpr uint32_t smem_seq(bool split) { return kIn[split] + kImg + SZ_SB + SZ_QG + SZ_XR + SZ_MISC + 1024; }
+// sequential kernel: inputs, P and T2 (hi, lo), S bf16, [Qg ; -W] stacked, the U tiles
+constexpr uint32_t SZ_PT2 = 24576, SZ_QGW = 32768;
+constexpr uint32_t smem_seq(bool split) { return kIn[split] + SZ_PT2 + SZ_SB + SZ_QGW + SZ_XR + SZ_MISC + 1024; }
 static_assert(smem_seq(true) <= 232448, "sequential kernel exceeds shared memory");
 static_assert(2 * (smem_prep(true) + 1024) <= 233472, "two prep CTAs must fit one SM");
 
@@ -98,6 +99,7 @@ constexpr uint32_t ID_KK = idesc_bf16_f32_major(128, 64, 0, 0);    // K-major A 
 constexpr uint32_t ID_MN_K = idesc_bf16_f32_major(128, 64, 1, 0);  // MN-major A, K-major B
 constexpr uint32_t ID_K_MN = idesc_bf16_f32_major(128, 64, 0, 1);  // K-major A, MN-major B
 constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 0, 1);    // state update (N = 128)
+constexpr uint32_t ID_KK128 = idesc_bf16_f32_major(128, 128, 0, 0);  // K-major A and B, N = 128
 
 struct GdnTcParams {
     CUtensorMap q[kMaxGroups], k[kMaxGroups], v[kMaxGroups], kl[kMaxGroups], vl[kMaxGroups];
@@ -417,16 +419,17 @@ __device__ __forceinline__ void mma_w(uint32_t base, uint32_t o1, uint32_t RW) {
     }
 }
 
-// Ut^T = V^T T2^T -> RU from the hi and lo tiles of T2 (split: + Vl^T T2h^T).
+// Ut^T = V^T T2^T -> RU from the hi and lo tiles of T2 (split: + Vl^T T2h^T);
+// with acc0 the first product adds to what RU holds.
 template <bool SPLIT>
-__device__ __forceinline__ void mma_ut(uint32_t base, uint32_t o2h, uint32_t o2l, uint32_t RU) {
+__device__ __forceinline__ void mma_ut(uint32_t base, uint32_t o2h, uint32_t o2l, uint32_t RU, bool acc0) {
     base = fresh(base);
     const uint64_t dv = sdesc_sw128(base + OFF_V, 8192, 1024);  // V as MN-major A (i blocks 8 KB apart)
     const uint64_t dvl = sdesc_sw128(base + OFF_VL, 8192, 1024);
     const uint64_t dh = sdesc_sw128(base + o2h, 16, 1024), dl = sdesc_sw128(base + o2l, 16, 1024);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dh, k * 32), ID_MN_K, k > 0);
+        mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dh, k * 32), ID_MN_K, k > 0 || acc0);
         mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dl, k * 32), ID_MN_K, 1);
         if (SPLIT) mma_bf16_ss(RU, dadd(dvl, k * 2048), dadd(dh, k * 32), ID_MN_K, 1);
     }
@@ -449,6 +452,19 @@ __device__ __forceinline__ void mma_sq(uint32_t base, uint32_t sb_off, uint32_t 
     for (int k = 0; k < 8; ++k)
         mma_bf16_ss(RO, dadd(da, (k >> 2) * 16384 + (k & 3) * 32), dadd(db, (k >> 2) * 8192 + (k & 3) * 32),
                     ID_KK, k > 0);
+}
+
+// [O^T | S (-W)^T] = S [Qg ; -W]^T -> RD (128 columns) in one product group:
+// S bf16 at sb_off, the stacked K-major tiles [Qg_j0 | -W_j0 | Qg_j1 | -W_j1]
+// (64 rows each) at qgw_off.
+__device__ __forceinline__ void mma_sqw(uint32_t base, uint32_t sb_off, uint32_t qgw_off, uint32_t RD) {
+    base = fresh(base);
+    const uint64_t da = sdesc_sw128(base + sb_off, 16, 1024), db = sdesc_sw128(base + qgw_off, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_bf16_ss(RD, dadd(da, off), dadd(db, off), ID_KK128, k > 0);
+    }
 }
 
 // S += (U diag)^T K -> RS and O^T += U^T P^T -> RO, from the U tiles (Udh, Udl,
@@ -496,9 +512,11 @@ __device__ __forceinline__ void state_copy(uint8_t *sm, uint32_t sb_off, uint32_
     tmem_st_wait();
 }
 
-// Qg = scale e^{gamma_t} Q (same swizzled geometry as the Q tiles) at qg_off.
-__device__ __forceinline__ void build_qg(uint8_t *sm, uint32_t qg_off, const float *gam, float scale, int tid) {
-    for (int e = tid; e < 1024; e += kThreads) {
+// Qg = scale e^{gamma_t} Q (same swizzled geometry as the Q tiles): the two
+// 64-column halves at qg_off and qg_off + half_stride; thread i of nthr.
+__device__ __forceinline__ void build_qg(uint8_t *sm, uint32_t qg_off, uint32_t half_stride, const float *gam,
+                                         float scale, int i, int nthr) {
+    for (int e = i; e < 1024; e += nthr) {
         const int sub = e >> 9, t = (e >> 3) & 63, ch = e & 7;
         const uint32_t off = sw128(t, ch);
         const uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_KQ + 8192 + sub * 16384 + off);
@@ -511,7 +529,7 @@ __device__ __forceinline__ void build_qg(uint8_t *sm, uint32_t qg_off, const flo
             const float2 xf = __bfloat1622float2(x2[q2]);
             wp[q2] = pack2(xf.x * f, xf.y * f);
         }
-        *reinterpret_cast<uint4 *>(sm + qg_off + sub * 8192 + off) = w;
+        *reinterpret_cast<uint4 *>(sm + qg_off + sub * half_stride + off) = w;
     }
 }
 
@@ -530,6 +548,22 @@ __device__ __forceinline__ void convert_w(uint8_t *sm, uint32_t w_off, uint32_t 
         w.w = pack2(-__uint_as_float(r[8 * q4 + 6]), -__uint_as_float(r[8 * q4 + 7]));
         *reinterpret_cast<uint4 *>(sm + w_off + sw128(row, 4 * half + q4)) = w;
     }
+}
+
+// -W (bf16) from TMEM RW (holding W^T: lane = j, columns = t) as the K-major
+// tiles [t][j] of j 0-63 at w_off and j 64-127 at w_off + 8 KB.
+__device__ __forceinline__ void convert_w_t(uint8_t *sm, uint32_t w_off, uint32_t RW, uint32_t lane_off, int half,
+                                            int row) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(RW + lane_off + 32 * half, r);
+    tmem_ld_wait();
+    uint8_t *wt = sm + w_off + (row >> 6) * 8192;
+    const uint32_t cofs = uint32_t(row & 7) * 2;
+    const uint32_t chunk = uint32_t(row & 63) >> 3;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        *reinterpret_cast<__nv_bfloat16 *>(wt + sw128(32 * half + e, chunk) + cofs) =
+            __float2bfloat16_rn(-__uint_as_float(r[e]));
 }
 
 // U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16) from TMEM RU as K-major
@@ -783,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         }
         // ---- meanwhile: bf16 copy of S (entering the chunk), S <- e^{gamma_C} S, and Qg
         state_copy(sm, oSB, R2, lane_off, half, row, __expf(gC));
-        build_qg(sm, oQG, gam, scale, tid);
+        build_qg(sm, oQG, 8192, gam, scale, tid, kThreads);
         fence_async_smem();
         tc_fence_before();
         if (check(true)) break;
@@ -811,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             if (!mbar_wait(bar_v, v_phase)) *abort_flag = 1;
             tc_fence_after();
             mma_w<SPLIT>(base, oTR, R1);
-            mma_ut<SPLIT>(base, oTR + 8192, oTR + 16384, R0);
+            mma_ut<SPLIT>(base, oTR + 8192, oTR + 16384, R0, false);
             mma_commit(bar_mma);
         }
         v_phase ^= 1;
@@ -910,11 +944,15 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
     const int row = quad * 32 + lane;
 
     // the sequence holding this slot: the largest n with floor(cu[n] / C) + n <= slot
-    int lo = 0, hi = p.n_seqs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.cu[mid] / C + mid <= slot) lo = mid;
-        else hi = mid - 1;
+    // (a key that grows with n).  Every warp narrows [lo, hi) 32-fold per round with
+    // one probe per lane, so a few hundred sequences take two rounds of loads.
+    int lo = 0, hi = p.n_seqs;
+    while (hi - lo > 1) {
+        const int step = (hi - lo + 31) >> 5, m = lo + lane * step;
+        const bool le = m < hi && p.cu[m] / C + m <= slot;
+        const int k = max(1, __popc(__ballot_sync(0xffffffffu, le)));  // the probes at or below: a prefix
+        hi = min(hi, lo + k * step);
+        lo += (k - 1) * step;
     }
     const int n = lo;
     int bos, eos;
@@ -924,21 +962,11 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
     const int clen = min(C, len - c * C), y = bos + c * C;
     const int hk = h / (p.h_v / p.h_k);
 
+    // the tiles and the gates are requested first; tensor memory is taken while they load
     if (tid == 0) {
         mbar_init(bar_in, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, 128);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot, R0 = tmem, R1 = tmem + 64;
-    const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    if (tid == 0) {
         const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mkl = &p.kl[gi];
         mbar_arrive_expect_tx(bar_in, SPLIT ? 49152u : 32768u);
         tma_load_2d(sm + OFF_KQ, mk, bar_in, hk * D, y);
@@ -950,11 +978,24 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
             tma_load_2d(sm + OFF_KL + 8192, mkl, bar_in, hk * D + 64, y);
         }
     }
-    // gates: gamma = inclusive prefix sum of g; padding has g = beta = 0
+    float g0 = 0.f, b0 = 0.f;  // padding has g = beta = 0
+    if (tid < clen) {
+        g0 = p.g[gi][size_t(y + tid) * p.h_v + h];
+        b0 = p.beta[gi][size_t(y + tid) * p.h_v + h];
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot, R0 = tmem, R1 = tmem + 64;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    // gates: gamma = inclusive prefix sum of g
     if (tid < C) {
-        const bool in = tid < clen;
-        gam[tid] = in ? p.g[gi][size_t(y + tid) * p.h_v + h] : 0.f;
-        bet[tid] = in ? p.beta[gi][size_t(y + tid) * p.h_v + h] : 0.f;
+        gam[tid] = g0;
+        bet[tid] = b0;
     }
     __syncthreads();
     if (warp == 0) gate_prefix(gam, lane);
@@ -981,11 +1022,15 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         mma_phase ^= 1;
         tc_fence_after();
         build_a_p<SPLIT>(sm, oP, Af, R0, R1, lane_off, quad, half, row, gam, bet, fb, eg, ei, fact, p.scale);
+        fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(w) != 0;
     }
+    // each tile of the image leaves as soon as it is formed
+    uint8_t *dst = p.img + ((size_t(gi) * p.slots + slot) * p.h_v + h) * kImg;
+    if (ok && tid == 0) bulk_store(dst + IMG_P, sm + oP, 8192);
     if (ok) {
-        // ---- the solve, T1 and T2, then W^T = K^T T1^T and -W^T
+        // ---- the solve, T1 and T2, then W^T = K^T T1^T and -W
         t_solve(Af, Tf, tid, warp, lane);
         write_t12(sm, Tf, bet, fb, oT1, oT2H, oT2L, tid);
         fence_async_smem();
@@ -995,25 +1040,25 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
             tc_fence_after();
             mma_w<SPLIT>(base, oT1, R0);
             mma_commit(bar_mma);
+            bulk_store(dst + IMG_T2H, sm + oT2H, 8192);
+            bulk_store(dst + IMG_T2L, sm + oT2L, 8192);
         }
         const bool w = mbar_wait(bar_mma, mma_phase);
         mma_phase ^= 1;
         tc_fence_after();
-        convert_w(sm, oW, R0, lane_off, half, row);
+        convert_w_t(sm, oW, R0, lane_off, half, row);
         fence_async_smem();
         ok = __syncthreads_and(w) != 0;
     }
     if (ok) {
         if (tid == 0) {
-            uint8_t *dst = p.img + ((size_t(gi) * p.slots + slot) * p.h_v + h) * kImg;
-            bulk_store(dst + IMG_P, sm + oP, 8192);
             bulk_store(dst + IMG_W, sm + oW, 16384);
-            bulk_store(dst + IMG_T2H, sm + oT2H, 8192);
-            bulk_store(dst + IMG_T2L, sm + oT2L, 8192);
             bulk_commit();
-            bulk_wait_all();
+            bulk_wait_read();  // shared memory may go; the writes complete with the grid
         }
     } else if (tid == 0) {
+        bulk_commit();
+        bulk_wait_read();
         atomicOr(p.status, SR_DEV_TIMEOUT);
         mma_commit(bar_mma);
         mbar_wait(bar_mma, mma_phase);
@@ -1056,8 +1101,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(sm);
-    constexpr uint32_t oIMG = kIn[SPLIT], oSB = oIMG + kImg, oQG = oSB + SZ_SB, oXR = oQG + SZ_QG;
-    constexpr uint32_t oMISC = oXR + SZ_XR;
+    constexpr uint32_t oP = kIn[SPLIT], oT2H = oP + 8192, oT2L = oP + 16384;
+    constexpr uint32_t oSB = oP + SZ_PT2, oQGW = oSB + SZ_SB, oXR = oQGW + SZ_QGW, oMISC = oXR + SZ_XR;
     float *gam = reinterpret_cast<float *>(sm + oMISC);  // [64]
     float *fu = gam + C;                                  // [64] e^{gamma_C - gamma_t}
     uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 1024);  // K (+ k low part) landed
@@ -1107,7 +1152,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t RU = tmem, RS = tmem + 128, RO0 = tmem + 256, RO1 = tmem + 320;
+    // S in columns 0-127; per chunk parity a 128-column pair [O | U]
+    const uint32_t RS = tmem, RO0 = tmem + 128, RO1 = tmem + 256;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
     state_init(RS, lane_off, half, row, h0, sbase);
@@ -1143,13 +1189,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
             tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * D + 64, y);
         }
     };
-    auto issue_w = [&](int c) {  // -W^T, T2 hi, T2 lo
+    auto issue_w = [&](int c) {  // -W (its halves beside those of Qg), T2 hi, T2 lo
+        const uint8_t *src = img_of(c);
         mbar_arrive_expect_tx(bar_w, kImg - IMG_W);
-        bulk_load(sm + oIMG + IMG_W, img_of(c) + IMG_W, kImg - IMG_W, bar_w);
+        bulk_load(sm + oQGW + 8192, src + IMG_W, 8192, bar_w);
+        bulk_load(sm + oQGW + 24576, src + IMG_W + 8192, 8192, bar_w);
+        bulk_load(sm + oT2H, src + IMG_T2H, kImg - IMG_T2H, bar_w);
     };
     auto issue_p = [&](int c) {
         mbar_arrive_expect_tx(bar_p, IMG_W - IMG_P);
-        bulk_load(sm + oIMG + IMG_P, img_of(c) + IMG_P, IMG_W - IMG_P, bar_p);
+        bulk_load(sm + oP, img_of(c) + IMG_P, IMG_W - IMG_P, bar_p);
     };
     if (tid == 0) {
         prefetch_tmap(mq); prefetch_tmap(mk); prefetch_tmap(mv);
@@ -1181,56 +1230,62 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     // gates of chunk c in gam (gamma = inclusive prefix sum of g; padding has g = 0),
     // fu, and Qg = scale e^{gamma_t} Q once Q has landed; false when a wait failed
     float g_next = 0.f;  // g of the next chunk (threads tid < C)
+    // (warp 0 issues the products and takes no part here: threads 64-127 hold the
+    // gates, warp 1 scans them, warps 1-7 form Qg)
+    const int gt = tid - 64;  // the token whose gate this thread holds, when in [0, C)
     auto next_gates_and_qg = [&](int c) -> bool {
-        if (tid < C) {
-            gam[tid] = g_next;
-            const int t = (c + 1) * C + tid;
+        if (gt >= 0 && gt < C) {
+            gam[gt] = g_next;
+            const int t = (c + 1) * C + gt;
             g_next = t < len ? gh[size_t(t) * h_v] : 0.f;
         }
         const bool qok = mbar_wait(bar_q, q_phase);
         q_phase ^= 1;
         __syncthreads();
-        if (warp == 0) gate_prefix(gam, lane);
+        if (warp == 1) gate_prefix(gam, lane);
         if (check(qok)) return false;
-        if (tid < C) fu[tid] = __expf(gam[C - 1] - gam[tid]);  // read after later barriers
-        build_qg(sm, oQG, gam, scale, tid);
+        if (gt >= 0 && gt < C) fu[gt] = __expf(gam[C - 1] - gam[gt]);  // read after later barriers
+        if (warp > 0) build_qg(sm, oQGW, 16384, gam, scale, tid - 32, kThreads - 32);
         fence_async_smem();
         return true;
     };
 
-    if (tid < C && tid < len) g_next = gh[size_t(tid) * h_v];
+    if (gt >= 0 && gt < C && gt < len) g_next = gh[size_t(gt) * h_v];
     bool ok = next_gates_and_qg(0);
     ok = ok && !check(true);
     if (ok && tid == 0 && nchunks > 1) issue_q(1);
 
     int c = 0;
     for (; ok && c < nchunks; ++c) {
-        const uint32_t RO = (c & 1) ? RO1 : RO0, RO_prev = (c & 1) ? RO0 : RO1;
+        const uint32_t RO = (c & 1) ? RO1 : RO0, RO_prev = (c & 1) ? RO0 : RO1, RU = RO + 64;
         // ---- bf16 copy of S (entering the chunk), then S <- e^{gamma_C} S
         state_copy(sm, oSB, RS, lane_off, half, row, __expf(gam[C - 1]));
         fence_async_smem();
         tc_fence_before();
         if (check(true)) break;
 
-        // ---- O(c) = S Qg^T ;  U^T = V^T T2^T + S (-W)^T
+        // ---- [O(c) | U^T] = S [Qg ; -W]^T, then U^T += V^T T2^T
         if (tid == 0) {
             const bool w = mbar_wait(bar_v, v_phase) && mbar_wait(bar_w, w_phase);
             if (!w) *abort_flag = 1;
             tc_fence_after();
-            mma_sq(base, oSB, oQG, RO);
-            mma_ut<SPLIT>(base, oIMG + IMG_T2H, oIMG + IMG_T2L, RU);
-            mma_sw(base, oSB, oIMG + IMG_W, RU);
+            mma_sqw(base, oSB, oQGW, RO);
+            mma_ut<SPLIT>(base, oT2H, oT2L, RU, true);
             mma_commit(bar_mma);
         }
         v_phase ^= 1;
         w_phase ^= 1;
-        // ---- meanwhile: o of the previous chunk
-        if (o && c > 0) out_direct(RO_prev, lane_off, half, row, o, size_t(bos) + size_t(c - 1) * C, C, v_stride, h);
+        // ---- meanwhile: o of the previous chunk (warp 4 also takes warp 0's share)
+        if (o && c > 0) {
+            const size_t tok0 = size_t(bos) + size_t(c - 1) * C;
+            if (warp != 0) out_direct(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h);
+            if (warp == 4) out_direct(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h);
+        }
         const bool m2 = wait_mma() && *abort_flag == 0;
         if (check(m2)) break;
-        if (tid == 0 && c + 1 < nchunks) {
-            issue_v(c + 1);
-            issue_w(c + 1);
+        if (c + 1 < nchunks) {  // issued from warps other than the product issuer
+            if (tid == 128) issue_v(c + 1);
+            if (tid == 160) issue_w(c + 1);
         }
 
         // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16): K-major tiles [i][t]
@@ -1244,21 +1299,21 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
             const bool w = mbar_wait(bar_k, k_phase) && mbar_wait(bar_p, p_phase);
             if (!w) *abort_flag = 1;
             tc_fence_after();
-            mma_update<SPLIT>(base, oXR, oIMG + IMG_P, RS, RO);
+            mma_update<SPLIT>(base, oXR, oP, RS, RO);
             mma_commit(bar_mma);
         }
         k_phase ^= 1;
         p_phase ^= 1;
-        // ---- meanwhile: gates and Qg of the next chunk (the Qg region was last read
+        // ---- meanwhile: gates and Qg of the next chunk (the Qg tiles were last read
         // by the first product group, complete at the previous wait)
         bool nok = true;
         if (c + 1 < nchunks) nok = next_gates_and_qg(c + 1);
         const bool m4 = wait_mma() && *abort_flag == 0 && nok;
         if (check(m4)) break;
-        if (tid == 0 && c + 1 < nchunks) {
-            issue_k(c + 1);
-            issue_p(c + 1);
-            if (c + 2 < nchunks) issue_q(c + 2);
+        if (c + 1 < nchunks) {
+            if (tid == 32) issue_k(c + 1);
+            if (tid == 64) issue_p(c + 1);
+            if (tid == 96 && c + 2 < nchunks) issue_q(c + 2);
         }
     }
 

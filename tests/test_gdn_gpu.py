@@ -159,15 +159,18 @@ def test_exact_resume_on_gpu(sr, algo, split_at):
     assert_close(o_b, full_o[split_at:].double().cpu().numpy(), OUT_TOL_BF16, "resumed outputs")
 
 
-def test_two_phase_equals_fused(sr):
+def test_two_phase_matches_fused(sr):
     """The two-phase tcgen05 form (state-free chunk work for all chunks first,
-    then the state chain) does the fused kernel's arithmetic in the same order:
-    the results are the same bits."""
+    then the state chain) forms the same products as the fused kernel; only the
+    order in which S (-W)^T and V^T T2^T enter the fp32 accumulator of U differs.
+    That moves a few bf16 roundings of the state copy, which the recurrence
+    carries on: the two agree far inside the tolerance each meets against the
+    oracle (a tenth of it here)."""
     x = W.raw_qwen()
     o2, s2 = run_gpu(sr, x, "tcgen05")
     o1, s1 = run_gpu(sr, x, "tcgen05_fused")
-    assert torch.equal(s1, s2)
-    assert torch.equal(o1, o2)
+    assert_close(s2, s1.double().cpu().numpy(), STATE_TOL / 10, "state, two-phase vs fused")
+    assert_close(o2, o1.double().cpu().numpy(), OUT_TOL_BF16 / 2, "o, two-phase vs fused")
 
 
 @pytest.mark.parametrize("algo", ["tcgen05", "tcgen05_fused"])
