@@ -51,8 +51,9 @@ L2_BYTES = 126 * 1024 * 1024
 MEASURED_TRAFFIC = {
     # in_proj of the 1-group workload with the fp8 low pass: 108.2 MB read + 39.1 MB written, x 8 groups
     "model_32k_5": ("gemm_tc.cu", "a8e892e37e32b385", 8 * 147.3e6),
-    # the raw workload's launch: 151.9 MB read + 54.4 MB written
-    "raw_qwen": ("gdn_tc.cu", "17abce7b1cf5d0e5", 206.4e6),
+    # the raw workload's call, both kernels of the two-phase form: prep 76.1 MB read +
+    # 133.6 MB written, sequential 340.4 MB read + 65.8 MB written
+    "raw_qwen": ("gdn_tc.cu", "6ee9786ec1a3d225", 615.9e6),
     # the Mamba2 workload's launch: 1270.8 MB read + 1216.6 MB written
     "mamba2": ("mamba2_tc.cu", "819b48f130629684", 2487.4e6),
 }
@@ -222,8 +223,10 @@ class RawGdn:
         return self.h_o.numel() * self.h_o.element_size() + self.h_s.numel() * 4
 
     def dominant(self):
-        # the default algorithm: the tcgen05 kernel at d = 128, the mma.sync one at d = 64
-        return {"name": "gdn_tc_kernel" if self.d == 128 else "gdn_chunk_kernel", "bound": "tensor",
+        # the default algorithm: at d = 128 the two tcgen05 kernels of one replay (the
+        # chunk-parallel prep, then the per-sequence state chain), timed as the pair;
+        # the mma.sync kernel at d = 64
+        return {"name": "gdn_prep_kernel + gdn_seq_kernel" if self.d == 128 else "gdn_chunk_kernel", "bound": "tensor",
                 "flop": self.flop_per_tok * self.tokens,
                 "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
 
