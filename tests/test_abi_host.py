@@ -67,6 +67,33 @@ def test_gdn_workspace_required():
     assert "workspace" in sr.last_error()
 
 
+def test_gdn_two_phase_workspace_holds_the_chunk_images():
+    """The default tcgen05 form (d = 128) keeps one 40 KB chunk image per (chunk
+    slot, V head), with floor(T / 64) + n_seqs slots; the fused form and the
+    other kernels need only the 256-byte header."""
+    kw = dict(d_k=128, d_v=128, h_k=16, h_v=32, n_seqs=8, total_tokens=8917, max_seqlen=2048)
+    slots = 8917 // 64 + 8
+    want = 256 + slots * 32 * 40960
+    assert sr.gdn_workspace_bytes(_gdn(**kw)) == want
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05, **kw)) == want
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED, **kw)) == 256
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_SEQUENTIAL, **kw)) == 256
+    # d = 64 takes the mma.sync kernel, which needs no scratch
+    assert sr.gdn_workspace_bytes(_gdn()) == 256
+    # the tcgen05 forms take bf16 at d = 128 only
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED)) == 0
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED, dtype=sr.SR_FP32, **kw)) == 0
+
+
+def test_group_workspace_holds_the_chunk_images():
+    """A replay group's workspace grows by the chunk images of its gated-delta
+    layers: 40 KB per (group, chunk slot, V head)."""
+    a16, a80 = _fake_group_args(total_tokens=16, max_seqlen=16), _fake_group_args(total_tokens=80, max_seqlen=80)
+    grow = sr.group_workspace_bytes(a80) - sr.group_workspace_bytes(a16)
+    # 64 more tokens: one more slot (80 // 64 - 16 // 64) of 4 V heads, plus the per-token buffers
+    assert grow >= 1 * 4 * 40960
+
+
 def test_gdn_workspace_too_small_and_misaligned():
     import torch
     a = _gdn()
