@@ -17,7 +17,9 @@
 //                            diagonal 64 x 64 blocks are the two heads' outputs
 //     S += [xw_h0^T; xw_h1^T] B   (xw = x diag(dt e^{gamma_C-gamma}) as hi + lo)
 // with Gm_h = (G o L_h), L_h[t][s] = e^{gamma_t-gamma_s} dt_s for s <= t.  C, B and
-// x tiles arrive by TMA (double-buffered); full chunks of y leave by TMA.
+// x tiles arrive by TMA (double-buffered); y goes from tensor memory straight to
+// global memory, a warp storing 32 consecutive channels of one token per
+// instruction.
 // Exponentials only ever see differences gamma_t - gamma_s with s <= t.
 // Every mbarrier wait is bounded; a timeout records SR_DEV_TIMEOUT, drains the
 // MMAs, frees tensor memory and ends the CTA.
@@ -46,13 +48,13 @@ constexpr uint32_t OFF_IN = 0;           // two buffers
 constexpr uint32_t OFF_SB = 2 * SZ_IN;   // bf16 state [(h,p)][n]: two 64-column halves of 16 KB
 constexpr uint32_t OFF_Q = OFF_SB + 32768;    // masked G rows [(h,t)][s], 16 KB
 constexpr uint32_t OFF_XW = OFF_Q + 16384;    // [xwh_h0][xwh_h1][xwl_h0][xwl_h1] tiles [t][p], 8 KB each
-constexpr uint32_t OFF_YS = OFF_XW + 32768;   // y staging [y_h0][y_h1] tiles [t][p]
+constexpr uint32_t OFF_YS = OFF_XW + 32768;   // G = C B^T staged for the mask rows
 constexpr uint32_t OFF_MISC = OFF_YS + 16384; // gates, tables, barriers
 constexpr uint32_t SZ_MISC = 3072;
 constexpr uint32_t kSmem = OFF_MISC + SZ_MISC + 1024;
 
 struct M2TcParams {
-    CUtensorMap mc, mb, mx, my;
+    CUtensorMap mc, mb, mx;
     const float *dt;
     const float *A;
     const int32_t *cu;
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     uint64_t *bar_y = bar_in + 4;    // chunk-internal part of y done
     uint64_t *bar_drain = bar_in + 5;  // every issued MMA done (abort path)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 6);
-    float *gs = reinterpret_cast<float *>(sm + OFF_YS);      // G = C B^T staged for the mask (before y uses it)
+    float *gs = reinterpret_cast<float *>(sm + OFF_YS);      // G = C B^T staged for the mask
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -164,7 +166,6 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     };
     if (tid == kIssueIn) {
         prefetch_tmap(&p.mc); prefetch_tmap(&p.mb); prefetch_tmap(&p.mx);
-        if (p.y) prefetch_tmap(&p.my);
         issue_in(0);
     }
 
@@ -200,7 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             dt_next = (t < len) ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
         }
         const bool tma_ok = mbar_wait(&bar_in[b], (c >> 1) & 1);
-        if (tid == 0) bulk_wait_read();  // the previous chunk's y tiles have left the staging area
         __syncthreads();
         if (warp < 2) {
             const float *d = dts + warp * C;
@@ -375,38 +375,20 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             tmem_ld_32x32b_x32(RI + lane_off + 32 * half, ri);
             tmem_ld_32x32b_x32(RY + lane_off + 64 * hrow + 32 * half, ry);
             tmem_ld_wait();
-            const float *eg = egs + hrow * C;
-            if (clen == C) {
-                uint8_t *yt = sm + OFF_YS + hrow * 8192;
-                const uint32_t cofs = uint32_t(prow & 7) * 2, chunk = uint32_t(prow) >> 3;
+            const float *eg = egs + hrow * C + 32 * half;
+            const size_t stride = size_t(H) * P;
+            __nv_bfloat16 *yd = p.y + (size_t(bos) + size_t(c) * C + 32 * half) * stride + size_t(2 * pair + hrow) * P + prow;
+            const int n_out = min(32, clen - 32 * half);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = 32 * half + e;
-                    *reinterpret_cast<__nv_bfloat16 *>(yt + sw128(t, chunk) + cofs) =
-                        __float2bfloat16_rn(eg[t] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
-                }
-                fence_async_smem();
-            } else {
-                const size_t tok0 = size_t(bos) + size_t(c) * C;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = 32 * half + e;
-                    if (t < clen)
-                        p.y[((tok0 + t) * H + 2 * pair + hrow) * P + prow] =
-                            __float2bfloat16_rn(eg[t] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
-                }
+            for (int e = 0; e < 32; ++e) {
+                if (e < n_out) *yd = __float2bfloat16_rn(eg[e] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
+                yd += stride;
             }
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0 && clen == C) {
-            tma_store_2d(&p.my, sm + OFF_YS, (2 * pair) * P, bos + c * C);
-            tma_store_2d(&p.my, sm + OFF_YS + 8192, (2 * pair + 1) * P, bos + c * C);
-            bulk_commit();
-        }
     }
-    if (tid == 0) bulk_wait_all();
 
     __syncthreads();
     ok = *abort_flag == 0;
@@ -449,7 +431,6 @@ cudaError_t mamba2_tc(const sr_mamba2_args &a, uint32_t *status, cudaStream_t st
     if (!make_map_bf16(&p.mc, a.C, T, NS, NS, 64, 64) || !make_map_bf16(&p.mb, a.B, T, NS, NS, 64, 64) ||
         !make_map_bf16(&p.mx, a.x, T, hp, hp, 64, 64))
         return cudaErrorInvalidValue;
-    if (a.y && !make_map_bf16(&p.my, a.y, T, hp, hp, 64, 64)) return cudaErrorInvalidValue;
     p.dt = a.dt;
     p.A = a.A;
     p.cu = a.cu_seqlens;
