@@ -38,8 +38,9 @@ using namespace tc;
 constexpr int C = 64, P = 64, NS = 128;
 constexpr int kThreads = 256;
 // MMA and TMA issue is spread over threads of warps that are idle at that point:
-// warp 7 (no gate-table work) loads the next chunk and forms C B^T at the chunk
-// start; warp 2 (no part in staging C B^T) issues the products after the state copy.
+// warp 7 (no gate-table work) forms C B^T at the chunk start and, with warp 2, has
+// no part in staging C B^T: after the state copy warp 7 loads the next chunk and
+// warp 2 issues the products.
 constexpr int kIssueIn = 224, kIssueMma = 64;
 
 // shared memory (bytes from a 1024-aligned base)
@@ -217,8 +218,6 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         }
         if (check(tma_ok)) break;
         if (tid == kIssueIn) {
-            // the input buffer of chunk c+1 last served chunk c-1, whose products have completed
-            if (c + 1 < nchunks) issue_in(c + 1);
             if (want_y) {  // G = [C;B] B^T -> RG needs only this chunk's inputs
                 tc_fence_after();
 #pragma unroll
@@ -288,6 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         tc_fence_before();
         if (check(true)) break;
 
+        // the input buffer of chunk c+1 last served chunk c-1, whose products have
+        // completed; its loads are issued here, where the issuing warp has no part in
+        // staging C B^T
+        if (tid == kIssueIn && c + 1 < nchunks) issue_in(c + 1);
         // ---- MMAs: Yi^T = [S] C^T -> RI; S += xw^T B (hi, lo)
         if (tid == kIssueMma) {
             tc_fence_after();
