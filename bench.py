@@ -205,7 +205,10 @@ class RawGdn:
         self.sr.gdn_replay(self.q, self.k, self.v, self.g, self.b, self.cu, max_seqlen=self.max_len,
                            o=self.o, s_out=self.s, ws=self.ws)
 
-    launches_per_step = 1
+    @property
+    def launches_per_step(self):
+        # d = 128: the two-phase tcgen05 pair (prep, then the state chain); d = 64: one kernel
+        return 2 if self.d == 128 else 1
 
     def step_e2e(self):
         for h, d in zip(self.h_in, self.d_in):
@@ -674,7 +677,9 @@ def run_ours(args):
         launches = 0
         for pr in profs:
             for kind, t in pr.times():
-                launches += 2 if kind == "conv" else 1  # conv: conv_gates + conv_state kernels
+                # two kernels per event pair: conv (conv_gates + conv_state) and gdn (the
+                # two-phase prep + state chain)
+                launches += 2 if kind in ("conv", "gdn") else 1
                 tot[kind] = tot.get(kind, 0.0) + t
                 cnt[kind] = cnt.get(kind, 0) + 1
         busy = sum(tot.values())
