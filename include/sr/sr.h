@@ -348,9 +348,11 @@ SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, siz
  * nothing and computes exactly what sr_group_replay computes.
  *
  * Limit: a replay whose sr_group_replay_workspace() exceeds
- * SR_GROUP_NOALLOC_SCRATCH_BYTES is rejected with SR_ERR_WORKSPACE (about
- * 150 KB per token per group at hidden 2560 with SR_PREC_SPLIT, so one group
- * of up to ~210 tokens fits; ~110 KB and ~290 tokens with SR_PREC_BF16).
+ * SR_GROUP_NOALLOC_SCRATCH_BYTES is rejected with SR_ERR_WORKSPACE.  At
+ * hidden 2560, intermediate 9216 and 32 V heads a group takes about 170 KB
+ * per token with SR_PREC_SPLIT (157 KB with SR_PREC_SPLIT_FP8, 132 KB with
+ * SR_PREC_BF16) plus 1.3 MB per sequence for the gated-delta chunk images,
+ * so one sequence of up to 191 tokens fits (207 and 254).
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture.  Sharing: every call on a device uses the same

@@ -90,7 +90,7 @@ def test_noalloc_rejects_replays_too_large_for_the_array():
     s = W.LayerShape()
     fake = 0x100000
     import ctypes
-    L, G, T = 3, 1, 4096  # ~150 KB per token: far beyond 32 MiB
+    L, G, T = 3, 1, 4096  # ~170 KB per token: far beyond 32 MiB
     w_arr = (sr.LayerWeights * (G * L))(*[sr.LayerWeights(*([fake] * 11)) for _ in range(G * L)])
     o_arr = (sr.LayerOutputs * (G * L))(*[sr.LayerOutputs(fake, fake, None) for _ in range(G * L)])
     anc = (ctypes.c_void_p * G)(fake)
