@@ -21,11 +21,11 @@ constexpr int kTokBatch = 16;  // tokens staged per shared-memory batch
 
 template <int DK, typename Tin>
 __global__ void __launch_bounds__(kRows)
-gdn_seq_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
-               const float *__restrict__ g, const float *__restrict__ beta,
-               const int32_t *__restrict__ cu, const float *__restrict__ h0,
-               Tin *__restrict__ o, float *__restrict__ s_out, int total, int max_len,
-               int h_k, int h_v, int d_v, float scale, uint32_t *status) {
+gdn_token_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                 const float *__restrict__ g, const float *__restrict__ beta,
+                 const int32_t *__restrict__ cu, const float *__restrict__ h0,
+                 Tin *__restrict__ o, float *__restrict__ s_out, int total, int max_len,
+                 int h_k, int h_v, int d_v, float scale, uint32_t *status) {
     const int n = blockIdx.z, h = blockIdx.y;
     const int row = blockIdx.x * kRows + threadIdx.x;
     const int hk = h / (h_v / h_k);
@@ -108,7 +108,7 @@ gdn_seq_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *
 template <int DK, typename Tin>
 cudaError_t launch(const sr_gdn_args &a, float scale, uint32_t *status, cudaStream_t st) {
     dim3 grid(a.d_v / kRows, a.h_v, a.n_seqs);
-    gdn_seq_kernel<DK, Tin><<<grid, kRows, 0, st>>>(
+    gdn_token_kernel<DK, Tin><<<grid, kRows, 0, st>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k), static_cast<const Tin *>(a.v),
         a.g, a.beta, a.cu_seqlens, a.h0, static_cast<Tin *>(a.o), a.s_out, a.total_tokens,
         a.max_seqlen, a.h_k, a.h_v, a.d_v, scale, status);
