@@ -89,8 +89,9 @@ typedef enum sr_gdn_algo {
                                (bf16, d_k = d_v = 128), two phases: the state-free part
                                of every chunk (masks, (I + A)^{-1}, W) for all chunks at
                                once, then the per-sequence state chain.  Workspace grows
-                               by 40 KB per (64-token chunk slot, V head).               */
-    SR_GDN_TCGEN05_FUSED = 4 /* the same in one kernel per (sequence, V head), every
+                               by 40 KB per (chunk slot, V head), with
+                               floor(total_tokens / 64) + n_seqs slots.                  */
+    SR_GDN_TCGEN05_FUSED = 4, /* the same in one kernel per (sequence, V head), every
                                step of a chunk in order; no scratch                     */
 } sr_gdn_algo;
 
