@@ -233,28 +233,21 @@ class RawGdn:
                 "flop": self.flop_per_tok * self.tokens,
                 "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
 
-    def oracle_sample(self, stride=1, min_s=0.0):
-        """Bounded oracle run over every stride-th (sequence, head) unit,
-        repeated until min_s seconds have passed; returns (tokens/s of a full
-        layer, description, threads used)."""
+    def oracle_piece(self, i):
+        """One bounded piece of the oracle's work on this workload: every
+        (sequence, V head) unit u with u % stride == i % stride (the whole
+        replay when it is small, every 8th unit of the 8-suffix one).  Returns
+        the replayed tokens the piece stands for (its head-tokens / H_v) and a
+        description."""
         import oracle
         x = self.x
         n_units = x.n_seqs * self.hv
-        lens = x.lengths
-        units = list(range(0, n_units, stride))
-        reps, t0 = 0, time.perf_counter()
-        while True:
-            oracle.gdn_replay(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, units=units)
-            reps += 1
-            dt = time.perf_counter() - t0
-            if dt >= min_s:
-                break
-        head_tokens = sum(lens[u // self.hv] for u in units) * reps
-        tok_per_s = head_tokens / self.hv / dt
-        return tok_per_s, (f"{len(units)} of {n_units} (sequence, head) units x {reps} reps, "
-                           f"{head_tokens} head-tokens, {dt:.1f} s; tokens/s = head-tokens / H_v / s"), \
-            oracle.num_threads()
-
+        stride = 1 if self.tokens * self.hv * self.d * self.d < 2**26 else 8
+        units = list(range(i % stride, n_units, stride))
+        oracle.gdn_replay(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, units=units)
+        head_tokens = sum(x.lengths[u // self.hv] for u in units)
+        return head_tokens / self.hv, (f"{len(units)} of the {n_units} (sequence, V head) units per piece, "
+                                       f"fp64 token-by-token recurrence; tokens = head-tokens / H_v")
 
 
 class GroupReplay:
@@ -285,6 +278,11 @@ class GroupReplay:
             self.gis = [W.anchor_pool_group(n_pages * W.SPARSE_PER_PAGE, k, seed=0x5EED0005 + 1000 * rank + g)
                         for g in range(8)]
             self.block_table = W.block_table(n_pages, 0x5EED0005 + 1000 * rank)
+            # pool rows of the last k anchors (page-tail layout: anchor a sits in page
+            # a // 4, slot a % 4), for the oracle's pieces, which run without the library
+            n_anchors = n_pages * W.SPARSE_PER_PAGE
+            self.h_rows = [self.block_table[a // W.SPARSE_PER_PAGE] * W.SPARSE_PER_PAGE + a % W.SPARSE_PER_PAGE
+                           for a in range(n_anchors - k, n_anchors)]
             self.desc = (f"whole model, token-sparse anchors: 8 groups replay k = {k} anchors gathered from "
                          f"pools of {n_pages * W.SPARSE_PER_PAGE} (32K prefix, 4 per 64-token page, "
                          f"shuffled block table)")
@@ -299,28 +297,45 @@ class GroupReplay:
         self.tokens = sum(self.gis[0].lengths)
         T, H, I = self.tokens, s.hidden, s.inter
         C = 64
+        # chunk-64 convention per token and V head: with the output o,
+        # 2 (C (3 d_k + 2 d_v) + 3 d_k d_v); without it (the last layer in skip
+        # mode) 2 (C 3 d_k + 2 d_k d_v)
+        gdn_o = float(T) * s.h_v * 2 * (C * (3 * s.d_k + 2 * s.d_v) + 3 * s.d_k * s.d_v) * self.G
+        gdn_no_o = float(T) * s.h_v * 2 * (C * 3 * s.d_k + 2 * s.d_k * s.d_v) * self.G
         self.flop = {  # algorithmic flops of one launch (all groups)
             "gemm_in": 2.0 * T * H * s.proj_dim * self.G,
             "gemm_out": 2.0 * T * s.v_dim * H * self.G,
             "gemm_gateup": 2.0 * T * H * 2 * I * self.G,
             "gemm_down": 2.0 * T * I * H * self.G,
-            "gdn": float(T) * s.h_v * 2 * (C * (3 * s.d_k + 2 * s.d_v) + 3 * s.d_k * s.d_v) * self.G,
+            # the mean over the step's GDN launches: L - 1 with o, the last without
+            "gdn": ((self.L - 1) * gdn_o + gdn_no_o) / self.L,
         }
         full = (self.flop["gemm_in"] + self.flop["gemm_out"] + self.flop["gemm_gateup"] + self.flop["gemm_down"]
-                + self.flop["gdn"])
-        last = self.flop["gemm_in"] + self.flop["gdn"]
+                + gdn_o)
+        last = self.flop["gemm_in"] + gdn_no_o
         self.step_flop = (self.L - 1) * full + last  # skip mode
         # algorithmic bytes of one launch (all groups) for the HBM-bound layer kernels
         split = 1 if precision == "bf16" else 2  # k, v: bf16, or hi + lo bf16
         act_out = {"split": 4, "split_fp8": 3, "bf16": 2}[precision]  # projection operand bytes per element
         qd, vd = s.qk_dim, s.v_dim
+        # algorithmic bytes per launch of the HBM-bound layer kernels: the
+        # operation's own inputs and outputs in bf16 (gates fp32), whatever the
+        # arithmetic carries
         self.bytes = {
-            # p (fp32) of the conv channels and gate columns in; q, k, v (hi/lo) and g, beta out
+            # [q|k|v] pre-conv channels and the b, a columns in; q, k, v out; g, beta (fp32) out
+            "conv": float(T) * self.G * ((s.conv_dim + 2 * s.h_v) * 2 + (2 * qd + vd) * 2 + 2 * s.h_v * 4),
+            # x in, RMSNorm(x) w out
+            "row_prep": float(T) * self.G * (H * 2 + H * 2),
+            # o and z in, y out
+            "gated_norm": float(T) * self.G * (vd * 2 * 3),
+        }
+        # the bytes the kernels move in this precision mode: the in_proj output p is
+        # fp32, the residual stream fp32, projection operands hi + lo (or hi + fp8 lo),
+        # k and v hi + lo in the split modes
+        self.bytes_impl = {
             "conv": float(T) * self.G * ((s.conv_dim + 2 * s.h_v) * 4 + qd * 2 + (qd + vd) * 2 * split
-                                          + 2 * s.h_v * 4),
-            # x in (fp32), x * w out (hi/lo), r out
+                                         + 2 * s.h_v * 4),
             "row_prep": float(T) * self.G * (H * 4 + H * act_out + 4),
-            # o (bf16) and z (fp32) in, y (hi/lo) out
             "gated_norm": float(T) * self.G * (vd * 2 + vd * 4 + vd * act_out),
         }
         self.input_bytes = self.G * T * H * 2 + sum(
@@ -364,7 +379,7 @@ class GroupReplay:
             _, rows = sr.sparse_anchor_plan(W.SPARSE_PREFIX, page_size=W.SPARSE_PAGE,
                                             anchors_per_page=W.SPARSE_PER_PAGE, k_max=W.SPARSE_K_MAX, ratio=0.05,
                                             block_table=self.block_table)
-            assert len(rows) == self.tokens
+            assert len(rows) == self.tokens and list(rows) == self.h_rows
             self.h_index = torch.tensor(rows, dtype=torch.int32).pin_memory()
             self.index = self.h_index.to(dev)
             self.kw["anchor_index"] = self.index
@@ -432,33 +447,22 @@ class GroupReplay:
     def d2h_bytes(self):
         return sum(hs.numel() * 4 + hc.numel() * 2 for row in self.h_out for hs, hc in row)
 
-    def oracle_sample(self, stride=1, min_s=0.0, tokens=None):
-        """Bounded oracle run: the first layer (in_proj, conv, recurrence,
-        gated norm, out_proj, MLP) of group 0 over the first `tokens` tokens,
-        repeated until min_s seconds; scaled by algorithmic flops to the
-        tokens/s of the whole step."""
-        import numpy as np
-        import oracle
+    def oracle_piece(self, i):
+        """One bounded piece of the oracle's work on this workload: the whole
+        replay of group i % G (every layer in skip mode, as the step computes
+        it, over the whole suffix).  Returns the replayed tokens the piece
+        stands for (the suffix over G: a step replays every token through all
+        G groups, which have the same shapes) and a description."""
         from oracle import layers as OL
-        gi = self.gis[0]
-        T = self.tokens if tokens is None else min(tokens, self.tokens)
-        x = oracle._f64(gi.anchors[:T])  # sparse pools: the first T rows (the cost does not depend on which)
-        cu = np.array([0, T])
-        reps, t0 = 0, time.perf_counter()
-        while True:
-            OL.gdn_layer(x, gi.layers[0], cu, gi.shape)
-            reps += 1
-            dt = time.perf_counter() - t0
-            if dt >= min_s:
-                break
-        full_layer_flop_per_tok = sum(v for k, v in self.flop.items()) / self.G / self.tokens
-        sample_flop = full_layer_flop_per_tok * T * reps
-        step_flop_per_tok = self.step_flop / self.tokens
-        tok_per_s = sample_flop / dt / step_flop_per_tok
-        return tok_per_s, (f"group 0, layer 0 (full layer incl. MLP) over {T} tokens x {reps} reps in {dt:.1f} s, "
-                           f"scaled by algorithmic flops to the whole step "
-                           f"({step_flop_per_tok / 1e6:.0f} MFLOP per replayed token)"), oracle.num_threads()
-
+        g = i % self.G
+        gi = self.gis[g]
+        if self.sparse:
+            OL.group_replay(gi, "skip", anchor_index=self.h_rows)
+        else:
+            OL.group_replay(gi, "skip")
+        return self.tokens / self.G, (f"one whole group per piece (group i mod {self.G}: {self.L} layers, skip "
+                                      f"mode, {self.tokens} tokens), fp64 numpy layer math + C recurrence; "
+                                      f"tokens = suffix / {self.G} groups per piece")
 
 
 class Mamba2Replay:
@@ -538,24 +542,21 @@ class Mamba2Replay:
         return {"name": "mamba2_tc_kernel", "bound": "hbm", "flop": self.flop_per_tok * self.tokens,
                 "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
 
-    def oracle_sample(self, stride=1, min_s=0.0, units=16):
-        """Bounded oracle run over `units` (sequence, head) pairs spread over the
-        batch, repeated until min_s seconds; tokens/s of the whole workload."""
+    def oracle_piece(self, i, units=16):
+        """One bounded piece of the oracle's work on this workload: `units`
+        (sequence, head) pairs spread over the batch (offset by i).  Returns
+        the replayed tokens the piece stands for (head-tokens / H) and a
+        description."""
         import oracle
         m = self.m
         n_units = len(m.lengths) * self.H
-        us = list(range(0, n_units, max(1, n_units // units)))[:units]
-        reps, t0 = 0, time.perf_counter()
-        while True:
-            oracle.mamba2_replay(m.x, m.B, m.C, m.dt, m.A, m.cu_seqlens, units=us)
-            reps += 1
-            dt = time.perf_counter() - t0
-            if dt >= min_s:
-                break
-        head_tokens = sum(m.lengths[u // self.H] for u in us) * reps
-        return head_tokens / self.H / dt, (f"{len(us)} of {n_units} (sequence, head) units x {reps} reps, "
-                                           f"{head_tokens} head-tokens in {dt:.1f} s; tokens/s = head-tokens / H / s"), \
-            oracle.num_threads()
+        step = max(1, n_units // units)
+        us = list(range(i % step, n_units, step))[:units]
+        oracle.mamba2_replay(m.x, m.B, m.C, m.dt, m.A, m.cu_seqlens, units=us)
+        head_tokens = sum(m.lengths[u // self.H] for u in us)
+        return head_tokens / self.H, (f"{len(us)} of the {n_units} (sequence, head) units per piece, fp64 "
+                                      f"token-by-token recurrence; tokens = head-tokens / H")
+
 
 WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "group": GroupReplay, "mamba2": Mamba2Replay,
              "sparse_32k": GroupReplay,
@@ -624,6 +625,29 @@ def max_over_ranks(ms, world, device):
 def job_throughput(units_per_step_per_rank, world, steps, ms):
     """Whole-job throughput: the units every rank processed over the slowest rank's time."""
     return units_per_step_per_rank * world * steps / (ms / 1e3)
+
+
+def workload_config(args, wl, world):
+    """The `config` object of the JSON line, the same for both arms."""
+    return {"workload": args.workload, "desc": wl.desc, "tokens_per_step_per_gpu": wl.tokens,
+            "l2": f"inputs {wl.input_bytes / 2**20:.0f} MiB > L2, no flush",
+            "parallelism": f"dp{world} (independent replays per GPU)"}
+
+
+def oracle_rate(wl, min_s):
+    """The oracle on the host cores: pieces i = 0, 1, ... of the workload until
+    min_s seconds have passed; returns (replayed tokens/s, pieces, seconds,
+    description, threads)."""
+    import oracle
+    tok, i, t0 = 0.0, 0, time.perf_counter()
+    while True:
+        n, desc = wl.oracle_piece(i)
+        tok += n
+        i += 1
+        secs = time.perf_counter() - t0
+        if secs >= min_s:
+            break
+    return tok / secs, i, secs, desc, oracle.num_threads()
 
 
 def run_ours(args):
@@ -695,7 +719,9 @@ def run_ours(args):
                            frac=round(tf / peaks_.get("bf16_tflops_sustained", peaks_["bf16_tflops"]), 4))
             elif k in wl.bytes:
                 gbs = wl.bytes[k] / (per_launch / 1e3) / 1e9
-                ent.update(bound="hbm", achieved_gbs=round(gbs, 1), frac=round(gbs / peaks_["hbm_gbs"], 4))
+                gbs_impl = wl.bytes_impl[k] / (per_launch / 1e3) / 1e9
+                ent.update(bound="hbm", achieved_gbs=round(gbs, 1), frac=round(gbs / peaks_["hbm_gbs"], 4),
+                           achieved_gbs_impl=round(gbs_impl, 1), frac_impl=round(gbs_impl / peaks_["hbm_gbs"], 4))
             kernels[k] = ent
     else:
         launches = wl.launches_per_step * args.steps
@@ -763,18 +789,17 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, cores = wl.oracle_sample(stride=1, min_s=10.0)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+        v, pieces, secs, desc, cores = oracle_rate(wl, min_s=10.0)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{pieces} pieces in {secs:.1f} s, timed (no extrapolation): {desc}"}
 
     line = {
         "metric": "replayed tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, workloads.py)",
-        "config": {"workload": args.workload, "desc": wl.desc, "tokens_per_step_per_gpu": wl.tokens,
-                   "precision": getattr(wl, "precision", "bf16 inputs"),
-                   "l2": f"inputs {wl.input_bytes / 2**20:.0f} MiB > L2, no flush",
-                   "parallelism": f"dp{world} (independent replays per GPU)"},
+        "config": workload_config(args, wl, world),
+        "precision": getattr(wl, "precision", "bf16 inputs"),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "serial_value": e2e_serial,
                 "copies": "overlapped with the replay (two buffer sets, copy streams)" if hasattr(wl, "e2e_inputs")
                 else "serialised with the replay", "h2d_bytes_per_step": wl.h2d_bytes,
@@ -796,26 +821,34 @@ def run_ours(args):
 
 
 def run_reference(args):
+    """The fp64 oracle as the reference arm: each step is one bounded piece of
+    the oracle's work on the workload (a whole group for the group workloads),
+    timed as it runs; the value is the replayed tokens the pieces stand for
+    over the time they took."""
     world, rank, local = dist_setup()
     if rank != 0:
         return
     wl = make_workload(args, 0)
-    kw = dict(stride=8) if isinstance(wl, RawGdn) else (dict(units=2) if isinstance(wl, Mamba2Replay)
-                                                        else dict(tokens=96))
-    for _ in range(args.warmup):
-        wl.oracle_sample(**kw)
-    vals = []
-    for _ in range(args.steps):
-        v, sample, cores = wl.oracle_sample(**kw)
-        vals.append(v)
-    value = statistics.mean(vals)
+    for i in range(args.warmup):
+        wl.oracle_piece(i)
+    tok, secs = 0.0, []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        n, desc = wl.oracle_piece(i)
+        secs.append(time.perf_counter() - t0)
+        tok += n
+    value = tok / sum(secs)
+    import oracle
+    cores = oracle.num_threads()
     line = {"impl": "reference", "metric": "replayed tokens/s", "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": wl.tokens / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1e3 * sum(secs) / len(secs), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, workloads.py)",
-            "config": {"workload": args.workload, "desc": wl.desc, "tokens_per_step_per_gpu": wl.tokens},
+            "config": workload_config(args, wl, world),
+            "precision": "fp64 (the oracle)",
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": f"one piece per step, {args.steps} pieces in {sum(secs):.1f} s, timed "
+                                       f"(no extrapolation): {desc}"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 

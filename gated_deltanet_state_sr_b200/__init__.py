@@ -317,6 +317,27 @@ def test_gemm(a, b0, *, b1=None, r=None, epi=EPI_STORE, c=None, ws=None, stream=
     return c
 
 
+_test_wait = _sig("sr_test_wait_timeout", _i32, ctypes.c_uint64, _i32, _vp, ctypes.c_size_t, _vp)
+WAIT_LIMIT_NS = 500_000_000  # the kernels' own limit on one mbarrier wait
+
+
+def test_wait_timeout(limit_ns, *, arrive=False, device="cuda", stream=None):
+    """sr_test_wait_timeout: one CTA waits on an mbarrier with a limit of
+    limit_ns (nothing arrives unless `arrive`), frees its tensor memory and
+    exits.  Returns (status flags, the wait's duration in ns) after a sync."""
+    torch = _torch()
+    ws = workspace(256, device)
+    _check(_test_wait(int(limit_ns), 1 if arrive else 0, _ptr(ws), ws.numel(), _stream_handle(stream)))
+    flags = device_status(ws, stream)
+    elapsed = int(ws[8:16].cpu().view(torch.int64).item())
+    return flags, elapsed
+
+
+def test_wait_call(limit_ns, arrive=0):
+    """Raw C call with no workspace (returns the sr_status; validation only)."""
+    return int(_test_wait(int(limit_ns), int(arrive), None, 0, None))
+
+
 # ------------------------------------------------------------------ group replay
 
 SR_PREC_SPLIT, SR_PREC_BF16, SR_PREC_SPLIT_FP8 = 0, 1, 2

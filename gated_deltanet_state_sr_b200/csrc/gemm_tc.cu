@@ -87,13 +87,16 @@ __device__ __forceinline__ uint2 lo8_pack8(const float (&lo)[8]) {
     return make_uint2(w[0], w[1]);
 }
 
-// Abort-aware bounded wait: gives up when another role has aborted.
+// Abort-aware bounded wait: gives up after tc::kWaitLimitNs, or as soon as
+// another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, volatile int *abort_flag) {
-    for (uint32_t i = 0; i < tc::kMaxPolls; ++i) {
-        if (tc::mbar_try_wait(bar, phase)) return true;
-        if ((i & 1023) == 1023 && *abort_flag) return false;
+    if (tc::mbar_try_wait(bar, phase)) return true;
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (tc::mbar_try_wait(bar, phase)) return true;
+        if (*abort_flag || tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) return false;
     }
-    return false;
 }
 
 template <int BN>

@@ -26,18 +26,29 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the array on the current device, looked up once per device.
-sr_status scratch_on_current_device(void **out) {
+// Device address of the array on the current device.  Outside a stream
+// capture it is looked up on every call, so a module that was reloaded (after
+// cudaDeviceReset, say) is found at its new address; inside a capture, where
+// a lookup might have to load the module, the address of the last call on this
+// device outside a capture is used.
+sr_status scratch_on_current_device(cudaStream_t stream, void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_error(e, "sr_group_replay_noalloc: cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return set_error(SR_ERR_UNSUPPORTED, "device index %d too large", dev);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return cuda_error(e, "sr_group_replay_noalloc: cudaStreamIsCapturing");
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_error(e, "sr_group_replay_noalloc: cudaGetSymbolAddress");
         g_scratch_ptr[dev] = p;
+    } else if (!g_scratch_ptr[dev]) {
+        return set_error(SR_ERR_INVALID_ARG,
+                         "sr_group_replay_noalloc: the first call on a device must come before any stream "
+                         "capture (it looks up the scratch array's device address)");
     }
     *out = g_scratch_ptr[dev];
     return SR_OK;
@@ -57,7 +68,7 @@ extern "C" sr_status sr_group_replay_noalloc(const sr_group_args *a, void *strea
                          "holds %zu; call sr_group_replay with a caller workspace instead",
                          need, size_t(SR_GROUP_NOALLOC_SCRATCH_BYTES));
     void *scratch = nullptr;
-    if (sr_status s = scratch_on_current_device(&scratch)) return s;
+    if (sr_status s = scratch_on_current_device(static_cast<cudaStream_t>(stream), &scratch)) return s;
     if (status_scratch) *status_scratch = scratch;
     // sr_group_replay clears the status word at the start of the array; every
     // other scratch byte is written before it is read within the call.

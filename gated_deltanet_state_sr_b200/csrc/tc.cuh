@@ -11,9 +11,18 @@
 namespace sr {
 namespace tc {
 
-// Upper bound on polls of one mbarrier wait before the kernel gives up and
-// reports SR_DEV_TIMEOUT (a healthy wait completes in microseconds).
-constexpr uint32_t kMaxPolls = 1u << 26;
+// Time limit of one mbarrier wait before the kernel gives up and reports
+// SR_DEV_TIMEOUT.  A healthy wait ends within one kernel's run time (at most
+// a few milliseconds here), so half a second only ever expires on a real
+// stall, and then the caller learns of it within about a second.
+constexpr uint64_t kWaitLimitNs = 500ull * 1000 * 1000;
+
+// The GPU's global nanosecond timer.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -48,11 +57,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     return ok != 0;
 }
 // Waits for the phase with parity `phase` to complete.  Returns false (and
-// leaves the barrier alone) after kMaxPolls unsuccessful polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(bar, phase)) return true;
-    return false;
+// leaves the barrier alone) once limit_ns nanoseconds of the global timer have
+// passed without it.  The timer is read only after a first unsuccessful poll,
+// and then once every 32 polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, phase)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, phase)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // ---------------------------------------------------------------- TMA

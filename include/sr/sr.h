@@ -354,9 +354,11 @@ SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, siz
  * per token with SR_PREC_SPLIT (157 KB with SR_PREC_SPLIT_FP8, 132 KB with
  * SR_PREC_BF16) plus 1.3 MB per sequence for the gated-delta chunk images,
  * so one sequence of up to 191 tokens fits (207 and 254).
- * Set-up: the first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Sharing: every call on a device uses the same
+ * Set-up: a call made outside a stream capture looks up the array's device
+ * address on the current device (cudaGetSymbolAddress), so the first call on
+ * a device must come before any stream capture; a call inside a capture
+ * reuses the address found by the last call outside one on that device (and
+ * fails with SR_ERR_INVALID_ARG if there was none).  Sharing: every call on a device uses the same
  * array, which keeps the previous call's contents, so calls whose kernels
  * overlap on the GPU (for example on two streams) race; serialise them.
  * status_scratch (may be NULL) receives the array's device address, which

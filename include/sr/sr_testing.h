@@ -27,6 +27,21 @@ SR_API sr_status sr_test_gemm(const void *a, const void *b0, const void *b1, voi
                               int32_t m, int32_t n, int32_t k, int32_t epi, void *workspace,
                               size_t workspace_bytes, void *stream);
 
+/* A bounded on-chip wait made to run out.  The paper has no counterpart: this
+ * checks the library's own failure detection.  Every tcgen05 / TMA kernel
+ * waits on mbarriers with a time limit (half a second), after which it sets
+ * SR_DEV_TIMEOUT in the status word, frees its tensor memory and returns.
+ * This call launches one CTA that allocates 128 tensor-memory columns, waits
+ * on an mbarrier through the same wait with the given limit_ns (0 < limit_ns
+ * <= the kernels' own limit, else SR_ERR_INVALID_ARG), then frees the tensor
+ * memory and exits.  With arrive == 0 nothing arrives at the barrier, so the
+ * wait runs out and SR_DEV_TIMEOUT is set; with arrive != 0 the CTA's first
+ * thread arrives before waiting, so the wait completes and no flag is set.
+ * The workspace (>= 256 bytes, 256-byte aligned) receives the status word at
+ * offset 0 and the wait's duration in nanoseconds (uint64) at offset 8. */
+SR_API sr_status sr_test_wait_timeout(uint64_t limit_ns, int32_t arrive, void *workspace, size_t workspace_bytes,
+                                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -12,11 +12,23 @@ FAKE = 0x10000  # an aligned, never-dereferenced address: validation fails first
 
 
 def test_exports_every_declared_symbol():
-    names = sr.declared_symbols()
-    assert {"sr_gdn_replay", "sr_group_replay", "sr_mamba2_replay", "sr_last_error",
-            "sr_device_status"} <= set(names)
+    import glob
+    import os
+    headers = sorted(glob.glob(os.path.join(os.path.dirname(sr.HEADER_PATH), "*.h")))
+    assert len(headers) >= 2
+    names = sorted({n for h in headers for n in sr.declared_symbols(h)})
+    assert {"sr_gdn_replay", "sr_group_replay", "sr_mamba2_replay", "sr_last_error", "sr_device_status",
+            "sr_group_replay_noalloc", "sr_test_gemm", "sr_test_wait_timeout"} <= set(names)
     for n in names:
         assert hasattr(sr.library(), n), f"libsr.so does not export {n}"
+
+
+def test_wait_timeout_validation():
+    """The test-only bounded-wait entry point refuses a zero limit, a limit
+    above the kernels' own, and a missing workspace, before any CUDA call."""
+    assert sr.test_wait_call(0) == sr.SR_ERR_INVALID_ARG
+    assert sr.test_wait_call(sr.WAIT_LIMIT_NS + 1) == sr.SR_ERR_INVALID_ARG
+    assert sr.test_wait_call(10_000) == sr.SR_ERR_WORKSPACE
 
 
 def test_version():

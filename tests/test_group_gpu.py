@@ -108,11 +108,24 @@ def test_group_parallel_equals_single(sr):
 
 def test_full_group_workload(sr):
     """The replay-group workload at full size: 3 layers, hidden 2560,
-    intermediate 9216, 16/32 heads, 1638-token suffix, skip mode."""
+    intermediate 9216, 16/32 heads, 1638-token suffix, skip mode; the states,
+    conv states and the hiddens after layers 1 and 2 against the oracle."""
     gi = W.group()
-    out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT)
+    out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT, want_hidden=True)
     ref = OL.group_replay(gi, "skip")
-    check_group(out[0], ref, STATE_TOL, "skip", False)
+    check_group(out[0], ref, STATE_TOL, "skip", True)
+    assert out[0][0][2] is not None and out[0][1][2] is not None
+
+
+def test_full_group_workload_full_mode(sr):
+    """The same group at full size in full mode (every layer to its MLP), in
+    the fp8-low-pass precision: all three layers' states and hiddens, the last
+    hidden included, against the oracle."""
+    gi = W.group()
+    out = run(sr, [gi], sr.SR_MODE_FULL, sr.SR_PREC_SPLIT_FP8, want_hidden=True)
+    ref = OL.group_replay(gi, "full")
+    check_group(out[0], ref, STATE_TOL, "full", True)
+    assert all(out[0][l][2] is not None for l in range(3))
 
 
 def test_prepare_lo8_matches_the_e5m2_format(sr):
@@ -135,20 +148,29 @@ def test_small_ragged_group_fp8_low_pass(sr, mode):
 
 def test_full_group_workload_fp8_low_pass(sr):
     """The full replay-group workload with the projections' low pass on the fp8
-    tensor cores, at the same state tolerance as the exact split."""
+    tensor cores, at the same state tolerance as the exact split; the hiddens
+    of layers 1 and 2 at the output tolerance."""
     gi = W.group()
-    out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8)
+    out = run(sr, [gi], sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8, want_hidden=True)
     ref = OL.group_replay(gi, "skip")
-    check_group(out[0], ref, STATE_TOL, "skip", False)
+    check_group(out[0], ref, STATE_TOL, "skip", True)
 
 
-@pytest.mark.parametrize("prefix,ratio", [(8192, 0.05), (32768, 0.05)])
-def test_whole_model_groups_0_and_7(sr, prefix, ratio):
+# Whole-model cases: every replay length k = ceil(r m) of the 8K/16K/32K
+# prefixes at 5 % and 10 % ("Tail-Replay", Sec. 3 and 4): 410, 820 (16K at 5 %
+# and 8K at 10 %), 1639 (32K at 5 % and 16K at 10 %) and 3277 (32K at 10 %).
+# Every group is checked where the oracle is quick; at the two longest
+# replays the first and the last group are, and the rest follow by the
+# bit-exact group independence test above.
+@pytest.mark.parametrize("prefix,ratio,checked", [
+    (8192, 0.05, range(8)), (16384, 0.05, range(8)), (32768, 0.05, (0, 7)), (32768, 0.10, (0, 7))])
+def test_whole_model_groups(sr, prefix, ratio, checked):
     """The whole-model replay (8 groups of 3 GDN layers, group-parallel, FA
-    skipped, suffix k = ceil(r m)) in the bench's default precision: all 8
-    groups in one call, the first and the last checked against the oracle."""
+    skipped) in the bench's default precision: all 8 groups in one call; the
+    checked groups' states, conv states and the hiddens of their first two
+    layers against the oracle."""
     gis = [W.model_group(prefix, ratio, g) for g in range(8)]
-    out = run(sr, gis, sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8)
-    for g in (0, 7):
+    out = run(sr, gis, sr.SR_MODE_SKIP, sr.SR_PREC_SPLIT_FP8, want_hidden=True)
+    for g in checked:
         ref = OL.group_replay(gis[g], "skip")
-        check_group(out[g], ref, STATE_TOL, "skip", False)
+        check_group(out[g], ref, STATE_TOL, "skip", True)
