@@ -207,8 +207,8 @@ class RawGdn:
 
     @property
     def launches_per_step(self):
-        # d = 128: the two-phase tcgen05 pair (prep, then the state chain); d = 64: one kernel
-        return 2 if self.d == 128 else 1
+        # the two-phase tcgen05 pair: the chunk-parallel prep, then the state chain
+        return 2
 
     def step_e2e(self):
         for h, d in zip(self.h_in, self.d_in):
@@ -226,10 +226,10 @@ class RawGdn:
         return self.h_o.numel() * self.h_o.element_size() + self.h_s.numel() * 4
 
     def dominant(self):
-        # the default algorithm: at d = 128 the two tcgen05 kernels of one replay (the
-        # chunk-parallel prep, then the per-sequence state chain), timed as the pair;
-        # the mma.sync kernel at d = 64
-        return {"name": "gdn_prep_kernel + gdn_seq_kernel" if self.d == 128 else "gdn_chunk_kernel", "bound": "tensor",
+        # the default algorithm: the two tcgen05 kernels of one replay (the chunk-parallel
+        # prep, then the per-sequence state chain), timed as the pair; at d = 64 they run
+        # on 128-wide tiles whose upper halves stay zero
+        return {"name": "gdn_prep_kernel + gdn_seq_kernel", "bound": "tensor",
                 "flop": self.flop_per_tok * self.tokens,
                 "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
 

@@ -47,7 +47,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int C = 64, D = 128;
+constexpr int C = 64;  // chunk length; every tile is 128 wide in the head dims (the state is 128 x 128 in TMEM)
 constexpr int kThreads = 256;
 constexpr int ROWA = C + 4;               // fp32 row pitch of A and T in the solve
 constexpr uint32_t SZ_AT = C * ROWA * 4;  // one fp32 64 x 64 matrix with padded rows
@@ -78,9 +78,11 @@ constexpr uint32_t IMG_T2H = 24576;  // T diag(beta), hi, K-major [t][s]
 constexpr uint32_t IMG_T2L = 32768;  // T diag(beta), lo
 constexpr uint32_t kImg = 40960;
 
-// prep kernel: K/Q (and Kl) tiles, then A and T fp32.  P and T2 hi reuse the
-// Q tiles once the first product has read them, T1 and T2 lo the A matrix
-// after the solve, -W^T the T matrix once T1 and T2 are formed.
+// prep kernel: K/Q (and Kl, right after them: the prep kernel reads no V) tiles,
+// then A and T fp32.  P and T2 hi reuse the Q tiles once the first product has
+// read them, T1 and T2 lo the A matrix after the solve, -W^T the T matrix once
+// T1 and T2 are formed.  Kl stays in place until W^T has been formed.
+constexpr uint32_t OFF_KL_PREP = 32768;
 constexpr uint32_t kPrepIn[2] = {32768, 49152};
 constexpr uint32_t smem_prep(bool split) { return kPrepIn[split] + 2 * SZ_AT + SZ_MISC + 1024; }
 
@@ -112,6 +114,7 @@ struct GdnTcParams {
     const int32_t *cu;
     uint8_t *img;  // two-phase: chunk images [group][slot][V head][kImg]
     int total, max_len, h_k, h_v, n_seqs, slots;
+    int d;  // head dim d_k = d_v: 128, or 64 (the upper half of every 128-wide tile stays zero)
     float scale;
     uint32_t *status;
 };
@@ -211,7 +214,7 @@ __device__ __forceinline__ uint32_t fresh(uint32_t base) {
 // [K;Q] K^T -> R0 (rows 0-63: K K^T, rows 64-127: Q K^T); with split k also
 // [K;Q] Kl^T into R0 and Kl K^T into R1 (rows 0-63).  One thread issues.
 template <bool SPLIT>
-__device__ __forceinline__ void mma_kqk(uint32_t base, uint32_t R0, uint32_t R1) {
+__device__ __forceinline__ void mma_kqk(uint32_t base, uint32_t R0, uint32_t R1, uint32_t kl_off = OFF_KL) {
     base = fresh(base);
     const uint64_t dk = sdesc_sw128(base + OFF_KQ, 16, 1024);
 #pragma unroll
@@ -220,7 +223,7 @@ __device__ __forceinline__ void mma_kqk(uint32_t base, uint32_t R0, uint32_t R1)
         mma_bf16_ss(R0, a, a, ID_KK, k > 0);
     }
     if (SPLIT) {
-        const uint64_t dl = sdesc_sw128(base + OFF_KL, 16, 1024);
+        const uint64_t dl = sdesc_sw128(base + kl_off, 16, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const uint64_t a = dadd(dk, (k >> 2) * 16384 + (k & 3) * 32);
@@ -405,12 +408,12 @@ __device__ __forceinline__ void write_t12(uint8_t *sm, const float *Tf, const fl
     }
 }
 
-// W^T = K^T T1^T -> RW (split: + Kl^T T1^T).  One thread issues.
+// W^T = K^T T1^T -> RW (split: + Kl^T T1^T, the low part of K at kl_off).  One thread issues.
 template <bool SPLIT>
-__device__ __forceinline__ void mma_w(uint32_t base, uint32_t o1, uint32_t RW) {
+__device__ __forceinline__ void mma_w(uint32_t base, uint32_t o1, uint32_t RW, uint32_t kl_off = OFF_KL) {
     base = fresh(base);
     const uint64_t dk = sdesc_sw128(base + OFF_KQ, 16384, 1024);  // K as MN-major A (j blocks 16 KB apart)
-    const uint64_t dl = sdesc_sw128(base + OFF_KL, 8192, 1024);
+    const uint64_t dl = sdesc_sw128(base + kl_off, 8192, 1024);
     const uint64_t dt = sdesc_sw128(base + o1, 16, 1024);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -594,6 +597,7 @@ __device__ __forceinline__ void convert_u(uint8_t *sm, uint32_t xr_off, uint32_t
 // chunk is staged as a [t][i] tile (two 64-channel halves) at stage_off for one
 // TMA store; the ragged last chunk is stored element by element, so that no row
 // of the next sequence is touched.
+template <int DH>
 __device__ __forceinline__ void out_chunk(uint8_t *sm, uint32_t stage_off, uint32_t RO, uint32_t lane_off, int half,
                                           int row, __nv_bfloat16 *o, size_t tok0, int clen, size_t v_stride, int h,
                                           bool tile_store) {
@@ -613,35 +617,43 @@ __device__ __forceinline__ void out_chunk(uint8_t *sm, uint32_t stage_off, uint3
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int t = 32 * half + e;
-            if (t < clen) o[(tok0 + t) * v_stride + size_t(h) * D + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
+            if (t < clen && row < 64 * DH)
+                o[(tok0 + t) * v_stride + size_t(h) * (64 * DH) + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
         }
     }
 }
 
 // Initial state (h0, or zero) into TMEM RS: thread -> row `row`, its column half.
+// With DH = 1 (d = 64) h0 is [64][64] and the rest of the 128 x 128 state is zero.
+template <int DH>
 __device__ __forceinline__ void state_init(uint32_t RS, uint32_t lane_off, int half, int row, const float *h0,
                                            size_t sbase) {
+    constexpr int d = 64 * DH;
     uint32_t r[32];
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
         const int j0 = 64 * half + 32 * part;
+        const bool in = h0 && row < d && j0 < d;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(h0 ? h0[sbase + size_t(row) * D + j0 + e] : 0.f);
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(in ? h0[sbase + size_t(row) * d + j0 + e] : 0.f);
         tmem_st_32x32b_x32(RS + lane_off + j0, r);
     }
     tmem_st_wait();
 }
 
-// Final state TMEM RS -> s_out.
+// Final state TMEM RS -> s_out (the d x d block of it).
+template <int DH>
 __device__ __forceinline__ void state_out(uint32_t RS, uint32_t lane_off, int half, int row, float *s_out,
                                           size_t sbase) {
+    constexpr int d = 64 * DH;
     uint32_t r[32];
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
         const int j0 = 64 * half + 32 * part;
         tmem_ld_32x32b_x32(RS + lane_off + j0, r);
         tmem_ld_wait();
-        float4 *dst = reinterpret_cast<float4 *>(s_out + sbase + size_t(row) * D + j0);
+        if (row >= d || j0 >= d) continue;
+        float4 *dst = reinterpret_cast<float4 *>(s_out + sbase + size_t(row) * d + j0);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
@@ -650,15 +662,17 @@ __device__ __forceinline__ void state_out(uint32_t RS, uint32_t lane_off, int ha
 }
 
 // Copies h0 (or zeros) to s_out for an empty sequence.
+template <int DH>
 __device__ __forceinline__ void state_passthrough(const float *h0, float *s_out, size_t sbase, int tid) {
-    for (int e = tid; e < D * D / 4; e += kThreads) {
+    constexpr int d = 64 * DH;
+    for (int e = tid; e < d * d / 4; e += kThreads) {
         const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
         reinterpret_cast<float4 *>(s_out + sbase)[e] = v;
     }
 }
 
 // ---------------------------------------------------------------- fused form
-template <bool SPLIT>
+template <bool SPLIT, int DH>
 __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -691,12 +705,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     const int len = eos - bos;
     const int nchunks = (len + C - 1) / C;
-    const size_t sbase = (size_t(n) * h_v + h) * D * D;
+    constexpr int d = 64 * DH;
+    const size_t sbase = (size_t(n) * h_v + h) * d * d;
     const float *h0 = p.h0[gi];
     float *s_out = p.s_out[gi];
 
     if (nchunks == 0) {  // empty sequence: the state is h0 (or zero)
-        state_passthrough(h0, s_out, sbase, tid);
+        state_passthrough<DH>(h0, s_out, sbase, tid);
         return;
     }
 
@@ -707,6 +722,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
         mbar_init(bar_mma, 1);
         *abort_flag = 0;
         fence_mbar_init();
+    }
+    if (DH == 1) {  // d = 64: the upper halves of the K, Q and V tiles are never loaded and stay zero
+        for (int e = tid; e < 3 * 512; e += kThreads) {
+            const uint32_t tile = e < 512 ? OFF_KQ + 16384 : (e < 1024 ? OFF_KQ + 24576 : OFF_V + 8192);
+            *reinterpret_cast<uint4 *>(sm + tile + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -719,35 +741,35 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const uint32_t R0 = tmem, R1 = tmem + 64, R2 = tmem + 128, R3 = tmem + 256;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    state_init(R2, lane_off, half, row, h0, sbase);
+    state_init<DH>(R2, lane_off, half, row, h0, sbase);
 
     const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const CUtensorMap *mo = &p.om[gi];
     // Each input is refilled as soon as the last product reading it has completed.
     auto issue_k = [&](int c) {
         const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_k, SPLIT ? 32768u : 16384u);
-        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * D, y);
-        tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * D + 64, y);
+        mbar_arrive_expect_tx(bar_k, DH * (SPLIT ? 16384u : 8192u));
+        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * d, y);
+        if (DH == 2) tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * d + 64, y);
         if (SPLIT) {
-            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * D, y);
-            tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * D + 64, y);
+            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * d, y);
+            if (DH == 2) tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * d + 64, y);
         }
     };
     auto issue_q = [&](int c) {
         const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_q, 16384u);
-        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * D, y);
-        tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * D + 64, y);
+        mbar_arrive_expect_tx(bar_q, DH * 8192u);
+        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * d, y);
+        if (DH == 2) tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * d + 64, y);
     };
     auto issue_v = [&](int c) {
         const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_v, SPLIT ? 32768u : 16384u);
-        tma_load_2d(sm + OFF_V, mv, bar_v, h * D, y);
-        tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * D + 64, y);
+        mbar_arrive_expect_tx(bar_v, DH * (SPLIT ? 16384u : 8192u));
+        tma_load_2d(sm + OFF_V, mv, bar_v, h * d, y);
+        if (DH == 2) tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * d + 64, y);
         if (SPLIT) {
-            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * D, y);
-            tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * D + 64, y);
+            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * d, y);
+            if (DH == 2) tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * d + 64, y);
         }
     };
     if (tid == 0) {
@@ -762,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const float *gh = p.g[gi] + size_t(bos) * h_v + h;
     const float *bh = p.beta[gi] + size_t(bos) * h_v + h;
     __nv_bfloat16 *o = p.o[gi];
-    const size_t v_stride = size_t(h_v) * D;
+    const size_t v_stride = size_t(h_v) * d;
     const float scale = p.scale;
     uint32_t kq_phase = 0, v_phase = 0, mma_phase = 0;
     float g_next = 0.f, b_next = 0.f;  // gates of the next chunk (threads tid < C)
@@ -885,13 +907,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
         // ---- o_t (bf16) through the (now free) Qg region
         const bool tile_store = o != nullptr && clen == C;
-        if (o) out_chunk(sm, oQG, R3, lane_off, half, row, o, size_t(bos) + size_t(c) * C, clen, v_stride, h, tile_store);
+        if (o) out_chunk<DH>(sm, oQG, R3, lane_off, half, row, o, size_t(bos) + size_t(c) * C, clen, v_stride, h, tile_store);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0 && tile_store) {
-            tma_store_2d(mo, sm + oQG, h * D, bos + c * C);
-            tma_store_2d(mo, sm + oQG + 8192, h * D + 64, bos + c * C);
+            tma_store_2d(mo, sm + oQG, h * d, bos + c * C);
+            if (DH == 2) tma_store_2d(mo, sm + oQG + 8192, h * d + 64, bos + c * C);
             bulk_commit();
         }
     }
@@ -899,7 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
     __syncthreads();
     if (*abort_flag == 0) {
-        state_out(R2, lane_off, half, row, s_out, sbase);
+        state_out<DH>(R2, lane_off, half, row, s_out, sbase);
     } else if (tid == 0) {
         atomicOr(p.status, SR_DEV_TIMEOUT);
         // let in-flight MMAs and TMA copies finish before tensor memory and shared memory are released
@@ -918,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 // ---------------------------------------------------------------- two-phase form: prep
 // One CTA per (chunk slot, V head, group).  Slots between two sequences' chunks
 // (at most one per sequence) exit at once.
-template <bool SPLIT>
+template <bool SPLIT, int DH>
 __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -968,15 +990,25 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         mbar_init(bar_mma, 1);
         fence_mbar_init();
         const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mkl = &p.kl[gi];
-        mbar_arrive_expect_tx(bar_in, SPLIT ? 49152u : 32768u);
-        tma_load_2d(sm + OFF_KQ, mk, bar_in, hk * D, y);
-        tma_load_2d(sm + OFF_KQ + 16384, mk, bar_in, hk * D + 64, y);
-        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_in, hk * D, y);
-        tma_load_2d(sm + OFF_KQ + 24576, mq, bar_in, hk * D + 64, y);
-        if (SPLIT) {
-            tma_load_2d(sm + OFF_KL, mkl, bar_in, hk * D, y);
-            tma_load_2d(sm + OFF_KL + 8192, mkl, bar_in, hk * D + 64, y);
+        constexpr int d = 64 * DH;
+        mbar_arrive_expect_tx(bar_in, DH * (SPLIT ? 24576u : 16384u));
+        tma_load_2d(sm + OFF_KQ, mk, bar_in, hk * d, y);
+        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_in, hk * d, y);
+        if (DH == 2) {
+            tma_load_2d(sm + OFF_KQ + 16384, mk, bar_in, hk * d + 64, y);
+            tma_load_2d(sm + OFF_KQ + 24576, mq, bar_in, hk * d + 64, y);
         }
+        if (SPLIT) {
+            tma_load_2d(sm + OFF_KL_PREP, mkl, bar_in, hk * d, y);
+            if (DH == 2) tma_load_2d(sm + OFF_KL_PREP + 8192, mkl, bar_in, hk * d + 64, y);
+        }
+    }
+    if (DH == 1) {  // d = 64: the upper halves of the K and Q tiles are never loaded and stay zero
+        for (int e = tid; e < 2 * 512; e += kThreads) {
+            const uint32_t tile = e < 512 ? OFF_KQ + 16384 : OFF_KQ + 24576;
+            *reinterpret_cast<uint4 *>(sm + tile + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
     }
     float g0 = 0.f, b0 = 0.f;  // padding has g = beta = 0
     if (tid < clen) {
@@ -1015,7 +1047,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         // ---- [K;Q] K^T, then A and P
         if (tid == 0) {
             tc_fence_after();
-            mma_kqk<SPLIT>(base, R0, R1);
+            mma_kqk<SPLIT>(base, R0, R1, OFF_KL_PREP);
             mma_commit(bar_mma);
         }
         const bool w = mbar_wait(bar_mma, mma_phase);
@@ -1038,7 +1070,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            mma_w<SPLIT>(base, oT1, R0);
+            mma_w<SPLIT>(base, oT1, R0, OFF_KL_PREP);
             mma_commit(bar_mma);
             bulk_store(dst + IMG_T2H, sm + oT2H, 8192);
             bulk_store(dst + IMG_T2L, sm + oT2L, 8192);
@@ -1075,13 +1107,14 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 // ---------------------------------------------------------------- two-phase form: sequential
 // o_t (bf16) of one chunk straight from TMEM RO to global memory: a warp stores
 // one token's 32 consecutive value channels per instruction (64 contiguous bytes).
+template <int DH>
 __device__ __forceinline__ void out_direct(uint32_t RO, uint32_t lane_off, int half, int row, __nv_bfloat16 *o,
                                            size_t tok0, int clen, size_t v_stride, int h) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(RO + lane_off + 32 * half, r);
     tmem_ld_wait();
-    __nv_bfloat16 *dst = o + (tok0 + size_t(32 * half)) * v_stride + size_t(h) * D + row;
-    const int n_out = min(32, clen - 32 * half);
+    __nv_bfloat16 *dst = o + (tok0 + size_t(32 * half)) * v_stride + size_t(h) * (64 * DH) + row;
+    const int n_out = row < 64 * DH ? min(32, clen - 32 * half) : 0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         if (e < n_out) *dst = __float2bfloat16_rn(__uint_as_float(r[e]));
@@ -1096,7 +1129,7 @@ __device__ __forceinline__ void out_direct(uint32_t RO, uint32_t lane_off, int h
 // products: o of chunk c-1 is written while the first group of products of c
 // runs (O alternates between two TMEM accumulators), and the gates and Qg of
 // chunk c+1 are formed while the state update of c runs.
-template <bool SPLIT>
+template <bool SPLIT, int DH>
 __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1125,12 +1158,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     const int len = eos - bos;
     const int nchunks = (len + C - 1) / C;
-    const size_t sbase = (size_t(n) * h_v + h) * D * D;
+    constexpr int d = 64 * DH;
+    const size_t sbase = (size_t(n) * h_v + h) * d * d;
     const float *h0 = p.h0[gi];
     float *s_out = p.s_out[gi];
 
     if (nchunks == 0) {
-        state_passthrough(h0, s_out, sbase, tid);
+        state_passthrough<DH>(h0, s_out, sbase, tid);
         return;
     }
 
@@ -1144,6 +1178,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (DH == 1) {  // d = 64: the upper halves of the K, Q and V tiles are never loaded and stay zero
+        for (int e = tid; e < 3 * 512; e += kThreads) {
+            const uint32_t tile = e < 512 ? OFF_KQ + 16384 : (e < 1024 ? OFF_KQ + 24576 : OFF_V + 8192);
+            *reinterpret_cast<uint4 *>(sm + tile + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
+    }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -1156,7 +1197,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     const uint32_t RS = tmem, RO0 = tmem + 128, RO1 = tmem + 256;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    state_init(RS, lane_off, half, row, h0, sbase);
+    state_init<DH>(RS, lane_off, half, row, h0, sbase);
 
     const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const uint8_t *img = p.img + (size_t(gi) * p.slots * h_v + h) * kImg;
@@ -1165,28 +1206,28 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     // Q once Qg is formed, V, T2 and -W^T once U is, K and P after the update.
     auto issue_k = [&](int c) {
         const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_k, SPLIT ? 32768u : 16384u);
-        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * D, y);
-        tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * D + 64, y);
+        mbar_arrive_expect_tx(bar_k, DH * (SPLIT ? 16384u : 8192u));
+        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * d, y);
+        if (DH == 2) tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * d + 64, y);
         if (SPLIT) {
-            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * D, y);
-            tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * D + 64, y);
+            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * d, y);
+            if (DH == 2) tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * d + 64, y);
         }
     };
     auto issue_q = [&](int c) {
         const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_q, 16384u);
-        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * D, y);
-        tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * D + 64, y);
+        mbar_arrive_expect_tx(bar_q, DH * 8192u);
+        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * d, y);
+        if (DH == 2) tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * d + 64, y);
     };
     auto issue_v = [&](int c) {
         const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_v, SPLIT ? 32768u : 16384u);
-        tma_load_2d(sm + OFF_V, mv, bar_v, h * D, y);
-        tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * D + 64, y);
+        mbar_arrive_expect_tx(bar_v, DH * (SPLIT ? 16384u : 8192u));
+        tma_load_2d(sm + OFF_V, mv, bar_v, h * d, y);
+        if (DH == 2) tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * d + 64, y);
         if (SPLIT) {
-            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * D, y);
-            tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * D + 64, y);
+            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * d, y);
+            if (DH == 2) tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * d + 64, y);
         }
     };
     auto issue_w = [&](int c) {  // -W (its halves beside those of Qg), T2 hi, T2 lo
@@ -1212,7 +1253,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
 
     const float *gh = p.g[gi] + size_t(bos) * h_v + h;
     __nv_bfloat16 *o = p.o[gi];
-    const size_t v_stride = size_t(h_v) * D;
+    const size_t v_stride = size_t(h_v) * d;
     const float scale = p.scale;
     uint32_t k_phase = 0, q_phase = 0, v_phase = 0, w_phase = 0, p_phase = 0, mma_phase = 0;
 
@@ -1278,8 +1319,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         // ---- meanwhile: o of the previous chunk (warp 4 also takes warp 0's share)
         if (o && c > 0) {
             const size_t tok0 = size_t(bos) + size_t(c - 1) * C;
-            if (warp != 0) out_direct(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h);
-            if (warp == 4) out_direct(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h);
+            if (warp != 0) out_direct<DH>(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h);
+            if (warp == 4) out_direct<DH>(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h);
         }
         const bool m2 = wait_mma() && *abort_flag == 0;
         if (check(m2)) break;
@@ -1320,9 +1361,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     __syncthreads();
     if (*abort_flag == 0) {
         const int cl = nchunks - 1;
-        if (o) out_direct(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C, len - cl * C,
+        if (o) out_direct<DH>(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C, len - cl * C,
                           v_stride, h);
-        state_out(RS, lane_off, half, row, s_out, sbase);
+        state_out<DH>(RS, lane_off, half, row, s_out, sbase);
     } else if (tid == 0) {
         atomicOr(p.status, SR_DEV_TIMEOUT);
         mma_commit(bar_mma);
@@ -1342,23 +1383,25 @@ bool map_64x64(CUtensorMap *m, const void *base, int rows, int cols) {
     return make_map_bf16(m, base, rows, cols, cols, 64, 64);
 }
 
-template <bool SPLIT>
+template <bool SPLIT, int DH>
 cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t st) {
     if (!p.img) {
         const int smem = int(smem_fused(SPLIT));
-        cudaError_t e = cudaFuncSetAttribute(gdn_tc_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e =
+            cudaFuncSetAttribute(gdn_tc_kernel<SPLIT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        gdn_tc_kernel<SPLIT><<<dim3(p.h_v, n_seqs, n_groups), kThreads, smem, st>>>(p);
+        gdn_tc_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kThreads, smem, st>>>(p);
         return cudaGetLastError();
     }
     const int s1 = int(smem_prep(SPLIT)), s2 = int(smem_seq(SPLIT));
-    cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
+    cudaError_t e =
+        cudaFuncSetAttribute(gdn_prep_kernel<SPLIT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gdn_seq_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
+    e = cudaFuncSetAttribute(gdn_seq_kernel<SPLIT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return e;
-    gdn_prep_kernel<SPLIT><<<dim3(p.slots, p.h_v, n_groups), kThreads, s1, st>>>(p);
+    gdn_prep_kernel<SPLIT, DH><<<dim3(p.slots, p.h_v, n_groups), kThreads, s1, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_seq_kernel<SPLIT><<<dim3(p.h_v, n_seqs, n_groups), kThreads, s2, st>>>(p);
+    gdn_seq_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kThreads, s2, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -1366,17 +1409,20 @@ int image_slots(int total, int n_seqs) { return total / C + n_seqs; }
 
 }  // namespace
 
-bool gdn_tc_supported(int d) { return d == 128; }
+// d = 128 natively; d = 64 runs the same kernels with the upper half of every
+// 128-wide K, Q and V tile left at zero, which keeps the upper rows and
+// columns of the state, W and U at zero (split precision: d = 128 only).
+bool gdn_tc_supported(int d) { return d == 128 || d == 64; }
 
 size_t gdn_tc_image_bytes(int total, int n_seqs, int h_v, int n_groups) {
     return size_t(n_groups) * size_t(image_slots(total, n_seqs)) * size_t(h_v) * kImg;
 }
 
-cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split, cudaStream_t st) {
-    if (n_seqs == 0 || n_groups == 0 || b.total == 0) return gdn_chunked_batch(b, n_groups, n_seqs, 128, split, st);
-    if (b.h_v > 65535) return cudaErrorInvalidValue;
+cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st) {
+    if (n_seqs == 0 || n_groups == 0 || b.total == 0) return gdn_chunked_batch(b, n_groups, n_seqs, d, split, st);
+    if (b.h_v > 65535 || !gdn_tc_supported(d) || (split && d != 128)) return cudaErrorInvalidValue;
     GdnTcParams p{};
-    const int T = b.total, qkw = b.h_k * D, vw = b.h_v * D;
+    const int T = b.total, qkw = b.h_k * d, vw = b.h_v * d;
     for (int g = 0; g < n_groups; ++g) {
         if (!map_64x64(&p.q[g], b.q[g], T, qkw) || !map_64x64(&p.k[g], b.k[g], T, qkw) ||
             !map_64x64(&p.v[g], b.v[g], T, vw))
@@ -1398,9 +1444,11 @@ cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split
     p.h_v = b.h_v;
     p.n_seqs = n_seqs;
     p.slots = image_slots(b.total, n_seqs);
+    p.d = d;
     p.scale = b.scale;
     p.status = b.status;
-    return split ? launch<true>(p, n_groups, n_seqs, st) : launch<false>(p, n_groups, n_seqs, st);
+    if (split) return launch<true, 2>(p, n_groups, n_seqs, st);
+    return d == 128 ? launch<false, 2>(p, n_groups, n_seqs, st) : launch<false, 1>(p, n_groups, n_seqs, st);
 }
 
 cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, void *img, cudaStream_t st) {
@@ -1421,7 +1469,7 @@ cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, void *im
     b.h_v = a.h_v;
     b.scale = scale;
     b.status = status;
-    return gdn_tc_batch(b, 1, a.n_seqs, false, st);
+    return gdn_tc_batch(b, 1, a.n_seqs, a.d_k, false, st);
 }
 
 }  // namespace sr

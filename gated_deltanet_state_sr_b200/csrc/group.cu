@@ -290,7 +290,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         gb.cu = a->cu_seqlens; gb.img = img; gb.total = T; gb.max_len = a->max_seqlen; gb.h_k = m.hk; gb.h_v = m.hv;
         gb.scale = 1.0f / sqrtf(float(m.d)); gb.status = status;
         SR_TRY(prof.begin(SR_K_GDN));
-        SR_TRY(gdn_tc_supported(m.d) ? gdn_tc_batch(gb, G, m.N, m.split, st)
+        SR_TRY(gdn_tc_supported(m.d) ? gdn_tc_batch(gb, G, m.N, m.d, m.split, st)
                                      : gdn_chunked_batch(gb, G, m.N, m.d, m.split, st));
         SR_TRY(prof.end());
         if (stop) break;

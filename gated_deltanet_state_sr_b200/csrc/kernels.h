@@ -37,12 +37,13 @@ struct GdnBatch {
     uint32_t *status;
 };
 cudaError_t gdn_chunked_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st);
-// The same on tcgen05 with the state in tensor memory (d = 128; gdn_tc.cu).
+// The same on tcgen05 with the state in tensor memory (d = 128, or d = 64 on
+// half-zero tiles; gdn_tc.cu).
 bool gdn_tc_supported(int d);
 cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, void *img, cudaStream_t st);
 // Scratch of the two-phase form: one 40 KB chunk image per (group, chunk slot, V head).
 size_t gdn_tc_image_bytes(int total, int n_seqs, int h_v, int n_groups);
-cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, bool split, cudaStream_t st);
+cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st);
 
 // 2-D bf16 TMA map (128-byte swizzle) over a row-major [rows, cols] matrix with row pitch `pitch`.
 bool make_map_bf16(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_cols, int box_rows);

@@ -81,12 +81,12 @@ typedef enum sr_dtype { SR_BF16 = 0, SR_FP32 = 1 } sr_dtype;
 
 /* Kernel selection for sr_gdn_replay. */
 typedef enum sr_gdn_algo {
-    SR_GDN_AUTO = 0,        /* bf16: tcgen05 two-phase form for d = 128, mma.sync kernel
-                               for d = 64; fp32: sequential                              */
+    SR_GDN_AUTO = 0,        /* bf16: the tcgen05 two-phase form; fp32: sequential      */
     SR_GDN_SEQUENTIAL = 1,  /* token-by-token fp32 FFMA recurrence (any dtype)          */
     SR_GDN_CHUNKED = 2,     /* chunked WY/UT form, warp-level mma.sync (bf16 only)      */
     SR_GDN_TCGEN05 = 3,     /* chunked WY/UT form on tcgen05, state in tensor memory
-                               (bf16, d_k = d_v = 128), two phases: the state-free part
+                               (bf16; d = 64 runs on 128-wide tiles whose upper halves
+                               stay zero), two phases: the state-free part
                                of every chunk (masks, (I + A)^{-1}, W) for all chunks at
                                once, then the per-sequence state chain.  Workspace grows
                                by 40 KB per (chunk slot, V head), with

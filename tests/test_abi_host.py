@@ -80,9 +80,9 @@ def test_gdn_workspace_required():
 
 
 def test_gdn_two_phase_workspace_holds_the_chunk_images():
-    """The default tcgen05 form (d = 128) keeps one 40 KB chunk image per (chunk
-    slot, V head), with floor(T / 64) + n_seqs slots; the fused form and the
-    other kernels need only the 256-byte header."""
+    """The default tcgen05 form keeps one 40 KB chunk image per (chunk slot, V
+    head), with floor(T / 64) + n_seqs slots, at d = 128 and at d = 64 alike;
+    the fused form and the other kernels need only the 256-byte header."""
     kw = dict(d_k=128, d_v=128, h_k=16, h_v=32, n_seqs=8, total_tokens=8917, max_seqlen=2048)
     slots = 8917 // 64 + 8
     want = 256 + slots * 32 * 40960
@@ -90,10 +90,11 @@ def test_gdn_two_phase_workspace_holds_the_chunk_images():
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05, **kw)) == want
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED, **kw)) == 256
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_SEQUENTIAL, **kw)) == 256
-    # d = 64 takes the mma.sync kernel, which needs no scratch
-    assert sr.gdn_workspace_bytes(_gdn()) == 256
-    # the tcgen05 forms take bf16 at d = 128 only
-    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED)) == 0
+    # d = 64 (100 tokens, 2 sequences, 4 V heads) takes the two-phase form too
+    assert sr.gdn_workspace_bytes(_gdn()) == 256 + (100 // 64 + 2) * 4 * 40960
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_CHUNKED)) == 256
+    assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED)) == 256
+    # the tcgen05 forms take bf16 only
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED, dtype=sr.SR_FP32, **kw)) == 0
 
 

@@ -27,8 +27,6 @@ def sr():
 
 
 def run_gpu(sr, x: W.GdnInputs, algo, want_o=True, dev="cuda"):
-    if algo.startswith("tcgen05") and x.q.shape[-1] != 128:
-        pytest.skip("the tcgen05 kernel takes d = 128 only")
     t = lambda a: None if a is None else a.to(dev).contiguous()
     o, s = sr.gdn_replay(t(x.q), t(x.k), t(x.v), t(x.g), t(x.beta), t(x.cu_seqlens),
                          max_seqlen=max(x.max_seqlen, 1), h0=t(x.h0), want_o=want_o, algo=algo)
@@ -77,10 +75,11 @@ def test_edge_lengths_with_initial_state(sr, algo, d):
 
 
 @pytest.mark.parametrize("algo", ALGOS)
-def test_strong_decay(sr, algo):
+@pytest.mark.parametrize("d", [64, 128])
+def test_strong_decay(sr, algo, d):
     """Gates of the group workload: g down to about -11 per token, so the
     cumulative decay over a chunk leaves the fp32 exp range."""
-    x = W.gdn_inputs(5, [300, 77], 2, 4, 128, 128, g_range=(-12.0, -0.5), norm_q=True)
+    x = W.gdn_inputs(5, [300, 77], 2, 4, d, d, g_range=(-12.0, -0.5), norm_q=True)
     o, s = run_gpu(sr, x, algo)
     o_ref, s_ref = run_oracle(x)
     assert_close(s, s_ref, STATE_TOL, "state")
@@ -133,16 +132,15 @@ def test_bad_cu_seqlens_flagged_on_device(sr, algo):
 
 @pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("split_at", [64, 100])
-def test_exact_resume_on_gpu(sr, algo, split_at):
+@pytest.mark.parametrize("dh", [64, 128])
+def test_exact_resume_on_gpu(sr, algo, split_at, dh):
     """Continuation: replaying b from h0 = Replay(a) gives Replay(a || b) ("Sparse
     Prefix Caching for Hybrid and Recurrent LLM Serving", exactness of resume; the
     replayed state hands over to the continuing tokens).  Split on and off a chunk
     boundary."""
     T = 300
-    x = W.gdn_inputs(15, [T], 2, 4, 128, 128)
+    x = W.gdn_inputs(15, [T], 2, 4, dh, dh)
     d = lambda a: a.cuda().contiguous()
-    if algo.startswith("tcgen05") and x.q.shape[-1] != 128:
-        pytest.skip("d = 128 only")
     full_o, full_s = sr.gdn_replay(d(x.q), d(x.k), d(x.v), d(x.g), d(x.beta), d(x.cu_seqlens), max_seqlen=T,
                                    algo=algo)
     cu_a = torch.tensor([0, split_at], dtype=torch.int32, device="cuda")
@@ -173,15 +171,29 @@ def test_two_phase_matches_fused(sr):
     assert_close(o2, o1.double().cpu().numpy(), OUT_TOL_BF16 / 2, "o, two-phase vs fused")
 
 
+def test_default_path_at_d64_is_tcgen05(sr):
+    """The small raw workload (d = 64) runs the tcgen05 two-phase kernels by
+    default, on 128-wide tiles whose upper halves stay zero: it agrees with the
+    explicitly selected two-phase form bit for bit and with the mma.sync chunk
+    kernel to a small fraction of the oracle tolerance."""
+    x = W.raw_small()
+    o0, s0 = run_gpu(sr, x, "auto")
+    o1, s1 = run_gpu(sr, x, "tcgen05")
+    o2, s2 = run_gpu(sr, x, "chunked")
+    assert torch.equal(s0, s1) and torch.equal(o0, o1)
+    assert_close(s1, s2.double().cpu().numpy(), STATE_TOL / 4, "state, tcgen05 vs mma.sync")
+
+
 @pytest.mark.parametrize("algo", ["tcgen05", "tcgen05_fused"])
-def test_many_short_sequences(sr, algo):
+@pytest.mark.parametrize("d", [64, 128])
+def test_many_short_sequences(sr, algo, d):
     """More sequences than the longest-first ranking handles (300), lengths
     0..140 with empty ones between: every chunk finds its image slot."""
     gen = torch.Generator().manual_seed(31)
     lengths = torch.randint(0, 141, (300,), generator=gen).tolist()
     for i in range(0, 300, 37):
         lengths[i] = 0
-    x = W.gdn_inputs(31, lengths, 1, 2, 128, 128, h0_std=0.2)
+    x = W.gdn_inputs(31, lengths, 1, 2, d, d, h0_std=0.2)
     o, s = run_gpu(sr, x, algo)
     units = [n * 2 + h for n in range(0, 300, 7) for h in range(2)]
     o_ref, s_ref = run_oracle(x, units=units)
