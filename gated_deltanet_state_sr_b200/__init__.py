@@ -20,7 +20,12 @@ import os
 import re
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsr.so")
+# SR_LIBRARY=libsr_checked.so selects the bounds-checked build (the same
+# kernels with every global index checked into the device status word).
+_LIB_NAME = os.environ.get("SR_LIBRARY", "libsr.so")
+if _LIB_NAME not in ("libsr.so", "libsr_checked.so"):
+    raise ImportError(f"SR_LIBRARY must be libsr.so or libsr_checked.so, not {_LIB_NAME!r}")
+LIB_PATH = os.path.join(_HERE, _LIB_NAME)
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sr", "sr.h")
 
 if not os.path.exists(LIB_PATH):
@@ -33,7 +38,8 @@ SR_OK, SR_ERR_INVALID_ARG, SR_ERR_UNSUPPORTED, SR_ERR_WORKSPACE, SR_ERR_CUDA, SR
 SR_BF16, SR_FP32 = 0, 1
 SR_GDN_AUTO, SR_GDN_SEQUENTIAL, SR_GDN_CHUNKED, SR_GDN_TCGEN05, SR_GDN_TCGEN05_FUSED = 0, 1, 2, 3, 4
 SR_MODE_SKIP, SR_MODE_FULL = 0, 1
-SR_DEV_BAD_CU_SEQLENS, SR_DEV_SEQ_TOO_LONG, SR_DEV_TIMEOUT, SR_DEV_BAD_INDEX = 0x1, 0x2, 0x4, 0x8
+SR_DEV_BAD_CU_SEQLENS, SR_DEV_SEQ_TOO_LONG, SR_DEV_TIMEOUT, SR_DEV_BAD_INDEX, SR_DEV_BAD_ACCESS = 0x1, 0x2, 0x4, 0x8, 0x10
+CHECKED = _LIB_NAME == "libsr_checked.so"
 _ALGOS = {"auto": SR_GDN_AUTO, "sequential": SR_GDN_SEQUENTIAL, "chunked": SR_GDN_CHUNKED,
           "tcgen05": SR_GDN_TCGEN05, "tcgen05_fused": SR_GDN_TCGEN05_FUSED}
 
@@ -88,7 +94,8 @@ class GroupArgs(ctypes.Structure):
                 ("max_seqlen", _i32), ("hidden", _i32), ("inter", _i32), ("h_k", _i32), ("h_v", _i32),
                 ("d_k", _i32), ("d_v", _i32), ("conv_width", _i32), ("eps", ctypes.c_float),
                 ("mode", _i32), ("precision", _i32), ("profile", ctypes.POINTER(Profile)),
-                ("initial", ctypes.POINTER(LayerState)), ("anchor_index", _vp), ("anchor_rows", _i32)]
+                ("initial", ctypes.POINTER(LayerState)), ("anchor_index", _vp), ("anchor_rows", _i32),
+                ("layer_done", ctypes.POINTER(_vp))]
 
 
 def _sig(name, restype, *argtypes):
@@ -346,7 +353,7 @@ _LAYER_FIELDS = [f for f, _ in LayerWeights._fields_]
 
 def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, inter, h_k, h_v, d=128,
                conv_width=4, eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, profile=None,
-               initial=None, anchor_index=None, total_tokens=None):
+               initial=None, anchor_index=None, total_tokens=None, layer_done=None):
     """Builds a GroupArgs (and keeps the ctypes arrays alive on it).
 
     anchors: list [G] of [T, hidden] bf16 CUDA tensors (the anchor pools
@@ -354,7 +361,9 @@ def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, int
     weights: list [G] of lists [L] of objects with the sr_layer_weights field
     names (CUDA tensors); outputs: list [G] of lists [L] of (s_out, conv_out,
     hidden_out-or-None); initial: None or list [G] of lists [L] of
-    (s_in-or-None, conv_in-or-None) to continue from."""
+    (s_in-or-None, conv_in-or-None) to continue from; layer_done: None or a
+    list [L] of torch.cuda.Event (or None), each recorded once that layer's
+    states are final."""
     G, L = len(anchors), len(weights[0])
     init_arr = None
     if initial is not None:
@@ -384,7 +393,15 @@ def group_args(anchors, cu_seqlens, weights, outputs, *, max_seqlen, hidden, int
                   ctypes.pointer(profile.struct) if profile is not None else None,
                   init_arr, None if anchor_index is None else anchor_index.data_ptr(),
                   0 if anchor_index is None else anchors[0].shape[0])
-    a._keep = (anc, w_arr, o_arr, profile, init_arr)
+    ev_arr = None
+    if layer_done is not None:
+        assert len(layer_done) == L
+        for e in layer_done:
+            if e is not None and e.cuda_event == 0:
+                e.record()  # torch creates the CUDA event lazily, at its first record
+        ev_arr = (_vp * L)(*[None if e is None else e.cuda_event for e in layer_done])
+        a.layer_done = ev_arr
+    a._keep = (anc, w_arr, o_arr, profile, init_arr, ev_arr)
     return a
 
 
@@ -418,7 +435,7 @@ def group_call(args: GroupArgs, ws, stream=None) -> int:
 
 def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k, h_v, d=128, conv_width=4,
                  eps=1e-6, mode=SR_MODE_SKIP, precision=SR_PREC_SPLIT, want_hidden=False, outputs=None,
-                 ws=None, stream=None, profile=None, initial=None, anchor_index=None):
+                 ws=None, stream=None, profile=None, initial=None, anchor_index=None, layer_done=None):
     """Replays every group of the call (see sr_group_replay).  Returns the
     outputs list [G][L] of (s_out, conv_out, hidden_out or None).
 
@@ -443,7 +460,7 @@ def group_replay(anchors, cu_seqlens, weights, *, max_seqlen, hidden, inter, h_k
             outputs.append(row)
     args = group_args(anchors, cu_seqlens, weights, outputs, max_seqlen=max_seqlen, hidden=hidden, inter=inter,
                       h_k=h_k, h_v=h_v, d=d, conv_width=conv_width, eps=eps, mode=mode, precision=precision,
-                      profile=profile, initial=initial, anchor_index=anchor_index)
+                      profile=profile, initial=initial, anchor_index=anchor_index, layer_done=layer_done)
     need = group_workspace_bytes(args)
     if need == 0:
         _check(group_call(args, None))

@@ -1,5 +1,7 @@
 """Build libsr.so in-tree: every csrc/*.cu compiled by nvcc for sm_100a only,
-linked into one shared library with a static CUDA runtime.
+linked into one shared library with a static CUDA runtime; and beside it
+libsr_checked.so, the same sources with -DSR_CHECKED (every global-memory
+index of the custom kernels is bounds-checked into the device status word).
 
     python gated_deltanet_state_sr_b200/build.py [--force] [--verbose]
 
@@ -18,6 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsr.so")
+OBJ_CHECKED = os.path.join(HERE, "_build_checked")
+LIB_CHECKED = os.path.join(HERE, "libsr_checked.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -31,10 +35,10 @@ def _deps():
                   glob.glob(os.path.join(INCLUDE, "sr", "*.h")))
 
 
-def _compile(src, verbose=False, extra=()):
-    obj = os.path.join(OBJ, os.path.basename(src) + ".o")
+def _compile(src, verbose=False, extra=(), obj_dir=OBJ):
+    obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
     newest_dep = max([os.path.getmtime(src)] + [os.path.getmtime(d) for d in _deps()])
-    if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep and not extra:
+    if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep:
         return obj, ""
     cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
@@ -45,28 +49,34 @@ def _compile(src, verbose=False, extra=()):
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def _build_one(obj_dir, lib, extra, force, verbose):
+    os.makedirs(obj_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     if force:
-        for o in glob.glob(os.path.join(OBJ, "*.o")):
+        for o in glob.glob(os.path.join(obj_dir, "*.o")):
             os.remove(o)
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose), srcs))
+        results = list(ex.map(lambda s: _compile(s, verbose, extra, obj_dir), srcs))
     objs = [o for o, _ in results]
     if verbose:
         for (_, log), s in zip(results, srcs):
             if log:
                 print(f"== {os.path.basename(s)}\n{log}")
-    if (not os.path.exists(LIB) or force or
-            max(os.path.getmtime(o) for o in objs) > os.path.getmtime(LIB)):
-        tmp = LIB + ".tmp"
+    if (not os.path.exists(lib) or force or
+            max(os.path.getmtime(o) for o in objs) > os.path.getmtime(lib)):
+        tmp = lib + ".tmp"
         cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs,
                "-Xlinker", "--exclude-libs,ALL"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    _build_one(OBJ, LIB, (), force, verbose)
+    _build_one(OBJ_CHECKED, LIB_CHECKED, ("-DSR_CHECKED",), force, False)
     return LIB
 
 

@@ -29,6 +29,23 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Bounds checks of the checked build.  Compiled with -DSR_CHECKED (the
+// library libsr_checked.so), SR_IN_BOUNDS(i, n, status) tests 0 <= i < n for a
+// global-memory index about to be used; on failure it ORs SR_DEV_BAD_ACCESS
+// into the status word and returns false, and the caller skips the access.
+// In the ordinary build it is the constant true and costs nothing.  A check
+// never traps: it is a stand-in for a memory checker that can run on any GPU.
+__device__ __forceinline__ bool in_bounds_checked(long long i, long long n, uint32_t *status) {
+    const bool ok = i >= 0 && i < n;
+    if (!ok && status) atomicOr(status, SR_DEV_BAD_ACCESS);
+    return ok;
+}
+#ifdef SR_CHECKED
+#define SR_IN_BOUNDS(i, n, status) ::sr::in_bounds_checked((long long)(i), (long long)(n), (status))
+#else
+#define SR_IN_BOUNDS(i, n, status) true
+#endif
+
 // Reads and checks the bounds of sequence n.  On a bad entry ORs a flag into
 // the status word and returns false; the caller then skips the sequence.
 __device__ __forceinline__ bool seq_bounds(const int32_t *cu, int n, int total, int max_len,

@@ -600,7 +600,7 @@ __device__ __forceinline__ void convert_u(uint8_t *sm, uint32_t xr_off, uint32_t
 template <int DH>
 __device__ __forceinline__ void out_chunk(uint8_t *sm, uint32_t stage_off, uint32_t RO, uint32_t lane_off, int half,
                                           int row, __nv_bfloat16 *o, size_t tok0, int clen, size_t v_stride, int h,
-                                          bool tile_store) {
+                                          bool tile_store, long long o_elems, uint32_t *status) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(RO + lane_off + 32 * half, r);
     tmem_ld_wait();
@@ -617,8 +617,9 @@ __device__ __forceinline__ void out_chunk(uint8_t *sm, uint32_t stage_off, uint3
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int t = 32 * half + e;
-            if (t < clen && row < 64 * DH)
-                o[(tok0 + t) * v_stride + size_t(h) * (64 * DH) + row] = __float2bfloat16_rn(__uint_as_float(r[e]));
+            const size_t idx = (tok0 + t) * v_stride + size_t(h) * (64 * DH) + row;
+            if (t < clen && row < 64 * DH && SR_IN_BOUNDS(idx, o_elems, status))
+                o[idx] = __float2bfloat16_rn(__uint_as_float(r[e]));
         }
     }
 }
@@ -627,13 +628,14 @@ __device__ __forceinline__ void out_chunk(uint8_t *sm, uint32_t stage_off, uint3
 // With DH = 1 (d = 64) h0 is [64][64] and the rest of the 128 x 128 state is zero.
 template <int DH>
 __device__ __forceinline__ void state_init(uint32_t RS, uint32_t lane_off, int half, int row, const float *h0,
-                                           size_t sbase) {
+                                           size_t sbase, long long s_elems, uint32_t *status) {
     constexpr int d = 64 * DH;
     uint32_t r[32];
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
         const int j0 = 64 * half + 32 * part;
-        const bool in = h0 && row < d && j0 < d;
+        const bool in = h0 && row < d && j0 < d &&
+                        SR_IN_BOUNDS(sbase + size_t(row) * d + j0 + 31, s_elems, status);
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(in ? h0[sbase + size_t(row) * d + j0 + e] : 0.f);
         tmem_st_32x32b_x32(RS + lane_off + j0, r);
@@ -644,7 +646,7 @@ __device__ __forceinline__ void state_init(uint32_t RS, uint32_t lane_off, int h
 // Final state TMEM RS -> s_out (the d x d block of it).
 template <int DH>
 __device__ __forceinline__ void state_out(uint32_t RS, uint32_t lane_off, int half, int row, float *s_out,
-                                          size_t sbase) {
+                                          size_t sbase, long long s_elems, uint32_t *status) {
     constexpr int d = 64 * DH;
     uint32_t r[32];
 #pragma unroll
@@ -653,6 +655,7 @@ __device__ __forceinline__ void state_out(uint32_t RS, uint32_t lane_off, int ha
         tmem_ld_32x32b_x32(RS + lane_off + j0, r);
         tmem_ld_wait();
         if (row >= d || j0 >= d) continue;
+        if (!SR_IN_BOUNDS(sbase + size_t(row) * d + j0 + 31, s_elems, status)) continue;
         float4 *dst = reinterpret_cast<float4 *>(s_out + sbase + size_t(row) * d + j0);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -663,9 +666,11 @@ __device__ __forceinline__ void state_out(uint32_t RS, uint32_t lane_off, int ha
 
 // Copies h0 (or zeros) to s_out for an empty sequence.
 template <int DH>
-__device__ __forceinline__ void state_passthrough(const float *h0, float *s_out, size_t sbase, int tid) {
+__device__ __forceinline__ void state_passthrough(const float *h0, float *s_out, size_t sbase, int tid,
+                                                  long long s_elems, uint32_t *status) {
     constexpr int d = 64 * DH;
     for (int e = tid; e < d * d / 4; e += kThreads) {
+        if (!SR_IN_BOUNDS(sbase + 4 * size_t(e) + 3, s_elems, status)) continue;
         const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
         reinterpret_cast<float4 *>(s_out + sbase)[e] = v;
     }
@@ -707,11 +712,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const int nchunks = (len + C - 1) / C;
     constexpr int d = 64 * DH;
     const size_t sbase = (size_t(n) * h_v + h) * d * d;
+    const long long s_elems = (long long)p.n_seqs * h_v * d * d, o_elems = (long long)p.total * h_v * d,
+                    gate_elems = (long long)p.total * h_v;
     const float *h0 = p.h0[gi];
     float *s_out = p.s_out[gi];
 
     if (nchunks == 0) {  // empty sequence: the state is h0 (or zero)
-        state_passthrough<DH>(h0, s_out, sbase, tid);
+        state_passthrough<DH>(h0, s_out, sbase, tid, s_elems, p.status);
         return;
     }
 
@@ -741,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const uint32_t R0 = tmem, R1 = tmem + 64, R2 = tmem + 128, R3 = tmem + 256;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    state_init<DH>(R2, lane_off, half, row, h0, sbase);
+    state_init<DH>(R2, lane_off, half, row, h0, sbase, s_elems, p.status);
 
     const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const CUtensorMap *mo = &p.om[gi];
@@ -788,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
     const float scale = p.scale;
     uint32_t kq_phase = 0, v_phase = 0, mma_phase = 0;
     float g_next = 0.f, b_next = 0.f;  // gates of the next chunk (threads tid < C)
-    if (tid < C && tid < len) {
+    if (tid < C && tid < len && SR_IN_BOUNDS((size_t(bos) + tid) * h_v + h, gate_elems, p.status)) {
         g_next = gh[size_t(tid) * h_v];
         b_next = bh[size_t(tid) * h_v];
     }
@@ -813,8 +820,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
             gam[tid] = g_next;
             bet[tid] = b_next;
             const int t = (c + 1) * C + tid;
-            g_next = t < len ? gh[size_t(t) * h_v] : 0.f;
-            b_next = t < len ? bh[size_t(t) * h_v] : 0.f;
+            const bool in = t < len && SR_IN_BOUNDS((size_t(bos) + t) * h_v + h, gate_elems, p.status);
+            g_next = in ? gh[size_t(t) * h_v] : 0.f;
+            b_next = in ? bh[size_t(t) * h_v] : 0.f;
         }
         const bool tma_ok = mbar_wait(bar_k, kq_phase) && mbar_wait(bar_q, kq_phase);
         kq_phase ^= 1;
@@ -907,7 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
         // ---- o_t (bf16) through the (now free) Qg region
         const bool tile_store = o != nullptr && clen == C;
-        if (o) out_chunk<DH>(sm, oQG, R3, lane_off, half, row, o, size_t(bos) + size_t(c) * C, clen, v_stride, h, tile_store);
+        if (o) out_chunk<DH>(sm, oQG, R3, lane_off, half, row, o, size_t(bos) + size_t(c) * C, clen, v_stride, h, tile_store, o_elems, p.status);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -921,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 
     __syncthreads();
     if (*abort_flag == 0) {
-        state_out<DH>(R2, lane_off, half, row, s_out, sbase);
+        state_out<DH>(R2, lane_off, half, row, s_out, sbase, s_elems, p.status);
     } else if (tid == 0) {
         atomicOr(p.status, SR_DEV_TIMEOUT);
         // let in-flight MMAs and TMA copies finish before tensor memory and shared memory are released
@@ -981,6 +989,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
     if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     const int len = eos - bos, c = slot - (bos / C + n);
     if (c < 0 || c * C >= len) return;
+    if (!SR_IN_BOUNDS(slot, p.slots, p.status)) return;
     const int clen = min(C, len - c * C), y = bos + c * C;
     const int hk = h / (p.h_v / p.h_k);
 
@@ -1011,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         fence_async_smem();
     }
     float g0 = 0.f, b0 = 0.f;  // padding has g = beta = 0
-    if (tid < clen) {
+    if (tid < clen && SR_IN_BOUNDS(size_t(y + tid) * p.h_v + h, (long long)p.total * p.h_v, p.status)) {
         g0 = p.g[gi][size_t(y + tid) * p.h_v + h];
         b0 = p.beta[gi][size_t(y + tid) * p.h_v + h];
     }
@@ -1109,12 +1118,15 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 // one token's 32 consecutive value channels per instruction (64 contiguous bytes).
 template <int DH>
 __device__ __forceinline__ void out_direct(uint32_t RO, uint32_t lane_off, int half, int row, __nv_bfloat16 *o,
-                                           size_t tok0, int clen, size_t v_stride, int h) {
+                                           size_t tok0, int clen, size_t v_stride, int h, long long o_elems,
+                                           uint32_t *status) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(RO + lane_off + 32 * half, r);
     tmem_ld_wait();
-    __nv_bfloat16 *dst = o + (tok0 + size_t(32 * half)) * v_stride + size_t(h) * (64 * DH) + row;
-    const int n_out = row < 64 * DH ? min(32, clen - 32 * half) : 0;
+    const size_t first = (tok0 + size_t(32 * half)) * v_stride + size_t(h) * (64 * DH) + row;
+    __nv_bfloat16 *dst = o + first;
+    int n_out = row < 64 * DH ? min(32, clen - 32 * half) : 0;
+    if (n_out > 0 && !SR_IN_BOUNDS(first + size_t(n_out - 1) * v_stride, o_elems, status)) n_out = 0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         if (e < n_out) *dst = __float2bfloat16_rn(__uint_as_float(r[e]));
@@ -1160,11 +1172,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     const int nchunks = (len + C - 1) / C;
     constexpr int d = 64 * DH;
     const size_t sbase = (size_t(n) * h_v + h) * d * d;
+    const long long s_elems = (long long)p.n_seqs * h_v * d * d, o_elems = (long long)p.total * h_v * d,
+                    gate_elems = (long long)p.total * h_v;
     const float *h0 = p.h0[gi];
     float *s_out = p.s_out[gi];
 
     if (nchunks == 0) {
-        state_passthrough<DH>(h0, s_out, sbase, tid);
+        state_passthrough<DH>(h0, s_out, sbase, tid, s_elems, p.status);
         return;
     }
 
@@ -1197,11 +1211,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     const uint32_t RS = tmem, RO0 = tmem + 128, RO1 = tmem + 256;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    state_init<DH>(RS, lane_off, half, row, h0, sbase);
+    state_init<DH>(RS, lane_off, half, row, h0, sbase, s_elems, p.status);
 
     const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const uint8_t *img = p.img + (size_t(gi) * p.slots * h_v + h) * kImg;
-    auto img_of = [&](int c) { return img + size_t(chunk_slot(bos, n, c)) * h_v * kImg; };
+    auto img_of = [&](int c) {
+        int sl = chunk_slot(bos, n, c);
+        if (!SR_IN_BOUNDS(sl, p.slots, p.status)) sl = 0;  // checked build: a slot past the images reads slot 0
+        return img + size_t(sl) * h_v * kImg;
+    };
     // Each input is refilled as soon as the last reader of its buffer is done:
     // Q once Qg is formed, V, T2 and -W^T once U is, K and P after the update.
     auto issue_k = [&](int c) {
@@ -1278,7 +1296,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         if (gt >= 0 && gt < C) {
             gam[gt] = g_next;
             const int t = (c + 1) * C + gt;
-            g_next = t < len ? gh[size_t(t) * h_v] : 0.f;
+            g_next = t < len && SR_IN_BOUNDS((size_t(bos) + t) * h_v + h, gate_elems, p.status)
+                         ? gh[size_t(t) * h_v] : 0.f;
         }
         const bool qok = mbar_wait(bar_q, q_phase);
         q_phase ^= 1;
@@ -1291,7 +1310,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         return true;
     };
 
-    if (gt >= 0 && gt < C && gt < len) g_next = gh[size_t(gt) * h_v];
+    if (gt >= 0 && gt < C && gt < len && SR_IN_BOUNDS((size_t(bos) + gt) * h_v + h, gate_elems, p.status))
+        g_next = gh[size_t(gt) * h_v];
     bool ok = next_gates_and_qg(0);
     ok = ok && !check(true);
     if (ok && tid == 0 && nchunks > 1) issue_q(1);
@@ -1319,8 +1339,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         // ---- meanwhile: o of the previous chunk (warp 4 also takes warp 0's share)
         if (o && c > 0) {
             const size_t tok0 = size_t(bos) + size_t(c - 1) * C;
-            if (warp != 0) out_direct<DH>(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h);
-            if (warp == 4) out_direct<DH>(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h);
+            if (warp != 0) out_direct<DH>(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h, o_elems, p.status);
+            if (warp == 4) out_direct<DH>(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h, o_elems, p.status);
         }
         const bool m2 = wait_mma() && *abort_flag == 0;
         if (check(m2)) break;
@@ -1362,8 +1382,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     if (*abort_flag == 0) {
         const int cl = nchunks - 1;
         if (o) out_direct<DH>(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C, len - cl * C,
-                          v_stride, h);
-        state_out<DH>(RS, lane_off, half, row, s_out, sbase);
+                          v_stride, h, o_elems, p.status);
+        state_out<DH>(RS, lane_off, half, row, s_out, sbase, s_elems, p.status);
     } else if (tid == 0) {
         atomicOr(p.status, SR_DEV_TIMEOUT);
         mma_commit(bar_mma);

@@ -250,7 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     tc::tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
                     tc::tmem_ld_wait();
                     const int col = nt * (BN / 2) + c;
-                    const int nvec = min(4, (p.N - col) / 8);  // 8-column groups in range
+                    int nvec = min(4, (p.N - col) / 8);  // 8-column groups in range
+                    if (row_ok && nvec > 0 &&
+                        !SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
+                        nvec = 0;
                     if (row_ok && nvec > 0) {
                         __nv_bfloat16 *cb = static_cast<__nv_bfloat16 *>(pr.c);
                         uint4 *dst = reinterpret_cast<uint4 *>(cb + size_t(row) * p.ldc + col);
@@ -292,6 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     const int col = nt * BN + c;
                     const int nvec = min(4, (p.N - col) / 8);
                     if (!row_ok || nvec <= 0) continue;
+                    if (!SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
+                        continue;
                     if (p.epi == EPI_F32_ROWSCALE || p.epi == EPI_F32_RESIDUAL) {
                         float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(pr.c) + size_t(row) * p.ldc + col);
                         const bool resid = p.epi == EPI_F32_RESIDUAL;

@@ -206,6 +206,8 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
                     SR_TRY(cudaMemsetAsync(o.conv_out, 0, c_bytes, st));
                 }
             }
+        for (int l = 0; a->layer_done && l < m.L; ++l)
+            if (a->layer_done[l]) SR_TRY(cudaEventRecord(static_cast<cudaEvent_t>(a->layer_done[l]), st));
         return SR_OK;
     }
     GroupBufs B[kMaxGroups];
@@ -293,6 +295,9 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         SR_TRY(gdn_tc_supported(m.d) ? gdn_tc_batch(gb, G, m.N, m.d, m.split, st)
                                      : gdn_chunked_batch(gb, G, m.N, m.d, m.split, st));
         SR_TRY(prof.end());
+        // layer l's states (s_out from this launch, conv_out from the conv launch) are final
+        if (a->layer_done && a->layer_done[l])
+            SR_TRY(cudaEventRecord(static_cast<cudaEvent_t>(a->layer_done[l]), st));
         if (stop) break;
 
         // (5) y = RMSNorm_head(o) w_gnorm * SiLU(z) -> A (hi/lo)
@@ -305,6 +310,7 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             gn.y_lo[g] = B[g].a_lo;
         }
         gn.T = T; gn.h_v = m.hv; gn.ld = m.proj; gn.z_off = m.conv_dim; gn.eps = a->eps; gn.lo8 = m.lo8;
+        gn.status = status;
         SR_TRY(prof.begin(SR_K_GATED_NORM));
         SR_TRY(gated_norm(gn, G, st));
         SR_TRY(prof.end());

@@ -97,6 +97,7 @@ struct GatedNormBatch {
     void *y_lo[kMaxGroups];               // may be null; bf16, or e4m3(lo * 2^8) when lo8
     int T, h_v, ld, z_off, lo8;
     float eps;
+    uint32_t *status;                     // device status word (bounds-checked build)
 };
 cudaError_t gated_norm(const GatedNormBatch &b, int n_groups, cudaStream_t st);
 

@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
         const int t1 = min(p.T, t0 + kConvTok);
         for (int e = tid; e < (t1 - t0) * p.h_v; e += blockDim.x) {
             const int t = t0 + e / p.h_v, h = e % p.h_v;
+            if (!SR_IN_BOUNDS(size_t(t) * p.h_v + h, (long long)p.T * p.h_v, p.status)) continue;
             const float b = P[size_t(t) * p.ld + p.b_off + h];
             const float a = P[size_t(t) * p.ld + p.b_off + p.h_v + h];
             p.gate[g][size_t(t) * p.h_v + h] = -expf(p.a_log[g][h]) * softplusf_(a + p.dt_bias[g][h]);
@@ -210,6 +211,10 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
         split2(c[0], c[1], hi[0], lo[0]);
         split2(c[2], c[3], hi[1], lo[1]);
         const uint2 hv = *reinterpret_cast<uint2 *>(hi), lv = *reinterpret_cast<uint2 *>(lo);
+        const long long w_out = head < n_qk ? (long long)p.T * p.h_k * 128 : (long long)p.T * p.h_v * 128;
+        const size_t o_first = size_t(t) * (head < n_qk ? p.h_k : p.h_v) * 128 +
+                               (ch - (head < p.h_k ? 0 : head < n_qk ? p.h_k * 128 : n_qk * 128));
+        if (!SR_IN_BOUNDS(o_first + 3, w_out, p.status)) return;
         if (head < p.h_k) {
             *reinterpret_cast<uint2 *>(p.q[g] + size_t(t) * p.h_k * 128 + ch) = hv;
         } else if (head < n_qk) {
@@ -272,9 +277,11 @@ __global__ void __launch_bounds__(128) conv_gates_kernel(const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 4; ++e) xm[j][e] = xr[e];
             } else if (p.conv_in[g]) {
-                const __nv_bfloat16 *hp = p.conv_in[g] + (size_t(n) * p.conv_dim + ch) * 3 + (3 - bos + tj);
+                const size_t hofs = (size_t(n) * p.conv_dim + ch) * 3 + (3 - bos + tj);
+                const bool hin = SR_IN_BOUNDS(hofs + 9, (long long)p.n_seqs * p.conv_dim * 3, p.status);
+                const __nv_bfloat16 *hp = p.conv_in[g] + hofs;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) xm[j][e] = __bfloat162float(hp[e * 3]);
+                for (int e = 0; e < 4; ++e) xm[j][e] = hin ? __bfloat162float(hp[e * 3]) : 0.f;
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) xm[j][e] = 0.f;
@@ -301,6 +308,7 @@ __global__ void __launch_bounds__(128) conv_state_kernel(const __grid_constant__
     if (ch >= p.conv_dim) return;
     const int bos = max(p.cu[n], 0), eos = min(p.cu[n + 1], p.T);
     const size_t off = (size_t(n) * p.conv_dim + ch) * 3;
+    if (!SR_IN_BOUNDS(off + 2, (long long)p.n_seqs * p.conv_dim * 3, p.status)) return;
     float hist[3] = {0.f, 0.f, 0.f};
     if (p.conv_in[g]) {
 #pragma unroll
@@ -311,7 +319,9 @@ __global__ void __launch_bounds__(128) conv_state_kernel(const __grid_constant__
     for (int j = 0; j < 3; ++j) {
         const int t = eos - 3 + j;
         const int hj = 3 - bos + t;  // history slot of a row before the start (in [0, 3) when t < bos)
-        val[j] = t >= bos ? p.p[g][size_t(t) * p.ld + ch] : (hj >= 0 ? hist[hj] : 0.f);
+        val[j] = t >= bos && SR_IN_BOUNDS(size_t(t) * p.ld + ch, (long long)p.T * p.ld, p.status)
+                     ? p.p[g][size_t(t) * p.ld + ch]
+                     : (t < bos && hj >= 0 ? hist[hj] : 0.f);
     }
     __nv_bfloat16 *out = p.conv_out[g] + off;
 #pragma unroll
@@ -327,6 +337,7 @@ __global__ void __launch_bounds__(256) gated_norm_kernel(const __grid_constant__
     if (item >= p.T * p.h_v) return;
     const int t = item / p.h_v, h = item % p.h_v;
     const int c = lane * 4;
+    if (!SR_IN_BOUNDS(size_t(item) * 128 + c + 3, (long long)p.T * p.h_v * 128, p.status)) return;
     const uint2 ou = *reinterpret_cast<const uint2 *>(p.o[g] + size_t(item) * 128 + c);
     const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ou);
     const float2 oa = __bfloat1622float2(o2[0]), ob = __bfloat1622float2(o2[1]);

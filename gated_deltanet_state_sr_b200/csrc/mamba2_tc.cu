@@ -62,7 +62,7 @@ struct M2TcParams {
     const float *h0;
     __nv_bfloat16 *y;
     float *s_out;
-    int total, max_len, H;
+    int total, max_len, H, n_seqs;
     uint32_t *status;
 };
 
@@ -107,11 +107,13 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     const int nchunks = (len + C - 1) / C;
     const int H = p.H;
     const size_t sbase0 = (size_t(n) * H + 2 * pair) * P * NS;  // state of head 2 pair; the pair is contiguous
+    const long long s_elems = (long long)p.n_seqs * H * P * NS, y_elems = (long long)p.total * H * P;
     const float *h0 = p.h0;
     float *s_out = p.s_out;
 
     if (nchunks == 0) {  // empty sequence: the states are h0 (or zero)
         for (int e = tid; e < 2 * P * NS / 4; e += kThreads) {
+            if (!SR_IN_BOUNDS(sbase0 + 4 * size_t(e) + 3, s_elems, p.status)) continue;
             const float4 v = h0 ? reinterpret_cast<const float4 *>(h0 + sbase0)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
             reinterpret_cast<float4 *>(s_out + sbase0)[e] = v;
         }
@@ -145,9 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
             const int n0 = 64 * half + 32 * part;
+            const bool in = h0 && SR_IN_BOUNDS(sbase0 + size_t(row) * NS + n0 + 31, s_elems, p.status);
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-                r[e] = __float_as_uint(h0 ? h0[sbase0 + size_t(row) * NS + n0 + e] : 0.f);
+                r[e] = __float_as_uint(in ? h0[sbase0 + size_t(row) * NS + n0 + e] : 0.f);
             tmem_st_32x32b_x32(RS + lane_off + n0, r);
         }
         tmem_st_wait();
@@ -173,7 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     // dt of the next chunk: thread tid < 128 holds token (tid & 63) of head (tid >> 6) of the pair
     const int dh = (tid >> 6) & 1, dtok = tid & 63;
     const float Ah = p.A[2 * pair + (warp & 1)];  // warps 0 and 1 scan heads 0 and 1
-    float dt_next = (tid < 128 && dtok < len) ? p.dt[(size_t(bos) + dtok) * H + 2 * pair + dh] : 0.f;
+    float dt_next = (tid < 128 && dtok < len &&
+                     SR_IN_BOUNDS((size_t(bos) + dtok) * H + 2 * pair + dh, (long long)p.total * H, p.status))
+                        ? p.dt[(size_t(bos) + dtok) * H + 2 * pair + dh] : 0.f;
     bool ok = true;
     // each MMA barrier completes once per chunk: its phase parity is the chunk's
     auto wait_on = [&](uint64_t *bar, int c) -> bool {
@@ -199,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         if (tid < 128) {
             dts[dh * C + dtok] = dt_next;
             const int t = (c + 1) * C + dtok;
-            dt_next = (t < len) ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
+            dt_next = (t < len && SR_IN_BOUNDS((size_t(bos) + t) * H + 2 * pair + dh, (long long)p.total * H, p.status))
+                          ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
         }
         const bool tma_ok = mbar_wait(&bar_in[b], (c >> 1) & 1);
         __syncthreads();
@@ -380,8 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             tmem_ld_wait();
             const float *eg = egs + hrow * C + 32 * half;
             const size_t stride = size_t(H) * P;
-            __nv_bfloat16 *yd = p.y + (size_t(bos) + size_t(c) * C + 32 * half) * stride + size_t(2 * pair + hrow) * P + prow;
-            const int n_out = min(32, clen - 32 * half);
+            const size_t y_first = (size_t(bos) + size_t(c) * C + 32 * half) * stride + size_t(2 * pair + hrow) * P + prow;
+            __nv_bfloat16 *yd = p.y + y_first;
+            int n_out = min(32, clen - 32 * half);
+            if (n_out > 0 && !SR_IN_BOUNDS(y_first + size_t(n_out - 1) * stride, y_elems, p.status)) n_out = 0;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 if (e < n_out) *yd = __float2bfloat16_rn(eg[e] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
@@ -402,6 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             const int n0 = 64 * half + 32 * part;
             tmem_ld_32x32b_x32(RS + lane_off + n0, r);
             tmem_ld_wait();
+            if (!SR_IN_BOUNDS(sbase0 + size_t(row) * NS + n0 + 31, s_elems, p.status)) continue;
             float4 *dst = reinterpret_cast<float4 *>(s_out + sbase0 + size_t(row) * NS + n0);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -443,6 +452,7 @@ cudaError_t mamba2_tc(const sr_mamba2_args &a, uint32_t *status, cudaStream_t st
     p.total = a.total_tokens;
     p.max_len = a.max_seqlen;
     p.H = a.n_heads;
+    p.n_seqs = a.n_seqs;
     p.status = status;
     cudaError_t e = cudaFuncSetAttribute(mamba2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
     if (e != cudaSuccess) return e;

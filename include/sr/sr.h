@@ -78,6 +78,8 @@ typedef enum sr_dtype { SR_BF16 = 0, SR_FP32 = 1 } sr_dtype;
 #define SR_DEV_SEQ_TOO_LONG 0x2u    /* a sequence is longer than max_seqlen       */
 #define SR_DEV_TIMEOUT 0x4u         /* a bounded on-chip wait gave up (kernel exited early) */
 #define SR_DEV_BAD_INDEX 0x8u       /* an anchor or row index outside its table (row read as zero / skipped) */
+#define SR_DEV_BAD_ACCESS 0x10u     /* bounds-checked build (libsr_checked.so) only: a global-memory access
+                                       outside its buffer was found and skipped */
 
 /* Kernel selection for sr_gdn_replay. */
 typedef enum sr_gdn_algo {
@@ -330,6 +332,16 @@ typedef struct sr_group_args {
      * anchors[g] holds the packed suffix itself ([total_tokens, hidden]). */
     const int32_t *anchor_index;
     int32_t anchor_rows;
+    /* Per-layer hand-off ("SuffixReplay", System Design, Pipelined Replay
+     * Path: the forward pass waits only at the layer that consumes a rebuilt
+     * state): a host array [n_layers] of cudaEvent_t handles the caller
+     * created, or NULL; NULL entries are skipped.  layer_done[l] is recorded on
+     * `stream` right after the launch that completes layer l's s_out and
+     * conv_out for every group, so work on another stream that needs only layer
+     * l's rebuilt state can wait on it instead of on the whole call.  It does
+     * not cover hidden_out[l], which the layer's MLP writes later.  Recording
+     * adds no synchronisation. */
+    void *const *layer_done;
 } sr_group_args;
 
 SR_API size_t sr_group_replay_workspace(const sr_group_args *args);

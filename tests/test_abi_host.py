@@ -23,6 +23,18 @@ def test_exports_every_declared_symbol():
         assert hasattr(sr.library(), n), f"libsr.so does not export {n}"
 
 
+def test_checked_build_exports_the_same_entry_points():
+    """The bounds-checked build (libsr_checked.so) is built beside libsr.so and
+    exports every entry point the headers declare."""
+    import ctypes as C
+    import glob
+    import os
+    lib = C.CDLL(os.path.join(os.path.dirname(sr.LIB_PATH), "libsr_checked.so"))
+    for h in glob.glob(os.path.join(os.path.dirname(sr.HEADER_PATH), "*.h")):
+        for n in sr.declared_symbols(h):
+            assert hasattr(lib, n), n
+
+
 def test_wait_timeout_validation():
     """The test-only bounded-wait entry point refuses a zero limit, a limit
     above the kernels' own, and a missing workspace, before any CUDA call."""

@@ -174,3 +174,39 @@ def test_whole_model_groups(sr, prefix, ratio, checked):
     for g in checked:
         ref = OL.group_replay(gis[g], "skip")
         check_group(out[g], ref, STATE_TOL, "skip", True)
+
+
+def test_layer_done_events_hand_off_each_layer(sr):
+    """Per-layer hand-off ("SuffixReplay", System Design, Pipelined Replay
+    Path): layer_done[l] is recorded right after the launch that completes
+    layer l's states, before any launch of layer l + 1, and a second stream
+    that waits only on it reads layer l's final state and conv state."""
+    s = small_shape()
+    gis = [W.group_inputs(44 + g, [70, 33], n_layers=3, shape=s) for g in range(2)]
+    anchors = [gi.anchors.cuda().contiguous() for gi in gis]
+    weights = [[DevLayer(lw) for lw in gi.layers] for gi in gis]
+    cu = gis[0].cu_seqlens.cuda()
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    prof = sr.LaunchProfiler(64)
+    out = sr.group_replay(anchors, cu, weights, max_seqlen=70, hidden=s.hidden, inter=s.inter, h_k=s.h_k,
+                          h_v=s.h_v, d=s.d_k, eps=s.eps, mode=sr.SR_MODE_FULL, precision=sr.SR_PREC_SPLIT,
+                          profile=prof, layer_done=events)
+    side = torch.cuda.Stream()
+    side.wait_event(events[0])
+    with torch.cuda.stream(side):
+        s0 = [out[g][0][0].clone() for g in range(2)]
+        c0 = [out[g][0][1].clone() for g in range(2)]
+    torch.cuda.synchronize()
+    for g in range(2):
+        assert torch.equal(s0[g], out[g][0][0]) and torch.equal(c0[g], out[g][0][1])
+    kinds = [k for k, _ in prof.times()]
+    gdn = [i for i, k in enumerate(kinds) if k == "gdn"]
+    assert len(gdn) == 3
+    for l in range(3):
+        end_of_recurrence = prof.ev[2 * gdn[l] + 1]
+        assert end_of_recurrence.elapsed_time(events[l]) >= 0
+        if gdn[l] + 1 < len(kinds):
+            next_launch = prof.ev[2 * (gdn[l] + 1)]
+            assert events[l].elapsed_time(next_launch) >= 0
+    ref = OL.group_replay(gis[1], "full")
+    check_group(out[1], ref, STATE_TOL, "full", False)
