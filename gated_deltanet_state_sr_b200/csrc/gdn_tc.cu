@@ -23,15 +23,17 @@
 //  * fused (gdn_tc_kernel): one CTA per (group, sequence, V head) runs every
 //    step of every chunk in order.  No scratch memory.
 //  * two-phase (gdn_prep_kernel, then gdn_seq_kernel): the gates, P, A, the
-//    solve, T2 and W of a chunk depend only on that chunk's q, k, g and beta,
-//    not on the state.  The prep kernel computes them for every (chunk, V
-//    head) at once (two CTAs per SM) and stores a 40 KB image per unit,
-//    [P | -W^T | T2 hi | T2 lo], in the operand layouts of the products that
-//    read it.  The sequential kernel then walks each sequence with only the
-//    state-dependent chain left per chunk:
-//        S -> bf16 and Qg;  O^T = S Qg^T,  U^T = V^T T2^T + S (-W)^T;
-//        U -> bf16;  S += (U diag)^T K,  O^T += U^T P^T;  o out,
-//    while the next chunk's tiles and image stream in behind each product.
+//    solve, T2, W and Qg of a chunk depend only on that chunk's q, k, g and
+//    beta, not on the state.  The prep kernel computes them for every (chunk,
+//    V head) at once (two CTAs per SM) and stores a 56.5 KB image per unit,
+//    [P | Qg, -W stacked | T2 hi | T2 lo | decay factors], in the operand
+//    layouts of the products that read it.  The sequential kernel then walks
+//    each sequence with only the state-dependent chain left per chunk:
+//        S -> bf16;  [O^T | U^T] = S [Qg ; -W]^T + [0 | V^T T2^T];
+//        U -> hi, lo, bf16;  S += (U diag)^T K;  O^T += U^T P^T;  o out,
+//    with the bf16 copy of S and U's tiles kept in tensor memory as the A
+//    operands of the products, while the next chunk's tiles and image stream
+//    in behind a whole chunk.
 // Every mbarrier wait is bounded; a timeout records SR_DEV_TIMEOUT, drains the
 // MMAs, frees tensor memory and ends the CTA.
 #include <cuda.h>
@@ -71,12 +73,15 @@ constexpr uint32_t smem_fused(bool split) {
 }
 
 // Chunk image of the two-phase form, per (group, chunk slot, V head): bf16
-// tiles in the 128-byte swizzled layouts of the products that read them.
+// tiles in the 128-byte swizzled layouts of the products that read them, and
+// the chunk's decay factors.  [Qg ; -W] is laid out as the sequential kernel's
+// stacked N = 128 operand, so one bulk copy brings it in.
 constexpr uint32_t IMG_P = 0;        // P, K-major [t][s]
-constexpr uint32_t IMG_W = 8192;     // -W, K-major [t][j], columns j 0-63 then 64-127 (16 KB)
-constexpr uint32_t IMG_T2H = 24576;  // T diag(beta), hi, K-major [t][s]
-constexpr uint32_t IMG_T2L = 32768;  // T diag(beta), lo
-constexpr uint32_t kImg = 40960;
+constexpr uint32_t IMG_QGW = 8192;   // [Qg_j0 | -W_j0 | Qg_j1 | -W_j1], K-major [t][j], 8 KB each
+constexpr uint32_t IMG_T2H = 40960;  // T diag(beta), hi, K-major [t][s]
+constexpr uint32_t IMG_T2L = 49152;  // T diag(beta), lo
+constexpr uint32_t IMG_GATE = 57344; // fp32 e^{gamma_C - gamma_t} for t < 64, then e^{gamma_C} (512 B)
+constexpr uint32_t kImg = 57856;
 
 // prep kernel: K/Q (and Kl, right after them: the prep kernel reads no V) tiles,
 // then A and T fp32.  P and T2 hi reuse the Q tiles once the first product has
@@ -86,10 +91,7 @@ constexpr uint32_t OFF_KL_PREP = 32768;
 constexpr uint32_t kPrepIn[2] = {32768, 49152};
 constexpr uint32_t smem_prep(bool split) { return kPrepIn[split] + 2 * SZ_AT + SZ_MISC + 1024; }
 
-// sequential kernel: inputs, P and T2 (hi, lo), S bf16, [Qg ; -W] stacked, the U tiles
-constexpr uint32_t SZ_PT2 = 24576, SZ_QGW = 32768;
-constexpr uint32_t smem_seq(bool split) { return kIn[split] + SZ_PT2 + SZ_SB + SZ_QGW + SZ_XR + SZ_MISC + 1024; }
-static_assert(smem_seq(true) <= 232448, "sequential kernel exceeds shared memory");
+
 static_assert(2 * (smem_prep(true) + 1024) <= 233472, "two prep CTAs must fit one SM");
 
 // Chunk c of the sequence n starting at token bos has the image slot
@@ -533,6 +535,29 @@ __device__ __forceinline__ void build_qg(uint8_t *sm, uint32_t qg_off, uint32_t 
             wp[q2] = pack2(xf.x * f, xf.y * f);
         }
         *reinterpret_cast<uint4 *>(sm + qg_off + sub * half_stride + off) = w;
+    }
+}
+
+// Qg = scale e^{gamma_t} Q, formed from the Q tiles (at OFF_KQ + 8192 and + 24576)
+// and written straight to global memory in the same swizzled tile layout, at dst
+// (j 0-63) and dst + 16 KB (j 64-127).  A warp writes four whole 128-byte rows per
+// instruction.
+__device__ __forceinline__ void build_qg_image(const uint8_t *sm, uint8_t *dst, const float *gam, float scale,
+                                               int tid) {
+    for (int e = tid; e < 1024; e += kThreads) {
+        const int sub = e >> 9, t = (e >> 3) & 63, ch = e & 7;
+        const uint32_t off = sw128(t, ch);
+        const uint4 u = *reinterpret_cast<const uint4 *>(sm + OFF_KQ + 8192 + sub * 16384 + off);
+        const float f = scale * __expf(gam[t]);
+        const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        uint4 w;
+        uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+            const float2 xf = __bfloat1622float2(x2[q2]);
+            wp[q2] = pack2(xf.x * f, xf.y * f);
+        }
+        *reinterpret_cast<uint4 *>(dst + sub * 16384 + off) = w;
     }
 }
 
@@ -1051,6 +1076,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
     const bool fact = gC > -80.f;
     uint32_t mma_phase = 0;
     bool ok = __syncthreads_and(mbar_wait(bar_in, 0)) != 0;
+    uint8_t *dst = p.img + ((size_t(gi) * p.slots + slot) * p.h_v + h) * kImg;
 
     if (ok) {
         // ---- [K;Q] K^T, then A and P
@@ -1059,6 +1085,11 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
             mma_kqk<SPLIT>(base, R0, R1, OFF_KL_PREP);
             mma_commit(bar_mma);
         }
+        // ---- meanwhile: Qg = scale e^{gamma_t} Q and the decay factors, straight to the image
+        build_qg_image(sm, dst + IMG_QGW, gam, p.scale, tid);
+        if (tid < C) reinterpret_cast<float *>(dst + IMG_GATE)[tid] = __expf(gC - gam[tid]);
+        if (tid == 0) reinterpret_cast<float *>(dst + IMG_GATE)[C] = __expf(gC);
+        __syncthreads();  // every Q read is done before P overwrites the first Q tile
         const bool w = mbar_wait(bar_mma, mma_phase);
         mma_phase ^= 1;
         tc_fence_after();
@@ -1068,7 +1099,6 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         ok = __syncthreads_and(w) != 0;
     }
     // each tile of the image leaves as soon as it is formed
-    uint8_t *dst = p.img + ((size_t(gi) * p.slots + slot) * p.h_v + h) * kImg;
     if (ok && tid == 0) bulk_store(dst + IMG_P, sm + oP, 8192);
     if (ok) {
         // ---- the solve, T1 and T2, then W^T = K^T T1^T and -W
@@ -1093,7 +1123,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
     }
     if (ok) {
         if (tid == 0) {
-            bulk_store(dst + IMG_W, sm + oW, 16384);
+            bulk_store(dst + IMG_QGW + 8192, sm + oW, 8192);
+            bulk_store(dst + IMG_QGW + 24576, sm + oW + 8192, 8192);
             bulk_commit();
             bulk_wait_read();  // shared memory may go; the writes complete with the grid
         }
@@ -1116,13 +1147,21 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 // ---------------------------------------------------------------- two-phase form: sequential
 // o_t (bf16) of one chunk straight from TMEM RO to global memory: a warp stores
 // one token's 32 consecutive value channels per instruction (64 contiguous bytes).
+// With `clear`, the columns read are then zeroed, so that the next product group
+// into this accumulator can add to it from the start.
 template <int DH>
 __device__ __forceinline__ void out_direct(uint32_t RO, uint32_t lane_off, int half, int row, __nv_bfloat16 *o,
                                            size_t tok0, int clen, size_t v_stride, int h, long long o_elems,
-                                           uint32_t *status) {
+                                           uint32_t *status, bool clear) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(RO + lane_off + 32 * half, r);
     tmem_ld_wait();
+    if (clear) {
+        uint32_t z[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) z[e] = 0u;
+        tmem_st_32x32b_x32(RO + lane_off + 32 * half, z);
+    }
     const size_t first = (tok0 + size_t(32 * half)) * v_stride + size_t(h) * (64 * DH) + row;
     __nv_bfloat16 *dst = o + first;
     int n_out = row < 64 * DH ? min(32, clen - 32 * half) : 0;
@@ -1132,35 +1171,150 @@ __device__ __forceinline__ void out_direct(uint32_t RO, uint32_t lane_off, int h
         if (e < n_out) *dst = __float2bfloat16_rn(__uint_as_float(r[e]));
         dst += v_stride;
     }
+    if (clear) tmem_st_wait();
 }
 
+// Zeroes the 64 O columns of an [O | U] accumulator (this thread's lane, its half).
+__device__ __forceinline__ void clear_o(uint32_t RO, uint32_t lane_off, int half) {
+    uint32_t z[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) z[e] = 0u;
+    tmem_st_32x32b_x32(RO + lane_off + 32 * half, z);
+    tmem_st_wait();
+}
+
+// The state chain keeps every A operand of its products in tensor memory
+// (tcgen05.mma with A from TMEM): the bf16 copy of S at RSB (64 columns, row
+// i of S in lane i, two values per column), and U's tiles written over U's own
+// fp32 columns RU and at RUB.  Only B operands live in shared memory.
+
+// bf16 copy of S (TMEM RS, this thread's row and column half) into RSB, then
+// S <- fC S in TMEM.
+__device__ __forceinline__ void state_copy_t(uint32_t RS, uint32_t RSB, uint32_t lane_off, int half, float fC) {
+    uint32_t r[32], b[16];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        tmem_ld_32x32b_x32(RS + lane_off + 64 * half + 32 * part, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) b[e] = pack2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+        tmem_st_32x32b_x16(RSB + lane_off + 32 * half + 16 * part, b);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
+        tmem_st_32x32b_x32(RS + lane_off + 64 * half + 32 * part, r);
+    }
+    tmem_st_wait();
+}
+
+// U's operands from its fp32 columns RU (lane i = value channel, column t =
+// token): U diag(e^{gamma_C - gamma}) as hi + lo written back over RU (tokens
+// 32 half .. 32 half + 31: hi at RU + 32 half, lo at RU + 32 half + 16, so a
+// thread overwrites only the columns it read) and U (bf16) at RUB + 16 half.
+__device__ __forceinline__ void convert_u_t(uint32_t RU, uint32_t RUB, uint32_t lane_off, int half, const float *fu) {
+    uint32_t r[32], wh[16], wl[16], wb[16];
+    tmem_ld_32x32b_x32(RU + lane_off + 32 * half, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const int t = 32 * half + 2 * e;
+        const float u0 = __uint_as_float(r[2 * e]), u1 = __uint_as_float(r[2 * e + 1]);
+        split2(u0 * fu[t], u1 * fu[t + 1], wh[e], wl[e]);
+        wb[e] = pack2(u0, u1);
+    }
+    tmem_st_32x32b_x16(RU + lane_off + 32 * half, wh);
+    tmem_st_32x32b_x16(RU + lane_off + 32 * half + 16, wl);
+    tmem_st_32x32b_x16(RUB + lane_off + 16 * half, wb);
+    tmem_st_wait();
+}
+
+// U^T = V^T T2^T -> RU (overwriting) from V at v_off and the hi and lo tiles of T2
+// (split: + Vl^T T2h^T, the low part of V at vl_off).
+template <bool SPLIT>
+__device__ __forceinline__ void mma_ut_s(uint32_t base, uint32_t v_off, uint32_t vl_off, uint32_t o2h, uint32_t o2l,
+                                         uint32_t RU) {
+    base = fresh(base);
+    const uint64_t dv = sdesc_sw128(base + v_off, 8192, 1024);  // V as MN-major A (i blocks 8 KB apart)
+    const uint64_t dvl = sdesc_sw128(base + vl_off, 8192, 1024);
+    const uint64_t dh = sdesc_sw128(base + o2h, 16, 1024), dl = sdesc_sw128(base + o2l, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dh, k * 32), ID_MN_K, k > 0);
+        mma_bf16_ss(RU, dadd(dv, k * 2048), dadd(dl, k * 32), ID_MN_K, 1);
+        if (SPLIT) mma_bf16_ss(RU, dadd(dvl, k * 2048), dadd(dh, k * 32), ID_MN_K, 1);
+    }
+}
+
+// [O^T | U^T] += S [Qg ; -W]^T -> RD (128 columns), S bf16 from TMEM RSB.
+__device__ __forceinline__ void mma_sqw_t(uint32_t base, uint32_t RSB, uint32_t qgw_off, uint32_t RD) {
+    base = fresh(base);
+    const uint64_t db = sdesc_sw128(base + qgw_off, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_bf16_ts(RD, RSB + 8 * k, dadd(db, (k >> 2) * 16384 + (k & 3) * 32), ID_KK128, 1);
+}
+
+// S += (U diag)^T K -> RS: hi + lo of U diag from TMEM RU, K at k_off as the
+// MN-major B operand (j blocks 8 KB apart); split: + hi times the low part of K.
+template <bool SPLIT>
+__device__ __forceinline__ void mma_s_update_t(uint32_t base, uint32_t k_off, uint32_t kl_off, uint32_t RU,
+                                               uint32_t RS) {
+    base = fresh(base);
+    const uint64_t dk = sdesc_sw128(base + k_off, 8192, 1024);
+    const uint64_t dkl = sdesc_sw128(base + kl_off, 8192, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t ah = RU + 32 * (k >> 1) + 8 * (k & 1);
+        mma_bf16_ts(RS, ah, dadd(dk, k * 2048), ID_S, 1);
+        mma_bf16_ts(RS, ah + 16, dadd(dk, k * 2048), ID_S, 1);
+        if (SPLIT) mma_bf16_ts(RS, ah, dadd(dkl, k * 2048), ID_S, 1);
+    }
+}
+
+// O^T += U^T P^T -> RO, U (bf16) from TMEM RUB and P at p_off.
+__device__ __forceinline__ void mma_o_update_t(uint32_t base, uint32_t RUB, uint32_t p_off, uint32_t RO) {
+    base = fresh(base);
+    const uint64_t dp = sdesc_sw128(base + p_off, 16, 1024);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mma_bf16_ts(RO, RUB + 8 * k, dadd(dp, k * 32), ID_KK, 1);
+}
+
+// Shared memory of the sequential kernel: K (and its low part) single-buffered;
+// V (and its low part) and the chunk image double-buffered, so the next chunk's
+// inputs stream in during a whole chunk.
+constexpr uint32_t SQ_K = 0, SQ_KL = 16384;   // [K_j0][K_j1], [Kl_j0][Kl_j1]
+constexpr uint32_t SQ_V = 32768;              // buffer b: [V_i0][V_i1] at SQ_V + 16 KB b
+constexpr uint32_t SQ_VL = 65536;             // buffer b: [Vl_i0][Vl_i1] at SQ_VL + 16 KB b
+constexpr uint32_t SQ_IMG = 98304;            // buffer b: the chunk image at SQ_IMG + SQ_IMG_STRIDE b
+constexpr uint32_t SQ_IMG_STRIDE = (kImg + 1023) / 1024 * 1024;
+constexpr uint32_t SQ_MISC = SQ_IMG + 2 * SQ_IMG_STRIDE;
+constexpr uint32_t smem_seq() { return SQ_MISC + 1024 + 1024; }
+static_assert(smem_seq() <= 232448, "sequential kernel exceeds shared memory");
+
 // One CTA per (V head, sequence rank, group).  Per chunk c the state chain is
-//   S(c) -> bf16;  [O(c) = S Qg^T,  U^T = V^T T2^T + S (-W)^T];  U -> bf16;
-//   [S += (U diag)^T K,  O(c) += U^T P^T]
-// and the work that feeds only the output or the next chunk runs beside the
-// products: o of chunk c-1 is written while the first group of products of c
-// runs (O alternates between two TMEM accumulators), and the gates and Qg of
-// chunk c+1 are formed while the state update of c runs.
+//   S(c) -> bf16 (TMEM);  [O(c) | U^T] += S [Qg ; -W]^T (U^T = V^T T2^T already
+//   there);  U -> hi, lo, bf16 (TMEM);  S += (U diag)^T K;
+// and the rest runs beside it: V^T T2^T of chunk c is formed while S is
+// copied; o of chunk c-1 is written (and its accumulator cleared for chunk
+// c+1) and chunk c+1's inputs are requested while the first product group of c
+// runs (O alternates between two TMEM accumulators); O(c) += U^T P^T is issued
+// after the state update and runs beside the next chunk's copy.  The chunk
+// image brings Qg and the decay factors, so no gate work is left here.
 template <bool SPLIT, int DH>
 __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(sm);
-    constexpr uint32_t oP = kIn[SPLIT], oT2H = oP + 8192, oT2L = oP + 16384;
-    constexpr uint32_t oSB = oP + SZ_PT2, oQGW = oSB + SZ_SB, oXR = oQGW + SZ_QGW, oMISC = oXR + SZ_XR;
-    float *gam = reinterpret_cast<float *>(sm + oMISC);  // [64]
-    float *fu = gam + C;                                  // [64] e^{gamma_C - gamma_t}
-    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + oMISC + 1024);  // K (+ k low part) landed
-    uint64_t *bar_q = bar_k + 1;                                          // Q landed
-    uint64_t *bar_v = bar_k + 2;                                          // V (+ v low part) landed
-    uint64_t *bar_w = bar_k + 3;                                          // -W^T and T2 landed
-    uint64_t *bar_p = bar_k + 4;                                          // P landed
-    uint64_t *bar_mma = bar_k + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + SQ_MISC);  // K (+ its low part) landed
+    uint64_t *bar_in = bar_k + 1;                                  // [2]: V and the image of buffer b landed
+    uint64_t *bar_g1 = bar_k + 3;                                  // [O | U] products done
+    uint64_t *bar_s = bar_k + 4;                                   // state update done
+    uint64_t *bar_o = bar_k + 5;                                   // output update done
+    uint64_t *bar_drain = bar_k + 6;                               // every issued MMA done (abort path)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_k + 7);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int h = blockIdx.x, gi = blockIdx.z;
-    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + oXR));
+    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + SQ_IMG));
     const int h_k = p.h_k, h_v = p.h_v;
     const int hk = h / (h_v / h_k);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1172,8 +1326,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     const int nchunks = (len + C - 1) / C;
     constexpr int d = 64 * DH;
     const size_t sbase = (size_t(n) * h_v + h) * d * d;
-    const long long s_elems = (long long)p.n_seqs * h_v * d * d, o_elems = (long long)p.total * h_v * d,
-                    gate_elems = (long long)p.total * h_v;
+    const long long s_elems = (long long)p.n_seqs * h_v * d * d, o_elems = (long long)p.total * h_v * d;
     const float *h0 = p.h0[gi];
     float *s_out = p.s_out[gi];
 
@@ -1183,18 +1336,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     }
 
     if (tid == 0) {
-        mbar_init(bar_k, 1);
-        mbar_init(bar_q, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_w, 1);
-        mbar_init(bar_p, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bar_k + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (DH == 1) {  // d = 64: the upper halves of the K, Q and V tiles are never loaded and stay zero
+    if (DH == 1) {  // d = 64: the upper halves of the K and V tiles are never loaded and stay zero
         for (int e = tid; e < 3 * 512; e += kThreads) {
-            const uint32_t tile = e < 512 ? OFF_KQ + 16384 : (e < 1024 ? OFF_KQ + 24576 : OFF_V + 8192);
+            const uint32_t tile = e < 512 ? SQ_K + 8192 : (e < 1024 ? SQ_V + 8192 : SQ_V + 16384 + 8192);
             *reinterpret_cast<uint4 *>(sm + tile + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_async_smem();
@@ -1207,77 +1355,57 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // S in columns 0-127; per chunk parity a 128-column pair [O | U]
-    const uint32_t RS = tmem, RO0 = tmem + 128, RO1 = tmem + 256;
+    // S fp32 in columns 0-127; per chunk parity a 128-column pair [O | U]; the bf16
+    // copy of S in 384-447; U (bf16) in 448-479
+    const uint32_t RS = tmem, RO0 = tmem + 128, RO1 = tmem + 256, RSB = tmem + 384, RUB = tmem + 448;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
     state_init<DH>(RS, lane_off, half, row, h0, sbase, s_elems, p.status);
+    clear_o(RO0, lane_off, half);
+    clear_o(RO1, lane_off, half);
 
-    const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
+    const CUtensorMap *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const uint8_t *img = p.img + (size_t(gi) * p.slots * h_v + h) * kImg;
     auto img_of = [&](int c) {
         int sl = chunk_slot(bos, n, c);
         if (!SR_IN_BOUNDS(sl, p.slots, p.status)) sl = 0;  // checked build: a slot past the images reads slot 0
         return img + size_t(sl) * h_v * kImg;
     };
-    // Each input is refilled as soon as the last reader of its buffer is done:
-    // Q once Qg is formed, V, T2 and -W^T once U is, K and P after the update.
     auto issue_k = [&](int c) {
         const int y = bos + c * C;
         mbar_arrive_expect_tx(bar_k, DH * (SPLIT ? 16384u : 8192u));
-        tma_load_2d(sm + OFF_KQ, mk, bar_k, hk * d, y);
-        if (DH == 2) tma_load_2d(sm + OFF_KQ + 16384, mk, bar_k, hk * d + 64, y);
+        tma_load_2d(sm + SQ_K, mk, bar_k, hk * d, y);
+        if (DH == 2) tma_load_2d(sm + SQ_K + 8192, mk, bar_k, hk * d + 64, y);
         if (SPLIT) {
-            tma_load_2d(sm + OFF_KL, mkl, bar_k, hk * d, y);
-            if (DH == 2) tma_load_2d(sm + OFF_KL + 8192, mkl, bar_k, hk * d + 64, y);
+            tma_load_2d(sm + SQ_KL, mkl, bar_k, hk * d, y);
+            if (DH == 2) tma_load_2d(sm + SQ_KL + 8192, mkl, bar_k, hk * d + 64, y);
         }
     };
-    auto issue_q = [&](int c) {
-        const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_q, DH * 8192u);
-        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_q, hk * d, y);
-        if (DH == 2) tma_load_2d(sm + OFF_KQ + 24576, mq, bar_q, hk * d + 64, y);
-    };
-    auto issue_v = [&](int c) {
-        const int y = bos + c * C;
-        mbar_arrive_expect_tx(bar_v, DH * (SPLIT ? 16384u : 8192u));
-        tma_load_2d(sm + OFF_V, mv, bar_v, h * d, y);
-        if (DH == 2) tma_load_2d(sm + OFF_V + 8192, mv, bar_v, h * d + 64, y);
+    auto issue_in = [&](int c) {  // V (+ low part) and the chunk image into buffer c & 1
+        const int y = bos + c * C, b = c & 1;
+        uint64_t *bar = &bar_in[b];
+        mbar_arrive_expect_tx(bar, DH * (SPLIT ? 16384u : 8192u) + kImg);
+        tma_load_2d(sm + SQ_V + 16384 * b, mv, bar, h * d, y);
+        if (DH == 2) tma_load_2d(sm + SQ_V + 16384 * b + 8192, mv, bar, h * d + 64, y);
         if (SPLIT) {
-            tma_load_2d(sm + OFF_VL, mvl, bar_v, h * d, y);
-            if (DH == 2) tma_load_2d(sm + OFF_VL + 8192, mvl, bar_v, h * d + 64, y);
+            tma_load_2d(sm + SQ_VL + 16384 * b, mvl, bar, h * d, y);
+            if (DH == 2) tma_load_2d(sm + SQ_VL + 16384 * b + 8192, mvl, bar, h * d + 64, y);
         }
-    };
-    auto issue_w = [&](int c) {  // -W (its halves beside those of Qg), T2 hi, T2 lo
-        const uint8_t *src = img_of(c);
-        mbar_arrive_expect_tx(bar_w, kImg - IMG_W);
-        bulk_load(sm + oQGW + 8192, src + IMG_W, 8192, bar_w);
-        bulk_load(sm + oQGW + 24576, src + IMG_W + 8192, 8192, bar_w);
-        bulk_load(sm + oT2H, src + IMG_T2H, kImg - IMG_T2H, bar_w);
-    };
-    auto issue_p = [&](int c) {
-        mbar_arrive_expect_tx(bar_p, IMG_W - IMG_P);
-        bulk_load(sm + oP, img_of(c) + IMG_P, IMG_W - IMG_P, bar_p);
+        bulk_load(sm + SQ_IMG + SQ_IMG_STRIDE * b, img_of(c), kImg, bar);
     };
     if (tid == 0) {
-        prefetch_tmap(mq); prefetch_tmap(mk); prefetch_tmap(mv);
+        prefetch_tmap(mk); prefetch_tmap(mv);
         if (SPLIT) { prefetch_tmap(mkl); prefetch_tmap(mvl); }
-        issue_q(0);
         issue_k(0);
-        issue_v(0);
-        issue_w(0);
-        issue_p(0);
+        issue_in(0);
+        if (nchunks > 1) issue_in(1);
     }
 
-    const float *gh = p.g[gi] + size_t(bos) * h_v + h;
     __nv_bfloat16 *o = p.o[gi];
     const size_t v_stride = size_t(h_v) * d;
-    const float scale = p.scale;
-    uint32_t k_phase = 0, q_phase = 0, v_phase = 0, w_phase = 0, p_phase = 0, mma_phase = 0;
 
-    auto wait_mma = [&]() -> bool {
-        const bool w = mbar_wait(bar_mma, mma_phase);
-        mma_phase ^= 1;
+    auto wait_on = [&](uint64_t *bar, int parity) -> bool {
+        const bool w = mbar_wait(bar, uint32_t(parity & 1));
         tc_fence_after();
         return w;
     };
@@ -1286,108 +1414,89 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         if (stop && tid == 0) *abort_flag = 1;
         return stop;
     };
-    // gates of chunk c in gam (gamma = inclusive prefix sum of g; padding has g = 0),
-    // fu, and Qg = scale e^{gamma_t} Q once Q has landed; false when a wait failed
-    float g_next = 0.f;  // g of the next chunk (threads tid < C)
-    // (warp 0 issues the products and takes no part here: threads 64-127 hold the
-    // gates, warp 1 scans them, warps 1-7 form Qg)
-    const int gt = tid - 64;  // the token whose gate this thread holds, when in [0, C)
-    auto next_gates_and_qg = [&](int c) -> bool {
-        if (gt >= 0 && gt < C) {
-            gam[gt] = g_next;
-            const int t = (c + 1) * C + gt;
-            g_next = t < len && SR_IN_BOUNDS((size_t(bos) + t) * h_v + h, gate_elems, p.status)
-                         ? gh[size_t(t) * h_v] : 0.f;
-        }
-        const bool qok = mbar_wait(bar_q, q_phase);
-        q_phase ^= 1;
-        __syncthreads();
-        if (warp == 1) gate_prefix(gam, lane);
-        if (check(qok)) return false;
-        if (gt >= 0 && gt < C) fu[gt] = __expf(gam[C - 1] - gam[gt]);  // read after later barriers
-        if (warp > 0) build_qg(sm, oQGW, 16384, gam, scale, tid - 32, kThreads - 32);
-        fence_async_smem();
-        return true;
-    };
-
-    if (gt >= 0 && gt < C && gt < len && SR_IN_BOUNDS((size_t(bos) + gt) * h_v + h, gate_elems, p.status))
-        g_next = gh[size_t(gt) * h_v];
-    bool ok = next_gates_and_qg(0);
-    ok = ok && !check(true);
-    if (ok && tid == 0 && nchunks > 1) issue_q(1);
 
     int c = 0;
-    for (; ok && c < nchunks; ++c) {
+    for (; c < nchunks; ++c) {
+        const int b = c & 1;
+        const uint32_t img_b = SQ_IMG + SQ_IMG_STRIDE * b;
+        const float *gate = reinterpret_cast<const float *>(sm + img_b + IMG_GATE);  // e^{gamma_C - gamma_t}, e^{gamma_C}
         const uint32_t RO = (c & 1) ? RO1 : RO0, RO_prev = (c & 1) ? RO0 : RO1, RU = RO + 64;
-        // ---- bf16 copy of S (entering the chunk), then S <- e^{gamma_C} S
-        state_copy(sm, oSB, RS, lane_off, half, row, __expf(gam[C - 1]));
-        fence_async_smem();
+        // ---- this chunk's V and image; U^T = V^T T2^T (state-free), formed while S is copied
+        const bool in_ok = wait_on(&bar_in[b], c >> 1);
+        if (tid == 0 && in_ok) {
+            mma_ut_s<SPLIT>(base, SQ_V + 16384 * b, SQ_VL + 16384 * b, img_b + IMG_T2H, img_b + IMG_T2L, RU);
+        }
+        // ---- bf16 copy of S (entering the chunk) into tensor memory, then S <- e^{gamma_C} S
+        state_copy_t(RS, RSB, lane_off, half, gate[C]);
         tc_fence_before();
-        if (check(true)) break;
+        if (check(in_ok)) break;
 
-        // ---- [O(c) | U^T] = S [Qg ; -W]^T, then U^T += V^T T2^T
+        // ---- [O(c) | U^T] += S [Qg ; -W]^T  (O(c) starts cleared)
         if (tid == 0) {
-            const bool w = mbar_wait(bar_v, v_phase) && mbar_wait(bar_w, w_phase);
-            if (!w) *abort_flag = 1;
             tc_fence_after();
-            mma_sqw(base, oSB, oQGW, RO);
-            mma_ut<SPLIT>(base, oT2H, oT2L, RU, true);
-            mma_commit(bar_mma);
+            mma_sqw_t(base, RSB, img_b + IMG_QGW, RO);
+            mma_commit(bar_g1);
         }
-        v_phase ^= 1;
-        w_phase ^= 1;
-        // ---- meanwhile: o of the previous chunk (warp 4 also takes warp 0's share)
-        if (o && c > 0) {
-            const size_t tok0 = size_t(bos) + size_t(c - 1) * C;
-            if (warp != 0) out_direct<DH>(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h, o_elems, p.status);
-            if (warp == 4) out_direct<DH>(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h, o_elems, p.status);
+        // ---- meanwhile: the next chunk's inputs into the other buffer, whose last
+        // reader (O(c - 1)'s update) is done, and o of the previous chunk (warp 4
+        // also takes warp 0's share), its accumulator cleared for chunk c + 1
+        bool ook = true;
+        if (c > 0) {
+            ook = wait_on(bar_o, c - 1);
+            if (tid == 192 && c + 1 < nchunks) issue_in(c + 1);
+            if (o) {
+                const size_t tok0 = size_t(bos) + size_t(c - 1) * C;
+                if (warp != 0)
+                    out_direct<DH>(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h, o_elems, p.status, true);
+                if (warp == 4)
+                    out_direct<DH>(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h, o_elems, p.status, true);
+            } else if (warp != 0) {
+                clear_o(RO_prev, lane_off, half);
+                if (warp == 4) clear_o(RO_prev, lane_off, 0);
+            }
         }
-        const bool m2 = wait_mma() && *abort_flag == 0;
+        const bool m2 = wait_on(bar_g1, c) && ook;
+        tc_fence_before();
         if (check(m2)) break;
-        if (c + 1 < nchunks) {  // issued from warps other than the product issuer
-            if (tid == 128) issue_v(c + 1);
-            if (tid == 160) issue_w(c + 1);
-        }
 
-        // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16): K-major tiles [i][t]
-        convert_u(sm, oXR, RU, lane_off, half, row, fu);
-        fence_async_smem();
+        // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16), in tensor memory
+        convert_u_t(RU, RUB, lane_off, half, gate);
         tc_fence_before();
         if (check(true)) break;
 
-        // ---- S += (U diag)^T K ;  O(c) += U^T P^T
+        // ---- S += (U diag)^T K
         if (tid == 0) {
-            const bool w = mbar_wait(bar_k, k_phase) && mbar_wait(bar_p, p_phase);
-            if (!w) *abort_flag = 1;
+            if (!mbar_wait(bar_k, uint32_t(c & 1))) *abort_flag = 1;
             tc_fence_after();
-            mma_update<SPLIT>(base, oXR, oP, RS, RO);
-            mma_commit(bar_mma);
+            mma_s_update_t<SPLIT>(base, SQ_K, SQ_KL, RU, RS);
+            mma_commit(bar_s);
         }
-        k_phase ^= 1;
-        p_phase ^= 1;
-        // ---- meanwhile: gates and Qg of the next chunk (the Qg tiles were last read
-        // by the first product group, complete at the previous wait)
-        bool nok = true;
-        if (c + 1 < nchunks) nok = next_gates_and_qg(c + 1);
-        const bool m4 = wait_mma() && *abort_flag == 0 && nok;
+        const bool m4 = wait_on(bar_s, c) && *abort_flag == 0;
+        tc_fence_before();
         if (check(m4)) break;
-        if (c + 1 < nchunks) {
-            if (tid == 32) issue_k(c + 1);
-            if (tid == 64) issue_p(c + 1);
-            if (tid == 96 && c + 2 < nchunks) issue_q(c + 2);
+        if (tid == 32 && c + 1 < nchunks) issue_k(c + 1);
+        // ---- O(c) += U^T P^T, off the state chain: it runs beside the next chunk's copy
+        if (tid == 0) {
+            tc_fence_after();
+            mma_o_update_t(base, RUB, img_b + IMG_P, RO);
+            mma_commit(bar_o);
         }
     }
 
     __syncthreads();
     if (*abort_flag == 0) {
         const int cl = nchunks - 1;
-        if (o) out_direct<DH>(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C, len - cl * C,
-                          v_stride, h, o_elems, p.status);
+        const bool w = wait_on(bar_o, cl);
+        if (o && w) out_direct<DH>(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C,
+                                   len - cl * C, v_stride, h, o_elems, p.status, false);
+        if (!w && tid == 0) atomicOr(p.status, SR_DEV_TIMEOUT);
         state_out<DH>(RS, lane_off, half, row, s_out, sbase, s_elems, p.status);
     } else if (tid == 0) {
+        // let every MMA this thread issued, and in-flight copies, finish before tensor
+        // and shared memory are released
         atomicOr(p.status, SR_DEV_TIMEOUT);
-        mma_commit(bar_mma);
-        mbar_wait(bar_mma, mma_phase);
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0);
         for (int i = 0; i < 64; ++i) __nanosleep(1000);
     }
     tc_fence_before();
@@ -1413,7 +1522,7 @@ cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t 
         gdn_tc_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kThreads, smem, st>>>(p);
         return cudaGetLastError();
     }
-    const int s1 = int(smem_prep(SPLIT)), s2 = int(smem_seq(SPLIT));
+    const int s1 = int(smem_prep(SPLIT)), s2 = int(smem_seq());
     cudaError_t e =
         cudaFuncSetAttribute(gdn_prep_kernel<SPLIT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return e;

@@ -41,7 +41,7 @@ cudaError_t gdn_chunked_batch(const GdnBatch &b, int n_groups, int n_seqs, int d
 // half-zero tiles; gdn_tc.cu).
 bool gdn_tc_supported(int d);
 cudaError_t gdn_tc(const sr_gdn_args &a, float scale, uint32_t *status, void *img, cudaStream_t st);
-// Scratch of the two-phase form: one 40 KB chunk image per (group, chunk slot, V head).
+// Scratch of the two-phase form: one 56.5 KB chunk image per (group, chunk slot, V head).
 size_t gdn_tc_image_bytes(int total, int n_seqs, int h_v, int n_groups);
 cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, bool split, cudaStream_t st);
 

@@ -92,18 +92,18 @@ def test_gdn_workspace_required():
 
 
 def test_gdn_two_phase_workspace_holds_the_chunk_images():
-    """The default tcgen05 form keeps one 40 KB chunk image per (chunk slot, V
+    """The default tcgen05 form keeps one 56.5 KB chunk image per (chunk slot, V
     head), with floor(T / 64) + n_seqs slots, at d = 128 and at d = 64 alike;
     the fused form and the other kernels need only the 256-byte header."""
     kw = dict(d_k=128, d_v=128, h_k=16, h_v=32, n_seqs=8, total_tokens=8917, max_seqlen=2048)
     slots = 8917 // 64 + 8
-    want = 256 + slots * 32 * 40960
+    want = 256 + slots * 32 * 57856
     assert sr.gdn_workspace_bytes(_gdn(**kw)) == want
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05, **kw)) == want
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED, **kw)) == 256
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_SEQUENTIAL, **kw)) == 256
     # d = 64 (100 tokens, 2 sequences, 4 V heads) takes the two-phase form too
-    assert sr.gdn_workspace_bytes(_gdn()) == 256 + (100 // 64 + 2) * 4 * 40960
+    assert sr.gdn_workspace_bytes(_gdn()) == 256 + (100 // 64 + 2) * 4 * 57856
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_CHUNKED)) == 256
     assert sr.gdn_workspace_bytes(_gdn(algo=sr.SR_GDN_TCGEN05_FUSED)) == 256
     # the tcgen05 forms take bf16 only
@@ -112,11 +112,11 @@ def test_gdn_two_phase_workspace_holds_the_chunk_images():
 
 def test_group_workspace_holds_the_chunk_images():
     """A replay group's workspace grows by the chunk images of its gated-delta
-    layers: 40 KB per (group, chunk slot, V head)."""
+    layers: 56.5 KB per (group, chunk slot, V head)."""
     a16, a80 = _fake_group_args(total_tokens=16, max_seqlen=16), _fake_group_args(total_tokens=80, max_seqlen=80)
     grow = sr.group_workspace_bytes(a80) - sr.group_workspace_bytes(a16)
     # 64 more tokens: one more slot (80 // 64 - 16 // 64) of 4 V heads, plus the per-token buffers
-    assert grow >= 1 * 4 * 40960
+    assert grow >= 1 * 4 * 57856
 
 
 def test_gdn_workspace_too_small_and_misaligned():
