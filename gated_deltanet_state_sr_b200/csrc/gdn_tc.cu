@@ -1290,17 +1290,25 @@ constexpr uint32_t SQ_MISC = SQ_IMG + 2 * SQ_IMG_STRIDE;
 constexpr uint32_t smem_seq() { return SQ_MISC + 1024 + 1024; }
 static_assert(smem_seq() <= 232448, "sequential kernel exceeds shared memory");
 
+// The sequential kernel runs 9 warps: warps 0-7 move data between tensor
+// memory and registers (warp w takes TMEM lanes 32 (w % 4) .. + 31 and column
+// half w / 4), warp 8 only waits for inputs and issues products and copies.
+constexpr int kSeqThreads = 288;
+constexpr int kIssuer = 256;
+
 // One CTA per (V head, sequence rank, group).  Per chunk c the state chain is
 //   S(c) -> bf16 (TMEM);  [O(c) | U^T] += S [Qg ; -W]^T (U^T = V^T T2^T already
 //   there);  U -> hi, lo, bf16 (TMEM);  S += (U diag)^T K;
-// and the rest runs beside it: V^T T2^T of chunk c is formed while S is
+// and the rest runs beside it: V^T T2^T of chunk c is issued while S is
 // copied; o of chunk c-1 is written (and its accumulator cleared for chunk
 // c+1) and chunk c+1's inputs are requested while the first product group of c
 // runs (O alternates between two TMEM accumulators); O(c) += U^T P^T is issued
-// after the state update and runs beside the next chunk's copy.  The chunk
-// image brings Qg and the decay factors, so no gate work is left here.
+// right behind the state update and runs beside the next chunk's copy.  The
+// chunk image brings Qg and the decay factors, so no gate work is left here.
+// Two block barriers per chunk hand work between the warps: after the state
+// copy and after U's conversion.
 template <bool SPLIT, int DH>
-__global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_constant__ GdnTcParams p) {
+__global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(sm);
@@ -1311,14 +1319,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     uint64_t *bar_o = bar_k + 5;                                   // output update done
     uint64_t *bar_drain = bar_k + 6;                               // every issued MMA done (abort path)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_k + 7);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int h = blockIdx.x, gi = blockIdx.z;
     const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + SQ_IMG));
     const int h_k = p.h_k, h_v = p.h_v;
     const int hk = h / (h_v / h_k);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const bool mover = warp < 8;              // warps 0-7
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const int row = quad * 32 + lane;
     int bos, eos;
     if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
@@ -1331,17 +1339,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     float *s_out = p.s_out[gi];
 
     if (nchunks == 0) {
-        state_passthrough<DH>(h0, s_out, sbase, tid, s_elems, p.status);
+        if (mover) state_passthrough<DH>(h0, s_out, sbase, tid, s_elems, p.status);
         return;
     }
 
-    if (tid == 0) {
+    if (tid == kIssuer) {
         for (int i = 0; i < 7; ++i) mbar_init(bar_k + i, 1);
-        *abort_flag = 0;
         fence_mbar_init();
     }
     if (DH == 1) {  // d = 64: the upper halves of the K and V tiles are never loaded and stay zero
-        for (int e = tid; e < 3 * 512; e += kThreads) {
+        for (int e = tid; e < 3 * 512; e += kSeqThreads) {
             const uint32_t tile = e < 512 ? SQ_K + 8192 : (e < 1024 ? SQ_V + 8192 : SQ_V + 16384 + 8192);
             *reinterpret_cast<uint4 *>(sm + tile + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -1360,9 +1367,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
     const uint32_t RS = tmem, RO0 = tmem + 128, RO1 = tmem + 256, RSB = tmem + 384, RUB = tmem + 448;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
-    state_init<DH>(RS, lane_off, half, row, h0, sbase, s_elems, p.status);
-    clear_o(RO0, lane_off, half);
-    clear_o(RO1, lane_off, half);
+    if (mover) {
+        state_init<DH>(RS, lane_off, half, row, h0, sbase, s_elems, p.status);
+        clear_o(RO0, lane_off, half);
+        clear_o(RO1, lane_off, half);
+    }
 
     const CUtensorMap *mk = &p.k[gi], *mv = &p.v[gi], *mkl = &p.kl[gi], *mvl = &p.vl[gi];
     const uint8_t *img = p.img + (size_t(gi) * p.slots * h_v + h) * kImg;
@@ -1393,7 +1402,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         }
         bulk_load(sm + SQ_IMG + SQ_IMG_STRIDE * b, img_of(c), kImg, bar);
     };
-    if (tid == 0) {
+    if (tid == kIssuer) {
         prefetch_tmap(mk); prefetch_tmap(mv);
         if (SPLIT) { prefetch_tmap(mkl); prefetch_tmap(mvl); }
         issue_k(0);
@@ -1409,89 +1418,79 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_seq_kernel(const __grid_const
         tc_fence_after();
         return w;
     };
-    auto check = [&](bool w) -> bool {
-        const bool stop = __syncthreads_or(!w) != 0;
-        if (stop && tid == 0) *abort_flag = 1;
-        return stop;
-    };
+    // block barrier that also tells every thread whether any thread's wait failed
+    auto check = [&](bool w) -> bool { return __syncthreads_or(!w) != 0; };
 
+    bool ok = true, carry = true;  // carry: this thread's wait for the previous state update
     int c = 0;
     for (; c < nchunks; ++c) {
         const int b = c & 1;
         const uint32_t img_b = SQ_IMG + SQ_IMG_STRIDE * b;
         const float *gate = reinterpret_cast<const float *>(sm + img_b + IMG_GATE);  // e^{gamma_C - gamma_t}, e^{gamma_C}
         const uint32_t RO = (c & 1) ? RO1 : RO0, RO_prev = (c & 1) ? RO0 : RO1, RU = RO + 64;
-        // ---- this chunk's V and image; U^T = V^T T2^T (state-free), formed while S is copied
-        const bool in_ok = wait_on(&bar_in[b], c >> 1);
-        if (tid == 0 && in_ok) {
+        // ---- this chunk's V and image: U^T = V^T T2^T (state-free) is issued while
+        // the movers copy S to bf16 in tensor memory and decay it
+        bool w = wait_on(&bar_in[b], c >> 1) && carry;
+        if (tid == kIssuer && w)
             mma_ut_s<SPLIT>(base, SQ_V + 16384 * b, SQ_VL + 16384 * b, img_b + IMG_T2H, img_b + IMG_T2L, RU);
-        }
-        // ---- bf16 copy of S (entering the chunk) into tensor memory, then S <- e^{gamma_C} S
-        state_copy_t(RS, RSB, lane_off, half, gate[C]);
+        if (mover && w) state_copy_t(RS, RSB, lane_off, half, gate[C]);
         tc_fence_before();
-        if (check(in_ok)) break;
+        if (check(w)) { ok = false; break; }
 
         // ---- [O(c) | U^T] += S [Qg ; -W]^T  (O(c) starts cleared)
-        if (tid == 0) {
+        if (tid == kIssuer) {
             tc_fence_after();
             mma_sqw_t(base, RSB, img_b + IMG_QGW, RO);
             mma_commit(bar_g1);
         }
-        // ---- meanwhile: the next chunk's inputs into the other buffer, whose last
-        // reader (O(c - 1)'s update) is done, and o of the previous chunk (warp 4
-        // also takes warp 0's share), its accumulator cleared for chunk c + 1
-        bool ook = true;
+        // ---- meanwhile: o of the previous chunk, its accumulator cleared for chunk
+        // c + 1, and the next chunk's inputs into the other buffer, whose last reader
+        // (O(c - 1)'s update) is then done
+        w = true;
         if (c > 0) {
-            ook = wait_on(bar_o, c - 1);
-            if (tid == 192 && c + 1 < nchunks) issue_in(c + 1);
-            if (o) {
-                const size_t tok0 = size_t(bos) + size_t(c - 1) * C;
-                if (warp != 0)
-                    out_direct<DH>(RO_prev, lane_off, half, row, o, tok0, C, v_stride, h, o_elems, p.status, true);
-                if (warp == 4)
-                    out_direct<DH>(RO_prev, lane_off, 0, row, o, tok0, C, v_stride, h, o_elems, p.status, true);
-            } else if (warp != 0) {
-                clear_o(RO_prev, lane_off, half);
-                if (warp == 4) clear_o(RO_prev, lane_off, 0);
+            w = wait_on(bar_o, c - 1);
+            if (tid == kIssuer && w && c + 1 < nchunks) issue_in(c + 1);
+            if (mover && w) {
+                if (o) {
+                    out_direct<DH>(RO_prev, lane_off, half, row, o, size_t(bos) + size_t(c - 1) * C, C, v_stride, h,
+                                   o_elems, p.status, true);
+                } else {
+                    clear_o(RO_prev, lane_off, half);
+                }
             }
         }
-        const bool m2 = wait_on(bar_g1, c) && ook;
-        tc_fence_before();
-        if (check(m2)) break;
-
+        w = wait_on(bar_g1, c) && w;
         // ---- U diag(e^{gamma_C - gamma}) (hi + lo) and U (bf16), in tensor memory
-        convert_u_t(RU, RUB, lane_off, half, gate);
+        if (mover && w) convert_u_t(RU, RUB, lane_off, half, gate);
         tc_fence_before();
-        if (check(true)) break;
+        if (check(w)) { ok = false; break; }
 
-        // ---- S += (U diag)^T K
-        if (tid == 0) {
-            if (!mbar_wait(bar_k, uint32_t(c & 1))) *abort_flag = 1;
+        // ---- S += (U diag)^T K, then right behind it O(c) += U^T P^T (off the chain)
+        if (tid == kIssuer) {
+            w = mbar_wait(bar_k, uint32_t(c & 1));
             tc_fence_after();
-            mma_s_update_t<SPLIT>(base, SQ_K, SQ_KL, RU, RS);
-            mma_commit(bar_s);
+            if (w) {
+                mma_s_update_t<SPLIT>(base, SQ_K, SQ_KL, RU, RS);
+                mma_commit(bar_s);
+                mma_o_update_t(base, RUB, img_b + IMG_P, RO);
+                mma_commit(bar_o);
+            }
         }
-        const bool m4 = wait_on(bar_s, c) && *abort_flag == 0;
-        tc_fence_before();
-        if (check(m4)) break;
-        if (tid == 32 && c + 1 < nchunks) issue_k(c + 1);
-        // ---- O(c) += U^T P^T, off the state chain: it runs beside the next chunk's copy
-        if (tid == 0) {
-            tc_fence_after();
-            mma_o_update_t(base, RUB, img_b + IMG_P, RO);
-            mma_commit(bar_o);
-        }
+        if (tid != kIssuer) w = true;
+        carry = wait_on(bar_s, c) && w;
+        if (tid == kIssuer && carry && c + 1 < nchunks) issue_k(c + 1);  // K's last reader is done
     }
+    if (ok) ok = __syncthreads_and(carry) != 0;
 
-    __syncthreads();
-    if (*abort_flag == 0) {
+    if (ok) {
         const int cl = nchunks - 1;
         const bool w = wait_on(bar_o, cl);
-        if (o && w) out_direct<DH>(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C,
-                                   len - cl * C, v_stride, h, o_elems, p.status, false);
-        if (!w && tid == 0) atomicOr(p.status, SR_DEV_TIMEOUT);
-        state_out<DH>(RS, lane_off, half, row, s_out, sbase, s_elems, p.status);
-    } else if (tid == 0) {
+        if (mover && o && w)
+            out_direct<DH>(cl & 1 ? RO1 : RO0, lane_off, half, row, o, size_t(bos) + size_t(cl) * C, len - cl * C,
+                           v_stride, h, o_elems, p.status, false);
+        if (!w && tid == kIssuer) atomicOr(p.status, SR_DEV_TIMEOUT);
+        if (mover) state_out<DH>(RS, lane_off, half, row, s_out, sbase, s_elems, p.status);
+    } else if (tid == kIssuer) {
         // let every MMA this thread issued, and in-flight copies, finish before tensor
         // and shared memory are released
         atomicOr(p.status, SR_DEV_TIMEOUT);
@@ -1530,7 +1529,7 @@ cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t 
     if (e != cudaSuccess) return e;
     gdn_prep_kernel<SPLIT, DH><<<dim3(p.slots, p.h_v, n_groups), kThreads, s1, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_seq_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kThreads, s2, st>>>(p);
+    gdn_seq_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kSeqThreads, s2, st>>>(p);
     return cudaGetLastError();
 }
 
