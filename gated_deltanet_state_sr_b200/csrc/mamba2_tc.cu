@@ -10,16 +10,19 @@
 //     S_C = e^{gamma_C} S_0 + sum_s dt_s e^{gamma_C-gamma_s} x_s B_s^T.
 // A CTA takes one sequence and two heads.  Their states (64 x 128 each) are
 // stacked into one 128 x 128 fp32 accumulator in tensor memory, so every
-// product is a tcgen05 MMA with M = 128, issued by one thread:
+// product is a tcgen05 MMA with M = 128, issued by one thread of a warp that
+// does nothing else:
 //     [C; B] B^T          -> G = C B^T in rows 0..63 (the B B^T rows are unused)
-//     [S_h0; S_h1] C^T    -> e^{-gamma} y's state part for both heads (bf16 copy of S)
+//     [S_h0; S_h1] C^T    -> e^{-gamma} y's state part for both heads
 //     [x_h0^T; x_h1^T] [Gm_h0 | Gm_h1]^T -> the chunk-internal part; the two
 //                            diagonal 64 x 64 blocks are the two heads' outputs
 //     S += [xw_h0^T; xw_h1^T] B   (xw = x diag(dt e^{gamma_C-gamma}) as hi + lo)
-// with Gm_h = (G o L_h), L_h[t][s] = e^{gamma_t-gamma_s} dt_s for s <= t.  C, B and
-// x tiles arrive by TMA (double-buffered); y goes from tensor memory straight to
-// global memory, a warp storing 32 consecutive channels of one token per
-// instruction.
+// with Gm_h = (G o L_h), L_h[t][s] = e^{gamma_t-gamma_s} dt_s for s <= t.  The A
+// operands of the state's own products (the bf16 copy of S and xw's hi and lo)
+// are written by the other eight warps into tensor memory and read from there;
+// C, B and x tiles arrive by TMA (double-buffered, two chunks ahead); y goes
+// from tensor memory straight to global memory, a warp storing 32 consecutive
+// channels of one token per instruction.
 // Exponentials only ever see differences gamma_t - gamma_s with s <= t.
 // Every mbarrier wait is bounded; a timeout records SR_DEV_TIMEOUT, drains the
 // MMAs, frees tensor memory and ends the CTA.
@@ -36,23 +39,21 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64, P = 64, NS = 128;
-constexpr int kThreads = 256;
-// MMA and TMA issue is spread over threads of warps that are idle at that point:
-// warp 7 (no gate-table work) forms C B^T at the chunk start and, with warp 2, has
-// no part in staging C B^T: after the state copy warp 7 loads the next chunk and
-// warp 2 issues the products.
-constexpr int kIssueIn = 224, kIssueMma = 64;
+// warps 0-7 move data (warp w: TMEM lanes 32 (w % 4) .. + 31, column half w / 4);
+// warp 8 waits for inputs and issues every product and copy
+constexpr int kMovers = 256, kThreads = 288, kIssuer = 256;
 
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t SZ_IN = 49152;        // one input buffer: [C_n0][B_n0][C_n1][B_n1][x_h0][x_h1], 8 KB each
 constexpr uint32_t OFF_IN = 0;           // two buffers
-constexpr uint32_t OFF_SB = 2 * SZ_IN;   // bf16 state [(h,p)][n]: two 64-column halves of 16 KB
-constexpr uint32_t OFF_Q = OFF_SB + 32768;    // masked G rows [(h,t)][s], 16 KB
-constexpr uint32_t OFF_XW = OFF_Q + 16384;    // [xwh_h0][xwh_h1][xwl_h0][xwl_h1] tiles [t][p], 8 KB each
-constexpr uint32_t OFF_YS = OFF_XW + 32768;   // G = C B^T staged for the mask rows
+constexpr uint32_t OFF_Q = 2 * SZ_IN;    // masked G rows [(h,t)][s], 16 KB
+constexpr uint32_t OFF_YS = OFF_Q + 16384;    // G = C B^T staged for the mask rows
 constexpr uint32_t OFF_MISC = OFF_YS + 16384; // gates, tables, barriers
 constexpr uint32_t SZ_MISC = 3072;
 constexpr uint32_t kSmem = OFF_MISC + SZ_MISC + 1024;
+
+// barrier of the eight data-moving warps only
+__device__ __forceinline__ void movers_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
 
 struct M2TcParams {
     CUtensorMap mc, mb, mx;
@@ -87,20 +88,20 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     float *wts = gam + 4 * C;                                // [2][64] dt e^{gamma_C - gamma}
     float *egs = gam + 6 * C;                                // [2][64] e^{gamma}
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 2048);  // [2] input buffers landed
-    uint64_t *bar_g = bar_in + 2;    // C B^T done
-    uint64_t *bar_mma = bar_in + 3;  // state part of y and the state update done
-    uint64_t *bar_y = bar_in + 4;    // chunk-internal part of y done
+    uint64_t *bar_g = bar_in + 2;      // C B^T done
+    uint64_t *bar_s = bar_in + 3;      // state part of y and the state update done
+    uint64_t *bar_y = bar_in + 4;      // chunk-internal part of y done
     uint64_t *bar_drain = bar_in + 5;  // every issued MMA done (abort path)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 6);
     float *gs = reinterpret_cast<float *>(sm + OFF_YS);      // G = C B^T staged for the mask
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const bool mover = tid < kMovers;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const int row = quad * 32 + lane;      // TMEM lane = stacked state row (head row >> 6, p = row & 63)
     const int hrow = row >> 6, prow = row & 63;
     const int pair = blockIdx.x;
-    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + OFF_SB));
+    const int n = longest_first(p.cu, gridDim.y, blockIdx.y, reinterpret_cast<int *>(sm + OFF_Q));
     int bos, eos;
     if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     const int len = eos - bos;
@@ -120,14 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         return;
     }
 
-    if (tid == 0) {
-        mbar_init(&bar_in[0], 1);
-        mbar_init(&bar_in[1], 1);
-        mbar_init(bar_g, 1);
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_y, 1);
-        mbar_init(bar_drain, 2);
-        *abort_flag = 0;
+    if (tid == kIssuer) {
+        for (int i = 0; i < 6; ++i) mbar_init(bar_in + i, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -138,11 +133,14 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // S (fp32) 0-127, G 128-191, the state part of y 192-255, the chunk-internal
+    // part 256-383, bf16 S 384-447, xw hi 448-479, xw lo 480-511
     const uint32_t RS = tmem, RG = tmem + 128, RI = tmem + 192, RY = tmem + 256;
+    const uint32_t RSB = tmem + 384, RXH = tmem + 448, RXL = tmem + 480;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
 
     // ---- initial states into TMEM: row (h, p), columns n in [64 half, 64 half + 64)
-    {
+    if (mover) {
         uint32_t r[32];
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -168,9 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         tma_load_2d(in + 32768, &p.mx, &bar_in[b], (2 * pair) * P, y0);
         tma_load_2d(in + 40960, &p.mx, &bar_in[b], (2 * pair + 1) * P, y0);
     };
-    if (tid == kIssueIn) {
+    if (tid == kIssuer) {
         prefetch_tmap(&p.mc); prefetch_tmap(&p.mb); prefetch_tmap(&p.mx);
         issue_in(0);
+        if (nchunks > 1) issue_in(1);
     }
 
     // dt of the next chunk: thread tid < 128 holds token (tid & 63) of head (tid >> 6) of the pair
@@ -179,253 +178,236 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     float dt_next = (tid < 128 && dtok < len &&
                      SR_IN_BOUNDS((size_t(bos) + dtok) * H + 2 * pair + dh, (long long)p.total * H, p.status))
                         ? p.dt[(size_t(bos) + dtok) * H + 2 * pair + dh] : 0.f;
-    bool ok = true;
-    // each MMA barrier completes once per chunk: its phase parity is the chunk's
-    auto wait_on = [&](uint64_t *bar, int c) -> bool {
-        const bool w = mbar_wait(bar, uint32_t(c & 1));
+    auto wait_on = [&](uint64_t *bar, int parity) -> bool {
+        const bool w = mbar_wait(bar, uint32_t(parity & 1));
         tc_fence_after();
         return w;
     };
-    auto check = [&](bool w) -> bool {
-        const bool stop = __syncthreads_or(!w) != 0;
-        if (stop && tid == 0) *abort_flag = 1;
-        return stop;
-    };
+    // block barrier that also tells every thread whether any thread's wait failed
+    auto check = [&](bool w) -> bool { return __syncthreads_or(!w) != 0; };
     constexpr uint32_t ID_G = idesc_bf16_f32_major(128, 64, 0, 0);      // [C;B] B^T, [S] C^T
     constexpr uint32_t ID_Y = idesc_bf16_f32_major(128, 128, 1, 0);     // x^T (MN-major) Q^T
-    constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 1, 1);     // xw^T (MN-major) B (MN-major)
+    constexpr uint32_t ID_S = idesc_bf16_f32_major(128, 128, 0, 1);     // xw^T (TMEM) B (MN-major)
     const bool want_y = p.y != nullptr;
 
+    bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
         const int b = c & 1;
         const uint32_t in = base + OFF_IN + b * SZ_IN;
         const int clen = min(C, len - c * C);
-        // ---- gates of the chunk: gamma = inclusive prefix sum of dt A (dt = 0 beyond the sequence)
-        if (tid < 128) {
-            dts[dh * C + dtok] = dt_next;
-            const int t = (c + 1) * C + dtok;
-            dt_next = (t < len && SR_IN_BOUNDS((size_t(bos) + t) * H + 2 * pair + dh, (long long)p.total * H, p.status))
-                          ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
-        }
-        const bool tma_ok = mbar_wait(&bar_in[b], (c >> 1) & 1);
-        __syncthreads();
-        if (warp < 2) {
-            const float *d = dts + warp * C;
-            const float a0 = d[2 * lane] * Ah, a1 = d[2 * lane + 1] * Ah;
-            float incl = a0 + a1;
+        bool w = wait_on(&bar_in[b], (c >> 1) & 1);
+        if (tid == kIssuer && w && want_y) {  // G = [C;B] B^T -> RG needs only this chunk's inputs
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
+                mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
             }
-            const float excl = incl - (a0 + a1);
-            gam[warp * C + 2 * lane] = excl + a0;
-            gam[warp * C + 2 * lane + 1] = excl + a0 + a1;
+            mma_commit(bar_g);
         }
-        if (check(tma_ok)) break;
-        if (tid == kIssueIn) {
-            if (want_y) {  // G = [C;B] B^T -> RG needs only this chunk's inputs
-                tc_fence_after();
+        if (mover) {
+            // ---- gates of the chunk: gamma = inclusive prefix sum of dt A (dt = 0 beyond the sequence)
+            if (tid < 128) {
+                dts[dh * C + dtok] = dt_next;
+                const int t = (c + 1) * C + dtok;
+                dt_next = (t < len && SR_IN_BOUNDS((size_t(bos) + t) * H + 2 * pair + dh, (long long)p.total * H,
+                                                   p.status))
+                              ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
+            }
+            movers_sync();
+            if (warp < 2) {
+                const float *d = dts + warp * C;
+                const float a0 = d[2 * lane] * Ah, a1 = d[2 * lane + 1] * Ah;
+                float incl = a0 + a1;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
                 }
-                mma_commit(bar_g);
+                const float excl = incl - (a0 + a1);
+                gam[warp * C + 2 * lane] = excl + a0;
+                gam[warp * C + 2 * lane + 1] = excl + a0 + a1;
             }
-        }
-        if (tid < 128) {
-            const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
-            wts[dh * C + dtok] = dts[dh * C + dtok] * __expf(gC - g);
-            egs[dh * C + dtok] = __expf(g);
-        }
-        __syncthreads();
-
-        // ---- bf16 copy of S (for y) and S <- e^{gamma_C} S in TMEM; xw = x diag(w) as hi + lo
-        {
-            const float fC = __expf(gam[hrow * C + C - 1]);
-            uint32_t r[32];
+            movers_sync();
+            if (tid < 128) {
+                const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
+                wts[dh * C + dtok] = dts[dh * C + dtok] * __expf(gC - g);
+                egs[dh * C + dtok] = __expf(g);
+            }
+            movers_sync();
+            // ---- bf16 copy of S (for y) into TMEM and S <- e^{gamma_C} S
+            {
+                const float fC = __expf(gam[hrow * C + C - 1]);
+                uint32_t r[32], bq[16];
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int n0 = 64 * half + 32 * part;
-                tmem_ld_32x32b_x32(RS + lane_off + n0, r);
-                tmem_ld_wait();
-                if (want_y) {
-                    uint8_t *sb = sm + OFF_SB + half * 16384;
+                for (int part = 0; part < 2; ++part) {
+                    const int n0 = 64 * half + 32 * part;
+                    tmem_ld_32x32b_x32(RS + lane_off + n0, r);
+                    tmem_ld_wait();
+                    if (want_y) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = pack2(__uint_as_float(r[8 * q4 + 0]), __uint_as_float(r[8 * q4 + 1]));
-                        w.y = pack2(__uint_as_float(r[8 * q4 + 2]), __uint_as_float(r[8 * q4 + 3]));
-                        w.z = pack2(__uint_as_float(r[8 * q4 + 4]), __uint_as_float(r[8 * q4 + 5]));
-                        w.w = pack2(__uint_as_float(r[8 * q4 + 6]), __uint_as_float(r[8 * q4 + 7]));
-                        *reinterpret_cast<uint4 *>(sb + sw128(row, 4 * part + q4)) = w;
+                        for (int e = 0; e < 16; ++e)
+                            bq[e] = pack2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                        tmem_st_32x32b_x16(RSB + lane_off + n0 / 2, bq);
                     }
-                }
 #pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
-                tmem_st_32x32b_x32(RS + lane_off + n0, r);
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * fC);
+                    tmem_st_32x32b_x32(RS + lane_off + n0, r);
+                }
+            }
+            // ---- xw = x diag(w) as hi + lo into TMEM: lane (h, p), tokens 32 half .. + 31
+            {
+                const uint8_t *xt = sm + OFF_IN + b * SZ_IN + 32768 + hrow * 8192;
+                const float *wv = wts + hrow * C + 32 * half;
+                const uint32_t pc = uint32_t(prow) >> 3, pb = (uint32_t(prow) & 7) * 2;
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int t = 32 * half + 2 * e;
+                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xt + sw128(t, pc) + pb));
+                    const float x1 =
+                        __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xt + sw128(t + 1, pc) + pb));
+                    split2(x0 * wv[2 * e], x1 * wv[2 * e + 1], hi[e], lo[e]);
+                }
+                tmem_st_32x32b_x16(RXH + lane_off + 16 * half, hi);
+                tmem_st_32x32b_x16(RXL + lane_off + 16 * half, lo);
             }
             tmem_st_wait();
         }
-        {
-            // thread: head hx, token tx, 32 p values (4 chunks of 8)
-            const int hx = tid >> 7, tx = (tid >> 1) & 63, c0 = (tid & 1) * 4;
-            const float wgt = wts[hx * C + tx];
-            const uint8_t *xt = sm + OFF_IN + b * SZ_IN + 32768 + hx * 8192;
-            uint8_t *xh = sm + OFF_XW + hx * 8192, *xl = sm + OFF_XW + 16384 + hx * 8192;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const uint32_t off = sw128(tx, c0 + v);
-                const uint4 u = *reinterpret_cast<const uint4 *>(xt + off);
-                const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(x2[e]);
-                    split2(f.x * wgt, f.y * wgt, hi[e], lo[e]);
-                }
-                *reinterpret_cast<uint4 *>(xh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(xl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-        }
-        fence_async_smem();
         tc_fence_before();
-        if (check(true)) break;
+        if (check(w)) { ok = false; break; }
 
-        // the input buffer of chunk c+1 last served chunk c-1, whose products have
-        // completed; its loads are issued here, where the issuing warp has no part in
-        // staging C B^T
-        if (tid == kIssueIn && c + 1 < nchunks) issue_in(c + 1);
-        // ---- MMAs: Yi^T = [S] C^T -> RI; S += xw^T B (hi, lo)
-        if (tid == kIssueMma) {
+        // ---- [S] C^T -> RI and S += xw^T B (hi, lo), one commit
+        if (tid == kIssuer) {
             tc_fence_after();
             if (want_y) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint32_t a = base + OFF_SB + (k >> 2) * 16384 + (k & 3) * 32;
                     const uint32_t bc = in + (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16_ss(RI, sdesc_sw128(a, 16, 1024), sdesc_sw128(bc, 16, 1024), ID_G, k > 0);
+                    mma_bf16_ts(RI, RSB + 8 * k, sdesc_sw128(bc, 16, 1024), ID_G, k > 0);
                 }
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const uint32_t bmn = in + 8192 + k * 2048;  // B as MN-major (n halves 16 KB apart)
-                mma_bf16_ss(RS, sdesc_sw128(base + OFF_XW + k * 2048, 8192, 1024), sdesc_sw128(bmn, 16384, 1024),
-                            ID_S, 1);
-                mma_bf16_ss(RS, sdesc_sw128(base + OFF_XW + 16384 + k * 2048, 8192, 1024),
-                            sdesc_sw128(bmn, 16384, 1024), ID_S, 1);
+                const uint64_t bmn = sdesc_sw128(in + 8192 + k * 2048, 16384, 1024);  // B as MN-major (n halves 16 KB apart)
+                mma_bf16_ts(RS, RXH + 8 * k, bmn, ID_S, 1);
+                mma_bf16_ts(RS, RXL + 8 * k, bmn, ID_S, 1);
             }
-            mma_commit(bar_mma);
-        }
-        if (!want_y) {
-            if (check(wait_on(bar_mma, c))) break;
-            continue;
+            mma_commit(bar_s);
         }
 
-        // ---- Gm_h rows: Q[(h, t)][s] = G[t][s] e^{gamma_h,t - gamma_h,s} dt_h,s (s <= t), bf16.
-        // G lives in TMEM lanes 0..63, which half of the warps can read: they stage it
-        // in shared memory (columns XOR-swizzled by row), then all warps build the rows
-        // while the other products run.
-        const bool mg = wait_on(bar_g, c);
-        if (quad < 2) {
-            const int t = row;
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(RG + lane_off + 32 * half, r);
-            tmem_ld_wait();
-            const int sw = (t & 7) << 2;
+        if (want_y) {
+            // ---- Gm_h rows: Q[(h, t)][s] = G[t][s] e^{gamma_h,t - gamma_h,s} dt_h,s (s <= t), bf16.
+            // G lives in TMEM lanes 0..63, which half of the movers can read: they stage it
+            // in shared memory (columns XOR-swizzled by row), then all movers build the rows
+            // while the other products run.
+            w = true;
+            if (mover) {
+                w = wait_on(bar_g, c);
+                if (quad < 2) {
+                    const int t = row;
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(RG + lane_off + 32 * half, r);
+                    tmem_ld_wait();
+                    const int sw = (t & 7) << 2;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<float4 *>(gs + t * C + ((32 * half + 4 * j) ^ sw)) =
-                    make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
-                                __uint_as_float(r[4 * j + 3]));
-        }
-        if (check(mg)) break;
-        {
-            // thread: head hq, token tq, 32 columns s0 .. s0 + 31
-            const int hq = tid >> 7, tq = (tid >> 1) & 63, s0 = (tid & 1) * 32;
-            const float gt = gam[hq * C + tq];
-            const float *gh = gam + hq * C, *dh2 = dts + hq * C;
-            const int sw = (tq & 7) << 2;
-            uint8_t *qrow = sm + OFF_Q;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const float4 ga = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4) ^ sw));
-                const float4 gb = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4 + 4) ^ sw));
-                const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int s = s0 + 8 * q4 + 2 * u;
-                    const float d0 = s <= tq ? __expf(gt - gh[s]) * dh2[s] : 0.f;
-                    const float d1 = s + 1 <= tq ? __expf(gt - gh[s + 1]) * dh2[s + 1] : 0.f;
-                    w[u] = pack2(d0 * gv[2 * u], d1 * gv[2 * u + 1]);
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4 *>(gs + t * C + ((32 * half + 4 * j) ^ sw)) =
+                            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
                 }
-                *reinterpret_cast<uint4 *>(qrow + sw128(hq * C + tq, (s0 >> 3) + q4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                movers_sync();
+                // thread: head hq, token tq, 32 columns s0 .. s0 + 31
+                const int hq = tid >> 7, tq = (tid >> 1) & 63, s0 = (tid & 1) * 32;
+                const float gt = gam[hq * C + tq];
+                const float *gh = gam + hq * C, *dh2 = dts + hq * C;
+                const int sw = (tq & 7) << 2;
+                uint8_t *qrow = sm + OFF_Q;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 ga = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4) ^ sw));
+                    const float4 gb = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4 + 4) ^ sw));
+                    const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    uint32_t wq[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s = s0 + 8 * q4 + 2 * u;
+                        const float d0 = s <= tq ? __expf(gt - gh[s]) * dh2[s] : 0.f;
+                        const float d1 = s + 1 <= tq ? __expf(gt - gh[s + 1]) * dh2[s + 1] : 0.f;
+                        wq[u] = pack2(d0 * gv[2 * u], d1 * gv[2 * u + 1]);
+                    }
+                    *reinterpret_cast<uint4 *>(qrow + sw128(hq * C + tq, (s0 >> 3) + q4)) =
+                        make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                }
+                fence_async_smem();
+            }
+            tc_fence_before();
+            if (check(w)) { ok = false; break; }
+            if (tid == kIssuer) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // [x_h0^T; x_h1^T] (MN-major, head blocks 8 KB apart) Q^T
+                    mma_bf16_ss(RY, sdesc_sw128(in + 32768 + k * 2048, 8192, 1024),
+                                sdesc_sw128(base + OFF_Q + k * 32, 16, 1024), ID_Y, k > 0);
+                mma_commit(bar_y);
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        if (check(true)) break;
-        if (tid == kIssueMma) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 4; ++k)  // [x_h0^T; x_h1^T] (MN-major, head blocks 8 KB apart) Q^T
-                mma_bf16_ss(RY, sdesc_sw128(in + 32768 + k * 2048, 8192, 1024),
-                            sdesc_sw128(base + OFF_Q + k * 32, 16, 1024), ID_Y, k > 0);
-            mma_commit(bar_y);
-        }
-        const bool m2 = wait_on(bar_mma, c) && wait_on(bar_y, c);
-        if (check(m2)) break;
 
-        // ---- y_t = e^{gamma_t} Yi + Y (own head's diagonal block); thread = (h, p), 32 tokens
-        {
-            uint32_t ri[32], ry[32];
-            tmem_ld_32x32b_x32(RI + lane_off + 32 * half, ri);
-            tmem_ld_32x32b_x32(RY + lane_off + 64 * hrow + 32 * half, ry);
-            tmem_ld_wait();
-            const float *eg = egs + hrow * C + 32 * half;
+        // ---- the products of this chunk are done: y out, and the input buffer of
+        // chunk c + 2 (this one) can be refilled
+        w = wait_on(bar_s, c);
+        if (want_y) w = wait_on(bar_y, c) && w;
+        if (tid == kIssuer && w && c + 2 < nchunks) issue_in(c + 2);
+        if (mover && want_y && w) {
+            // y_t = e^{gamma_t} Yi + Y (own head's diagonal block); thread = (h, p), 32 tokens
+            // in two passes of 16
             const size_t stride = size_t(H) * P;
             const size_t y_first = (size_t(bos) + size_t(c) * C + 32 * half) * stride + size_t(2 * pair + hrow) * P + prow;
             __nv_bfloat16 *yd = p.y + y_first;
             int n_out = min(32, clen - 32 * half);
             if (n_out > 0 && !SR_IN_BOUNDS(y_first + size_t(n_out - 1) * stride, y_elems, p.status)) n_out = 0;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                if (e < n_out) *yd = __float2bfloat16_rn(eg[e] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
-                yd += stride;
+            for (int part = 0; part < 2; ++part) {
+                uint32_t ri[16], ry[16];
+                tmem_ld_32x32b_x16(RI + lane_off + 32 * half + 16 * part, ri);
+                tmem_ld_32x32b_x16(RY + lane_off + 64 * hrow + 32 * half + 16 * part, ry);
+                tmem_ld_wait();
+                const float *eg = egs + hrow * C + 32 * half + 16 * part;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    if (16 * part + e < n_out)
+                        *yd = __float2bfloat16_rn(eg[e] * __uint_as_float(ri[e]) + __uint_as_float(ry[e]));
+                    yd += stride;
+                }
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        if (!w) { ok = false; }
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
     }
 
-    __syncthreads();
-    ok = *abort_flag == 0;
     if (ok) {
-        uint32_t r[32];
+        if (mover) {
+            uint32_t r[32];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int n0 = 64 * half + 32 * part;
-            tmem_ld_32x32b_x32(RS + lane_off + n0, r);
-            tmem_ld_wait();
-            if (!SR_IN_BOUNDS(sbase0 + size_t(row) * NS + n0 + 31, s_elems, p.status)) continue;
-            float4 *dst = reinterpret_cast<float4 *>(s_out + sbase0 + size_t(row) * NS + n0);
+            for (int part = 0; part < 2; ++part) {
+                const int n0 = 64 * half + 32 * part;
+                tmem_ld_32x32b_x32(RS + lane_off + n0, r);
+                tmem_ld_wait();
+                if (!SR_IN_BOUNDS(sbase0 + size_t(row) * NS + n0 + 31, s_elems, p.status)) continue;
+                float4 *dst = reinterpret_cast<float4 *>(s_out + sbase0 + size_t(row) * NS + n0);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                     __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                for (int e = 0; e < 8; ++e)
+                    dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                         __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+            }
         }
-    } else {
-        // let in-flight MMAs (of both issuing threads) and TMA copies finish before
+    } else if (tid == kIssuer) {
+        // let every MMA this thread issued, and in-flight TMA copies, finish before
         // tensor and shared memory are released
-        if (tid == kIssueIn || tid == kIssueMma) mma_commit(bar_drain);
-        if (tid == kIssueMma) {
-            atomicOr(p.status, SR_DEV_TIMEOUT);
-            mbar_wait(bar_drain, 0);
-            for (int i = 0; i < 64; ++i) __nanosleep(1000);
-        }
+        atomicOr(p.status, SR_DEV_TIMEOUT);
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0);
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
     }
     tc_fence_before();
     __syncthreads();
