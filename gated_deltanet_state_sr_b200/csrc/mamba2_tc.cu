@@ -16,7 +16,9 @@
 //     [S_h0; S_h1] C^T    -> e^{-gamma} y's state part for both heads
 //     [x_h0^T; x_h1^T] [Gm_h0 | Gm_h1]^T -> the chunk-internal part; the two
 //                            diagonal 64 x 64 blocks are the two heads' outputs
-//     S += [xw_h0^T; xw_h1^T] B   (xw = x diag(dt e^{gamma_C-gamma}) as hi + lo)
+//     [x_h0^T; x_h1^T] [D_h0 | D_h1]^T -> x diag(w) for both heads (diagonal blocks),
+//                            D_h = diag(w_h) as hi + lo bf16 tiles, w = dt e^{gamma_C-gamma}
+//     S += [xw_h0^T; xw_h1^T] B   (xw = x diag(w) as hi + lo)
 // with Gm_h = (G o L_h), L_h[t][s] = e^{gamma_t-gamma_s} dt_s for s <= t.  The A
 // operands of the state's own products (the bf16 copy of S and xw's hi and lo)
 // are written by the other eight warps into tensor memory and read from there;
@@ -48,7 +50,8 @@ constexpr uint32_t SZ_IN = 49152;        // one input buffer: [C_n0][B_n0][C_n1]
 constexpr uint32_t OFF_IN = 0;           // two buffers
 constexpr uint32_t OFF_Q = 2 * SZ_IN;    // masked G rows [(h,t)][s], 16 KB
 constexpr uint32_t OFF_YS = OFF_Q + 16384;    // G = C B^T staged for the mask rows
-constexpr uint32_t OFF_MISC = OFF_YS + 16384; // gates, tables, barriers
+constexpr uint32_t OFF_DW = OFF_YS + 16384;   // diag(w) per head as hi and lo tiles [t][s]: [h0 hi][h1 hi][h0 lo][h1 lo]
+constexpr uint32_t OFF_MISC = OFF_DW + 32768; // gates, tables, barriers
 constexpr uint32_t SZ_MISC = 3072;
 constexpr uint32_t kSmem = OFF_MISC + SZ_MISC + 1024;
 
@@ -92,7 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     uint64_t *bar_s = bar_in + 3;      // state part of y and the state update done
     uint64_t *bar_y = bar_in + 4;      // chunk-internal part of y done
     uint64_t *bar_drain = bar_in + 5;  // every issued MMA done (abort path)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 6);
+    uint64_t *bar_xw = bar_in + 6;     // x diag(w) done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_in + 7);
     float *gs = reinterpret_cast<float *>(sm + OFF_YS);      // G = C B^T staged for the mask
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -122,9 +126,13 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     }
 
     if (tid == kIssuer) {
-        for (int i = 0; i < 6; ++i) mbar_init(bar_in + i, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bar_in + i, 1);
         fence_mbar_init();
     }
+    // diag(w) tiles: zero off the diagonal for good; the diagonal is rewritten per chunk
+    for (int e = tid; e < 32768 / 16; e += kThreads)
+        *reinterpret_cast<uint4 *>(sm + OFF_DW + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_smem();
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -134,7 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // S (fp32) 0-127, G 128-191, the state part of y 192-255, the chunk-internal
-    // part 256-383, bf16 S 384-447, xw hi 448-479, xw lo 480-511
+    // part 256-383 (before it, x diag(w) in fp32), bf16 S 384-447, xw hi 448-479,
+    // xw lo 480-511
     const uint32_t RS = tmem, RG = tmem + 128, RI = tmem + 192, RY = tmem + 256;
     const uint32_t RSB = tmem + 384, RXH = tmem + 448, RXL = tmem + 480;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
@@ -230,10 +239,33 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             movers_sync();
             if (tid < 128) {
                 const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
-                wts[dh * C + dtok] = dts[dh * C + dtok] * __expf(gC - g);
+                const float wv = dts[dh * C + dtok] * __expf(gC - g);
+                wts[dh * C + dtok] = wv;
                 egs[dh * C + dtok] = __expf(g);
+                // diag(w) of head dh: entry (t, t) of its hi and lo tiles
+                uint32_t whi, wlo;
+                split2(wv, 0.f, whi, wlo);
+                const uint32_t off = sw128(dtok, dtok >> 3) + (dtok & 7) * 2;
+                *reinterpret_cast<uint16_t *>(sm + OFF_DW + dh * 8192 + off) = uint16_t(whi & 0xffffu);
+                *reinterpret_cast<uint16_t *>(sm + OFF_DW + 16384 + dh * 8192 + off) = uint16_t(wlo & 0xffffu);
             }
-            movers_sync();
+            fence_async_smem();
+        }
+        // ---- x diag(w) (hi + lo of w) -> the chunk-internal part's columns, on the
+        // tensor cores while the movers copy S
+        tc_fence_before();
+        if (check(w)) { ok = false; break; }
+        if (tid == kIssuer) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {  // [x_h0^T; x_h1^T] (MN-major) [Dh_h0; Dh_h1]^T, then the lo tiles
+                const uint64_t ax = sdesc_sw128(in + 32768 + k * 2048, 8192, 1024);
+                mma_bf16_ss(RY, ax, sdesc_sw128(base + OFF_DW + k * 32, 16, 1024), ID_Y, k > 0);
+                mma_bf16_ss(RY, ax, sdesc_sw128(base + OFF_DW + 16384 + k * 32, 16, 1024), ID_Y, 1);
+            }
+            mma_commit(bar_xw);
+        }
+        if (mover) {
             // ---- bf16 copy of S (for y) into TMEM and S <- e^{gamma_C} S
             {
                 const float fC = __expf(gam[hrow * C + C - 1]);
@@ -254,20 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
                     tmem_st_32x32b_x32(RS + lane_off + n0, r);
                 }
             }
-            // ---- xw = x diag(w) as hi + lo into TMEM: lane (h, p), tokens 32 half .. + 31
+            // ---- xw (own head's diagonal block of the product) as hi + lo into TMEM:
+            // lane (h, p), tokens 32 half .. + 31
+            w = wait_on(bar_xw, c);
             {
-                const uint8_t *xt = sm + OFF_IN + b * SZ_IN + 32768 + hrow * 8192;
-                const float *wv = wts + hrow * C + 32 * half;
-                const uint32_t pc = uint32_t(prow) >> 3, pb = (uint32_t(prow) & 7) * 2;
-                uint32_t hi[16], lo[16];
+                uint32_t r[32], hi[16], lo[16];
+                tmem_ld_32x32b_x32(RY + lane_off + 64 * hrow + 32 * half, r);
+                tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int t = 32 * half + 2 * e;
-                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xt + sw128(t, pc) + pb));
-                    const float x1 =
-                        __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xt + sw128(t + 1, pc) + pb));
-                    split2(x0 * wv[2 * e], x1 * wv[2 * e + 1], hi[e], lo[e]);
-                }
+                for (int e = 0; e < 16; ++e) split2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), hi[e], lo[e]);
                 tmem_st_32x32b_x16(RXH + lane_off + 16 * half, hi);
                 tmem_st_32x32b_x16(RXL + lane_off + 16 * half, lo);
             }
@@ -322,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
                 const float *gh = gam + hq * C, *dh2 = dts + hq * C;
                 const int sw = (tq & 7) << 2;
                 uint8_t *qrow = sm + OFF_Q;
-#pragma unroll
+#pragma unroll 1
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const float4 ga = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4) ^ sw));
                     const float4 gb = *reinterpret_cast<const float4 *>(gs + tq * C + ((s0 + 8 * q4 + 4) ^ sw));
