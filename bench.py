@@ -49,8 +49,9 @@ L2_BYTES = 126 * 1024 * 1024
 # the kernel source it was taken on; once that file changes the figure no
 # longer describes the kernel and the bench reports null.
 MEASURED_TRAFFIC = {
-    # in_proj of the 1-group workload with the fp8 low pass: 108.3 MB read + 41.4 MB written, x 8 groups
-    "model_32k_5": ("gemm_tc.cu", "8f8d09eb72f61537", 8 * 149.7e6),
+    # gate/up (single-CTA tiles) of the 1-group workload with the fp8 low pass: 155.4 MB read +
+    # 28.1 MB written, x 8 groups
+    "model_32k_5": ("gemm_tc.cu", "03b6ae2b55b1cbf3", 8 * 183.5e6),
     # the raw workload's call, both kernels of the two-phase form: prep 76.3 MB read +
     # 208.0 MB written, sequential 379.2 MB read + 64.4 MB written
     "raw_qwen": ("gdn_tc.cu", "8dae5304f374db1e", 727.9e6),
@@ -302,17 +303,19 @@ class GroupReplay:
         # mode) 2 (C 3 d_k + 2 d_k d_v)
         gdn_o = float(T) * s.h_v * 2 * (C * (3 * s.d_k + 2 * s.d_v) + 3 * s.d_k * s.d_v) * self.G
         gdn_no_o = float(T) * s.h_v * 2 * (C * 3 * s.d_k + 2 * s.d_k * s.d_v) * self.G
+        in_full = 2.0 * T * H * s.proj_dim * self.G
+        in_last = 2.0 * T * H * (s.proj_dim - s.v_dim) * self.G  # skip mode: the last layer needs no z
         self.flop = {  # algorithmic flops of one launch (all groups)
-            "gemm_in": 2.0 * T * H * s.proj_dim * self.G,
+            # the mean over the step's in_proj launches: L - 1 full, the last without z
+            "gemm_in": ((self.L - 1) * in_full + in_last) / self.L,
             "gemm_out": 2.0 * T * s.v_dim * H * self.G,
             "gemm_gateup": 2.0 * T * H * 2 * I * self.G,
             "gemm_down": 2.0 * T * I * H * self.G,
             # the mean over the step's GDN launches: L - 1 with o, the last without
             "gdn": ((self.L - 1) * gdn_o + gdn_no_o) / self.L,
         }
-        full = (self.flop["gemm_in"] + self.flop["gemm_out"] + self.flop["gemm_gateup"] + self.flop["gemm_down"]
-                + gdn_o)
-        last = self.flop["gemm_in"] + gdn_no_o
+        full = in_full + self.flop["gemm_out"] + self.flop["gemm_gateup"] + self.flop["gemm_down"] + gdn_o
+        last = in_last + gdn_no_o
         self.step_flop = (self.L - 1) * full + last  # skip mode
         # algorithmic bytes of one launch (all groups) for the HBM-bound layer kernels
         split = 1 if precision == "bf16" else 2  # k, v: bf16, or hi + lo bf16
@@ -335,7 +338,9 @@ class GroupReplay:
         self.bytes_impl = {
             "conv": float(T) * self.G * ((s.conv_dim + 2 * s.h_v) * 4 + qd * 2 + (qd + vd) * 2 * split
                                          + 2 * s.h_v * 4),
-            "row_prep": float(T) * self.G * (H * 4 + H * act_out + 4),
+            # layer 0 only (later layers get the operand from the residual GEMMs' epilogues):
+            # bf16 anchors in, the fp32 residual stream, the operand and r out
+            "row_prep": float(T) * self.G * (H * 2 + H * 4 + H * act_out + 4),
             "gated_norm": float(T) * self.G * (vd * 2 + vd * 4 + vd * act_out),
         }
         self.input_bytes = self.G * T * H * 2 + sum(

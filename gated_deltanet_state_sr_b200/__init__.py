@@ -304,14 +304,16 @@ def default_scale(d_k):
 
 # ------------------------------------------------------------------ test support (include/sr/sr_testing.h)
 
-_test_gemm = _sig("sr_test_gemm", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp,
+_test_gemm = _sig("sr_test_gemm", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
                   ctypes.c_size_t, _vp)
 EPI_STORE, EPI_RESIDUAL, EPI_SWIGLU = 0, 1, 2
+GEMM_FORM_DEFAULT, GEMM_FORM_SINGLE, GEMM_FORM_PAIR = 0, 1, 2
 
 
-def test_gemm(a, b0, *, b1=None, r=None, epi=EPI_STORE, c=None, ws=None, stream=None):
+def test_gemm(a, b0, *, b1=None, r=None, epi=EPI_STORE, c=None, ws=None, stream=None, form=GEMM_FORM_DEFAULT):
     """One tcgen05 GEMM through sr_test_gemm: c = a b0^T, r + a b0^T, or
-    SiLU(a b0^T) * (a b1^T).  bf16 CUDA tensors, row-major."""
+    SiLU(a b0^T) * (a b1^T).  bf16 CUDA tensors, row-major.  form: the
+    library default, one CTA per tile, or CTA pairs."""
     torch = _torch()
     m, k = a.shape
     n = b0.shape[0]
@@ -319,8 +321,8 @@ def test_gemm(a, b0, *, b1=None, r=None, epi=EPI_STORE, c=None, ws=None, stream=
         c = torch.empty(m, n, dtype=torch.bfloat16, device=a.device)
     if ws is None:
         ws = workspace(256, a.device)
-    _check(_test_gemm(_ptr(a), _ptr(b0), _ptr(b1), _ptr(c), _ptr(r), m, n, k, epi, _ptr(ws), ws.numel(),
-                      _stream_handle(stream)))
+    _check(_test_gemm(_ptr(a), _ptr(b0), _ptr(b1), _ptr(c), _ptr(r), m, n, k, epi, int(form), _ptr(ws),
+                      ws.numel(), _stream_handle(stream)))
     return c
 
 

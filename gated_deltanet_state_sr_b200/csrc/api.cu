@@ -186,11 +186,12 @@ sr_status sr_device_status(const void *ws, void *stream, uint32_t *flags) {
 #include "sr/sr_testing.h"
 
 extern "C" sr_status sr_test_gemm(const void *a, const void *b0, const void *b1, void *c, const void *r,
-                                  int32_t m, int32_t n, int32_t k, int32_t epi, void *ws, size_t ws_bytes,
-                                  void *stream) {
+                                  int32_t m, int32_t n, int32_t k, int32_t epi, int32_t form, void *ws,
+                                  size_t ws_bytes, void *stream) {
     if (!a || !b0 || !c || (epi == EPI_SWIGLU && !b1) || (epi == EPI_RESIDUAL && !r))
         return set_error(SR_ERR_INVALID_ARG, "sr_test_gemm: missing operand");
     if (epi < 0 || epi > 2) return set_error(SR_ERR_INVALID_ARG, "sr_test_gemm: bad epilogue");
+    if (form < 0 || form > 2) return set_error(SR_ERR_INVALID_ARG, "sr_test_gemm: bad form");
     if (m <= 0 || n <= 0 || k <= 0 || k % 64 || n % 32)
         return set_error(SR_ERR_UNSUPPORTED, "sr_test_gemm: need m, n, k > 0, k %% 64 == 0, n %% 32 == 0");
     if (sr_status s = check_workspace(ws, ws_bytes, kWsHeader)) return s;
@@ -198,7 +199,9 @@ extern "C" sr_status sr_test_gemm(const void *a, const void *b0, const void *b1,
     uint32_t *status = static_cast<uint32_t *>(ws);
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st);
     GemmProblemDesc d{a, nullptr, b0, b1, c, r, nullptr, nullptr};
-    if (e == cudaSuccess) e = gemm_tc(&d, 1, m, n, k, n, epi, 1, 0, status, st);
+    GemmOptions opt;
+    opt.form = form;
+    if (e == cudaSuccess) e = gemm_tc(&d, 1, m, n, k, n, epi, 1, 0, status, st, opt);
     if (e != cudaSuccess) return cuda_error(e, "sr_test_gemm");
     return SR_OK;
 }

@@ -6,7 +6,10 @@
 //   EPI_SWIGLU        C = SiLU(r A Bg^T) * (r A Bu^T) bf16 out, optional lo part   (MLP gate/up)
 //   EPI_F32_ROWSCALE  C = r A B^T                     fp32 out                     (in_proj)
 //   EPI_F32_RESIDUAL  C += A B^T                      fp32 in place                (out_proj, down)
-// r is an optional fp32 per-row scale (the folded RMSNorm factor).  With two
+//                     and optionally the next RMSNorm's operand from the new C:
+//                     C * w as hi + lo, and each row's sum of C^2 over the tile
+// r is an optional fp32 per-row scale (the folded RMSNorm factor), given as
+// such or formed from the producing GEMM's per-tile sums of squares.  With two
 // passes the A operand is an exact hi + lo pair of bf16 matrices
 // (A = A_hi + A_lo) and both products accumulate into the same TMEM tile, so
 // the result carries ~16 mantissa bits of the activations: the weights are
@@ -52,6 +55,11 @@ struct Problem {
     const __nv_bfloat16 *r;
     void *c_lo;              // SwiGLU: low part of the output (bf16, or e4m3 of lo * 2^8; may be null)
     const float *rowscale;   // per-row scale (may be null)
+    const float *ssq_in;     // per-row partial sums of squares -> RMSNorm row scale (may be null)
+    const __nv_bfloat16 *nw; // EPI_F32_RESIDUAL: next norm weight (may be null)
+    __nv_bfloat16 *n_hi;     // x * nw, hi part, row pitch N
+    void *n_lo;              // low part (bf16, or e4m3 of lo * 2^8; may be null)
+    float *ssq_out;          // [n_tiles, M] sums of x^2 per N-tile
 };
 
 struct Params {
@@ -63,8 +71,22 @@ struct Params {
     int epi;
     int n_pass;  // 1: A; 2: A_hi then A_lo
     int lo_fp8;  // the A_lo pass on the fp8 tensor cores (128-byte K blocks of 128 elements)
+    int ssq_parts;  // partial sums per row in ssq_in
+    float eps;      // RMSNorm epsilon of the row scale formed from ssq_in
+    int nt_skip_at, nt_skip;  // N tiles nt_skip_at .. + nt_skip - 1 are not computed (n_tiles excludes them)
+    int ssq_slots;  // partial sums per row written by the next-norm epilogue: one per 256-column tile
     uint32_t *status;
 };
+
+// Problem, N tile and M tile of work item `tile` (M tiles fastest).
+__device__ __forceinline__ void decode_tile(const Params &p, int tile, int &pi, int &nt, int &mt) {
+    const int tiles_per_prob = p.m_tiles * p.n_tiles;
+    pi = tile / tiles_per_prob;
+    const int rem = tile % tiles_per_prob;
+    nt = rem / p.m_tiles;
+    mt = rem % p.m_tiles;
+    if (nt >= p.nt_skip_at) nt += p.nt_skip;
+}
 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -96,6 +118,163 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
         for (int i = 0; i < 32; ++i)
             if (tc::mbar_try_wait(bar, phase)) return true;
         if (*abort_flag || tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) return false;
+    }
+}
+
+// Epilogue of one output tile for the calling thread's row: reads `width`
+// accumulator columns from tensor memory at tbase (SwiGLU: the gate products
+// in the first half, the up products in the second) whose outputs go to
+// columns col0.. of the row, and writes the epilogue's outputs (see the file
+// comment).  With the next norm's operand, the row's sum of squares over those
+// columns goes to partial-sum slot ssq_slot.
+__device__ __forceinline__ void epilogue_row(const Params &p, const Problem &pr, uint32_t tbase, int row, int width,
+                                             int col0, int ssq_slot) {
+    const bool row_ok = row < p.M;
+    float rs = 1.f;
+    if (row_ok && pr.ssq_in) {
+        // RMSNorm factor from the producer's per-tile sums of squares, added in order
+        float ss = 0.f;
+        for (int t = 0; t < p.ssq_parts; ++t)
+            if (SR_IN_BOUNDS(size_t(t) * p.M + row, (long long)p.ssq_parts * p.M, p.status))
+                ss += pr.ssq_in[size_t(t) * p.M + row];
+        rs = 1.f / sqrtf(ss / float(p.K) + p.eps);
+    } else if (row_ok && pr.rowscale) {
+        rs = pr.rowscale[row];
+    }
+    if (p.epi == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < width / 2; c += 32) {
+            uint32_t g[32], u[32];
+            tc::tmem_ld_32x32b_x32(tbase + c, g);
+            tc::tmem_ld_32x32b_x32(tbase + width / 2 + c, u);
+            tc::tmem_ld_wait();
+            const int col = col0 + c;
+            int nvec = min(4, (p.N - col) / 8);  // 8-column groups in range
+            if (row_ok && nvec > 0 &&
+                !SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
+                nvec = 0;
+            if (row_ok && nvec > 0) {
+                __nv_bfloat16 *cb = static_cast<__nv_bfloat16 *>(pr.c);
+                uint4 *dst = reinterpret_cast<uint4 *>(cb + size_t(row) * p.ldc + col);
+                uint4 *dlo = pr.c_lo && !p.lo_fp8
+                                 ? reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c_lo) +
+                                                             size_t(row) * p.ldc + col)
+                                 : nullptr;
+                uint2 *dlo8 = pr.c_lo && p.lo_fp8
+                                  ? reinterpret_cast<uint2 *>(static_cast<uint8_t *>(pr.c_lo) +
+                                                              size_t(row) * p.ldc + col)
+                                  : nullptr;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    if (v >= nvec) break;
+                    uint32_t w[4], wl[4];
+                    float lo[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = v * 8 + e * 2;
+                        const float h0 = silu(rs * __uint_as_float(g[j])) * (rs * __uint_as_float(u[j]));
+                        const float h1 = silu(rs * __uint_as_float(g[j + 1])) * (rs * __uint_as_float(u[j + 1]));
+                        w[e] = pack2(h0, h1);
+                        lo[2 * e] = h0 - bf_lo(w[e]);
+                        lo[2 * e + 1] = h1 - bf_hi(w[e]);
+                        wl[e] = pack2(lo[2 * e], lo[2 * e + 1]);
+                    }
+                    dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (dlo) dlo[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                    if (dlo8) dlo8[v] = lo8_pack8(lo);
+                }
+            }
+        }
+    } else {
+        // the next RMSNorm's operand (EPI_F32_RESIDUAL with nw): x * nw and sum x^2
+        const bool norm_out = p.epi == EPI_F32_RESIDUAL && pr.nw != nullptr;
+        float ssq = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < width; c += 32) {
+            uint32_t x[32];
+            tc::tmem_ld_32x32b_x32(tbase + c, x);
+            tc::tmem_ld_wait();
+            const int col = col0 + c;
+            const int nvec = min(4, (p.N - col) / 8);
+            if (!row_ok || nvec <= 0) continue;
+            if (!SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
+                continue;
+            if (p.epi == EPI_F32_ROWSCALE || p.epi == EPI_F32_RESIDUAL) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(pr.c) + size_t(row) * p.ldc + col);
+                const bool resid = p.epi == EPI_F32_RESIDUAL;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    if (v >= 2 * nvec) break;
+                    float4 o = make_float4(rs * __uint_as_float(x[4 * v]), rs * __uint_as_float(x[4 * v + 1]),
+                                           rs * __uint_as_float(x[4 * v + 2]), rs * __uint_as_float(x[4 * v + 3]));
+                    if (resid) {
+                        const float4 rv = dst[v];
+                        o.x += rv.x; o.y += rv.y; o.z += rv.z; o.w += rv.w;
+                    }
+                    dst[v] = o;
+                    x[4 * v] = __float_as_uint(o.x);
+                    x[4 * v + 1] = __float_as_uint(o.y);
+                    x[4 * v + 2] = __float_as_uint(o.z);
+                    x[4 * v + 3] = __float_as_uint(o.w);
+                }
+                if (norm_out &&
+                    SR_IN_BOUNDS(size_t(row) * p.N + col + 8 * nvec - 1, (long long)p.M * p.N, p.status)) {
+                    uint4 *dhi = reinterpret_cast<uint4 *>(pr.n_hi + size_t(row) * p.N + col);
+                    const uint4 *wv = reinterpret_cast<const uint4 *>(pr.nw + col);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (v >= nvec) break;
+                        const uint4 wq = wv[v];
+                        const uint32_t ww[4] = {wq.x, wq.y, wq.z, wq.w};
+                        uint32_t w[4], wl[4];
+                        float lo[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = v * 8 + e * 2;
+                            const float x0 = __uint_as_float(x[j]), x1 = __uint_as_float(x[j + 1]);
+                            ssq = fmaf(x0, x0, ssq);
+                            ssq = fmaf(x1, x1, ssq);
+                            const float h0 = x0 * bf_lo(ww[e]), h1 = x1 * bf_hi(ww[e]);
+                            w[e] = pack2(h0, h1);
+                            lo[2 * e] = h0 - bf_lo(w[e]);
+                            lo[2 * e + 1] = h1 - bf_hi(w[e]);
+                            wl[e] = pack2(lo[2 * e], lo[2 * e + 1]);
+                        }
+                        dhi[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                        if (pr.n_lo && p.lo_fp8)
+                            reinterpret_cast<uint2 *>(static_cast<uint8_t *>(pr.n_lo) + size_t(row) * p.N + col)[v] =
+                                lo8_pack8(lo);
+                        else if (pr.n_lo)
+                            reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.n_lo) + size_t(row) * p.N +
+                                                      col)[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                    }
+                }
+                continue;
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c) + size_t(row) * p.ldc + col);
+            const uint4 *res = p.epi == EPI_RESIDUAL
+                                   ? reinterpret_cast<const uint4 *>(pr.r + size_t(row) * p.ldc + col)
+                                   : nullptr;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                if (v >= nvec) break;
+                uint32_t rr[4] = {0u, 0u, 0u, 0u};
+                if (res) {
+                    const uint4 rv = res[v];
+                    rr[0] = rv.x; rr[1] = rv.y; rr[2] = rv.z; rr[3] = rv.w;
+                }
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = v * 8 + e * 2;
+                    w[e] = pack2(bf_lo(rr[e]) + rs * __uint_as_float(x[j]),
+                                 bf_hi(rr[e]) + rs * __uint_as_float(x[j + 1]));
+                }
+                dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        const size_t si = size_t(ssq_slot) * p.M + row;
+        if (norm_out && row_ok && SR_IN_BOUNDS(si, (long long)p.ssq_slots * p.M, p.status)) pr.ssq_out[si] = ssq;
     }
 }
 
@@ -166,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             int stage = 0;
             uint32_t phase = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-                const int pi = tile / tiles_per_prob, rem = tile % tiles_per_prob;
-                const int nt = rem / p.m_tiles, mt = rem % p.m_tiles;
+                int pi, nt, mt;
+                decode_tile(p, tile, pi, nt, mt);
                 const Problem &pr = p.prob[pi];
                 for (int kk = 0; kk < kblocks_all; ++kk) {
                     const bool lo = kk >= kblocks;
@@ -191,11 +370,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
-            constexpr uint32_t idesc_f8 = tc::idesc_e4m3_e5m2_f32(BM, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                // a last N tile narrower than BN runs products of its own width (a multiple of 16)
+                int pi, nt, mt;
+                decode_tile(p, tile, pi, nt, mt);
+                const int ncols = p.epi == EPI_SWIGLU ? BN : min(BN, (p.N - nt * BN + 15) / 16 * 16);
+                const uint32_t idesc = tc::idesc_bf16_f32(BM, ncols);
+                const uint32_t idesc_f8 = tc::idesc_e4m3_e5m2_f32(BM, ncols);
                 if (!wait_or_abort(&tempty[acc], acc_phase ^ 1, abort_flag)) { fail(); break; }
                 tc::tc_fence_after();
                 const uint32_t d = tmem + uint32_t(acc * BN);
@@ -233,109 +416,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-            const int pi = tile / tiles_per_prob, rem = tile % tiles_per_prob;
-            const int nt = rem / p.m_tiles, mt = rem % p.m_tiles;
+            int pi, nt, mt;
+            decode_tile(p, tile, pi, nt, mt);
             const Problem &pr = p.prob[pi];
             if (!wait_or_abort(&tfull[acc], acc_phase, abort_flag)) { fail(); break; }
             tc::tc_fence_after();
-            const int row = mt * BM + quad * 32 + lane;
-            const bool row_ok = row < p.M;
-            const uint32_t tbase = tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN);
-            const float rs = (pr.rowscale && row_ok) ? pr.rowscale[row] : 1.f;
-            if (p.epi == EPI_SWIGLU) {
-#pragma unroll 1
-                for (int c = 0; c < BN / 2; c += 32) {
-                    uint32_t g[32], u[32];
-                    tc::tmem_ld_32x32b_x32(tbase + c, g);
-                    tc::tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
-                    tc::tmem_ld_wait();
-                    const int col = nt * (BN / 2) + c;
-                    int nvec = min(4, (p.N - col) / 8);  // 8-column groups in range
-                    if (row_ok && nvec > 0 &&
-                        !SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
-                        nvec = 0;
-                    if (row_ok && nvec > 0) {
-                        __nv_bfloat16 *cb = static_cast<__nv_bfloat16 *>(pr.c);
-                        uint4 *dst = reinterpret_cast<uint4 *>(cb + size_t(row) * p.ldc + col);
-                        uint4 *dlo = pr.c_lo && !p.lo_fp8
-                                         ? reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c_lo) +
-                                                                     size_t(row) * p.ldc + col)
-                                         : nullptr;
-                        uint2 *dlo8 = pr.c_lo && p.lo_fp8
-                                          ? reinterpret_cast<uint2 *>(static_cast<uint8_t *>(pr.c_lo) +
-                                                                      size_t(row) * p.ldc + col)
-                                          : nullptr;
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            if (v >= nvec) break;
-                            uint32_t w[4], wl[4];
-                            float lo[8];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = v * 8 + e * 2;
-                                const float h0 = silu(rs * __uint_as_float(g[j])) * (rs * __uint_as_float(u[j]));
-                                const float h1 = silu(rs * __uint_as_float(g[j + 1])) * (rs * __uint_as_float(u[j + 1]));
-                                w[e] = pack2(h0, h1);
-                                lo[2 * e] = h0 - bf_lo(w[e]);
-                                lo[2 * e + 1] = h1 - bf_hi(w[e]);
-                                wl[e] = pack2(lo[2 * e], lo[2 * e + 1]);
-                            }
-                            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                            if (dlo) dlo[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                            if (dlo8) dlo8[v] = lo8_pack8(lo);
-                        }
-                    }
-                }
-            } else {
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t x[32];
-                    tc::tmem_ld_32x32b_x32(tbase + c, x);
-                    tc::tmem_ld_wait();
-                    const int col = nt * BN + c;
-                    const int nvec = min(4, (p.N - col) / 8);
-                    if (!row_ok || nvec <= 0) continue;
-                    if (!SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
-                        continue;
-                    if (p.epi == EPI_F32_ROWSCALE || p.epi == EPI_F32_RESIDUAL) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(pr.c) + size_t(row) * p.ldc + col);
-                        const bool resid = p.epi == EPI_F32_RESIDUAL;
-#pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            if (v >= 2 * nvec) break;
-                            float4 o = make_float4(rs * __uint_as_float(x[4 * v]), rs * __uint_as_float(x[4 * v + 1]),
-                                                   rs * __uint_as_float(x[4 * v + 2]), rs * __uint_as_float(x[4 * v + 3]));
-                            if (resid) {
-                                const float4 rv = dst[v];
-                                o.x += rv.x; o.y += rv.y; o.z += rv.z; o.w += rv.w;
-                            }
-                            dst[v] = o;
-                        }
-                        continue;
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c) + size_t(row) * p.ldc + col);
-                    const uint4 *res = p.epi == EPI_RESIDUAL
-                                           ? reinterpret_cast<const uint4 *>(pr.r + size_t(row) * p.ldc + col)
-                                           : nullptr;
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (v >= nvec) break;
-                        uint32_t rr[4] = {0u, 0u, 0u, 0u};
-                        if (res) {
-                            const uint4 rv = res[v];
-                            rr[0] = rv.x; rr[1] = rv.y; rr[2] = rv.z; rr[3] = rv.w;
-                        }
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = v * 8 + e * 2;
-                            w[e] = pack2(bf_lo(rr[e]) + rs * __uint_as_float(x[j]),
-                                         bf_hi(rr[e]) + rs * __uint_as_float(x[j + 1]));
-                        }
-                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                }
-            }
+            epilogue_row(p, pr, tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN), mt * BM + quad * 32 + lane, BN,
+                         p.epi == EPI_SWIGLU ? nt * (BN / 2) : nt * BN, nt);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&tempty[acc]);
@@ -353,6 +440,199 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, 2 * BN);
     }
+}
+
+// ------------------------------------------------------------------ CTA pairs
+// The same GEMM with each output tile of 256 rows x 256 columns computed by a
+// cluster of two CTAs on two SMs through cta_group::2 products: CTA r of the
+// pair loads rows r*128.. of the tile's A rows and its half of the tile's B
+// rows (for SwiGLU: the gate rows in CTA 0, the up rows in CTA 1) into its own
+// shared memory, and holds rows r*128.. of the accumulator in its own tensor
+// memory.  Each SM thus streams 32 KB per 64-deep K block instead of 48 KB,
+// for the same tensor work.  The even CTA issues every product; both CTAs'
+// loads signal its stage barriers, its commits arrive at both CTAs' stage and
+// accumulator barriers, and both CTAs' epilogue warps release its accumulator
+// buffers.  The arithmetic of every output element (the K blocks in order,
+// fp32 accumulation in tensor memory) is that of the single-CTA form.
+constexpr int kPairStages = 6;
+constexpr int kPairSmemBytes = kPairStages * 2 * kTileA + 1024 /*align*/ + 256 /*barriers*/;
+
+__device__ __forceinline__ bool wait_or_abort_cluster(uint64_t *bar, uint32_t phase, volatile int *abort_flag) {
+    if (tc::mbar_try_wait_cluster(bar, phase)) return true;
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (tc::mbar_try_wait_cluster(bar, phase)) return true;
+        if (*abort_flag || tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) return false;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_constant__ Params p) {
+    constexpr int BN = 256, STAGES = kPairStages, kTileB = kTileA;  // B: this CTA's 128 rows
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * kTileA;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + STAGES * kTileB);  // used in the even CTA
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;  // used in the even CTA: 4 epilogue warps of each CTA arrive
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = tc::cluster_ctarank();
+    const bool leader = rank == 0;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&tfull[b], 1);
+            tc::mbar_init(&tempty[b], 8);
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc_pair(tmem_slot, 2 * BN);
+        tc::tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < p.n_problems; ++i) {
+            tc::prefetch_tmap(&p.prob[i].a);
+            if (p.n_pass == 2) tc::prefetch_tmap(&p.prob[i].a_lo);
+            if (p.lo_fp8) {
+                tc::prefetch_tmap(&p.prob[i].b0_lo);
+                if (p.epi == EPI_SWIGLU) tc::prefetch_tmap(&p.prob[i].b1_lo);
+            }
+            tc::prefetch_tmap(&p.prob[i].b0);
+            if (p.epi == EPI_SWIGLU) tc::prefetch_tmap(&p.prob[i].b1);
+        }
+    }
+    // the barriers of both CTAs are initialised before either CTA uses its pair's
+    __syncwarp();
+    tc::tc_fence_before();
+    tc::cluster_sync();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int tiles_per_prob = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row tiles here
+    const int total = p.n_problems * tiles_per_prob;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int kblocks = p.K / BK;
+    const int kblocks_lo = p.n_pass == 2 ? (p.lo_fp8 ? p.K / (2 * BK) : kblocks) : 0;
+    const int kblocks_all = kblocks + kblocks_lo;
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(p.status, SR_DEV_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t full0 = tc::mapa_shared(tc::smem_u32(full), 0);  // the even CTA's stage barriers
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = pair; tile < total && !*abort_flag; tile += n_pairs) {
+                int pi, nt, mt;
+                decode_tile(p, tile, pi, nt, mt);
+                const Problem &pr = p.prob[pi];
+                for (int kk = 0; kk < kblocks_all; ++kk) {
+                    const bool lo = kk >= kblocks;
+                    const bool f8 = lo && p.lo_fp8;
+                    const int kb = lo ? kk - kblocks : kk;
+                    const int kx = f8 ? kb * 2 * BK : kb * BK;
+                    const CUtensorMap *mb0 = f8 ? &pr.b0_lo : &pr.b0, *mb1 = f8 ? &pr.b1_lo : &pr.b1;
+                    if (!wait_or_abort(&empty[stage], phase ^ 1, abort_flag)) { fail(); break; }
+                    // the even CTA's barrier expects both CTAs' bytes of the stage
+                    if (leader) tc::mbar_arrive_expect_tx(&full[stage], 2 * (kTileA + kTileB));
+                    const uint32_t fb = full0 + uint32_t(stage) * 8u;
+                    tc::tma_load_2d_pair(sA + stage * kTileA, lo ? &pr.a_lo : &pr.a, fb, kx,
+                                         mt * 2 * BM + int(rank) * BM);
+                    if (p.epi == EPI_SWIGLU)
+                        tc::tma_load_2d_pair(sB + stage * kTileB, leader ? mb0 : mb1, fb, kx, nt * (BN / 2));
+                    else
+                        tc::tma_load_2d_pair(sB + stage * kTileB, mb0, fb, kx, nt * BN + int(rank) * (BN / 2));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(2 * BM, BN);
+            constexpr uint32_t idesc_f8 = tc::idesc_e4m3_e5m2_f32(2 * BM, BN);
+            for (int tile = pair; tile < total && !*abort_flag; tile += n_pairs) {
+                if (!wait_or_abort_cluster(&tempty[acc], acc_phase ^ 1, abort_flag)) { fail(); break; }
+                tc::tc_fence_after();
+                const uint32_t d = tmem + uint32_t(acc * BN);
+                bool ok = true;
+                for (int kb = 0; kb < kblocks_all; ++kb) {
+                    if (!wait_or_abort(&full[stage], phase, abort_flag)) { fail(); ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint32_t a0 = tc::smem_u32(sA + stage * kTileA);
+                    const uint32_t b0 = tc::smem_u32(sB + stage * kTileB);
+                    if (p.lo_fp8 && kb >= kblocks) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_f8_ss_pair(d, tc::sdesc_k_sw128(a0 + k * 32), tc::sdesc_k_sw128(b0 + k * 32),
+                                               idesc_f8, 1);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            tc::mma_bf16_ss_pair(d, tc::sdesc_k_sw128(a0 + k * 32), tc::sdesc_k_sw128(b0 + k * 32),
+                                                 idesc, (kb | k) != 0);
+                    }
+                    tc::mma_commit_pair(&empty[stage], 0x3);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc::mma_commit_pair(&tfull[acc], 0x3);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            tc::mma_commit_pair(drain, 0x3);
+        }
+        // in both CTAs: every product writing this CTA's tensor memory has completed
+        if (lane == 0 && !tc::mbar_wait(drain, 0)) atomicOr(p.status, SR_DEV_TIMEOUT);
+    } else {
+        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        const uint32_t tempty0 = tc::mapa_shared(tc::smem_u32(tempty), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < total && !*abort_flag; tile += n_pairs) {
+            int pi, nt, mt;
+            decode_tile(p, tile, pi, nt, mt);
+            const Problem &pr = p.prob[pi];
+            if (!wait_or_abort(&tfull[acc], acc_phase, abort_flag)) { fail(); break; }
+            tc::tc_fence_after();
+            epilogue_row(p, pr, tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN),
+                         mt * 2 * BM + int(rank) * BM + quad * 32 + lane, BN,
+                         p.epi == EPI_SWIGLU ? nt * (BN / 2) : nt * BN, nt);
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+
+    if (*abort_flag) {
+        // let TMA copies already in flight land before the shared memory is released
+        for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    }
+    __syncwarp();
+    tc::tc_fence_before();
+    tc::cluster_sync();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc_pair(tmem, 2 * BN);
+    }
+    // neither CTA leaves while the other may still arrive at its barriers
+    __syncwarp();
+    tc::cluster_sync();
 }
 
 // ------------------------------------------------------------------ host
@@ -429,12 +709,10 @@ bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int pitch, i
 
 namespace {
 
-template <int BN>
-cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
-                        int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st) {
-    Params local{};
-    const int bn_out = epi == EPI_SWIGLU ? BN / 2 : BN;
-    const int bn_rows = epi == EPI_SWIGLU ? BN / 2 : BN;  // rows of each weight box
+// Tensor maps and scalars shared by both forms.  b_rows: rows of each weight box.
+cudaError_t fill_params(Params &local, const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc,
+                        int epi, int n_pass, int lo_fp8, uint32_t *status, GemmOptions norm, int b_rows, int bn_out,
+                        int bm_tile) {
     for (int i = 0; i < n_problems; ++i) {
         const GemmProblemDesc &d = probs[i];
         if (!make_map(&local.prob[i].a, d.a, M, K, K, BM)) return cudaErrorInvalidValue;
@@ -443,30 +721,53 @@ cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int
                                    : make_map(&local.prob[i].a_lo, d.a_lo, M, K, K, BM);
             if (!ok) return cudaErrorInvalidValue;
         }
-        if (!make_map(&local.prob[i].b0, d.b0, N, K, K, bn_rows)) return cudaErrorInvalidValue;
-        if (epi == EPI_SWIGLU && !make_map(&local.prob[i].b1, d.b1, N, K, K, bn_rows)) return cudaErrorInvalidValue;
+        if (!make_map(&local.prob[i].b0, d.b0, N, K, K, b_rows)) return cudaErrorInvalidValue;
+        if (epi == EPI_SWIGLU && !make_map(&local.prob[i].b1, d.b1, N, K, K, b_rows)) return cudaErrorInvalidValue;
         if (n_pass == 2 && lo_fp8) {
-            if (!d.b0_lo || !make_map_u8(&local.prob[i].b0_lo, d.b0_lo, N, K, K, 2 * BK, bn_rows))
+            if (!d.b0_lo || !make_map_u8(&local.prob[i].b0_lo, d.b0_lo, N, K, K, 2 * BK, b_rows))
                 return cudaErrorInvalidValue;
-            if (epi == EPI_SWIGLU && (!d.b1_lo || !make_map_u8(&local.prob[i].b1_lo, d.b1_lo, N, K, K, 2 * BK, bn_rows)))
+            if (epi == EPI_SWIGLU && (!d.b1_lo || !make_map_u8(&local.prob[i].b1_lo, d.b1_lo, N, K, K, 2 * BK, b_rows)))
                 return cudaErrorInvalidValue;
         }
         local.prob[i].c = d.c;
         local.prob[i].r = static_cast<const __nv_bfloat16 *>(d.r);
         local.prob[i].c_lo = d.c_lo;
         local.prob[i].rowscale = d.rowscale;
+        local.prob[i].ssq_in = d.ssq_in;
+        local.prob[i].nw = static_cast<const __nv_bfloat16 *>(d.nw);
+        local.prob[i].n_hi = static_cast<__nv_bfloat16 *>(d.n_hi);
+        local.prob[i].n_lo = d.n_lo;
+        local.prob[i].ssq_out = d.ssq_out;
     }
     local.n_problems = n_problems;
     local.M = M;
     local.N = N;
     local.K = K;
     local.ldc = ldc;
-    local.m_tiles = (M + BM - 1) / BM;
+    local.m_tiles = (M + bm_tile - 1) / bm_tile;
     local.n_tiles = (N + bn_out - 1) / bn_out;
     local.epi = epi;
     local.n_pass = n_pass;
     local.lo_fp8 = n_pass == 2 && lo_fp8;
+    local.ssq_parts = norm.ssq_parts;
+    local.eps = norm.eps;
+    local.nt_skip_at = norm.n_skip_lo / kGemmTileN;
+    local.nt_skip = (norm.n_skip_hi - norm.n_skip_lo) / kGemmTileN;
+    local.ssq_slots = local.n_tiles;
+    local.n_tiles -= local.nt_skip;
     local.status = status;
+    return cudaSuccess;
+}
+
+template <int BN>
+cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
+                        int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st, GemmOptions norm) {
+    Params local{};
+    const int bn_out = epi == EPI_SWIGLU ? BN / 2 : BN;
+    const int bn_rows = epi == EPI_SWIGLU ? BN / 2 : BN;  // rows of each weight box
+    cudaError_t e0 = fill_params(local, probs, n_problems, M, N, K, ldc, epi, n_pass, lo_fp8, status, norm, bn_rows,
+                                 bn_out, BM);
+    if (e0 != cudaSuccess) return e0;
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<BN>::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -477,18 +778,64 @@ cudaError_t launch_gemm(const GemmProblemDesc *probs, int n_problems, int M, int
     return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_pair(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
+                             int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st, GemmOptions norm) {
+    constexpr int BN = 256;
+    Params local{};
+    const int bn_out = epi == EPI_SWIGLU ? BN / 2 : BN;
+    // each CTA of a pair loads 128 weight rows: half the tile's B rows, or for
+    // SwiGLU the tile's gate rows (even CTA) or up rows (odd CTA)
+    cudaError_t e = fill_params(local, probs, n_problems, M, N, K, ldc, epi, n_pass, lo_fp8, status, norm, BN / 2,
+                                bn_out, 2 * BM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int total = n_problems * local.m_tiles * local.n_tiles;
+    const int pairs = sm_count() / 2;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * (total < pairs ? total : pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, local);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
-                    int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st) {
+                    int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st, GemmOptions norm) {
     if (n_problems <= 0 || n_problems > kMaxGemmProblems || M <= 0 || N <= 0 || K <= 0 || K % BK != 0 ||
         N % 8 != 0 || ldc % 8 != 0 || ldc < N || (n_pass != 1 && n_pass != 2) ||
         (n_pass == 2 && lo_fp8 && K % (2 * BK) != 0))
         return cudaErrorInvalidValue;
+    for (int i = 0; i < n_problems; ++i) {
+        const GemmProblemDesc &d = probs[i];
+        if (d.ssq_in && (norm.ssq_parts <= 0 || !(norm.eps > 0.f) || epi == EPI_F32_RESIDUAL || epi == EPI_STORE ||
+                         epi == EPI_RESIDUAL))
+            return cudaErrorInvalidValue;
+        if (d.nw && (epi != EPI_F32_RESIDUAL || !d.n_hi || !d.ssq_out || (n_pass == 2) != (d.n_lo != nullptr)))
+            return cudaErrorInvalidValue;
+        if (norm.n_skip_hi > norm.n_skip_lo && d.nw) return cudaErrorInvalidValue;
+    }
+    if (norm.n_skip_lo < 0 || norm.n_skip_hi < norm.n_skip_lo || norm.n_skip_lo % kGemmTileN ||
+        norm.n_skip_hi % kGemmTileN || norm.n_skip_hi >= N || (norm.n_skip_hi > norm.n_skip_lo && epi == EPI_SWIGLU))
+        return cudaErrorInvalidValue;
     // 256-wide tiles: measured against 128-wide ones on the group shapes, they stay
     // ahead even where the 128-wide tiling fills the last wave of SMs better
     // (the A tile is then streamed twice as often).
-    return launch_gemm<256>(probs, n_problems, M, N, K, ldc, epi, n_pass, lo_fp8, status, st);
+    static_assert(kGemmTileN == 256, "the partial sums of squares come one per 256-wide tile");
+    if (norm.form == GEMM_FORM_PAIR)
+        return launch_gemm_pair(probs, n_problems, M, N, K, ldc, epi, n_pass, lo_fp8, status, st, norm);
+    return launch_gemm<256>(probs, n_problems, M, N, K, ldc, epi, n_pass, lo_fp8, status, st, norm);
 }
 
 }  // namespace sr

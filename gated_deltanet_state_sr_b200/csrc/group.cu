@@ -11,8 +11,13 @@
 // every group through per-group pointers):
 //   row_prep(x, w_in_norm) -> in_proj GEMM (fp32 out, RMSNorm factor in the
 //   epilogue) -> conv + gates (+ conv state) -> chunked gated-delta recurrence
-//   -> gated norm -> out_proj GEMM (+= residual) -> row_prep(x, w_post_norm)
-//   -> gate/up GEMM (SwiGLU epilogue) -> down GEMM (+= residual).
+//   -> gated norm -> out_proj GEMM (+= residual) -> gate/up GEMM (SwiGLU
+//   epilogue) -> down GEMM (+= residual).
+// Only layer 0 runs row_prep (it also gathers the anchors): the out_proj and
+// down epilogues form the next RMSNorm's operand (x * w as hi + lo) from the
+// updated residual rows, with each row's sum of squares per 256-column tile,
+// and the GEMM that consumes the operand adds those sums in order into its
+// RMSNorm factor.
 // In skip mode the last layer stops after its recurrence: its gated norm,
 // out_proj and MLP change no state ("Tail-Replay", Sec. 3 omits the final
 // group FFN).  The residual stream is kept in fp32 between layers.
@@ -52,10 +57,13 @@ Dims dims_of(const sr_group_args &a) {
 }
 
 struct GroupBufs {
-    float *x32, *r, *p, *gate, *beta;
+    float *x32, *r, *ssq, *p, *gate, *beta;
     __nv_bfloat16 *a_hi, *q, *k, *k_lo, *v, *v_lo, *o, *h_hi;
     void *a_lo, *h_lo;  // bf16, or e4m3 bytes with the fp8 low pass
 };
+
+// Partial sums of squares per hidden row: one per 256-column GEMM tile.
+int ssq_parts(const Dims &m) { return (m.H + kGemmTileN - 1) / kGemmTileN; }
 
 // Carves the per-group scratch buffers, then the chunk images of the two-phase
 // gated-delta kernels (shared by the layers; *img), out of the workspace
@@ -69,25 +77,28 @@ size_t carve(const Dims &m, char *base, GroupBufs *out, void **img = nullptr) {
         return ptr;
     };
     const size_t T = size_t(m.T);
-    const size_t amax = size_t(m.H > m.vd ? m.H : m.vd);
+    // A holds the RMSNorm operands [T, H]; the MLP buffer h holds the SwiGLU output
+    // [T, I] and, before out_proj, the gated norm's y [T, h_v d_v]
+    const size_t hmax = size_t(m.I > m.vd ? m.I : m.vd);
     for (int g = 0; g < m.G; ++g) {
         GroupBufs b;
         b.x32 = reinterpret_cast<float *>(take(T * m.H * 4));
         b.r = reinterpret_cast<float *>(take(T * 4));
+        b.ssq = reinterpret_cast<float *>(take(T * ssq_parts(m) * 4));
         b.p = reinterpret_cast<float *>(take(T * m.proj * 4));
         b.gate = reinterpret_cast<float *>(take(T * m.hv * 4));
         b.beta = reinterpret_cast<float *>(take(T * m.hv * 4));
-        b.a_hi = reinterpret_cast<__nv_bfloat16 *>(take(T * amax * 2));
+        b.a_hi = reinterpret_cast<__nv_bfloat16 *>(take(T * m.H * 2));
         const size_t lo_elem = m.lo8 ? 1 : 2;
-        b.a_lo = m.split ? take(T * amax * lo_elem) : nullptr;
+        b.a_lo = m.split ? take(T * m.H * lo_elem) : nullptr;
         b.q = reinterpret_cast<__nv_bfloat16 *>(take(T * m.qd * 2));
         b.k = reinterpret_cast<__nv_bfloat16 *>(take(T * m.qd * 2));
         b.k_lo = m.split ? reinterpret_cast<__nv_bfloat16 *>(take(T * m.qd * 2)) : nullptr;
         b.v = reinterpret_cast<__nv_bfloat16 *>(take(T * m.vd * 2));
         b.v_lo = m.split ? reinterpret_cast<__nv_bfloat16 *>(take(T * m.vd * 2)) : nullptr;
         b.o = reinterpret_cast<__nv_bfloat16 *>(take(T * m.vd * 2));
-        b.h_hi = reinterpret_cast<__nv_bfloat16 *>(take(T * m.I * 2));
-        b.h_lo = m.split ? take(T * m.I * lo_elem) : nullptr;
+        b.h_hi = reinterpret_cast<__nv_bfloat16 *>(take(T * hmax * 2));
+        b.h_lo = m.split ? take(T * hmax * lo_elem) : nullptr;
         if (out) out[g] = b;
     }
     void *im = take(gdn_tc_supported(m.d) ? gdn_tc_image_bytes(m.T, m.N, m.hv, m.G) : 0);
@@ -225,31 +236,54 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         auto O = [&](int g) -> const sr_layer_outputs & { return a->outputs[g * m.L + l]; };
         auto I = [&](int g) -> const sr_layer_state * { return a->initial ? &a->initial[g * m.L + l] : nullptr; };
 
-        // (1) A = x * w_in_norm (hi/lo), r = RMSNorm factor; layer 0 also seeds the fp32 residual stream
-        RowPrepBatch rp{};
-        for (int g = 0; g < G; ++g) {
-            rp.x[g] = l == 0 ? a->anchors[g] : static_cast<const void *>(B[g].x32);
-            rp.w[g] = static_cast<const __nv_bfloat16 *>(W(g).w_in_norm);
-            rp.a_hi[g] = B[g].a_hi;
-            rp.a_lo[g] = B[g].a_lo;
-            rp.r[g] = B[g].r;
-            rp.x32_out[g] = l == 0 ? B[g].x32 : nullptr;
+        // (1) layer 0: A = x * w_in_norm (hi/lo) and r = RMSNorm factor from the anchors
+        // (gathered through the index table for sparse anchors), and the fp32 residual
+        // stream; later layers find A and the partial sums in place (step 8)
+        if (l == 0) {
+            RowPrepBatch rp{};
+            for (int g = 0; g < G; ++g) {
+                rp.x[g] = a->anchors[g];
+                rp.w[g] = static_cast<const __nv_bfloat16 *>(W(g).w_in_norm);
+                rp.a_hi[g] = B[g].a_hi;
+                rp.a_lo[g] = B[g].a_lo;
+                rp.r[g] = B[g].r;
+                rp.x32_out[g] = B[g].x32;
+            }
+            rp.T = T; rp.H = m.H; rp.x_f32 = 0; rp.eps = a->eps; rp.lo8 = m.lo8;
+            rp.idx = a->anchor_index;
+            rp.x_rows = a->anchor_index ? a->anchor_rows : T;
+            rp.status = status;
+            SR_TRY(prof.begin(SR_K_ROW_PREP));
+            SR_TRY(row_prep(rp, G, st));
+            SR_TRY(prof.end());
         }
-        rp.T = T; rp.H = m.H; rp.x_f32 = l == 0 ? 0 : 1; rp.eps = a->eps; rp.lo8 = m.lo8;
-        rp.idx = l == 0 ? a->anchor_index : nullptr;  // sparse anchors: gather from the pool
-        rp.x_rows = a->anchor_index ? a->anchor_rows : T;
-        rp.status = status;
-        SR_TRY(prof.begin(SR_K_ROW_PREP));
-        SR_TRY(row_prep(rp, G, st));
-        SR_TRY(prof.end());
+        GemmOptions rn;
+        rn.ssq_parts = ssq_parts(m);
+        rn.eps = a->eps;
+        // Tile form per projection, as measured on the whole-model replay (8 groups of
+        // 1639 tokens, hidden 2560): CTA pairs for in_proj, out_proj and down_proj, whose
+        // tiles then take 13 % less time per round; one CTA per tile for gate/up, where
+        // the pairs' padding of M to 256 rows costs more than their rounds gain.
+        GemmOptions pair_opt;
+        pair_opt.form = GEMM_FORM_PAIR;
 
-        // (2) p = r * (A W_in^T), fp32
+        // (2) p = r * (A W_in^T), fp32.  When the layer stops after its recurrence, the
+        // z columns (read only by the gated norm) are not computed where they span
+        // whole GEMM tiles.
         GemmProblemDesc gp[kMaxGemmProblems];
-        for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_in, nullptr, B[g].p, nullptr, nullptr, B[g].r,
-                                    W(g).w_in_lo8, nullptr};
+        for (int g = 0; g < G; ++g) {
+            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_in, nullptr, B[g].p, nullptr, nullptr,
+                                    l == 0 ? B[g].r : nullptr, W(g).w_in_lo8, nullptr};
+            if (l > 0) gp[g].ssq_in = B[g].ssq;
+        }
+        GemmOptions in_opt = rn;
+        in_opt.form = GEMM_FORM_PAIR;
+        if (stop && m.conv_dim % kGemmTileN == 0 && m.vd % kGemmTileN == 0) {
+            in_opt.n_skip_lo = m.conv_dim;
+            in_opt.n_skip_hi = m.conv_dim + m.vd;
+        }
         SR_TRY(prof.begin(SR_K_GEMM_IN));
-        SR_TRY(gemm_tc(gp, G, T, m.proj, m.H, m.proj, EPI_F32_ROWSCALE, npass, m.lo8, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.proj, m.H, m.proj, EPI_F32_ROWSCALE, npass, m.lo8, status, st, in_opt));
         SR_TRY(prof.end());
 
         // (3) conv + SiLU + L2 norm + gates, conv state
@@ -300,14 +334,15 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
             SR_TRY(cudaEventRecord(static_cast<cudaEvent_t>(a->layer_done[l]), st));
         if (stop) break;
 
-        // (5) y = RMSNorm_head(o) w_gnorm * SiLU(z) -> A (hi/lo)
+        // (5) y = RMSNorm_head(o) w_gnorm * SiLU(z) (hi/lo), into the MLP activation buffer
+        // (free here; the out_proj epilogue writes the next operand into A)
         GatedNormBatch gn{};
         for (int g = 0; g < G; ++g) {
             gn.o[g] = B[g].o;
             gn.p[g] = B[g].p;
             gn.w[g] = static_cast<const __nv_bfloat16 *>(W(g).w_gnorm);
-            gn.y_hi[g] = B[g].a_hi;
-            gn.y_lo[g] = B[g].a_lo;
+            gn.y_hi[g] = B[g].h_hi;
+            gn.y_lo[g] = B[g].h_lo;
         }
         gn.T = T; gn.h_v = m.hv; gn.ld = m.proj; gn.z_off = m.conv_dim; gn.eps = a->eps; gn.lo8 = m.lo8;
         gn.status = status;
@@ -315,44 +350,48 @@ extern "C" sr_status sr_group_replay(const sr_group_args *a, void *ws, size_t ws
         SR_TRY(gated_norm(gn, G, st));
         SR_TRY(prof.end());
 
-        // (6) x += y W_out^T
-        for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_out, nullptr, B[g].x32, nullptr, nullptr, nullptr,
-                                    W(g).w_out_lo8, nullptr};
-        SR_TRY(prof.begin(SR_K_GEMM_OUT));
-        SR_TRY(gemm_tc(gp, G, T, m.H, m.vd, m.H, EPI_F32_RESIDUAL, npass, m.lo8, status, st));
-        SR_TRY(prof.end());
-
-        // (7) A = x * w_post_norm, r
+        // (6) x += y W_out^T; the epilogue also forms A = x * w_post_norm (hi/lo) and the
+        // partial sums of x^2 of the post-attention RMSNorm
         for (int g = 0; g < G; ++g) {
-            rp.x[g] = B[g].x32;
-            rp.w[g] = static_cast<const __nv_bfloat16 *>(W(g).w_post_norm);
-            rp.x32_out[g] = nullptr;
+            gp[g] = GemmProblemDesc{B[g].h_hi, B[g].h_lo, W(g).w_out, nullptr, B[g].x32, nullptr, nullptr, nullptr,
+                                    W(g).w_out_lo8, nullptr};
+            gp[g].nw = W(g).w_post_norm;
+            gp[g].n_hi = B[g].a_hi;
+            gp[g].n_lo = B[g].a_lo;
+            gp[g].ssq_out = B[g].ssq;
         }
-        rp.x_f32 = 1;
-        rp.idx = nullptr;
-        rp.x_rows = T;
-        SR_TRY(prof.begin(SR_K_ROW_PREP));
-        SR_TRY(row_prep(rp, G, st));
+        SR_TRY(prof.begin(SR_K_GEMM_OUT));
+        SR_TRY(gemm_tc(gp, G, T, m.H, m.vd, m.H, EPI_F32_RESIDUAL, npass, m.lo8, status, st, pair_opt));
         SR_TRY(prof.end());
 
-        // (8) h = SiLU(r A W_gate^T) * (r A W_up^T) (hi/lo)
-        for (int g = 0; g < G; ++g)
-            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_gate, W(g).w_up, B[g].h_hi, nullptr, B[g].h_lo, B[g].r,
-                                    W(g).w_gate_lo8, W(g).w_up_lo8};
+        // (7) h = SiLU(r A W_gate^T) * (r A W_up^T) (hi/lo), r from the partial sums
+        for (int g = 0; g < G; ++g) {
+            gp[g] = GemmProblemDesc{B[g].a_hi, B[g].a_lo, W(g).w_gate, W(g).w_up, B[g].h_hi, nullptr, B[g].h_lo,
+                                    nullptr, W(g).w_gate_lo8, W(g).w_up_lo8};
+            gp[g].ssq_in = B[g].ssq;
+        }
         SR_TRY(prof.begin(SR_K_GEMM_GATEUP));
-        SR_TRY(gemm_tc(gp, G, T, m.I, m.H, m.I, EPI_SWIGLU, npass, m.lo8, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.I, m.H, m.I, EPI_SWIGLU, npass, m.lo8, status, st, rn));
         SR_TRY(prof.end());
 
-        // (9) x += h W_down^T
-        for (int g = 0; g < G; ++g)
+        // (8) x += h W_down^T; unless this is the last layer, the epilogue also forms the
+        // next layer's A = x * w_in_norm (hi/lo) and partial sums of x^2
+        const bool next = l + 1 < m.L;
+        for (int g = 0; g < G; ++g) {
             gp[g] = GemmProblemDesc{B[g].h_hi, B[g].h_lo, W(g).w_down, nullptr, B[g].x32, nullptr, nullptr, nullptr,
                                     W(g).w_down_lo8, nullptr};
+            if (next) {
+                gp[g].nw = a->weights[g * m.L + l + 1].w_in_norm;
+                gp[g].n_hi = B[g].a_hi;
+                gp[g].n_lo = B[g].a_lo;
+                gp[g].ssq_out = B[g].ssq;
+            }
+        }
         SR_TRY(prof.begin(SR_K_GEMM_DOWN));
-        SR_TRY(gemm_tc(gp, G, T, m.H, m.I, m.H, EPI_F32_RESIDUAL, npass, m.lo8, status, st));
+        SR_TRY(gemm_tc(gp, G, T, m.H, m.I, m.H, EPI_F32_RESIDUAL, npass, m.lo8, status, st, pair_opt));
         SR_TRY(prof.end());
 
-        // (10) optional bf16 copy of the hidden after this layer
+        // (9) optional bf16 copy of the hidden after this layer
         CastBatch cast{};
         int n_cast = 0;
         for (int g = 0; g < G; ++g)

@@ -129,11 +129,38 @@ struct GemmProblemDesc {
     const float *rowscale;  // [M] fp32 per-row scale, may be null (= 1)
     const void *b0_lo = nullptr;  // lo_fp8: e5m2(b0 * 2^-8) bytes [N, K]
     const void *b1_lo = nullptr;  // lo_fp8: e5m2(b1 * 2^-8) bytes [N, K] (SwiGLU)
+    // The next RMSNorm's operand, formed in the EPI_F32_RESIDUAL epilogue from the
+    // updated fp32 rows x: n_hi/n_lo = x * nw as hi + lo (lo as bf16, or as
+    // e4m3(lo * 2^8) bytes when lo_fp8; null in one-pass mode), row pitch N, and
+    // ssq_out[t * M + row] = sum of x^2 over the columns of N-tile t, in column order.
+    const void *nw = nullptr;     // [N] bf16 norm weight; null: no operand is formed
+    void *n_hi = nullptr;
+    void *n_lo = nullptr;
+    float *ssq_out = nullptr;     // [ceil(N / kGemmTileN), M]
+    // Row scale from such partial sums (in place of rowscale): 1 / sqrt(sum / K + eps),
+    // the parts added in order.
+    const float *ssq_in = nullptr;  // [ssq_parts, M]
+};
+// Output columns per GEMM tile (the partial sums of squares come one per tile).
+constexpr int kGemmTileN = 256;
+// How output tiles map to CTAs: one CTA per 128 x 256 tile (the default), or a
+// cluster of two CTAs (two SMs) per 256 x 256 tile sharing cta_group::2
+// products, which streams a third fewer operand bytes per SM for the same
+// tensor work but pads M to a multiple of 256.
+enum GemmForm { GEMM_FORM_DEFAULT = 0, GEMM_FORM_SINGLE = 1, GEMM_FORM_PAIR = 2 };
+struct GemmOptions {
+    int ssq_parts = 0;  // partial sums per row in ssq_in
+    float eps = 0.f;
+    int form = GEMM_FORM_DEFAULT;
+    // Output columns [n_skip_lo, n_skip_hi) that nobody reads: their tiles are not
+    // computed and those columns of C are left as they are.  Both bounds are
+    // multiples of kGemmTileN and n_skip_hi < N (not with EPI_SWIGLU or nw).
+    int n_skip_lo = 0, n_skip_hi = 0;
 };
 // n_pass 1: A only; 2: A_hi then A_lo.  lo_fp8: the A_lo pass runs on the fp8
 // tensor cores (e4m3 A_lo * 2^8 times e5m2 B * 2^-8); needs K % 128 == 0.
 cudaError_t gemm_tc(const GemmProblemDesc *probs, int n_problems, int M, int N, int K, int ldc, int epi,
-                    int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st);
+                    int n_pass, int lo_fp8, uint32_t *status, cudaStream_t st, GemmOptions norm = GemmOptions{});
 // fp8 low-pass helpers (layer_kernels.cu): e5m2(w * 2^-8) for n bf16 weights.
 cudaError_t prepare_lo8(const void *w, void *w_lo8, int64_t n, cudaStream_t st);
 

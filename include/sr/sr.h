@@ -216,7 +216,7 @@ SR_API sr_status sr_mamba2_replay(const sr_mamba2_args *args, void *workspace, s
  * Supported: n_groups <= 8, d_k = d_v = 128, conv_width = 4, hidden % 64 == 0,
  * inter % 64 == 0, (h_v d_v) % 64 == 0, h_v % h_k == 0.  Workspace: the size
  * sr_group_replay_workspace() returns (it grows linearly with total_tokens
- * and n_groups; about 160-175 KB per token per group at hidden 2560).
+ * and n_groups; about 135-170 KB per token per group at hidden 2560).
  * ---------------------------------------------------------------------- */
 typedef struct sr_layer_weights {
     const void *w_in_norm;   /* [hidden] bf16 */
@@ -362,10 +362,10 @@ SR_API sr_status sr_group_replay(const sr_group_args *args, void *workspace, siz
  *
  * Limit: a replay whose sr_group_replay_workspace() exceeds
  * SR_GROUP_NOALLOC_SCRATCH_BYTES is rejected with SR_ERR_WORKSPACE.  At
- * hidden 2560, intermediate 9216 and 32 V heads a group takes about 175 KB
- * per token with SR_PREC_SPLIT (162 KB with SR_PREC_SPLIT_FP8, 137 KB with
+ * hidden 2560, intermediate 9216 and 32 V heads a group takes about 169 KB
+ * per token with SR_PREC_SPLIT (158 KB with SR_PREC_SPLIT_FP8, 134 KB with
  * SR_PREC_BF16) plus 1.8 MB per sequence for the gated-delta chunk images,
- * so one sequence of up to 186 tokens fits (191 and 235).
+ * so one sequence of up to 191 tokens fits (197 and 241).
  * Set-up: a call made outside a stream capture looks up the array's device
  * address on the current device (cudaGetSymbolAddress), so the first call on
  * a device must come before any stream capture; a call inside a capture

@@ -22,9 +22,11 @@ extern "C" {
  *   epi 1:  c = r + a b0^T
  *   epi 2:  c = SiLU(a b0^T) * (a b1^T)
  * a [m, k], b0 / b1 [n, k], c and r [m, n]; all bf16 row-major; k % 64 == 0,
- * n % 32 == 0.  workspace >= 256 bytes. */
+ * n % 32 == 0.  workspace >= 256 bytes.  form: 0 the library's default, 1 one
+ * CTA per 128 x 256 output tile, 2 a cluster of two CTAs (two SMs) per
+ * 256 x 256 tile sharing cta_group::2 products; both give bit-identical c. */
 SR_API sr_status sr_test_gemm(const void *a, const void *b0, const void *b1, void *c, const void *r,
-                              int32_t m, int32_t n, int32_t k, int32_t epi, void *workspace,
+                              int32_t m, int32_t n, int32_t k, int32_t epi, int32_t form, void *workspace,
                               size_t workspace_bytes, void *stream);
 
 /* A bounded on-chip wait made to run out.  The paper has no counterpart: this

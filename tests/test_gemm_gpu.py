@@ -73,3 +73,36 @@ def test_swiglu(sr, m, n, k):
     ws = sr.workspace(256)
     sr.test_gemm(a, bg, b1=bu, epi=sr.EPI_SWIGLU, ws=ws)
     assert sr.device_status(ws) == 0
+
+
+@pytest.mark.parametrize("epi,m,n,k", [
+    ("store", 130, 96, 128),      # one pair tile, the odd CTA's rows past m
+    ("store", 64, 256, 128),      # one pair tile, the odd CTA's rows all past m
+    ("store", 257, 544, 192),     # ragged M across two pair tiles, ragged N
+    ("residual", 300, 352, 320),  # residual epilogue, ragged N in the odd CTA's half
+    ("swiglu", 5, 128, 64),       # gate rows in the even CTA, up rows in the odd one
+    ("swiglu", 1638, 9216, 2560),
+    ("store", 1638, 12352, 2560),
+])
+def test_cta_pair_form_is_bit_identical_to_single_cta_form(sr, epi, m, n, k):
+    """Both forms run the same K blocks in the same order into fp32 tensor
+    memory, so every output element must come out bit-identical; the pair
+    form is also checked against fp64 like the default path above."""
+    a = W.normal(6, "a", (m, k)).cuda()
+    b0 = W.normal(6, "b0", (n, k), 0.02).cuda()
+    b1 = W.normal(6, "b1", (n, k), 0.02).cuda() if epi == "swiglu" else None
+    r = W.normal(6, "r", (m, n)).cuda() if epi == "residual" else None
+    e = {"store": sr.EPI_STORE, "residual": sr.EPI_RESIDUAL, "swiglu": sr.EPI_SWIGLU}[epi]
+    out = {}
+    for form in (sr.GEMM_FORM_SINGLE, sr.GEMM_FORM_PAIR):
+        ws = sr.workspace(256)
+        out[form] = sr.test_gemm(a, b0, b1=b1, r=r, epi=e, ws=ws, form=form)
+        assert sr.device_status(ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(out[sr.GEMM_FORM_SINGLE], out[sr.GEMM_FORM_PAIR])
+    A = f64(a)
+    if epi == "swiglu":
+        ref = silu(A @ f64(b0).T) * (A @ f64(b1).T)
+    else:
+        ref = A @ f64(b0).T + (f64(r) if r is not None else 0.0)
+    assert_close(out[sr.GEMM_FORM_PAIR], ref, OUT_TOL_BF16, f"pair form, {epi}")

@@ -16,7 +16,7 @@ sr = pytest.importorskip("gated_deltanet_state_sr_b200")
 
 # Longest single-sequence replay whose split-precision scratch fits the array
 # at hidden 2560, intermediate 9216, 16/32 heads of 128, three layers.
-NOALLOC_SPLIT_MAX_TOKENS = 186
+NOALLOC_SPLIT_MAX_TOKENS = 191
 
 
 class DevLayer:
@@ -49,7 +49,7 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
     sr_group_replay, so its results must be bit-identical, on the first call
     and on a second call that finds the first call's leftovers in the array.
     The capacity case is the longest split-precision replay the array holds
-    (one sequence of 186 tokens at hidden 2560), whose scratch ends within
+    (one sequence of 191 tokens at hidden 2560), whose scratch ends within
     1 MB of the array's end."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -118,18 +118,18 @@ def _host_args(T, precision=None):
 def test_noalloc_rejects_replays_too_large_for_the_array():
     """A replay whose scratch would exceed the built-in array is refused before
     any GPU work (no device needed for this check)."""
-    a = _host_args(4096)  # ~170 KB per token: far beyond 32 MiB
+    a = _host_args(4096)  # ~169 KB per token: far beyond 32 MiB
     assert sr.group_workspace_bytes(a) > sr.NOALLOC_SCRATCH_BYTES
     assert sr.group_noalloc_call(a) == sr.SR_ERR_WORKSPACE
     assert "built-in array" in sr.last_error()
 
 
 def test_noalloc_capacity_edge():
-    """The stated capacity at hidden 2560: 186 tokens fit in split precision,
-    187 do not and are refused before any GPU work; with the fp8 low pass
-    191 fit and 192 do not, in bf16 235 and 236."""
-    for prec, fits in ((sr.SR_PREC_SPLIT, NOALLOC_SPLIT_MAX_TOKENS), (sr.SR_PREC_SPLIT_FP8, 191),
-                       (sr.SR_PREC_BF16, 235)):
+    """The stated capacity at hidden 2560: 191 tokens fit in split precision,
+    192 do not and are refused before any GPU work; with the fp8 low pass
+    197 fit and 198 do not, in bf16 241 and 242."""
+    for prec, fits in ((sr.SR_PREC_SPLIT, NOALLOC_SPLIT_MAX_TOKENS), (sr.SR_PREC_SPLIT_FP8, 197),
+                       (sr.SR_PREC_BF16, 241)):
         assert sr.group_workspace_bytes(_host_args(fits, prec)) <= sr.NOALLOC_SCRATCH_BYTES
         too_big = _host_args(fits + 1, prec)
         assert sr.group_workspace_bytes(too_big) > sr.NOALLOC_SCRATCH_BYTES
