@@ -37,11 +37,15 @@ namespace {
 constexpr int BM = 128, BK = 64;
 constexpr int kTileA = BM * BK * 2;  // 16 KB
 constexpr int kThreads = 192;
+// Staging of the epilogue's outputs, per epilogue warp (its 32 rows x 32 columns
+// per step): fp32 4 KB at 0, bf16 hi 2 KB at 4 KB, low part (<= 2 KB) at 6 KB.
+constexpr int kStageWarpBytes = 8192;
+constexpr int kEpiStageBytes = 4 * kStageWarpBytes;
 // Tile width BN fixes the stage count (the launcher uses 256).
 template <int BN> struct Cfg {
     static constexpr int STAGES = BN == 256 ? 4 : 6;
     static constexpr int kTileB = BN * BK * 2;
-    static constexpr int kSmemBytes = STAGES * (kTileA + kTileB) + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int kSmemBytes = STAGES * (kTileA + kTileB) + kEpiStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 };
 
 struct Problem {
@@ -51,6 +55,10 @@ struct Problem {
     CUtensorMap b1;  // up [N, K] box {64, 128} (SwiGLU only)
     CUtensorMap b0_lo;  // fp8 low pass: e5m2 bytes of b0 * 2^-8, box {128 B, as b0}
     CUtensorMap b1_lo;  // fp8 low pass: e5m2 bytes of b1 * 2^-8 (SwiGLU only)
+    // outputs of the staged epilogue, written by TMA stores of 32 x 32 boxes:
+    CUtensorMap o_f32;  // fp32 C (EPI_F32_*), 128-byte swizzle; also the residual's loads
+    CUtensorMap o_hi;   // bf16 hi part: SwiGLU C, or the next norm's n_hi; 64-byte swizzle
+    CUtensorMap o_lo;   // its low part: e4m3 bytes (32-byte swizzle) or bf16 (64-byte swizzle)
     void *c;
     const __nv_bfloat16 *r;
     void *c_lo;              // SwiGLU: low part of the output (bf16, or e4m3 of lo * 2^8; may be null)
@@ -121,161 +129,218 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t phase, vol
     }
 }
 
-// Epilogue of one output tile for the calling thread's row: reads `width`
-// accumulator columns from tensor memory at tbase (SwiGLU: the gate products
-// in the first half, the up products in the second) whose outputs go to
-// columns col0.. of the row, and writes the epilogue's outputs (see the file
-// comment).  With the next norm's operand, the row's sum of squares over those
-// columns goes to partial-sum slot ssq_slot.
-__device__ __forceinline__ void epilogue_row(const Params &p, const Problem &pr, uint32_t tbase, int row, int width,
-                                             int col0, int ssq_slot) {
-    const bool row_ok = row < p.M;
-    float rs = 1.f;
-    if (row_ok && pr.ssq_in) {
-        // RMSNorm factor from the producer's per-tile sums of squares, added in order
+// Byte offset of 16-byte chunk v of row r in a staging box whose rows are 128,
+// 64 or 32 bytes, under the TMA swizzle of that row size (the chunk index XOR
+// address bits 7.. of the row start; boxes start 1024-byte aligned).
+__device__ __forceinline__ uint32_t sw128(int r, int v) { return uint32_t(r * 128 + ((v ^ (r & 7)) << 4)); }
+__device__ __forceinline__ uint32_t sw64(int r, int v) { return uint32_t(r * 64 + ((v ^ ((r >> 1) & 3)) << 4)); }
+__device__ __forceinline__ uint32_t sw32(int r, int v) { return uint32_t(r * 32 + ((v ^ ((r >> 2) & 1)) << 4)); }
+
+// RMSNorm row factor of the calling thread's row: from the producer's per-tile
+// sums of squares (added in order), or given, or 1.
+__device__ __forceinline__ float row_scale(const Params &p, const Problem &pr, int row) {
+    if (row >= p.M) return 1.f;
+    if (pr.ssq_in) {
         float ss = 0.f;
         for (int t = 0; t < p.ssq_parts; ++t)
             if (SR_IN_BOUNDS(size_t(t) * p.M + row, (long long)p.ssq_parts * p.M, p.status))
                 ss += pr.ssq_in[size_t(t) * p.M + row];
-        rs = 1.f / sqrtf(ss / float(p.K) + p.eps);
-    } else if (row_ok && pr.rowscale) {
-        rs = pr.rowscale[row];
+        return 1.f / sqrtf(ss / float(p.K) + p.eps);
     }
+    return pr.rowscale ? pr.rowscale[row] : 1.f;
+}
+
+// x (8 values) -> bf16 hi in `hi` and the low part as bf16 in `lo` and as e4m3
+// bytes of lo * 2^8 in `lo8`.
+__device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo, uint2 &lo8) {
+    uint32_t w[4], wl[4];
+    float l[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        w[e] = pack2(x[2 * e], x[2 * e + 1]);
+        l[2 * e] = x[2 * e] - bf_lo(w[e]);
+        l[2 * e + 1] = x[2 * e + 1] - bf_hi(w[e]);
+        wl[e] = pack2(l[2 * e], l[2 * e + 1]);
+    }
+    hi = make_uint4(w[0], w[1], w[2], w[3]);
+    lo = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+    lo8 = lo8_pack8(l);
+}
+
+// Staged epilogue of one output tile for one warp's 32 rows (row0 + lane): per
+// 32 accumulator columns, the warp writes its outputs into its staging boxes in
+// shared memory and one lane stores each box with a TMA store (coalesced, and
+// clipped at the tensor's bounds); the residual of EPI_F32_RESIDUAL comes in by
+// a TMA load of the same box.  `width` accumulator columns at tbase (SwiGLU:
+// gate products in the first half, up products in the second) produce output
+// columns col0..; with the next norm's operand, the row's sum of squares over
+// those columns goes to partial-sum slot ssq_slot.  Returns false if the
+// residual's load timed out.
+__device__ __forceinline__ bool epilogue_staged(const Params &p, const Problem &pr, uint32_t tbase, int row0,
+                                                int lane, int width, int col0, int ssq_slot, uint8_t *stg,
+                                                uint64_t *rbar, uint32_t &rphase) {
+    // a warp whose 32 rows all lie past M has nothing to write (and issues no
+    // store that would start outside the tensor)
+    if (row0 >= p.M) return true;
+    const int row = row0 + lane;
+    const float rs = row_scale(p, pr, row);
+    uint8_t *sf = stg, *sh = stg + 4096, *sl = stg + 6144;
+    const bool f8 = p.lo_fp8 != 0;
+    bool ok = true;
     if (p.epi == EPI_SWIGLU) {
+        const bool has_lo = pr.c_lo != nullptr;
 #pragma unroll 1
-        for (int c = 0; c < width / 2; c += 32) {
+        for (int c = 0; c < width / 2 && col0 + c < p.N; c += 32) {
             uint32_t g[32], u[32];
             tc::tmem_ld_32x32b_x32(tbase + c, g);
             tc::tmem_ld_32x32b_x32(tbase + width / 2 + c, u);
+            if (lane == 0) tc::bulk_wait_read();  // the previous boxes have left shared memory
+            __syncwarp();
             tc::tmem_ld_wait();
-            const int col = col0 + c;
-            int nvec = min(4, (p.N - col) / 8);  // 8-column groups in range
-            if (row_ok && nvec > 0 &&
-                !SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
-                nvec = 0;
-            if (row_ok && nvec > 0) {
-                __nv_bfloat16 *cb = static_cast<__nv_bfloat16 *>(pr.c);
-                uint4 *dst = reinterpret_cast<uint4 *>(cb + size_t(row) * p.ldc + col);
-                uint4 *dlo = pr.c_lo && !p.lo_fp8
-                                 ? reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c_lo) +
-                                                             size_t(row) * p.ldc + col)
-                                 : nullptr;
-                uint2 *dlo8 = pr.c_lo && p.lo_fp8
-                                  ? reinterpret_cast<uint2 *>(static_cast<uint8_t *>(pr.c_lo) +
-                                                              size_t(row) * p.ldc + col)
-                                  : nullptr;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (v >= nvec) break;
-                    uint32_t w[4], wl[4];
-                    float lo[8];
+            for (int v = 0; v < 4; ++v) {
+                float h[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = v * 8 + e * 2;
-                        const float h0 = silu(rs * __uint_as_float(g[j])) * (rs * __uint_as_float(u[j]));
-                        const float h1 = silu(rs * __uint_as_float(g[j + 1])) * (rs * __uint_as_float(u[j + 1]));
-                        w[e] = pack2(h0, h1);
-                        lo[2 * e] = h0 - bf_lo(w[e]);
-                        lo[2 * e + 1] = h1 - bf_hi(w[e]);
-                        wl[e] = pack2(lo[2 * e], lo[2 * e + 1]);
-                    }
-                    dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                    if (dlo) dlo[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                    if (dlo8) dlo8[v] = lo8_pack8(lo);
-                }
+                for (int e = 0; e < 8; ++e)
+                    h[e] = silu(rs * __uint_as_float(g[8 * v + e])) * (rs * __uint_as_float(u[8 * v + e]));
+                uint4 hi, lo;
+                uint2 lo8;
+                split8(h, hi, lo, lo8);
+                *reinterpret_cast<uint4 *>(sh + sw64(lane, v)) = hi;
+                if (has_lo && !f8) *reinterpret_cast<uint4 *>(sl + sw64(lane, v)) = lo;
+                if (has_lo && f8) *reinterpret_cast<uint2 *>(sl + sw32(lane, v >> 1) + 8 * (v & 1)) = lo8;
+            }
+            tc::fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tc::tma_store_2d(&pr.o_hi, sh, col0 + c, row0);
+                if (has_lo) tc::tma_store_2d(&pr.o_lo, sl, col0 + c, row0);
+                tc::bulk_commit();
             }
         }
     } else {
-        // the next RMSNorm's operand (EPI_F32_RESIDUAL with nw): x * nw and sum x^2
-        const bool norm_out = p.epi == EPI_F32_RESIDUAL && pr.nw != nullptr;
+        const bool resid = p.epi == EPI_F32_RESIDUAL;
+        const bool norm_out = resid && pr.nw != nullptr;
+        const bool has_lo = norm_out && pr.n_lo != nullptr;
         float ssq = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < width; c += 32) {
+        for (int c = 0; c < width && col0 + c < p.N; c += 32) {
+            const int col = col0 + c;
+            if (lane == 0) {
+                tc::bulk_wait_read();  // the previous boxes have left shared memory
+                if (resid) {
+                    tc::mbar_arrive_expect_tx(rbar, 4096);
+                    tc::tma_load_2d(sf, &pr.o_f32, rbar, col, row0);
+                }
+            }
+            __syncwarp();
             uint32_t x[32];
             tc::tmem_ld_32x32b_x32(tbase + c, x);
             tc::tmem_ld_wait();
-            const int col = col0 + c;
-            const int nvec = min(4, (p.N - col) / 8);
-            if (!row_ok || nvec <= 0) continue;
-            if (!SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status))
-                continue;
-            if (p.epi == EPI_F32_ROWSCALE || p.epi == EPI_F32_RESIDUAL) {
-                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(pr.c) + size_t(row) * p.ldc + col);
-                const bool resid = p.epi == EPI_F32_RESIDUAL;
+            float xv[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) xv[e] = rs * __uint_as_float(x[e]);
+            if (resid) {
+                if (!tc::mbar_wait(rbar, rphase)) ok = false;
+                rphase ^= 1;
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
-                    if (v >= 2 * nvec) break;
-                    float4 o = make_float4(rs * __uint_as_float(x[4 * v]), rs * __uint_as_float(x[4 * v + 1]),
-                                           rs * __uint_as_float(x[4 * v + 2]), rs * __uint_as_float(x[4 * v + 3]));
-                    if (resid) {
-                        const float4 rv = dst[v];
-                        o.x += rv.x; o.y += rv.y; o.z += rv.z; o.w += rv.w;
-                    }
-                    dst[v] = o;
-                    x[4 * v] = __float_as_uint(o.x);
-                    x[4 * v + 1] = __float_as_uint(o.y);
-                    x[4 * v + 2] = __float_as_uint(o.z);
-                    x[4 * v + 3] = __float_as_uint(o.w);
+                    const float4 r = *reinterpret_cast<const float4 *>(sf + sw128(lane, v));
+                    xv[4 * v] += r.x;
+                    xv[4 * v + 1] += r.y;
+                    xv[4 * v + 2] += r.z;
+                    xv[4 * v + 3] += r.w;
                 }
-                if (norm_out &&
-                    SR_IN_BOUNDS(size_t(row) * p.N + col + 8 * nvec - 1, (long long)p.M * p.N, p.status)) {
-                    uint4 *dhi = reinterpret_cast<uint4 *>(pr.n_hi + size_t(row) * p.N + col);
-                    const uint4 *wv = reinterpret_cast<const uint4 *>(pr.nw + col);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (v >= nvec) break;
-                        const uint4 wq = wv[v];
-                        const uint32_t ww[4] = {wq.x, wq.y, wq.z, wq.w};
-                        uint32_t w[4], wl[4];
-                        float lo[8];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = v * 8 + e * 2;
-                            const float x0 = __uint_as_float(x[j]), x1 = __uint_as_float(x[j + 1]);
-                            ssq = fmaf(x0, x0, ssq);
-                            ssq = fmaf(x1, x1, ssq);
-                            const float h0 = x0 * bf_lo(ww[e]), h1 = x1 * bf_hi(ww[e]);
-                            w[e] = pack2(h0, h1);
-                            lo[2 * e] = h0 - bf_lo(w[e]);
-                            lo[2 * e + 1] = h1 - bf_hi(w[e]);
-                            wl[e] = pack2(lo[2 * e], lo[2 * e + 1]);
-                        }
-                        dhi[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                        if (pr.n_lo && p.lo_fp8)
-                            reinterpret_cast<uint2 *>(static_cast<uint8_t *>(pr.n_lo) + size_t(row) * p.N + col)[v] =
-                                lo8_pack8(lo);
-                        else if (pr.n_lo)
-                            reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.n_lo) + size_t(row) * p.N +
-                                                      col)[v] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                    }
-                }
-                continue;
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c) + size_t(row) * p.ldc + col);
-            const uint4 *res = p.epi == EPI_RESIDUAL
-                                   ? reinterpret_cast<const uint4 *>(pr.r + size_t(row) * p.ldc + col)
-                                   : nullptr;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                if (v >= nvec) break;
-                uint32_t rr[4] = {0u, 0u, 0u, 0u};
-                if (res) {
-                    const uint4 rv = res[v];
-                    rr[0] = rv.x; rr[1] = rv.y; rr[2] = rv.z; rr[3] = rv.w;
-                }
-                uint32_t w[4];
+            for (int v = 0; v < 8; ++v)
+                *reinterpret_cast<float4 *>(sf + sw128(lane, v)) =
+                    make_float4(xv[4 * v], xv[4 * v + 1], xv[4 * v + 2], xv[4 * v + 3]);
+            if (norm_out) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = v * 8 + e * 2;
-                    w[e] = pack2(bf_lo(rr[e]) + rs * __uint_as_float(x[j]),
-                                 bf_hi(rr[e]) + rs * __uint_as_float(x[j + 1]));
+                for (int v = 0; v < 4; ++v) {
+                    // norm weights of columns past N read as zero (N is a multiple of 8)
+                    const uint4 wq = col + 8 * v < p.N ? reinterpret_cast<const uint4 *>(pr.nw + col)[v]
+                                                       : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t ww[4] = {wq.x, wq.y, wq.z, wq.w};
+                    float h[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = xv[8 * v + 2 * e], x1 = xv[8 * v + 2 * e + 1];
+                        ssq = fmaf(x0, x0, ssq);
+                        ssq = fmaf(x1, x1, ssq);
+                        h[2 * e] = x0 * bf_lo(ww[e]);
+                        h[2 * e + 1] = x1 * bf_hi(ww[e]);
+                    }
+                    uint4 hi, lo;
+                    uint2 lo8;
+                    split8(h, hi, lo, lo8);
+                    *reinterpret_cast<uint4 *>(sh + sw64(lane, v)) = hi;
+                    if (has_lo && !f8) *reinterpret_cast<uint4 *>(sl + sw64(lane, v)) = lo;
+                    if (has_lo && f8) *reinterpret_cast<uint2 *>(sl + sw32(lane, v >> 1) + 8 * (v & 1)) = lo8;
                 }
-                dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            tc::fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tc::tma_store_2d(&pr.o_f32, sf, col, row0);
+                if (norm_out) tc::tma_store_2d(&pr.o_hi, sh, col, row0);
+                if (has_lo) tc::tma_store_2d(&pr.o_lo, sl, col, row0);
+                tc::bulk_commit();
             }
         }
         const size_t si = size_t(ssq_slot) * p.M + row;
-        if (norm_out && row_ok && SR_IN_BOUNDS(si, (long long)p.ssq_slots * p.M, p.status)) pr.ssq_out[si] = ssq;
+        if (norm_out && row < p.M && SR_IN_BOUNDS(si, (long long)p.ssq_slots * p.M, p.status)) pr.ssq_out[si] = ssq;
     }
+    return ok;
+}
+
+// Per-thread epilogue of the bf16 test epilogues (EPI_STORE, EPI_RESIDUAL): the
+// calling thread's row, `width` accumulator columns at tbase, output columns col0..
+__device__ __forceinline__ void epilogue_row_bf16(const Params &p, const Problem &pr, uint32_t tbase, int row,
+                                                  int width, int col0) {
+    const bool row_ok = row < p.M;
+    const float rs = row_scale(p, pr, row);
+#pragma unroll 1
+    for (int c = 0; c < width; c += 32) {
+        uint32_t x[32];
+        tc::tmem_ld_32x32b_x32(tbase + c, x);
+        tc::tmem_ld_wait();
+        const int col = col0 + c;
+        const int nvec = min(4, (p.N - col) / 8);
+        if (!row_ok || nvec <= 0) continue;
+        if (!SR_IN_BOUNDS(size_t(row) * p.ldc + col + 8 * nvec - 1, (long long)p.M * p.ldc, p.status)) continue;
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(pr.c) + size_t(row) * p.ldc + col);
+        const uint4 *res =
+            p.epi == EPI_RESIDUAL ? reinterpret_cast<const uint4 *>(pr.r + size_t(row) * p.ldc + col) : nullptr;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            if (v >= nvec) break;
+            uint32_t rr[4] = {0u, 0u, 0u, 0u};
+            if (res) {
+                const uint4 rv = res[v];
+                rr[0] = rv.x; rr[1] = rv.y; rr[2] = rv.z; rr[3] = rv.w;
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = v * 8 + e * 2;
+                w[e] = pack2(bf_lo(rr[e]) + rs * __uint_as_float(x[j]), bf_hi(rr[e]) + rs * __uint_as_float(x[j + 1]));
+            }
+            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+// Epilogue of one output tile for one epilogue warp (rows row0 .. row0 + 31).
+__device__ __forceinline__ bool epilogue_warp(const Params &p, const Problem &pr, uint32_t tbase, int row0, int lane,
+                                              int width, int col0, int ssq_slot, uint8_t *stg, uint64_t *rbar,
+                                              uint32_t &rphase) {
+    if (p.epi == EPI_STORE || p.epi == EPI_RESIDUAL) {
+        epilogue_row_bf16(p, pr, tbase, row0 + lane, width, col0);
+        return true;
+    }
+    return epilogue_staged(p, pr, tbase, row0, lane, width, col0, ssq_slot, stg, rbar, rphase);
 }
 
 template <int BN>
@@ -286,12 +351,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * kTileA;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + STAGES * kTileB);
+    uint8_t *stage_out = sB + STAGES * kTileB;  // the epilogue warps' staging boxes (1024-aligned)
+    uint64_t *full = reinterpret_cast<uint64_t *>(stage_out + kEpiStageBytes);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *rbar = drain + 1;  // [4] residual loads of the epilogue warps
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(rbar + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -305,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             tc::mbar_init(&tempty[b], 4);
         }
         tc::mbar_init(drain, 1);
+        for (int w = 0; w < 4; ++w) tc::mbar_init(&rbar[w], 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -413,6 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
     } else {
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        uint8_t *stg = stage_out + (warp - 2) * kStageWarpBytes;
+        uint64_t *rb = &rbar[warp - 2];
+        uint32_t rphase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
@@ -421,13 +492,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const Problem &pr = p.prob[pi];
             if (!wait_or_abort(&tfull[acc], acc_phase, abort_flag)) { fail(); break; }
             tc::tc_fence_after();
-            epilogue_row(p, pr, tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN), mt * BM + quad * 32 + lane, BN,
-                         p.epi == EPI_SWIGLU ? nt * (BN / 2) : nt * BN, nt);
+            const bool ok = epilogue_warp(p, pr, tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN),
+                                          mt * BM + quad * 32, lane, BN, p.epi == EPI_SWIGLU ? nt * (BN / 2) : nt * BN,
+                                          nt, stg, rb, rphase);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            if (!ok) { fail(); break; }
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (lane == 0) tc::bulk_wait_all();  // the output boxes are written before the CTA leaves
     }
 
     if (*abort_flag) {
@@ -455,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // buffers.  The arithmetic of every output element (the K blocks in order,
 // fp32 accumulation in tensor memory) is that of the single-CTA form.
 constexpr int kPairStages = 6;
-constexpr int kPairSmemBytes = kPairStages * 2 * kTileA + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kPairSmemBytes = kPairStages * 2 * kTileA + kEpiStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 __device__ __forceinline__ bool wait_or_abort_cluster(uint64_t *bar, uint32_t phase, volatile int *abort_flag) {
     if (tc::mbar_try_wait_cluster(bar, phase)) return true;
@@ -473,12 +547,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * kTileA;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + STAGES * kTileB);  // used in the even CTA
+    uint8_t *stage_out = sB + STAGES * kTileB;  // the epilogue warps' staging boxes (1024-aligned)
+    uint64_t *full = reinterpret_cast<uint64_t *>(stage_out + kEpiStageBytes);  // used in the even CTA
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;  // used in the even CTA: 4 epilogue warps of each CTA arrive
     uint64_t *drain = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *rbar = drain + 1;  // [4] residual loads of the epilogue warps
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(rbar + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -494,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
             tc::mbar_init(&tempty[b], 8);
         }
         tc::mbar_init(drain, 1);
+        for (int w = 0; w < 4; ++w) tc::mbar_init(&rbar[w], 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -601,6 +678,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     } else {
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
         const uint32_t tempty0 = tc::mapa_shared(tc::smem_u32(tempty), 0);
+        uint8_t *stg = stage_out + (warp - 2) * kStageWarpBytes;
+        uint64_t *rb = &rbar[warp - 2];
+        uint32_t rphase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = pair; tile < total && !*abort_flag; tile += n_pairs) {
@@ -609,14 +689,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
             const Problem &pr = p.prob[pi];
             if (!wait_or_abort(&tfull[acc], acc_phase, abort_flag)) { fail(); break; }
             tc::tc_fence_after();
-            epilogue_row(p, pr, tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN),
-                         mt * 2 * BM + int(rank) * BM + quad * 32 + lane, BN,
-                         p.epi == EPI_SWIGLU ? nt * (BN / 2) : nt * BN, nt);
+            const bool ok = epilogue_warp(p, pr, tmem + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN),
+                                          mt * 2 * BM + int(rank) * BM + quad * 32, lane, BN,
+                                          p.epi == EPI_SWIGLU ? nt * (BN / 2) : nt * BN, nt, stg, rb, rphase);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+            if (!ok) { fail(); break; }
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (lane == 0) tc::bulk_wait_all();  // the output boxes are written before the CTA leaves
     }
 
     if (*abort_flag) {
@@ -705,6 +787,22 @@ namespace {
 bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int pitch, int box_rows) {
     return make_map_bf16(m, base, rows, cols, pitch, 64, box_rows);
 }
+// Map of an epilogue output [rows, cols] (row pitch `pitch` elements of `esize`
+// bytes) in 32 x 32 boxes with the swizzle of the box's row size.
+bool make_map_out(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, int rows, int cols,
+                  int pitch) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(pitch) * esize};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t es[2] = {1u, 1u};
+    const CUtensorMapSwizzle sw = esize == 4   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : esize == 2 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_32B;
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 }  // namespace
 
 namespace {
@@ -729,6 +827,24 @@ cudaError_t fill_params(Params &local, const GemmProblemDesc *probs, int n_probl
             if (epi == EPI_SWIGLU && (!d.b1_lo || !make_map_u8(&local.prob[i].b1_lo, d.b1_lo, N, K, K, 2 * BK, b_rows)))
                 return cudaErrorInvalidValue;
         }
+        // outputs of the staged epilogue
+        const bool lo8 = n_pass == 2 && lo_fp8;
+        bool ok_out = true;
+        if (epi == EPI_F32_ROWSCALE || epi == EPI_F32_RESIDUAL)
+            ok_out = make_map_out(&local.prob[i].o_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d.c, M, N, ldc);
+        if (ok_out && epi == EPI_F32_RESIDUAL && d.nw) {
+            ok_out = make_map_out(&local.prob[i].o_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.n_hi, M, N, N);
+            if (ok_out && d.n_lo)
+                ok_out = lo8 ? make_map_out(&local.prob[i].o_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d.n_lo, M, N, N)
+                                : make_map_out(&local.prob[i].o_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.n_lo, M, N, N);
+        }
+        if (ok_out && epi == EPI_SWIGLU) {
+            ok_out = make_map_out(&local.prob[i].o_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.c, M, N, ldc);
+            if (ok_out && d.c_lo)
+                ok_out = lo8 ? make_map_out(&local.prob[i].o_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d.c_lo, M, N, ldc)
+                                : make_map_out(&local.prob[i].o_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.c_lo, M, N, ldc);
+        }
+        if (!ok_out) return cudaErrorInvalidValue;
         local.prob[i].c = d.c;
         local.prob[i].r = static_cast<const __nv_bfloat16 *>(d.r);
         local.prob[i].c_lo = d.c_lo;
