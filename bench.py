@@ -49,9 +49,9 @@ L2_BYTES = 126 * 1024 * 1024
 # the kernel source it was taken on; once that file changes the figure no
 # longer describes the kernel and the bench reports null.
 MEASURED_TRAFFIC = {
-    # gate/up (single-CTA tiles) of the 1-group workload with the fp8 low pass: 155.4 MB read +
-    # 28.1 MB written, x 8 groups
-    "model_32k_5": ("gemm_tc.cu", "03b6ae2b55b1cbf3", 8 * 183.5e6),
+    # gate/up (single-CTA tiles) of the 1-group workload with the fp8 low pass: 155.8 MB read +
+    # 30.0 MB written, x 8 groups
+    "model_32k_5": ("gemm_tc.cu", "1f99993d9cfa0691", 8 * 185.8e6),
     # the raw workload's call, both kernels of the two-phase form: prep 76.3 MB read +
     # 208.0 MB written, sequential 379.2 MB read + 64.4 MB written
     "raw_qwen": ("gdn_tc.cu", "8dae5304f374db1e", 727.9e6),
@@ -149,9 +149,15 @@ class RawGdn:
 
     def __init__(self, name, rank):
         self.name = name
-        if name == "raw_qwen":
+        self.f32 = name == "raw_qwen_f32"
+        if name in ("raw_qwen", "raw_qwen_f32"):
             self.x = W.raw_qwen(seed=0x5EED0001 + rank)
             self.desc = "one GDN layer, 8 suffixes ~U{512..2048} tok, H_k=16 H_v=32 d=128"
+            if self.f32:
+                # the fp32-input mode: the same values carried as fp32 q, k, v (and o)
+                x = self.x
+                x.q, x.k, x.v = x.q.float(), x.k.float(), x.v.float()
+                self.desc += ", fp32 q/k/v/o (the fp32-input mode)"
         elif name == "raw_small":
             self.x = W.raw_small(seed=0x5EED0000 + rank)
             self.desc = "one GDN layer, 1 suffix of 256 tok, H_k=2 H_v=4 d=64"
@@ -164,8 +170,14 @@ class RawGdn:
         self.hv, self.d, self.hk = hv, d, hk
         # algorithmic work (chunk-64 convention) and bytes per replayed token
         C = 64
-        self.flop_per_tok = hv * 2 * (C * (3 * d + 2 * d) + 3 * d * d)
-        self.bytes_per_tok = hk * 2 * d * 2 + hv * (2 * d * 2 + 8)
+        if self.f32:
+            # the token recurrence's multiply-adds per token and V head: S k, the
+            # rank-one update and S q, 3 d_k d_v FMAs = 6 d_k d_v flops
+            self.flop_per_tok = hv * 6 * d * d
+        else:
+            self.flop_per_tok = hv * 2 * (C * (3 * d + 2 * d) + 3 * d * d)
+        esz = 4 if self.f32 else 2
+        self.bytes_per_tok = hk * 2 * d * esz + hv * (2 * d * esz + 8)
         self.state_bytes = x.n_seqs * hv * d * d * 4
         self.input_bytes = sum(t.numel() * t.element_size() for t in (x.q, x.k, x.v, x.g, x.beta))
 
@@ -208,8 +220,9 @@ class RawGdn:
 
     @property
     def launches_per_step(self):
-        # the two-phase tcgen05 pair: the chunk-parallel prep, then the state chain
-        return 2
+        # the two-phase tcgen05 pair: the chunk-parallel prep, then the state chain;
+        # the fp32-input mode: one token-by-token launch
+        return 1 if self.f32 else 2
 
     def step_e2e(self):
         for h, d in zip(self.h_in, self.d_in):
@@ -227,6 +240,10 @@ class RawGdn:
         return self.h_o.numel() * self.h_o.element_size() + self.h_s.numel() * 4
 
     def dominant(self):
+        if self.f32:
+            # fp32 inputs run the token-by-token recurrence on the fp32 FMA units
+            return {"name": "gdn_token_kernel", "bound": "alu", "flop": self.flop_per_tok * self.tokens,
+                    "bytes": self.bytes_per_tok * self.tokens + self.state_bytes}
         # the default algorithm: the two tcgen05 kernels of one replay (the chunk-parallel
         # prep, then the per-sequence state chain), timed as the pair; at d = 64 they run
         # on 128-wide tiles whose upper halves stay zero
@@ -563,10 +580,12 @@ class Mamba2Replay:
                                       f"token-by-token recurrence; tokens = head-tokens / H")
 
 
-WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "group": GroupReplay, "mamba2": Mamba2Replay,
+WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "raw_qwen_f32": RawGdn, "group": GroupReplay,
+             "mamba2": Mamba2Replay,
              "sparse_32k": GroupReplay,
              **{f"model_{m}_{r}": GroupReplay for m in ("8k", "16k", "32k") for r in ("5", "10")}}
 DEFAULT_WORKLOAD = "model_32k_5"
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 74.4
 
 
 # ------------------------------------------------------------------ arms
@@ -779,7 +798,15 @@ def run_ours(args):
         kern_ms = ms_per_step  # the dominant kernel is the whole step for the raw workloads
         tflops = dom["flop"] / (kern_ms / 1e3) / 1e12
         hbm_gbs = dom["bytes"] / (kern_ms / 1e3) / 1e9
-        if dom["bound"] == "hbm":
+        if dom["bound"] == "alu":
+            # fp32 FMA peak from the unit counts: 148 SMs x 128 fp32 lanes x 2 flop x the
+            # maximum SM clock (1965 MHz) = 74.4 TFLOP/s
+            peak = FP32_FMA_TFLOPS
+            roofline = {"kernel": dom["name"], "bound": "alu", "achieved": round(tflops, 2), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": measured_traffic(args.workload),
+                        "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 flop x 1965 MHz",
+                        "hbm_gbs": round(hbm_gbs, 1), "hbm_frac": round(hbm_gbs / peaks["hbm_gbs"], 4)}
+        elif dom["bound"] == "hbm":
             roofline = {"kernel": dom["name"], "bound": "hbm", "achieved": round(hbm_gbs, 1),
                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(hbm_gbs / peaks["hbm_gbs"], 4),
                         "traffic": measured_traffic(args.workload), "peak_source": f"{src} (HBM copy)",
@@ -801,10 +828,11 @@ def run_ours(args):
     line = {
         "metric": "replayed tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if getattr(wl, "f32", False) else "bf16",
         "data": "synthetic (seeded, workloads.py)",
         "config": workload_config(args, wl, world),
-        "precision": getattr(wl, "precision", "bf16 inputs"),
+        "precision": getattr(wl, "precision", "fp32 inputs" if getattr(wl, "f32", False) else "bf16 inputs"),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "serial_value": e2e_serial,
                 "copies": "overlapped with the replay (two buffer sets, copy streams)" if hasattr(wl, "e2e_inputs")
                 else "serialised with the replay", "h2d_bytes_per_step": wl.h2d_bytes,

@@ -105,6 +105,20 @@ def test_fp32_input_mode(sr):
     assert_close(o, o_ref, TOL_FP32, "o (fp32 mode)")
 
 
+def test_fp32_input_mode_full_size(sr):
+    """The fp32-input mode at the 8-suffix workload's full size (the same values
+    as fp32 q, k, v; 16/32 heads, d = 128): states and outputs within the fp32
+    tolerance, every sequence on its own."""
+    x = W.raw_qwen()
+    x.q, x.k, x.v = x.q.float(), x.k.float(), x.v.float()
+    o, s = run_gpu(sr, x, "auto")
+    assert o.dtype == torch.float32
+    o_ref, s_ref = run_oracle(x)
+    assert_close(o, o_ref, TOL_FP32, "o (fp32 mode)")
+    for n in range(x.n_seqs):
+        assert_close(s[n], s_ref[n], TOL_FP32, f"state seq {n} (fp32 mode)")
+
+
 @pytest.mark.parametrize("algo", ALGOS)
 def test_bad_cu_seqlens_flagged_on_device(sr, algo):
     """A decreasing cu_seqlens entry is caught by the kernel's own bounds check:
