@@ -83,16 +83,17 @@ constexpr uint32_t IMG_T2L = 49152;  // T diag(beta), lo
 constexpr uint32_t IMG_GATE = 57344; // fp32 e^{gamma_C - gamma_t} for t < 64, then e^{gamma_C} (512 B)
 constexpr uint32_t kImg = 57856;
 
-// prep kernel: K/Q (and Kl, right after them: the prep kernel reads no V) tiles,
-// then A and T fp32.  P and T2 hi reuse the Q tiles once the first product has
+// prep kernel: K/Q tiles at 0 (32 KB), then two fp32 64 x 64 slots (A and T),
+// then the gates.  P and T2 hi reuse the Q tiles once the first product has
 // read them, T1 and T2 lo the A matrix after the solve, -W^T the T matrix once
-// T1 and T2 are formed.  Kl stays in place until W^T has been formed.
+// T1 and T2 are formed.  With split k the low part of K arrives at 32 KB and the
+// first product reads it there; T then takes that slot (A the next), and the
+// low part is loaded again for W^T once T1 and T2 are formed.  Both forms take
+// 69 KB, three CTAs per SM.
 constexpr uint32_t OFF_KL_PREP = 32768;
-constexpr uint32_t kPrepIn[2] = {32768, 49152};
-constexpr uint32_t smem_prep(bool split) { return kPrepIn[split] + 2 * SZ_AT + SZ_MISC + 1024; }
+constexpr uint32_t smem_prep() { return 32768 + 2 * SZ_AT + SZ_MISC + 1024; }
 
-
-static_assert(2 * (smem_prep(true) + 1024) <= 233472, "two prep CTAs must fit one SM");
+static_assert(3 * (smem_prep() + 1024) <= 233472, "three prep CTAs must fit one SM");
 
 // Chunk c of the sequence n starting at token bos has the image slot
 // floor(bos / C) + n + c: distinct chunks get distinct slots, all below
@@ -974,16 +975,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_tc_kernel(const __grid_consta
 // One CTA per (chunk slot, V head, group).  Slots between two sequences' chunks
 // (at most one per sequence) exit at once.
 template <bool SPLIT, int DH>
-__global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnTcParams p) {
+__global__ void __launch_bounds__(kThreads, 3) gdn_prep_kernel(const __grid_constant__ GdnTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(sm);
-    constexpr uint32_t oXR = kPrepIn[SPLIT], oMISC = oXR + 2 * SZ_AT;
+    // split k: T over the low part of K (read by the first product, loaded again for W)
+    constexpr uint32_t oT = SPLIT ? OFF_KL_PREP : 32768 + SZ_AT, oA = SPLIT ? OFF_KL_PREP + SZ_AT : 32768;
+    constexpr uint32_t oMISC = 32768 + 2 * SZ_AT;
     constexpr uint32_t oP = OFF_KQ + 8192, oT2H = OFF_KQ + 24576;  // the Q tiles
-    constexpr uint32_t oT1 = oXR, oT2L = oXR + 8192;                // A
-    constexpr uint32_t oW = oXR + SZ_AT;                            // T
-    float *Af = reinterpret_cast<float *>(sm + oXR);
-    float *Tf = reinterpret_cast<float *>(sm + oXR + SZ_AT);
+    constexpr uint32_t oT1 = oA, oT2L = oA + 8192;                  // A
+    constexpr uint32_t oW = oT;                                     // T
+    float *Af = reinterpret_cast<float *>(sm + oA);
+    float *Tf = reinterpret_cast<float *>(sm + oT);
     float *gam = reinterpret_cast<float *>(sm + oMISC);  // [64]
     float *bet = gam + C;                                 // [64]
     float *fb = gam + 2 * C;                              // [64] beta_s e^{gamma_s}
@@ -1107,13 +1110,29 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        bool wk = true;
         if (tid == 0) {
             tc_fence_after();
-            mma_w<SPLIT>(base, oT1, R0, OFF_KL_PREP);
-            mma_commit(bar_mma);
+            if (SPLIT) {  // the low part of K again, over the spent T
+                constexpr int d = 64 * DH;
+                mbar_arrive_expect_tx(bar_in, DH * 8192u);
+                tma_load_2d(sm + OFF_KL_PREP, &p.kl[gi], bar_in, hk * d, y);
+                if (DH == 2) tma_load_2d(sm + OFF_KL_PREP + 8192, &p.kl[gi], bar_in, hk * d + 64, y);
+                wk = mbar_wait(bar_in, 1);
+            }
+            if (wk) {
+                mma_w<SPLIT>(base, oT1, R0, OFF_KL_PREP);
+                mma_commit(bar_mma);
+            }
             bulk_store(dst + IMG_T2H, sm + oT2H, 8192);
             bulk_store(dst + IMG_T2L, sm + oT2L, 8192);
         }
+        // a failed wait for the reload skips W's product; every thread learns of it here
+        if (__syncthreads_or(!wk)) {
+            ok = false;
+        }
+    }
+    if (ok) {
         const bool w = mbar_wait(bar_mma, mma_phase);
         mma_phase ^= 1;
         tc_fence_after();
@@ -1521,7 +1540,7 @@ cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t 
         gdn_tc_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kThreads, smem, st>>>(p);
         return cudaGetLastError();
     }
-    const int s1 = int(smem_prep(SPLIT)), s2 = int(smem_seq());
+    const int s1 = int(smem_prep()), s2 = int(smem_seq());
     cudaError_t e =
         cudaFuncSetAttribute(gdn_prep_kernel<SPLIT, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return e;
