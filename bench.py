@@ -51,20 +51,24 @@ L2_BYTES = 126 * 1024 * 1024
 MEASURED_TRAFFIC = {
     # gate/up (single-CTA tiles) of the 1-group workload with the fp8 low pass: 155.8 MB read +
     # 30.0 MB written, x 8 groups
-    "model_32k_5": ("gemm_tc.cu", "1f99993d9cfa0691", 8 * 185.8e6),
-    # the raw workload's call, both kernels of the two-phase form: prep 76.3 MB read +
-    # 208.0 MB written, sequential 379.2 MB read + 64.4 MB written
-    "raw_qwen": ("gdn_tc.cu", "8dae5304f374db1e", 727.9e6),
+    "model_32k_5": ("gemm_tc.cu", "1f99993d9cfa0691", 8 * 185.8e6, "gemm_gateup"),
+    # the raw workload's call, both kernels of the two-phase form: prep 76.4 MB read +
+    # 207.5 MB written, sequential 379.3 MB read + 64.2 MB written
+    "raw_qwen": ("gdn_tc.cu", "27fad40539b0f525", 727.4e6, None),
     # the Mamba2 workload's launch: 1273.9 MB read + 1222.0 MB written
-    "mamba2": ("mamba2_tc.cu", "53e6f86ec1f409d3", 2495.9e6),
+    "mamba2": ("mamba2_tc.cu", "53e6f86ec1f409d3", 2495.9e6, None),
 }
 
 
-def measured_traffic(workload):
+def measured_traffic(workload, kind=None):
+    """The recorded DRAM traffic per launch of the workload's dominant kernel, or
+    None when there is none for this kernel kind or its source has changed."""
     ent = MEASURED_TRAFFIC.get(workload)
     if ent is None:
         return None
-    fn, digest, nbytes = ent
+    fn, digest, nbytes, ent_kind = ent
+    if ent_kind is not None and ent_kind != kind:
+        return None
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "gated_deltanet_state_sr_b200", "csrc", fn)
     try:
         with open(path, "rb") as f:
@@ -784,10 +788,13 @@ def run_ours(args):
         per_launch_ms = kernels[dom_kind]["ms_per_step"] / kernels[dom_kind]["launches_per_step"]
         achieved = wl.flop[dom_kind] / (per_launch_ms / 1e3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roofline = {"kernel": f"gemm_tc_kernel ({dom_kind})" if dom_kind.startswith("gemm") else dom_kind,
+        names = {"gemm_in": "gemm_pair_kernel (in_proj)", "gemm_out": "gemm_pair_kernel (out_proj)",
+                 "gemm_down": "gemm_pair_kernel (down)", "gemm_gateup": "gemm_tc_kernel (gate/up)",
+                 "gdn": "gdn_prep_kernel + gdn_seq_kernel"}
+        roofline = {"kernel": names.get(dom_kind, dom_kind),
                     "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                     "frac": round(achieved / peak, 4),
-                    "traffic": measured_traffic(args.workload) if dom_kind == "gemm_in" else None,
+                    "traffic": measured_traffic(args.workload, dom_kind),
                     "peak_source": f"{src} (sustained bf16: kernel timed inside a long step)",
                     "flop_per_launch": wl.flop[dom_kind], "ms_per_launch": round(per_launch_ms, 4),
                     "mma_passes": {"split": "2 bf16", "split_fp8": "1 bf16 + 1 fp8 (e4m3 x e5m2)",
