@@ -51,7 +51,7 @@ L2_BYTES = 126 * 1024 * 1024
 MEASURED_TRAFFIC = {
     # gate/up (single-CTA tiles) of the 1-group workload with the fp8 low pass: 155.8 MB read +
     # 30.0 MB written, x 8 groups
-    "model_32k_5": ("gemm_tc.cu", "1f99993d9cfa0691", 8 * 185.8e6, "gemm_gateup"),
+    "model_32k_5": ("gemm_tc.cu", "47f52f1e08eba982", 8 * 185.8e6, "gemm_gateup"),
     # the raw workload's call, both kernels of the two-phase form: prep 76.4 MB read +
     # 207.5 MB written, sequential 379.3 MB read + 64.2 MB written
     "raw_qwen": ("gdn_tc.cu", "27fad40539b0f525", 727.4e6, None),

@@ -18,10 +18,14 @@
 // warp 1 allocates TMEM and issues tcgen05.mma (M=128, N=256, K=16) from one
 // thread, warps 2-5 drain the double-buffered TMEM accumulator (2 x 256
 // columns) with tcgen05.ld and apply the epilogue while the next tile's MMAs
-// run.  Tiles walk M fastest so CTAs running together share the weight tile
-// through L2.  Several problems with identical shapes (one per replay group)
-// are scheduled as one launch.  Every mbarrier wait is bounded; on timeout
-// the kernel records SR_DEV_TIMEOUT, drains its MMAs, frees TMEM and exits.
+// run; each epilogue warp stages its outputs 32 x 32 at a time in shared
+// memory and writes them with TMA stores.  Tiles walk M fastest so CTAs
+// running together share the weight tile through L2.  Several problems with
+// identical shapes (one per replay group) are scheduled as one launch.  A
+// second form (gemm_pair_kernel, below) computes 256 x 256 tiles with a
+// cluster of two CTAs and cta_group::2 products.  Every mbarrier wait is
+// bounded; on timeout the kernel records SR_DEV_TIMEOUT, drains its MMAs,
+// frees TMEM and exits.
 #include <cuda.h>
 
 #include "common.cuh"
