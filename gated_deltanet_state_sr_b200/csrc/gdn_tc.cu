@@ -118,6 +118,7 @@ struct GdnTcParams {
     uint8_t *img;  // two-phase: chunk images [group][slot][V head][kImg]
     int total, max_len, h_k, h_v, n_seqs, slots;
     int d;  // head dim d_k = d_v: 128, or 64 (the upper half of every 128-wide tile stays zero)
+    int want_o;  // 0: no group writes o, so the two-phase form neither forms nor moves P and Qg
     float scale;
     uint32_t *status;
 };
@@ -245,7 +246,7 @@ template <bool SPLIT>
 __device__ __forceinline__ void build_a_p(uint8_t *sm, uint32_t p_off, float *Af, uint32_t R0, uint32_t R1,
                                           uint32_t lane_off, int quad, int half, int row, const float *gam,
                                           const float *bet, const float *fb, const float *eg, const float *ei,
-                                          bool fact, float scale) {
+                                          bool fact, float scale, bool want_p = true) {
     uint32_t r[32], r2[32];
     tmem_ld_32x32b_x32(R0 + lane_off + 32 * half, r);
     if (SPLIT && quad < 2) tmem_ld_32x32b_x32(R1 + lane_off + 32 * half, r2);
@@ -266,7 +267,7 @@ __device__ __forceinline__ void build_a_p(uint8_t *sm, uint32_t p_off, float *Af
             }
             *reinterpret_cast<float4 *>(&Af[t * ROWA + 32 * half + e]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
         }
-    } else {
+    } else if (want_p) {
         const int t = row - 64;
         const float gt = gam[t], st = scale * eg[t];
 #pragma unroll
@@ -1028,12 +1029,13 @@ __global__ void __launch_bounds__(kThreads, 3) gdn_prep_kernel(const __grid_cons
         fence_mbar_init();
         const CUtensorMap *mq = &p.q[gi], *mk = &p.k[gi], *mkl = &p.kl[gi];
         constexpr int d = 64 * DH;
-        mbar_arrive_expect_tx(bar_in, DH * (SPLIT ? 24576u : 16384u));
+        // without o, Q is not needed: P and Qg are neither formed nor stored
+        mbar_arrive_expect_tx(bar_in, DH * ((SPLIT ? 24576u : 16384u) - (p.want_o ? 0u : 8192u)));
         tma_load_2d(sm + OFF_KQ, mk, bar_in, hk * d, y);
-        tma_load_2d(sm + OFF_KQ + 8192, mq, bar_in, hk * d, y);
+        if (p.want_o) tma_load_2d(sm + OFF_KQ + 8192, mq, bar_in, hk * d, y);
         if (DH == 2) {
             tma_load_2d(sm + OFF_KQ + 16384, mk, bar_in, hk * d + 64, y);
-            tma_load_2d(sm + OFF_KQ + 24576, mq, bar_in, hk * d + 64, y);
+            if (p.want_o) tma_load_2d(sm + OFF_KQ + 24576, mq, bar_in, hk * d + 64, y);
         }
         if (SPLIT) {
             tma_load_2d(sm + OFF_KL_PREP, mkl, bar_in, hk * d, y);
@@ -1089,20 +1091,21 @@ __global__ void __launch_bounds__(kThreads, 3) gdn_prep_kernel(const __grid_cons
             mma_commit(bar_mma);
         }
         // ---- meanwhile: Qg = scale e^{gamma_t} Q and the decay factors, straight to the image
-        build_qg_image(sm, dst + IMG_QGW, gam, p.scale, tid);
+        if (p.want_o) build_qg_image(sm, dst + IMG_QGW, gam, p.scale, tid);
         if (tid < C) reinterpret_cast<float *>(dst + IMG_GATE)[tid] = __expf(gC - gam[tid]);
         if (tid == 0) reinterpret_cast<float *>(dst + IMG_GATE)[C] = __expf(gC);
         __syncthreads();  // every Q read is done before P overwrites the first Q tile
         const bool w = mbar_wait(bar_mma, mma_phase);
         mma_phase ^= 1;
         tc_fence_after();
-        build_a_p<SPLIT>(sm, oP, Af, R0, R1, lane_off, quad, half, row, gam, bet, fb, eg, ei, fact, p.scale);
+        build_a_p<SPLIT>(sm, oP, Af, R0, R1, lane_off, quad, half, row, gam, bet, fb, eg, ei, fact, p.scale,
+                         p.want_o != 0);
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(w) != 0;
     }
     // each tile of the image leaves as soon as it is formed
-    if (ok && tid == 0) bulk_store(dst + IMG_P, sm + oP, 8192);
+    if (ok && tid == 0 && p.want_o) bulk_store(dst + IMG_P, sm + oP, 8192);
     if (ok) {
         // ---- the solve, T1 and T2, then W^T = K^T T1^T and -W
         t_solve(Af, Tf, tid, warp, lane);
@@ -1412,14 +1415,24 @@ __global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_co
     auto issue_in = [&](int c) {  // V (+ low part) and the chunk image into buffer c & 1
         const int y = bos + c * C, b = c & 1;
         uint64_t *bar = &bar_in[b];
-        mbar_arrive_expect_tx(bar, DH * (SPLIT ? 16384u : 8192u) + kImg);
+        mbar_arrive_expect_tx(bar, DH * (SPLIT ? 16384u : 8192u) + (p.want_o ? kImg : 16384u + (kImg - IMG_T2H)));
         tma_load_2d(sm + SQ_V + 16384 * b, mv, bar, h * d, y);
         if (DH == 2) tma_load_2d(sm + SQ_V + 16384 * b + 8192, mv, bar, h * d + 64, y);
         if (SPLIT) {
             tma_load_2d(sm + SQ_VL + 16384 * b, mvl, bar, h * d, y);
             if (DH == 2) tma_load_2d(sm + SQ_VL + 16384 * b + 8192, mvl, bar, h * d + 64, y);
         }
-        bulk_load(sm + SQ_IMG + SQ_IMG_STRIDE * b, img_of(c), kImg, bar);
+        if (p.want_o) {
+            bulk_load(sm + SQ_IMG + SQ_IMG_STRIDE * b, img_of(c), kImg, bar);
+        } else {
+            // no o: only -W, T2 (hi and lo) and the decay factors; P and Qg were not formed
+            // (the products that read their slots feed only the O accumulator, never output)
+            uint8_t *dsm = sm + SQ_IMG + SQ_IMG_STRIDE * b;
+            const uint8_t *src = img_of(c);
+            bulk_load(dsm + IMG_QGW + 8192, src + IMG_QGW + 8192, 8192, bar);
+            bulk_load(dsm + IMG_QGW + 24576, src + IMG_QGW + 24576, 8192, bar);
+            bulk_load(dsm + IMG_T2H, src + IMG_T2H, kImg - IMG_T2H, bar);
+        }
     };
     if (tid == kIssuer) {
         prefetch_tmap(mk); prefetch_tmap(mv);
@@ -1592,6 +1605,8 @@ cudaError_t gdn_tc_batch(const GdnBatch &b, int n_groups, int n_seqs, int d, boo
     p.n_seqs = n_seqs;
     p.slots = image_slots(b.total, n_seqs);
     p.d = d;
+    p.want_o = 0;
+    for (int g = 0; g < n_groups; ++g) p.want_o |= b.o[g] != nullptr;
     p.scale = b.scale;
     p.status = b.status;
     if (split) return launch<true, 2>(p, n_groups, n_seqs, st);
