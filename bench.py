@@ -192,8 +192,11 @@ class RawGdn:
         self.q, self.k, self.v, self.g, self.b, self.cu = map(d, (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens))
         self.o = torch.empty_like(self.v)
         self.s = torch.empty(x.n_seqs, self.hv, self.d, self.d, dtype=torch.float32, device=dev)
-        self.ws = sr.workspace(1 << 20, dev)
         self.max_len = x.max_seqlen
+        # the call's own scratch (the two-phase form's chunk images), sized once
+        args = sr.gdn_args(self.q, self.k, self.v, self.g, self.b, self.cu, n_seqs=x.n_seqs, max_seqlen=self.max_len,
+                           o=self.o, s_out=self.s)
+        self.ws = sr.workspace(max(sr.gdn_workspace_bytes(args), 1 << 20), dev)
         # pinned host copies for the end-to-end leg
         pin = lambda t: t.contiguous().pin_memory()
         self.h_in = [pin(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens)]
@@ -589,6 +592,7 @@ WORKLOADS = {"raw_qwen": RawGdn, "raw_small": RawGdn, "raw_qwen_f32": RawGdn, "g
              "sparse_32k": GroupReplay,
              **{f"model_{m}_{r}": GroupReplay for m in ("8k", "16k", "32k") for r in ("5", "10")}}
 DEFAULT_WORKLOAD = "model_32k_5"
+L2_BYTES = 126 * 10**6  # B200 L2
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 74.4
 
 
@@ -657,8 +661,10 @@ def job_throughput(units_per_step_per_rank, world, steps, ms):
 
 def workload_config(args, wl, world):
     """The `config` object of the JSON line, the same for both arms."""
-    return {"workload": args.workload, "desc": wl.desc, "tokens_per_step_per_gpu": wl.tokens,
-            "l2": f"inputs {wl.input_bytes / 2**20:.0f} MiB > L2, no flush",
+    mib = wl.input_bytes / 2**20
+    l2 = (f"inputs {mib:.0f} MiB > L2, no flush" if wl.input_bytes > L2_BYTES else
+          f"inputs {mib:.1f} MiB < L2: flushed by a 256 MiB write before every step, each step timed alone")
+    return {"workload": args.workload, "desc": wl.desc, "tokens_per_step_per_gpu": wl.tokens, "l2": l2,
             "parallelism": f"dp{world} (independent replays per GPU)"}
 
 
@@ -701,6 +707,26 @@ def run_ours(args):
     barrier()
     profiled = isinstance(wl, GroupReplay)
     profs = [sr.LaunchProfiler(64) for _ in range(args.steps)] if profiled else None
+    # The single-call workloads (one replay call of a few tens of microseconds of GPU
+    # work) are launch-bound from the host; as a serving engine would, they run as a
+    # CUDA graph of the call, replayed per step.  The group workloads (28 launches,
+    # milliseconds of GPU work per call) run eagerly, with per-launch events.
+    graph = None
+    if not profiled and not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            wl.step()
+        torch.cuda.synchronize(dev)
+        for _ in range(args.warmup):
+            graph.replay()
+        barrier()
+    step = graph.replay if graph is not None else wl.step
+    # inputs that fit in L2: a 256 MiB write flushes it before every step, and each
+    # step is timed by its own events (the flushes stay outside the timed sum)
+    flush = None
+    if wl.input_bytes <= L2_BYTES and not profiled:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
@@ -708,16 +734,22 @@ def run_ours(args):
         for i in range(args.steps):
             if profiled:
                 wl.step(profs[i])
+            elif flush is not None:
+                flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                step()
+                ev[i][1].record(stream)
             else:
-                wl.step()
+                step()
         e1.record(stream)
         barrier()
         # keep the GPU busy long enough for the clock sampler to see load
         t_end = time.perf_counter() + 0.6
         while time.perf_counter() < t_end:
-            wl.step()
+            step()
         torch.cuda.synchronize(dev)
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_dev = sum(a.elapsed_time(b) for a, b in ev) if flush is not None else e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_dev, world, dev)
     ms_per_step = ms / args.steps
     value = job_throughput(wl.tokens, world, args.steps, ms)
 
@@ -845,6 +877,7 @@ def run_ours(args):
                 else "serialised with the replay", "h2d_bytes_per_step": wl.h2d_bytes,
                 "d2h_bytes_per_step": wl.d2h_bytes},
         "gpu_launches": launches,
+        "launch": "cuda graph of the call" if graph is not None else "eager",
         "roofline": roofline,
         "kernels": kernels,
         "clocks": clk.summary(),
@@ -900,6 +933,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="run the single-call workloads eagerly instead of as a CUDA graph")
     ap.add_argument("--precision", choices=["split", "split_fp8", "bf16"], default="split_fp8",
                     help="group workloads: split_fp8 (hi/lo activations, low pass on the fp8 tensor cores; "
                          "parity-checked, the default), split (both passes bf16; parity-checked) or bf16 "
