@@ -1003,19 +1003,38 @@ __global__ void __launch_bounds__(kThreads, 3) gdn_prep_kernel(const __grid_cons
     const int row = quad * 32 + lane;
 
     // the sequence holding this slot: the largest n with floor(cu[n] / C) + n <= slot
-    // (a key that grows with n).  Every warp narrows [lo, hi) 32-fold per round with
-    // one probe per lane, so a few hundred sequences take two rounds of loads.
-    int lo = 0, hi = p.n_seqs;
-    while (hi - lo > 1) {
-        const int step = (hi - lo + 31) >> 5, m = lo + lane * step;
-        const bool le = m < hi && p.cu[m] / C + m <= slot;
-        const int k = max(1, __popc(__ballot_sync(0xffffffffu, le)));  // the probes at or below: a prefix
-        hi = min(hi, lo + k * step);
-        lo += (k - 1) * step;
+    // (a key that grows with n).  Up to 31 sequences: one load per lane brings
+    // cu[0 .. n_seqs], and the sequence's bounds come from the lanes by shuffles.
+    // More: every warp narrows [lo, hi) 32-fold per round with one probe per lane,
+    // so a few hundred sequences take two rounds of loads.
+    int n, bos, eos;
+    if (p.n_seqs < 32) {
+        const int v = lane <= p.n_seqs ? p.cu[lane] : 0;
+        const bool le = lane < p.n_seqs && v / C + lane <= slot;
+        n = max(1, __popc(__ballot_sync(0xffffffffu, le))) - 1;
+        bos = __shfl_sync(0xffffffffu, v, n);
+        eos = __shfl_sync(0xffffffffu, v, n + 1);
+        // the checks of seq_bounds on the values in hand
+        if (!(bos >= 0 && bos <= eos && eos <= p.total && (n != 0 || bos == 0))) {
+            if (tid == 0) atomicOr(p.status, SR_DEV_BAD_CU_SEQLENS);
+            return;
+        }
+        if (eos - bos > p.max_len) {
+            if (tid == 0) atomicOr(p.status, SR_DEV_SEQ_TOO_LONG);
+            return;
+        }
+    } else {
+        int lo = 0, hi = p.n_seqs;
+        while (hi - lo > 1) {
+            const int step = (hi - lo + 31) >> 5, m = lo + lane * step;
+            const bool le = m < hi && p.cu[m] / C + m <= slot;
+            const int k = max(1, __popc(__ballot_sync(0xffffffffu, le)));  // the probes at or below: a prefix
+            hi = min(hi, lo + k * step);
+            lo += (k - 1) * step;
+        }
+        n = lo;
+        if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     }
-    const int n = lo;
-    int bos, eos;
-    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
     const int len = eos - bos, c = slot - (bos / C + n);
     if (c < 0 || c * C >= len) return;
     if (!SR_IN_BOUNDS(slot, p.slots, p.status)) return;
