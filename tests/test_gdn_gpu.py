@@ -216,3 +216,37 @@ def test_many_short_sequences(sr, algo, d):
         n, h = divmod(u, 2)
         assert_close(s[n, h], s_ref[n, h], STATE_TOL, f"state seq {n} head {h}")
         assert_close(o[cu[n]:cu[n + 1], h], o_ref[cu[n]:cu[n + 1], h], OUT_TOL_BF16, f"o seq {n} head {h}")
+
+
+@pytest.mark.parametrize("want_o", [True, False])
+def test_replay_call_captures_in_a_cuda_graph(sr, want_o):
+    """The replay call issues only stream work (a status clear and its kernels)
+    with no host synchronisation, so a serving engine can capture it in a CUDA
+    graph: replaying the graph gives the eager call's results bit for bit,
+    also after the inputs change in place between replays."""
+    x = W.raw_qwen()
+    d = lambda a: a.cuda().contiguous()
+    q, k, v, g, b, cu = map(d, (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens))
+    o = torch.empty_like(v) if want_o else None
+    s = torch.empty(x.n_seqs, v.shape[1], v.shape[2], v.shape[2], dtype=torch.float32, device="cuda")
+    args = sr.gdn_args(q, k, v, g, b, cu, n_seqs=x.n_seqs, max_seqlen=x.max_seqlen, o=o, s_out=s)
+    ws = sr.workspace(sr.gdn_workspace_bytes(args))
+    call = lambda: sr.gdn_replay(q, k, v, g, b, cu, max_seqlen=x.max_seqlen, want_o=want_o, o=o, s_out=s, ws=ws)
+    call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for scale in (1.0, 0.5):
+        v.mul_(scale)
+        call()
+        torch.cuda.synchronize()
+        s_eager = s.clone()
+        o_eager = o.clone() if want_o else None
+        s.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(s, s_eager)
+        if want_o:
+            assert torch.equal(o, o_eager)
+    assert sr.device_status(ws) == 0

@@ -99,3 +99,26 @@ def test_exact_resume_on_gpu(sr, algo):
     torch.cuda.synchronize()
     assert_close(sb, s.double().cpu().numpy(), STATE_TOL, "resumed state")
     assert_close(yb, y[j:].double().cpu().numpy(), OUT_TOL_BF16, "resumed outputs")
+
+
+def test_replay_call_captures_in_a_cuda_graph(sr):
+    """As for the gated-delta call: captured in a CUDA graph, the Mamba2 replay
+    gives the eager call's results bit for bit."""
+    m = W.mamba2_inputs(23, [300, 65, 1, 128], H=8, h0_std=0.2)
+    d = lambda a: a.cuda().contiguous()
+    x, B, C, dt, A, cu, h0 = map(d, (m.x, m.B, m.C, m.dt, m.A, m.cu_seqlens, m.h0))
+    y, s = torch.empty_like(x), torch.empty(4, 8, x.shape[2], B.shape[2], dtype=torch.float32, device="cuda")
+    args = sr.mamba2_args(x, B, C, dt, A, cu, n_seqs=4, max_seqlen=m.max_seqlen, h0=h0, y=y, s_out=s)
+    ws = sr.workspace(sr.mamba2_workspace_bytes(args))
+    call = lambda: sr.mamba2_replay(x, B, C, dt, A, cu, max_seqlen=m.max_seqlen, h0=h0, y=y, s_out=s, ws=ws)
+    call()
+    torch.cuda.synchronize()
+    y_eager, s_eager = y.clone(), s.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    y.zero_()
+    s.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager) and torch.equal(s, s_eager)
