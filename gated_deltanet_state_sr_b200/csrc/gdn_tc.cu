@@ -1001,6 +1001,10 @@ __global__ void __launch_bounds__(kThreads, 3) gdn_prep_kernel(const __grid_cons
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
+    // the state chain (launched as this grid's programmatic dependent) may start
+    // its set-up once every CTA of this grid is running; it waits for this whole
+    // grid, and its memory, before it reads an image
+    grid_launch_dependents();
 
     // the sequence holding this slot: the largest n with floor(cu[n] / C) + n <= slot
     // (a key that grows with n).  Up to 31 sequences: one load per lane brings
@@ -1370,7 +1374,12 @@ __global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_co
     const int quad = warp & 3, half = (warp >> 2) & 1;
     const int row = quad * 32 + lane;
     int bos, eos;
-    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) return;
+    // every CTA waits for the prep grid before it exits, so that this grid's
+    // completion implies the prep's for the work that follows in the stream
+    if (!seq_bounds(p.cu, n, p.total, p.max_len, p.status, bos, eos)) {
+        grid_dependency_wait();
+        return;
+    }
     const int len = eos - bos;
     const int nchunks = (len + C - 1) / C;
     constexpr int d = 64 * DH;
@@ -1381,6 +1390,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_co
 
     if (nchunks == 0) {
         if (mover) state_passthrough<DH>(h0, s_out, sbase, tid, s_elems, p.status);
+        grid_dependency_wait();
         return;
     }
 
@@ -1431,7 +1441,9 @@ __global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_co
             if (DH == 2) tma_load_2d(sm + SQ_KL + 8192, mkl, bar_k, hk * d + 64, y);
         }
     };
-    auto issue_in = [&](int c) {  // V (+ low part) and the chunk image into buffer c & 1
+    // V (+ low part) and the chunk image into buffer c & 1, on one barrier; the
+    // two halves may be issued apart (the image only after the prep grid is done)
+    auto issue_v = [&](int c) {
         const int y = bos + c * C, b = c & 1;
         uint64_t *bar = &bar_in[b];
         mbar_arrive_expect_tx(bar, DH * (SPLIT ? 16384u : 8192u) + (p.want_o ? kImg : 16384u + (kImg - IMG_T2H)));
@@ -1441,6 +1453,10 @@ __global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_co
             tma_load_2d(sm + SQ_VL + 16384 * b, mvl, bar, h * d, y);
             if (DH == 2) tma_load_2d(sm + SQ_VL + 16384 * b + 8192, mvl, bar, h * d + 64, y);
         }
+    };
+    auto issue_img = [&](int c) {
+        const int b = c & 1;
+        uint64_t *bar = &bar_in[b];
         if (p.want_o) {
             bulk_load(sm + SQ_IMG + SQ_IMG_STRIDE * b, img_of(c), kImg, bar);
         } else {
@@ -1453,12 +1469,19 @@ __global__ void __launch_bounds__(kSeqThreads, 1) gdn_seq_kernel(const __grid_co
             bulk_load(dsm + IMG_T2H, src + IMG_T2H, kImg - IMG_T2H, bar);
         }
     };
+    auto issue_in = [&](int c) {
+        issue_v(c);
+        issue_img(c);
+    };
     if (tid == kIssuer) {
         prefetch_tmap(mk); prefetch_tmap(mv);
         if (SPLIT) { prefetch_tmap(mkl); prefetch_tmap(mvl); }
         issue_k(0);
-        issue_in(0);
-        if (nchunks > 1) issue_in(1);
+        issue_v(0);
+        if (nchunks > 1) issue_v(1);
+        grid_dependency_wait();  // the images are the prep grid's output
+        issue_img(0);
+        if (nchunks > 1) issue_img(1);
     }
 
     __nv_bfloat16 *o = p.o[gi];
@@ -1580,7 +1603,21 @@ cudaError_t launch(const GdnTcParams &p, int n_groups, int n_seqs, cudaStream_t 
     if (e != cudaSuccess) return e;
     gdn_prep_kernel<SPLIT, DH><<<dim3(p.slots, p.h_v, n_groups), kThreads, s1, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_seq_kernel<SPLIT, DH><<<dim3(p.h_v, n_seqs, n_groups), kSeqThreads, s2, st>>>(p);
+    // the state chain as the prep's programmatic dependent: its CTAs take their
+    // SMs, tensor memory, initial state and first K and V tiles while the prep's
+    // last units run, and wait for the prep grid only before loading an image
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.h_v, n_seqs, n_groups);
+    cfg.blockDim = dim3(kSeqThreads);
+    cfg.dynamicSmemBytes = size_t(s2);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gdn_seq_kernel<SPLIT, DH>, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

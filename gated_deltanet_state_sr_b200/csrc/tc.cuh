@@ -130,6 +130,15 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 }
+// Programmatic dependent launch.  grid_launch_dependents: once every CTA of this
+// grid has executed it (or exited), the grid launched after it with programmatic
+// stream serialization may start.  grid_dependency_wait: blocks the thread until
+// the grids this one depends on have completed and their memory is visible (at
+// once when there are none).
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 // Makes generic-proxy shared-memory writes visible to the async proxy (tensor core / TMA).
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
