@@ -88,6 +88,20 @@ def test_strong_decay(sr, algo, d):
 
 @pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("d", [64, 128])
+def test_decay_around_the_factorisation_bound(sr, algo, d):
+    """g ~ U(-2.6, -0.001): a chunk's decay e^{gamma_C} lands on both sides of
+    e^{-80}, so one sequence mixes chunks whose masks the tcgen05 kernels form as
+    e^{gamma_t} e^{-gamma_s} with chunks that take an exponential per masked
+    difference (23 and 17 of the 40 (chunk, head) pairs here); q not normalised."""
+    x = W.gdn_inputs(9, [300, 77, 130], 2, 4, d, d, g_range=(-2.6, -0.001), norm_q=False, h0_std=0.2)
+    o, s = run_gpu(sr, x, algo)
+    o_ref, s_ref = run_oracle(x)
+    assert_close(s, s_ref, STATE_TOL, "state")
+    assert_close(o, o_ref, OUT_TOL_BF16, "o")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("d", [64, 128])
 def test_state_only_mode(sr, algo, d):
     x = W.gdn_inputs(6, [150, 40], 2, 4, d, d)
     o, s = run_gpu(sr, x, algo, want_o=False)
