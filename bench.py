@@ -52,8 +52,8 @@ MEASURED_TRAFFIC = {
     # gate/up (single-CTA tiles) of the 1-group workload with the fp8 low pass: 155.8 MB read +
     # 30.0 MB written, x 8 groups
     "model_32k_5": ("gemm_tc.cu", "47f52f1e08eba982", 8 * 185.8e6, "gemm_gateup"),
-    # the raw workload's call, both kernels of the two-phase form: prep 76.4 MB read +
-    # 207.5 MB written, sequential 379.3 MB read + 64.2 MB written
+    # the raw workload's call, both kernels of the two-phase form: prep 76.3 MB read +
+    # 208.0 MB written, sequential 379.1 MB read + 64.2 MB written
     "raw_qwen": ("gdn_tc.cu", "caa0762384027f6e", 727.6e6, None),
     # the Mamba2 workload's launch: 1273.9 MB read + 1222.0 MB written
     "mamba2": ("mamba2_tc.cu", "53e6f86ec1f409d3", 2495.9e6, None),
