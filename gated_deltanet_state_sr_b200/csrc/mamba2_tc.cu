@@ -22,6 +22,9 @@
 // with Gm_h = (G o L_h), L_h[t][s] = e^{gamma_t-gamma_s} dt_s for s <= t.  The A
 // operands of the state's own products (the bf16 copy of S and xw's hi and lo)
 // are written by the other eight warps into tensor memory and read from there;
+// A chunk's gates (gamma, e^{gamma}, the diagonal of diag(w)) are formed by the
+// data warps during the chunk before it, while that chunk's last products run,
+// so the products of a chunk can start as soon as its inputs have landed.
 // C, B and x tiles arrive by TMA (double-buffered, two chunks ahead); y goes
 // from tensor memory straight to global memory, a warp storing 32 consecutive
 // channels of one token per instruction.
@@ -50,9 +53,12 @@ constexpr uint32_t SZ_IN = 49152;        // one input buffer: [C_n0][B_n0][C_n1]
 constexpr uint32_t OFF_IN = 0;           // two buffers
 constexpr uint32_t OFF_Q = 2 * SZ_IN;    // masked G rows [(h,t)][s], 16 KB
 constexpr uint32_t OFF_YS = OFF_Q + 16384;    // G = C B^T staged for the mask rows
-constexpr uint32_t OFF_DW = OFF_YS + 16384;   // diag(w) per head as hi and lo tiles [t][s]: [h0 hi][h1 hi][h0 lo][h1 lo]
-constexpr uint32_t OFF_MISC = OFF_DW + 32768; // gates, tables, barriers
-constexpr uint32_t SZ_MISC = 3072;
+// diag(w) per head as hi and lo tiles [t][s]: [h0 hi][h1 hi][h0 lo][h1 lo], one set
+// per chunk parity (a chunk's set is formed during the chunk before it)
+constexpr uint32_t OFF_DW = OFF_YS + 16384;
+constexpr uint32_t SZ_DW = 32768;
+constexpr uint32_t OFF_MISC = OFF_DW + 2 * SZ_DW; // gate tables (per chunk parity), barriers
+constexpr uint32_t SZ_MISC = 4096;
 constexpr uint32_t kSmem = OFF_MISC + SZ_MISC + 1024;
 
 // barrier of the eight data-moving warps only
@@ -86,11 +92,11 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(sm);
-    float *gam = reinterpret_cast<float *>(sm + OFF_MISC);  // [2][64] gamma
-    float *dts = gam + 2 * C;                                // [2][64] dt (0 beyond the sequence)
-    float *wts = gam + 4 * C;                                // [2][64] dt e^{gamma_C - gamma}
-    float *egs = gam + 6 * C;                                // [2][64] e^{gamma}
-    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 2048);  // [2] input buffers landed
+    // per chunk parity and head: gamma, dt (0 beyond the sequence) and e^{gamma}, [2][2][64] each
+    float *gam_all = reinterpret_cast<float *>(sm + OFF_MISC);
+    float *dts_all = gam_all + 4 * C;
+    float *egs_all = gam_all + 8 * C;
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 3072);  // [2] input buffers landed
     uint64_t *bar_g = bar_in + 2;      // C B^T done
     uint64_t *bar_s = bar_in + 3;      // state part of y and the state update done
     uint64_t *bar_y = bar_in + 4;      // chunk-internal part of y done
@@ -130,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         fence_mbar_init();
     }
     // diag(w) tiles: zero off the diagonal for good; the diagonal is rewritten per chunk
-    for (int e = tid; e < 32768 / 16; e += kThreads)
+    for (int e = tid; e < 2 * SZ_DW / 16; e += kThreads)
         *reinterpret_cast<uint4 *>(sm + OFF_DW + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
     fence_async_smem();
     if (warp == 0) {
@@ -181,12 +187,57 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         if (nchunks > 1) issue_in(1);
     }
 
-    // dt of the next chunk: thread tid < 128 holds token (tid & 63) of head (tid >> 6) of the pair
+    // dt of the next chunk whose gates are formed: thread tid < 128 holds token
+    // (tid & 63) of head (tid >> 6) of the pair
     const int dh = (tid >> 6) & 1, dtok = tid & 63;
     const float Ah = p.A[2 * pair + (warp & 1)];  // warps 0 and 1 scan heads 0 and 1
     float dt_next = (tid < 128 && dtok < len &&
                      SR_IN_BOUNDS((size_t(bos) + dtok) * H + 2 * pair + dh, (long long)p.total * H, p.status))
                         ? p.dt[(size_t(bos) + dtok) * H + 2 * pair + dh] : 0.f;
+    // ---- the gates of chunk cc into the tables and diag(w) tiles of parity cc & 1
+    // (movers only): gamma = inclusive prefix sum of dt A, e^{gamma}, and the
+    // diagonal entries w = dt e^{gamma_C - gamma} of diag(w) as hi and lo.  Chunk
+    // cc's dt is in dt_next, which then moves on to chunk cc + 1.
+    auto gates = [&](int cc) {
+        const int gb = cc & 1;
+        float *gam = gam_all + gb * 2 * C, *dts = dts_all + gb * 2 * C, *egs = egs_all + gb * 2 * C;
+        if (tid < 128) {
+            dts[dh * C + dtok] = dt_next;
+            const int t = (cc + 1) * C + dtok;
+            dt_next = (t < len && SR_IN_BOUNDS((size_t(bos) + t) * H + 2 * pair + dh, (long long)p.total * H,
+                                               p.status))
+                          ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
+        }
+        movers_sync();
+        if (warp < 2) {
+            const float *d = dts + warp * C;
+            const float a0 = d[2 * lane] * Ah, a1 = d[2 * lane + 1] * Ah;
+            float incl = a0 + a1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const float excl = incl - (a0 + a1);
+            gam[warp * C + 2 * lane] = excl + a0;
+            gam[warp * C + 2 * lane + 1] = excl + a0 + a1;
+        }
+        movers_sync();
+        if (tid < 128) {
+            const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
+            const float wv = dts[dh * C + dtok] * __expf(gC - g);
+            egs[dh * C + dtok] = __expf(g);
+            uint32_t whi, wlo;
+            split2(wv, 0.f, whi, wlo);
+            const uint32_t off = OFF_DW + gb * SZ_DW + sw128(dtok, dtok >> 3) + (dtok & 7) * 2;
+            *reinterpret_cast<uint16_t *>(sm + off + dh * 8192) = uint16_t(whi & 0xffffu);
+            *reinterpret_cast<uint16_t *>(sm + off + 16384 + dh * 8192) = uint16_t(wlo & 0xffffu);
+        }
+        fence_async_smem();
+    };
+    if (mover) gates(0);
+    __syncthreads();  // chunk 0's tables and diag(w) tiles, before the first product reads them
+
     auto wait_on = [&](uint64_t *bar, int parity) -> bool {
         const bool w = mbar_wait(bar, uint32_t(parity & 1));
         tc_fence_after();
@@ -204,64 +255,25 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
         const int b = c & 1;
         const uint32_t in = base + OFF_IN + b * SZ_IN;
         const int clen = min(C, len - c * C);
+        const float *gam = gam_all + b * 2 * C, *dts = dts_all + b * 2 * C, *egs = egs_all + b * 2 * C;
         bool w = wait_on(&bar_in[b], (c >> 1) & 1);
-        if (tid == kIssuer && w && want_y) {  // G = [C;B] B^T -> RG needs only this chunk's inputs
+        if (tid == kIssuer && w) {
+            // G = [C;B] B^T -> RG, and x diag(w) (hi + lo of w) -> the chunk-internal part's
+            // columns: both need only this chunk's inputs and its gates (formed a chunk ago)
+            if (want_y) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
-                mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
-            }
-            mma_commit(bar_g);
-        }
-        if (mover) {
-            // ---- gates of the chunk: gamma = inclusive prefix sum of dt A (dt = 0 beyond the sequence)
-            if (tid < 128) {
-                dts[dh * C + dtok] = dt_next;
-                const int t = (c + 1) * C + dtok;
-                dt_next = (t < len && SR_IN_BOUNDS((size_t(bos) + t) * H + 2 * pair + dh, (long long)p.total * H,
-                                                   p.status))
-                              ? p.dt[(size_t(bos) + t) * H + 2 * pair + dh] : 0.f;
-            }
-            movers_sync();
-            if (warp < 2) {
-                const float *d = dts + warp * C;
-                const float a0 = d[2 * lane] * Ah, a1 = d[2 * lane + 1] * Ah;
-                float incl = a0 + a1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += v;
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t a = in + (k >> 2) * 16384 + (k & 3) * 32;
+                    mma_bf16_ss(RG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a + 8192, 16, 1024), ID_G, k > 0);
                 }
-                const float excl = incl - (a0 + a1);
-                gam[warp * C + 2 * lane] = excl + a0;
-                gam[warp * C + 2 * lane + 1] = excl + a0 + a1;
+                mma_commit(bar_g);
             }
-            movers_sync();
-            if (tid < 128) {
-                const float g = gam[dh * C + dtok], gC = gam[dh * C + C - 1];
-                const float wv = dts[dh * C + dtok] * __expf(gC - g);
-                wts[dh * C + dtok] = wv;
-                egs[dh * C + dtok] = __expf(g);
-                // diag(w) of head dh: entry (t, t) of its hi and lo tiles
-                uint32_t whi, wlo;
-                split2(wv, 0.f, whi, wlo);
-                const uint32_t off = sw128(dtok, dtok >> 3) + (dtok & 7) * 2;
-                *reinterpret_cast<uint16_t *>(sm + OFF_DW + dh * 8192 + off) = uint16_t(whi & 0xffffu);
-                *reinterpret_cast<uint16_t *>(sm + OFF_DW + 16384 + dh * 8192 + off) = uint16_t(wlo & 0xffffu);
-            }
-            fence_async_smem();
-        }
-        // ---- x diag(w) (hi + lo of w) -> the chunk-internal part's columns, on the
-        // tensor cores while the movers copy S
-        tc_fence_before();
-        if (check(w)) { ok = false; break; }
-        if (tid == kIssuer) {
-            tc_fence_after();
+            const uint32_t dw = base + OFF_DW + b * SZ_DW;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {  // [x_h0^T; x_h1^T] (MN-major) [Dh_h0; Dh_h1]^T, then the lo tiles
                 const uint64_t ax = sdesc_sw128(in + 32768 + k * 2048, 8192, 1024);
-                mma_bf16_ss(RY, ax, sdesc_sw128(base + OFF_DW + k * 32, 16, 1024), ID_Y, k > 0);
-                mma_bf16_ss(RY, ax, sdesc_sw128(base + OFF_DW + 16384 + k * 32, 16, 1024), ID_Y, 1);
+                mma_bf16_ss(RY, ax, sdesc_sw128(dw + k * 32, 16, 1024), ID_Y, k > 0);
+                mma_bf16_ss(RY, ax, sdesc_sw128(dw + 16384 + k * 32, 16, 1024), ID_Y, 1);
             }
             mma_commit(bar_xw);
         }
@@ -288,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             }
             // ---- xw (own head's diagonal block of the product) as hi + lo into TMEM:
             // lane (h, p), tokens 32 half .. + 31
-            w = wait_on(bar_xw, c);
+            w = wait_on(bar_xw, c) && w;
             {
                 uint32_t r[32], hi[16], lo[16];
                 tmem_ld_32x32b_x32(RY + lane_off + 64 * hrow + 32 * half, r);
@@ -321,7 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             }
             mma_commit(bar_s);
         }
-
         if (want_y) {
             // ---- Gm_h rows: Q[(h, t)][s] = G[t][s] e^{gamma_h,t - gamma_h,s} dt_h,s (s <= t), bf16.
             // G lives in TMEM lanes 0..63, which half of the movers can read: they stage it
@@ -379,6 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1) mamba2_tc_kernel(const __grid_con
             }
         }
 
+        // ---- the next chunk's gates, while this chunk's last products run (the tables
+        // and diag(w) tiles of that parity were last read by chunk c - 1)
+        if (mover && c + 1 < nchunks) gates(c + 1);
         // ---- the products of this chunk are done: y out, and the input buffer of
         // chunk c + 2 (this one) can be refilled
         w = wait_on(bar_s, c);
